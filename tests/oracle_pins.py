@@ -1,0 +1,291 @@
+"""Pins of the fp64 oracle to results fixed by the pages or by mathematics.
+
+Each ``pin_*`` function takes an oracle library handle (``oracle.load(path)``)
+and raises AssertionError when the oracle disagrees.  ``test_oracle_pins``
+runs them on the real oracle; ``test_oracle_mutants`` runs them on copies of
+the oracle with planted mistakes and checks that some pin fails each time.
+
+Sources ("MDN: Parallelizing Stepwise Momentum for Delta Linear Attention"):
+  recurrence ............ paper.rainbus.top summary, step 1; ijyty.com, section 3
+  unrolled closed form .. summary, step 2 (eta_i on write i: this build's reading)
+  row<->column reordering summary, step 3; ijyty.com, section 4
+  chunkwise form ........ summary, step 4
+  spectrum lambda+- ..... summary, step 6; novelty paragraph; ijyty.com, section 5
+  mu = 0 ablation ....... ijyty.com, section 8 (reduces to a gated delta rule)
+"""
+from __future__ import annotations
+
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import oracle
+from chunk_reference import chunk_forward
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _frac(x) -> float:
+    return float(Fraction(x))
+
+
+def _rand_case(rng, B, T, H, d, state=True, alpha_lo=0.3, alpha_hi=0.95,
+               mu_lo=0.4, mu_hi=0.95):
+    q = rng.standard_normal((B, T, H, d))
+    k = rng.standard_normal((B, T, H, d))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, d))
+    al = np.log(rng.uniform(alpha_lo, alpha_hi, (B, T, H)))
+    ml = np.log(rng.uniform(mu_lo, mu_hi, (B, T, H)))
+    be = rng.uniform(0.05, 0.6, (B, T, H))
+    et = rng.uniform(0.2, 1.8, (B, T, H))
+    S0 = rng.standard_normal((B, H, d, d)) * 0.3 if state else None
+    M0 = rng.standard_normal((B, H, d, d)) * 0.3 if state else None
+    return q, k, v, al, ml, be, et, S0, M0
+
+
+def _close(a, b, tol, what):
+    a, b = np.asarray(a), np.asarray(b)
+    err = np.max(np.abs(a - b)) / max(1.0, np.max(np.abs(b)))
+    assert err <= tol, f"{what}: max err {err:.3e} > {tol:.1e}"
+
+
+# ---------------------------------------------------------------- hand-worked
+def _golden_case(lib, name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        g = json.load(f)
+    T, d = len(g["q"]), len(g["q"][0])
+    shp = (1, T, 1, d)
+    q = np.array(g["q"], dtype=np.float64).reshape(shp)
+    k = np.array(g["k"], dtype=np.float64).reshape(shp)
+    v = np.array(g["v"], dtype=np.float64).reshape(shp)
+    gate = lambda key: np.array(g[key], dtype=np.float64).reshape(1, T, 1)
+    al, ml = np.log(gate("alpha")), np.log(gate("mu"))
+    S0 = None
+    if "S0" in g:
+        S0 = np.array([[_frac(x) for x in row] for row in g["S0"]]).reshape(1, 1, d, d)
+    o, vt, S_T, M_T = oracle.chunk_fwd(q, k, v, al, ml, gate("beta"), gate("eta"),
+                                       g["d"], S0, None, lib=lib)
+    exp = g["expected"]
+    conv = lambda m: np.array([[_frac(x) for x in row] for row in m])
+    _close(vt.reshape(T, d), conv(exp["vtilde"]), 1e-14, f"{name} vtilde")
+    _close(o.reshape(T, d), conv(exp["o"]), 1e-14, f"{name} o")
+    _close(S_T.reshape(d, d), conv(exp["S_T"]), 1e-14, f"{name} S_T")
+    _close(M_T.reshape(d, d), conv(exp["M_T"]), 1e-14, f"{name} M_T")
+
+
+def pin_hand_scalar(lib):
+    _golden_case(lib, "hand_scalar_d1_T3.json")
+
+
+def pin_hand_matrix(lib):
+    _golden_case(lib, "hand_matrix_d2_T2.json")
+
+
+# ---------------------------------------------------------------- closed form
+def pin_closed_form(lib):
+    """Unrolled form (summary step 2, with eta_i on write i) at every prefix t."""
+    rng = np.random.default_rng(11)
+    T, d = 24, 5
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, 1, T, 1, d)
+    dcorr = 0.5
+    _, vt, _, _ = oracle.chunk_fwd(q, k, v, al, ml, be, et, dcorr, S0, M0, lib=lib)
+    a, m, b_, e = al[0, :, 0], ml[0, :, 0], be[0, :, 0], et[0, :, 0]
+    K, V, Vt, Q = k[0, :, 0], v[0, :, 0], vt[0, :, 0], q[0, :, 0]
+    abar, mbar = np.exp(np.cumsum(a)), np.exp(np.cumsum(m))
+    c = np.cumsum(b_ * mbar / abar)
+    for t in range(1, T + 1):
+        # M_t = mubar_t M0 - sum_i (mubar_t/mubar_i) eta_i k_i vt_i^T
+        Mt = mbar[t - 1] * M0[0, 0].copy()
+        St = abar[t - 1] * S0[0, 0] - abar[t - 1] * c[t - 1] * M0[0, 0]
+        for i in range(1, t + 1):
+            outer = np.outer(K[i - 1], Vt[i - 1])
+            Mt -= (mbar[t - 1] / mbar[i - 1]) * e[i - 1] * outer
+            c_im1 = c[i - 2] if i >= 2 else 0.0
+            gam = abar[t - 1] / mbar[i - 1] * (c[t - 1] - c_im1)
+            St += gam * e[i - 1] * outer
+        o_t, _, S_t, M_t = oracle.chunk_fwd(q[:, :t], k[:, :t], v[:, :t], al[:, :t],
+                                            ml[:, :t], be[:, :t], et[:, :t], dcorr,
+                                            S0, M0, lib=lib)
+        _close(S_t[0, 0], St, 1e-11, f"closed-form S_{t}")
+        _close(M_t[0, 0], Mt, 1e-11, f"closed-form M_{t}")
+        qh = Q[t - 1] - dcorr * K[t - 1]
+        _close(o_t[0, t - 1, 0], St.T @ qh, 1e-11, f"closed-form o_{t}")
+    # vtilde against its definition using the closed-form S_{t-1}
+    S_prev = S0[0, 0].copy()
+    for t in range(1, T + 1):
+        _close(Vt[t - 1], V[t - 1] - np.exp(a[t - 1]) * S_prev.T @ K[t - 1], 1e-11,
+               f"vtilde_{t}")
+        _, _, S_pt, _ = oracle.chunk_fwd(q[:, :t], k[:, :t], v[:, :t], al[:, :t],
+                                         ml[:, :t], be[:, :t], et[:, :t], dcorr,
+                                         S0, M0, lib=lib)
+        S_prev = S_pt[0, 0]
+
+
+# ---------------------------------------------------------------- mu = 0
+def pin_mu_zero_gated_delta_rule(lib):
+    """mu = 0: S_t = alpha_t (I - beta_t eta_t k_t k_t^T) S_{t-1} + beta_t eta_t k_t v_t^T."""
+    rng = np.random.default_rng(12)
+    T, d = 20, 6
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, 1, T, 1, d)
+    ml[:] = -np.inf
+    dcorr = 0.25
+    o, vt, S_T, M_T = oracle.chunk_fwd(q, k, v, al, ml, be, et, dcorr, S0, M0, lib=lib)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        kt, vv = k[0, t, 0], v[0, t, 0]
+        w = be[0, t, 0] * et[0, t, 0]
+        S = np.exp(al[0, t, 0]) * (np.eye(d) - w * np.outer(kt, kt)) @ S + w * np.outer(kt, vv)
+        _close(o[0, t, 0], S.T @ (q[0, t, 0] - dcorr * kt), 1e-12, f"GDN o_{t}")
+    _close(S_T[0, 0], S, 1e-12, "GDN S_T")
+
+
+# ---------------------------------------------------------------- spectrum
+def _one_step_matrix(lib, dk, dv, alpha, mu, beta, eta, kvec):
+    n = dk * dv
+    A = np.zeros((2 * n, 2 * n))
+    zero = np.zeros((1, 1, dk))
+    g = lambda x: np.array([[x]], dtype=np.float64)
+    for col in range(2 * n):
+        e = np.zeros(2 * n)
+        e[col] = 1.0
+        S = e[:n].reshape(1, 1, dk, dv)
+        M = e[n:].reshape(1, 1, dk, dv)
+        _, _, S1, M1 = oracle.step(zero, kvec.reshape(1, 1, dk), np.zeros((1, 1, dv)),
+                                   g(np.log(alpha)), g(np.log(mu)), g(beta), g(eta), 0.0,
+                                   S, M, lib=lib)
+        A[:, col] = np.concatenate([S1.ravel(), M1.ravel()])
+    return A
+
+
+def _match_multiset(got, want, tol):
+    got = list(got)
+    for w in want:
+        j = int(np.argmin([abs(g - w) for g in got]))
+        assert abs(got[j] - w) <= tol, f"eigenvalue {w} not found (closest {got[j]})"
+        got.pop(j)
+
+
+def pin_spectrum(lib):
+    """Block transition [S;M]_t = A_t [S;M]_{t-1} at d=2 (and d_k=3, d_v=2 via dk=dv=3):
+    spectrum {alpha x (d_k-1)d_v, mu x (d_k-1)d_v, lambda+- x d_v each} with
+    lambda+- = (tau +- sqrt(tau^2 - 4 alpha mu)) / 2, tau = alpha + mu - alpha beta eta |k|^2."""
+    cases = [  # (alpha, mu, beta, eta, k): complex pair, real pair, |k| != 1
+        (0.7, 0.6, 0.3, 0.9, np.array([0.6, 0.8])),
+        (0.2, 0.9, 0.7, 1.9, np.array([1.0, 0.0])),
+        (0.5, 0.5, 0.25, 1.0, np.array([0.9, -0.7])),
+        (0.6, 0.45, 0.35, 1.3, np.array([0.3, -0.5, 0.8])),
+    ]
+    for alpha, mu, beta, eta, kv in cases:
+        dk = dv = kv.size
+        A = _one_step_matrix(lib, dk, dv, alpha, mu, beta, eta, kv)
+        kappa = float(kv @ kv)
+        tau = alpha + mu - alpha * beta * eta * kappa
+        disc = complex(tau * tau - 4 * alpha * mu)
+        lp, lm_ = (tau + disc ** 0.5) / 2, (tau - disc ** 0.5) / 2
+        want = ([alpha] * ((dk - 1) * dv) + [mu] * ((dk - 1) * dv)
+                + [lp] * dv + [lm_] * dv)
+        _match_multiset(np.linalg.eigvals(A), want, 1e-7)
+
+
+# ---------------------------------------------------------------- chunk form
+def pin_chunked_form(lib):
+    """The chunkwise restatement equals the stepwise oracle for every chunk length,
+    ragged tails included, with non-zero entering states."""
+    rng = np.random.default_rng(13)
+    B, T, H, d = 2, 37, 2, 4
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    ref = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0, lib=lib)
+    for C in (1, 2, 4, 16, 64):
+        got = chunk_forward(q, k, v, al, ml, be, et, 0.5, S0, M0, C=C)
+        for name, x, y in zip(("o", "vtilde", "S_T", "M_T"), got, ref):
+            _close(x, y, 1e-10, f"chunked C={C} {name}")
+
+
+# ---------------------------------------------------------------- coefficients
+def pin_chunk_coeffs(lib):
+    """Per-chunk la, lm, lc, Gamma reproduce the chunk-end state through the unrolled
+    form; Gamma's diagonal is beta_r eta_r and Gamma obeys
+    Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r mubar_r / mubar_i."""
+    rng = np.random.default_rng(14)
+    B, T, H, d, C = 1, 45, 2, 3, 16
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    la, lm, lc, G = oracle.chunk_coeffs(al, ml, be, et, C, lib=lib)
+    _, vt, _, _ = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0, lib=lib)
+    NT = (T + C - 1) // C
+    for h in range(H):
+        S, M = S0[0, h].copy(), M0[0, h].copy()
+        for n in range(NT):
+            t0, t1 = n * C, min(T, n * C + C)
+            L = t1 - t0
+            Gn = G[0, h, n]
+            a_c, m_c, c_c = la[0, h, t0:t1], lm[0, h, t0:t1], lc[0, h, t0:t1]
+            # log-domain quantities against cumulative products of the gates
+            assert np.allclose(np.exp(a_c), np.cumprod(np.exp(al[0, t0:t1, h])), rtol=1e-12)
+            assert np.allclose(np.exp(m_c), np.cumprod(np.exp(ml[0, t0:t1, h])), rtol=1e-12)
+            terms = be[0, t0:t1, h] * np.exp(m_c) / np.exp(a_c)
+            assert np.allclose(np.exp(c_c), np.cumsum(terms), rtol=1e-12)
+            alpha = np.exp(al[0, t0:t1, h])
+            for r in range(L):
+                assert abs(Gn[r, r] - be[0, t0 + r, h] * et[0, t0 + r, h]) < 1e-13
+                for i in range(r):
+                    want = (alpha[r] * Gn[r - 1, i]
+                            + et[0, t0 + i, h] * be[0, t0 + r, h] * np.exp(m_c[r] - m_c[i]))
+                    assert abs(Gn[r, i] - want) <= 1e-12 * max(1.0, abs(want))
+            assert np.all(np.triu(Gn, 1) == 0)
+            assert np.all(Gn[L:, :] == 0) and np.all(Gn[:, L:] == 0)
+            K, Vt = k[0, t0:t1, h], vt[0, t0:t1, h]
+            abarL, bL = np.exp(a_c[-1]), np.exp(a_c[-1] + c_c[-1])
+            w_m = et[0, t0:t1, h] * np.exp(m_c[-1] - m_c)
+            S_new = abarL * S - bL * M + K.T @ (Gn[L - 1, :L][:, None] * Vt)
+            M_new = np.exp(m_c[-1]) * M - K.T @ (w_m[:, None] * Vt)
+            S, M = S_new, M_new
+        _, _, S_T, M_T = oracle.chunk_fwd(q[:, :, h:h + 1], k[:, :, h:h + 1],
+                                          v[:, :, h:h + 1], al[:, :, h:h + 1],
+                                          ml[:, :, h:h + 1], be[:, :, h:h + 1],
+                                          et[:, :, h:h + 1], 0.5, S0[:, h:h + 1],
+                                          M0[:, h:h + 1], lib=lib)
+        _close(S, S_T[0, 0], 1e-11, f"coeffs S_T head {h}")
+        _close(M, M_T[0, 0], 1e-11, f"coeffs M_T head {h}")
+
+
+# ---------------------------------------------------------------- decode step
+def pin_step_matches_sequence(lib):
+    """T calls of the one-token step equal one pass over the T tokens (the pages'
+    claim that stepwise decoding behaves exactly as chunkwise training)."""
+    rng = np.random.default_rng(15)
+    B, T, H, d = 2, 9, 3, 4
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    o_ref, vt_ref, S_ref, M_ref = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0,
+                                                   lib=lib)
+    S, M = S0, M0
+    for t in range(T):
+        o, vt, S, M = oracle.step(q[:, t], k[:, t], v[:, t], al[:, t], ml[:, t], be[:, t],
+                                  et[:, t], 0.5, S, M, lib=lib)
+        _close(o, o_ref[:, t], 1e-13, f"step o_{t}")
+        _close(vt, vt_ref[:, t], 1e-13, f"step vtilde_{t}")
+    _close(S, S_ref, 1e-13, "step S_T")
+    _close(M, M_ref, 1e-13, "step M_T")
+
+
+def pin_resume(lib):
+    """Running [0, T1) then [T1, T) with the first call's S_T, M_T as the second's
+    S0, M0 equals one call over [0, T)."""
+    rng = np.random.default_rng(16)
+    B, T, H, d = 1, 30, 2, 4
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    ref = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0, lib=lib)
+    T1 = 13
+    a = oracle.chunk_fwd(q[:, :T1], k[:, :T1], v[:, :T1], al[:, :T1], ml[:, :T1],
+                         be[:, :T1], et[:, :T1], 0.5, S0, M0, lib=lib)
+    b = oracle.chunk_fwd(q[:, T1:], k[:, T1:], v[:, T1:], al[:, T1:], ml[:, T1:],
+                         be[:, T1:], et[:, T1:], 0.5, a[2], a[3], lib=lib)
+    _close(np.concatenate([a[0], b[0]], axis=1), ref[0], 1e-13, "resume o")
+    _close(b[2], ref[2], 1e-13, "resume S_T")
+
+
+ALL_PINS = [pin_hand_scalar, pin_hand_matrix, pin_closed_form, pin_mu_zero_gated_delta_rule,
+            pin_spectrum, pin_chunked_form, pin_chunk_coeffs, pin_step_matches_sequence,
+            pin_resume]
