@@ -1,0 +1,447 @@
+"""Benchmark of the MDN hot path: one step = mdn_chunk_fwd over one batch of the
+workload plus one mdn_step decode token continuing from the pass's (S_T, M_T).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME|INDEX]
+
+Prints ONE JSON line on rank 0.  For N > 1 launch with torch.distributed.run:
+each rank processes its own independently seeded batch (heads are independent,
+so there is no collective on the data path); the step time is the max over
+ranks.  ``--impl reference`` times the fp64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mdn_inputs as mi  # noqa: E402
+
+METRIC = "MDN chunk-fwd tokens/s (d=128, bf16 in/fp32 state) and % tensor/HBM roofline"
+DEFAULT_WORKLOAD = 1           # B=4, H=8, T=2048, d=128, bf16
+L2_FLUSH_BYTES = 256 << 20     # > 126 MB of L2
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x FP32 lanes x FMA x max clock
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def load_traffic():
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def kernel_work(name: str, spec: mi.Spec):
+    """Algorithmic work of one launch of a kernel: (bound, amount, unit-of-peak).
+    Chunk kernels process every token-head of the batch per launch; the decode
+    kernel processes every head once."""
+    th = spec.B * spec.T * spec.H          # token-heads
+    d, C = spec.d, spec.C
+    heads = spec.B * spec.H
+    states = 2 * heads * d * d * 4 * (2 if spec.state_std > 0 else 1)  # S_T,M_T (+S0,M0)
+    if name in ("chunk_tc", "inter_tc"):
+        # whole pass: q,k,v,o,vtilde bf16 + 4 fp32 gates, plus states
+        return "hbm", th * (5 * d * 2 + 16) + states, "GB/s"
+    if name == "inter_simt":
+        return "alu", th * 12.0 * d * d, "TFLOP/s"
+    if name == "intra_simt":
+        return "alu", th * 5.0 * C * d, "TFLOP/s"
+    if name == "output_simt":
+        return "alu", th * 4.0 * C * d, "TFLOP/s"
+    if name == "gate_prep":
+        return "hbm", th * (16 + 16 + 4 * C), "GB/s"
+    if name == "step":
+        return "hbm", heads * (4 * d * d * 4 + 3 * d * 2 + 16 + 2 * d * 2), "GB/s"
+    return None, 0.0, ""
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clock record
+            self.err = str(e)
+
+    _NAMES = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+              0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+              0x100: "display_clock_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self._NAMES.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "source": "nvml"}
+
+
+# ---------------------------------------------------------------- our path
+def decode_token(spec: mi.Spec, seed: int):
+    """One decode token per (b, h): q, k, v [B,H,d] and gates [B,H] (stored dtypes)."""
+    s = mi.replace(spec, T=1, seed=seed, state_std=0.0)
+    inp = mi.make_inputs(s)
+    return inp
+
+
+def run_ours(args, rank, world, device):
+    import momentum_delta_rule_mdn_b200 as mdn
+
+    spec0 = workload_spec(args.workload)
+    spec = mi.replace(spec0, seed=spec0.seed + 7919 * rank)
+    inp = mi.make_inputs(spec)
+    tok = decode_token(spec, spec.seed + 1)
+    dev = mi.to_torch(inp, device)
+    dtok = {k: (v[:, 0].contiguous() if v is not None else None)
+            for k, v in mi.to_torch(tok, device).items()}
+    B, T, H, d = spec.B, spec.T, spec.H, spec.d
+    ws = torch.empty(mdn.chunk_fwd_workspace_size(B, T, H, d, spec.C, dev["q"].dtype),
+                     dtype=torch.uint8, device=device)
+    o = torch.empty_like(dev["q"])
+    vt = torch.empty_like(dev["q"])
+    S_T = torch.empty((B, H, d, d), dtype=torch.float32, device=device)
+    M_T = torch.empty_like(S_T)
+    o1 = torch.empty_like(dtok["q"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    gates = ("alpha_log", "mu_log", "beta", "eta")
+
+    def step():
+        mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), inp.d_corr,
+                      dev["S0"], dev["M0"], spec.C, out=(o, vt, S_T, M_T), workspace=ws)
+        mdn.step(dtok["q"], dtok["k"], dtok["v"], *(dtok[g] for g in gates), inp.d_corr,
+                 S_T, M_T, o=o1, want_vtilde=False)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed (untimed) before each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    mdn.profile_enable(True)
+    mdn.profile_read(reset=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    kernels = mdn.profile_read(reset=True)
+    mdn.profile_enable(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = float(np.mean(step_ms))
+    ms_max = max_over_ranks(ms, world, device)
+
+    tokens_per_rank = B * T
+    value = tokens_per_rank * world / (ms_max * 1e-3)
+
+    # ---- dominant kernel and its roofline
+    hbm, bf16, peak_src = load_peaks()
+    dom = max(kernels.items(), key=lambda kv: kv[1][0]) if kernels else None
+    roofline = None
+    gpu_launches = sum(n for _, n in kernels.values())
+    if dom:
+        name, (tot_ms, n) = dom
+        bound, work, unit = kernel_work(name, spec)
+        avg_s = tot_ms / n * 1e-3
+        if bound == "hbm":
+            achieved, peak = work / avg_s / 1e9, hbm
+        elif bound == "tensor":
+            achieved, peak = work / avg_s / 1e12, bf16
+        else:
+            achieved, peak = work / avg_s / 1e12, FP32_ALU_PEAK_TFLOPS
+        tr = load_traffic().get(name, {})
+        traffic = tr.get("bytes_per_launch") if tr.get("workload") == spec0.name else None
+        roofline = {"kernel": name, "bound": bound, "achieved": round(achieved, 3),
+                    "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
+                    "traffic": traffic,
+                    "peak_source": peak_src if bound != "alu" else
+                    "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz",
+                    "kernel_ms_avg": round(tot_ms / n, 5),
+                    "share_of_step": round(tot_ms / args.steps / ms, 4)}
+
+    # ---- end to end through the public call, host (pinned) buffers
+    e2e = run_e2e(args, mdn, inp, tok, spec, device, world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if "chunk_tc" in kernels else "f32",
+        "data": "synthetic (seeded generator; gates from the stable parameterisation)",
+        "config": {"workload": spec0.name, "B": B, "T": T, "H": H, "d_k": d, "d_v": d,
+                   "C": spec.C, "inputs": spec.dtype, "state": "fp32",
+                   "step": "mdn_chunk_fwd over the batch + 1 mdn_step token",
+                   "l2": "flushed before every timed step (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{world} (independent heads, no collective)",
+                   "global_batch": B * world, "seq_len": T},
+        "roofline": roofline,
+        "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1]} for k, v in kernels.items()},
+        "gpu_launches": gpu_launches,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+    }
+    return line, spec
+
+
+def run_e2e(args, mdn, inp, tok, spec, device, world):
+    """Same metric through the public API with pinned host inputs: per step the
+    inputs are copied host->device, the pass runs, and every result is read back."""
+    host = mi.to_torch(inp, "cpu", pin=True)
+    htok = {k: (v[:, 0].contiguous().pin_memory() if v is not None else None)
+            for k, v in mi.to_torch(tok, "cpu").items()}
+    gates = ("alpha_log", "mu_log", "beta", "eta")
+    B, T, H, d = spec.B, spec.T, spec.H, spec.d
+    out_h = (torch.empty_like(host["q"]).pin_memory(), torch.empty_like(host["q"]).pin_memory(),
+             torch.empty((B, H, d, d)).pin_memory(), torch.empty((B, H, d, d)).pin_memory())
+    o1_h = torch.empty_like(htok["q"]).pin_memory()
+    ws = torch.empty(mdn.chunk_fwd_workspace_size(B, T, H, d, spec.C, host["q"].dtype),
+                     dtype=torch.uint8, device=device)
+    h2d = sum(t.numel() * t.element_size() for k, t in host.items() if t is not None) + \
+        sum(t.numel() * t.element_size() for t in htok.values() if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in out_h) + o1_h.numel() * o1_h.element_size()
+
+    def step():
+        o, vt, S_T, M_T = mdn.chunk_fwd(host["q"], host["k"], host["v"],
+                                        *(host[g] for g in gates), inp.d_corr, host["S0"],
+                                        host["M0"], spec.C, out=out_h, workspace=ws)
+        dt = {k: v.to(device, non_blocking=True) for k, v in htok.items() if v is not None}
+        # the decode token continues from the device copies of (S_T, M_T)
+        S_d = S_T.to(device, non_blocking=True)
+        M_d = M_T.to(device, non_blocking=True)
+        o1, _ = mdn.step(dt["q"], dt["k"], dt["v"], *(dt[g] for g in gates), inp.d_corr,
+                         S_d, M_d, want_vtilde=False)
+        o1_h.copy_(o1, non_blocking=True)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / n, world, device)
+    # (S_T, M_T) go host->device again for the decode token
+    h2d += 2 * B * H * d * d * 4
+    return {"value": round(B * T * world / (ms * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_baseline(spec: mi.Spec, inp=None, budget_s: float = 10.0):
+    """The fp64 oracle as it stands, on the host cores, over the same workload
+    (the whole batch per repetition), repeated until ~budget_s of CPU work."""
+    import oracle
+    inp = inp or mi.make_inputs(spec)
+    args = (inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log, inp.beta, inp.eta, inp.d_corr,
+            inp.S0, inp.M0)
+    args64 = [None if a is None else (np.asarray(a, dtype=np.float64) if isinstance(a, np.ndarray) else a)
+              for a in args]
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.chunk_fwd(*args64)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(spec.B * spec.T / dt, 1), "unit": "tokens/s",
+            "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{spec.name}: the full batch ({spec.B}x{spec.T} tokens x {spec.H} heads, "
+                      f"fp64 stepwise recurrence), {reps} repetition(s), {dt:.2f} s each",
+            "seconds_per_batch": round(dt, 3)}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    spec = workload_spec(args.workload)
+    inp = mi.make_inputs(spec)
+    tok = decode_token(spec, spec.seed + 1)
+    c64 = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
+    full = [c64(x) for x in (inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log, inp.beta, inp.eta)]
+    s0, m0 = c64(inp.S0), c64(inp.M0)
+    # bounded sample per step: the first `hs` heads of every batch row
+    t0 = time.perf_counter()
+    oracle.chunk_fwd(*[x[:, :, :1] for x in full], inp.d_corr,
+                     None if s0 is None else s0[:, :1], None if m0 is None else m0[:, :1])
+    per_head = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)   # whole run within ~2.5 minutes
+    hs = int(max(1, min(spec.H, budget / max(per_head, 1e-6))))
+
+    def one():
+        o, vt, S, M = oracle.chunk_fwd(*[x[:, :, :hs] for x in full], inp.d_corr,
+                                       None if s0 is None else s0[:, :hs],
+                                       None if m0 is None else m0[:, :hs])
+        oracle.step(*[c64(x)[:, 0, :hs] for x in (tok.q, tok.k, tok.v, tok.alpha_log,
+                                                  tok.mu_log, tok.beta, tok.eta)],
+                    inp.d_corr, S, M)
+
+    for _ in range(args.warmup):
+        one()
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        one()
+        times.append(time.perf_counter() - t)
+    sec = float(np.mean(times))
+    tokens = spec.B * spec.T * hs / spec.H          # token-heads processed / heads per token
+    value = tokens / sec
+    cb = {"value": round(value, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+          "kind": "oracle",
+          "sample": f"{spec.name}: {hs} of {spec.H} heads per batch row each step "
+                    f"(token rate scaled by {hs}/{spec.H})"}
+    return {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
+                       "d_k": spec.d, "d_v": spec.d, "C": spec.C,
+                       "step": "oracle forward over the sample + 1 decode token",
+                       "global_batch": spec.B, "seq_len": spec.T},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- plumbing
+def workload_spec(w):
+    if w is None:
+        return mi.CONFIGS[DEFAULT_WORKLOAD]
+    if str(w).isdigit():
+        return mi.CONFIGS[int(w)]
+    for s in mi.CONFIGS:
+        if s.name == w:
+            return s
+    raise SystemExit(f"unknown workload {w!r}")
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line, spec = run_ours(args, rank, world, device)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(spec)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

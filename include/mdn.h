@@ -1,0 +1,180 @@
+/*
+ * mdn.h -- C ABI of libmdn: the Momentum DeltaNet (MDN) chunkwise forward
+ * pass and single-token decode step on NVIDIA B200 (sm_100a).
+ *
+ * The method ("MDN: Parallelizing Stepwise Momentum for Delta Linear
+ * Attention", arXiv 2605.05838; paper.rainbus.top summary, steps 1-7;
+ * ijyty.com article, sections 3-6).  Per (batch b, head h), with fast weight S
+ * and momentum M, both d_k x d_v fp32, and alpha_t = exp(alpha_log_t),
+ * mu_t = exp(mu_log_t):
+ *
+ *     p_t      = alpha_t k_t
+ *     vtilde_t = v_t - S_{t-1}^T p_t                   (corrected value)
+ *     M_t      = mu_t M_{t-1} - eta_t k_t vtilde_t^T
+ *     S_t      = alpha_t S_{t-1} - beta_t M_t
+ *     o_t      = S_t^T qhat_t,   qhat_t = q_t - d k_t  (output correction)
+ *
+ * mdn_chunk_fwd computes o, vtilde and the final (S_T, M_T) for a whole
+ * sequence with the chunkwise-parallel form (summary, step 4); mdn_step runs
+ * the recurrence for one token (the decoding form, ijyty.com section 6).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates or frees memory; scratch space is passed in explicitly.
+ *  - Layouts are dense, row-major, without padding:
+ *        q, k, v, o, vtilde : [B, T, H, d]        (mdn_step: [B, H, d])
+ *        gates              : [B, T, H] fp32      (mdn_step: [B, H])
+ *        S0, M0, S_T, M_T, S, M : [B, H, d_k, d_v] fp32, row index over d_k
+ *    q, k, v, o and vtilde use the element type `in_dtype`; everything else
+ *    is fp32.  Alignment: mdn_chunk_fwd wants q, k, v, o, vtilde and the
+ *    states 16-byte aligned and the workspace 256-byte aligned; mdn_step wants
+ *    S and M 16-byte aligned; every other pointer needs only the alignment of
+ *    its element type (la, lm, lc, b of mdn_chunk_gate_prep: 8 bytes).
+ *  - Work is enqueued on `stream` (NULL = the legacy default stream) and runs
+ *    asynchronously; the call returns once the work is enqueued.
+ *  - Arguments are validated on the host before anything is enqueued; a call
+ *    that fails validation writes nothing.  No entry point aborts or exits.
+ *  - Gates are taken as given: the library applies no clamp or activation.
+ *  - Calls that share output or scratch buffers must be ordered by the caller.
+ */
+#ifndef MDN_H
+#define MDN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *mdn_stream_t;
+
+typedef enum {
+    MDN_OK = 0,
+    MDN_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment, bad size  */
+    MDN_ERR_UNSUPPORTED = 2,  /* valid but outside this build's support (d, C, dtype) */
+    MDN_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed                 */
+    MDN_ERR_NONFINITE = 4,    /* MDN_CHECK_FINITE found a NaN/Inf in an output        */
+    MDN_ERR_TIMEOUT = 5       /* a bounded on-device wait ran out (kernel gave up)    */
+} mdn_status;
+
+typedef enum {
+    MDN_F32 = 0,   /* IEEE fp32 */
+    MDN_BF16 = 1   /* bfloat16  */
+} mdn_dtype;
+
+/* Flags for mdn_chunk_fwd. */
+#define MDN_CHECK_FINITE 0x1  /* after the pass, synchronise `stream` and return
+                                 MDN_ERR_NONFINITE if o, vtilde, S_T or M_T holds
+                                 a NaN or Inf, and MDN_ERR_TIMEOUT if a kernel
+                                 reported a wait that ran out */
+#define MDN_FORCE_SIMT   0x2  /* use the fp32 CUDA-core kernels even for bf16 input */
+
+/* Version of this ABI (incremented on any incompatible change). */
+int mdn_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mdn_status_string(mdn_status status);
+
+/*
+ * Bytes of device scratch that mdn_chunk_fwd needs for these sizes, or 0 if
+ * the sizes are invalid or unsupported.  Pure host function.
+ */
+size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    mdn_dtype in_dtype);
+
+/*
+ * Chunkwise forward pass over a whole sequence (summary, steps 2-5; the
+ * chunk form Vtilde = U - Y S + Z M, U = T V, Y = T Diag(alphabar) P,
+ * Z = T Diag(b) P, T = (I + P K^T o Gamma-)^{-1}, with o from the reordered
+ * sum (Qhat K^T o Gamma) Vtilde plus the carried-state term).
+ *
+ *   q, k, v     [B,T,H,d] in_dtype.  d_k = d_v = d.
+ *   alpha_log, mu_log, beta, eta  [B,T,H] fp32.
+ *   d_corr      the scalar d of qhat = q - d k.
+ *   S0, M0      [B,H,d,d] fp32 entering states; either may be NULL (zeros).
+ *   C           chunk length; this build supports C = 64.
+ *   o, vtilde   [B,T,H,d] in_dtype outputs (vtilde is the materialised Vtilde).
+ *   S_T, M_T    [B,H,d,d] fp32 outputs: the states after token T.  They may
+ *               alias S0 / M0 (read before written, per head).
+ *   workspace   device scratch of at least mdn_chunk_fwd_workspace_size(...)
+ *               bytes, 256-byte aligned; its contents on entry do not matter.
+ *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT.
+ *
+ * Support: d in {64, 128}, C = 64, any T >= 0 (a short last chunk is handled
+ * as if padded with steps that leave S and M unchanged), B, H >= 0 with
+ * B*H*ceil(T/C) < 2^31.  T = 0 copies S0, M0 (or zeros) to S_T, M_T.
+ * Errors: MDN_ERR_INVALID_ARG (null required pointer, negative size,
+ * unaligned pointer, too-small workspace), MDN_ERR_UNSUPPORTED (d, C or dtype
+ * outside support), MDN_ERR_CUDA (launch failure), and with MDN_CHECK_FINITE
+ * also MDN_ERR_NONFINITE / MDN_ERR_TIMEOUT.
+ */
+mdn_status mdn_chunk_fwd(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                         const float *alpha_log, const float *mu_log,
+                         const float *beta, const float *eta, float d_corr,
+                         const float *S0, const float *M0,
+                         int B, int T, int H, int dk, int dv, int C,
+                         void *o, void *vtilde, float *S_T, float *M_T,
+                         void *workspace, size_t ws_bytes, int flags,
+                         mdn_stream_t stream);
+
+/*
+ * One decode token for every (b, h): the stepwise recurrence above, applied
+ * in place (ijyty.com section 6: decoding runs the recurrence token by token).
+ *
+ *   q, k, v     [B,H,d] in_dtype;  gates [B,H] fp32;  d_corr as above.
+ *   S, M        [B,H,d,d] fp32, read and overwritten with S_t, M_t.
+ *   o           [B,H,d] in_dtype output;  vtilde [B,H,d] in_dtype or NULL.
+ *
+ *   flags       must be 0 (reserved).
+ * Support: d in {64, 128}.  Each state element is read once and written once.
+ * Errors: MDN_ERR_INVALID_ARG, MDN_ERR_UNSUPPORTED, MDN_ERR_CUDA.
+ */
+mdn_status mdn_step(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                    const float *alpha_log, const float *mu_log,
+                    const float *beta, const float *eta, float d_corr,
+                    float *S, float *M, int B, int H, int dk, int dv,
+                    void *o, void *vtilde, int flags, mdn_stream_t stream);
+
+/*
+ * The chunk coefficients alone (the gate-preparation stage of mdn_chunk_fwd;
+ * summary step 5), each cumulative quantity restarting at every chunk start:
+ *
+ *   la_r = sum_{j<=r} alpha_log_j            lm_r = sum_{j<=r} mu_log_j
+ *   lc_r = logcumsumexp_{j<=r}(log beta_j + lm_j - la_j)     (-inf if all beta = 0)
+ *   b_r  = exp(la_r + lc_r)                   (= alphabar_r c_r)
+ *   gamma_{r,i} = eta_i (alphabar_r / mubar_i)(c_r - c_{i-1})  for i <= r, else 0
+ *
+ *   la, lm, lc, b   [B,H,NT*C] fp32 outputs, NT = ceil(T/C); positions past T
+ *                   hold the values of steps that leave the state unchanged.
+ *   gamma           [B,H,NT,C,C] fp32 output, or NULL to skip it.
+ * Support: C = 64.  Errors: MDN_ERR_INVALID_ARG, MDN_ERR_UNSUPPORTED, MDN_ERR_CUDA.
+ */
+mdn_status mdn_chunk_gate_prep(const float *alpha_log, const float *mu_log,
+                               const float *beta, const float *eta,
+                               int B, int T, int H, int C,
+                               float *la, float *lm, float *lc, float *b, float *gamma,
+                               mdn_stream_t stream);
+
+/*
+ * Optional per-kernel timing (no counterpart in the method; a measurement aid).
+ * mdn_profile_enable(1) makes every later kernel launch of the library record a
+ * CUDA event pair on its launch stream (the events are created on the first
+ * enable, so that call needs a current CUDA device); mdn_profile_enable(0)
+ * stops recording.  Returns the previous state, or -1 if events could not be
+ * created.
+ * mdn_profile_read synchronises the recorded events and writes, for up to
+ * `capacity` kernel names, the name (static string), total device time in ms
+ * and launch count since the last reset; returns the number written, or -1 on
+ * a CUDA error.  `reset` != 0 clears the totals afterwards.  Any output array
+ * may be NULL.
+ */
+int mdn_profile_enable(int on);
+int mdn_profile_read(int reset, const char **names, double *total_ms,
+                     long long *launches, int capacity);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MDN_H */

@@ -1,0 +1,187 @@
+"""Thin torch binding of libmdn.  Argument marshalling only: every step of the
+forward pass and of the decode step runs in the library's CUDA kernels.
+
+Device tensors in -> device tensors out, on the current CUDA stream.  Host
+(CPU) tensors are copied to the current device first and the results copied
+back (pinned host memory makes those copies asynchronous).
+"""
+from __future__ import annotations
+
+import threading
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_lock = threading.Lock()
+_handle = None
+
+
+def library():
+    """The loaded libmdn (ctypes.CDLL)."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            _handle = _lib.load()
+        return _handle
+
+
+class MDNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def status_string(status: int) -> str:
+    return library().mdn_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return _lib.MDN_F32
+    if t.dtype == torch.bfloat16:
+        return _lib.MDN_BF16
+    raise TypeError(f"q, k, v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _check(status: int, where: str):
+    if status != _lib.MDN_OK:
+        raise MDNError(status, where)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: Optional[torch.Tensor], dtype, shape, name):
+    if t is None:
+        return
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()}")
+
+
+def chunk_fwd_workspace_size(B: int, T: int, H: int, d: int, C: int = 64,
+                             dtype: torch.dtype = torch.bfloat16) -> int:
+    code = _lib.MDN_BF16 if dtype == torch.bfloat16 else _lib.MDN_F32
+    return int(library().mdn_chunk_fwd_workspace_size(B, T, H, d, d, C, code))
+
+
+def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0=None,
+              C: int = 64, *, out=None, workspace: Optional[torch.Tensor] = None,
+              flags: int = 0, stream: Optional[torch.cuda.Stream] = None):
+    """Chunkwise MDN forward pass.  Returns (o, vtilde, S_T, M_T).
+
+    q, k, v: [B,T,H,d] float32 or bfloat16; gates [B,T,H] float32; S0, M0
+    [B,H,d,d] float32 or None.  ``out`` may hold preallocated (o, vtilde, S_T,
+    M_T).  Host inputs are copied to the current device and results back.
+    """
+    if not q.is_cuda:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        mv = lambda t: None if t is None else t.to(dev, non_blocking=True)
+        res = chunk_fwd(mv(q), mv(k), mv(v), mv(alpha_log), mv(mu_log), mv(beta), mv(eta),
+                        d, mv(S0), mv(M0), C, workspace=workspace, flags=flags,
+                        stream=stream)
+        if out is not None:
+            for dst, src in zip(out, res):
+                dst.copy_(src, non_blocking=True)
+            return out
+        return tuple(t.to("cpu") for t in res)
+    B, T, H, D = q.shape
+    code = _dtype_code(q)
+    for name, t in (("k", k), ("v", v)):
+        _need(t, q.dtype, q.shape, name)
+    _need(q, q.dtype, q.shape, "q")
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (B, T, H), name)
+    _need(S0, torch.float32, (B, H, D, D), "S0")
+    _need(M0, torch.float32, (B, H, D, D), "M0")
+    if out is None:
+        o = torch.empty_like(q)
+        vt = torch.empty_like(q)
+        S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+        M_T = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    else:
+        o, vt, S_T, M_T = out
+        _need(o, q.dtype, q.shape, "o")
+        _need(vt, q.dtype, q.shape, "vtilde")
+        _need(S_T, torch.float32, (B, H, D, D), "S_T")
+        _need(M_T, torch.float32, (B, H, D, D), "M_T")
+    lib = library()
+    ws_bytes = int(lib.mdn_chunk_fwd_workspace_size(B, T, H, D, D, C, code))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    status = lib.mdn_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta),
+        float(d), _ptr(S0), _ptr(M0), B, T, H, D, D, C, _ptr(o), _ptr(vt), _ptr(S_T), _ptr(M_T),
+        _ptr(workspace), workspace.numel(), int(flags), _stream_handle(stream))
+    _check(status, "mdn_chunk_fwd")
+    return o, vt, S_T, M_T
+
+
+def step(q, k, v, alpha_log, mu_log, beta, eta, d: float, S: torch.Tensor, M: torch.Tensor,
+         *, o: Optional[torch.Tensor] = None, vtilde: Optional[torch.Tensor] = None,
+         want_vtilde: bool = True, stream: Optional[torch.cuda.Stream] = None):
+    """One decode token: S, M [B,H,d,d] float32 are updated in place.
+    q, k, v: [B,H,d]; gates [B,H].  Returns (o, vtilde or None)."""
+    B, H, D = q.shape
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, q.dtype, (B, H, D), name)
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (B, H), name)
+    _need(S, torch.float32, (B, H, D, D), "S")
+    _need(M, torch.float32, (B, H, D, D), "M")
+    if o is None:
+        o = torch.empty_like(q)
+    if vtilde is None and want_vtilde:
+        vtilde = torch.empty_like(q)
+    status = library().mdn_step(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta),
+        float(d), _ptr(S), _ptr(M), B, H, D, D, _ptr(o), _ptr(vtilde), 0, _stream_handle(stream))
+    _check(status, "mdn_step")
+    return o, vtilde
+
+
+def chunk_gate_prep(alpha_log, mu_log, beta, eta, C: int = 64, with_gamma: bool = True,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """Chunk coefficients: (la, lm, lc, b) [B,H,NT*C] and gamma [B,H,NT,C,C] (or None)."""
+    B, T, H = alpha_log.shape
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (B, T, H), name)
+    NT = (T + C - 1) // C
+    mk = lambda *s: torch.empty(s, dtype=torch.float32, device=alpha_log.device)
+    la, lm, lc, bco = (mk(B, H, NT * C) for _ in range(4))
+    gamma = mk(B, H, NT, C, C) if with_gamma else None
+    status = library().mdn_chunk_gate_prep(
+        _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta), B, T, H, C, _ptr(la), _ptr(lm),
+        _ptr(lc), _ptr(bco), _ptr(gamma), _stream_handle(stream))
+    _check(status, "mdn_chunk_gate_prep")
+    return la, lm, lc, bco, gamma
+
+
+def profile_enable(on: bool = True) -> bool:
+    """Start/stop per-kernel event timing inside the library (see mdn.h)."""
+    prev = library().mdn_profile_enable(1 if on else 0)
+    if prev < 0:
+        raise RuntimeError("mdn_profile_enable: could not create CUDA events")
+    return bool(prev)
+
+
+def profile_read(reset: bool = True) -> dict:
+    """{kernel name: (total device ms, launches)} since the last reset."""
+    import ctypes
+    cap = 32
+    names = (ctypes.c_char_p * cap)()
+    ms = (ctypes.c_double * cap)()
+    cnt = (ctypes.c_longlong * cap)()
+    n = library().mdn_profile_read(1 if reset else 0, names, ms, cnt, cap)
+    if n < 0:
+        raise RuntimeError("mdn_profile_read failed")
+    return {names[i].decode(): (ms[i], int(cnt[i])) for i in range(n)}

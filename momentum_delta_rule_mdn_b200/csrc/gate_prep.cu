@@ -1,0 +1,143 @@
+// K-1: chunk coefficients in the log domain (la, lm, lc, b) and Gamma.
+//
+// "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
+// paper.rainbus.top summary, step 5: every cumulative product of the chunk
+// (alphabar, mubar, c) is kept in the log domain, built with cumsum and
+// logcumsumexp.  One warp owns one chunk of 64 positions (two per lane); the
+// prefix sums and the log-sum-exp prefix are warp-shuffle scans.
+//
+// Positions past the end of the sequence act as steps that leave S and M
+// unchanged (alpha = mu = 1, beta = eta = 0), so a short last chunk needs no
+// special case downstream.
+//
+// Gamma_{r,i} = eta_i (alphabar_r / mubar_i)(c_r - c_{i-1}) is accumulated
+// down each column i by its first-order recurrence
+//     Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r exp(lm_r - lm_i),
+// a sum of non-negative terms.  Evaluating the difference c_r - c_{i-1} from
+// lc (the pages' log-broadcast) cancels catastrophically in fp32 when
+// mu/alpha < 1 over a run of tokens; the recurrence has no subtraction.
+#include "mdn_internal.cuh"
+
+namespace mdn {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_incl_sum(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(kFull, x, off);
+        if (lane >= off) x += y;
+    }
+    return x;
+}
+
+__device__ __forceinline__ float warp_incl_lse(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(kFull, x, off);
+        if (lane >= off) x = log_add_exp(x, y);
+    }
+    return x;
+}
+
+__global__ void __launch_bounds__(128)
+gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
+                 const float* __restrict__ beta, const float* __restrict__ eta,
+                 int B, int T, int H, int NT, float* __restrict__ la, float* __restrict__ lm,
+                 float* __restrict__ lc, float* __restrict__ bco, float* __restrict__ gamma)
+{
+    const int lane = threadIdx.x & 31;
+    const long long chunk = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (chunk >= (long long)B * H * NT) return;
+    const int n = (int)(chunk % NT);
+    const long long bh = chunk / NT;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+
+    // Positions 2*lane and 2*lane+1 of chunk n.
+    const int t0 = n * kChunk + 2 * lane;
+    float a[2] = {0.f, 0.f}, m[2] = {0.f, 0.f}, be[2] = {0.f, 0.f}, et[2] = {0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int t = t0 + e;
+        if (t < T) {
+            const size_t g = ((size_t)b * T + t) * H + h;
+            a[e] = alpha_log[g];
+            m[e] = mu_log[g];
+            be[e] = beta[g];
+            et[e] = eta[g];
+        }
+    }
+    // la, lm: inclusive prefix sums over the chunk.
+    const float sa = warp_incl_sum(a[0] + a[1], lane);
+    const float sm = warp_incl_sum(m[0] + m[1], lane);
+    float pa = __shfl_up_sync(kFull, sa, 1), pm = __shfl_up_sync(kFull, sm, 1);
+    if (lane == 0) pa = pm = 0.f;
+    float la_v[2], lm_v[2];
+    la_v[0] = pa + a[0];
+    la_v[1] = la_v[0] + a[1];
+    lm_v[0] = pm + m[0];
+    lm_v[1] = lm_v[0] + m[1];
+    // lc: logcumsumexp of x_j = log beta_j + lm_j - la_j  (beta = 0 -> -inf).
+    float x[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) x[e] = (be[e] > 0.f) ? logf(be[e]) + lm_v[e] - la_v[e] : -INFINITY;
+    const float sx = warp_incl_lse(log_add_exp(x[0], x[1]), lane);
+    float px = __shfl_up_sync(kFull, sx, 1);
+    if (lane == 0) px = -INFINITY;
+    float lc_v[2];
+    lc_v[0] = log_add_exp(px, x[0]);
+    lc_v[1] = log_add_exp(lc_v[0], x[1]);
+
+    const size_t row = (size_t)bh * NT * kChunk + (size_t)n * kChunk + 2 * lane;
+    reinterpret_cast<float2*>(la + row)[0] = make_float2(la_v[0], la_v[1]);
+    reinterpret_cast<float2*>(lm + row)[0] = make_float2(lm_v[0], lm_v[1]);
+    reinterpret_cast<float2*>(lc + row)[0] = make_float2(lc_v[0], lc_v[1]);
+    reinterpret_cast<float2*>(bco + row)[0] =
+        make_float2(expf(la_v[0] + lc_v[0]), expf(la_v[1] + lc_v[1]));
+
+    if (gamma == nullptr) return;
+    // Column recurrence; this lane owns columns i0 = lane and i1 = lane + 32.
+    const float ea[2] = {expf(a[0]), expf(a[1])};
+    const int i0 = lane, i1 = lane + 32;
+    // Position p sits in lane p/2, element p%2: fetch both elements, pick locally.
+    auto fetch = [&](const float (&x)[2], int p) {
+        const float e0 = __shfl_sync(kFull, x[0], p >> 1);
+        const float e1 = __shfl_sync(kFull, x[1], p >> 1);
+        return (p & 1) ? e1 : e0;
+    };
+    const float eta_i0 = fetch(et, i0), lm_i0 = fetch(lm_v, i0);
+    const float eta_i1 = fetch(et, i1), lm_i1 = fetch(lm_v, i1);
+    float g0 = 0.f, g1 = 0.f;
+    float* G = gamma + (size_t)chunk * kChunk * kChunk;
+    for (int r = 0; r < kChunk; ++r) {
+        const int src = r >> 1;
+        const bool odd = r & 1;
+        const float ar = __shfl_sync(kFull, odd ? ea[1] : ea[0], src);
+        const float br = __shfl_sync(kFull, odd ? be[1] : be[0], src);
+        const float lmr = __shfl_sync(kFull, odd ? lm_v[1] : lm_v[0], src);
+        g0 = (r >= i0) ? fmaf(ar, g0, eta_i0 * br * expf(lmr - lm_i0)) : 0.f;
+        g1 = (r >= i1) ? fmaf(ar, g1, eta_i1 * br * expf(lmr - lm_i1)) : 0.f;
+        G[r * kChunk + i0] = g0;
+        G[r * kChunk + i1] = g1;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
+                             const float* eta, int B, int T, int H, float* la, float* lm,
+                             float* lc, float* bco, float* gamma, cudaStream_t s)
+{
+    const int NT = (T + kChunk - 1) / kChunk;
+    const long long chunks = (long long)B * H * NT;
+    if (chunks == 0) return cudaSuccess;
+    const int warps_per_block = 4;
+    const long long blocks = (chunks + warps_per_block - 1) / warps_per_block;
+    ProfScope ps(kGatePrep, s);
+    gate_prep_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, s>>>(
+        alpha_log, mu_log, beta, eta, B, T, H, NT, la, lm, lc, bco, gamma);
+    return cudaGetLastError();
+}
+
+}  // namespace mdn

@@ -1,0 +1,241 @@
+// The C ABI of libmdn (see include/mdn.h): argument validation, workspace
+// layout and kernel dispatch.  Nothing here allocates device memory.
+#include <stdint.h>
+#include <string.h>
+
+#include "mdn_internal.cuh"
+
+using namespace mdn;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned_elem(const void* p, mdn_dtype dt) {
+    return (reinterpret_cast<uintptr_t>(p) & (dt == MDN_F32 ? 3u : 1u)) == 0;
+}
+
+struct WsLayout {
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, total;
+};
+
+// Byte offsets of every scratch region for these sizes.
+WsLayout ws_layout(long long BH, int NT, int D)
+{
+    const size_t rows = (size_t)BH * NT * kChunk;  // positions, padded to whole chunks
+    WsLayout w;
+    size_t off = 0;
+    w.status = off; off += align_up(64);
+    w.la = off;     off += align_up(rows * sizeof(float));
+    w.lm = off;     off += align_up(rows * sizeof(float));
+    w.lc = off;     off += align_up(rows * sizeof(float));
+    w.bco = off;    off += align_up(rows * sizeof(float));
+    w.gamma = off;  off += align_up(rows * kChunk * sizeof(float));
+    w.U = off;      off += align_up(rows * D * sizeof(float));
+    w.Y = off;      off += align_up(rows * D * sizeof(float));
+    w.Z = off;      off += align_up(rows * D * sizeof(float));
+    w.Oi = off;     off += align_up(rows * D * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+mdn_status check_sizes(int B, int T, int H, int dk, int dv, int C, mdn_dtype dt)
+{
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0 || C <= 0) return MDN_ERR_INVALID_ARG;
+    if (dt != MDN_F32 && dt != MDN_BF16) return MDN_ERR_UNSUPPORTED;
+    if (dk != dv) return MDN_ERR_UNSUPPORTED;
+    if (dk != 64 && dk != 128) return MDN_ERR_UNSUPPORTED;
+    if (C != kChunk) return MDN_ERR_UNSUPPORTED;
+    const long long NT = ((long long)T + C - 1) / C;
+    if ((long long)B * H * NT >= (1LL << 31) || (long long)B * H >= (1LL << 31) / 2)
+        return MDN_ERR_UNSUPPORTED;
+    return MDN_OK;
+}
+
+mdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDN_OK : MDN_ERR_CUDA; }
+
+}  // namespace
+
+// ---------------------------------------------------------------- finite check
+namespace mdn {
+namespace {
+__global__ void finite_check_kernel(const void* x, size_t n, bool bf16, unsigned* flag)
+{
+    unsigned bad = 0;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        if (bf16) {
+            const unsigned short u = static_cast<const unsigned short*>(x)[i];
+            bad |= ((u & 0x7f80u) == 0x7f80u);
+        } else {
+            bad |= !isfinite(static_cast<const float*>(x)[i]);
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(flag, 1u);
+}
+}  // namespace
+
+cudaError_t launch_finite_check(const void* x, size_t n, bool bf16, unsigned* flag,
+                                cudaStream_t s)
+{
+    if (n == 0) return cudaSuccess;
+    size_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    ProfScope ps(kFiniteCheck, s);
+    finite_check_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, n, bf16, flag);
+    return cudaGetLastError();
+}
+}  // namespace mdn
+
+// ---------------------------------------------------------------- exports
+extern "C" {
+
+int mdn_abi_version(void) { return kAbiVersion; }
+
+const char* mdn_status_string(mdn_status s)
+{
+    switch (s) {
+        case MDN_OK: return "MDN_OK";
+        case MDN_ERR_INVALID_ARG: return "MDN_ERR_INVALID_ARG: invalid argument";
+        case MDN_ERR_UNSUPPORTED: return "MDN_ERR_UNSUPPORTED: sizes or dtype outside this build's support";
+        case MDN_ERR_CUDA: return "MDN_ERR_CUDA: a CUDA launch or runtime call failed";
+        case MDN_ERR_NONFINITE: return "MDN_ERR_NONFINITE: an output holds NaN or Inf";
+        case MDN_ERR_TIMEOUT: return "MDN_ERR_TIMEOUT: a bounded device wait ran out";
+    }
+    return "unknown mdn_status";
+}
+
+size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    mdn_dtype in_dtype)
+{
+    if (check_sizes(B, T, H, dk, dv, C, in_dtype) != MDN_OK) return 0;
+    const int NT = (T + C - 1) / C;
+    return ws_layout((long long)B * H, NT, dk).total;
+}
+
+mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                         const float* alpha_log, const float* mu_log, const float* beta,
+                         const float* eta, float d_corr, const float* S0, const float* M0,
+                         int B, int T, int H, int dk, int dv, int C, void* o, void* vtilde,
+                         float* S_T, float* M_T, void* workspace, size_t ws_bytes, int flags,
+                         mdn_stream_t stream)
+{
+    mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
+    if (st != MDN_OK) return st;
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT)) return MDN_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return MDN_OK;
+    if (!S_T || !M_T || !aligned16(S_T) || !aligned16(M_T)) return MDN_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (M0 && !aligned16(M0))) return MDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = dk;
+    const size_t state_bytes = (size_t)B * H * D * D * sizeof(float);
+    if (T == 0) {
+        cudaError_t e = cudaSuccess;
+        if (S0) { if (S0 != S_T) e = cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, s); }
+        else e = cudaMemsetAsync(S_T, 0, state_bytes, s);
+        if (e == cudaSuccess) {
+            if (M0) { if (M0 != M_T) e = cudaMemcpyAsync(M_T, M0, state_bytes, cudaMemcpyDeviceToDevice, s); }
+            else e = cudaMemsetAsync(M_T, 0, state_bytes, s);
+        }
+        return cuda_status(e);
+    }
+    const void* tok[] = {q, k, v, o, vtilde};
+    for (const void* p : tok)
+        if (!p || !aligned16(p)) return MDN_ERR_INVALID_ARG;
+    const void* gates[] = {alpha_log, mu_log, beta, eta};
+    for (const void* p : gates)
+        if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MDN_ERR_INVALID_ARG;
+    const int NT = (T + C - 1) / C;
+    const WsLayout w = ws_layout((long long)B * H, NT, D);
+    if (ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
+
+    char* ws = static_cast<char*>(workspace);
+    ChunkArgs a;
+    a.q = q; a.k = k; a.v = v;
+    a.alpha_log = alpha_log; a.mu_log = mu_log; a.beta = beta; a.eta = eta;
+    a.dcorr = d_corr; a.S0 = S0; a.M0 = M0;
+    a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
+    a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
+    a.status = reinterpret_cast<unsigned*>(ws + w.status);
+    a.la = reinterpret_cast<float*>(ws + w.la);
+    a.lm = reinterpret_cast<float*>(ws + w.lm);
+    a.lc = reinterpret_cast<float*>(ws + w.lc);
+    a.bco = reinterpret_cast<float*>(ws + w.bco);
+    a.gamma = reinterpret_cast<float*>(ws + w.gamma);
+    a.U = reinterpret_cast<float*>(ws + w.U);
+    a.Y = reinterpret_cast<float*>(ws + w.Y);
+    a.Z = reinterpret_cast<float*>(ws + w.Z);
+    a.Oi = reinterpret_cast<float*>(ws + w.Oi);
+
+    cudaError_t e;
+    const bool check = flags & MDN_CHECK_FINITE;
+    if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return MDN_ERR_CUDA;
+    if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
+                              a.gamma, s)))
+        return MDN_ERR_CUDA;
+    if ((e = launch_chunk_simt(a, in_dtype, s))) return MDN_ERR_CUDA;
+    if (!check) return MDN_OK;
+
+    const size_t ntok = (size_t)B * T * H * D;
+    const bool bf = in_dtype == MDN_BF16;
+    if ((e = launch_finite_check(o, ntok, bf, a.status, s))) return MDN_ERR_CUDA;
+    if ((e = launch_finite_check(vtilde, ntok, bf, a.status, s))) return MDN_ERR_CUDA;
+    if ((e = launch_finite_check(S_T, (size_t)B * H * D * D, false, a.status, s))) return MDN_ERR_CUDA;
+    if ((e = launch_finite_check(M_T, (size_t)B * H * D * D, false, a.status, s))) return MDN_ERR_CUDA;
+    unsigned host_status[2] = {0, 0};
+    if ((e = cudaMemcpyAsync(host_status, a.status, sizeof(host_status), cudaMemcpyDeviceToHost, s)))
+        return MDN_ERR_CUDA;
+    if ((e = cudaStreamSynchronize(s))) return MDN_ERR_CUDA;
+    if (host_status[1]) return MDN_ERR_TIMEOUT;
+    if (host_status[0]) return MDN_ERR_NONFINITE;
+    return MDN_OK;
+}
+
+mdn_status mdn_step(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                    const float* alpha_log, const float* mu_log, const float* beta,
+                    const float* eta, float d_corr, float* S, float* M, int B, int H, int dk,
+                    int dv, void* o, void* vtilde, int flags, mdn_stream_t stream)
+{
+    mdn_status st = check_sizes(B, 1, H, dk, dv, kChunk, in_dtype);
+    if (st != MDN_OK) return st;
+    if (flags != 0) return MDN_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return MDN_OK;
+    const void* tok[] = {q, k, v, o};
+    for (const void* p : tok)
+        if (!p || !aligned_elem(p, in_dtype)) return MDN_ERR_INVALID_ARG;
+    if (vtilde && !aligned_elem(vtilde, in_dtype)) return MDN_ERR_INVALID_ARG;
+    const void* gates[] = {alpha_log, mu_log, beta, eta};
+    for (const void* p : gates)
+        if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    if (!S || !M || !aligned16(S) || !aligned16(M)) return MDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(launch_step(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S,
+                                   M, B, H, dk, o, vtilde, s));
+}
+
+mdn_status mdn_chunk_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
+                               const float* eta, int B, int T, int H, int C, float* la,
+                               float* lm, float* lc, float* b, float* gamma,
+                               mdn_stream_t stream)
+{
+    mdn_status st = check_sizes(B, T, H, 64, 64, C, MDN_F32);
+    if (st != MDN_OK) return st;
+    if (B == 0 || H == 0 || T == 0) return MDN_OK;
+    const void* gates[] = {alpha_log, mu_log, beta, eta};
+    for (const void* p : gates)
+        if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    const void* outs[] = {la, lm, lc, b};
+    for (const void* p : outs)
+        if (!p || (reinterpret_cast<uintptr_t>(p) & 7u)) return MDN_ERR_INVALID_ARG;
+    if (gamma && !aligned4(gamma)) return MDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, la, lm, lc, b,
+                                        gamma, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// K-5: one decode token, the stepwise recurrence applied in place.
+//
+// "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
+// paper.rainbus.top summary, step 1; ijyty.com article, section 6 (decoding
+// switches to the token-by-token recurrence):
+//   vtilde_j = v_j - alpha sum_i S_ij k_i
+//   M_ij <- mu M_ij - eta k_i vtilde_j
+//   S_ij <- alpha S_ij - beta M_ij
+//   o_j   = sum_i S_ij (q_i - d k_i)
+//
+// Bound by HBM: each state element is read once and written once.  Columns
+// are independent, so one block owns one (b, h) and 64 columns; a thread owns
+// RP rows x 4 adjacent columns (float4), so each row access of a warp-half is
+// 256 contiguous bytes.  The two column sums are block reductions in shared
+// memory.  All state loads are issued before the first reduction.
+#include "mdn_internal.cuh"
+
+namespace mdn {
+namespace {
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256)
+step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+            const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
+            const float* __restrict__ beta, const float* __restrict__ eta, float dcorr,
+            float* __restrict__ S, float* __restrict__ M, Tin* __restrict__ o,
+            Tin* __restrict__ vt_out)
+{
+    constexpr int NC = 64;          // columns per block
+    constexpr int CG = NC / 4;      // float4 column groups
+    constexpr int RG = 256 / CG;    // row groups
+    constexpr int RP = D / RG;      // rows per thread
+    constexpr int HALVES = D / NC;
+    __shared__ float ks[D], qs[D];
+    __shared__ float red[RG][NC + 4];
+    __shared__ float vts[NC];
+
+    const int tid = threadIdx.x;
+    const long long bh = blockIdx.x / HALVES;
+    const int col_base = (blockIdx.x % HALVES) * NC;
+    const int cg = tid % CG, rg = tid / CG;
+    const int col = col_base + cg * 4;
+
+    float* Sh = S + (size_t)bh * D * D;
+    float* Mh = M + (size_t)bh * D * D;
+    float4 s4[RP], m4[RP];
+#pragma unroll
+    for (int e = 0; e < RP; ++e) {
+        const int i = rg * RP + e;
+        s4[e] = __ldcs(reinterpret_cast<const float4*>(Sh + (size_t)i * D + col));
+        m4[e] = __ldcs(reinterpret_cast<const float4*>(Mh + (size_t)i * D + col));
+    }
+    const float alpha = expf(alpha_log[bh]);
+    const float mu = expf(mu_log[bh]);
+    const float be = beta[bh];
+    const float et = eta[bh];
+    for (int i = tid; i < D; i += 256) {
+        const float kv = ld_elem(k + (size_t)bh * D + i);
+        ks[i] = kv;
+        qs[i] = ld_elem(q + (size_t)bh * D + i) - dcorr * kv;
+    }
+    __syncthreads();
+
+    // vtilde = v - S^T (alpha k)
+    float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < RP; ++e) {
+        const float kv = ks[rg * RP + e];
+        p[0] = fmaf(s4[e].x, kv, p[0]);
+        p[1] = fmaf(s4[e].y, kv, p[1]);
+        p[2] = fmaf(s4[e].z, kv, p[2]);
+        p[3] = fmaf(s4[e].w, kv, p[3]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[rg][cg * 4 + c] = p[c];
+    __syncthreads();
+    if (tid < NC) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) s += red[g][tid];
+        const float vtj = ld_elem(v + (size_t)bh * D + col_base + tid) - alpha * s;
+        vts[tid] = vtj;
+        if (vt_out) st_elem(vt_out + (size_t)bh * D + col_base + tid, vtj);
+    }
+    __syncthreads();
+
+    float vv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) vv[c] = vts[cg * 4 + c];
+    float po[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < RP; ++e) {
+        const int i = rg * RP + e;
+        const float ek = et * ks[i];
+        const float qv = qs[i];
+        float* sp = &s4[e].x;
+        float* mp = &m4[e].x;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float mnew = fmaf(mu, mp[c], -ek * vv[c]);
+            const float snew = fmaf(alpha, sp[c], -be * mnew);
+            mp[c] = mnew;
+            sp[c] = snew;
+            po[c] = fmaf(snew, qv, po[c]);
+        }
+        __stcs(reinterpret_cast<float4*>(Sh + (size_t)i * D + col), s4[e]);
+        __stcs(reinterpret_cast<float4*>(Mh + (size_t)i * D + col), m4[e]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) red[rg][cg * 4 + c] = po[c];
+    __syncthreads();
+    if (tid < NC) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) s += red[g][tid];
+        st_elem(o + (size_t)bh * D + col_base + tid, s);
+    }
+}
+
+template <typename Tin, int D>
+cudaError_t launch_step_typed(const void* q, const void* k, const void* v,
+                              const float* alpha_log, const float* mu_log, const float* beta,
+                              const float* eta, float dcorr, float* S, float* M, int B, int H,
+                              void* o, void* vt, cudaStream_t s)
+{
+    const long long blocks = (long long)B * H * (D / 64);
+    if (blocks == 0) return cudaSuccess;
+    ProfScope ps(kStep, s);
+    step_kernel<Tin, D><<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
+        alpha_log, mu_log, beta, eta, dcorr, S, M, static_cast<Tin*>(o), static_cast<Tin*>(vt));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
+                        const float* alpha_log, const float* mu_log, const float* beta,
+                        const float* eta, float dcorr, float* S, float* M, int B, int H,
+                        int D, void* o, void* vt, cudaStream_t s)
+{
+    if (dt == MDN_F32)
+        return D == 64 ? launch_step_typed<float, 64>(q, k, v, alpha_log, mu_log, beta, eta,
+                                                      dcorr, S, M, B, H, o, vt, s)
+                       : launch_step_typed<float, 128>(q, k, v, alpha_log, mu_log, beta, eta,
+                                                       dcorr, S, M, B, H, o, vt, s);
+    return D == 64 ? launch_step_typed<__nv_bfloat16, 64>(q, k, v, alpha_log, mu_log, beta, eta,
+                                                          dcorr, S, M, B, H, o, vt, s)
+                   : launch_step_typed<__nv_bfloat16, 128>(q, k, v, alpha_log, mu_log, beta,
+                                                           eta, dcorr, S, M, B, H, o, vt, s);
+}
+
+}  // namespace mdn

@@ -1,0 +1,119 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/*.h declares, and its host-side validation rejects bad arguments
+before touching the device."""
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from momentum_delta_rule_mdn_b200 import _lib, build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return _lib.load()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(mdn_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("mdn_chunk_fwd", "mdn_step", "mdn_chunk_fwd_workspace_size", "mdn_status_string",
+              "mdn_chunk_gate_prep", "mdn_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mdn_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert set(_lib.SIGNATURES) <= exported
+
+
+def test_status_strings(lib):
+    assert lib.mdn_abi_version() == 1
+    for s in range(6):
+        assert lib.mdn_status_string(s).decode().startswith("MDN_")
+    assert b"unknown" in lib.mdn_status_string(99)
+
+
+def test_workspace_size_rules(lib):
+    ws = lib.mdn_chunk_fwd_workspace_size
+    assert ws(8, 4096, 16, 128, 128, 64, _lib.MDN_BF16) > 0
+    assert ws(1, 0, 1, 64, 64, 64, _lib.MDN_F32) > 0
+    assert ws(1, 256, 1, 96, 96, 64, _lib.MDN_F32) == 0      # unsupported d
+    assert ws(1, 256, 1, 64, 128, 64, _lib.MDN_F32) == 0     # d_k != d_v
+    assert ws(1, 256, 1, 64, 64, 32, _lib.MDN_F32) == 0      # unsupported C
+    assert ws(-1, 256, 1, 64, 64, 64, _lib.MDN_F32) == 0
+    assert ws(1, 256, 1, 64, 64, 64, 7) == 0                 # unknown dtype
+    # grows with T and covers whole chunks of a ragged tail
+    assert ws(1, 65, 1, 64, 64, 64, 0) == ws(1, 128, 1, 64, 64, 64, 0)
+    assert ws(1, 129, 1, 64, 64, 64, 0) > ws(1, 128, 1, 64, 64, 64, 0)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=_lib.MDN_BF16, al=FAKE, ml=FAKE, be=FAKE, et=FAKE,
+             d=0.5, S0=None, M0=None, B=1, T=128, H=1, dk=64, dv=64, C=64, o=FAKE, vt=FAKE,
+             ST=FAKE, MT=FAKE, ws=FAKE, wsb=0, flags=0)
+    a.update(kw)
+    return lib.mdn_chunk_fwd(a["q"], a["k"], a["v"], a["dt"], a["al"], a["ml"], a["be"],
+                             a["et"], a["d"], a["S0"], a["M0"], a["B"], a["T"], a["H"],
+                             a["dk"], a["dv"], a["C"], a["o"], a["vt"], a["ST"], a["MT"],
+                             a["ws"], a["wsb"], a["flags"], None)
+
+
+def test_chunk_fwd_validation(lib):
+    E = _lib
+    assert _chunk(lib, dk=96, dv=96) == E.MDN_ERR_UNSUPPORTED
+    assert _chunk(lib, C=32) == E.MDN_ERR_UNSUPPORTED
+    assert _chunk(lib, dt=5) == E.MDN_ERR_UNSUPPORTED
+    assert _chunk(lib, B=-1) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, C=0) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, flags=0x100) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, q=None) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, vt=None) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, ST=None) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, k=FAKE + 4) == E.MDN_ERR_INVALID_ARG           # unaligned
+    assert _chunk(lib, al=FAKE + 2) == E.MDN_ERR_INVALID_ARG          # gate not 4-byte aligned
+    assert _chunk(lib, ws=FAKE + 16) == E.MDN_ERR_INVALID_ARG         # workspace not 256-aligned
+    need = lib.mdn_chunk_fwd_workspace_size(1, 128, 1, 64, 64, 64, _lib.MDN_BF16)
+    assert _chunk(lib, wsb=need - 1) == E.MDN_ERR_INVALID_ARG         # workspace too small
+    assert _chunk(lib, B=0) == E.MDN_OK                               # nothing to do
+    assert _chunk(lib, H=0, q=None) == E.MDN_OK
+
+
+def test_step_and_gate_prep_validation(lib):
+    E = _lib
+    st = lambda **kw: lib.mdn_step(kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 1), FAKE, FAKE,
+                                   FAKE, FAKE, 0.5, kw.get("S", FAKE), FAKE, kw.get("B", 2), 3,
+                                   kw.get("d", 128), kw.get("d", 128), FAKE, None,
+                                   kw.get("flags", 0), None)
+    assert st(d=32) == E.MDN_ERR_UNSUPPORTED
+    assert st(q=None) == E.MDN_ERR_INVALID_ARG
+    assert st(S=FAKE + 8) == E.MDN_ERR_INVALID_ARG
+    assert st(q=FAKE + 1) == E.MDN_ERR_INVALID_ARG                   # bf16 needs 2-byte alignment
+    assert st(flags=1) == E.MDN_ERR_INVALID_ARG
+    assert st(B=0) == E.MDN_OK
+    gp = lambda **kw: lib.mdn_chunk_gate_prep(FAKE, FAKE, FAKE, FAKE, 1, kw.get("T", 100), 1,
+                                              kw.get("C", 64), kw.get("la", FAKE), FAKE, FAKE,
+                                              FAKE, None, None)
+    assert gp(C=16) == E.MDN_ERR_UNSUPPORTED
+    assert gp(la=None) == E.MDN_ERR_INVALID_ARG
+    assert gp(T=0) == E.MDN_OK
