@@ -158,6 +158,41 @@ mdn_status mdn_chunk_gate_prep(const float *alpha_log, const float *mu_log,
                                mdn_stream_t stream);
 
 /*
+ * mdn_chunk_fwd without a caller-supplied workspace.  The paper has no
+ * counterpart: this is a deployment aid of this library.
+ *
+ * Some callers cannot call cudaMalloc or hand out scratch memory: for example
+ * a plug-in that runs inside another runtime's execution phase, where that
+ * runtime owns all device memory and forbids allocation there, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation.  Such callers still own and pass q, k, v, the gates, the
+ * states and the outputs; only the scratch space comes from the library.
+ *
+ * The scratch is one fixed array of 64 MiB in device memory per GPU, created
+ * when the library is loaded on that GPU and held until the process exits.
+ * Arguments and results are exactly those of mdn_chunk_fwd (minus workspace
+ * and ws_bytes).  Sizes whose scratch need, mdn_chunk_fwd_workspace_size(...),
+ * exceeds 64 MiB are rejected with MDN_ERR_UNSUPPORTED before anything runs.
+ *
+ * - The scratch of the CURRENT device is used; `stream` must belong to it.
+ * - The first call on a device looks up the array's device address (a
+ *   one-time set-up, no allocation); make that first call before any stream
+ *   capture is begun on the device.
+ * - All calls on a device share the one array and it keeps the last call's
+ *   contents.  The pass never relies on them, but calls that overlap on the
+ *   GPU (e.g. on two unordered streams) race on the array and corrupt each
+ *   other's results: order such calls on one stream or with events.
+ * - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+mdn_status mdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 mdn_dtype in_dtype, const float *alpha_log,
+                                 const float *mu_log, const float *beta, const float *eta,
+                                 float d_corr, const float *S0, const float *M0,
+                                 int B, int T, int H, int dk, int dv, int C,
+                                 void *o, void *vtilde, float *S_T, float *M_T,
+                                 int flags, mdn_stream_t stream);
+
+/*
  * Optional per-kernel timing (no counterpart in the method; a measurement aid).
  * mdn_profile_enable(1) makes every later kernel launch of the library record a
  * CUDA event pair on its launch stream (the events are created on the first

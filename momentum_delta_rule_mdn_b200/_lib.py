@@ -26,6 +26,8 @@ SIGNATURES = {
                       _i, _i, _i, _i, _vp, _vp, _i, _vp]),
     "mdn_chunk_gate_prep": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                  _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mdn_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                   _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp]),
     "mdn_profile_enable": (_i, [_i]),
     "mdn_profile_read": (_i, [_i, ctypes.POINTER(ctypes.c_char_p),
                               ctypes.POINTER(ctypes.c_double),
