@@ -228,6 +228,7 @@ def run_ours(args, rank, world, device):
 
     # ---- end to end through the public call, host (pinned) buffers
     e2e = run_e2e(args, mdn, inp, tok, spec, device, world)
+    decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -247,7 +248,41 @@ def run_ours(args, rank, world, device):
         "e2e": e2e,
         "clocks": clk.summary(),
     }
+    if decode:
+        line["decode"] = decode
     return line, spec
+
+
+def run_decode(args, mdn, device, hbm_peak):
+    """mdn_step at the decode workload's shape (B=256, H=16, d=128): S and M
+    (2 x 268 MB fp32) are read and written once per token, so no L2 flush is
+    needed.  Reports tokens/s and the kernel's HBM fraction."""
+    spec = mi.CONFIGS[4]
+    B, H, d = spec.B, spec.H, spec.d
+    tok = mi.make_inputs(mi.replace(spec, T=1, seed=spec.seed + 11))
+    t = {k: v[:, 0].contiguous() for k, v in mi.to_torch(tok, device).items() if v is not None}
+    S = torch.randn((B, H, d, d), device=device) * 0.01
+    M = torch.randn((B, H, d, d), device=device) * 0.01
+    o = torch.empty_like(t["q"])
+    gates = ("alpha_log", "mu_log", "beta", "eta")
+    for _ in range(3):
+        mdn.step(t["q"], t["k"], t["v"], *(t[g] for g in gates), spec.q_corr, S, M, o=o,
+                 want_vtilde=False)
+    n = max(5, min(args.steps, 50))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        mdn.step(t["q"], t["k"], t["v"], *(t[g] for g in gates), spec.q_corr, S, M, o=o,
+                 want_vtilde=False)
+    b.record()
+    torch.cuda.synchronize()
+    sec = a.elapsed_time(b) / n * 1e-3
+    _, bytes_per_step, _ = kernel_work("step", spec)
+    gbs = bytes_per_step / sec / 1e9
+    return {"workload": spec.name, "tokens_per_s": round(B / sec, 1),
+            "us_per_step": round(sec * 1e6, 2), "achieved_gbs": round(gbs, 1),
+            "peak_gbs": hbm_peak, "frac": round(gbs / hbm_peak, 4), "steps": n}
 
 
 def run_e2e(args, mdn, inp, tok, spec, device, world):
@@ -412,6 +447,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-shape measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

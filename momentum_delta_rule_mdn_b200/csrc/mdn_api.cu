@@ -20,7 +20,7 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, total;
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, total;
 };
 
 // Byte offsets of every scratch region for these sizes.
@@ -39,6 +39,7 @@ WsLayout ws_layout(long long BH, int NT, int D)
     w.Y = off;      off += align_up(rows * D * sizeof(float));
     w.Z = off;      off += align_up(rows * D * sizeof(float));
     w.Oi = off;     off += align_up(rows * D * sizeof(float));
+    w.rec = off;    off += align_up(rows * 6 * sizeof(float));
     w.total = off;
     return w;
 }
@@ -171,14 +172,20 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.Y = reinterpret_cast<float*>(ws + w.Y);
     a.Z = reinterpret_cast<float*>(ws + w.Z);
     a.Oi = reinterpret_cast<float*>(ws + w.Oi);
+    a.rec = reinterpret_cast<float*>(ws + w.rec);
 
     cudaError_t e;
     const bool check = flags & MDN_CHECK_FINITE;
     if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return MDN_ERR_CUDA;
-    if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
-                              a.gamma, s)))
-        return MDN_ERR_CUDA;
-    if ((e = launch_chunk_simt(a, in_dtype, s))) return MDN_ERR_CUDA;
+    const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
+    if (tensor_cores) {
+        if ((e = launch_chunk_tc(a, s))) return MDN_ERR_CUDA;
+    } else {
+        if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
+                                  a.gamma, s)))
+            return MDN_ERR_CUDA;
+        if ((e = launch_chunk_simt(a, in_dtype, s))) return MDN_ERR_CUDA;
+    }
     if (!check) return MDN_OK;
 
     const size_t ntok = (size_t)B * T * H * D;

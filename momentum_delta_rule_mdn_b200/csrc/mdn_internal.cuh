@@ -53,6 +53,8 @@ struct ChunkArgs {
     float* Y;
     float* Z;
     float* Oi;         // [B*H, NT*C, D]  carried-state part of o
+    float* rec;        // [B*H*NT, 6, C]  packed coefficients (tensor-core path)
+    float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
 };
 
 // Kernel kinds known to the optional timing facility (profile.cu).
@@ -75,7 +77,12 @@ struct ProfScope {
 cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
                              const float* eta, int B, int T, int H, float* la, float* lm,
                              float* lc, float* bco, float* gamma, cudaStream_t s);
+cudaError_t launch_gate_pack(const float* alpha_log, const float* mu_log, const float* beta,
+                             const float* eta, int B, int T, int H, float* rec, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
+// Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
+// when the arguments are outside what it handles.
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
                         const float* eta, float dcorr, float* S, float* M, int B, int H,
