@@ -60,9 +60,12 @@ def kernel_work(name: str, spec: mi.Spec):
     d, C = spec.d, spec.C
     heads = spec.B * spec.H
     states = 2 * heads * d * d * 4 * (2 if spec.state_std > 0 else 1)  # S_T,M_T (+S0,M0)
-    if name in ("chunk_tc", "inter_tc"):
-        # whole pass: q,k,v,o,vtilde bf16 + 4 fp32 gates, plus states
-        return "hbm", th * (5 * d * 2 + 16) + states, "GB/s"
+    if name == "inter_tc":
+        # the bytes it must move: q, k, v read and o, vtilde written (bf16), plus the states
+        return "hbm", th * (5 * d * 2) + states, "GB/s"
+    if name == "intra_tc":
+        # q, k read; T and Att (bf16 C x C per chunk) written
+        return "hbm", th * (2 * d * 2 + 2 * C * 2), "GB/s"
     if name == "inter_simt":
         return "alu", th * 12.0 * d * d, "TFLOP/s"
     if name == "intra_simt":
@@ -234,7 +237,7 @@ def run_ours(args, rank, world, device):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if "chunk_tc" in kernels else "f32",
+        "dtype": "bf16" if "inter_tc" in kernels else "f32",
         "data": "synthetic (seeded generator; gates from the stable parameterisation)",
         "config": {"workload": spec0.name, "B": B, "T": T, "H": H, "d_k": d, "d_v": d,
                    "C": spec.C, "inputs": spec.dtype, "state": "fp32",

@@ -1,0 +1,333 @@
+// K-2 on sm_100a: the intra-chunk part of the chunkwise MDN forward pass,
+// one CTA per chunk, all chunks in parallel.
+//
+// "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
+// paper.rainbus.top summary, steps 3-5.  Per chunk (positions r, i inside it):
+//   G      = [K; Qhat] [K; Qhat]^T     tcgen05.mma, M=128, N=128, K=128, bf16 in, fp32 in TMEM
+//            lane i < 64: k_i.k_r (cols 0..63);  lane 64+r: qhat_r.k_i (cols 0..63)
+//   Gamma  down each column i by Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r mubar_r/mubar_i
+//          (mubar_r/mubar_i as a running product of mu: non-negative terms only)
+//   A      = (P K^T) o Gamma-:  A_{r,i} = alpha_r k_r.k_i Gamma_{r-1,i}  (i < r)
+//   Att    = (Qhat K^T) o Gamma:  Att_{r,i} = qhat_r.k_i Gamma_{r,i}  (i <= r)
+//   T      = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution, then the
+//            off-diagonal blocks by distance from the diagonal, fp32.
+// Writes T and Att (bf16, row-major 64 x 64 per chunk) and Gamma_{C,.} (the
+// last row of Gamma, into row 6 of the chunk's coefficient record).  The
+// inter-chunk kernel turns them into its operands.
+#include "mdn_internal.cuh"
+#include "tc_common.cuh"
+
+namespace mdn {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int kThreads = 128;
+constexpr uint32_t KQ = 0;                  // [K; Qhat], 2 feature panels x (128 rows x 128 B)
+constexpr uint32_t GM = 32768;              // fp32 [64][LDF] Gamma
+constexpr uint32_t AM = GM + 64 * LDF * 4;  // fp32 [64][LDF] A (upper blocks: solve scratch)
+constexpr uint32_t TMF = AM + 64 * LDF * 4; // fp32 [64][LDF] T
+constexpr uint32_t REC = TMF + 64 * LDF * 4;// record rows 0..5
+constexpr uint32_t MU = REC + 1536;         // mu_r
+constexpr uint32_t BARS = MU + 256;
+constexpr uint32_t MISC = BARS + 16;
+constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTxBytes = 32768 + 1536;
+
+struct IntraArgs {
+    float* rec;            // [chunks][7][64]: rows 0..5 read, row 6 written
+    __nv_bfloat16* tmat;   // [chunks][64][64]
+    __nv_bfloat16* att;    // [chunks][64][64]
+    unsigned* status;
+    float* dbg;            // diagnostics: phase clocks of CTA 0 (null in normal use)
+    float dcorr;
+    int H, NT;
+};
+
+__global__ void __launch_bounds__(kThreads)
+chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const IntraArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const long long chunk = blockIdx.x;
+    const int n = (int)(chunk % a.NT);
+    const long long bh = chunk / a.NT;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BARS);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
+    float* Gm = reinterpret_cast<float*>(sm + GM);
+    float* Am = reinterpret_cast<float*>(sm + AM);
+    float* Tm = reinterpret_cast<float*>(sm + TMF);
+    const float* rec = reinterpret_cast<const float*>(sm + REC);
+    float* mu = reinterpret_cast<float*>(sm + MU);
+    PhaseClock clk;
+    clk.start((a.dbg && chunk == 0 && tid == 0) ? a.dbg : nullptr);
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+        mbar_arrive_expect_tx(&bars[0], kTxBytes);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_4d(sm + KQ + p * 16384, &tm_k, p * 64, h, n * C, b, &bars[0]);
+            tma_load_4d(sm + KQ + p * 16384 + 8192, &tm_q, p * 64, h, n * C, b, &bars[0]);
+        }
+        bulk_load(sm + REC, a.rec + chunk * kRecFloats, 1536, &bars[0]);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
+
+    bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
+    clk.lap(0);
+    if (ok) {
+        // Qhat = Q - d K in place (rows 64..127 of both panels)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = tid + 128 * u;
+            const int pn = idx >> 9, w = idx & 511, r = w >> 3, c = w & 7;
+            const uint4 kw = *reinterpret_cast<const uint4*>(sm + KQ + pn * 16384 + sw128_off(r, c));
+            uint8_t* qp = sm + KQ + pn * 16384 + sw128_off(r + 64, c);
+            float kx[8], qx[8];
+            unpack_bf16x8(kw, kx);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(qp), qx);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qx[e] -= a.dcorr * kx[e];
+            st_bf16x8(qp, qx);
+        }
+        if (tid < C) {
+            const float* lm = rec + C;
+            mu[tid] = expf(lm[tid] - (tid > 0 ? lm[tid - 1] : 0.f));
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        clk.lap(1);
+        if (tid == 0) {
+            tc_fence_after_sync();
+            const uint32_t id = idesc_bf16(128, 128, false, false);
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad =
+                    smem_desc(sbase + KQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128);
+                mma_bf16(tmem, ad, ad, id, ks > 0);
+            }
+            mma_commit(&bars[1]);
+        }
+        ok = mbar_wait(&bars[1], 0);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok);
+        clk.lap(2);
+    }
+    if (ok) {
+        // lane i < 64: k_i.k_r;  lane 64 + r: qhat_r.k_i   (columns 0..63)
+        float gv[64];
+        tmem_ld32(tmem + lane_sel, *reinterpret_cast<float(*)[32]>(gv));
+        tmem_ld32(tmem + lane_sel + 32, *reinterpret_cast<float(*)[32]>(gv + 32));
+        tmem_wait_ld();
+        if (tid < C) {
+            // column i of Gamma and A
+            const int i = tid;
+            const float* al = rec + 3 * C;
+            const float* be = rec + 4 * C;
+            const float eta_i = rec[5 * C + i];
+            float gam = 0.f, f = 1.f;
+#pragma unroll
+            for (int r4 = 0; r4 < C; r4 += 4) {
+                const float4 a4 = lds4(al + r4), b4 = lds4(be + r4), m4 = lds4(mu + r4);
+                const float ar_[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float br_[4] = {b4.x, b4.y, b4.z, b4.w};
+                const float mr_[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r4 + e;
+                    Am[r * LDF + i] = (r > i) ? ar_[e] * gv[r] * gam : 0.f;
+                    f = (r > i) ? f * mr_[e] : 1.f;
+                    gam = (r >= i) ? fmaf(ar_[e], gam, eta_i * br_[e] * f) : 0.f;
+                    Gm[r * LDF + i] = gam;
+                }
+            }
+            a.rec[chunk * kRecFloats + 6 * C + i] = gam;  // Gamma_{C,i}
+        } else {
+            // zero the six blocks of T above the diagonal
+            for (int idx = tid - C; idx < 6 * 64; idx += 64) {
+                const int blkid = idx >> 6, e = idx & 63;
+                const int bi = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
+                const int bj = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
+                *reinterpret_cast<float4*>(Tm + (16 * bi + (e >> 2)) * LDF + 16 * bj + 4 * (e & 3)) =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        __syncthreads();
+        clk.lap(3);
+        if (tid >= C) {
+            // row r of Att, straight to global memory
+            const int r = tid - C;
+            uint4* dst = reinterpret_cast<uint4*>(a.att + (chunk * C + r) * C);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 g0 = lds4(Gm + r * LDF + 8 * c), g1 = lds4(Gm + r * LDF + 8 * c + 4);
+                const float gr[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= r) ? gv[8 * c + e] * gr[e] : 0.f;
+                dst[c] = bf16x8(x);
+            }
+        } else {
+            // diagonal 16x16 blocks of T by forward substitution, one column per thread
+            const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) t[r] = (r == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int r = 1; r < 16; ++r) {
+                float av[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 v4 = lds4(Am + (o + r) * LDF + o + 4 * q4);
+                    av[4 * q4] = v4.x;
+                    av[4 * q4 + 1] = v4.y;
+                    av[4 * q4 + 2] = v4.z;
+                    av[4 * q4 + 3] = v4.w;
+                }
+                float acc = 0.f;
+#pragma unroll
+                for (int k = 0; k < r; ++k) acc = fmaf(av[k], t[k], acc);
+                if (r > c) t[r] = -acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tm[(o + r) * LDF + o + c] = t[r];
+        }
+        __syncthreads();
+        clk.lap(4);
+        // Off-diagonal blocks by distance L: W = sum_{k=j}^{i-1} A_{i,k} T_{k,j},
+        // T_{i,j} = -T_{i,i} W (j = i - L).  W goes to block (L-1, i) of Am.  A
+        // thread owns a 2 x 4 tile of a block.
+        for (int L = 1; L < 4; ++L) {
+            const int tasks = (4 - L) * 32;
+            const int task = tid;
+            const bool mine = task < tasks;
+            const int i = L + (task >> 5), j = i - L, r0 = 2 * ((task >> 2) & 7), c4 = task & 3;
+            if (mine) {
+                float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+                for (int kb = j; kb < i; ++kb) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 a0 = lds4(Am + (16 * i + r0) * LDF + 16 * kb + 4 * k4);
+                        const float4 a1 = lds4(Am + (16 * i + r0 + 1) * LDF + 16 * kb + 4 * k4);
+                        const float x0[4] = {a0.x, a0.y, a0.z, a0.w};
+                        const float x1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float4 t4 = lds4(Tm + (16 * kb + 4 * k4 + e) * LDF + 16 * j + 4 * c4);
+                            acc0.x = fmaf(x0[e], t4.x, acc0.x);
+                            acc0.y = fmaf(x0[e], t4.y, acc0.y);
+                            acc0.z = fmaf(x0[e], t4.z, acc0.z);
+                            acc0.w = fmaf(x0[e], t4.w, acc0.w);
+                            acc1.x = fmaf(x1[e], t4.x, acc1.x);
+                            acc1.y = fmaf(x1[e], t4.y, acc1.y);
+                            acc1.z = fmaf(x1[e], t4.z, acc1.z);
+                            acc1.w = fmaf(x1[e], t4.w, acc1.w);
+                        }
+                    }
+                }
+                float* w = Am + (16 * (L - 1) + r0) * LDF + 16 * i + 4 * c4;
+                *reinterpret_cast<float4*>(w) = acc0;
+                *reinterpret_cast<float4*>(w + LDF) = acc1;
+            }
+            __syncthreads();
+            if (mine) {
+                float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 t0 = lds4(Tm + (16 * i + r0) * LDF + 16 * i + 4 * k4);
+                    const float4 t1 = lds4(Tm + (16 * i + r0 + 1) * LDF + 16 * i + 4 * k4);
+                    const float x0[4] = {t0.x, t0.y, t0.z, t0.w};
+                    const float x1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 w4 =
+                            lds4(Am + (16 * (L - 1) + 4 * k4 + e) * LDF + 16 * i + 4 * c4);
+                        acc0.x = fmaf(x0[e], w4.x, acc0.x);
+                        acc0.y = fmaf(x0[e], w4.y, acc0.y);
+                        acc0.z = fmaf(x0[e], w4.z, acc0.z);
+                        acc0.w = fmaf(x0[e], w4.w, acc0.w);
+                        acc1.x = fmaf(x1[e], w4.x, acc1.x);
+                        acc1.y = fmaf(x1[e], w4.y, acc1.y);
+                        acc1.z = fmaf(x1[e], w4.z, acc1.z);
+                        acc1.w = fmaf(x1[e], w4.w, acc1.w);
+                    }
+                }
+                float* t = Tm + (16 * i + r0) * LDF + 16 * j + 4 * c4;
+                *reinterpret_cast<float4*>(t) = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
+                *reinterpret_cast<float4*>(t + LDF) = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
+            }
+            __syncthreads();
+        }
+        clk.lap(5);
+        // T to global memory (bf16, row-major): thread = (row, half)
+        {
+            const int r = tid >> 1, hf = tid & 1;
+            uint4* dst = reinterpret_cast<uint4*>(a.tmat + (chunk * C + r) * C + 32 * hf);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float4 t0 = lds4(Tm + r * LDF + 32 * hf + 8 * c);
+                const float4 t1 = lds4(Tm + r * LDF + 32 * hf + 8 * c + 4);
+                const float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                dst[c] = bf16x8(x);
+            }
+        }
+        clk.lap(6);
+    }
+    if (!ok && tid == 0) {
+        atomicOr(a.status + 1, 1u);
+        (void)mbar_wait(&bars[0], 0);  // the loads must land before shared memory goes away
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
+{
+    CUtensorMap mq, mk;
+    if (!make_token_map(&mq, a.q, a.B, a.T, a.H, 64, true) ||
+        !make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true))
+        return cudaErrorInvalidValue;
+    IntraArgs t;
+    t.rec = a.rec;
+    t.tmat = a.tmat;
+    t.att = a.att;
+    t.status = a.status;
+    t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
+    t.dcorr = a.dcorr;
+    t.H = a.H;
+    t.NT = a.NT;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_intra_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    ProfScope ps(kIntraTc, s);
+    chunk_intra_kernel<<<(unsigned)chunks, kThreads, SMEM_BYTES, s>>>(mq, mk, t);
+    return cudaGetLastError();
+}
+
+}  // namespace mdn

@@ -123,9 +123,10 @@ gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
     }
 }
 
-// Packed per-chunk coefficient record for the tensor-core path: six rows of
-// 64 floats, [la | lm | b | alpha | beta | eta], positions past T holding the
-// values of steps that leave the state unchanged.  One bulk copy per chunk.
+// Packed per-chunk coefficient record for the tensor-core path: seven rows of
+// 64 floats, [la | lm | b | alpha | beta | eta | Gamma_{C,.}]; this kernel
+// writes the first six (the intra-chunk kernel writes the last), positions past
+// T holding the values of steps that leave the state unchanged.
 __global__ void __launch_bounds__(128)
 gate_pack_kernel(const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
                  const float* __restrict__ beta, const float* __restrict__ eta,
@@ -169,7 +170,7 @@ gate_pack_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
     lc_v[0] = log_add_exp(px, x[0]);
     lc_v[1] = log_add_exp(lc_v[0], x[1]);
 
-    float2* r = reinterpret_cast<float2*>(rec + (size_t)chunk * 6 * kChunk) + lane;
+    float2* r = reinterpret_cast<float2*>(rec + (size_t)chunk * 7 * kChunk) + lane;
     r[0 * kChunk / 2] = make_float2(la_v[0], la_v[1]);
     r[1 * kChunk / 2] = make_float2(lm_v[0], lm_v[1]);
     r[2 * kChunk / 2] = make_float2(expf(la_v[0] + lc_v[0]), expf(la_v[1] + lc_v[1]));

@@ -20,7 +20,7 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, total;
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, tmat, att, total;
 };
 
 // Byte offsets of every scratch region for these sizes.
@@ -39,7 +39,9 @@ WsLayout ws_layout(long long BH, int NT, int D)
     w.Y = off;      off += align_up(rows * D * sizeof(float));
     w.Z = off;      off += align_up(rows * D * sizeof(float));
     w.Oi = off;     off += align_up(rows * D * sizeof(float));
-    w.rec = off;    off += align_up(rows * 6 * sizeof(float));
+    w.rec = off;    off += align_up(rows * 7 * sizeof(float));
+    w.tmat = off;   off += align_up(rows * kChunk * 2);
+    w.att = off;    off += align_up(rows * kChunk * 2);
     w.total = off;
     return w;
 }
@@ -173,6 +175,8 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.Z = reinterpret_cast<float*>(ws + w.Z);
     a.Oi = reinterpret_cast<float*>(ws + w.Oi);
     a.rec = reinterpret_cast<float*>(ws + w.rec);
+    a.tmat = reinterpret_cast<__nv_bfloat16*>(ws + w.tmat);
+    a.att = reinterpret_cast<__nv_bfloat16*>(ws + w.att);
 
     cudaError_t e;
     const bool check = flags & MDN_CHECK_FINITE;

@@ -53,7 +53,9 @@ struct ChunkArgs {
     float* Y;
     float* Z;
     float* Oi;         // [B*H, NT*C, D]  carried-state part of o
-    float* rec;        // [B*H*NT, 6, C]  packed coefficients (tensor-core path)
+    float* rec;        // [B*H*NT, 7, C]  packed coefficients (tensor-core path)
+    __nv_bfloat16* tmat;  // [B*H*NT, C, C]  T = (I + A)^{-1}, bf16 (tensor-core path)
+    __nv_bfloat16* att;   // [B*H*NT, C, C]  (Qhat K^T) o Gamma, bf16 (tensor-core path)
     float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
 };
 
@@ -83,6 +85,8 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s);
+cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s);
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
                         const float* eta, float dcorr, float* S, float* M, int B, int H,
