@@ -3,6 +3,7 @@
 //
 // "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
 // paper.rainbus.top summary, steps 3-5.  Per chunk (positions r, i inside it):
+//   Qhat   = Q - d K
 //   G      = [K; Qhat] [K; Qhat]^T     tcgen05.mma, M=128, N=128, K=128, bf16 in, fp32 in TMEM
 //            lane i < 64: k_i.k_r (cols 0..63);  lane 64+r: qhat_r.k_i (cols 0..63)
 //   Gamma  down each column i by Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r mubar_r/mubar_i
@@ -10,10 +11,14 @@
 //   A      = (P K^T) o Gamma-:  A_{r,i} = alpha_r k_r.k_i Gamma_{r-1,i}  (i < r)
 //   Att    = (Qhat K^T) o Gamma:  Att_{r,i} = qhat_r.k_i Gamma_{r,i}  (i <= r)
 //   T      = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution, then the
-//            off-diagonal blocks by distance from the diagonal, fp32.
-// Writes T and Att (bf16, row-major 64 x 64 per chunk) and Gamma_{C,.} (the
-// last row of Gamma, into row 6 of the chunk's coefficient record).  The
-// inter-chunk kernel turns them into its operands.
+//            off-diagonal blocks by distance from the diagonal, fp32
+//   P      = [I; Att] T = [T; Att T]                    (M=128, N=64,  K=64)
+//   R      = K^T [Diag(Gamma_C) T | -Diag(w) T]          (M=128, N=128, K=64)
+//            with w_r = eta_r mubar_C / mubar_r
+// and writes, per chunk, the operands of the sequential inter-chunk kernel in
+// bf16: Qhat [64 x 128], [T; Att T] [128 x 64], A2T = [R_S; R_M] [256 x 64],
+// plus the per-position coefficients alphabar_r, alpha_r b_{r-1}, b_r and the
+// chunk scalars alphabar_C, b_C, mubar_C (fp32).
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -24,22 +29,30 @@ using namespace sm100;
 using namespace tc;
 
 constexpr int kThreads = 128;
-constexpr uint32_t KQ = 0;                  // [K; Qhat], 2 feature panels x (128 rows x 128 B)
-constexpr uint32_t GM = 32768;              // fp32 [64][LDF] Gamma
-constexpr uint32_t AM = GM + 64 * LDF * 4;  // fp32 [64][LDF] A (upper blocks: solve scratch)
-constexpr uint32_t TMF = AM + 64 * LDF * 4; // fp32 [64][LDF] T
-constexpr uint32_t REC = TMF + 64 * LDF * 4;// record rows 0..5
-constexpr uint32_t MU = REC + 1536;         // mu_r
-constexpr uint32_t BARS = MU + 256;
+constexpr uint32_t KQ = 0;                   // [K; Qhat], 2 feature panels x (128 rows x 128 B)
+constexpr uint32_t GM = 32768;               // fp32 [64][LDF] Gamma;  later [D_G T | -D_w T] bf16
+constexpr uint32_t AM = GM + 64 * LDF * 4;   // fp32 [64][LDF] A (upper blocks: scratch); later T bf16
+constexpr uint32_t TMF = AM + 64 * LDF * 4;  // fp32 [64][LDF] T
+constexpr uint32_t IATT = TMF + 64 * LDF * 4;// [I; Att] 128 x 64 bf16, K-major SW128
+constexpr uint32_t REC = IATT + 16384;       // record rows 0..5
+constexpr uint32_t VEC = REC + 1536;         // mu_r, w_r, Gamma_{C,r}
+constexpr uint32_t BARS = VEC + 768;
 constexpr uint32_t MISC = BARS + 16;
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t DT = GM;                  // aliases: written after Gamma and A are dead
+constexpr uint32_t TB = AM;
+static_assert(GM % 1024 == 0 && AM % 1024 == 0 && IATT % 1024 == 0, "operand alignment");
+static_assert(SMEM_BYTES <= 116 * 1024, "two CTAs per SM");
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t TM_G = 0, TM_P = 0, TM_R = 128;  // P reuses G's columns once G is read
 constexpr uint32_t kTxBytes = 32768 + 1536;
 
 struct IntraArgs {
-    float* rec;            // [chunks][7][64]: rows 0..5 read, row 6 written
-    __nv_bfloat16* tmat;   // [chunks][64][64]
-    __nv_bfloat16* att;    // [chunks][64][64]
+    const float* rec;      // [chunks][7][64] packed gate coefficients (rows 0..5 used)
+    __nv_bfloat16* qhat;   // [chunks][64][128]
+    __nv_bfloat16* tat;    // [chunks][128][64]
+    __nv_bfloat16* a2t;    // [chunks][256][64]
+    float* crec;           // [chunks][256]
     unsigned* status;
     float* dbg;            // diagnostics: phase clocks of CTA 0 (null in normal use)
     float dcorr;
@@ -65,7 +78,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* Am = reinterpret_cast<float*>(sm + AM);
     float* Tm = reinterpret_cast<float*>(sm + TMF);
     const float* rec = reinterpret_cast<const float*>(sm + REC);
-    float* mu = reinterpret_cast<float*>(sm + MU);
+    float* mu = reinterpret_cast<float*>(sm + VEC);
+    float* wv = mu + C;    // w_r = eta_r mubar_C / mubar_r
+    float* wg = wv + C;    // Gamma_{C,r}
     PhaseClock clk;
     clk.start((a.dbg && chunk == 0 && tid == 0) ? a.dbg : nullptr);
 
@@ -85,6 +100,14 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    if (tid < C) {  // identity rows 0..63 of [I; Att]
+        for (int c = 0; c < 8; ++c) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e == tid) ? 1.f : 0.f;
+            st_bf16x8(sm + IATT + sw128_off(tid, c), x);
+        }
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -94,7 +117,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
     clk.lap(0);
     if (ok) {
-        // Qhat = Q - d K in place (rows 64..127 of both panels)
+        // Qhat = Q - d K in place (rows 64..127 of both panels) and to global memory
+        __nv_bfloat16* qg = a.qhat + chunk * C * D;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u;
@@ -106,11 +130,26 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             unpack_bf16x8(*reinterpret_cast<const uint4*>(qp), qx);
 #pragma unroll
             for (int e = 0; e < 8; ++e) qx[e] -= a.dcorr * kx[e];
-            st_bf16x8(qp, qx);
+            const uint4 qw = bf16x8(qx);
+            *reinterpret_cast<uint4*>(qp) = qw;
+            *reinterpret_cast<uint4*>(qg + r * D + 64 * pn + 8 * c) = qw;
         }
         if (tid < C) {
+            const int r = tid;
+            const float* la = rec;
             const float* lm = rec + C;
-            mu[tid] = expf(lm[tid] - (tid > 0 ? lm[tid - 1] : 0.f));
+            const float* bb = rec + 2 * C;
+            mu[r] = expf(lm[r] - (r > 0 ? lm[r - 1] : 0.f));
+            wv[r] = rec[5 * C + r] * expf(lm[C - 1] - lm[r]);
+            float* cr = a.crec + chunk * 256;
+            cr[r] = expf(la[r]);
+            cr[C + r] = rec[3 * C + r] * (r > 0 ? bb[r - 1] : 0.f);
+            cr[2 * C + r] = bb[r];
+            if (r == 0) {
+                cr[3 * C] = expf(la[C - 1]);
+                cr[3 * C + 1] = bb[C - 1];
+                cr[3 * C + 2] = expf(lm[C - 1]);
+            }
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -121,7 +160,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t ad =
                     smem_desc(sbase + KQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128);
-                mma_bf16(tmem, ad, ad, id, ks > 0);
+                mma_bf16(tmem + TM_G, ad, ad, id, ks > 0);
             }
             mma_commit(&bars[1]);
         }
@@ -133,8 +172,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (ok) {
         // lane i < 64: k_i.k_r;  lane 64 + r: qhat_r.k_i   (columns 0..63)
         float gv[64];
-        tmem_ld32(tmem + lane_sel, *reinterpret_cast<float(*)[32]>(gv));
-        tmem_ld32(tmem + lane_sel + 32, *reinterpret_cast<float(*)[32]>(gv + 32));
+        tmem_ld32(tmem + lane_sel + TM_G, *reinterpret_cast<float(*)[32]>(gv));
+        tmem_ld32(tmem + lane_sel + TM_G + 32, *reinterpret_cast<float(*)[32]>(gv + 32));
         tmem_wait_ld();
         if (tid < C) {
             // column i of Gamma and A
@@ -158,7 +197,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     Gm[r * LDF + i] = gam;
                 }
             }
-            a.rec[chunk * kRecFloats + 6 * C + i] = gam;  // Gamma_{C,i}
+            wg[i] = gam;  // Gamma_{C,i}
         } else {
             // zero the six blocks of T above the diagonal
             for (int idx = tid - C; idx < 6 * 64; idx += 64) {
@@ -172,9 +211,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncthreads();
         clk.lap(3);
         if (tid >= C) {
-            // row r of Att, straight to global memory
+            // row r of Att into rows 64..127 of [I; Att]
             const int r = tid - C;
-            uint4* dst = reinterpret_cast<uint4*>(a.att + (chunk * C + r) * C);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const float4 g0 = lds4(Gm + r * LDF + 8 * c), g1 = lds4(Gm + r * LDF + 8 * c + 4);
@@ -182,7 +220,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 float x[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= r) ? gv[8 * c + e] * gr[e] : 0.f;
-                dst[c] = bf16x8(x);
+                st_bf16x8(sm + IATT + sw128_off(tid, c), x);
             }
         } else {
             // diagonal 16x16 blocks of T by forward substitution, one column per thread
@@ -276,19 +314,60 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             __syncthreads();
         }
         clk.lap(5);
-        // T to global memory (bf16, row-major): thread = (row, half)
+        // T (bf16, rows k) and [Diag(Gamma_C) T | -Diag(w) T]; thread = (row, half)
         {
-            const int r = tid >> 1, hf = tid & 1;
-            uint4* dst = reinterpret_cast<uint4*>(a.tmat + (chunk * C + r) * C + 32 * hf);
+            const int r = tid & 63, hf = tid >> 6;
+            const float wr = hf ? -wv[r] : wg[r];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float4 t0 = lds4(Tm + r * LDF + 32 * hf + 8 * c);
-                const float4 t1 = lds4(Tm + r * LDF + 32 * hf + 8 * c + 4);
-                const float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                dst[c] = bf16x8(x);
+            for (int c = 0; c < 8; ++c) {
+                const float4 t0 = lds4(Tm + r * LDF + 8 * c), t1 = lds4(Tm + r * LDF + 8 * c + 4);
+                float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                if (hf == 0) st_bf16x8(sm + TB + sw128_off(r, c), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= wr;
+                st_bf16x8(sm + DT + hf * 8192 + sw128_off(r, c), x);
             }
         }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
         clk.lap(6);
+        if (tid == 0) {
+            tc_fence_after_sync();
+            const uint32_t idp = idesc_bf16(128, 64, false, true);
+            const uint32_t idr = idesc_bf16(128, 128, true, true);
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_P, smem_desc(sbase + IATT + ks * 32, 16, 1024, kSw128),
+                         smem_desc(sbase + TB + ks * 2048, 8192, 1024, kSw128), idp, ks > 0);
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_R, smem_desc(sbase + KQ + ks * 2048, 16384, 1024, kSw128),
+                         smem_desc(sbase + DT + ks * 2048, 8192, 1024, kSw128), idr, ks > 0);
+            mma_commit(&bars[1]);
+        }
+        ok = mbar_wait(&bars[1], 1);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok);
+        clk.lap(7);
+    }
+    if (ok) {
+        // [T; Att T] row = lane, and the two A2T rows (lane, 128 + lane), to global memory
+        float v[64];
+        tmem_ld32(tmem + lane_sel + TM_P, *reinterpret_cast<float(*)[32]>(v));
+        tmem_ld32(tmem + lane_sel + TM_P + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        tmem_wait_ld();
+        uint4* d = reinterpret_cast<uint4*>(a.tat + (chunk * 2 * C + tid) * C);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) d[c] = bf16x8(v + 8 * c);
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            tmem_ld32(tmem + lane_sel + TM_R + 64 * q2, *reinterpret_cast<float(*)[32]>(v));
+            tmem_ld32(tmem + lane_sel + TM_R + 64 * q2 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tmem_wait_ld();
+            uint4* e = reinterpret_cast<uint4*>(a.a2t + (chunk * 2 * D + q2 * D + tid) * C);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) e[c] = bf16x8(v + 8 * c);
+        }
+        clk.lap(8);
     }
     if (!ok && tid == 0) {
         atomicOr(a.status + 1, 1u);
@@ -309,8 +388,10 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
         return cudaErrorInvalidValue;
     IntraArgs t;
     t.rec = a.rec;
-    t.tmat = a.tmat;
-    t.att = a.att;
+    t.qhat = a.qhat;
+    t.tat = a.tat;
+    t.a2t = a.a2t;
+    t.crec = a.crec;
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
     t.dcorr = a.dcorr;

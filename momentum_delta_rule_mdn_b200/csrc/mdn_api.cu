@@ -20,7 +20,7 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, tmat, att, total;
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, qhat, tat, a2t, crec, total;
 };
 
 // Byte offsets of every scratch region for these sizes.
@@ -40,8 +40,10 @@ WsLayout ws_layout(long long BH, int NT, int D)
     w.Z = off;      off += align_up(rows * D * sizeof(float));
     w.Oi = off;     off += align_up(rows * D * sizeof(float));
     w.rec = off;    off += align_up(rows * 7 * sizeof(float));
-    w.tmat = off;   off += align_up(rows * kChunk * 2);
-    w.att = off;    off += align_up(rows * kChunk * 2);
+    w.qhat = off;   off += align_up(rows * D * 2);
+    w.tat = off;    off += align_up(rows * 2 * kChunk * 2);
+    w.a2t = off;    off += align_up(rows * 2 * D * 2);
+    w.crec = off;   off += align_up(rows * 4 * sizeof(float));
     w.total = off;
     return w;
 }
@@ -175,8 +177,10 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.Z = reinterpret_cast<float*>(ws + w.Z);
     a.Oi = reinterpret_cast<float*>(ws + w.Oi);
     a.rec = reinterpret_cast<float*>(ws + w.rec);
-    a.tmat = reinterpret_cast<__nv_bfloat16*>(ws + w.tmat);
-    a.att = reinterpret_cast<__nv_bfloat16*>(ws + w.att);
+    a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + w.qhat);
+    a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
+    a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);
+    a.crec = reinterpret_cast<float*>(ws + w.crec);
 
     cudaError_t e;
     const bool check = flags & MDN_CHECK_FINITE;

@@ -54,8 +54,12 @@ struct ChunkArgs {
     float* Z;
     float* Oi;         // [B*H, NT*C, D]  carried-state part of o
     float* rec;        // [B*H*NT, 7, C]  packed coefficients (tensor-core path)
-    __nv_bfloat16* tmat;  // [B*H*NT, C, C]  T = (I + A)^{-1}, bf16 (tensor-core path)
-    __nv_bfloat16* att;   // [B*H*NT, C, C]  (Qhat K^T) o Gamma, bf16 (tensor-core path)
+    // operands the intra-chunk kernel prepares for the inter-chunk kernel (bf16, per chunk)
+    __nv_bfloat16* qhat;  // [B*H*NT, C, D]      qhat = q - d k
+    __nv_bfloat16* tat;   // [B*H*NT, 2C, C]     [T; Att T]
+    __nv_bfloat16* a2t;   // [B*H*NT, 2D, C]     [K^T Diag(Gamma_C) T; -K^T Diag(w) T]
+    float* crec;          // [B*H*NT, 256]       alphabar_r, alpha_r b_{r-1}, b_r, then
+                          //                     alphabar_C, b_C, mubar_C
     float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
 };
 
