@@ -50,7 +50,8 @@ constexpr uint32_t ST = A2T0 + 2 * 32768;    // [S | M] bf16, 128 rows x (32 + 3
 constexpr uint32_t YB = ST + 16384;          // Y 64 x 32 bf16, MN-major SW64
 constexpr uint32_t V0 = YB + 4096;           // V slice 64 x 32 bf16 (plain rows), 2 buffers
 constexpr uint32_t CR0 = V0 + 8192;          // chunk coefficients (256 floats), 2 buffers
-constexpr uint32_t BARS = CR0 + 2 * 1024;
+constexpr uint32_t OST0 = CR0 + 2 * 1024;    // output staging: [Vtilde | o] 64 x 32 bf16 each, 2 buffers
+constexpr uint32_t BARS = OST0 + 2 * 8192;
 constexpr uint32_t MISC = BARS + 128;
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory map too large");
@@ -98,7 +99,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_qh,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tat,
-                   const __grid_constant__ CUtensorMap tm_a2t, const InterArgs a)
+                   const __grid_constant__ CUtensorMap tm_a2t, const __grid_constant__ CUtensorMap tm_vt,
+                   const __grid_constant__ CUtensorMap tm_o, const InterArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -108,6 +110,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int lane = ((warp & 3) << 5) | (tid & 31);  // TMEM lane = operand row
     const int hc = warp >> 2;                          // column half: columns 16*hc .. 16*hc+15
     const int r = lane & 63;
+    const bool producer = tid == 128;  // issues every TMA load and store of the CTA
     const int slice = blockIdx.x % (D / NS);
     const int bh = blockIdx.x / (D / NS);
     const int b = bh / a.H, h = bh % a.H;
@@ -118,6 +121,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (tid == 0) {
         for (int k = 0; k < 7; ++k) mbar_init(&bars[k], 1);
         mbar_fence_init();
+        *reinterpret_cast<volatile int*>(sm + MISC + 4) = 0;
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -167,12 +171,13 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tma_load_3d(sm + A2T0 + buf * 32768, &tm_a2t, 0, 0, (int)chunk, fb);
         tma_load_3d(sm + A2T0 + buf * 32768 + 16384, &tm_a2t, 0, 128, (int)chunk, fb);
     };
-    if (tid == 0) {
+    if (producer) {
         for (int n = 0; n < 2 && n < a.NT; ++n) {
             load_a(n);
             load_b(n);
         }
     }
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + MISC + 4);
 
     bool ok = true;
     PhaseClock clk;
@@ -183,55 +188,79 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     auto store_outputs = [&](int n) -> bool {
         if (!mbar_wait(&bars[B_M3], n & 1)) return false;
         tc_fence_after_sync();
-        if (tid == 0 && n + 2 < a.NT) load_b(n + 2);
+        if (producer && n + 2 < a.NT) load_b(n + 2);
         float o3[NH];
         tmem_ld16(tl + TM_A3, o3);
         tmem_wait_ld();
         if (a.dbg != nullptr && blockIdx.x == 0 && n == 0)
             for (int j = 0; j < NH; ++j) a.dbg[DBG_A3 + lane * 32 + NH * hc + j] = o3[j];
-        const int t = n * C + r;
-        if (t < a.T) {
-            __nv_bfloat16* dst =
-                (lane < C ? a.vt : a.o) + (((size_t)b * a.T + t) * a.H + h) * D + j0 + NH * hc;
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
+        // rows of Vtilde (lanes 0..63) and o (lanes 64..127) into the staging tile;
+        // a TMA store (rows past T are clipped) writes them out
+        uint8_t* stg = sm + OST0 + (n & 1) * 8192 + (lane < C ? 0 : 4096) + r * 64 + 32 * hc;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float w[8];
+        for (int c = 0; c < 2; ++c) {
+            float w[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    w[e] = (lane < C) ? o3[8 * c + e] : o3[8 * c + e] + oi[8 * c + e];
-                d4[c] = bf16x8(w);
-            }
+            for (int e = 0; e < 8; ++e)
+                w[e] = (lane < C) ? o3[8 * c + e] : o3[8 * c + e] + oi[8 * c + e];
+            *reinterpret_cast<uint4*>(stg + 16 * c) = bf16x8(w);
         }
+        fence_proxy_async_smem();
         return true;
     };
 
+    auto issue_stores = [&](int n) {  // thread 0, after a barrier that follows store_outputs(n)
+        const uint8_t* stg = sm + OST0 + (n & 1) * 8192;
+        tma_store_4d(&tm_vt, j0, h, n * C, b, stg);
+        tma_store_4d(&tm_o, j0, h, n * C, b, stg + 4096);
+        bulk_commit_group();
+    };
+    // MMA descriptors: base descriptors plus start-address offsets (16-byte units)
+    const uint64_t d_kq0 = smem_desc(sbase + KQ0, 16, 1024, kSw128);
+    const uint64_t d_st = smem_desc(sbase + ST, 8192, 1024, kSw128);
+    const uint64_t d_a20 = smem_desc(sbase + A2T0, 16, 1024, kSw128);
+    const uint64_t d_tat0 = smem_desc(sbase + TAT0, 16, 1024, kSw128);
+    const uint64_t d_y = smem_desc(sbase + YB, 4096, 512, kSw64);
+    const uint32_t id1 = idesc_bf16(128, 64, false, true);
+    const uint32_t id2 = idesc_bf16(128, 32, false, true);
+
+    // A wait that runs out sets the abort flag before the next barrier; every
+    // thread reads it after that barrier, so all leave the loop together.
+    auto fail = [&](bool w) {
+        if (!w) *abort_flag = 1;
+    };
     for (int n = 0; n < a.NT; ++n) {
         const int buf = n & 1;
-        const uint32_t kq = KQ0 + buf * 32768;
         const float* cr = reinterpret_cast<const float*>(sm + CR0 + buf * 1024);
         const bool dump = a.dbg != nullptr && blockIdx.x == 0 && n == 0;
-        ok = __syncthreads_and(mbar_wait(&bars[B_FA0 + buf], (n >> 1) & 1));
-        if (!ok) break;
+        // the staging tile about to be written (chunk n-1) was last stored for chunk n-3
+        if (producer) bulk_wait_group_read<1>();
+        fail(mbar_wait(&bars[B_FA0 + buf], (n >> 1) & 1));
+        __syncthreads();
+        if (*abort_flag) break;
         clk.lap(0);
         const float c_ab = cr[r], c_d2 = cr[C + r], c_b = cr[2 * C + r];
         const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
 
-        // A1 = [K; Qhat] [S | M]
-        if (tid == 0) {
+        // A1 = [K; Qhat] [S | M]   (warp 0, one elected lane issues)
+        if (warp == 0) {
             tc_fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 64, false, true);
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_A1,
-                         smem_desc(sbase + kq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128),
-                         smem_desc(sbase + ST + ks * 2048, 8192, 1024, kSw128), id, ks > 0);
-            mma_commit(&bars[B_M1]);
+            const uint64_t dkq = d_kq0 + buf * (32768 >> 4);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad = dkq + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+                const uint64_t bd = d_st + ks * (2048 >> 4);
+                if (elect_one()) mma_bf16(tmem + TM_A1, ad, bd, id1, ks > 0);
+            }
+            if (elect_one()) mma_commit(&bars[B_M1]);
+            __syncwarp();
         }
-        if (n > 0) ok = store_outputs(n - 1);
-        ok = mbar_wait(&bars[B_M1], n & 1) && ok;
+        if (n > 0) fail(store_outputs(n - 1));
+        fail(mbar_wait(&bars[B_M1], n & 1));
         tc_fence_after_sync();
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
+        __syncthreads();
+        if (*abort_flag) break;
+        if (producer && n > 0) issue_stores(n - 1);
         clk.lap(1);
 
         // Y = V - X (rows 0..63); Oi kept in registers (rows 64..127)
@@ -262,40 +291,40 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     for (int j = 0; j < NH; ++j) a.dbg[DBG_Y + r * NS + NH * hc + j] = yy[j];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) st_bf16x8(sm + YB + sw64_off(r, 2 * hc + c), yy + 8 * c);
+                fence_proxy_async_smem();
             } else {
 #pragma unroll
                 for (int j = 0; j < NH; ++j) oi[j] = c_ab * x[j] - c_b * y[j];
             }
         }
-        fence_proxy_async_smem();
         tc_fence_before_sync();
-        ok = __syncthreads_and(mbar_wait(&bars[B_FB0 + buf], (n >> 1) & 1));
-        if (!ok) break;
+        fail(mbar_wait(&bars[B_FB0 + buf], (n >> 1) & 1));
+        __syncthreads();
+        if (*abort_flag) break;
         clk.lap(2);
 
-        if (tid == 0) {
-            // A2 = [A2T_S; A2T_M] Y, then A3 = [T; Att T] Y
+        // A2 = [A2T_S; A2T_M] Y, then A3 = [T; Att T] Y   (warp 0)
+        if (warp == 0) {
             tc_fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 32, false, true);
-            const uint32_t a2 = A2T0 + buf * 32768, tat = TAT0 + buf * 16384;
+            const uint64_t da2 = d_a20 + buf * (32768 >> 4), dtat = d_tat0 + buf * (16384 >> 4);
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t yd = smem_desc(sbase + YB + ks * 1024, 4096, 512, kSw64);
-                mma_bf16(tmem + TM_A2, smem_desc(sbase + a2 + ks * 32, 16, 1024, kSw128), yd, id,
-                         ks > 0);
-                mma_bf16(tmem + TM_A2 + 32, smem_desc(sbase + a2 + 16384 + ks * 32, 16, 1024, kSw128),
-                         yd, id, ks > 0);
+                const uint64_t yd = d_y + ks * (1024 >> 4);
+                if (elect_one()) mma_bf16(tmem + TM_A2, da2 + ks * 2, yd, id2, ks > 0);
+                if (elect_one()) mma_bf16(tmem + TM_A2 + 32, da2 + (16384 >> 4) + ks * 2, yd, id2, ks > 0);
             }
-            mma_commit(&bars[B_M2]);
+            if (elect_one()) mma_commit(&bars[B_M2]);
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t yd = smem_desc(sbase + YB + ks * 1024, 4096, 512, kSw64);
-                mma_bf16(tmem + TM_A3, smem_desc(sbase + tat + ks * 32, 16, 1024, kSw128), yd, id,
-                         ks > 0);
+                const uint64_t yd = d_y + ks * (1024 >> 4);
+                if (elect_one()) mma_bf16(tmem + TM_A3, dtat + ks * 2, yd, id2, ks > 0);
             }
-            mma_commit(&bars[B_M3]);
-            // K, Qhat, V and the coefficients of this buffer are no longer needed
-            if (n + 2 < a.NT) load_a(n + 2);
+            if (elect_one()) mma_commit(&bars[B_M3]);
+            __syncwarp();
         }
-        ok = mbar_wait(&bars[B_M2], n & 1);
+        // K, Qhat, V and the coefficients of this buffer are no longer needed
+        if (producer && n + 2 < a.NT) load_a(n + 2);
+        fail(mbar_wait(&bars[B_M2], n & 1));
         tc_fence_after_sync();
         clk.lap(3);
 
@@ -329,12 +358,16 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
         clk.lap(4);
     }
-    if (ok && a.NT > 0) ok = store_outputs(a.NT - 1);
-    ok = __syncthreads_and(ok);
+    ok = *abort_flag == 0;
+    __syncthreads();
+    ok = *abort_flag == 0;
+    if (ok && a.NT > 0) fail(store_outputs(a.NT - 1));
+    __syncthreads();
+    ok = *abort_flag == 0;
+    if (ok && producer && a.NT > 0) issue_stores(a.NT - 1);
+    if (producer) bulk_wait_group_all();  // every output tile has been written out
     if (ok) {
         const size_t row = ((size_t)bh * D + lane) * D + j0 + NH * hc;
 #pragma unroll
@@ -342,7 +375,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             a.S_T[row + j] = s[j];
             a.M_T[row + j] = m[j];
         }
-    } else if (tid == 0) {
+    } else if (producer) {
         atomicOr(a.status + 1, 1u);
         // Loads that were issued must land before the CTA's shared memory is
         // released; only the last two chunks' buffers can still be in flight.
@@ -357,33 +390,19 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// 3-D map over per-chunk bf16 matrices [chunks, rows, cols]; box = {64, box_rows, 1}, 128B swizzle.
-bool make_chunk_map(CUtensorMap* map, const void* base, long long chunks, int rows, int cols,
-                    int box_rows)
-{
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)chunks};
-    cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s)
 {
-    CUtensorMap mk, mqh, mv, mtat, ma2t;
+    CUtensorMap mk, mqh, mv, mtat, ma2t, mvt, mo;
     const long long chunks = (long long)a.B * a.H * a.NT;
     if (!make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
         !make_chunk_map(&mqh, a.qhat, chunks, C, D, C) ||
         !make_token_map(&mv, a.v, a.B, a.T, a.H, NS, false) ||
         !make_chunk_map(&mtat, a.tat, chunks, 2 * C, C, 2 * C) ||
-        !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128))
+        !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128) ||
+        !make_token_map(&mvt, a.vt, a.B, a.T, a.H, NS, false) ||
+        !make_token_map(&mo, a.o, a.B, a.T, a.H, NS, false))
         return cudaErrorInvalidValue;
     InterArgs t;
     t.crec = a.crec;
@@ -408,18 +427,18 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s)
     }
     const long long blocks = (long long)a.B * a.H * (D / NS);
     ProfScope ps(kInterTc, s);
-    chunk_inter_kernel<<<(unsigned)blocks, kThreads, SMEM_BYTES, s>>>(mk, mqh, mv, mtat, ma2t, t);
+    chunk_inter_kernel<<<(unsigned)blocks, kThreads, SMEM_BYTES, s>>>(mk, mqh, mv, mtat, ma2t, mvt,
+                                                                       mo, t);
     return cudaGetLastError();
 }
 
-// The tensor-core path: coefficients, then the intra-chunk kernel, then the
-// sequential inter-chunk kernel, all on stream s.
+// The tensor-core path: the intra-chunk kernel, then the sequential
+// inter-chunk kernel, both on stream s.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s)
 {
     if (a.D != D) return cudaErrorNotSupported;
-    cudaError_t e = launch_gate_pack(a.alpha_log, a.mu_log, a.beta, a.eta, a.B, a.T, a.H, a.rec, s);
+    cudaError_t e = launch_chunk_intra_tc(a, s);
     if (e != cudaSuccess) return e;
-    if ((e = launch_chunk_intra_tc(a, s)) != cudaSuccess) return e;
     return launch_chunk_inter_tc(a, s);
 }
 

@@ -45,10 +45,17 @@ static_assert(GM % 1024 == 0 && AM % 1024 == 0 && IATT % 1024 == 0, "operand ali
 static_assert(SMEM_BYTES <= 116 * 1024, "two CTAs per SM");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t TM_G = 0, TM_P = 0, TM_R = 128;  // P reuses G's columns once G is read
-constexpr uint32_t kTxBytes = 32768 + 1536;
+constexpr uint32_t kTxBytes = 32768;
+// staging of the outputs for the TMA stores (regions dead by then)
+constexpr uint32_t STG_TAT = IATT;           // 128 x 64 bf16
+constexpr uint32_t STG_A2T = GM;             // 256 x 64 bf16 (spans GM and AM)
+static_assert(STG_A2T + 32768 <= TMF, "A2T staging overlaps T");
 
 struct IntraArgs {
-    const float* rec;      // [chunks][7][64] packed gate coefficients (rows 0..5 used)
+    const float* alpha_log;  // [B, T, H] gates
+    const float* mu_log;
+    const float* beta;
+    const float* eta;
     __nv_bfloat16* qhat;   // [chunks][64][128]
     __nv_bfloat16* tat;    // [chunks][128][64]
     __nv_bfloat16* a2t;    // [chunks][256][64]
@@ -56,12 +63,13 @@ struct IntraArgs {
     unsigned* status;
     float* dbg;            // diagnostics: phase clocks of CTA 0 (null in normal use)
     float dcorr;
-    int H, NT;
+    int T, H, NT;
 };
 
 __global__ void __launch_bounds__(kThreads)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const IntraArgs a)
+                   const __grid_constant__ CUtensorMap tm_qh, const __grid_constant__ CUtensorMap tm_tat,
+                   const __grid_constant__ CUtensorMap tm_a2t, const IntraArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -77,7 +85,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* Gm = reinterpret_cast<float*>(sm + GM);
     float* Am = reinterpret_cast<float*>(sm + AM);
     float* Tm = reinterpret_cast<float*>(sm + TMF);
-    const float* rec = reinterpret_cast<const float*>(sm + REC);
+    float* rec = reinterpret_cast<float*>(sm + REC);
     float* mu = reinterpret_cast<float*>(sm + VEC);
     float* wv = mu + C;    // w_r = eta_r mubar_C / mubar_r
     float* wg = wv + C;    // Gamma_{C,r}
@@ -94,7 +102,32 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tma_load_4d(sm + KQ + p * 16384, &tm_k, p * 64, h, n * C, b, &bars[0]);
             tma_load_4d(sm + KQ + p * 16384 + 8192, &tm_q, p * 64, h, n * C, b, &bars[0]);
         }
-        bulk_load(sm + REC, a.rec + chunk * kRecFloats, 1536, &bars[0]);
+    }
+    if (warp == 3) {
+        // per-position coefficients: la, lm, b, alpha, beta, eta (positions past T are
+        // steps that leave the state unchanged)
+        const int lane = tid & 31;
+        const int t0 = n * C + 2 * lane;
+        float ga[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gb[2] = {0.f, 0.f}, ge[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            if (t0 + e < a.T) {
+                const size_t gi = ((size_t)b * a.T + t0 + e) * a.H + h;
+                ga[e] = a.alpha_log[gi];
+                gm[e] = a.mu_log[gi];
+                gb[e] = a.beta[gi];
+                ge[e] = a.eta[gi];
+            }
+        }
+        float la[2], lm[2], lc[2];
+        chunk_log_coeffs(ga, gm, gb, lane, la, lm, lc);
+        float2* r2 = reinterpret_cast<float2*>(rec) + lane;
+        r2[0] = make_float2(la[0], la[1]);
+        r2[32] = make_float2(lm[0], lm[1]);
+        r2[64] = make_float2(expf(la[0] + lc[0]), expf(la[1] + lc[1]));
+        r2[96] = make_float2(expf(ga[0]), expf(ga[1]));
+        r2[128] = make_float2(gb[0], gb[1]);
+        r2[160] = make_float2(ge[0], ge[1]);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -118,7 +151,6 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     clk.lap(0);
     if (ok) {
         // Qhat = Q - d K in place (rows 64..127 of both panels) and to global memory
-        __nv_bfloat16* qg = a.qhat + chunk * C * D;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u;
@@ -130,9 +162,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             unpack_bf16x8(*reinterpret_cast<const uint4*>(qp), qx);
 #pragma unroll
             for (int e = 0; e < 8; ++e) qx[e] -= a.dcorr * kx[e];
-            const uint4 qw = bf16x8(qx);
-            *reinterpret_cast<uint4*>(qp) = qw;
-            *reinterpret_cast<uint4*>(qg + r * D + 64 * pn + 8 * c) = qw;
+            *reinterpret_cast<uint4*>(qp) = bf16x8(qx);
         }
         if (tid < C) {
             const int r = tid;
@@ -155,6 +185,10 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncthreads();
         clk.lap(1);
         if (tid == 0) {
+            // Qhat (rows 64..127 of both panels) to global memory
+            tma_store_3d(&tm_qh, 0, 0, (int)chunk, sm + KQ + 8192);
+            tma_store_3d(&tm_qh, 64, 0, (int)chunk, sm + KQ + 16384 + 8192);
+            bulk_commit_group();
             tc_fence_after_sync();
             const uint32_t id = idesc_bf16(128, 128, false, false);
             for (int ks = 0; ks < 8; ++ks) {
@@ -350,22 +384,30 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         clk.lap(7);
     }
     if (ok) {
-        // [T; Att T] row = lane, and the two A2T rows (lane, 128 + lane), to global memory
+        // [T; Att T] row = lane and the two A2T rows (lane, 128 + lane) into the
+        // swizzled staging tiles, then TMA stores
         float v[64];
         tmem_ld32(tmem + lane_sel + TM_P, *reinterpret_cast<float(*)[32]>(v));
         tmem_ld32(tmem + lane_sel + TM_P + 32, *reinterpret_cast<float(*)[32]>(v + 32));
         tmem_wait_ld();
-        uint4* d = reinterpret_cast<uint4*>(a.tat + (chunk * 2 * C + tid) * C);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) d[c] = bf16x8(v + 8 * c);
+        for (int c = 0; c < 8; ++c) st_bf16x8(sm + STG_TAT + sw128_off(tid, c), v + 8 * c);
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2, *reinterpret_cast<float(*)[32]>(v));
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
             tmem_wait_ld();
-            uint4* e = reinterpret_cast<uint4*>(a.a2t + (chunk * 2 * D + q2 * D + tid) * C);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) e[c] = bf16x8(v + 8 * c);
+            for (int c = 0; c < 8; ++c)
+                st_bf16x8(sm + STG_A2T + q2 * 16384 + sw128_off(tid, c), v + 8 * c);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_3d(&tm_tat, 0, 0, (int)chunk, sm + STG_TAT);
+            tma_store_3d(&tm_a2t, 0, 0, (int)chunk, sm + STG_A2T);
+            tma_store_3d(&tm_a2t, 0, 128, (int)chunk, sm + STG_A2T + 16384);
+            bulk_commit_group();
         }
         clk.lap(8);
     }
@@ -373,6 +415,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         atomicOr(a.status + 1, 1u);
         (void)mbar_wait(&bars[0], 0);  // the loads must land before shared memory goes away
     }
+    if (tid == 0) bulk_wait_group_all();  // the stores have read their shared-memory tiles
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -382,12 +425,19 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
 {
-    CUtensorMap mq, mk;
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    CUtensorMap mq, mk, mqh, mtat, ma2t;
     if (!make_token_map(&mq, a.q, a.B, a.T, a.H, 64, true) ||
-        !make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true))
+        !make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
+        !make_chunk_map(&mqh, a.qhat, chunks, C, D, C) ||
+        !make_chunk_map(&mtat, a.tat, chunks, 2 * C, C, 2 * C) ||
+        !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
     IntraArgs t;
-    t.rec = a.rec;
+    t.alpha_log = a.alpha_log;
+    t.mu_log = a.mu_log;
+    t.beta = a.beta;
+    t.eta = a.eta;
     t.qhat = a.qhat;
     t.tat = a.tat;
     t.a2t = a.a2t;
@@ -395,6 +445,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
     t.dcorr = a.dcorr;
+    t.T = a.T;
     t.H = a.H;
     t.NT = a.NT;
     static bool attr_set = false;
@@ -405,9 +456,8 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const long long chunks = (long long)a.B * a.H * a.NT;
     ProfScope ps(kIntraTc, s);
-    chunk_intra_kernel<<<(unsigned)chunks, kThreads, SMEM_BYTES, s>>>(mq, mk, t);
+    chunk_intra_kernel<<<(unsigned)chunks, kThreads, SMEM_BYTES, s>>>(mq, mk, mqh, mtat, ma2t, t);
     return cudaGetLastError();
 }
 

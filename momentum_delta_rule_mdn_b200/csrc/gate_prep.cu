@@ -23,24 +23,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-__device__ __forceinline__ float warp_incl_sum(float x, int lane) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(kFull, x, off);
-        if (lane >= off) x += y;
-    }
-    return x;
-}
-
-__device__ __forceinline__ float warp_incl_lse(float x, int lane) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(kFull, x, off);
-        if (lane >= off) x = log_add_exp(x, y);
-    }
-    return x;
-}
-
 __global__ void __launch_bounds__(128)
 gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
                  const float* __restrict__ beta, const float* __restrict__ eta,
@@ -68,26 +50,8 @@ gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
             et[e] = eta[g];
         }
     }
-    // la, lm: inclusive prefix sums over the chunk.
-    const float sa = warp_incl_sum(a[0] + a[1], lane);
-    const float sm = warp_incl_sum(m[0] + m[1], lane);
-    float pa = __shfl_up_sync(kFull, sa, 1), pm = __shfl_up_sync(kFull, sm, 1);
-    if (lane == 0) pa = pm = 0.f;
-    float la_v[2], lm_v[2];
-    la_v[0] = pa + a[0];
-    la_v[1] = la_v[0] + a[1];
-    lm_v[0] = pm + m[0];
-    lm_v[1] = lm_v[0] + m[1];
-    // lc: logcumsumexp of x_j = log beta_j + lm_j - la_j  (beta = 0 -> -inf).
-    float x[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) x[e] = (be[e] > 0.f) ? logf(be[e]) + lm_v[e] - la_v[e] : -INFINITY;
-    const float sx = warp_incl_lse(log_add_exp(x[0], x[1]), lane);
-    float px = __shfl_up_sync(kFull, sx, 1);
-    if (lane == 0) px = -INFINITY;
-    float lc_v[2];
-    lc_v[0] = log_add_exp(px, x[0]);
-    lc_v[1] = log_add_exp(lc_v[0], x[1]);
+    float la_v[2], lm_v[2], lc_v[2];
+    chunk_log_coeffs(a, m, be, lane, la_v, lm_v, lc_v);
 
     const size_t row = (size_t)bh * NT * kChunk + (size_t)n * kChunk + 2 * lane;
     reinterpret_cast<float2*>(la + row)[0] = make_float2(la_v[0], la_v[1]);
@@ -123,76 +87,7 @@ gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
     }
 }
 
-// Packed per-chunk coefficient record for the tensor-core path: seven rows of
-// 64 floats, [la | lm | b | alpha | beta | eta | Gamma_{C,.}]; this kernel
-// writes the first six (the intra-chunk kernel writes the last), positions past
-// T holding the values of steps that leave the state unchanged.
-__global__ void __launch_bounds__(128)
-gate_pack_kernel(const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
-                 const float* __restrict__ beta, const float* __restrict__ eta,
-                 int B, int T, int H, int NT, float* __restrict__ rec)
-{
-    const int lane = threadIdx.x & 31;
-    const long long chunk = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (chunk >= (long long)B * H * NT) return;
-    const int n = (int)(chunk % NT);
-    const long long bh = chunk / NT;
-    const int b = (int)(bh / H), h = (int)(bh % H);
-    const int t0 = n * kChunk + 2 * lane;
-    float a[2] = {0.f, 0.f}, m[2] = {0.f, 0.f}, be[2] = {0.f, 0.f}, et[2] = {0.f, 0.f};
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int t = t0 + e;
-        if (t < T) {
-            const size_t g = ((size_t)b * T + t) * H + h;
-            a[e] = alpha_log[g];
-            m[e] = mu_log[g];
-            be[e] = beta[g];
-            et[e] = eta[g];
-        }
-    }
-    const float sa = warp_incl_sum(a[0] + a[1], lane);
-    const float sm = warp_incl_sum(m[0] + m[1], lane);
-    float pa = __shfl_up_sync(kFull, sa, 1), pm = __shfl_up_sync(kFull, sm, 1);
-    if (lane == 0) pa = pm = 0.f;
-    float la_v[2], lm_v[2];
-    la_v[0] = pa + a[0];
-    la_v[1] = la_v[0] + a[1];
-    lm_v[0] = pm + m[0];
-    lm_v[1] = lm_v[0] + m[1];
-    float x[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) x[e] = (be[e] > 0.f) ? logf(be[e]) + lm_v[e] - la_v[e] : -INFINITY;
-    const float sx = warp_incl_lse(log_add_exp(x[0], x[1]), lane);
-    float px = __shfl_up_sync(kFull, sx, 1);
-    if (lane == 0) px = -INFINITY;
-    float lc_v[2];
-    lc_v[0] = log_add_exp(px, x[0]);
-    lc_v[1] = log_add_exp(lc_v[0], x[1]);
-
-    float2* r = reinterpret_cast<float2*>(rec + (size_t)chunk * 7 * kChunk) + lane;
-    r[0 * kChunk / 2] = make_float2(la_v[0], la_v[1]);
-    r[1 * kChunk / 2] = make_float2(lm_v[0], lm_v[1]);
-    r[2 * kChunk / 2] = make_float2(expf(la_v[0] + lc_v[0]), expf(la_v[1] + lc_v[1]));
-    r[3 * kChunk / 2] = make_float2(expf(a[0]), expf(a[1]));
-    r[4 * kChunk / 2] = make_float2(be[0], be[1]);
-    r[5 * kChunk / 2] = make_float2(et[0], et[1]);
-}
-
 }  // namespace
-
-cudaError_t launch_gate_pack(const float* alpha_log, const float* mu_log, const float* beta,
-                             const float* eta, int B, int T, int H, float* rec, cudaStream_t s)
-{
-    const int NT = (T + kChunk - 1) / kChunk;
-    const long long chunks = (long long)B * H * NT;
-    if (chunks == 0) return cudaSuccess;
-    const long long blocks = (chunks + 3) / 4;
-    ProfScope ps(kGatePrep, s);
-    gate_pack_kernel<<<(unsigned)blocks, 128, 0, s>>>(alpha_log, mu_log, beta, eta, B, T, H, NT,
-                                                      rec);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
                              const float* eta, int B, int T, int H, float* la, float* lm,

@@ -20,7 +20,7 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, rec, qhat, tat, a2t, crec, total;
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, qhat, tat, a2t, crec, total;
 };
 
 // Byte offsets of every scratch region for these sizes.
@@ -39,7 +39,6 @@ WsLayout ws_layout(long long BH, int NT, int D)
     w.Y = off;      off += align_up(rows * D * sizeof(float));
     w.Z = off;      off += align_up(rows * D * sizeof(float));
     w.Oi = off;     off += align_up(rows * D * sizeof(float));
-    w.rec = off;    off += align_up(rows * 7 * sizeof(float));
     w.qhat = off;   off += align_up(rows * D * 2);
     w.tat = off;    off += align_up(rows * 2 * kChunk * 2);
     w.a2t = off;    off += align_up(rows * 2 * D * 2);
@@ -176,7 +175,6 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.Y = reinterpret_cast<float*>(ws + w.Y);
     a.Z = reinterpret_cast<float*>(ws + w.Z);
     a.Oi = reinterpret_cast<float*>(ws + w.Oi);
-    a.rec = reinterpret_cast<float*>(ws + w.rec);
     a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + w.qhat);
     a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
     a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);

@@ -25,6 +25,49 @@ __device__ __forceinline__ float log_add_exp(float a, float b) {
     return m + log1pf(expf(-fabsf(a - b)));
 }
 
+// Inclusive warp scans (lane order) of a sum and of a log-sum-exp.
+__device__ __forceinline__ float warp_incl_sum(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    return x;
+}
+__device__ __forceinline__ float warp_incl_lse(float x, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x = log_add_exp(x, y);
+    }
+    return x;
+}
+
+// Log-domain coefficients of one chunk of 64 positions, computed by one warp
+// (lane owns positions 2*lane and 2*lane+1): from alpha_log, mu_log, beta in
+// a[], m[], be[], the chunk-local prefix sums la, lm and lc = logcumsumexp of
+// (log beta + lm - la), lc = -inf while every beta so far is 0.
+__device__ __forceinline__ void chunk_log_coeffs(const float (&a)[2], const float (&m)[2],
+                                                 const float (&be)[2], int lane, float (&la)[2],
+                                                 float (&lm)[2], float (&lc)[2]) {
+    const float sa = warp_incl_sum(a[0] + a[1], lane);
+    const float sm = warp_incl_sum(m[0] + m[1], lane);
+    float pa = __shfl_up_sync(0xffffffffu, sa, 1), pm = __shfl_up_sync(0xffffffffu, sm, 1);
+    if (lane == 0) pa = pm = 0.f;
+    la[0] = pa + a[0];
+    la[1] = la[0] + a[1];
+    lm[0] = pm + m[0];
+    lm[1] = lm[0] + m[1];
+    float x[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) x[e] = (be[e] > 0.f) ? logf(be[e]) + lm[e] - la[e] : -INFINITY;
+    const float sx = warp_incl_lse(log_add_exp(x[0], x[1]), lane);
+    float px = __shfl_up_sync(0xffffffffu, sx, 1);
+    if (lane == 0) px = -INFINITY;
+    lc[0] = log_add_exp(px, x[0]);
+    lc[1] = log_add_exp(lc[0], x[1]);
+}
+
 // Everything one mdn_chunk_fwd call needs, with the workspace already carved.
 struct ChunkArgs {
     const void* q;
@@ -53,7 +96,6 @@ struct ChunkArgs {
     float* Y;
     float* Z;
     float* Oi;         // [B*H, NT*C, D]  carried-state part of o
-    float* rec;        // [B*H*NT, 7, C]  packed coefficients (tensor-core path)
     // operands the intra-chunk kernel prepares for the inter-chunk kernel (bf16, per chunk)
     __nv_bfloat16* qhat;  // [B*H*NT, C, D]      qhat = q - d k
     __nv_bfloat16* tat;   // [B*H*NT, 2C, C]     [T; Att T]
@@ -83,8 +125,6 @@ struct ProfScope {
 cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
                              const float* eta, int B, int T, int H, float* la, float* lm,
                              float* lc, float* bco, float* gamma, cudaStream_t s);
-cudaError_t launch_gate_pack(const float* alpha_log, const float* mu_log, const float* beta,
-                             const float* eta, int B, int T, int H, float* rec, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.

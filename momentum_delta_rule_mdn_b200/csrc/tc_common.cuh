@@ -15,9 +15,6 @@ namespace tc {
 constexpr int C = 64;          // chunk length
 constexpr int D = 128;         // d_k = d_v
 constexpr int LDF = 68;        // leading dimension of fp32 64x64 matrices (16-byte rows)
-constexpr int kRecRows = 7;    // packed per-chunk record: la, lm, b, alpha, beta, eta, Gamma_{C,.}
-constexpr int kRecFloats = kRecRows * C;
-constexpr uint32_t kRecBytes = kRecFloats * 4;
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -61,6 +58,16 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sm100::smem_u32(bar)) : "memory");
+}
+// True in exactly one (the lowest) active lane of the warp.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
 }
 __device__ __forceinline__ long long clock_now() {
     long long t;
@@ -117,14 +124,15 @@ inline bool make_token_map(CUtensorMap* map, const void* base, int B, int T, int
            CUDA_SUCCESS;
 }
 
-// 3-D map over per-chunk 64 x 64 bf16 matrices [chunks, 64, 64]; box = one matrix, 128B swizzle.
-inline bool make_mat_map(CUtensorMap* map, const void* base, long long chunks)
+// 3-D map over per-chunk bf16 matrices [chunks, rows, cols]; box = {64, box_rows, 1}, 128B swizzle.
+inline bool make_chunk_map(CUtensorMap* map, const void* base, long long chunks, int rows, int cols,
+                           int box_rows)
 {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {64, 64, (cuuint64_t)chunks};
-    cuuint64_t strides[2] = {64 * 2, 64 * 64 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)chunks};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
