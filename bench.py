@@ -230,7 +230,7 @@ def run_ours(args, rank, world, device):
                     "share_of_step": round(tot_ms / args.steps / ms, 4)}
 
     # ---- end to end through the public call, host (pinned) buffers
-    e2e = run_e2e(args, mdn, inp, tok, spec, device, world)
+    e2e = None if args.no_e2e else run_e2e(args, mdn, inp, tok, spec, device, world)
     decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
 
     line = {
@@ -451,6 +451,7 @@ def main():
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-shape measurement")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

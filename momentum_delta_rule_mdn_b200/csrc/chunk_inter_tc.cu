@@ -361,6 +361,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         clk.lap(4);
     }
     ok = *abort_flag == 0;
+    clk.flush();
     __syncthreads();
     ok = *abort_flag == 0;
     if (ok && a.NT > 0) fail(store_outputs(a.NT - 1));

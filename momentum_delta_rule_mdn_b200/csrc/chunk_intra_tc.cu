@@ -415,6 +415,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         atomicOr(a.status + 1, 1u);
         (void)mbar_wait(&bars[0], 0);  // the loads must land before shared memory goes away
     }
+    clk.flush();
     if (tid == 0) bulk_wait_group_all();  // the stores have read their shared-memory tiles
     tc_fence_before_sync();
     __syncthreads();

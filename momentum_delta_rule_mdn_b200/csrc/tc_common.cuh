@@ -74,20 +74,29 @@ __device__ __forceinline__ long long clock_now() {
     asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
     return t;
 }
-// Cycle counts of a kernel's phases, summed over chunks (diagnostic dump only).
+// Cycle counts of a kernel's phases, summed over chunks in registers and
+// written out once (diagnostic dump only; inert when `out` is null).
 struct PhaseClock {
+    static constexpr int kMax = 20;
     float* out;
     long long t;
+    float acc[kMax];
     __device__ __forceinline__ void start(float* o) {
         out = o;
+#pragma unroll
+        for (int k = 0; k < kMax; ++k) acc[k] = 0.f;
         t = clock_now();
     }
     __device__ __forceinline__ void lap(int k) {
         if (out) {
             const long long now = clock_now();
-            out[k] += (float)(now - t);
+            acc[k] += (float)(now - t);
             t = now;
         }
+    }
+    __device__ __forceinline__ void flush() {
+        if (out)
+            for (int k = 0; k < kMax; ++k) out[k] += acc[k];
     }
 };
 
