@@ -65,7 +65,7 @@ def kernel_work(name: str, spec: mi.Spec):
         return "hbm", th * (5 * d * 2) + states, "GB/s"
     if name == "intra_tc":
         # q, k, gates read; Qhat, [T; Att T], A2T and the chunk record written
-        return "hbm", th * (2 * d * 2 + 16) + th * (d * 2 + 2 * C * 2 + 4 * d * 2 + 16), "GB/s"
+        return "hbm", th * (2 * d * 2 + 16) + th * (d * 2 + 2 * C * 2 + 2 * d * 2 + 16), "GB/s"
     if name == "inter_simt":
         return "alu", th * 12.0 * d * d, "TFLOP/s"
     if name == "intra_simt":
