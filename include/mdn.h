@@ -70,12 +70,26 @@ typedef enum {
                                  a NaN or Inf, and MDN_ERR_TIMEOUT if a kernel
                                  reported a wait that ran out */
 #define MDN_FORCE_SIMT   0x2  /* use the fp32 CUDA-core kernels even for bf16 input */
+#define MDN_SLICE32      0x4  /* tensor-core path: the inter-chunk kernel gives each CTA
+                                 32 columns of d_v (four CTAs per head) */
+#define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head).  Neither flag:
+                                 64 when B*H*2 reaches the SM count, else 32.  Both
+                                 widths compute the same result; the flags exist
+                                 for tuning and testing. */
 
 /* Version of this ABI (incremented on any incompatible change). */
 int mdn_abi_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *mdn_status_string(mdn_status status);
+
+/*
+ * The CUDA error behind the last MDN_ERR_CUDA that a call returned on the
+ * calling thread: "<name> (<code>): <description>".  The string belongs to
+ * the library and stays valid until the next failing call on this thread.
+ * Before any failure it says that no error was recorded.  Never NULL.
+ */
+const char *mdn_last_cuda_error(void);
 
 /*
  * Bytes of device scratch that mdn_chunk_fwd needs for these sizes, or 0 if
@@ -100,7 +114,8 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *               alias S0 / M0 (read before written, per head).
  *   workspace   device scratch of at least mdn_chunk_fwd_workspace_size(...)
  *               bytes, 256-byte aligned; its contents on entry do not matter.
- *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT.
+ *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT, plus at most one of
+ *               MDN_SLICE32 / MDN_SLICE64.
  *
  * Support: d in {64, 128}, C = 64, any T >= 0 (a short last chunk is handled
  * as if padded with steps that leave S and M unchanged), B, H >= 0 with

@@ -12,6 +12,8 @@ MDN_OK, MDN_ERR_INVALID_ARG, MDN_ERR_UNSUPPORTED, MDN_ERR_CUDA, MDN_ERR_NONFINIT
 MDN_F32, MDN_BF16 = 0, 1
 MDN_CHECK_FINITE = 0x1
 MDN_FORCE_SIMT = 0x2
+MDN_SLICE32 = 0x4
+MDN_SLICE64 = 0x8
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -19,6 +21,7 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 SIGNATURES = {
     "mdn_abi_version": (_i, []),
     "mdn_status_string": (ctypes.c_char_p, [_i]),
+    "mdn_last_cuda_error": (ctypes.c_char_p, []),
     "mdn_chunk_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "mdn_chunk_fwd": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                            _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp]),

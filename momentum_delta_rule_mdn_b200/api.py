@@ -30,7 +30,10 @@ def library():
 class MDNError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)}")
+        msg = f"{where}: {status_string(status)}"
+        if status == _lib.MDN_ERR_CUDA:
+            msg += f" [{library().mdn_last_cuda_error().decode()}]"
+        super().__init__(msg)
 
 
 def status_string(status: int) -> str:

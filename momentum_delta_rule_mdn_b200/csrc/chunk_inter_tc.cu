@@ -11,23 +11,34 @@
 // chunk-end update S' = alphabar_C S - b_C M + K^T Diag(Gamma_{C,.}) T Y,
 // M' = mubar_C M - K^T Diag(eta_i mubar_C / mubar_i) T Y.
 //
-// One CTA owns one (b, h) and 32 of the d_v = 128 columns (columns of S, M and
-// Vtilde are independent) and walks the chunks in order.  The intra-chunk
-// kernel has prepared Qhat, [T; Att T] and A2T = [K^T Diag(Gamma_C) T;
+// One CTA owns one (b, h) and NS (32 or 64) of the d_v = 128 columns (columns
+// of S, M and Vtilde are independent) and walks the chunks in order.  The
+// intra-chunk kernel has prepared Qhat, [T; Att T] and A2T = [K^T Diag(Gamma_C) T;
 // -K^T Diag(w) T] for every chunk.  Per chunk n:
-//     A1 = [K; Qhat] [S | M]                      (M=128, N=64, K=128)
-//     Y  = V - (D1 KS - D2 KM);   Oi = Diag(alphabar) QhatS - Diag(b) QhatM
-//     A2 = [A2T_S; A2T_M] Y   (two M=128, N=32, K=64)
+//     A1 = [K; Qhat] [S | M]                      (M=128, N=2 NS, K=128)
+//     Y  = V - (D1 KS - D2 KM)
+//     A2 = [A2T_S; A2T_M] Y   (two M=128, N=NS, K=64)
 //     S, M <- (alphabar_C S - b_C M, mubar_C M) + A2
-//     A3 = [T; Att T] Y  (M=128, N=32, K=64):  Vtilde = A3[0:64],  o = Oi + A3[64:128]
-// The critical path of a chunk is A1 -> Y -> A2 -> state; the stores of chunk
-// n-1 run while A1 of chunk n executes.  Eight warps: warp w owns TMEM lanes
-// 32(w%4).. and columns 16(w/4).. of the CTA's 32, so a thread holds 16
-// columns of one row of S and M in fp32 registers; their bf16 copy in shared
-// memory is the B operand of A1.  Loads are double-buffered in two groups by
-// lifetime (K, Qhat, V, coefficients: free after A1; [T; Att T], A2T: free
-// after A2, A3).  Every mbarrier wait is bounded; a wait that runs out sets
-// status[1] and the CTA stops.
+//     A3 = [T; Att T] Y  (M=128, N=NS, K=64):
+//     Vtilde = A3[0:64],  o = Diag(alphabar) QhatS - Diag(b) QhatM + A3[64:128]
+// A tcgen05.mma of N <= 128 costs about the same whatever N is, so a wider
+// slice does more work per instruction; NS = 64 halves the CTAs per head
+// and the operand traffic for the same chain length.
+// Only A1 -> Y -> A2 -> state is sequential; the warps are specialised so
+// that nothing else sits on that chain:
+//   warp 0      one lane issues every tcgen05.mma and commit
+//   warp 1      one lane issues every TMA load, up to two chunks ahead
+//   NS/4 chain warps: warp w owns TMEM lanes 32(w%4).. and 16 columns; it
+//               holds those columns of one row of S and M in fp32 registers
+//               for the whole sequence (their bf16 copy in shared memory is
+//               the B operand of A1); the warps on lanes 0..63 also form Y
+//   4 output warps: Vtilde and o of chunk n from A3 and A1, written to
+//               global memory while the chain runs on
+// Hand-offs are mbarriers only (no CTA-wide barrier inside the loop).  TMEM
+// holds A1 and A3 twice (chunk parity) so the outputs of chunk n can be read
+// while chunk n+1 computes.  Every wait is bounded; a wait that runs out
+// raises the CTA's abort flag, every role leaves its loop, in-flight copies
+// and MMAs are drained, and status[1] is set.
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -37,33 +48,65 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int NS = 32;         // d_v columns per CTA
-constexpr int NH = 16;         // columns per thread
-constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 256;
+constexpr int NH = 16;           // columns per chain thread
+constexpr int kChainWarp0 = 2;   // warps 0, 1: MMA issue, loads
 
-// Shared memory map (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t KQ0 = 0;                  // [K; Qhat], 2 buffers x 2 panels x (128 x 128 B)
-constexpr uint32_t TAT0 = 2 * 32768;         // [T; Att T] 128 x 64 bf16 (K-major SW128), 2 buffers
-constexpr uint32_t A2T0 = TAT0 + 2 * 16384;  // [A2T_S | A2T_M] 2 panels of 128 x 64, 2 buffers
-constexpr uint32_t ST = A2T0 + 2 * 32768;    // [S | M] bf16, 128 rows x (32 + 32), MN-major SW128
-constexpr uint32_t YB = ST + 16384;          // Y 64 x 32 bf16, MN-major SW64
-constexpr uint32_t V0 = YB + 4096;           // V slice 64 x 32 bf16 (plain rows), 2 buffers
-constexpr uint32_t CR0 = V0 + 8192;          // chunk coefficients (256 floats), 2 buffers
-constexpr uint32_t OST0 = CR0 + 2 * 1024;    // output staging: [Vtilde | o] 64 x 32 bf16 each, 2 buffers
-constexpr uint32_t BARS = OST0 + 2 * 8192;
-constexpr uint32_t MISC = BARS + 128;
-constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory map too large");
+// Per-width layout.  NS = d_v columns per CTA (32 or 64).
+template <int NS>
+struct Cfg {
+    static constexpr int CW = NS / 4;                 // chain warps: 4 lane quadrants x NS/16 column groups
+    static constexpr int kOutWarp0 = kChainWarp0 + CW;
+    static constexpr int kThreads = (kOutWarp0 + 4) * 32;
+    // one CTA per SM; registers are granted to warps in groups of four
+    static constexpr int kMaxRegs = (65536 / (((kThreads / 32 + 3) / 4) * 128)) & ~7;
+    static constexpr int NVC = NS == 32 ? 4 : 2;      // V / coefficient slots
+    static constexpr uint32_t kTmemCols = NS == 32 ? 256 : 512;
+    // shared memory (byte offsets from a 1024-byte aligned base)
+    static constexpr uint32_t KQ0 = 0;                // [K; Qhat], 2 slots x 2 panels x (128 rows x 128 B)
+    static constexpr uint32_t FB0 = 2 * 32768;        // [T; Att T] (16 KB), [A2T_S | A2T_M] (2 x 16 KB), 2 slots
+    static constexpr uint32_t FB_BYTES = 49152;
+    static constexpr uint32_t ST = FB0 + 2 * FB_BYTES;  // [S | M] bf16, 128 rows, MN-major 128-byte swizzle
+    static constexpr uint32_t ST_BYTES = 128 * 2 * NS * 2;
+    static constexpr uint32_t YB = ST + ST_BYTES;      // Y 64 rows x NS bf16, MN-major (64 / 128-byte swizzle)
+    static constexpr uint32_t YB_BYTES = 64 * NS * 2;
+    static constexpr uint32_t V0 = YB + YB_BYTES;      // V slice 64 rows x NS bf16 (plain rows), NVC slots
+    static constexpr uint32_t V_BYTES = 64 * NS * 2;
+    static constexpr uint32_t CR0 = V0 + NVC * V_BYTES;  // chunk coefficients (256 floats), NVC slots
+    static constexpr uint32_t BARS = CR0 + NVC * 1024;
+    static constexpr uint32_t MISC = BARS + 256;
+    static constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
+    static_assert(SMEM_BYTES <= 232448, "shared memory map too large");
+    static_assert(ST % 1024 == 0 && YB % 1024 == 0 && V0 % 16 == 0, "operand alignment");
+    // TMEM columns: A1 (KS | KM, QhatS | QhatM) in two slots, A2 (dS | dM), A3 in two slots
+    static constexpr uint32_t TM_A1 = 0, TM_A2 = 4 * NS, TM_A3 = 6 * NS;
+    static constexpr uint32_t kTxVC = V_BYTES + 1024;
+    // byte offset of 16-byte chunk c (8 columns) of row i of S, resp. M, in ST
+    __device__ static __forceinline__ uint32_t s_off(int i, int c) { return sw128_off(i, c); }
+    __device__ static __forceinline__ uint32_t m_off(int i, int c) {
+        return NS == 32 ? sw128_off(i, 4 + c) : 16384 + sw128_off(i, c);
+    }
+    // byte offset of chunk c of row r of Y in YB
+    __device__ static __forceinline__ uint32_t y_off(int r, int c) {
+        return NS == 32 ? sw64_off(r, c) : sw128_off(r, c);
+    }
+};
 
-// TMEM columns
-constexpr uint32_t TM_A1 = 0, TM_A2 = 64, TM_A3 = 128;
+constexpr uint32_t kTxKQ = 32768;   // K, Qhat
+constexpr uint32_t kTxFB = 49152;   // [T; Att T], A2T
 
-constexpr uint32_t kTxA = 32768 + 4096 + 1024;   // K, Qhat, V, coefficients
-constexpr uint32_t kTxB = 16384 + 32768;         // [T; Att T], A2T
-
-// mbarriers
-constexpr int B_FA0 = 0, B_FB0 = 2, B_M1 = 4, B_M2 = 5, B_M3 = 6;
+// mbarriers (index into the array at BARS)
+constexpr int B_FKQ = 0;   // [2] K, Qhat landed
+constexpr int B_FFB = 2;   // [2] [T; Att T], A2T landed
+constexpr int B_FVC = 4;   // [4] V, coefficients landed
+constexpr int B_EVC = 8;   // [4] V, coefficients slot released (chain + output warps)
+constexpr int B_M1 = 12;   // [2] A1 complete
+constexpr int B_M2 = 14;   //     A2 complete
+constexpr int B_M3 = 15;   // [2] A3 complete (and every earlier MMA)
+constexpr int B_YR = 17;   //     Y written (the chain warps on lanes 0..63)
+constexpr int B_SR = 18;   //     next state written (every chain warp)
+constexpr int B_OD = 19;   // [2] A1 / A3 slot read by the output warps (4 warps)
+constexpr int B_FIN = 21;  //     every MMA complete (exit)
+constexpr int kBars = 22;
 
 struct InterArgs {
     const float* crec;
@@ -74,13 +117,9 @@ struct InterArgs {
     __nv_bfloat16* o;
     __nv_bfloat16* vt;
     unsigned* status;
-    float* dbg;  // diagnostics: CTA 0 dumps its first chunk's intermediates and phase clocks
+    float* dbg;  // diagnostics: phase clocks of the MMA and load lanes of CTA 0 (null in normal use)
     int T, H, NT;
 };
-
-// Offsets (floats) of the diagnostic dump.
-constexpr int DBG_A1 = 49152, DBG_Y = 57344, DBG_A2 = 59392, DBG_A3 = 67584, DBG_S = 71680,
-              DBG_M = 75776, DBG_CLK = 80400;
 
 // 16 consecutive 32-bit TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -96,40 +135,74 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
+
+// Wait for the phase of `bar` with this parity.  Gives up when another role
+// has raised the abort flag, or after ~1 s (then raises it itself).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitNs || i > (1u << 26)) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+// Warp-uniform form: every lane waits, and the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
+}
+
+template <int NS>
+__global__ void __launch_bounds__(Cfg<NS>::kThreads) __maxnreg__(Cfg<NS>::kMaxRegs)
 chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_qh,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tat,
-                   const __grid_constant__ CUtensorMap tm_a2t, const __grid_constant__ CUtensorMap tm_vt,
-                   const __grid_constant__ CUtensorMap tm_o, const InterArgs a)
+                   const __grid_constant__ CUtensorMap tm_a2t, const InterArgs a)
 {
+    using L = Cfg<NS>;
+    constexpr int CW = L::CW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int lane = ((warp & 3) << 5) | (tid & 31);  // TMEM lane = operand row
-    const int hc = warp >> 2;                          // column half: columns 16*hc .. 16*hc+15
-    const int r = lane & 63;
-    const bool producer = tid == 128;  // issues every TMA load and store of the CTA
+    const int tid = threadIdx.x, warp = tid >> 5, lid = tid & 31;
+    const int quad = warp & 3;                   // TMEM lane quadrant this warp may access
+    const int lane = (quad << 5) | lid;          // TMEM lane = operand row
     const int slice = blockIdx.x % (D / NS);
     const int bh = blockIdx.x / (D / NS);
     const int b = bh / a.H, h = bh % a.H;
     const int j0 = slice * NS;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BARS);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
+    const int NT = a.NT;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
 
     if (tid == 0) {
-        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], 1);
+        for (int k = 0; k < kBars; ++k) {
+            uint32_t count = 1;  // TMA (expect_tx) and tcgen05.commit barriers
+            if (k >= B_EVC && k < B_EVC + 4) count = CW + 4;
+            if (k == B_YR) count = CW / 2;
+            if (k == B_OD || k == B_OD + 1) count = 4;
+            if (k == B_SR) count = CW;
+            mbar_init(&bars[k], count);
+        }
         mbar_fence_init();
-        *reinterpret_cast<volatile int*>(sm + MISC + 4) = 0;
+        *abort_flag = 0;
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(tmem_slot, L::kTmemCols);
         tmem_relinquish();
     }
-    // entering state: row `lane` of S and M, columns j0 + 16 hc ..
+    // chain warps: the entering state, row `lane`, columns j0 + NH hc ..
+    const bool chain = warp >= kChainWarp0 && warp < L::kOutWarp0;
+    const int hc = (warp - kChainWarp0) >> 2;  // column group of a chain warp
     float s[NH], m[NH];
-    {
+    if (chain) {
         const size_t row = ((size_t)bh * D + lane) * D + j0 + NH * hc;
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
@@ -137,273 +210,283 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             m[j] = a.M0 ? a.M0[row + j] : 0.f;
         }
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            st_bf16x8(sm + ST + sw128_off(lane, 2 * hc + c), s + 8 * c);
-            st_bf16x8(sm + ST + sw128_off(lane, 4 + 2 * hc + c), m + 8 * c);
+        for (int c = 0; c < NH / 8; ++c) {
+            st_bf16x8(sm + L::ST + L::s_off(lane, hc * (NH / 8) + c), s + 8 * c);
+            st_bf16x8(sm + L::ST + L::m_off(lane, hc * (NH / 8) + c), m + 8 * c);
         }
+        fence_proxy_async_smem();
     }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + NH * hc;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);  // this warp's lane base
 
-    auto load_a = [&](int n) {  // K, Qhat, V, coefficients of chunk n
-        const int buf = n & 1;
-        uint64_t* fb = &bars[B_FA0 + buf];
-        const long long chunk = (long long)bh * a.NT + n;
-        mbar_arrive_expect_tx(fb, kTxA);
+    if (warp == 0) {
+        // ------------------------------------------------------------ MMA issue
+        if (lid == 0) {
+            PhaseClock clk;
+            clk.start((a.dbg && blockIdx.x == 0) ? a.dbg : nullptr);
+            const uint64_t d_kq0 = smem_desc(sbase + L::KQ0, 16, 1024, kSw128);
+            // B of A1: [S | M], N = 2 NS; for NS = 64 the S and M halves are two 128-byte panels
+            const uint64_t d_st = smem_desc(sbase + L::ST, NS == 32 ? 8192 : 16384, 1024, kSw128);
+            const uint64_t d_fb0 = smem_desc(sbase + L::FB0, 16, 1024, kSw128);
+            const uint64_t d_y = NS == 32 ? smem_desc(sbase + L::YB, 4096, 512, kSw64)
+                                          : smem_desc(sbase + L::YB, 8192, 1024, kSw128);
+            constexpr uint32_t ystep = (16 * NS * 2) >> 4;  // 16 rows of Y
+            constexpr uint32_t id1 = idesc_bf16(128, 2 * NS, false, true);
+            constexpr uint32_t id2 = idesc_bf16(128, NS, false, true);
+            // K, Qhat of chunk n and the A1 / A3 slot of chunk n are waited for
+            // while chunk n - 1 waits for its Y, so that only the state hand-off
+            // separates the last product of one chunk from the first of the next.
+            bool ready = NT > 0 && wait_bar(&bars[B_FKQ], 0, abort_flag);
+            for (int n = 0; n < NT && ready; ++n) {
+                const int s2 = n & 1;
+                clk.lap(0);
+                if (n >= 1 && !wait_bar(&bars[B_SR], (n - 1) & 1, abort_flag)) break;
+                clk.lap(1);
+                tc_fence_after_sync();
+                const uint64_t dkq = d_kq0 + s2 * (32768 >> 4);
+                const uint32_t a1 = tmem + L::TM_A1 + 2 * NS * s2;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            tma_load_4d(sm + KQ0 + buf * 32768 + p * 16384, &tm_k, p * 64, h, n * C, b, fb);
-            tma_load_3d(sm + KQ0 + buf * 32768 + p * 16384 + 8192, &tm_qh, p * 64, 0, (int)chunk, fb);
-        }
-        tma_load_4d(sm + V0 + buf * 4096, &tm_v, j0, h, n * C, b, fb);
-        bulk_load(sm + CR0 + buf * 1024, a.crec + chunk * 256, 1024, fb);
-    };
-    auto load_b = [&](int n) {  // [T; Att T] and A2T of chunk n
-        const int buf = n & 1;
-        uint64_t* fb = &bars[B_FB0 + buf];
-        const long long chunk = (long long)bh * a.NT + n;
-        mbar_arrive_expect_tx(fb, kTxB);
-        tma_load_3d(sm + TAT0 + buf * 16384, &tm_tat, 0, 0, (int)chunk, fb);
-        tma_load_3d(sm + A2T0 + buf * 32768, &tm_a2t, 0, 0, (int)chunk, fb);
-        tma_load_3d(sm + A2T0 + buf * 32768 + 16384, &tm_a2t, 0, 128, (int)chunk, fb);
-    };
-    if (producer) {
-        for (int n = 0; n < 2 && n < a.NT; ++n) {
-            load_a(n);
-            load_b(n);
-        }
-    }
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + MISC + 4);
-
-    bool ok = true;
-    PhaseClock clk;
-    clk.start((a.dbg && blockIdx.x == 0 && tid == 0) ? a.dbg + DBG_CLK + 16 : nullptr);
-    float oi[NH];
-    // Vtilde and o of chunk n once its A3 product has completed; then the
-    // [T; Att T] / A2T buffer of chunk n is free for chunk n + 2.
-    auto store_outputs = [&](int n) -> bool {
-        if (!mbar_wait(&bars[B_M3], n & 1)) return false;
-        tc_fence_after_sync();
-        if (producer && n + 2 < a.NT) load_b(n + 2);
-        float o3[NH];
-        tmem_ld16(tl + TM_A3, o3);
-        tmem_wait_ld();
-        if (a.dbg != nullptr && blockIdx.x == 0 && n == 0)
-            for (int j = 0; j < NH; ++j) a.dbg[DBG_A3 + lane * 32 + NH * hc + j] = o3[j];
-        // rows of Vtilde (lanes 0..63) and o (lanes 64..127) into the staging tile;
-        // a TMA store (rows past T are clipped) writes them out
-        uint8_t* stg = sm + OST0 + (n & 1) * 8192 + (lane < C ? 0 : 4096) + r * 64 + 32 * hc;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            float w[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                w[e] = (lane < C) ? o3[8 * c + e] : o3[8 * c + e] + oi[8 * c + e];
-            *reinterpret_cast<uint4*>(stg + 16 * c) = bf16x8(w);
-        }
-        fence_proxy_async_smem();
-        return true;
-    };
-
-    auto issue_stores = [&](int n) {  // thread 0, after a barrier that follows store_outputs(n)
-        const uint8_t* stg = sm + OST0 + (n & 1) * 8192;
-        tma_store_4d(&tm_vt, j0, h, n * C, b, stg);
-        tma_store_4d(&tm_o, j0, h, n * C, b, stg + 4096);
-        bulk_commit_group();
-    };
-    // MMA descriptors: base descriptors plus start-address offsets (16-byte units)
-    const uint64_t d_kq0 = smem_desc(sbase + KQ0, 16, 1024, kSw128);
-    const uint64_t d_st = smem_desc(sbase + ST, 8192, 1024, kSw128);
-    const uint64_t d_a20 = smem_desc(sbase + A2T0, 16, 1024, kSw128);
-    const uint64_t d_tat0 = smem_desc(sbase + TAT0, 16, 1024, kSw128);
-    const uint64_t d_y = smem_desc(sbase + YB, 4096, 512, kSw64);
-    const uint32_t id1 = idesc_bf16(128, 64, false, true);
-    const uint32_t id2 = idesc_bf16(128, 32, false, true);
-
-    // A wait that runs out sets the abort flag before the next barrier; every
-    // thread reads it after that barrier, so all leave the loop together.
-    auto fail = [&](bool w) {
-        if (!w) *abort_flag = 1;
-    };
-    for (int n = 0; n < a.NT; ++n) {
-        const int buf = n & 1;
-        const float* cr = reinterpret_cast<const float*>(sm + CR0 + buf * 1024);
-        const bool dump = a.dbg != nullptr && blockIdx.x == 0 && n == 0;
-        // the staging tile about to be written (chunk n-1) was last stored for chunk n-3
-        if (producer) bulk_wait_group_read<1>();
-        fail(mbar_wait(&bars[B_FA0 + buf], (n >> 1) & 1));
-        __syncthreads();
-        if (*abort_flag) break;
-        clk.lap(0);
-        const float c_ab = cr[r], c_d2 = cr[C + r], c_b = cr[2 * C + r];
-        const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
-
-        // A1 = [K; Qhat] [S | M]   (warp 0, one elected lane issues)
-        if (warp == 0) {
-            tc_fence_after_sync();
-            const uint64_t dkq = d_kq0 + buf * (32768 >> 4);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = dkq + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-                const uint64_t bd = d_st + ks * (2048 >> 4);
-                if (elect_one()) mma_bf16(tmem + TM_A1, ad, bd, id1, ks > 0);
-            }
-            if (elect_one()) mma_commit(&bars[B_M1]);
-            __syncwarp();
-        }
-        if (n > 0) fail(store_outputs(n - 1));
-        fail(mbar_wait(&bars[B_M1], n & 1));
-        tc_fence_after_sync();
-        __syncthreads();
-        if (*abort_flag) break;
-        if (producer && n > 0) issue_stores(n - 1);
-        clk.lap(1);
-
-        // Y = V - X (rows 0..63); Oi kept in registers (rows 64..127)
-        {
-            float x[NH], y[NH];
-            tmem_ld16(tl + TM_A1, x);
-            tmem_ld16(tl + TM_A1 + 32, y);
-            tmem_wait_ld();
-            if (dump)
-                for (int j = 0; j < NH; ++j) {
-                    a.dbg[DBG_A1 + lane * 64 + NH * hc + j] = x[j];
-                    a.dbg[DBG_A1 + lane * 64 + 32 + NH * hc + j] = y[j];
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(a1, dkq + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
+                             d_st + ks * (2048 >> 4), id1, ks > 0);
+                mma_commit(&bars[B_M1 + s2]);
+                clk.lap(2);
+                if (!wait_bar(&bars[B_FFB + s2], (n >> 1) & 1, abort_flag)) break;
+                if (n + 1 < NT) {
+                    const int t2 = (n + 1) & 1;
+                    if (!wait_bar(&bars[B_FKQ + t2], ((n + 1) >> 1) & 1, abort_flag)) break;
+                    if (n >= 1 && !wait_bar(&bars[B_OD + t2], ((n - 1) >> 1) & 1, abort_flag)) break;
                 }
-            if (lane < C) {
-                const uint4* vrow = reinterpret_cast<const uint4*>(sm + V0 + buf * 4096 + r * 64) + 2 * hc;
-                float yy[NH];
+                clk.lap(3);
+                if (!wait_bar(&bars[B_YR], n & 1, abort_flag)) break;
+                clk.lap(4);
+                tc_fence_after_sync();
+                const uint64_t dfb = d_fb0 + s2 * (L::FB_BYTES >> 4);
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float vv[8];
-                    unpack_bf16x8(vrow[c], vv);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t yd = d_y + ks * ystep;
+                    mma_bf16(tmem + L::TM_A2, dfb + (16384 >> 4) + ks * 2, yd, id2, ks > 0);
+                    mma_bf16(tmem + L::TM_A2 + NS, dfb + (32768 >> 4) + ks * 2, yd, id2, ks > 0);
+                }
+                mma_commit(&bars[B_M2]);
+                clk.lap(5);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = 8 * c + e;
-                        yy[j] = vv[e] - (c_ab * x[j] - c_d2 * y[j]);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + L::TM_A3 + NS * s2, dfb + ks * 2, d_y + ks * ystep, id2, ks > 0);
+                mma_commit(&bars[B_M3 + s2]);
+                clk.lap(6);
+            }
+            clk.flush();
+            // every issued MMA has completed before TMEM and shared memory are released
+            mma_commit(&bars[B_FIN]);
+            (void)mbar_wait(&bars[B_FIN], 0);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ TMA loads
+        if (lid == 0) {
+            PhaseClock clk;
+            clk.start((a.dbg && blockIdx.x == 0) ? a.dbg + 20 : nullptr);
+            int issued_kq = 0, issued_fb = 0, issued_vc = 0;
+            for (int n = 0; n < NT; ++n) {
+                const int s2 = n & 1, sv = n % L::NVC;
+                const long long chunk = (long long)bh * NT + n;
+                if (n >= 2 && !wait_bar(&bars[B_M1 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
+                clk.lap(0);
+                uint64_t* fb = &bars[B_FKQ + s2];
+                mbar_arrive_expect_tx(fb, kTxKQ);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    uint8_t* dst = sm + L::KQ0 + s2 * 32768 + p * 16384;
+                    tma_load_4d(dst, &tm_k, p * 64, h, n * C, b, fb);
+                    tma_load_3d(dst + 8192, &tm_qh, p * 64, 0, (int)chunk, fb);
+                }
+                issued_kq = n + 1;
+                if (n >= 2 && !wait_bar(&bars[B_M3 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
+                clk.lap(1);
+                fb = &bars[B_FFB + s2];
+                mbar_arrive_expect_tx(fb, kTxFB);
+                uint8_t* dst = sm + L::FB0 + s2 * L::FB_BYTES;
+                tma_load_3d(dst, &tm_tat, 0, 0, (int)chunk, fb);
+                tma_load_3d(dst + 16384, &tm_a2t, 0, 0, (int)chunk, fb);
+                tma_load_3d(dst + 32768, &tm_a2t, 0, 128, (int)chunk, fb);
+                issued_fb = n + 1;
+                if (n >= L::NVC &&
+                    !wait_bar(&bars[B_EVC + sv], ((n / L::NVC) - 1) & 1, abort_flag))
+                    break;
+                clk.lap(2);
+                fb = &bars[B_FVC + sv];
+                mbar_arrive_expect_tx(fb, L::kTxVC);
+                tma_load_4d(sm + L::V0 + sv * L::V_BYTES, &tm_v, j0, h, n * C, b, fb);
+                bulk_load(sm + L::CR0 + sv * 1024, a.crec + chunk * 256, 1024, fb);
+                issued_vc = n + 1;
+            }
+            clk.flush();
+            // Copies that were issued must land before shared memory is
+            // released (after an abort some were never consumed).  A phase
+            // that has completed passes at once.
+            for (int n = issued_kq - 2; n < issued_kq; ++n)
+                if (n >= 0) (void)mbar_wait(&bars[B_FKQ + (n & 1)], (n >> 1) & 1);
+            for (int n = issued_fb - 2; n < issued_fb; ++n)
+                if (n >= 0) (void)mbar_wait(&bars[B_FFB + (n & 1)], (n >> 1) & 1);
+            for (int n = issued_vc - L::NVC; n < issued_vc; ++n)
+                if (n >= 0) (void)mbar_wait(&bars[B_FVC + n % L::NVC], (n / L::NVC) & 1);
+        }
+        __syncwarp();
+    } else if (chain) {
+        // ------------------------------------------------------------ chain epilogues
+        const bool ypart = quad < 2;  // lanes 0..63: rows of K, so this warp forms Y
+        const int r = lane & 63;
+        PhaseClock clk;
+        clk.start((a.dbg && blockIdx.x == 0 && warp == kChainWarp0 + 2 && lid == 0) ? a.dbg + 40 : nullptr);
+        for (int n = 0; n < NT; ++n) {
+            const int s2 = n & 1, sv = n % L::NVC;
+            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
+            clk.lap(0);
+            const float* cr = reinterpret_cast<const float*>(sm + L::CR0 + sv * 1024);
+            const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
+            if (ypart) {
+                const float c_ab = cr[r], c_d2 = cr[C + r];
+                const uint4* vrow =
+                    reinterpret_cast<const uint4*>(sm + L::V0 + sv * L::V_BYTES + r * (NS * 2)) + hc * (NH / 8);
+                if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
+                clk.lap(1);
+                tc_fence_after_sync();
+                const uint32_t a1 = tq + L::TM_A1 + 2 * NS * s2 + NH * hc;
+#pragma unroll
+                for (int q16 = 0; q16 < NH / 16; ++q16) {
+                    float x[16], y[16];
+                    tmem_ld16(a1 + 16 * q16, x);
+                    tmem_ld16(a1 + NS + 16 * q16, y);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float vv[8];
+                        unpack_bf16x8(vrow[2 * q16 + c], vv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) vv[e] -= fmaf(c_ab, x[8 * c + e], -c_d2 * y[8 * c + e]);
+                        st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + 2 * q16 + c), vv);
                     }
                 }
-                if (dump)
-                    for (int j = 0; j < NH; ++j) a.dbg[DBG_Y + r * NS + NH * hc + j] = yy[j];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) st_bf16x8(sm + YB + sw64_off(r, 2 * hc + c), yy + 8 * c);
+                clk.lap(2);
                 fence_proxy_async_smem();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lid == 0) {
+                    mbar_arrive(&bars[B_YR]);
+                    mbar_arrive(&bars[B_EVC + sv]);
+                }
+                clk.lap(3);
             } else {
-#pragma unroll
-                for (int j = 0; j < NH; ++j) oi[j] = c_ab * x[j] - c_b * y[j];
+                __syncwarp();
+                if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
             }
-        }
-        tc_fence_before_sync();
-        fail(mbar_wait(&bars[B_FB0 + buf], (n >> 1) & 1));
-        __syncthreads();
-        if (*abort_flag) break;
-        clk.lap(2);
-
-        // A2 = [A2T_S; A2T_M] Y, then A3 = [T; Att T] Y   (warp 0)
-        if (warp == 0) {
+            if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
+            clk.lap(4);
             tc_fence_after_sync();
-            const uint64_t da2 = d_a20 + buf * (32768 >> 4), dtat = d_tat0 + buf * (16384 >> 4);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t yd = d_y + ks * (1024 >> 4);
-                if (elect_one()) mma_bf16(tmem + TM_A2, da2 + ks * 2, yd, id2, ks > 0);
-                if (elect_one()) mma_bf16(tmem + TM_A2 + 32, da2 + (16384 >> 4) + ks * 2, yd, id2, ks > 0);
-            }
-            if (elect_one()) mma_commit(&bars[B_M2]);
+            for (int q16 = 0; q16 < NH / 16; ++q16) {
+                float dS[16], dM[16];
+                tmem_ld16(tq + L::TM_A2 + NH * hc + 16 * q16, dS);
+                tmem_ld16(tq + L::TM_A2 + NS + NH * hc + 16 * q16, dM);
+                tmem_wait_ld();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t yd = d_y + ks * (1024 >> 4);
-                if (elect_one()) mma_bf16(tmem + TM_A3, dtat + ks * 2, yd, id2, ks > 0);
+                for (int j = 0; j < 16; ++j) {
+                    const int jj = 16 * q16 + j;
+                    const float sn = fmaf(abC, s[jj], fmaf(-bC, m[jj], dS[j]));
+                    m[jj] = fmaf(mbC, m[jj], dM[j]);
+                    s[jj] = sn;
+                }
             }
-            if (elect_one()) mma_commit(&bars[B_M3]);
+#pragma unroll
+            for (int c = 0; c < NH / 8; ++c) {
+                st_bf16x8(sm + L::ST + L::s_off(lane, hc * (NH / 8) + c), s + 8 * c);
+                st_bf16x8(sm + L::ST + L::m_off(lane, hc * (NH / 8) + c), m + 8 * c);
+            }
+            clk.lap(5);
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
             __syncwarp();
+            if (lid == 0) mbar_arrive(&bars[B_SR]);
+            clk.lap(6);
         }
-        // K, Qhat, V and the coefficients of this buffer are no longer needed
-        if (producer && n + 2 < a.NT) load_a(n + 2);
-        fail(mbar_wait(&bars[B_M2], n & 1));
-        tc_fence_after_sync();
-        clk.lap(3);
-
-        // state update
-        {
-            float dS[NH], dM[NH];
-            tmem_ld16(tl + TM_A2, dS);
-            tmem_ld16(tl + TM_A2 + 32, dM);
-            tmem_wait_ld();
-            if (dump)
-                for (int j = 0; j < NH; ++j) {
-                    a.dbg[DBG_A2 + lane * 64 + NH * hc + j] = dS[j];
-                    a.dbg[DBG_A2 + lane * 64 + 32 + NH * hc + j] = dM[j];
-                }
+        clk.flush();
+    } else {
+        // ------------------------------------------------------------ outputs
+        const bool orow = quad >= 2;  // lanes 64..127: rows of o; lanes 0..63: rows of Vtilde
+        const int r = lane & 63;
+        __nv_bfloat16* const out = orow ? a.o : a.vt;
+        for (int n = 0; n < NT; ++n) {
+            const int s2 = n & 1, sv = n % L::NVC;
+            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
+            const float* cr = reinterpret_cast<const float*>(sm + L::CR0 + sv * 1024);
+            const float c_ab = cr[r], c_b = cr[2 * C + r];
+            __syncwarp();
+            if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
+            if (!warp_wait(&bars[B_M3 + s2], (n >> 1) & 1, abort_flag)) break;
+            tc_fence_after_sync();
+            const int t = n * C + r;
+            uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * a.T + t) * a.H + h) * D + j0);
+#pragma unroll 1
+            for (int q16 = 0; q16 < NS / 16; ++q16) {
+                float x[16], y[16];
+                if (orow) {
+                    tmem_ld16(tq + L::TM_A1 + 2 * NS * s2 + 16 * q16, x);       // Qhat S
+                    tmem_ld16(tq + L::TM_A1 + 2 * NS * s2 + NS + 16 * q16, y);  // Qhat M
+                    tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < NH; ++j) {
-                const float sn = fmaf(abC, s[j], fmaf(-bC, m[j], dS[j]));
-                m[j] = fmaf(mbC, m[j], dM[j]);
-                s[j] = sn;
-            }
+                    for (int j = 0; j < 16; ++j) x[j] = fmaf(c_ab, x[j], -c_b * y[j]);
+                    tmem_ld16(tq + L::TM_A3 + NS * s2 + 16 * q16, y);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                st_bf16x8(sm + ST + sw128_off(lane, 2 * hc + c), s + 8 * c);
-                st_bf16x8(sm + ST + sw128_off(lane, 4 + 2 * hc + c), m + 8 * c);
-            }
-            if (dump)
-                for (int j = 0; j < NH; ++j) {
-                    a.dbg[DBG_S + lane * NS + NH * hc + j] = s[j];
-                    a.dbg[DBG_M + lane * NS + NH * hc + j] = m[j];
+                    for (int j = 0; j < 16; ++j) x[j] += y[j];
+                } else {
+                    tmem_ld16(tq + L::TM_A3 + NS * s2 + 16 * q16, x);
+                    tmem_wait_ld();
                 }
+                if (t < a.T) {
+                    dst[2 * q16] = bf16x8(x);
+                    dst[2 * q16 + 1] = bf16x8(x + 8);
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lid == 0) mbar_arrive(&bars[B_OD + s2]);
         }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        clk.lap(4);
     }
-    ok = *abort_flag == 0;
-    clk.flush();
+
+    tc_fence_before_sync();
     __syncthreads();
-    ok = *abort_flag == 0;
-    if (ok && a.NT > 0) fail(store_outputs(a.NT - 1));
-    __syncthreads();
-    ok = *abort_flag == 0;
-    if (ok && producer && a.NT > 0) issue_stores(a.NT - 1);
-    if (producer) bulk_wait_group_all();  // every output tile has been written out
-    if (ok) {
+    const bool ok = *abort_flag == 0;
+    if (chain && ok) {
         const size_t row = ((size_t)bh * D + lane) * D + j0 + NH * hc;
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             a.S_T[row + j] = s[j];
             a.M_T[row + j] = m[j];
         }
-    } else if (producer) {
-        atomicOr(a.status + 1, 1u);
-        // Loads that were issued must land before the CTA's shared memory is
-        // released; only the last two chunks' buffers can still be in flight.
-        for (int n = a.NT - 2; n < a.NT; ++n)
-            if (n >= 0) {
-                (void)mbar_wait(&bars[B_FA0 + (n & 1)], (n >> 1) & 1);
-                (void)mbar_wait(&bars[B_FB0 + (n & 1)], (n >> 1) & 1);
-            }
     }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (!ok && tid == 0) atomicOr(a.status + 1, 1u);
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, L::kTmemCols);
+    }
 }
 
-}  // namespace
-
-cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s)
+template <int NS>
+cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
 {
-    CUtensorMap mk, mqh, mv, mtat, ma2t, mvt, mo;
+    using L = Cfg<NS>;
+    CUtensorMap mk, mqh, mv, mtat, ma2t;
     const long long chunks = (long long)a.B * a.H * a.NT;
     if (!make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
         !make_chunk_map(&mqh, a.qhat, chunks, C, D, C) ||
         !make_token_map(&mv, a.v, a.B, a.T, a.H, NS, false) ||
         !make_chunk_map(&mtat, a.tat, chunks, 2 * C, C, 2 * C) ||
-        !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128) ||
-        !make_token_map(&mvt, a.vt, a.B, a.T, a.H, NS, false) ||
-        !make_token_map(&mo, a.o, a.B, a.T, a.H, NS, false))
+        !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
     InterArgs t;
     t.crec = a.crec;
@@ -418,29 +501,39 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s)
     t.T = a.T;
     t.H = a.H;
     t.NT = a.NT;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_inter_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = cudaFuncSetAttribute(chunk_inter_kernel<NS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     const long long blocks = (long long)a.B * a.H * (D / NS);
     ProfScope ps(kInterTc, s);
-    chunk_inter_kernel<<<(unsigned)blocks, kThreads, SMEM_BYTES, s>>>(mk, mqh, mv, mtat, ma2t, mvt,
-                                                                       mo, t);
+    chunk_inter_kernel<NS><<<(unsigned)blocks, L::kThreads, L::SMEM_BYTES, s>>>(mk, mqh, mv, mtat, ma2t, t);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// Slice width: 64 columns (two CTAs per head) when that already gives one CTA
+// per SM or more, otherwise 32 (four per head) to spread short batches.
+cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s, int ns)
+{
+    if (ns == 0) {
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        ns = (long long)a.B * a.H * 2 >= sms ? 64 : 32;
+    }
+    return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
 }
 
 // The tensor-core path: the intra-chunk kernel, then the sequential
 // inter-chunk kernel, both on stream s.
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s)
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
     cudaError_t e = launch_chunk_intra_tc(a, s);
     if (e != cudaSuccess) return e;
-    return launch_chunk_inter_tc(a, s);
+    return launch_chunk_inter_tc(a, s, ns);
 }
 
 }  // namespace mdn

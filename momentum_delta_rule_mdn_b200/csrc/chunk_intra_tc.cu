@@ -91,6 +91,11 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* wg = wv + C;    // Gamma_{C,r}
     PhaseClock clk;
     clk.start((a.dbg && chunk == 0 && tid == 0) ? a.dbg : nullptr);
+#ifdef MDN_PHASE_CLOCKS
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    const uint64_t t_begin = global_timer_ns();
+#endif
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -420,6 +425,14 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+#ifdef MDN_PHASE_CLOCKS
+    if (a.dbg && tid == 0 && chunk < 4096) {
+        double* tl = reinterpret_cast<double*>(a.dbg + 64);
+        tl[3 * chunk] = (double)t_begin;
+        tl[3 * chunk + 1] = (double)global_timer_ns();
+        tl[3 * chunk + 2] = (double)smid;
+    }
+#endif
 }
 
 }  // namespace

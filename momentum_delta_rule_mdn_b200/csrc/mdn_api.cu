@@ -3,6 +3,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <cstdio>
+
 #include "mdn_internal.cuh"
 
 using namespace mdn;
@@ -60,9 +62,26 @@ mdn_status check_sizes(int B, int T, int H, int dk, int dv, int C, mdn_dtype dt)
     return MDN_OK;
 }
 
-mdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDN_OK : MDN_ERR_CUDA; }
+mdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDN_OK : mdn::cuda_fail(e); }
 
 }  // namespace
+
+// ---------------------------------------------------------------- CUDA errors
+namespace mdn {
+namespace {
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+thread_local char t_last_cuda_text[160] = "no CUDA error recorded on this thread";
+}  // namespace
+mdn_status cuda_fail(cudaError_t e)
+{
+    t_last_cuda_error = e;
+    snprintf(t_last_cuda_text, sizeof(t_last_cuda_text), "%s (%d): %s", cudaGetErrorName(e),
+             (int)e, cudaGetErrorString(e));
+    return MDN_ERR_CUDA;
+}
+}  // namespace mdn
+
+extern "C" const char* mdn_last_cuda_error(void) { return mdn::t_last_cuda_text; }
 
 // ---------------------------------------------------------------- finite check
 namespace mdn {
@@ -130,7 +149,9 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 {
     mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
     if (st != MDN_OK) return st;
-    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT)) return MDN_ERR_INVALID_ARG;
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64))
+        return MDN_ERR_INVALID_ARG;
+    if ((flags & MDN_SLICE32) && (flags & MDN_SLICE64)) return MDN_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return MDN_OK;
     if (!S_T || !M_T || !aligned16(S_T) || !aligned16(M_T)) return MDN_ERR_INVALID_ARG;
     if ((S0 && !aligned16(S0)) || (M0 && !aligned16(M0))) return MDN_ERR_INVALID_ARG;
@@ -182,28 +203,29 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 
     cudaError_t e;
     const bool check = flags & MDN_CHECK_FINITE;
-    if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return MDN_ERR_CUDA;
+    if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
     const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
     if (tensor_cores) {
-        if ((e = launch_chunk_tc(a, s))) return MDN_ERR_CUDA;
+        const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
+        if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
     } else {
         if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
                                   a.gamma, s)))
-            return MDN_ERR_CUDA;
-        if ((e = launch_chunk_simt(a, in_dtype, s))) return MDN_ERR_CUDA;
+            return mdn::cuda_fail(e);
+        if ((e = launch_chunk_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
     }
     if (!check) return MDN_OK;
 
     const size_t ntok = (size_t)B * T * H * D;
     const bool bf = in_dtype == MDN_BF16;
-    if ((e = launch_finite_check(o, ntok, bf, a.status, s))) return MDN_ERR_CUDA;
-    if ((e = launch_finite_check(vtilde, ntok, bf, a.status, s))) return MDN_ERR_CUDA;
-    if ((e = launch_finite_check(S_T, (size_t)B * H * D * D, false, a.status, s))) return MDN_ERR_CUDA;
-    if ((e = launch_finite_check(M_T, (size_t)B * H * D * D, false, a.status, s))) return MDN_ERR_CUDA;
+    if ((e = launch_finite_check(o, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(vtilde, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(S_T, (size_t)B * H * D * D, false, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(M_T, (size_t)B * H * D * D, false, a.status, s))) return mdn::cuda_fail(e);
     unsigned host_status[2] = {0, 0};
     if ((e = cudaMemcpyAsync(host_status, a.status, sizeof(host_status), cudaMemcpyDeviceToHost, s)))
-        return MDN_ERR_CUDA;
-    if ((e = cudaStreamSynchronize(s))) return MDN_ERR_CUDA;
+        return mdn::cuda_fail(e);
+    if ((e = cudaStreamSynchronize(s))) return mdn::cuda_fail(e);
     if (host_status[1]) return MDN_ERR_TIMEOUT;
     if (host_status[0]) return MDN_ERR_NONFINITE;
     return MDN_OK;

@@ -128,9 +128,12 @@ cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const 
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s);
+// Records e as this thread's last CUDA error (mdn_last_cuda_error) and
+// returns MDN_ERR_CUDA.
+mdn_status cuda_fail(cudaError_t e);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);  // ns: see launch_chunk_inter_tc
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s);
-cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s);
+cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s, int ns);  // ns = 0: choose
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
                         const float* eta, float dcorr, float* S, float* M, int B, int H,

@@ -50,7 +50,8 @@ extern "C" mdn_status mdn_chunk_fwd_noalloc(
     const size_t need = mdn_chunk_fwd_workspace_size(B, T, H, dk, dv, C, in_dtype);
     if (need > kStaticScratchBytes) return MDN_ERR_UNSUPPORTED;
     void* ws = nullptr;
-    if (scratch_on_current_device(&ws) != cudaSuccess) return MDN_ERR_CUDA;
+    const cudaError_t e = scratch_on_current_device(&ws);
+    if (e != cudaSuccess) return mdn::cuda_fail(e);
     return mdn_chunk_fwd(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S0, M0, B, T,
                          H, dk, dv, C, o, vtilde, S_T, M_T, ws, kStaticScratchBytes, flags,
                          stream);

@@ -75,7 +75,9 @@ __device__ __forceinline__ long long clock_now() {
     return t;
 }
 // Cycle counts of a kernel's phases, summed over chunks in registers and
-// written out once (diagnostic dump only; inert when `out` is null).
+// written out once.  Diagnostic builds only (MDN_PHASE_CLOCKS); otherwise
+// every call is empty and costs nothing.
+#ifdef MDN_PHASE_CLOCKS
 struct PhaseClock {
     static constexpr int kMax = 20;
     float* out;
@@ -99,6 +101,13 @@ struct PhaseClock {
             for (int k = 0; k < kMax; ++k) out[k] += acc[k];
     }
 };
+#else
+struct PhaseClock {
+    __device__ __forceinline__ void start(float*) {}
+    __device__ __forceinline__ void lap(int) {}
+    __device__ __forceinline__ void flush() {}
+};
+#endif
 
 // ------------------------------------------------------------------ host side
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn()

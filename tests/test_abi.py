@@ -87,6 +87,7 @@ def test_chunk_fwd_validation(lib):
     assert _chunk(lib, B=-1) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, C=0) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, flags=0x100) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, flags=_lib.MDN_SLICE32 | _lib.MDN_SLICE64) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, q=None) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, vt=None) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, ST=None) == E.MDN_ERR_INVALID_ARG

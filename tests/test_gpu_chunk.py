@@ -55,7 +55,17 @@ def test_small_cases(name, B, T, H, d, dtype, std):
     compare_heads(run(inp), inp, all_heads(inp.spec), TOL[dtype])
 
 
-@pytest.mark.parametrize("flags", [0, _lib.MDN_FORCE_SIMT])
+@pytest.mark.parametrize("flags", [_lib.MDN_SLICE32, _lib.MDN_SLICE64])
+@pytest.mark.parametrize("name,B,T,H", [("ragged", 2, 200, 3), ("T1", 1, 1, 2), ("T65", 1, 65, 1),
+                                         ("long", 1, 1000, 2)])
+def test_inter_slice_widths(name, B, T, H, flags):
+    """Both column-slice widths of the inter-chunk kernel against the oracle."""
+    inp = mi.make_inputs(mi.Spec("slice_" + name, B=B, T=T, H=H, d=128, dtype="bf16",
+                                 state_std=0.01, seed=zlib.crc32(name.encode()) % 1000 + 3000))
+    compare_heads(run(inp, flags=flags), inp, all_heads(inp.spec), TOL["bf16"])
+
+
+@pytest.mark.parametrize("flags", [0, _lib.MDN_FORCE_SIMT, _lib.MDN_SLICE32, _lib.MDN_SLICE64])
 @pytest.mark.parametrize("cfg,heads", [
     (1, [(0, 0), (1, 3), (2, 7), (3, 5)]),
     (2, [(0, 0), (3, 9), (5, 15), (7, 2)]),
