@@ -1,17 +1,17 @@
-// K-2 on sm_100a: the intra-chunk part of the chunkwise MDN forward pass,
-// one CTA per chunk, all chunks in parallel.
+// K-2 on sm_100a: the intra-chunk part of the chunkwise MDN forward pass.
 //
 // "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
 // paper.rainbus.top summary, steps 3-5.  Per chunk (positions r, i inside it):
 //   Qhat   = Q - d K
 //   G      = [K; Qhat] [K; Qhat]^T     tcgen05.mma, M=128, N=128, K=128, bf16 in, fp32 in TMEM
-//            lane i < 64: k_i.k_r (cols 0..63);  lane 64+r: qhat_r.k_i (cols 0..63)
+//            lane i < 64: k_i.k_r (columns r), k_i.qhat_r (columns 64 + r)
 //   Gamma  down each column i by Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r mubar_r/mubar_i
 //          (mubar_r/mubar_i as a running product of mu: non-negative terms only)
 //   A      = (P K^T) o Gamma-:  A_{r,i} = alpha_r k_r.k_i Gamma_{r-1,i}  (i < r)
 //   Att    = (Qhat K^T) o Gamma:  Att_{r,i} = qhat_r.k_i Gamma_{r,i}  (i <= r)
-//   T      = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution, then the
-//            off-diagonal blocks by distance from the diagonal, fp32
+//   T      = (I + A)^{-1} in fp32 over 16 x 16 blocks: diagonal blocks by forward
+//            substitution, B_ik = -T_ii A_ik, then T_ij = sum_{k=j}^{i-1} B_ik T_kj
+//            by distance from the diagonal
 //   P      = [I; Att] T = [T; Att T]                    (M=128, N=64,  K=64)
 //   R      = K^T [Diag(Gamma_C) T | -Diag(w) T]          (M=128, N=128, K=64)
 //            with w_r = eta_r mubar_C / mubar_r
@@ -19,6 +19,15 @@
 // bf16: Qhat [64 x 128], [T; Att T] [128 x 64], A2T = [R_S; R_M] [256 x 64],
 // plus the per-position coefficients alphabar_r, alpha_r b_{r-1}, b_r and the
 // chunk scalars alphabar_C, b_C, mubar_C (fp32).
+//
+// The CTAs are persistent (two per SM) and take chunks in chunk-major order
+// (chunk 0 of every head first).  K and Q of a CTA's next chunk are loaded by
+// TMA into a second buffer while the current chunk computes, and the gate
+// scan of the next chunk runs on the warps that the column pass leaves idle.
+// Column i of Gamma never leaves the registers of the thread that owns it:
+// that thread writes column i of A and K-row i of the MN-major [I; Att]
+// operand directly.  T is solved in place over A: the diagonal blocks replace
+// A_ii, B_ik replaces A_ik, and T_ij (i > j) goes to the unused block (j, i).
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -29,42 +38,101 @@ using namespace sm100;
 using namespace tc;
 
 constexpr int kThreads = 128;
-constexpr uint32_t KQ = 0;                   // [K; Qhat], 2 feature panels x (128 rows x 128 B)
-constexpr uint32_t GM = 32768;               // fp32 [64][LDF] Gamma;  later [D_G T | -D_w T] bf16
-constexpr uint32_t AM = GM + 64 * LDF * 4;   // fp32 [64][LDF] A (upper blocks: scratch); later T bf16
-constexpr uint32_t TMF = AM + 64 * LDF * 4;  // fp32 [64][LDF] T
-constexpr uint32_t IATT = TMF + 64 * LDF * 4;// [I; Att] 128 x 64 bf16, K-major SW128
-constexpr uint32_t REC = IATT + 16384;       // record rows 0..5
-constexpr uint32_t VEC = REC + 1536;         // mu_r, w_r, Gamma_{C,r}
+// Shared memory (byte offsets from a 1024-byte aligned base).
+constexpr uint32_t KQ0 = 0;                   // [K; Q] of a chunk, 2 buffers; a buffer holds 2
+                                              // feature panels of (64 rows of K, 64 rows of Q) x 128 B
+constexpr uint32_t KQ_BYTES = 32768;
+constexpr uint32_t AM = 2 * KQ_BYTES;         // fp32 [64][LDF]: A, then T and B in place
+constexpr uint32_t IATT = AM + 17408;         // [I; Att] MN-major: 2 M-panels x 64 K-rows x 128 B
+constexpr uint32_t DT1 = IATT + 16384;        // N-panel 1 of [D_G T | -D_w T] (8 KB)
+constexpr uint32_t REC = DT1 + 8192;          // gate record, 2 buffers x 6 x 64 floats
+constexpr uint32_t VEC = REC + 2 * 1536;      // mu_r, w_r, Gamma_{C,r}
 constexpr uint32_t BARS = VEC + 768;
-constexpr uint32_t MISC = BARS + 16;
-constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
-constexpr uint32_t DT = GM;                  // aliases: written after Gamma and A are dead
-constexpr uint32_t TB = AM;
-static_assert(GM % 1024 == 0 && AM % 1024 == 0 && IATT % 1024 == 0, "operand alignment");
-static_assert(SMEM_BYTES <= 116 * 1024, "two CTAs per SM");
+constexpr uint32_t MISC = BARS + 32;
+constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
+static_assert(AM % 1024 == 0 && IATT % 1024 == 0 && DT1 % 1024 == 0, "operand alignment");
+static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
+// Aliases, each written only once its previous contents are dead.
+constexpr uint32_t TB_OFF = 8192;    // T bf16 (B of P): the Q half of panel 0 of the current buffer
+constexpr uint32_t DT0_OFF = 24576;  // N-panel 0 of [D_G T | -D_w T] (B of R): the Q half of panel 1
+constexpr uint32_t STG_TAT = AM;     // [T; Att T] staging: over T once the bf16 copies are made
+// TMEM columns
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t TM_G = 0, TM_P = 0, TM_R = 128;  // P reuses G's columns once G is read
-constexpr uint32_t kTxBytes = 32768;
-// staging of the outputs for the TMA stores (regions dead by then)
-constexpr uint32_t STG_TAT = IATT;           // 128 x 64 bf16
-constexpr uint32_t STG_A2T = GM;             // 256 x 64 bf16 (spans GM and AM)
-static_assert(STG_A2T + 32768 <= TMF, "A2T staging overlaps T");
+// mbarriers: two K/Q buffers, one for the MMA commits
+constexpr int B_LD = 0, B_MMA = 2;
 
 struct IntraArgs {
     const float* alpha_log;  // [B, T, H] gates
     const float* mu_log;
     const float* beta;
     const float* eta;
-    __nv_bfloat16* qhat;   // [chunks][64][128]
-    __nv_bfloat16* tat;    // [chunks][128][64]
-    __nv_bfloat16* a2t;    // [chunks][256][64]
-    float* crec;           // [chunks][256]
+    float* crec;             // [chunks][256]
     unsigned* status;
-    float* dbg;            // diagnostics: phase clocks of CTA 0 (null in normal use)
+    float* dbg;              // diagnostics: phase clocks of CTA 0 (null in normal use)
     float dcorr;
-    int T, H, NT;
+    int T, H, NT, BH;
 };
+
+// Chunk-major order: the c-th chunk is chunk n of head bh; returns its index
+// in the head-major layout of the workspace.
+__device__ __forceinline__ long long chunk_of(long long c, const IntraArgs& a, int& n, int& bh) {
+    n = (int)(c / a.BH);
+    bh = (int)(c % a.BH);
+    return (long long)bh * a.NT + n;
+}
+
+// Gate record of one chunk (one warp): la, lm, b, alpha, beta, eta per
+// position; positions past T are steps that leave the state unchanged.
+__device__ __forceinline__ void gate_record(const IntraArgs& a, int n, int bh, float* rec, int lane) {
+    const int b = bh / a.H, h = bh % a.H;
+    const int t0 = n * C + 2 * lane;
+    float ga[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gb[2] = {0.f, 0.f}, ge[2] = {0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        if (t0 + e < a.T) {
+            const size_t gi = ((size_t)b * a.T + t0 + e) * a.H + h;
+            ga[e] = a.alpha_log[gi];
+            gm[e] = a.mu_log[gi];
+            gb[e] = a.beta[gi];
+            ge[e] = a.eta[gi];
+        }
+    }
+    float la[2], lm[2], lc[2];
+    chunk_log_coeffs(ga, gm, gb, lane, la, lm, lc);
+    float2* r2 = reinterpret_cast<float2*>(rec) + lane;
+    r2[0] = make_float2(la[0], la[1]);
+    r2[32] = make_float2(lm[0], lm[1]);
+    r2[64] = make_float2(expf(la[0] + lc[0]), expf(la[1] + lc[1]));
+    r2[96] = make_float2(expf(ga[0]), expf(ga[1]));
+    r2[128] = make_float2(gb[0], gb[1]);
+    r2[160] = make_float2(ge[0], ge[1]);
+}
+
+// acc += rows r0, r0 + 1 of X times columns c0 .. c0 + 3 of Y, for 16 x 16
+// blocks X (at x) and Y (at y), both with row stride LDF.
+__device__ __forceinline__ void tile_2x4(const float* x, const float* y, int r0, int c0,
+                                         float4& acc0, float4& acc1) {
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 a0 = lds4(x + r0 * LDF + 4 * k4);
+        const float4 a1 = lds4(x + (r0 + 1) * LDF + 4 * k4);
+        const float x0[4] = {a0.x, a0.y, a0.z, a0.w};
+        const float x1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float4 t4 = lds4(y + (4 * k4 + e) * LDF + c0);
+            acc0.x = fmaf(x0[e], t4.x, acc0.x);
+            acc0.y = fmaf(x0[e], t4.y, acc0.y);
+            acc0.z = fmaf(x0[e], t4.z, acc0.z);
+            acc0.w = fmaf(x0[e], t4.w, acc0.w);
+            acc1.x = fmaf(x1[e], t4.x, acc1.x);
+            acc1.y = fmaf(x1[e], t4.y, acc1.y);
+            acc1.z = fmaf(x1[e], t4.z, acc1.z);
+            acc1.w = fmaf(x1[e], t4.w, acc1.w);
+        }
+    }
+}
 
 __global__ void __launch_bounds__(kThreads)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -75,75 +143,65 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const long long chunk = blockIdx.x;
-    const int n = (int)(chunk % a.NT);
-    const long long bh = chunk / a.NT;
-    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long chunks = (long long)a.BH * a.NT;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BARS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
-    float* Gm = reinterpret_cast<float*>(sm + GM);
     float* Am = reinterpret_cast<float*>(sm + AM);
-    float* Tm = reinterpret_cast<float*>(sm + TMF);
-    float* rec = reinterpret_cast<float*>(sm + REC);
     float* mu = reinterpret_cast<float*>(sm + VEC);
     float* wv = mu + C;    // w_r = eta_r mubar_C / mubar_r
     float* wg = wv + C;    // Gamma_{C,r}
     PhaseClock clk;
-    clk.start((a.dbg && chunk == 0 && tid == 0) ? a.dbg : nullptr);
+    clk.start((a.dbg && blockIdx.x == 0 && tid == 0) ? a.dbg : nullptr);
 #ifdef MDN_PHASE_CLOCKS
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
     const uint64_t t_begin = global_timer_ns();
 #endif
 
-    if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_fence_init();
-        mbar_arrive_expect_tx(&bars[0], kTxBytes);
+    // K and Q of the c-th chunk into buffer buf (thread 0); the pending load
+    // is remembered so that an abort can drain it.
+    int pend_buf = -1;
+    uint32_t pend_par = 0;
+    auto load_kq = [&](long long c, int iter) {
+        int n, bh;
+        (void)chunk_of(c, a, n, bh);
+        const int b = bh / a.H, h = bh % a.H, buf = iter & 1;
+        uint64_t* bar = &bars[B_LD + buf];
+        mbar_arrive_expect_tx(bar, KQ_BYTES);
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-            tma_load_4d(sm + KQ + p * 16384, &tm_k, p * 64, h, n * C, b, &bars[0]);
-            tma_load_4d(sm + KQ + p * 16384 + 8192, &tm_q, p * 64, h, n * C, b, &bars[0]);
+            uint8_t* dst = sm + KQ0 + buf * KQ_BYTES + p * 16384;
+            tma_load_4d(dst, &tm_k, p * 64, h, n * C, b, bar);
+            tma_load_4d(dst + 8192, &tm_q, p * 64, h, n * C, b, bar);
         }
+        pend_buf = buf;
+        pend_par = (iter >> 1) & 1;
+    };
+
+    if (tid == 0) {
+        mbar_init(&bars[B_LD], 1);
+        mbar_init(&bars[B_LD + 1], 1);
+        mbar_init(&bars[B_MMA], 1);
+        mbar_fence_init();
+        if (blockIdx.x < chunks) load_kq(blockIdx.x, 0);
     }
-    if (warp == 3) {
-        // per-position coefficients: la, lm, b, alpha, beta, eta (positions past T are
-        // steps that leave the state unchanged)
-        const int lane = tid & 31;
-        const int t0 = n * C + 2 * lane;
-        float ga[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gb[2] = {0.f, 0.f}, ge[2] = {0.f, 0.f};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            if (t0 + e < a.T) {
-                const size_t gi = ((size_t)b * a.T + t0 + e) * a.H + h;
-                ga[e] = a.alpha_log[gi];
-                gm[e] = a.mu_log[gi];
-                gb[e] = a.beta[gi];
-                ge[e] = a.eta[gi];
-            }
-        }
-        float la[2], lm[2], lc[2];
-        chunk_log_coeffs(ga, gm, gb, lane, la, lm, lc);
-        float2* r2 = reinterpret_cast<float2*>(rec) + lane;
-        r2[0] = make_float2(la[0], la[1]);
-        r2[32] = make_float2(lm[0], lm[1]);
-        r2[64] = make_float2(expf(la[0] + lc[0]), expf(la[1] + lc[1]));
-        r2[96] = make_float2(expf(ga[0]), expf(ga[1]));
-        r2[128] = make_float2(gb[0], gb[1]);
-        r2[160] = make_float2(ge[0], ge[1]);
+    if (warp == 3 && blockIdx.x < chunks) {
+        int n, bh;
+        (void)chunk_of(blockIdx.x, a, n, bh);
+        gate_record(a, n, bh, reinterpret_cast<float*>(sm + REC), lane);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (tid < C) {  // identity rows 0..63 of [I; Att]
-        for (int c = 0; c < 8; ++c) {
+    if (tid < C) {  // K-row tid of the identity M-panel of [I; Att]; never overwritten
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = (8 * c + e == tid) ? 1.f : 0.f;
-            st_bf16x8(sm + IATT + sw128_off(tid, c), x);
+            for (int e = 0; e < 8; ++e) x[e] = (8 * cc + e == tid) ? 1.f : 0.f;
+            st_bf16x8(sm + IATT + sw128_off(tid, cc), x);
         }
     }
     tc_fence_before_sync();
@@ -152,16 +210,32 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
 
-    bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
-    clk.lap(0);
-    if (ok) {
-        // Qhat = Q - d K in place (rows 64..127 of both panels) and to global memory
+    bool ok = true;
+    uint32_t mma_phase = 0;
+    int k = 0;
+    for (long long c = blockIdx.x; c < chunks; c += gridDim.x, ++k) {
+        const int buf = k & 1;
+        uint8_t* kq = sm + KQ0 + buf * KQ_BYTES;
+        const uint32_t kq_s = sbase + KQ0 + buf * KQ_BYTES;
+        const float* rec = reinterpret_cast<const float*>(sm + REC + buf * 1536);
+        int n, bh;
+        const long long chunk = chunk_of(c, a, n, bh);
+        const long long c_next = c + gridDim.x;
+        // A is about to be overwritten: the store of [T; Att T] from its staging
+        // tile (all store groups but the newest) must have read it
+        if (tid == 0) bulk_wait_group_read<1>();
+        ok = __syncthreads_and(mbar_wait(&bars[B_LD + buf], (k >> 1) & 1));
+        if (!ok) break;
+        if (tid == 0 && pend_buf == buf) pend_buf = -1;
+        clk.lap(0);
+
+        // ---- Qhat = Q - d K in place (the Q rows of both panels); chunk record
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u;
-            const int pn = idx >> 9, w = idx & 511, r = w >> 3, c = w & 7;
-            const uint4 kw = *reinterpret_cast<const uint4*>(sm + KQ + pn * 16384 + sw128_off(r, c));
-            uint8_t* qp = sm + KQ + pn * 16384 + sw128_off(r + 64, c);
+            const int pn = idx >> 9, w = idx & 511, r = w >> 3, cc = w & 7;
+            const uint4 kw = *reinterpret_cast<const uint4*>(kq + pn * 16384 + sw128_off(r, cc));
+            uint8_t* qp = kq + pn * 16384 + sw128_off(r + 64, cc);
             float kx[8], qx[8];
             unpack_bf16x8(kw, kx);
             unpack_bf16x8(*reinterpret_cast<const uint4*>(qp), qx);
@@ -190,247 +264,284 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncthreads();
         clk.lap(1);
         if (tid == 0) {
-            // Qhat (rows 64..127 of both panels) to global memory
-            tma_store_3d(&tm_qh, 0, 0, (int)chunk, sm + KQ + 8192);
-            tma_store_3d(&tm_qh, 64, 0, (int)chunk, sm + KQ + 16384 + 8192);
+            tma_store_3d(&tm_qh, 0, 0, (int)chunk, kq + 8192);
+            tma_store_3d(&tm_qh, 64, 0, (int)chunk, kq + 16384 + 8192);
             bulk_commit_group();
             tc_fence_after_sync();
             const uint32_t id = idesc_bf16(128, 128, false, false);
+#pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t ad =
-                    smem_desc(sbase + KQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128);
+                    smem_desc(kq_s + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128);
                 mma_bf16(tmem + TM_G, ad, ad, id, ks > 0);
             }
-            mma_commit(&bars[1]);
+            mma_commit(&bars[B_MMA]);
         }
-        ok = mbar_wait(&bars[1], 0);
+        ok = mbar_wait(&bars[B_MMA], mma_phase);
+        mma_phase ^= 1;
         tc_fence_after_sync();
         ok = __syncthreads_and(ok);
+        if (!ok) break;
         clk.lap(2);
-    }
-    if (ok) {
-        // lane i < 64: k_i.k_r;  lane 64 + r: qhat_r.k_i   (columns 0..63)
-        float gv[64];
-        tmem_ld32(tmem + lane_sel + TM_G, *reinterpret_cast<float(*)[32]>(gv));
-        tmem_ld32(tmem + lane_sel + TM_G + 32, *reinterpret_cast<float(*)[32]>(gv + 32));
-        tmem_wait_ld();
+
+        // ---- column pass: thread i < 64 owns column i of Gamma, A and Att
         if (tid < C) {
-            // column i of Gamma and A
+            if (tid == 0 && c_next < chunks) {
+                // K, Q of the next chunk into the other buffer, once the stores of the
+                // previous chunk's A2T (all groups but the newest, Qhat) have read it
+                bulk_wait_group_read<1>();
+                load_kq(c_next, k + 1);
+            }
             const int i = tid;
             const float* al = rec + 3 * C;
             const float* be = rec + 4 * C;
             const float eta_i = rec[5 * C + i];
             float gam = 0.f, f = 1.f;
 #pragma unroll
-            for (int r4 = 0; r4 < C; r4 += 4) {
-                const float4 a4 = lds4(al + r4), b4 = lds4(be + r4), m4 = lds4(mu + r4);
-                const float ar_[4] = {a4.x, a4.y, a4.z, a4.w};
-                const float br_[4] = {b4.x, b4.y, b4.z, b4.w};
-                const float mr_[4] = {m4.x, m4.y, m4.z, m4.w};
+            for (int r16 = 0; r16 < C; r16 += 16) {
+                float kk[16], kh[16];
+                tmem_ld16(tmem + lane_sel + TM_G + r16, kk);      // k_i.k_r
+                tmem_ld16(tmem + lane_sel + TM_G + C + r16, kh);  // k_i.qhat_r
+                tmem_wait_ld();
+                float att[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = r4 + e;
-                    Am[r * LDF + i] = (r > i) ? ar_[e] * gv[r] * gam : 0.f;
-                    f = (r > i) ? f * mr_[e] : 1.f;
-                    gam = (r >= i) ? fmaf(ar_[e], gam, eta_i * br_[e] * f) : 0.f;
-                    Gm[r * LDF + i] = gam;
+                for (int r4 = 0; r4 < 16; r4 += 4) {
+                    const float4 a4 = lds4(al + r16 + r4), b4 = lds4(be + r16 + r4),
+                                 m4 = lds4(mu + r16 + r4);
+                    const float ar_[4] = {a4.x, a4.y, a4.z, a4.w};
+                    const float br_[4] = {b4.x, b4.y, b4.z, b4.w};
+                    const float mr_[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r16 + r4 + e;
+                        Am[r * LDF + i] = (r > i) ? ar_[e] * kk[r4 + e] * gam : 0.f;
+                        f = (r > i) ? f * mr_[e] : 1.f;
+                        gam = (r >= i) ? fmaf(ar_[e], gam, eta_i * br_[e] * f) : 0.f;
+                        att[r4 + e] = kh[r4 + e] * gam;  // gam = 0 above the diagonal
+                    }
                 }
+                // column i of Att, rows r16 .. r16 + 15: M-panel 1, K-row i
+                st_bf16x8(sm + IATT + 8192 + sw128_off(i, r16 / 8), att);
+                st_bf16x8(sm + IATT + 8192 + sw128_off(i, r16 / 8 + 1), att + 8);
             }
             wg[i] = gam;  // Gamma_{C,i}
-        } else {
-            // zero the six blocks of T above the diagonal
-            for (int idx = tid - C; idx < 6 * 64; idx += 64) {
-                const int blkid = idx >> 6, e = idx & 63;
-                const int bi = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
-                const int bj = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
-                *reinterpret_cast<float4*>(Tm + (16 * bi + (e >> 2)) * LDF + 16 * bj + 4 * (e & 3)) =
-                    make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        } else if (warp == 3 && c_next < chunks) {
+            int n2, bh2;
+            (void)chunk_of(c_next, a, n2, bh2);
+            gate_record(a, n2, bh2, reinterpret_cast<float*>(sm + REC + (buf ^ 1) * 1536), lane);
         }
         __syncthreads();
         clk.lap(3);
-        if (tid >= C) {
-            // row r of Att into rows 64..127 of [I; Att]
-            const int r = tid - C;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 g0 = lds4(Gm + r * LDF + 8 * c), g1 = lds4(Gm + r * LDF + 8 * c + 4);
-                const float gr[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = (8 * c + e <= r) ? gv[8 * c + e] * gr[e] : 0.f;
-                st_bf16x8(sm + IATT + sw128_off(tid, c), x);
-            }
-        } else {
-            // diagonal 16x16 blocks of T by forward substitution, one column per thread
-            const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
+
+        // ---- diagonal blocks of T by forward substitution, one column per thread
+        {
+            const int blk = tid >> 4, cl = tid & 15, o = 16 * blk;
             float t[16];
+            if (tid < C) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) t[r] = (r == c) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) t[r] = (r == cl) ? 1.f : 0.f;
 #pragma unroll
-            for (int r = 1; r < 16; ++r) {
-                float av[16];
+                for (int r = 1; r < 16; ++r) {
+                    float av[16];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 v4 = lds4(Am + (o + r) * LDF + o + 4 * q4);
-                    av[4 * q4] = v4.x;
-                    av[4 * q4 + 1] = v4.y;
-                    av[4 * q4 + 2] = v4.z;
-                    av[4 * q4 + 3] = v4.w;
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 v4 = lds4(Am + (o + r) * LDF + o + 4 * q4);
+                        av[4 * q4] = v4.x;
+                        av[4 * q4 + 1] = v4.y;
+                        av[4 * q4 + 2] = v4.z;
+                        av[4 * q4 + 3] = v4.w;
+                    }
+                    float acc = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < r; ++kk) acc = fmaf(av[kk], t[kk], acc);
+                    if (r > cl) t[r] = -acc;
                 }
-                float acc = 0.f;
-#pragma unroll
-                for (int k = 0; k < r; ++k) acc = fmaf(av[k], t[k], acc);
-                if (r > c) t[r] = -acc;
             }
+            __syncthreads();  // A_ii has been read
+            if (tid < C) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(o + r) * LDF + o + c] = t[r];
+                for (int r = 0; r < 16; ++r) Am[(o + r) * LDF + o + cl] = t[r];
+            }
         }
         __syncthreads();
         clk.lap(4);
-        // Off-diagonal blocks by distance L: W = sum_{k=j}^{i-1} A_{i,k} T_{k,j},
-        // T_{i,j} = -T_{i,i} W (j = i - L).  W goes to block (L-1, i) of Am.  A
-        // thread owns a 2 x 4 tile of a block.
+
+        // ---- B_ik = -T_ii A_ik for the six blocks below the diagonal, in place
+        {
+            // blocks (i, k): (1,0) (2,0) (2,1) (3,0) (3,1) (3,2), 32 tiles of 2 x 4 each
+            float4 res[2][2];
+            int where[2];
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+                const int tile = tid + 128 * rep;
+                where[rep] = -1;
+                if (tile < 192) {
+                    const int bidx = tile >> 5;
+                    const int bi = bidx < 1 ? 1 : (bidx < 3 ? 2 : 3);
+                    const int bk = bidx < 1 ? 0 : (bidx < 3 ? bidx - 1 : bidx - 3);
+                    const int r0 = 2 * ((tile >> 2) & 7), c0 = 4 * (tile & 3);
+                    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+                    tile_2x4(Am + 16 * bi * LDF + 16 * bi, Am + 16 * bi * LDF + 16 * bk, r0, c0,
+                             acc0, acc1);
+                    res[rep][0] = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
+                    res[rep][1] = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
+                    where[rep] = (16 * bi + r0) * LDF + 16 * bk + c0;
+                }
+            }
+            __syncthreads();  // every read of A_ik precedes its overwrite
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep)
+                if (where[rep] >= 0) {
+                    *reinterpret_cast<float4*>(Am + where[rep]) = res[rep][0];
+                    *reinterpret_cast<float4*>(Am + where[rep] + LDF) = res[rep][1];
+                }
+        }
+        __syncthreads();
+        clk.lap(5);
+
+        // ---- T_ij = sum_{k=j}^{i-1} B_ik T_kj by distance L = i - j, into block (j, i)
         for (int L = 1; L < 4; ++L) {
-            const int tasks = (4 - L) * 32;
-            const int task = tid;
-            const bool mine = task < tasks;
-            const int i = L + (task >> 5), j = i - L, r0 = 2 * ((task >> 2) & 7), c4 = task & 3;
-            if (mine) {
+            if (tid < (4 - L) * 32) {
+                const int i = L + (tid >> 5), j = i - L;
+                const int r0 = 2 * ((tid >> 2) & 7), c0 = 4 * (tid & 3);
                 float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
                 for (int kb = j; kb < i; ++kb) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float4 a0 = lds4(Am + (16 * i + r0) * LDF + 16 * kb + 4 * k4);
-                        const float4 a1 = lds4(Am + (16 * i + r0 + 1) * LDF + 16 * kb + 4 * k4);
-                        const float x0[4] = {a0.x, a0.y, a0.z, a0.w};
-                        const float x1[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float4 t4 = lds4(Tm + (16 * kb + 4 * k4 + e) * LDF + 16 * j + 4 * c4);
-                            acc0.x = fmaf(x0[e], t4.x, acc0.x);
-                            acc0.y = fmaf(x0[e], t4.y, acc0.y);
-                            acc0.z = fmaf(x0[e], t4.z, acc0.z);
-                            acc0.w = fmaf(x0[e], t4.w, acc0.w);
-                            acc1.x = fmaf(x1[e], t4.x, acc1.x);
-                            acc1.y = fmaf(x1[e], t4.y, acc1.y);
-                            acc1.z = fmaf(x1[e], t4.z, acc1.z);
-                            acc1.w = fmaf(x1[e], t4.w, acc1.w);
-                        }
-                    }
+                    // T_kj: the diagonal block for kb == j, else stored at block (j, kb)
+                    tile_2x4(Am + 16 * i * LDF + 16 * kb, Am + 16 * j * LDF + 16 * kb, r0, c0,
+                             acc0, acc1);
                 }
-                float* w = Am + (16 * (L - 1) + r0) * LDF + 16 * i + 4 * c4;
-                *reinterpret_cast<float4*>(w) = acc0;
-                *reinterpret_cast<float4*>(w + LDF) = acc1;
-            }
-            __syncthreads();
-            if (mine) {
-                float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 t0 = lds4(Tm + (16 * i + r0) * LDF + 16 * i + 4 * k4);
-                    const float4 t1 = lds4(Tm + (16 * i + r0 + 1) * LDF + 16 * i + 4 * k4);
-                    const float x0[4] = {t0.x, t0.y, t0.z, t0.w};
-                    const float x1[4] = {t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float4 w4 =
-                            lds4(Am + (16 * (L - 1) + 4 * k4 + e) * LDF + 16 * i + 4 * c4);
-                        acc0.x = fmaf(x0[e], w4.x, acc0.x);
-                        acc0.y = fmaf(x0[e], w4.y, acc0.y);
-                        acc0.z = fmaf(x0[e], w4.z, acc0.z);
-                        acc0.w = fmaf(x0[e], w4.w, acc0.w);
-                        acc1.x = fmaf(x1[e], w4.x, acc1.x);
-                        acc1.y = fmaf(x1[e], w4.y, acc1.y);
-                        acc1.z = fmaf(x1[e], w4.z, acc1.z);
-                        acc1.w = fmaf(x1[e], w4.w, acc1.w);
-                    }
-                }
-                float* t = Tm + (16 * i + r0) * LDF + 16 * j + 4 * c4;
-                *reinterpret_cast<float4*>(t) = make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w);
-                *reinterpret_cast<float4*>(t + LDF) = make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w);
+                float* t = Am + (16 * j + r0) * LDF + 16 * i + c0;
+                *reinterpret_cast<float4*>(t) = acc0;
+                *reinterpret_cast<float4*>(t + LDF) = acc1;
             }
             __syncthreads();
         }
-        clk.lap(5);
-        // T (bf16, rows k) and [Diag(Gamma_C) T | -Diag(w) T]; thread = (row, half)
+        clk.lap(6);
+
+        // ---- bf16 copies of T: T (B of P) into the Q half of panel 0, and
+        //      [D_G T | -D_w T] (B of R) into the Q half of panel 1 and DT1.  The
+        //      store of Qhat must have read both halves.
+        if (tid == 0) bulk_wait_group_read<0>();
+        __syncthreads();
         {
-            const int r = tid & 63, hf = tid >> 6;
-            const float wr = hf ? -wv[r] : wg[r];
+            const int r = tid & 63, hf = tid >> 6;  // row r of T, columns 32 hf .. 32 hf + 31
+            const int bi = r >> 4;
+            const float g = wg[r], w = -wv[r];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 t0 = lds4(Tm + r * LDF + 8 * c), t1 = lds4(Tm + r * LDF + 8 * c + 4);
-                float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                if (hf == 0) st_bf16x8(sm + TB + sw128_off(r, c), x);
+            for (int q = 0; q < 2; ++q) {
+                const int bj = 2 * hf + q;  // 16-column block of T
+                float x[16];
+                if (bj <= bi) {
+                    const float* src = (bj == bi) ? Am + r * LDF + 16 * bi
+                                                  : Am + (16 * bj + (r & 15)) * LDF + 16 * bi;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= wr;
-                st_bf16x8(sm + DT + hf * 8192 + sw128_off(r, c), x);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 v4 = lds4(src + 4 * q4);
+                        x[4 * q4] = v4.x;
+                        x[4 * q4 + 1] = v4.y;
+                        x[4 * q4 + 2] = v4.z;
+                        x[4 * q4 + 3] = v4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x[e] = 0.f;
+                }
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    const uint32_t off = sw128_off(r, 2 * bj + h8);
+                    float y[8], z[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        y[e] = g * x[8 * h8 + e];
+                        z[e] = w * x[8 * h8 + e];
+                    }
+                    st_bf16x8(kq + TB_OFF + off, x + 8 * h8);
+                    st_bf16x8(kq + DT0_OFF + off, y);
+                    st_bf16x8(sm + DT1 + off, z);
+                }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncthreads();
-        clk.lap(6);
+        clk.lap(7);
         if (tid == 0) {
             tc_fence_after_sync();
-            const uint32_t idp = idesc_bf16(128, 64, false, true);
+            const uint32_t idp = idesc_bf16(128, 64, true, true);
             const uint32_t idr = idesc_bf16(128, 128, true, true);
+            const uint32_t dt_lbo = (sbase + DT1) - (kq_s + DT0_OFF);  // N-panel 0 -> 1
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_P, smem_desc(sbase + IATT + ks * 32, 16, 1024, kSw128),
-                         smem_desc(sbase + TB + ks * 2048, 8192, 1024, kSw128), idp, ks > 0);
+                mma_bf16(tmem + TM_P, smem_desc(sbase + IATT + ks * 2048, 8192, 1024, kSw128),
+                         smem_desc(kq_s + TB_OFF + ks * 2048, 8192, 1024, kSw128), idp, ks > 0);
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_R, smem_desc(sbase + KQ + ks * 2048, 16384, 1024, kSw128),
-                         smem_desc(sbase + DT + ks * 2048, 8192, 1024, kSw128), idr, ks > 0);
-            mma_commit(&bars[1]);
+                mma_bf16(tmem + TM_R, smem_desc(kq_s + ks * 2048, 16384, 1024, kSw128),
+                         smem_desc(kq_s + DT0_OFF + ks * 2048, dt_lbo, 1024, kSw128), idr, ks > 0);
+            mma_commit(&bars[B_MMA]);
         }
-        ok = mbar_wait(&bars[1], 1);
+        ok = mbar_wait(&bars[B_MMA], mma_phase);
+        mma_phase ^= 1;
         tc_fence_after_sync();
         ok = __syncthreads_and(ok);
-        clk.lap(7);
-    }
-    if (ok) {
-        // [T; Att T] row = lane and the two A2T rows (lane, 128 + lane) into the
-        // swizzled staging tiles, then TMA stores
+        if (!ok) break;
+        clk.lap(8);
+
+        // ---- [T; Att T] row = lane into its staging tile over A, then its store
         float v[64];
         tmem_ld32(tmem + lane_sel + TM_P, *reinterpret_cast<float(*)[32]>(v));
         tmem_ld32(tmem + lane_sel + TM_P + 32, *reinterpret_cast<float(*)[32]>(v + 32));
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) st_bf16x8(sm + STG_TAT + sw128_off(tid, c), v + 8 * c);
+        for (int cc = 0; cc < 8; ++cc) st_bf16x8(sm + STG_TAT + sw128_off(tid, cc), v + 8 * cc);
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_3d(&tm_tat, 0, 0, (int)chunk, sm + STG_TAT);
+            bulk_commit_group();
+        }
+        clk.lap(9);
+
+        // ---- A2T rows (lane, 128 + lane) into the current K/Q buffer (K has been read)
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2, *reinterpret_cast<float(*)[32]>(v));
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_bf16x8(sm + STG_A2T + q2 * 16384 + sw128_off(tid, c), v + 8 * c);
+            for (int cc = 0; cc < 8; ++cc) st_bf16x8(kq + q2 * 16384 + sw128_off(tid, cc), v + 8 * cc);
         }
         fence_proxy_async_smem();
+        tc_fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-            tma_store_3d(&tm_tat, 0, 0, (int)chunk, sm + STG_TAT);
-            tma_store_3d(&tm_a2t, 0, 0, (int)chunk, sm + STG_A2T);
-            tma_store_3d(&tm_a2t, 0, 128, (int)chunk, sm + STG_A2T + 16384);
+            tma_store_3d(&tm_a2t, 0, 0, (int)chunk, kq);
+            tma_store_3d(&tm_a2t, 0, 128, (int)chunk, kq + 16384);
             bulk_commit_group();
         }
-        clk.lap(8);
-    }
-    if (!ok && tid == 0) {
-        atomicOr(a.status + 1, 1u);
-        (void)mbar_wait(&bars[0], 0);  // the loads must land before shared memory goes away
+        clk.lap(10);
     }
     clk.flush();
-    if (tid == 0) bulk_wait_group_all();  // the stores have read their shared-memory tiles
+    if (tid == 0) {
+        if (!ok) {
+            atomicOr(a.status + 1, 1u);
+            // a load that was issued must land before shared memory goes away
+            if (pend_buf >= 0) (void)mbar_wait(&bars[B_LD + pend_buf], pend_par);
+        }
+        bulk_wait_group_all();  // the stores have read their shared-memory tiles
+    }
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 #ifdef MDN_PHASE_CLOCKS
-    if (a.dbg && tid == 0 && chunk < 4096) {
+    if (a.dbg && tid == 0 && blockIdx.x < 2048) {
         double* tl = reinterpret_cast<double*>(a.dbg + 64);
-        tl[3 * chunk] = (double)t_begin;
-        tl[3 * chunk + 1] = (double)global_timer_ns();
-        tl[3 * chunk + 2] = (double)smid;
+        tl[3 * blockIdx.x] = (double)t_begin;
+        tl[3 * blockIdx.x + 1] = (double)global_timer_ns();
+        tl[3 * blockIdx.x + 2] = (double)smid;
     }
 #endif
 }
@@ -452,9 +563,6 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
     t.mu_log = a.mu_log;
     t.beta = a.beta;
     t.eta = a.eta;
-    t.qhat = a.qhat;
-    t.tat = a.tat;
-    t.a2t = a.a2t;
     t.crec = a.crec;
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
@@ -462,16 +570,19 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
     t.T = a.T;
     t.H = a.H;
     t.NT = a.NT;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_intra_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    t.BH = a.B * a.H;
+    cudaError_t e = cudaFuncSetAttribute(chunk_intra_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    // persistent: two CTAs per SM, each taking every grid-th chunk
+    const long long grid = chunks < 2LL * sms ? chunks : 2LL * sms;
     ProfScope ps(kIntraTc, s);
-    chunk_intra_kernel<<<(unsigned)chunks, kThreads, SMEM_BYTES, s>>>(mq, mk, mqh, mtat, ma2t, t);
+    chunk_intra_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mqh, mtat, ma2t, t);
     return cudaGetLastError();
 }
 
