@@ -110,6 +110,7 @@ constexpr int kBars = 22;
 
 struct InterArgs {
     const float* crec;
+    const unsigned* ready;  // [chunks] set by the intra-chunk kernel once a chunk is written
     const float* S0;
     const float* M0;
     float* S_T;
@@ -139,6 +140,25 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
         }
     }
 }
+// Wait until the intra-chunk kernel has published a chunk (it may still be
+// running: this kernel is launched as its programmatic dependent).  Gives up
+// like wait_bar.
+__device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* abort_flag) {
+    if (ld_acquire_gpu(flag) != 0u) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(flag) != 0u) return true;
+        if ((i & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitNs || i > (1u << 24)) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
 // Warp-uniform form: every lane waits, and the warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
@@ -281,6 +301,9 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const int s2 = n & 1, sv = n % L::NVC;
                 const long long chunk = (long long)bh * NT + n;
                 if (n >= 2 && !wait_bar(&bars[B_M1 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
+                // the operands of chunk n are in global memory
+                if (!wait_ready(a.ready + chunk, abort_flag)) break;
+                fence_proxy_async_global();
                 clk.lap(0);
                 uint64_t* fb = &bars[B_FKQ + s2];
                 mbar_arrive_expect_tx(fb, kTxKQ);
@@ -476,6 +499,7 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
         return cudaErrorInvalidValue;
     InterArgs t;
     t.crec = a.crec;
+    t.ready = a.ready;
     t.S0 = a.S0;
     t.M0 = a.M0;
     t.S_T = a.S_T;
@@ -493,33 +517,49 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)a.B * a.H * (D / NS);
     ProfScope ps(kInterTc, s);
-    chunk_inter_kernel<NS><<<(unsigned)blocks, L::kThreads, L::SMEM_BYTES, s>>>(mk, mqh, mv, mtat, ma2t, t);
-    return cudaGetLastError();
+    // Programmatic dependent launch: the CTAs may start while the intra-chunk
+    // kernel (launched just before on s) still runs; each chunk is read only
+    // after its ready flag.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(L::kThreads);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk_inter_kernel<NS>, mk, mqh, mv, mtat, ma2t, t);
 }
 
 }  // namespace
 
-// Slice width: 64 columns (two CTAs per head) when that already gives one CTA
-// per SM or more, otherwise 32 (four per head) to spread short batches.
-cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s, int ns)
-{
-    if (ns == 0) {
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        ns = (long long)a.B * a.H * 2 >= sms ? 64 : 32;
-    }
-    return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
-}
-
 // The tensor-core path: the intra-chunk kernel, then the sequential
-// inter-chunk kernel, both on stream s.
+// inter-chunk kernel as its programmatic dependent, both on stream s.
+//
+// Slice width (ns = 0 chooses) and overlap: the inter-chunk kernel's CTAs
+// can only start on SMs that the intra-chunk kernel has left.  When its CTAs
+// fit in the SMs minus a share kept for the intra-chunk kernel, that many SMs
+// are reserved: the intra-chunk CTAs there take a single chunk, and the chain
+// starts one chunk's time after launch while the other SMs produce the rest
+// ahead of it.  Four slices per head when they fit in one wave (their chain
+// is the shortest per chunk), else two; SMs are reserved only when the
+// slices fit beside the intra-chunk kernel's share.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
-    cudaError_t e = launch_chunk_intra_tc(a, s);
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    return launch_chunk_inter_tc(a, s, ns);
+    const long long heads = (long long)a.B * a.H;
+    const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
+    if (ns == 0) ns = heads * 4 <= sms ? 32 : 64;
+    const long long ctas = heads * (D / ns);
+    const int reserve = ctas <= room ? (int)ctas : 0;
+    if ((e = launch_chunk_intra_tc(a, s, reserve)) != cudaSuccess) return e;
+    return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
 }
 
 }  // namespace mdn

@@ -20,14 +20,18 @@
 // plus the per-position coefficients alphabar_r, alpha_r b_{r-1}, b_r and the
 // chunk scalars alphabar_C, b_C, mubar_C (fp32).
 //
-// The CTAs are persistent (two per SM) and take chunks in chunk-major order
-// (chunk 0 of every head first).  K and Q of a CTA's next chunk are loaded by
-// TMA into a second buffer while the current chunk computes, and the gate
-// scan of the next chunk runs on the warps that the column pass leaves idle.
-// Column i of Gamma never leaves the registers of the thread that owns it:
-// that thread writes column i of A and K-row i of the MN-major [I; Att]
-// operand directly.  T is solved in place over A: the diagonal blocks replace
-// A_ii, B_ik replaces A_ik, and T_ij (i > j) goes to the unused block (j, i).
+// The CTAs are persistent (two per SM) and take chunks from a global counter
+// in chunk-major order (chunk 0 of every head first), publishing a ready flag
+// per chunk; the inter-chunk kernel, launched as their programmatic
+// dependent, starts on the SMs whose CTAs leave first (the CTAs on a reserved
+// set of SMs take a single chunk) and follows the flags.  K and Q of a CTA's
+// next chunk are loaded by TMA into a second buffer while the current chunk
+// computes, and the gate scan of the next chunk runs on a warp that the
+// column pass leaves idle.  Column i of Gamma never leaves the registers of
+// the thread that owns it: that thread writes column i of A and K-row i of
+// the MN-major [I; Att] operand directly.  T is solved in place over A: the
+// diagonal blocks replace A_ii, B_ik replaces A_ik, and T_ij (i > j) goes to
+// the unused block (j, i).
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -38,6 +42,7 @@ using namespace sm100;
 using namespace tc;
 
 constexpr int kThreads = 128;
+constexpr int kTmaTid = 64;  // issues every TMA load and store (its warp idles in the column pass)
 // Shared memory (byte offsets from a 1024-byte aligned base).
 constexpr uint32_t KQ0 = 0;                   // [K; Q] of a chunk, 2 buffers; a buffer holds 2
                                               // feature panels of (64 rows of K, 64 rows of Q) x 128 B
@@ -48,8 +53,8 @@ constexpr uint32_t DT1 = IATT + 16384;        // N-panel 1 of [D_G T | -D_w T] (
 constexpr uint32_t REC = DT1 + 8192;          // gate record, 2 buffers x 6 x 64 floats
 constexpr uint32_t VEC = REC + 2 * 1536;      // mu_r, w_r, Gamma_{C,r}
 constexpr uint32_t BARS = VEC + 768;
-constexpr uint32_t MISC = BARS + 32;
-constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
+constexpr uint32_t MISC = BARS + 32;          // TMEM address; chunk indices of the next two iterations
+constexpr uint32_t SMEM_BYTES = MISC + 32 + 1024;  // + alignment slack
 static_assert(AM % 1024 == 0 && IATT % 1024 == 0 && DT1 % 1024 == 0, "operand alignment");
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 // Aliases, each written only once its previous contents are dead.
@@ -68,10 +73,14 @@ struct IntraArgs {
     const float* beta;
     const float* eta;
     float* crec;             // [chunks][256]
+    unsigned* ready;         // [chunks] set to 1 once a chunk's operands are in global memory
+    unsigned* queue;         // next chunk (in chunk-major order) to hand out; zero on entry
     unsigned* status;
     float* dbg;              // diagnostics: phase clocks of CTA 0 (null in normal use)
     float dcorr;
     int T, H, NT, BH;
+    int reserve;             // CTAs on SMs 0 .. reserve-1 take one chunk only, freeing
+                             // those SMs early for the inter-chunk kernel
 };
 
 // Chunk-major order: the c-th chunk is chunk n of head bh; returns its index
@@ -80,6 +89,14 @@ __device__ __forceinline__ long long chunk_of(long long c, const IntraArgs& a, i
     n = (int)(c / a.BH);
     bh = (int)(c % a.BH);
     return (long long)bh * a.NT + n;
+}
+
+// Marks a chunk's operands as written: its bulk stores have completed (the
+// caller waited for them) and the chunk record was stored before a CTA barrier.
+__device__ __forceinline__ void publish_chunk(unsigned* ready, long long chunk) {
+    fence_proxy_async_global();
+    __threadfence();
+    st_release_gpu(ready + chunk, 1u);
 }
 
 // Gate record of one chunk (one warp): la, lm, b, alpha, beta, eta per
@@ -151,6 +168,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* mu = reinterpret_cast<float*>(sm + VEC);
     float* wv = mu + C;    // w_r = eta_r mubar_C / mubar_r
     float* wg = wv + C;    // Gamma_{C,r}
+    // The inter-chunk kernel may be scheduled as soon as every CTA of this grid
+    // has started; it waits for each chunk's ready flag before reading it.
+    pdl_launch_dependents();
     PhaseClock clk;
     clk.start((a.dbg && blockIdx.x == 0 && tid == 0) ? a.dbg : nullptr);
 #ifdef MDN_PHASE_CLOCKS
@@ -179,17 +199,27 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         pend_par = (iter >> 1) & 1;
     };
 
-    if (tid == 0) {
+    // chunk indices of the next two iterations (slot = iteration & 1)
+    long long* cslot = reinterpret_cast<long long*>(sm + MISC + 16);
+    int fetched = 0, limit = 1 << 30;  // TMA thread: chunks taken from the counter
+    auto fetch = [&]() -> long long {
+        if (fetched >= limit) return chunks;
+        ++fetched;
+        const unsigned c = atomicAdd(a.queue, 1u);
+        return c < chunks ? (long long)c : chunks;
+    };
+    if (tid == kTmaTid) {
+        uint32_t smid_;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));
+        if ((int)smid_ < a.reserve) limit = 1;
         mbar_init(&bars[B_LD], 1);
         mbar_init(&bars[B_LD + 1], 1);
         mbar_init(&bars[B_MMA], 1);
         mbar_fence_init();
-        if (blockIdx.x < chunks) load_kq(blockIdx.x, 0);
-    }
-    if (warp == 3 && blockIdx.x < chunks) {
-        int n, bh;
-        (void)chunk_of(blockIdx.x, a, n, bh);
-        gate_record(a, n, bh, reinterpret_cast<float*>(sm + REC), lane);
+        const long long c0 = fetch();
+        cslot[0] = c0;
+        cslot[1] = c0 < chunks ? fetch() : chunks;
+        if (c0 < chunks) load_kq(c0, 0);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -209,24 +239,30 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
+    if (warp == 3 && cslot[0] < chunks) {  // ordered before use by the loop's first barrier
+        int n, bh;
+        (void)chunk_of(cslot[0], a, n, bh);
+        gate_record(a, n, bh, reinterpret_cast<float*>(sm + REC), lane);
+    }
 
     bool ok = true;
     uint32_t mma_phase = 0;
     int k = 0;
-    for (long long c = blockIdx.x; c < chunks; c += gridDim.x, ++k) {
+    long long prev_chunk = -1;  // thread 0: the chunk whose stores were issued last
+    for (long long c = cslot[0]; c < chunks; ++k) {
         const int buf = k & 1;
         uint8_t* kq = sm + KQ0 + buf * KQ_BYTES;
         const uint32_t kq_s = sbase + KQ0 + buf * KQ_BYTES;
         const float* rec = reinterpret_cast<const float*>(sm + REC + buf * 1536);
         int n, bh;
         const long long chunk = chunk_of(c, a, n, bh);
-        const long long c_next = c + gridDim.x;
+        const long long c_next = cslot[buf ^ 1];  // written an iteration ago (or before the loop)
         // A is about to be overwritten: the store of [T; Att T] from its staging
         // tile (all store groups but the newest) must have read it
-        if (tid == 0) bulk_wait_group_read<1>();
+        if (tid == kTmaTid) bulk_wait_group_read<1>();
         ok = __syncthreads_and(mbar_wait(&bars[B_LD + buf], (k >> 1) & 1));
         if (!ok) break;
-        if (tid == 0 && pend_buf == buf) pend_buf = -1;
+        if (tid == kTmaTid && pend_buf == buf) pend_buf = -1;
         clk.lap(0);
 
         // ---- Qhat = Q - d K in place (the Q rows of both panels); chunk record
@@ -263,10 +299,12 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         fence_proxy_async_smem();
         __syncthreads();
         clk.lap(1);
-        if (tid == 0) {
+        if (tid == kTmaTid) {
             tma_store_3d(&tm_qh, 0, 0, (int)chunk, kq + 8192);
             tma_store_3d(&tm_qh, 64, 0, (int)chunk, kq + 16384 + 8192);
             bulk_commit_group();
+        }
+        if (tid == 0) {
             tc_fence_after_sync();
             const uint32_t id = idesc_bf16(128, 128, false, false);
 #pragma unroll
@@ -286,12 +324,6 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
         // ---- column pass: thread i < 64 owns column i of Gamma, A and Att
         if (tid < C) {
-            if (tid == 0 && c_next < chunks) {
-                // K, Q of the next chunk into the other buffer, once the stores of the
-                // previous chunk's A2T (all groups but the newest, Qhat) have read it
-                bulk_wait_group_read<1>();
-                load_kq(c_next, k + 1);
-            }
             const int i = tid;
             const float* al = rec + 3 * C;
             const float* be = rec + 4 * C;
@@ -325,6 +357,15 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 st_bf16x8(sm + IATT + 8192 + sw128_off(i, r16 / 8 + 1), att + 8);
             }
             wg[i] = gam;  // Gamma_{C,i}
+        } else if (tid == kTmaTid) {
+            // every store group but the newest (Qhat) has completed: the previous
+            // chunk is in global memory, and its A2T staging buffer is free for
+            // K, Q of the next chunk
+            bulk_wait_group<1>();
+            if (prev_chunk >= 0) publish_chunk(a.ready, prev_chunk);
+            if (c_next < chunks) load_kq(c_next, k + 1);
+            // the chunk after next; every thread has read this slot's old value
+            cslot[buf] = c_next < chunks ? fetch() : chunks;
         } else if (warp == 3 && c_next < chunks) {
             int n2, bh2;
             (void)chunk_of(c_next, a, n2, bh2);
@@ -421,7 +462,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // ---- bf16 copies of T: T (B of P) into the Q half of panel 0, and
         //      [D_G T | -D_w T] (B of R) into the Q half of panel 1 and DT1.  The
         //      store of Qhat must have read both halves.
-        if (tid == 0) bulk_wait_group_read<0>();
+        if (tid == kTmaTid) bulk_wait_group_read<0>();
         __syncthreads();
         {
             const int r = tid & 63, hf = tid >> 6;  // row r of T, columns 32 hf .. 32 hf + 31
@@ -496,7 +537,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int cc = 0; cc < 8; ++cc) st_bf16x8(sm + STG_TAT + sw128_off(tid, cc), v + 8 * cc);
         fence_proxy_async_smem();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == kTmaTid) {
             tma_store_3d(&tm_tat, 0, 0, (int)chunk, sm + STG_TAT);
             bulk_commit_group();
         }
@@ -514,21 +555,24 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == kTmaTid) {
             tma_store_3d(&tm_a2t, 0, 0, (int)chunk, kq);
             tma_store_3d(&tm_a2t, 0, 128, (int)chunk, kq + 16384);
             bulk_commit_group();
+            prev_chunk = chunk;
         }
         clk.lap(10);
+        c = c_next;
     }
     clk.flush();
-    if (tid == 0) {
+    if (tid == kTmaTid) {
         if (!ok) {
             atomicOr(a.status + 1, 1u);
             // a load that was issued must land before shared memory goes away
             if (pend_buf >= 0) (void)mbar_wait(&bars[B_LD + pend_buf], pend_par);
         }
-        bulk_wait_group_all();  // the stores have read their shared-memory tiles
+        bulk_wait_group_all();  // the stores have completed
+        if (ok && prev_chunk >= 0) publish_chunk(a.ready, prev_chunk);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -548,7 +592,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 }  // namespace
 
-cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve)
 {
     const long long chunks = (long long)a.B * a.H * a.NT;
     CUtensorMap mq, mk, mqh, mtat, ma2t;
@@ -564,6 +608,9 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
     t.beta = a.beta;
     t.eta = a.eta;
     t.crec = a.crec;
+    t.ready = a.ready;
+    t.queue = a.ready + chunks;
+    t.reserve = reserve;
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
     t.dcorr = a.dcorr;
@@ -579,7 +626,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s)
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    // persistent: two CTAs per SM, each taking every grid-th chunk
+    // persistent: two CTAs per SM
     const long long grid = chunks < 2LL * sms ? chunks : 2LL * sms;
     ProfScope ps(kIntraTc, s);
     chunk_intra_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mqh, mtat, ma2t, t);

@@ -22,7 +22,7 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, qhat, tat, a2t, crec, total;
+    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, qhat, tat, a2t, crec, ready, total;
 };
 
 // Byte offsets of every scratch region for these sizes.
@@ -45,6 +45,7 @@ WsLayout ws_layout(long long BH, int NT, int D)
     w.tat = off;    off += align_up(rows * 2 * kChunk * 2);
     w.a2t = off;    off += align_up(rows * 2 * D * 2);
     w.crec = off;   off += align_up(rows * 4 * sizeof(float));
+    w.ready = off;  off += align_up(((size_t)BH * NT + 1) * sizeof(unsigned));
     w.total = off;
     return w;
 }
@@ -200,6 +201,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
     a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);
     a.crec = reinterpret_cast<float*>(ws + w.crec);
+    a.ready = reinterpret_cast<unsigned*>(ws + w.ready);
 
     cudaError_t e;
     const bool check = flags & MDN_CHECK_FINITE;
@@ -207,6 +209,8 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
     if (tensor_cores) {
         const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
+        if ((e = cudaMemsetAsync(a.ready, 0, ((size_t)B * H * NT + 1) * sizeof(unsigned), s)))
+            return mdn::cuda_fail(e);
         if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
     } else {
         if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,

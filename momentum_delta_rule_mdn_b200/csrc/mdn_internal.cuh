@@ -100,6 +100,8 @@ struct ChunkArgs {
     __nv_bfloat16* qhat;  // [B*H*NT, C, D]      qhat = q - d k
     __nv_bfloat16* tat;   // [B*H*NT, 2C, C]     [T; Att T]
     __nv_bfloat16* a2t;   // [B*H*NT, 2D, C]     [K^T Diag(Gamma_C) T; -K^T Diag(w) T]
+    unsigned* ready;      // [B*H*NT + 1] chunk operands written (tensor-core path), then the
+                          // intra-chunk kernel's work counter; zeroed per call
     float* crec;          // [B*H*NT, 256]       alphabar_r, alpha_r b_{r-1}, b_r, then
                           //                     alphabar_C, b_C, mubar_C
     float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
@@ -131,9 +133,9 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and
 // returns MDN_ERR_CUDA.
 mdn_status cuda_fail(cudaError_t e);
-cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);  // ns: see launch_chunk_inter_tc
-cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s);
-cudaError_t launch_chunk_inter_tc(const ChunkArgs& a, cudaStream_t s, int ns);  // ns = 0: choose
+// ns: columns of d_v per inter-chunk CTA (32 or 64), 0 = choose by batch size
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve);
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
                         const float* eta, float dcorr, float* S, float* M, int B, int H,
