@@ -151,7 +151,7 @@ def run_ours(args, rank, world, device):
     import momentum_delta_rule_mdn_b200 as mdn
 
     spec0 = workload_spec(args.workload)
-    spec = mi.replace(spec0, seed=spec0.seed + 7919 * rank)
+    spec = rank_spec(spec0, rank)
     inp = mi.make_inputs(spec)
     tok = decode_token(spec, spec.seed + 1)
     dev = mi.to_torch(inp, device)
@@ -209,8 +209,7 @@ def run_ours(args, rank, world, device):
     ms = float(np.mean(step_ms))
     ms_max = max_over_ranks(ms, world, device)
 
-    tokens_per_rank = B * T
-    value = tokens_per_rank * world / (ms_max * 1e-3)
+    value = whole_job_value(B * T, world, ms_max)
 
     # ---- dominant kernel and its roofline
     hbm, bf16, peak_src = load_peaks()
@@ -435,6 +434,18 @@ def workload_spec(w):
         if s.name == w:
             return s
     raise SystemExit(f"unknown workload {w!r}")
+
+
+def rank_spec(spec0: mi.Spec, rank: int) -> mi.Spec:
+    """The workload of one rank: same shape, its own seed (ranks are replicas
+    over independent batches; no two ranks draw the same inputs)."""
+    return mi.replace(spec0, seed=spec0.seed + 7919 * rank)
+
+
+def whole_job_value(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Weak-scaling throughput: the tokens every rank processed over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
 
 
 def barrier(world):
