@@ -9,16 +9,26 @@
 //   o_j   = sum_i S_ij (q_i - d k_i)
 //
 // Bound by HBM: each state element is read once and written once.  Columns
-// are independent, so one block owns one (b, h) and 64 columns; a thread owns
-// RP rows x 4 adjacent columns (float4), so each row access of a warp-half is
-// 256 contiguous bytes.  The two column sums are block reductions in shared
-// memory.  All state loads are issued before the first reduction.
+// are independent, so one block owns one (b, h) and NC columns (64 for large
+// batches; 32 or 16 when fewer blocks would leave SMs idle); a thread owns RP
+// rows x 4 adjacent columns (float4).  The two column sums over rows reduce
+// within a warp by shuffles, then across the 8 warps in shared memory.  All
+// state loads are issued before the first reduction.
 #include "mdn_internal.cuh"
 
 namespace mdn {
 namespace {
 
-template <typename Tin, int D>
+// Sum of x over the lanes of this warp that share lane % CG (the row groups of
+// one column group); the result is valid in every lane.
+template <int CG>
+__device__ __forceinline__ float rows_sum(float x) {
+#pragma unroll
+    for (int off = CG; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+template <typename Tin, int D, int NC>
 __global__ void __launch_bounds__(256)
 step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
             const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
@@ -26,18 +36,18 @@ step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __r
             float* __restrict__ S, float* __restrict__ M, Tin* __restrict__ o,
             Tin* __restrict__ vt_out)
 {
-    constexpr int NC = 64;          // columns per block
     constexpr int CG = NC / 4;      // float4 column groups
     constexpr int RG = 256 / CG;    // row groups
     constexpr int RP = D / RG;      // rows per thread
-    constexpr int HALVES = D / NC;
+    constexpr int PARTS = D / NC;   // blocks per head
+    static_assert(RP >= 1 && CG <= 32, "shape");
     __shared__ float ks[D], qs[D];
-    __shared__ float red[RG][NC + 4];
+    __shared__ float red[8][NC];
     __shared__ float vts[NC];
 
-    const int tid = threadIdx.x;
-    const long long bh = blockIdx.x / HALVES;
-    const int col_base = (blockIdx.x % HALVES) * NC;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long bh = blockIdx.x / PARTS;
+    const int col_base = (blockIdx.x % PARTS) * NC;
     const int cg = tid % CG, rg = tid / CG;
     const int col = col_base + cg * 4;
 
@@ -72,13 +82,17 @@ step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __r
         p[3] = fmaf(s4[e].w, kv, p[3]);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) red[rg][cg * 4 + c] = p[c];
+    for (int c = 0; c < 4; ++c) p[c] = rows_sum<CG>(p[c]);
+    if (lane < CG) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[warp][cg * 4 + c] = p[c];
+    }
     __syncthreads();
     if (tid < NC) {
-        float s = 0.f;
+        float sum = 0.f;
 #pragma unroll
-        for (int g = 0; g < RG; ++g) s += red[g][tid];
-        const float vtj = ld_elem(v + (size_t)bh * D + col_base + tid) - alpha * s;
+        for (int g = 0; g < 8; ++g) sum += red[g][tid];
+        const float vtj = ld_elem(v + (size_t)bh * D + col_base + tid) - alpha * sum;
         vts[tid] = vtj;
         if (vt_out) st_elem(vt_out + (size_t)bh * D + col_base + tid, vtj);
     }
@@ -107,13 +121,17 @@ step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __r
         __stcs(reinterpret_cast<float4*>(Mh + (size_t)i * D + col), m4[e]);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) red[rg][cg * 4 + c] = po[c];
+    for (int c = 0; c < 4; ++c) po[c] = rows_sum<CG>(po[c]);
+    if (lane < CG) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) red[warp][cg * 4 + c] = po[c];
+    }
     __syncthreads();
     if (tid < NC) {
-        float s = 0.f;
+        float sum = 0.f;
 #pragma unroll
-        for (int g = 0; g < RG; ++g) s += red[g][tid];
-        st_elem(o + (size_t)bh * D + col_base + tid, s);
+        for (int g = 0; g < 8; ++g) sum += red[g][tid];
+        st_elem(o + (size_t)bh * D + col_base + tid, sum);
     }
 }
 
@@ -123,12 +141,29 @@ cudaError_t launch_step_typed(const void* q, const void* k, const void* v,
                               const float* eta, float dcorr, float* S, float* M, int B, int H,
                               void* o, void* vt, cudaStream_t s)
 {
-    const long long blocks = (long long)B * H * (D / 64);
-    if (blocks == 0) return cudaSuccess;
+    const long long heads = (long long)B * H;
+    if (heads == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // narrowest column split that still reaches two blocks per SM
+    const int nc = heads * (D / 64) >= 2LL * sms ? 64 : (heads * (D / 32) >= 2LL * sms ? 32 : 16);
     ProfScope ps(kStep, s);
-    step_kernel<Tin, D><<<(unsigned)blocks, 256, 0, s>>>(
-        static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
-        alpha_log, mu_log, beta, eta, dcorr, S, M, static_cast<Tin*>(o), static_cast<Tin*>(vt));
+    const Tin* qq = static_cast<const Tin*>(q);
+    const Tin* kk = static_cast<const Tin*>(k);
+    const Tin* vv = static_cast<const Tin*>(v);
+    Tin* oo = static_cast<Tin*>(o);
+    Tin* tt = static_cast<Tin*>(vt);
+    if (nc == 64)
+        step_kernel<Tin, D, 64><<<(unsigned)(heads * (D / 64)), 256, 0, s>>>(
+            qq, kk, vv, alpha_log, mu_log, beta, eta, dcorr, S, M, oo, tt);
+    else if (nc == 32)
+        step_kernel<Tin, D, 32><<<(unsigned)(heads * (D / 32)), 256, 0, s>>>(
+            qq, kk, vv, alpha_log, mu_log, beta, eta, dcorr, S, M, oo, tt);
+    else
+        step_kernel<Tin, D, 16><<<(unsigned)(heads * (D / 16)), 256, 0, s>>>(
+            qq, kk, vv, alpha_log, mu_log, beta, eta, dcorr, S, M, oo, tt);
     return cudaGetLastError();
 }
 

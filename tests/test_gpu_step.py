@@ -16,9 +16,14 @@ def _seq_to_steps(t):
     return t.transpose(0, 1).contiguous()
 
 
-@pytest.mark.parametrize("dtype,d", [("f32", 64), ("f32", 128), ("bf16", 64), ("bf16", 128)])
-def test_step_small(dtype, d):
-    spec = mi.Spec("step_small", B=2, T=24, H=3, d=d, dtype=dtype, state_std=0.05, seed=77)
+@pytest.mark.parametrize("dtype,d,B,H", [
+    ("f32", 64, 2, 3), ("f32", 128, 2, 3), ("bf16", 64, 2, 3), ("bf16", 128, 2, 3),
+    # head counts at which the kernel splits d_v into 32 and 64 columns per block
+    ("bf16", 128, 10, 8), ("bf16", 128, 40, 8), ("f32", 64, 10, 16), ("f32", 64, 40, 8),
+])
+def test_step_small(dtype, d, B, H):
+    spec = mi.Spec("step_small", B=B, T=24 if B * H < 50 else 4, H=H, d=d, dtype=dtype,
+                   state_std=0.05, seed=77)
     inp = mi.make_inputs(spec)
     dev = mi.to_torch(inp, "cuda")
     S, M = dev["S0"].clone(), dev["M0"].clone()
