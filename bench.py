@@ -83,7 +83,7 @@ def kernel_work(name: str, spec: mi.Spec):
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
         self.samples = []
         self.reasons = set()

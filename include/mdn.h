@@ -124,6 +124,12 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  * unaligned pointer, too-small workspace), MDN_ERR_UNSUPPORTED (d, C or dtype
  * outside support), MDN_ERR_CUDA (launch failure), and with MDN_CHECK_FINITE
  * also MDN_ERR_NONFINITE / MDN_ERR_TIMEOUT.
+ *
+ * Asynchronous on `stream` (except with MDN_CHECK_FINITE).  The bf16 d = 128
+ * path enqueues a small memset of the workspace and two kernels, the second
+ * launched as the first one's programmatic dependent; the sequence can be
+ * captured in a CUDA graph and replayed.  Calls that may run concurrently
+ * need separate workspaces.
  */
 mdn_status mdn_chunk_fwd(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
                          const float *alpha_log, const float *mu_log,
