@@ -73,9 +73,15 @@ typedef enum {
 #define MDN_SLICE32      0x4  /* tensor-core path: the inter-chunk kernel gives each CTA
                                  32 columns of d_v (four CTAs per head) */
 #define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head).  Neither flag:
-                                 64 when B*H*2 reaches the SM count, else 32.  Both
-                                 widths compute the same result; the flags exist
-                                 for tuning and testing. */
+                                 32 when B*H*4 CTAs fit on the SMs at once, else 64.
+                                 Both widths compute the same result; the flags
+                                 exist for tuning and testing. */
+#define MDN_TEST_NO_INTRA 0x100 /* testing the failure path only: the tensor-core
+                                 path does not launch its intra-chunk kernel, so the
+                                 inter-chunk kernel's wait for each chunk's operands
+                                 runs out (after about 1 s), its CTAs stop cleanly,
+                                 and with MDN_CHECK_FINITE the call returns
+                                 MDN_ERR_TIMEOUT.  The outputs are not written. */
 
 /* Version of this ABI (incremented on any incompatible change). */
 int mdn_abi_version(void);
@@ -115,7 +121,7 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   workspace   device scratch of at least mdn_chunk_fwd_workspace_size(...)
  *               bytes, 256-byte aligned; its contents on entry do not matter.
  *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT, plus at most one of
- *               MDN_SLICE32 / MDN_SLICE64.
+ *               MDN_SLICE32 / MDN_SLICE64 (and MDN_TEST_NO_INTRA in tests).
  *
  * Support: d in {64, 128}, C = 64, any T >= 0 (a short last chunk is handled
  * as if padded with steps that leave S and M unchanged), B, H >= 0 with

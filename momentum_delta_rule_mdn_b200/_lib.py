@@ -14,6 +14,7 @@ MDN_CHECK_FINITE = 0x1
 MDN_FORCE_SIMT = 0x2
 MDN_SLICE32 = 0x4
 MDN_SLICE64 = 0x8
+MDN_TEST_NO_INTRA = 0x100
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 

@@ -227,6 +227,9 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);  // this warp's lane base
+#ifdef MDN_PHASE_CLOCKS
+    const uint64_t t_start = global_timer_ns();
+#endif
 
     if (warp == 0) {
         // ------------------------------------------------------------ MMA issue
@@ -483,6 +486,13 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tc_fence_after_sync();
         tmem_dealloc(tmem, L::kTmemCols);
     }
+#ifdef MDN_PHASE_CLOCKS
+    if (a.dbg && tid == 0 && blockIdx.x < 1024) {
+        double* tl = reinterpret_cast<double*>(a.dbg + 30000);
+        tl[2 * blockIdx.x] = (double)t_start;
+        tl[2 * blockIdx.x + 1] = (double)global_timer_ns();
+    }
+#endif
 }
 
 template <int NS>
@@ -558,7 +568,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     if (ns == 0) ns = heads * 4 <= sms ? 32 : 64;
     const long long ctas = heads * (D / ns);
     const int reserve = ctas <= room ? (int)ctas : 0;
-    if ((e = launch_chunk_intra_tc(a, s, reserve)) != cudaSuccess) return e;
+    if (!a.test_no_intra && (e = launch_chunk_intra_tc(a, s, reserve)) != cudaSuccess) return e;
     return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
 }
 

@@ -150,7 +150,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 {
     mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
     if (st != MDN_OK) return st;
-    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64))
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64 | MDN_TEST_NO_INTRA))
         return MDN_ERR_INVALID_ARG;
     if ((flags & MDN_SLICE32) && (flags & MDN_SLICE64)) return MDN_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return MDN_OK;
@@ -211,6 +211,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
         const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
         if ((e = cudaMemsetAsync(a.ready, 0, ((size_t)B * H * NT + 1) * sizeof(unsigned), s)))
             return mdn::cuda_fail(e);
+        a.test_no_intra = (flags & MDN_TEST_NO_INTRA) != 0;
         if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
     } else {
         if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,

@@ -104,6 +104,7 @@ struct ChunkArgs {
                           // intra-chunk kernel's work counter; zeroed per call
     float* crec;          // [B*H*NT, 256]       alphabar_r, alpha_r b_{r-1}, b_r, then
                           //                     alphabar_C, b_C, mubar_C
+    bool test_no_intra = false;  // failure-path test: skip the intra-chunk kernel
     float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
 };
 

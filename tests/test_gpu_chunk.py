@@ -201,3 +201,16 @@ def test_chunk_fwd_cuda_graph_replay():
         g.replay()
         torch.cuda.synchronize()
         compare_heads(out, inps[r], all_heads(inps[r].spec), TOL["bf16"])
+
+
+def test_timeout_path_reports_and_recovers():
+    """Failure injected on the host: the intra-chunk kernel is not launched, so
+    the inter-chunk kernel's bounded wait for the first chunk's operands runs
+    out; its CTAs stop cleanly and the call reports MDN_ERR_TIMEOUT.  The
+    context stays usable: the next normal call is correct."""
+    inp = mi.make_inputs(mi.Spec("timeout", B=1, T=130, H=2, d=128, dtype="bf16",
+                                 state_std=0.01, seed=4200))
+    with pytest.raises(mdn.MDNError) as err:
+        run(inp, flags=_lib.MDN_TEST_NO_INTRA | _lib.MDN_CHECK_FINITE)
+    assert err.value.status == _lib.MDN_ERR_TIMEOUT
+    compare_heads(run(inp), inp, all_heads(inp.spec), TOL["bf16"])
