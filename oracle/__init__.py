@@ -63,6 +63,9 @@ def _bind(path: str) -> ctypes.CDLL:
     lib.mdn_oracle_step.restype = i
     lib.mdn_oracle_chunk_coeffs.argtypes = [_D, _D, _D, _D, i, i, i, i, _D, _D, _D, _D]
     lib.mdn_oracle_chunk_coeffs.restype = i
+    lib.mdn_oracle_gates.argtypes = [_D, _D, _D, _D, ctypes.c_ssize_t, ctypes.c_double,
+                                     ctypes.c_double, i, _D, _D, _D, _D]
+    lib.mdn_oracle_gates.restype = i
     lib.mdn_oracle_max_threads.argtypes = []
     lib.mdn_oracle_max_threads.restype = i
     return lib
@@ -150,3 +153,26 @@ def chunk_coeffs(alpha_log, mu_log, beta, eta, C: int, with_gamma: bool = True,
     if rc != 0:
         raise RuntimeError(f"mdn_oracle_chunk_coeffs failed ({rc})")
     return la, lm, lc, gamma
+
+
+def gates(x_eta, a, b, c, s: float = 1.0, mu_log_min: float = -1.0, eta_act: str = "tanh",
+          lib: Optional[ctypes.CDLL] = None):
+    """Gates from pre-activations (any equal shapes).  Returns fp64
+    (alpha_log, mu_log, beta, eta)."""
+    lib = lib or load()
+    x, aa, bb, cc = (_f64(t) for t in (x_eta, a, b, c))
+    assert x.shape == aa.shape == bb.shape == cc.shape
+    out = [np.empty(x.shape) for _ in range(4)]
+    act = {"tanh": 0, "2sigmoid": 1}[eta_act]
+    rc = lib.mdn_oracle_gates(_ptr(x), _ptr(aa), _ptr(bb), _ptr(cc), x.size, float(s),
+                              float(mu_log_min), act, *(_ptr(o) for o in out))
+    if rc != 0:
+        raise RuntimeError(f"mdn_oracle_gates failed ({rc})")
+    return tuple(out)
+
+
+def step_delta_norm(S_old, S_new) -> np.ndarray:
+    """Frobenius norm of the fast-weight change of one decode step, per head:
+    ||S_t - S_{t-1}||_F (ijyty.com article, section 8)."""
+    dS = np.asarray(S_new, dtype=np.float64) - np.asarray(S_old, dtype=np.float64)
+    return np.sqrt((dS * dS).sum(axis=(-2, -1)))

@@ -32,6 +32,13 @@
  *   gates              : [B, T, H]        (decode step: [B, H])
  *   S0, M0, S_T, M_T   : [B, H, d_k, d_v], row index over d_k
  *
+ * mdn_oracle_gates maps raw per-token pre-activations to the four gates by the
+ * stable parameterisation (summary, step 6; article, sections 5 and 8):
+ *     eta   = tanh(x) + 1            (or 2 sigmoid(x), the ablated variant)
+ *     theta = arctan(eta * s)
+ *     alpha = cos^2(theta) sigmoid(a),  beta = sin^2(theta) sigmoid(b)
+ *     log mu = max(log sigmoid(c), mu_log_min)
+ *
  * Parity pins: every function here is checked against results the pages or
  * the mathematics fix (closed form, special cases, spectrum, hand-worked
  * values) by the CPU tests; none is unpinned.
@@ -239,6 +246,34 @@ int mdn_oracle_chunk_coeffs(const double *alpha_log, const double *mu_log,
                     G[(ptrdiff_t)r * C + i] = acc;
                 }
         }
+    }
+    return 0;
+}
+
+/* log(sigmoid(x)) without overflow for either sign of x. */
+static double log_sigmoid(double x)
+{
+    return x >= 0.0 ? -log1p(exp(-x)) : x - log1p(exp(x));
+}
+
+/* The four gates of n tokens from their pre-activations (see the header).
+ * eta_act: 0 = tanh(x) + 1, 1 = 2 sigmoid(x).  Outputs: alpha_log = log alpha,
+ * mu_log, beta, eta, each [n]. */
+int mdn_oracle_gates(const double *x_eta, const double *a, const double *b,
+                     const double *c, ptrdiff_t n, double s, double mu_log_min,
+                     int eta_act, double *alpha_log, double *mu_log, double *beta,
+                     double *eta)
+{
+    if (n < 0 || (eta_act != 0 && eta_act != 1)) return -1;
+    for (ptrdiff_t i = 0; i < n; ++i) {
+        const double e = eta_act == 0 ? tanh(x_eta[i]) + 1.0 : 2.0 / (1.0 + exp(-x_eta[i]));
+        const double theta = atan(e * s);
+        const double ct = cos(theta), st = sin(theta);
+        eta[i] = e;
+        alpha_log[i] = log(ct * ct) + log_sigmoid(a[i]);
+        beta[i] = st * st * exp(log_sigmoid(b[i]));
+        const double lm = log_sigmoid(c[i]);
+        mu_log[i] = lm > mu_log_min ? lm : mu_log_min;
     }
     return 0;
 }

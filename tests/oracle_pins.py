@@ -12,6 +12,8 @@ Sources ("MDN: Parallelizing Stepwise Momentum for Delta Linear Attention"):
   chunkwise form ........ summary, step 4
   spectrum lambda+- ..... summary, step 6; novelty paragraph; ijyty.com, section 5
   mu = 0 ablation ....... ijyty.com, section 8 (reduces to a gated delta rule)
+  gate parameterisation . summary, step 6; ijyty.com, sections 5 and 8
+  ||Delta S_t||_F ........ ijyty.com, section 8 (decoding diagnostic)
 """
 from __future__ import annotations
 
@@ -286,6 +288,71 @@ def pin_resume(lib):
     _close(b[2], ref[2], 1e-13, "resume S_T")
 
 
+# ---------------------------------------------------------------- gates
+def _logsig(x):
+    return -np.logaddexp(0.0, -np.asarray(x, dtype=np.float64))
+
+
+def pin_gates_special_points(lib):
+    """theta = arctan(eta s): s = 0 gives theta = 0 (alpha = sigmoid(a), beta = 0);
+    x = 0 gives eta = 1 for both activations, so s = 1 gives theta = pi/4
+    (cos^2 = sin^2 = 1/2).  mu_log is log sigmoid(c) above the clamp, the clamp
+    below it."""
+    a = np.array([-3.0, 0.0, 2.5]); b = np.array([1.0, -0.5, 0.0]); c = np.array([0.0, -5.0, 4.0])
+    x0 = np.zeros(3)
+    for act in ("tanh", "2sigmoid"):
+        al, ml, be, et = oracle.gates(np.array([0.3, -1.2, 2.0]), a, b, c, s=0.0,
+                                      mu_log_min=-1.0, eta_act=act, lib=lib)
+        _close(al, _logsig(a), 1e-15, f"{act} s=0 alpha_log")
+        _close(be, np.zeros(3), 1e-15, f"{act} s=0 beta")
+        al, ml, be, et = oracle.gates(x0, a, b, c, s=1.0, mu_log_min=-1.0, eta_act=act, lib=lib)
+        _close(et, np.ones(3), 1e-15, f"{act} eta(0)")
+        _close(al, np.log(0.5) + _logsig(a), 1e-14, f"{act} theta=pi/4 alpha_log")
+        _close(be, 0.5 / (1.0 + np.exp(-b)), 1e-14, f"{act} theta=pi/4 beta")
+        # log sigmoid(0) = -log 2 > -1; log sigmoid(-5) < -1 clamps; log sigmoid(4) ~ -0.018
+        _close(ml, [-np.log(2.0), -1.0, -np.log1p(np.exp(-4.0))], 1e-15, f"{act} mu_log")
+
+
+def pin_gates_identities(lib):
+    """On random pre-activations: alpha/sigmoid(a) + beta/sigmoid(b) = 1
+    (cos^2 + sin^2); cos^2(arctan u) = 1/(1+u^2) with u = eta s; and the two
+    eta activations agree through tanh(x) + 1 = 2 sigmoid(2x)."""
+    rng = np.random.default_rng(21)
+    n = 257
+    x, a, b, c = (rng.standard_normal(n) * 2.0 for _ in range(4))
+    s = 1.7
+    al, ml, be, et = oracle.gates(x, a, b, c, s=s, mu_log_min=-2.0, eta_act="tanh", lib=lib)
+    sa, sb = 1.0 / (1.0 + np.exp(-a)), 1.0 / (1.0 + np.exp(-b))
+    _close(np.exp(al) / sa + be / sb, np.ones(n), 1e-13, "cos^2 + sin^2")
+    _close(al, -np.log1p((et * s) ** 2) + _logsig(a), 1e-13, "cos^2(arctan u)")
+    assert np.all(et > 0.0) and np.all(et < 2.0), "eta in (0, 2)"
+    assert np.all(ml >= -2.0) and np.all(ml < 0.0), "mu_log in [clamp, 0)"
+    al2, ml2, be2, et2 = oracle.gates(2.0 * x, a, b, c, s=s, mu_log_min=-2.0,
+                                      eta_act="2sigmoid", lib=lib)
+    _close(et2, et, 1e-14, "tanh(x)+1 = 2 sigmoid(2x)")
+    _close(al2, al, 1e-13, "same alpha through either activation")
+    _close(be2, be, 1e-13, "same beta through either activation")
+
+
+def pin_step_delta_norm(lib):
+    """||S_t - S_{t-1}||_F of one decode step: from zero states the first write is
+    S_1 = beta eta k v^T, so the norm is beta eta ||k|| ||v||; with alpha = 1 and
+    beta = 0 the fast weight does not move."""
+    rng = np.random.default_rng(23)
+    B, H, d = 2, 3, 5
+    q, k, v = (rng.standard_normal((B, H, d)) for _ in range(3))
+    be, et = rng.uniform(0.1, 0.9, (B, H)), rng.uniform(0.2, 1.8, (B, H))
+    al, ml = np.log(rng.uniform(0.3, 0.9, (B, H))), np.log(rng.uniform(0.4, 0.9, (B, H)))
+    Z = np.zeros((B, H, d, d))
+    _, _, S1, _ = oracle.step(q, k, v, al, ml, be, et, 0.5, Z, Z, lib=lib)
+    want = be * et * np.linalg.norm(k, axis=-1) * np.linalg.norm(v, axis=-1)
+    _close(oracle.step_delta_norm(Z, S1), want, 1e-13, "first write norm")
+    S0, M0 = rng.standard_normal((B, H, d, d)), rng.standard_normal((B, H, d, d))
+    _, _, S2, _ = oracle.step(q, k, v, np.zeros((B, H)), ml, np.zeros((B, H)), et, 0.5, S0, M0,
+                              lib=lib)
+    _close(oracle.step_delta_norm(S0, S2), np.zeros((B, H)), 1e-15, "alpha=1, beta=0")
+
+
 ALL_PINS = [pin_hand_scalar, pin_hand_matrix, pin_closed_form, pin_mu_zero_gated_delta_rule,
             pin_spectrum, pin_chunked_form, pin_chunk_coeffs, pin_step_matches_sequence,
-            pin_resume]
+            pin_resume, pin_gates_special_points, pin_gates_identities, pin_step_delta_norm]

@@ -43,6 +43,14 @@ MUTANTS = {
                      "s += exp(lm_c[j] - la_c[j] - mx);"),
     "la_off_by_one": ("la_c[r] = sa;\n", "la_c[r] = sa - alpha_log[g];\n"),
     "gamma_strict_lower": ("if (r < L && i <= r) {", "if (r < L && i < r) {"),
+    "gates_cos_sin_swapped": ("alpha_log[i] = log(ct * ct) + log_sigmoid(a[i]);",
+                              "alpha_log[i] = log(st * st) + log_sigmoid(a[i]);"),
+    "gates_theta_without_s": ("const double theta = atan(e * s);", "const double theta = atan(e);"),
+    "gates_eta_tanh_without_shift": ("? tanh(x_eta[i]) + 1.0 :", "? tanh(x_eta[i]) :"),
+    "gates_clamp_as_upper_bound": ("mu_log[i] = lm > mu_log_min ? lm : mu_log_min;",
+                                   "mu_log[i] = lm < mu_log_min ? lm : mu_log_min;"),
+    "gates_beta_not_squared": ("beta[i] = st * st * exp(log_sigmoid(b[i]));",
+                               "beta[i] = st * exp(log_sigmoid(b[i]));"),
 }
 
 
