@@ -239,6 +239,7 @@ def run_ours(args, rank, world, device):
     # ---- end to end through the public call, host (pinned) buffers
     e2e = None if args.no_e2e else run_e2e(args, mdn, inp, tok, spec, device, world)
     decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
+    gates = None if args.no_decode else run_gate_params(args, mdn, device, hbm, B * T * H)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -260,6 +261,8 @@ def run_ours(args, rank, world, device):
     }
     if decode:
         line["decode"] = decode
+    if gates:
+        line["gate_params"] = gates
     return line, spec
 
 
@@ -290,10 +293,64 @@ def run_decode(args, mdn, device, hbm_peak):
     sec = a.elapsed_time(b) / n * 1e-3
     _, bytes_per_step, _ = kernel_work("step", spec)
     gbs = bytes_per_step / sec / 1e9
+    # the same token with ||S_t - S_{t-1}||_F per head (memset + step + sqrt)
+    ds = torch.empty((B, H), device=device)
+    for _ in range(3):
+        mdn.step_with_delta_norm(t["q"], t["k"], t["v"], *(t[g] for g in gates), spec.q_corr,
+                                 S, M, o=o, ds_norm=ds, want_vtilde=False)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        mdn.step_with_delta_norm(t["q"], t["k"], t["v"], *(t[g] for g in gates), spec.q_corr,
+                                 S, M, o=o, ds_norm=ds, want_vtilde=False)
+    b.record()
+    torch.cuda.synchronize()
+    sec_dn = a.elapsed_time(b) / n * 1e-3
+    gbs_dn = bytes_per_step / sec_dn / 1e9
     return {"workload": spec.name, "tokens_per_s": round(B / sec, 1),
             "us_per_step": round(sec * 1e6, 2), "achieved_gbs": round(gbs, 1),
-            "peak_gbs": hbm_peak, "frac": round(gbs / hbm_peak, 4), "steps": n}
+            "peak_gbs": hbm_peak, "frac": round(gbs / hbm_peak, 4), "steps": n,
+            "with_delta_norm": {"us_per_step": round(sec_dn * 1e6, 2),
+                                "achieved_gbs": round(gbs_dn, 1),
+                                "frac": round(gbs_dn / hbm_peak, 4)}}
 
+
+def run_gate_params(args, mdn, device, hbm_peak, workload_n: int):
+    """K-0 (gates from pre-activations): 16 bytes read + 16 written per
+    element.  Timed at the workload's token-head count and at 2^26 elements
+    (512 MiB per launch, far above L2) for the HBM fraction.  The launches are
+    captured in a CUDA graph and replayed, so host overhead is not timed."""
+    out = {}
+    reps = 20
+    for label, n in (("workload", workload_n), ("hbm", 1 << 26)):
+        g = torch.Generator(device=device).manual_seed(5)
+        pre = [torch.randn(n, device=device, generator=g) for _ in range(4)]
+        res = tuple(torch.empty(n, device=device) for _ in range(4))
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                mdn.gate_params(*pre, s=1.0, mu_log_min=-1.0, out=res)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(reps):
+                mdn.gate_params(*pre, s=1.0, mu_log_min=-1.0, out=res)
+        graph.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        sec = a.elapsed_time(b) / reps * 1e-3
+        gbs = 32.0 * n / sec / 1e9
+        out[label] = {"elements": n, "us_per_launch": round(sec * 1e6, 2),
+                      "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
+        del graph, pre, res
+    out["peak_gbs"] = hbm_peak
+    out["timing"] = f"CUDA graph of {reps} back-to-back launches, replayed once after a warm replay"
+    return out
 
 def run_e2e(args, mdn, inp, tok, spec, device, world):
     """Same metric through the public API with pinned host inputs: per step the
@@ -469,7 +526,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode-shape measurement")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-shape and gate-kernel side measurements")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -165,6 +165,54 @@ mdn_status mdn_step(const void *q, const void *k, const void *v, mdn_dtype in_dt
                     void *o, void *vtilde, int flags, mdn_stream_t stream);
 
 /*
+ * mdn_step that also measures how far the fast weight moved:
+ *
+ *   ds_norm     [B,H] fp32 output: ||S_t - S_{t-1}||_F of each head (the
+ *               decoding diagnostic of ijyty.com section 8, which averages it
+ *               over steps).  Must not be NULL when B*H > 0.
+ *
+ * Enqueues a memset of ds_norm, the step (whose blocks add their shares of
+ * the squared norm atomically) and an in-place square root.  o, vtilde, S and
+ * M come out bit-identical to mdn_step's.  Everything else as mdn_step.
+ */
+mdn_status mdn_step_delta_norm(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                               const float *alpha_log, const float *mu_log,
+                               const float *beta, const float *eta, float d_corr,
+                               float *S, float *M, int B, int H, int dk, int dv,
+                               void *o, void *vtilde, float *ds_norm, int flags,
+                               mdn_stream_t stream);
+
+/* Activations of eta for mdn_gate_params. */
+#define MDN_ETA_TANH     0  /* eta = tanh(x) + 1 (the pages' choice) */
+#define MDN_ETA_2SIGMOID 1  /* eta = 2 sigmoid(x) (their ablation, article section 8) */
+
+/*
+ * The four gates from raw per-token pre-activations, by the pages' stable
+ * parameterisation (summary step 6; ijyty.com sections 5 and 8):
+ *
+ *   eta       = tanh(x_eta) + 1   (or 2 sigmoid(x_eta), eta_act)
+ *   theta     = arctan(eta * s)
+ *   alpha_log = log(cos^2(theta) sigmoid(a))
+ *   beta      = sin^2(theta) sigmoid(b)
+ *   mu_log    = max(log sigmoid(c), mu_log_min)
+ *
+ *   x_eta, a, b, c   n fp32 pre-activations each (any layout; elementwise).
+ *   s                the scale of theta (finite).
+ *   mu_log_min       the lower clamp of log mu (finite; the pages use -2, their
+ *                    ablations -1.5 .. -1).
+ *   alpha_log, mu_log, beta, eta   n fp32 outputs, ready for mdn_chunk_fwd /
+ *                    mdn_step.  Outputs may not alias inputs.
+ *
+ * Pointers 4-byte aligned (16-byte alignment and n % 4 == 0 take a vectorised
+ * path).  Errors: MDN_ERR_INVALID_ARG (n < 0, null or unaligned pointer,
+ * unknown eta_act, non-finite s or clamp), MDN_ERR_CUDA.
+ */
+mdn_status mdn_gate_params(const float *x_eta, const float *a, const float *b, const float *c,
+                           long long n, float s, float mu_log_min, int eta_act,
+                           float *alpha_log, float *mu_log, float *beta, float *eta,
+                           mdn_stream_t stream);
+
+/*
  * The chunk coefficients alone (the gate-preparation stage of mdn_chunk_fwd;
  * summary step 5), each cumulative quantity restarting at every chunk start:
  *

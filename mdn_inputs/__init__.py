@@ -89,6 +89,12 @@ class Inputs:
     eta: np.ndarray
     S0: Optional[np.ndarray]
     M0: Optional[np.ndarray]
+    # the gate pre-activations as float32 (what a gate-parameterisation kernel
+    # reads); the gates above were formed from their float64 draws
+    x_eta: Optional[np.ndarray] = None
+    a_pre: Optional[np.ndarray] = None
+    b_pre: Optional[np.ndarray] = None
+    c_pre: Optional[np.ndarray] = None
 
     @property
     def d_corr(self) -> float:
@@ -152,7 +158,8 @@ def make_inputs(spec: Spec) -> Inputs:
     return Inputs(spec=spec, q=q, k=k, v=v, q_store=q_store, k_store=k_store,
                   v_store=v_store, alpha_log=np.log(alpha).astype(f32),
                   mu_log=mu_log.astype(f32), beta=beta.astype(f32),
-                  eta=eta.astype(f32), S0=S0, M0=M0)
+                  eta=eta.astype(f32), S0=S0, M0=M0, x_eta=x.astype(f32),
+                  a_pre=a.astype(f32), b_pre=b.astype(f32), c_pre=c.astype(f32))
 
 
 def to_torch(inp: Inputs, device="cpu", pin: bool = False) -> dict:

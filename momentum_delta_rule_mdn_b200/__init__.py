@@ -5,4 +5,5 @@ The compute lives in ``lib/libmdn.so`` (hand-written CUDA behind the C ABI of
 library is loaded on first use and there is no CPU fallback.
 """
 from .api import (MDNError, chunk_fwd, chunk_fwd_workspace_size, chunk_gate_prep,  # noqa: F401
-                  step, status_string, library, profile_enable, profile_read)
+                  step, step_with_delta_norm, gate_params, status_string, library,
+                  profile_enable, profile_read)

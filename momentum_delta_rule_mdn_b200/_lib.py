@@ -15,6 +15,8 @@ MDN_FORCE_SIMT = 0x2
 MDN_SLICE32 = 0x4
 MDN_SLICE64 = 0x8
 MDN_TEST_NO_INTRA = 0x100
+MDN_ETA_TANH = 0
+MDN_ETA_2SIGMOID = 1
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -28,6 +30,10 @@ SIGNATURES = {
                            _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp]),
     "mdn_step": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                       _i, _i, _i, _i, _vp, _vp, _i, _vp]),
+    "mdn_step_delta_norm": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                 _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
+    "mdn_gate_params": (_i, [_vp, _vp, _vp, _vp, ctypes.c_longlong, _f, _f, _i,
+                             _vp, _vp, _vp, _vp, _vp]),
     "mdn_chunk_gate_prep": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                  _vp, _vp, _vp, _vp, _vp, _vp]),
     "mdn_chunk_fwd_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,

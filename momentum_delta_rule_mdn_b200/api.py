@@ -152,6 +152,57 @@ def step(q, k, v, alpha_log, mu_log, beta, eta, d: float, S: torch.Tensor, M: to
     return o, vtilde
 
 
+def step_with_delta_norm(q, k, v, alpha_log, mu_log, beta, eta, d: float, S: torch.Tensor,
+                         M: torch.Tensor, *, o: Optional[torch.Tensor] = None,
+                         vtilde: Optional[torch.Tensor] = None, ds_norm: Optional[torch.Tensor] = None,
+                         want_vtilde: bool = True, stream: Optional[torch.cuda.Stream] = None):
+    """As :func:`step`, and also returns ds_norm [B,H] = ||S_t - S_{t-1}||_F per head."""
+    B, H, D = q.shape
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, q.dtype, (B, H, D), name)
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (B, H), name)
+    _need(S, torch.float32, (B, H, D, D), "S")
+    _need(M, torch.float32, (B, H, D, D), "M")
+    if o is None:
+        o = torch.empty_like(q)
+    if vtilde is None and want_vtilde:
+        vtilde = torch.empty_like(q)
+    if ds_norm is None:
+        ds_norm = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _need(ds_norm, torch.float32, (B, H), "ds_norm")
+    status = library().mdn_step_delta_norm(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta),
+        float(d), _ptr(S), _ptr(M), B, H, D, D, _ptr(o), _ptr(vtilde), _ptr(ds_norm), 0,
+        _stream_handle(stream))
+    _check(status, "mdn_step_delta_norm")
+    return o, vtilde, ds_norm
+
+
+_ETA_ACT = {"tanh": 0, "2sigmoid": 1}
+
+
+def gate_params(x_eta, a, b, c, s: float = 1.0, mu_log_min: float = -2.0,
+                eta_act: str = "tanh", *, out=None, stream: Optional[torch.cuda.Stream] = None):
+    """The four gates from pre-activations of any common shape (fp32, contiguous).
+    Returns (alpha_log, mu_log, beta, eta) of that shape."""
+    if eta_act not in _ETA_ACT:
+        raise ValueError(f"eta_act must be one of {sorted(_ETA_ACT)}, got {eta_act!r}")
+    shape = tuple(x_eta.shape)
+    for name, t in (("x_eta", x_eta), ("a", a), ("b", b), ("c", c)):
+        _need(t, torch.float32, shape, name)
+    if out is None:
+        out = tuple(torch.empty_like(x_eta) for _ in range(4))
+    for name, t in zip(("alpha_log", "mu_log", "beta", "eta"), out):
+        _need(t, torch.float32, shape, name)
+    status = library().mdn_gate_params(
+        _ptr(x_eta), _ptr(a), _ptr(b), _ptr(c), x_eta.numel(), float(s), float(mu_log_min),
+        _ETA_ACT[eta_act], *(_ptr(t) for t in out), _stream_handle(stream))
+    _check(status, "mdn_gate_params")
+    return tuple(out)
+
+
 def chunk_gate_prep(alpha_log, mu_log, beta, eta, C: int = 64, with_gamma: bool = True,
                     stream: Optional[torch.cuda.Stream] = None):
     """Chunk coefficients: (la, lm, lc, b) [B,H,NT*C] and gamma [B,H,NT,C,C] (or None)."""

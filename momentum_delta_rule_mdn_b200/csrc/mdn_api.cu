@@ -3,6 +3,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <cmath>
 #include <cstdio>
 
 #include "mdn_internal.cuh"
@@ -236,10 +237,12 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     return MDN_OK;
 }
 
-mdn_status mdn_step(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
-                    const float* alpha_log, const float* mu_log, const float* beta,
-                    const float* eta, float d_corr, float* S, float* M, int B, int H, int dk,
-                    int dv, void* o, void* vtilde, int flags, mdn_stream_t stream)
+namespace {
+mdn_status step_impl(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                     const float* alpha_log, const float* mu_log, const float* beta,
+                     const float* eta, float d_corr, float* S, float* M, int B, int H, int dk,
+                     int dv, void* o, void* vtilde, float* ds_norm, int flags,
+                     mdn_stream_t stream)
 {
     mdn_status st = check_sizes(B, 1, H, dk, dv, kChunk, in_dtype);
     if (st != MDN_OK) return st;
@@ -253,9 +256,48 @@ mdn_status mdn_step(const void* q, const void* k, const void* v, mdn_dtype in_dt
     for (const void* p : gates)
         if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
     if (!S || !M || !aligned16(S) || !aligned16(M)) return MDN_ERR_INVALID_ARG;
+    if (ds_norm && !aligned4(ds_norm)) return MDN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return cuda_status(launch_step(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S,
-                                   M, B, H, dk, o, vtilde, s));
+                                   M, B, H, dk, o, vtilde, ds_norm, s));
+}
+}  // namespace
+
+mdn_status mdn_step(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                    const float* alpha_log, const float* mu_log, const float* beta,
+                    const float* eta, float d_corr, float* S, float* M, int B, int H, int dk,
+                    int dv, void* o, void* vtilde, int flags, mdn_stream_t stream)
+{
+    return step_impl(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S, M, B, H, dk,
+                     dv, o, vtilde, nullptr, flags, stream);
+}
+
+mdn_status mdn_step_delta_norm(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                               const float* alpha_log, const float* mu_log, const float* beta,
+                               const float* eta, float d_corr, float* S, float* M, int B, int H,
+                               int dk, int dv, void* o, void* vtilde, float* ds_norm, int flags,
+                               mdn_stream_t stream)
+{
+    if (!ds_norm && B > 0 && H > 0) return MDN_ERR_INVALID_ARG;
+    return step_impl(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S, M, B, H, dk,
+                     dv, o, vtilde, ds_norm, flags, stream);
+}
+
+mdn_status mdn_gate_params(const float* x_eta, const float* a, const float* b, const float* c,
+                           long long n, float s, float mu_log_min, int eta_act,
+                           float* alpha_log, float* mu_log, float* beta, float* eta,
+                           mdn_stream_t stream)
+{
+    if (n < 0) return MDN_ERR_INVALID_ARG;
+    if (eta_act != MDN_ETA_TANH && eta_act != MDN_ETA_2SIGMOID) return MDN_ERR_INVALID_ARG;
+    if (!std::isfinite(s) || !std::isfinite(mu_log_min)) return MDN_ERR_INVALID_ARG;
+    if (n == 0) return MDN_OK;
+    const void* ptrs[] = {x_eta, a, b, c, alpha_log, mu_log, beta, eta};
+    for (const void* p : ptrs)
+        if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    return cuda_status(launch_gate_params(x_eta, a, b, c, n, s, mu_log_min, eta_act, alpha_log,
+                                          mu_log, beta, eta,
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 mdn_status mdn_chunk_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,

@@ -111,7 +111,7 @@ struct ChunkArgs {
 // Kernel kinds known to the optional timing facility (profile.cu).
 enum KernelKind {
     kGatePrep = 0, kIntraSimt, kInterSimt, kOutputSimt, kStep, kFiniteCheck,
-    kChunkTc, kIntraTc, kInterTc, kOutputTc, kKernelKinds
+    kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kKernelKinds
 };
 // Record a start event for a launch of kind k on s (returns a slot, or -1 when
 // timing is off); prof_end records the matching stop event.
@@ -137,10 +137,16 @@ mdn_status cuda_fail(cudaError_t e);
 // ns: columns of d_v per inter-chunk CTA (32 or 64), 0 = choose by batch size
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve);
+// ds_norm (nullable, [B*H]): receives ||S_t - S_{t-1}||_F of each head.
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
                         const float* eta, float dcorr, float* S, float* M, int B, int H,
-                        int D, void* o, void* vt, cudaStream_t s);
+                        int D, void* o, void* vt, float* ds_norm, cudaStream_t s);
+// Gates from pre-activations (K-0), n elements; eta_act 0 = tanh + 1, 1 = 2 sigmoid.
+cudaError_t launch_gate_params(const float* x_eta, const float* a, const float* b, const float* c,
+                               long long n, float s_scale, float mu_log_min, int eta_act,
+                               float* alpha_log, float* mu_log, float* beta, float* eta,
+                               cudaStream_t s);
 cudaError_t launch_finite_check(const void* x, size_t n, bool bf16, unsigned* flag,
                                 cudaStream_t s);
 

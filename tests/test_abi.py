@@ -118,3 +118,28 @@ def test_step_and_gate_prep_validation(lib):
     assert gp(C=16) == E.MDN_ERR_UNSUPPORTED
     assert gp(la=None) == E.MDN_ERR_INVALID_ARG
     assert gp(T=0) == E.MDN_OK
+
+
+def test_gate_params_and_delta_norm_validation(lib):
+    E = _lib
+    inf = float("inf")
+
+    def gp(n=10, s=1.0, mn=-2.0, act=E.MDN_ETA_TANH, x=FAKE, out=FAKE):
+        return lib.mdn_gate_params(x, FAKE, FAKE, FAKE, n, s, mn, act, out, FAKE, FAKE, FAKE,
+                                   None)
+    assert gp(n=-1) == E.MDN_ERR_INVALID_ARG
+    assert gp(act=2) == E.MDN_ERR_INVALID_ARG
+    assert gp(s=inf) == E.MDN_ERR_INVALID_ARG
+    assert gp(mn=float("nan")) == E.MDN_ERR_INVALID_ARG
+    assert gp(x=None) == E.MDN_ERR_INVALID_ARG
+    assert gp(out=FAKE + 2) == E.MDN_ERR_INVALID_ARG                 # not 4-byte aligned
+    assert gp(n=0) == E.MDN_OK
+    assert gp(n=0, act=E.MDN_ETA_2SIGMOID, x=None) == E.MDN_OK       # nothing to read
+
+    def dn(B=2, ds=FAKE, d=128):
+        return lib.mdn_step_delta_norm(FAKE, FAKE, FAKE, E.MDN_BF16, FAKE, FAKE, FAKE, FAKE, 0.5,
+                                       FAKE, FAKE, B, 3, d, d, FAKE, None, ds, 0, None)
+    assert dn(ds=None) == E.MDN_ERR_INVALID_ARG
+    assert dn(ds=FAKE + 1) == E.MDN_ERR_INVALID_ARG
+    assert dn(d=32) == E.MDN_ERR_UNSUPPORTED
+    assert dn(B=0, ds=None) == E.MDN_OK
