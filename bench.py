@@ -240,6 +240,7 @@ def run_ours(args, rank, world, device):
     e2e = None if args.no_e2e else run_e2e(args, mdn, inp, tok, spec, device, world)
     decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
     gates = None if args.no_decode else run_gate_params(args, mdn, device, hbm, B * T * H)
+    varlen = None if args.no_decode else run_varlen(args, mdn, device, spec0)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -263,6 +264,8 @@ def run_ours(args, rank, world, device):
         line["decode"] = decode
     if gates:
         line["gate_params"] = gates
+    if varlen:
+        line["varlen"] = varlen
     return line, spec
 
 
@@ -313,6 +316,57 @@ def run_decode(args, mdn, device, hbm_peak):
             "with_delta_norm": {"us_per_step": round(sec_dn * 1e6, 2),
                                 "achieved_gbs": round(gbs_dn, 1),
                                 "frac": round(gbs_dn / hbm_peak, 4)}}
+
+
+VARLEN_LENGTHS = (3000, 1500, 64, 2500, 1, 700, 300, 127)
+
+
+def run_varlen(args, mdn, device, spec0):
+    """mdn_chunk_fwd_varlen on the workload's token budget (B*T tokens, same H
+    and d) split into sequences of mixed lengths (the fixed list above, the
+    remainder as a last sequence).  L2 flushed before every timed call, as in
+    the main step."""
+    total = spec0.B * spec0.T
+    lens = []
+    for x in VARLEN_LENGTHS:
+        if sum(lens) + x <= total:
+            lens.append(x)
+    if sum(lens) < total:
+        lens.append(total - sum(lens))
+    H, d = spec0.H, spec0.d
+    inp = mi.make_inputs(mi.replace(spec0, B=1, T=total, seed=spec0.seed + 21))
+    dev = {k: v[0] for k, v in mi.to_torch(inp, device).items() if v is not None}
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=device)
+    N = len(lens)
+    lib = mdn.library()
+    code = 1 if dev["q"].dtype == torch.bfloat16 else 0
+    ws = torch.empty(int(lib.mdn_chunk_fwd_varlen_workspace_size(N, total, H, d, d, spec0.C, code)),
+                     dtype=torch.uint8, device=device)
+    out = (torch.empty_like(dev["q"]), torch.empty_like(dev["q"]),
+           torch.empty((N, H, d, d), device=device), torch.empty((N, H, d, d), device=device))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    gates = ("alpha_log", "mu_log", "beta", "eta")
+
+    def call():
+        mdn.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), cu,
+                             inp.d_corr, None, None, spec0.C, out=out, workspace=ws)
+    for _ in range(3):
+        flush.zero_()
+        call()
+    n = max(5, min(args.steps, 50))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush.zero_()
+        ev[i][0].record()
+        call()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    return {"lengths": lens, "tokens": total, "H": H, "d": d, "ms": round(ms, 5),
+            "tokens_per_s": round(total / (ms * 1e-3), 1), "calls": n,
+            "includes": "checked offsets, chunk-aligned gather, intra + inter kernels"}
 
 
 def run_gate_params(args, mdn, device, hbm_peak, workload_n: int):
@@ -526,7 +580,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode-shape and gate-kernel side measurements")
+    ap.add_argument("--no-decode", action="store_true", help="skip the side measurements (decode shape, gate kernel, packed sequences)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

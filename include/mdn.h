@@ -147,6 +147,48 @@ mdn_status mdn_chunk_fwd(const void *q, const void *k, const void *v, mdn_dtype 
                          mdn_stream_t stream);
 
 /*
+ * Bytes of device scratch that mdn_chunk_fwd_varlen needs, or 0 if the sizes
+ * are invalid or unsupported.  Pure host function.
+ */
+size_t mdn_chunk_fwd_varlen_workspace_size(int N, int total_T, int H, int dk, int dv, int C,
+                                           mdn_dtype in_dtype);
+
+/*
+ * mdn_chunk_fwd over N independent sequences of different lengths packed
+ * along the token axis.  The pages run one sequence per batch row; this is
+ * the plain extension: sequence s is the recurrence above over its own
+ * tokens, from its own entering state.
+ *
+ *   q, k, v, o, vtilde  [total_T,H,d] in_dtype, the sequences back to back.
+ *   alpha_log, mu_log, beta, eta  [total_T,H] fp32.
+ *   cu_seqlens  DEVICE pointer to N+1 ints: sequence s is tokens
+ *               [cu_seqlens[s], cu_seqlens[s+1]); cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[N] = total_T.  Empty sequences
+ *               are allowed (their S_T, M_T are S0, M0).
+ *   S0, M0      [N,H,d,d] fp32 or NULL (zeros); S_T, M_T  [N,H,d,d] fp32.
+ *   workspace   at least mdn_chunk_fwd_varlen_workspace_size(...) bytes,
+ *               256-byte aligned.
+ *   flags       as mdn_chunk_fwd (without MDN_TEST_NO_INTRA).
+ *
+ * The inputs are first copied into a chunk-aligned layout (each sequence
+ * padded to a whole number of chunks with steps that leave S and M
+ * unchanged); the chain kernels write o and vtilde straight back to the
+ * packed rows.  cu_seqlens is read on the device only.  If it breaks the
+ * rules above, every sequence is treated as empty (S_T = S0, M_T = M0, o and
+ * vtilde untouched) and, with MDN_CHECK_FINITE, the call returns
+ * MDN_ERR_INVALID_ARG.  Other errors as mdn_chunk_fwd.  Asynchronous on
+ * `stream` (except with MDN_CHECK_FINITE).
+ */
+mdn_status mdn_chunk_fwd_varlen(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                                const float *alpha_log, const float *mu_log,
+                                const float *beta, const float *eta, float d_corr,
+                                const int *cu_seqlens, int N, int total_T,
+                                const float *S0, const float *M0, int H, int dk, int dv, int C,
+                                void *o, void *vtilde, float *S_T, float *M_T,
+                                void *workspace, size_t ws_bytes, int flags,
+                                mdn_stream_t stream);
+
+/*
  * One decode token for every (b, h): the stepwise recurrence above, applied
  * in place (ijyty.com section 6: decoding runs the recurrence token by token).
  *

@@ -128,6 +128,52 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0
     return o, vt, S_T, M_T
 
 
+def chunk_fwd_varlen(q, k, v, alpha_log, mu_log, beta, eta, cu_seqlens: torch.Tensor,
+                     d: float = 0.5, S0=None, M0=None, C: int = 64, *, out=None,
+                     workspace: Optional[torch.Tensor] = None, flags: int = 0,
+                     stream: Optional[torch.cuda.Stream] = None):
+    """Chunkwise pass over N sequences packed along the token axis.
+
+    q, k, v: [total_T,H,d]; gates [total_T,H] float32; cu_seqlens: int32
+    [N+1] on the device (sequence s is tokens cu_seqlens[s]:cu_seqlens[s+1]);
+    S0, M0: [N,H,d,d] float32 or None.  Returns (o, vtilde, S_T, M_T)."""
+    total_T, H, D = q.shape
+    N = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous() or N < 0:
+        raise ValueError("cu_seqlens: expected a contiguous int32 tensor of N+1 offsets")
+    if cu_seqlens.device != q.device:
+        raise ValueError("cu_seqlens must be on the same device as q")
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, q.dtype, q.shape, name)
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (total_T, H), name)
+    _need(S0, torch.float32, (N, H, D, D), "S0")
+    _need(M0, torch.float32, (N, H, D, D), "M0")
+    if out is None:
+        o = torch.empty_like(q)
+        vt = torch.empty_like(q)
+        S_T = torch.empty((N, H, D, D), dtype=torch.float32, device=q.device)
+        M_T = torch.empty((N, H, D, D), dtype=torch.float32, device=q.device)
+    else:
+        o, vt, S_T, M_T = out
+        _need(o, q.dtype, q.shape, "o")
+        _need(vt, q.dtype, q.shape, "vtilde")
+        _need(S_T, torch.float32, (N, H, D, D), "S_T")
+        _need(M_T, torch.float32, (N, H, D, D), "M_T")
+    lib = library()
+    ws_bytes = int(lib.mdn_chunk_fwd_varlen_workspace_size(N, total_T, H, D, D, C, code))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    status = lib.mdn_chunk_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta),
+        float(d), _ptr(cu_seqlens), N, total_T, _ptr(S0), _ptr(M0), H, D, D, C, _ptr(o),
+        _ptr(vt), _ptr(S_T), _ptr(M_T), _ptr(workspace), workspace.numel(), int(flags),
+        _stream_handle(stream))
+    _check(status, "mdn_chunk_fwd_varlen")
+    return o, vt, S_T, M_T
+
+
 def step(q, k, v, alpha_log, mu_log, beta, eta, d: float, S: torch.Tensor, M: torch.Tensor,
          *, o: Optional[torch.Tensor] = None, vtilde: Optional[torch.Tensor] = None,
          want_vtilde: bool = True, stream: Optional[torch.cuda.Stream] = None):

@@ -120,6 +120,8 @@ struct InterArgs {
     unsigned* status;
     float* dbg;  // diagnostics: phase clocks of the MMA and load lanes of CTA 0 (null in normal use)
     int T, H, NT;
+    const int* cu_seqlens;  // variable-length mode (see ChunkArgs); null otherwise
+    const int* cu_chunks;
 };
 
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
@@ -180,10 +182,10 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int quad = warp & 3;                   // TMEM lane quadrant this warp may access
     const int lane = (quad << 5) | lid;          // TMEM lane = operand row
     const int slice = blockIdx.x % (D / NS);
-    const int bh = blockIdx.x / (D / NS);
-    const int b = bh / a.H, h = bh % a.H;
+    const Chain ch = chain_of(a, blockIdx.x / (D / NS));
+    const int b = ch.b, h = ch.h;
     const int j0 = slice * NS;
-    const int NT = a.NT;
+    const int NT = ch.nt;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BARS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC + 4);
@@ -209,7 +211,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int hc = (warp - kChainWarp0) >> 2;  // column group of a chain warp
     float s[NH], m[NH];
     if (chain) {
-        const size_t row = ((size_t)bh * D + lane) * D + j0 + NH * hc;
+        const size_t row = ((size_t)ch.sh * D + lane) * D + j0 + NH * hc;
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             s[j] = a.S0 ? a.S0[row + j] : 0.f;
@@ -302,7 +304,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             int issued_kq = 0, issued_fb = 0, issued_vc = 0;
             for (int n = 0; n < NT; ++n) {
                 const int s2 = n & 1, sv = n % L::NVC;
-                const long long chunk = (long long)bh * NT + n;
+                const long long chunk = ch.chunk0 + n;
                 if (n >= 2 && !wait_bar(&bars[B_M1 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
                 // the operands of chunk n are in global memory
                 if (!wait_ready(a.ready + chunk, abort_flag)) break;
@@ -313,7 +315,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     uint8_t* dst = sm + L::KQ0 + s2 * 32768 + p * 16384;
-                    tma_load_4d(dst, &tm_k, p * 64, h, n * C, b, fb);
+                    tma_load_4d(dst, &tm_k, p * 64, h, (ch.n0 + n) * C, b, fb);
                     tma_load_3d(dst + 8192, &tm_qh, p * 64, 0, (int)chunk, fb);
                 }
                 issued_kq = n + 1;
@@ -332,7 +334,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 clk.lap(2);
                 fb = &bars[B_FVC + sv];
                 mbar_arrive_expect_tx(fb, L::kTxVC);
-                tma_load_4d(sm + L::V0 + sv * L::V_BYTES, &tm_v, j0, h, n * C, b, fb);
+                tma_load_4d(sm + L::V0 + sv * L::V_BYTES, &tm_v, j0, h, (ch.n0 + n) * C, b, fb);
                 bulk_load(sm + L::CR0 + sv * 1024, a.crec + chunk * 256, 1024, fb);
                 issued_vc = n + 1;
             }
@@ -440,8 +442,8 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
             if (!warp_wait(&bars[B_M3 + s2], (n >> 1) & 1, abort_flag)) break;
             tc_fence_after_sync();
-            const int t = n * C + r;
-            uint4* dst = reinterpret_cast<uint4*>(out + (((size_t)b * a.T + t) * a.H + h) * D + j0);
+            const int t = n * C + r;  // token of the chain
+            uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(ch.out0 + t) * a.H + h) * D + j0);
 #pragma unroll 1
             for (int q16 = 0; q16 < NS / 16; ++q16) {
                 float x[16], y[16];
@@ -459,7 +461,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     tmem_ld16(tq + L::TM_A3 + NS * s2 + 16 * q16, x);
                     tmem_wait_ld();
                 }
-                if (t < a.T) {
+                if (t < ch.len) {
                     dst[2 * q16] = bf16x8(x);
                     dst[2 * q16 + 1] = bf16x8(x + 8);
                 }
@@ -474,7 +476,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __syncthreads();
     const bool ok = *abort_flag == 0;
     if (chain && ok) {
-        const size_t row = ((size_t)bh * D + lane) * D + j0 + NH * hc;
+        const size_t row = ((size_t)ch.sh * D + lane) * D + j0 + NH * hc;
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             a.S_T[row + j] = s[j];
@@ -521,11 +523,14 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
     t.T = a.T;
     t.H = a.H;
     t.NT = a.NT;
+    t.cu_seqlens = a.cu_seqlens;
+    t.cu_chunks = a.cu_chunks;
     cudaError_t e = cudaFuncSetAttribute(chunk_inter_kernel<NS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const long long blocks = (long long)a.B * a.H * (D / NS);
+    const long long chains = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
+    const long long blocks = chains * (D / NS);
     ProfScope ps(kInterTc, s);
     // Programmatic dependent launch: the CTAs may start while the intra-chunk
     // kernel (launched just before on s) still runs; each chunk is read only
@@ -563,7 +568,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const long long heads = (long long)a.B * a.H;
+    const long long heads = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
     const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
     if (ns == 0) ns = heads * 4 <= sms ? 32 : 64;
     const long long ctas = heads * (D / ns);

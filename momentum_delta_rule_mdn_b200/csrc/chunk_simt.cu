@@ -140,21 +140,22 @@ inter_simt_kernel(ChunkArgs a)
     const int tid = threadIdx.x;
     const int nslices = D / NS;
     const int slice = blockIdx.x % nslices;
-    const long long bh = blockIdx.x / nslices;
-    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const Chain ch = chain_of(a, blockIdx.x / nslices);
+    const int b = ch.b, h = ch.h;
     const int j0 = slice * NS;
     const int j = tid % NS;        // column inside the slice
     const int rg = tid / NS;       // 0..7
 
-    const size_t st_base = (size_t)bh * D * D;
+    const size_t st_base = (size_t)ch.sh * D * D;
     for (int e = 0; e < EPT; ++e) {
         const int i = rg + 8 * e;
         Ss[i * NS + j] = a.S0 ? a.S0[st_base + (size_t)i * D + j0 + j] : 0.f;
         Ms[i * NS + j] = a.M0 ? a.M0[st_base + (size_t)i * D + j0 + j] : 0.f;
     }
 
-    for (int n = 0; n < a.NT; ++n) {
-        const size_t chunk = (size_t)bh * a.NT + n;
+    for (int nc = 0; nc < ch.nt; ++nc) {
+        const int n = ch.n0 + nc;  // chunk of the input rows
+        const size_t chunk = (size_t)ch.chunk0 + nc;
         const size_t crow = chunk * C;
         const size_t cmat = chunk * C * D;
         __syncthreads();  // previous chunk's state update is complete
@@ -191,9 +192,9 @@ inter_simt_kernel(ChunkArgs a)
             float s = acc[e];
             for (int i = 0; i < D; ++i) s = fmaf(tile[r * KS + i], Ms[i * NS + j], s);
             Vs[r * VS + j] = s;
-            const int t = n * C + r;
-            if (t < a.T)
-                st_elem(static_cast<Tin*>(a.vt) + (((size_t)b * a.T + t) * a.H + h) * D + j0 + j, s);
+            const int t = nc * C + r;  // token of the chain
+            if (t < ch.len)
+                st_elem(static_cast<Tin*>(a.vt) + ((size_t)(ch.out0 + t) * a.H + h) * D + j0 + j, s);
         }
         __syncthreads();
         // Qhat tile, then the carried-state part of o.
@@ -266,14 +267,15 @@ output_simt_kernel(ChunkArgs a)
     const long long bh = blockIdx.x / a.NT;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x;
+    const ChunkOut co = chunk_out(a, b, n);  // where this chunk's rows of vt and o live
     for (int idx = tid; idx < C * D; idx += 256) {
         const int r = idx / D, c = idx % D, t = n * C + r;
         float qv = 0.f, kv = 0.f, vv = 0.f;
-        if (t < a.T) {
+        if (r < co.valid) {
             const size_t g = (((size_t)b * a.T + t) * a.H + h) * D + c;
             kv = ld_tok<Tin>(a.k, g);
             qv = ld_tok<Tin>(a.q, g) - a.dcorr * kv;
-            vv = ld_tok<Tin>(a.vt, g);
+            vv = ld_tok<Tin>(a.vt, ((size_t)(co.row0 + r) * a.H + h) * D + c);
         }
         Qs[r * KS + c] = qv;
         Ks[r * KS + c] = kv;
@@ -295,11 +297,11 @@ output_simt_kernel(ChunkArgs a)
     __syncthreads();
     const size_t orow = chunk * C * D;  // Oi is [B*H, NT*C, D]
     for (int idx = tid; idx < C * D; idx += 256) {
-        const int r = idx / D, c = idx % D, t = n * C + r;
+        const int r = idx / D, c = idx % D;
         float s = a.Oi[orow + idx];
         for (int i = 0; i <= r; ++i) s = fmaf(As[r * AS + i], Vs[i * D + c], s);
-        if (t < a.T)
-            st_elem(static_cast<Tin*>(a.o) + (((size_t)b * a.T + t) * a.H + h) * D + c, s);
+        if (r < co.valid)
+            st_elem(static_cast<Tin*>(a.o) + ((size_t)(co.row0 + r) * a.H + h) * D + c, s);
     }
 }
 
@@ -328,8 +330,8 @@ cudaError_t launch_simt_typed(const ChunkArgs& a, cudaStream_t s)
     if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(kInterSimt, s);
-        inter_simt_kernel<Tin, D>
-            <<<(unsigned)((long long)a.B * a.H * (D / kSlice)), 256, smem3, s>>>(a);
+        const long long chains = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
+        inter_simt_kernel<Tin, D><<<(unsigned)(chains * (D / kSlice)), 256, smem3, s>>>(a);
     }
     if ((e = cudaGetLastError())) return e;
     {

@@ -66,6 +66,65 @@ mdn_status check_sizes(int B, int T, int H, int dk, int dv, int C, mdn_dtype dt)
 
 mdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDN_OK : mdn::cuda_fail(e); }
 
+// Points the scratch members of a at their regions of ws.
+void carve(ChunkArgs& a, char* ws, const WsLayout& w)
+{
+    a.status = reinterpret_cast<unsigned*>(ws + w.status);
+    a.la = reinterpret_cast<float*>(ws + w.la);
+    a.lm = reinterpret_cast<float*>(ws + w.lm);
+    a.lc = reinterpret_cast<float*>(ws + w.lc);
+    a.bco = reinterpret_cast<float*>(ws + w.bco);
+    a.gamma = reinterpret_cast<float*>(ws + w.gamma);
+    a.U = reinterpret_cast<float*>(ws + w.U);
+    a.Y = reinterpret_cast<float*>(ws + w.Y);
+    a.Z = reinterpret_cast<float*>(ws + w.Z);
+    a.Oi = reinterpret_cast<float*>(ws + w.Oi);
+    a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + w.qhat);
+    a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
+    a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);
+    a.crec = reinterpret_cast<float*>(ws + w.crec);
+    a.ready = reinterpret_cast<unsigned*>(ws + w.ready);
+}
+
+// The chunk pass over a (scratch carved; status zeroed by the caller when
+// MDN_CHECK_FINITE is set).  ntok: elements of o and of vt; nstate: heads of
+// S_T and M_T.
+mdn_status run_pass(ChunkArgs& a, mdn_dtype in_dtype, int flags, cudaStream_t s, size_t ntok,
+                    size_t nstate)
+{
+    cudaError_t e;
+    const int D = a.D;
+    const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
+    if (tensor_cores) {
+        const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
+        if ((e = cudaMemsetAsync(a.ready, 0, ((size_t)a.B * a.H * a.NT + 1) * sizeof(unsigned), s)))
+            return mdn::cuda_fail(e);
+        a.test_no_intra = (flags & MDN_TEST_NO_INTRA) != 0;
+        if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
+    } else {
+        if ((e = launch_gate_prep(a.alpha_log, a.mu_log, a.beta, a.eta, a.B, a.T, a.H, a.la, a.lm,
+                                  a.lc, a.bco, a.gamma, s)))
+            return mdn::cuda_fail(e);
+        if ((e = launch_chunk_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
+    }
+    if (!(flags & MDN_CHECK_FINITE)) return MDN_OK;
+
+    const bool bf = in_dtype == MDN_BF16;
+    const size_t nst = nstate * D * D;
+    if ((e = launch_finite_check(a.o, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(a.vt, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(a.S_T, nst, false, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(a.M_T, nst, false, a.status, s))) return mdn::cuda_fail(e);
+    unsigned host_status[3] = {0, 0, 0};
+    if ((e = cudaMemcpyAsync(host_status, a.status, sizeof(host_status), cudaMemcpyDeviceToHost, s)))
+        return mdn::cuda_fail(e);
+    if ((e = cudaStreamSynchronize(s))) return mdn::cuda_fail(e);
+    if (host_status[2]) return MDN_ERR_INVALID_ARG;
+    if (host_status[1]) return MDN_ERR_TIMEOUT;
+    if (host_status[0]) return MDN_ERR_NONFINITE;
+    return MDN_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- CUDA errors
@@ -181,60 +240,123 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     const WsLayout w = ws_layout((long long)B * H, NT, D);
     if (ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
 
-    char* ws = static_cast<char*>(workspace);
     ChunkArgs a;
     a.q = q; a.k = k; a.v = v;
     a.alpha_log = alpha_log; a.mu_log = mu_log; a.beta = beta; a.eta = eta;
     a.dcorr = d_corr; a.S0 = S0; a.M0 = M0;
     a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
     a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
-    a.status = reinterpret_cast<unsigned*>(ws + w.status);
-    a.la = reinterpret_cast<float*>(ws + w.la);
-    a.lm = reinterpret_cast<float*>(ws + w.lm);
-    a.lc = reinterpret_cast<float*>(ws + w.lc);
-    a.bco = reinterpret_cast<float*>(ws + w.bco);
-    a.gamma = reinterpret_cast<float*>(ws + w.gamma);
-    a.U = reinterpret_cast<float*>(ws + w.U);
-    a.Y = reinterpret_cast<float*>(ws + w.Y);
-    a.Z = reinterpret_cast<float*>(ws + w.Z);
-    a.Oi = reinterpret_cast<float*>(ws + w.Oi);
-    a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + w.qhat);
-    a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
-    a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);
-    a.crec = reinterpret_cast<float*>(ws + w.crec);
-    a.ready = reinterpret_cast<unsigned*>(ws + w.ready);
+    carve(a, static_cast<char*>(workspace), w);
+    cudaError_t e;
+    if ((flags & MDN_CHECK_FINITE) && (e = cudaMemsetAsync(a.status, 0, 64, s)))
+        return mdn::cuda_fail(e);
+    return run_pass(a, in_dtype, flags, s, (size_t)B * T * H * D, (size_t)B * H);
+}
+
+// ---------------------------------------------------------------- variable length
+namespace {
+
+struct VarlenLayout {
+    size_t cu_s, cu_c, q, k, v, al, ml, be, et, chunk, total;
+    int NT;  // padded chunks (an upper bound on the sequences' chunk count)
+};
+
+// NT = floor(total_T / C) + N bounds sum_s ceil(len_s / C) for any split of
+// total_T tokens into N sequences.
+mdn_status varlen_layout(int N, int total_T, int H, int dk, int dv, int C, mdn_dtype dt,
+                         VarlenLayout& v)
+{
+    if (N < 0 || total_T < 0 || C <= 0) return MDN_ERR_INVALID_ARG;
+    const long long NT = (long long)total_T / (C > 0 ? C : 1) + N;
+    if (NT * C >= (1LL << 31)) return MDN_ERR_UNSUPPORTED;
+    mdn_status st = check_sizes(1, (int)(NT * C), H, dk, dv, C, dt);
+    if (st != MDN_OK) return st;
+    if ((long long)N * H >= (1LL << 31) / 2) return MDN_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)NT * C * H;  // padded token-heads
+    const size_t elt = dt == MDN_F32 ? 4 : 2;
+    v.NT = (int)NT;
+    size_t off = 0;
+    v.cu_s = off; off += align_up((size_t)(N + 1) * sizeof(int));
+    v.cu_c = off; off += align_up((size_t)(N + 1) * sizeof(int));
+    v.q = off;    off += align_up(rows * dk * elt);
+    v.k = off;    off += align_up(rows * dk * elt);
+    v.v = off;    off += align_up(rows * dv * elt);
+    v.al = off;   off += align_up(rows * sizeof(float));
+    v.ml = off;   off += align_up(rows * sizeof(float));
+    v.be = off;   off += align_up(rows * sizeof(float));
+    v.et = off;   off += align_up(rows * sizeof(float));
+    v.chunk = off;
+    v.total = off + ws_layout(H, v.NT, dk).total;
+    return MDN_OK;
+}
+
+}  // namespace
+
+size_t mdn_chunk_fwd_varlen_workspace_size(int N, int total_T, int H, int dk, int dv, int C,
+                                           mdn_dtype in_dtype)
+{
+    VarlenLayout v;
+    if (varlen_layout(N, total_T, H, dk, dv, C, in_dtype, v) != MDN_OK) return 0;
+    return v.total;
+}
+
+mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                                const float* alpha_log, const float* mu_log, const float* beta,
+                                const float* eta, float d_corr, const int* cu_seqlens, int N,
+                                int total_T, const float* S0, const float* M0, int H, int dk,
+                                int dv, int C, void* o, void* vtilde, float* S_T, float* M_T,
+                                void* workspace, size_t ws_bytes, int flags, mdn_stream_t stream)
+{
+    VarlenLayout L;
+    mdn_status st = varlen_layout(N, total_T, H, dk, dv, C, in_dtype, L);
+    if (st != MDN_OK) return st;
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64))
+        return MDN_ERR_INVALID_ARG;
+    if ((flags & MDN_SLICE32) && (flags & MDN_SLICE64)) return MDN_ERR_INVALID_ARG;
+    if (N == 0 || H == 0) return MDN_OK;
+    if (!cu_seqlens || !aligned4(cu_seqlens)) return MDN_ERR_INVALID_ARG;
+    if (!S_T || !M_T || !aligned16(S_T) || !aligned16(M_T)) return MDN_ERR_INVALID_ARG;
+    if ((S0 && !aligned16(S0)) || (M0 && !aligned16(M0))) return MDN_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        const void* tok[] = {q, k, v, o, vtilde};
+        for (const void* p : tok)
+            if (!p || !aligned16(p)) return MDN_ERR_INVALID_ARG;
+        const void* gates[] = {alpha_log, mu_log, beta, eta};
+        for (const void* p : gates)
+            if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    }
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MDN_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return MDN_ERR_INVALID_ARG;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = dk;
+    char* ws = static_cast<char*>(workspace);
+    int* cu_s = reinterpret_cast<int*>(ws + L.cu_s);
+    int* cu_c = reinterpret_cast<int*>(ws + L.cu_c);
+    ChunkArgs a;
+    a.q = ws + L.q; a.k = ws + L.k; a.v = ws + L.v;
+    a.alpha_log = reinterpret_cast<float*>(ws + L.al);
+    a.mu_log = reinterpret_cast<float*>(ws + L.ml);
+    a.beta = reinterpret_cast<float*>(ws + L.be);
+    a.eta = reinterpret_cast<float*>(ws + L.et);
+    a.dcorr = d_corr; a.S0 = S0; a.M0 = M0;
+    a.B = 1; a.T = L.NT * C; a.H = H; a.D = D; a.NT = L.NT;
+    a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
+    a.cu_seqlens = cu_s; a.cu_chunks = cu_c; a.nseq = N;
+    carve(a, ws + L.chunk, ws_layout(H, L.NT, D));
 
     cudaError_t e;
-    const bool check = flags & MDN_CHECK_FINITE;
-    if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
-    const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
-    if (tensor_cores) {
-        const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
-        if ((e = cudaMemsetAsync(a.ready, 0, ((size_t)B * H * NT + 1) * sizeof(unsigned), s)))
-            return mdn::cuda_fail(e);
-        a.test_no_intra = (flags & MDN_TEST_NO_INTRA) != 0;
-        if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
-    } else {
-        if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
-                                  a.gamma, s)))
-            return mdn::cuda_fail(e);
-        if ((e = launch_chunk_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
-    }
-    if (!check) return MDN_OK;
-
-    const size_t ntok = (size_t)B * T * H * D;
-    const bool bf = in_dtype == MDN_BF16;
-    if ((e = launch_finite_check(o, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
-    if ((e = launch_finite_check(vtilde, ntok, bf, a.status, s))) return mdn::cuda_fail(e);
-    if ((e = launch_finite_check(S_T, (size_t)B * H * D * D, false, a.status, s))) return mdn::cuda_fail(e);
-    if ((e = launch_finite_check(M_T, (size_t)B * H * D * D, false, a.status, s))) return mdn::cuda_fail(e);
-    unsigned host_status[2] = {0, 0};
-    if ((e = cudaMemcpyAsync(host_status, a.status, sizeof(host_status), cudaMemcpyDeviceToHost, s)))
+    if ((e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
+    if ((e = launch_varlen_setup(cu_seqlens, N, total_T, cu_s, cu_c, a.status + 2, s)))
         return mdn::cuda_fail(e);
-    if ((e = cudaStreamSynchronize(s))) return mdn::cuda_fail(e);
-    if (host_status[1]) return MDN_ERR_TIMEOUT;
-    if (host_status[0]) return MDN_ERR_NONFINITE;
-    return MDN_OK;
+    const size_t elt = in_dtype == MDN_F32 ? 4 : 2;
+    if ((e = launch_varlen_gather(q, k, v, elt, alpha_log, mu_log, beta, eta, cu_s, cu_c, N, H, D,
+                                  L.NT, const_cast<void*>(a.q), const_cast<void*>(a.k),
+                                  const_cast<void*>(a.v), const_cast<float*>(a.alpha_log),
+                                  const_cast<float*>(a.mu_log), const_cast<float*>(a.beta),
+                                  const_cast<float*>(a.eta), s)))
+        return mdn::cuda_fail(e);
+    return run_pass(a, in_dtype, flags, s, (size_t)total_T * H * D, (size_t)N * H);
 }
 
 namespace {

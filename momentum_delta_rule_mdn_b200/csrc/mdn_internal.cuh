@@ -86,7 +86,7 @@ struct ChunkArgs {
     float* S_T;
     float* M_T;
     // scratch (workspace)
-    unsigned* status;  // [0]: non-finite flag, [1]: timeout flag
+    unsigned* status;  // [0]: non-finite flag, [1]: timeout flag, [2]: bad cu_seqlens
     float* la;         // [B*H, NT*C]
     float* lm;
     float* lc;
@@ -106,12 +106,96 @@ struct ChunkArgs {
                           //                     alphabar_C, b_C, mubar_C
     bool test_no_intra = false;  // failure-path test: skip the intra-chunk kernel
     float* dbg = nullptr;  // diagnostics: if set, CTA 0 dumps its first chunk's intermediates
+    // Variable-length mode (cu_chunks != null).  q, k, v and the gates are then
+    // the chunk-aligned padded copy, seen as one batch row (B = 1, T = NT*C):
+    // sequence s owns padded chunks [cu_chunks[s], cu_chunks[s+1]) and packed
+    // tokens [cu_seqlens[s], cu_seqlens[s+1]) of o and vt; S0 .. M_T are
+    // [nseq, H, D, D].
+    const int* cu_seqlens = nullptr;
+    const int* cu_chunks = nullptr;
+    int nseq = 0;
 };
+
+// One chain of the sequential pass: a state head and its run of chunks.
+struct Chain {
+    long long sh;      // state head (index into S0 .. M_T, in units of D*D)
+    int b, h;          // batch row and head of the inputs
+    long long chunk0;  // its first chunk in the per-chunk buffers
+    int n0;            // its first chunk in the input rows (token row n0*C of batch row b)
+    int nt;            // chunks in the chain
+    long long out0;    // token row (of o, vt) of its first token
+    int len;           // tokens of the chain written to o, vt
+};
+
+// A: ChunkArgs or a kernel's own argument block with the same fields.
+template <class A>
+__device__ __forceinline__ Chain chain_of(const A& a, long long sh)
+{
+    Chain c;
+    c.sh = sh;
+    c.h = (int)(sh % a.H);
+    if (a.cu_chunks) {
+        const int seq = (int)(sh / a.H);
+        const int c0 = a.cu_chunks[seq];
+        c.b = 0;
+        c.chunk0 = (long long)c.h * a.NT + c0;
+        c.n0 = c0;
+        c.nt = a.cu_chunks[seq + 1] - c0;
+        c.out0 = a.cu_seqlens[seq];
+        c.len = a.cu_seqlens[seq + 1] - a.cu_seqlens[seq];
+    } else {
+        c.b = (int)(sh / a.H);
+        c.chunk0 = sh * a.NT;
+        c.n0 = 0;
+        c.nt = a.NT;
+        c.out0 = (long long)c.b * a.T;
+        c.len = a.T;
+    }
+    return c;
+}
+
+// The sequence that owns padded chunk n (variable-length mode), or -1 for
+// the unused chunks past the last sequence.  Empty sequences own no chunk.
+__device__ __forceinline__ int varlen_seq_of_chunk(const int* cu_chunks, int nseq, int n)
+{
+    if (n >= cu_chunks[nseq]) return -1;
+    int lo = 0, hi = nseq - 1;  // the last s with cu_chunks[s] <= n
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu_chunks[mid] <= n) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Output rows of input chunk n of batch row b: row r (< valid) of the chunk
+// is token row row0 + r of o and vt.
+struct ChunkOut {
+    long long row0;
+    int valid;
+};
+
+__device__ __forceinline__ ChunkOut chunk_out(const ChunkArgs& a, int b, int n)
+{
+    ChunkOut o;
+    int rest;
+    if (a.cu_chunks) {
+        const int seq = varlen_seq_of_chunk(a.cu_chunks, a.nseq, n);
+        if (seq < 0) return ChunkOut{0, 0};
+        const int local0 = (n - a.cu_chunks[seq]) * kChunk;
+        o.row0 = (long long)a.cu_seqlens[seq] + local0;
+        rest = a.cu_seqlens[seq + 1] - a.cu_seqlens[seq] - local0;
+    } else {
+        o.row0 = (long long)b * a.T + (long long)n * kChunk;
+        rest = a.T - n * kChunk;
+    }
+    o.valid = rest < 0 ? 0 : (rest > kChunk ? kChunk : rest);
+    return o;
+}
 
 // Kernel kinds known to the optional timing facility (profile.cu).
 enum KernelKind {
     kGatePrep = 0, kIntraSimt, kInterSimt, kOutputSimt, kStep, kFiniteCheck,
-    kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kKernelKinds
+    kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kVarlen, kKernelKinds
 };
 // Record a start event for a launch of kind k on s (returns a slot, or -1 when
 // timing is off); prof_end records the matching stop event.
@@ -149,5 +233,18 @@ cudaError_t launch_gate_params(const float* x_eta, const float* a, const float* 
                                cudaStream_t s);
 cudaError_t launch_finite_check(const void* x, size_t n, bool bf16, unsigned* flag,
                                 cudaStream_t s);
+// Variable-length mode.  Setup: checks cu_seqlens (N+1 device ints: 0, non-
+// decreasing, ending at total_T), writes the checked copy to cu_s and the
+// chunk offsets to cu_c (N+1 each); an invalid cu_seqlens sets *bad and
+// makes every sequence empty.  Gather: the chunk-aligned padded inputs
+// (NT*C rows; padding rows are steps that change nothing: k = v = q = 0,
+// alpha = mu = 1, beta = eta = 0).
+cudaError_t launch_varlen_setup(const int* cu_seqlens, int N, int total_T, int* cu_s, int* cu_c,
+                                unsigned* bad, cudaStream_t s);
+cudaError_t launch_varlen_gather(const void* q, const void* k, const void* v, size_t elt,
+                                 const float* alpha_log, const float* mu_log, const float* beta,
+                                 const float* eta, const int* cu_s, const int* cu_c, int N, int H,
+                                 int D, int NT, void* qp, void* kp, void* vp, float* alp,
+                                 float* mlp, float* bep, float* etp, cudaStream_t s);
 
 }  // namespace mdn

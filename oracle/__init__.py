@@ -116,6 +116,33 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d, S0=None, M0=None,
     return o, vt, S_T, M_T
 
 
+def chunk_fwd_varlen(q, k, v, alpha_log, mu_log, beta, eta, cu_seqlens, d, S0=None, M0=None,
+                     lib: Optional[ctypes.CDLL] = None):
+    """N sequences packed along the token axis: q, k, v [total_T,H,d], gates
+    [total_T,H], cu_seqlens [N+1] (sequence s = tokens cu[s]:cu[s+1]), S0, M0
+    [N,H,d,d] or None.  The pages run one sequence per batch row; packing is
+    the plain extension, each sequence its own recurrence from its own
+    entering state.  Returns fp64 (o, vtilde, S_T, M_T)."""
+    cu = [int(x) for x in np.asarray(cu_seqlens)]
+    N = len(cu) - 1
+    total_T, H, dk = np.shape(q)
+    dv = np.shape(v)[-1]
+    assert N >= 0 and cu[0] == 0 and cu[-1] == total_T
+    assert all(cu[i] <= cu[i + 1] for i in range(N))
+    o = np.zeros((total_T, H, dv))
+    vt = np.zeros((total_T, H, dv))
+    S_T = np.empty((N, H, dk, dv))
+    M_T = np.empty((N, H, dk, dv))
+    for s in range(N):
+        a, b = cu[s], cu[s + 1]
+        seq = lambda x: np.asarray(x)[a:b][None]
+        st = lambda x: None if x is None else np.asarray(x)[s:s + 1]
+        ro, rvt, rS, rM = chunk_fwd(seq(q), seq(k), seq(v), seq(alpha_log), seq(mu_log),
+                                    seq(beta), seq(eta), d, st(S0), st(M0), lib=lib)
+        o[a:b], vt[a:b], S_T[s], M_T[s] = ro[0], rvt[0], rS[0], rM[0]
+    return o, vt, S_T, M_T
+
+
 def step(q, k, v, alpha_log, mu_log, beta, eta, d, S, M,
          lib: Optional[ctypes.CDLL] = None):
     """One decode token over [B,H,d] inputs.  Returns fp64 (o, vtilde, S_new, M_new);

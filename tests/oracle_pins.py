@@ -14,6 +14,8 @@ Sources ("MDN: Parallelizing Stepwise Momentum for Delta Linear Attention"):
   mu = 0 ablation ....... ijyty.com, section 8 (reduces to a gated delta rule)
   gate parameterisation . summary, step 6; ijyty.com, sections 5 and 8
   ||Delta S_t||_F ........ ijyty.com, section 8 (decoding diagnostic)
+  packed sequences ...... the pages' one-sequence recurrence per sequence (their
+                          silence on packing read as independence)
 """
 from __future__ import annotations
 
@@ -288,6 +290,45 @@ def pin_resume(lib):
     _close(b[2], ref[2], 1e-13, "resume S_T")
 
 
+
+def pin_varlen(lib):
+    """Sequences packed along the token axis: (1) N sequences of one length equal
+    the batched pass with B = N; (2) lengths 0, 1, 5, 13 equal the one-token
+    step run over the packed rows with the state reset to S0[s] at every
+    sequence start; (3) an empty sequence returns its S0, M0."""
+    rng = np.random.default_rng(17)
+    N, L, H, d = 3, 7, 2, 4
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, N, L, H, d)
+    flat = lambda x: x.reshape((N * L,) + x.shape[2:])
+    cu = np.arange(N + 1) * L
+    ref = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0, lib=lib)
+    got = oracle.chunk_fwd_varlen(flat(q), flat(k), flat(v), flat(al), flat(ml), flat(be),
+                                  flat(et), cu, 0.5, S0, M0, lib=lib)
+    for name, g, r in zip(("o", "vtilde"), got[:2], ref[:2]):
+        assert np.array_equal(g, flat(r)), f"varlen equal-length {name}"
+    assert np.array_equal(got[2], ref[2]) and np.array_equal(got[3], ref[3])
+
+    lens = [0, 5, 1, 13, 0]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    Tt, N = int(cu[-1]), len(lens)
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, 1, Tt, H, d)
+    q, k, v, al, ml, be, et = (x[0] for x in (q, k, v, al, ml, be, et))
+    S0 = rng.standard_normal((N, H, d, d))
+    M0 = rng.standard_normal((N, H, d, d))
+    o, vt, S_T, M_T = oracle.chunk_fwd_varlen(q, k, v, al, ml, be, et, cu, 0.5, S0, M0, lib=lib)
+    for s in range(N):
+        S, M = S0[s:s + 1], M0[s:s + 1]
+        for t in range(cu[s], cu[s + 1]):
+            to, tvt, S, M = oracle.step(q[t][None], k[t][None], v[t][None], al[t][None],
+                                        ml[t][None], be[t][None], et[t][None], 0.5, S, M,
+                                        lib=lib)
+            _close(o[t], to[0], 1e-13, f"varlen o seq {s} token {t}")
+            _close(vt[t], tvt[0], 1e-13, f"varlen vtilde seq {s} token {t}")
+        _close(S_T[s], S[0], 1e-13, f"varlen S_T seq {s}")
+        _close(M_T[s], M[0], 1e-13, f"varlen M_T seq {s}")
+        if lens[s] == 0:
+            assert np.array_equal(S_T[s], S0[s]) and np.array_equal(M_T[s], M0[s])
+
 # ---------------------------------------------------------------- gates
 def _logsig(x):
     return -np.logaddexp(0.0, -np.asarray(x, dtype=np.float64))
@@ -355,4 +396,5 @@ def pin_step_delta_norm(lib):
 
 ALL_PINS = [pin_hand_scalar, pin_hand_matrix, pin_closed_form, pin_mu_zero_gated_delta_rule,
             pin_spectrum, pin_chunked_form, pin_chunk_coeffs, pin_step_matches_sequence,
-            pin_resume, pin_gates_special_points, pin_gates_identities, pin_step_delta_norm]
+            pin_resume, pin_varlen, pin_gates_special_points, pin_gates_identities,
+            pin_step_delta_norm]

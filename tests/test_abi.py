@@ -143,3 +143,30 @@ def test_gate_params_and_delta_norm_validation(lib):
     assert dn(ds=FAKE + 1) == E.MDN_ERR_INVALID_ARG
     assert dn(d=32) == E.MDN_ERR_UNSUPPORTED
     assert dn(B=0, ds=None) == E.MDN_OK
+
+
+def test_varlen_workspace_and_validation(lib):
+    E = _lib
+    ws = lib.mdn_chunk_fwd_varlen_workspace_size
+    assert ws(4, 8192, 8, 128, 128, 64, E.MDN_BF16) > 0
+    assert ws(0, 0, 8, 128, 128, 64, E.MDN_BF16) > 0
+    assert ws(-1, 100, 8, 128, 128, 64, E.MDN_BF16) == 0
+    assert ws(2, -5, 8, 128, 128, 64, E.MDN_BF16) == 0
+    assert ws(2, 100, 8, 96, 96, 64, E.MDN_BF16) == 0                  # unsupported d
+    # room for the worst split: every sequence ends one token into a chunk
+    assert ws(5, 640, 1, 64, 64, 64, E.MDN_F32) == ws(10, 320, 1, 64, 64, 64, E.MDN_F32)
+    assert ws(5, 641, 1, 64, 64, 64, E.MDN_F32) == ws(5, 640, 1, 64, 64, 64, E.MDN_F32)
+    need = ws(2, 100, 1, 64, 64, 64, E.MDN_F32)
+
+    def vl(N=2, total=100, cu=FAKE, wsb=need, flags=0, q=FAKE, S_T=FAKE):
+        return lib.mdn_chunk_fwd_varlen(q, FAKE, FAKE, E.MDN_F32, FAKE, FAKE, FAKE, FAKE, 0.5,
+                                        cu, N, total, None, None, 1, 64, 64, 64, FAKE, FAKE,
+                                        S_T, FAKE, FAKE, wsb, flags, None)
+    assert vl(cu=None) == E.MDN_ERR_INVALID_ARG
+    assert vl(cu=FAKE + 2) == E.MDN_ERR_INVALID_ARG
+    assert vl(q=None) == E.MDN_ERR_INVALID_ARG
+    assert vl(S_T=FAKE + 4) == E.MDN_ERR_INVALID_ARG
+    assert vl(wsb=need - 1) == E.MDN_ERR_INVALID_ARG
+    assert vl(flags=E.MDN_TEST_NO_INTRA) == E.MDN_ERR_INVALID_ARG
+    assert vl(N=-1) == E.MDN_ERR_INVALID_ARG
+    assert vl(N=0, cu=None) == E.MDN_OK
