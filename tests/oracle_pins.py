@@ -16,6 +16,8 @@ Sources ("MDN: Parallelizing Stepwise Momentum for Delta Linear Attention"):
   ||Delta S_t||_F ........ ijyty.com, section 8 (decoding diagnostic)
   packed sequences ...... the pages' one-sequence recurrence per sequence (their
                           silence on packing read as independence)
+  gradients ............. summary, step 7; ijyty.com, section 6 (training saves
+                          vtilde, rebuilds S and M in the backward pass)
 """
 from __future__ import annotations
 
@@ -329,6 +331,78 @@ def pin_varlen(lib):
         if lens[s] == 0:
             assert np.array_equal(S_T[s], S0[s]) and np.array_equal(M_T[s], M0[s])
 
+
+# ---------------------------------------------------------------- backward
+def pin_backward_forward_is_the_oracle(lib):
+    """The torch recurrence that the gradient oracle differentiates equals the
+    C oracle's forward pass (o, vtilde, S_T, M_T)."""
+    from oracle import backward as ob
+    import torch
+    rng = np.random.default_rng(31)
+    B, T, H, d = 2, 11, 2, 5
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    ref = oracle.chunk_fwd(q, k, v, al, ml, be, et, 0.5, S0, M0, lib=lib)
+    tt = lambda x: torch.as_tensor(x, dtype=torch.float64)
+    got = ob.forward(*(tt(x) for x in (q, k, v, al, ml, be, et)), 0.5, tt(S0), tt(M0))
+    for name, g, r in zip(("o", "vtilde", "S_T", "M_T"), got, ref):
+        _close(g.numpy(), r, 1e-12, f"torch forward {name}")
+
+
+def pin_backward_finite_differences(lib):
+    """Every gradient entry against a central difference of the loss
+    (h = 1e-6, fp64) on a case with non-zero entering states and all three
+    cotangents."""
+    from oracle import backward as ob
+    rng = np.random.default_rng(32)
+    B, T, H, d = 1, 6, 2, 3
+    q, k, v, al, ml, be, et, S0, M0 = _rand_case(rng, B, T, H, d)
+    do = rng.standard_normal((B, T, H, d))
+    dS = rng.standard_normal((B, H, d, d))
+    dM = rng.standard_normal((B, H, d, d))
+    args = dict(q=q, k=k, v=v, alpha_log=al, mu_log=ml, beta=be, eta=et)
+    g = ob.chunk_bwd(q, k, v, al, ml, be, et, 0.5, S0, M0, do, dS, dM)
+    states = dict(S0=S0, M0=M0)
+    h = 1e-6
+    for name in list(args) + list(states):
+        base = args if name in args else states
+        x = base[name]
+        grad = g["d" + name]
+        assert grad.shape == x.shape, name
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            lp = ob.loss_value(**{**args, **states, name: xp}, d=0.5, do=do, dS_T=dS, dM_T=dM)
+            lm = ob.loss_value(**{**args, **states, name: xm}, d=0.5, do=do, dS_T=dS, dM_T=dM)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def pin_backward_single_token(lib):
+    """One token from zero states: S_1 = beta eta k v^T and o = beta eta (k.qhat) v,
+    so with L = <do, o> + <dS, S_1>: dv = beta eta ((k.qhat) do + dS^T k),
+    dq = beta eta (v.do) k, dk = beta eta ((v.do)(qhat - d k) + dS v),
+    dbeta = eta X, deta = beta X with X = (k.qhat)(v.do) + k^T dS v, and no
+    dependence on alpha or mu (the states they scale are zero)."""
+    from oracle import backward as ob
+    rng = np.random.default_rng(33)
+    d, dc = 4, 0.5
+    q, k, v, do = (rng.standard_normal((1, 1, 1, d)) for _ in range(4))
+    dS = rng.standard_normal((1, 1, d, d))
+    al, ml = np.full((1, 1, 1), -0.3), np.full((1, 1, 1), -0.7)
+    be, et = np.full((1, 1, 1), 0.6), np.full((1, 1, 1), 1.3)
+    g = ob.chunk_bwd(q, k, v, al, ml, be, et, dc, None, None, do, dS, None)
+    kk, vv, qq, oo, SS = k[0, 0, 0], v[0, 0, 0], q[0, 0, 0], do[0, 0, 0], dS[0, 0]
+    qh = qq - dc * kk
+    c, w = 0.6 * 1.3, (kk @ qh) * (vv @ oo) + kk @ SS @ vv
+    _close(g["dv"][0, 0, 0], c * ((kk @ qh) * oo + SS.T @ kk), 1e-13, "1-token dv")
+    _close(g["dq"][0, 0, 0], c * (vv @ oo) * kk, 1e-13, "1-token dq")
+    _close(g["dk"][0, 0, 0], c * ((vv @ oo) * (qh - dc * kk) + SS @ vv), 1e-13, "1-token dk")
+    _close(g["dbeta"][0, 0, 0], 1.3 * w, 1e-13, "1-token dbeta")
+    _close(g["deta"][0, 0, 0], 0.6 * w, 1e-13, "1-token deta")
+    _close(g["dalpha_log"], np.zeros((1, 1, 1)), 1e-15, "1-token dalpha")
+    _close(g["dmu_log"], np.zeros((1, 1, 1)), 1e-15, "1-token dmu")
+
 # ---------------------------------------------------------------- gates
 def _logsig(x):
     return -np.logaddexp(0.0, -np.asarray(x, dtype=np.float64))
@@ -397,4 +471,5 @@ def pin_step_delta_norm(lib):
 ALL_PINS = [pin_hand_scalar, pin_hand_matrix, pin_closed_form, pin_mu_zero_gated_delta_rule,
             pin_spectrum, pin_chunked_form, pin_chunk_coeffs, pin_step_matches_sequence,
             pin_resume, pin_varlen, pin_gates_special_points, pin_gates_identities,
-            pin_step_delta_norm]
+            pin_step_delta_norm, pin_backward_forward_is_the_oracle,
+            pin_backward_finite_differences, pin_backward_single_token]
