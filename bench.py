@@ -241,6 +241,7 @@ def run_ours(args, rank, world, device):
     decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
     gates = None if args.no_decode else run_gate_params(args, mdn, device, hbm, B * T * H)
     varlen = None if args.no_decode else run_varlen(args, mdn, device, spec0)
+    backward = None if args.no_decode else run_backward(args, mdn, device, spec0)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -266,6 +267,8 @@ def run_ours(args, rank, world, device):
         line["gate_params"] = gates
     if varlen:
         line["varlen"] = varlen
+    if backward:
+        line["backward"] = backward
     return line, spec
 
 
@@ -367,6 +370,50 @@ def run_varlen(args, mdn, device, spec0):
     return {"lengths": lens, "tokens": total, "H": H, "d": d, "ms": round(ms, 5),
             "tokens_per_s": round(total / (ms * 1e-3), 1), "calls": n,
             "includes": "checked offsets, chunk-aligned gather, intra + inter kernels"}
+
+
+def run_backward(args, mdn, device, spec0):
+    """mdn_chunk_bwd at the workload's shape from the forward pass's saved
+    vtilde and a random cotangent of o; per-kernel device times from the
+    library's events (a separate pass)."""
+    inp = mi.make_inputs(spec0)
+    dev = mi.to_torch(inp, device)
+    gates = ("alpha_log", "mu_log", "beta", "eta")
+    B, T, H, d = spec0.B, spec0.T, spec0.H, spec0.d
+    o, vt, _, _ = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates),
+                                inp.d_corr)
+    do = torch.randn_like(o)
+    code = 1 if o.dtype == torch.bfloat16 else 0
+    ws = torch.empty(int(mdn.library().mdn_chunk_bwd_workspace_size(B, T, H, d, d, spec0.C, code)),
+                     dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def call():
+        mdn.chunk_bwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), inp.d_corr, vt,
+                      do, workspace=ws)
+    for _ in range(2):
+        call()
+    n = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush.zero_()
+        ev[i][0].record()
+        call()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    mdn.profile_enable(True)
+    mdn.profile_read(reset=True)
+    for _ in range(n):
+        call()
+    torch.cuda.synchronize()
+    kern = mdn.profile_read(reset=True)
+    mdn.profile_enable(False)
+    return {"workload": spec0.name, "ms": round(ms, 4), "tokens_per_s": round(B * T / (ms * 1e-3), 1),
+            "calls": n, "path": "fp32 CUDA cores",
+            "kernels_ms": {k: round(v[0] / v[1], 4) for k, v in kern.items()}}
 
 
 def run_gate_params(args, mdn, device, hbm_peak, workload_n: int):
@@ -580,7 +627,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the side measurements (decode shape, gate kernel, packed sequences)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the side measurements (decode shape, gate kernel, packed sequences, backward)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

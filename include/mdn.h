@@ -147,6 +147,47 @@ mdn_status mdn_chunk_fwd(const void *q, const void *k, const void *v, mdn_dtype 
                          mdn_stream_t stream);
 
 /*
+ * Bytes of device scratch that mdn_chunk_bwd needs, or 0 if the sizes are
+ * invalid or unsupported.  Pure host function.
+ */
+size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    mdn_dtype in_dtype);
+
+/*
+ * The backward pass of mdn_chunk_fwd: gradients of
+ * L = <d_o, o> + <dS_T, S_T> + <dM_T, M_T> with respect to every input.  As
+ * the pages train (summary, step 7; article, section 6), it takes the Vtilde
+ * that the forward pass saved and rebuilds the chunk-entering states from it,
+ * then runs the adjoints of S and M backwards over the chunks and forms every
+ * other gradient chunk by chunk.
+ *
+ *   q .. M0, d_corr   the forward pass's inputs (same layouts and dtypes).
+ *   vtilde      [B,T,H,d] in_dtype: the forward pass's vtilde output.
+ *   d_o         [B,T,H,d] in_dtype: the cotangent of o.
+ *   dS_T, dM_T  [B,H,d,d] fp32 cotangents of S_T, M_T, or NULL (zero).
+ *   dq, dk, dv  [B,T,H,d] fp32 outputs.
+ *   dalpha_log, dmu_log, dbeta, deta  [B,T,H] fp32 outputs.
+ *   dS0, dM0    [B,H,d,d] fp32 outputs (the gradients of the entering states).
+ *   workspace   at least mdn_chunk_bwd_workspace_size(...) bytes, 256-byte
+ *               aligned (about (4 d^2 + 3 C^2 + 10 C) x 4 bytes per chunk of C
+ *               tokens of each head).
+ *   flags       0.
+ *
+ * This build computes the backward pass in fp32 on CUDA cores, for every
+ * supported d and dtype.  Support and errors as mdn_chunk_fwd (T = 0 copies
+ * dS_T, dM_T to dS0, dM0).  Asynchronous on `stream`; enqueues six kernels.
+ */
+mdn_status mdn_chunk_bwd(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                         const float *alpha_log, const float *mu_log,
+                         const float *beta, const float *eta, float d_corr,
+                         const float *S0, const float *M0, const void *vtilde,
+                         const void *d_o, const float *dS_T, const float *dM_T,
+                         int B, int T, int H, int dk, int dv, int C,
+                         float *dq, float *dk_out, float *dv_out, float *dalpha_log,
+                         float *dmu_log, float *dbeta, float *deta, float *dS0, float *dM0,
+                         void *workspace, size_t ws_bytes, int flags, mdn_stream_t stream);
+
+/*
  * Bytes of device scratch that mdn_chunk_fwd_varlen needs, or 0 if the sizes
  * are invalid or unsupported.  Pure host function.
  */

@@ -34,6 +34,10 @@ SIGNATURES = {
                                  _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     "mdn_gate_params": (_i, [_vp, _vp, _vp, _vp, ctypes.c_longlong, _f, _f, _i,
                              _vp, _vp, _vp, _vp, _vp]),
+    "mdn_chunk_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "mdn_chunk_bwd": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp,
+                           _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                           _vp, _vp, _vp, _vp, _sz, _i, _vp]),
     "mdn_chunk_fwd_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "mdn_chunk_fwd_varlen": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _i, _i,
                                   _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i,

@@ -128,6 +128,37 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0
     return o, vt, S_T, M_T
 
 
+def chunk_bwd(q, k, v, alpha_log, mu_log, beta, eta, d: float, vtilde, d_o, S0=None, M0=None,
+              dS_T=None, dM_T=None, C: int = 64, *, workspace: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Backward pass of :func:`chunk_fwd` from its saved ``vtilde``.  Returns a
+    dict of fp32 tensors: dq, dk, dv, dalpha_log, dmu_log, dbeta, deta, dS0, dM0."""
+    B, T, H, D = q.shape
+    code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("vtilde", vtilde), ("d_o", d_o)):
+        _need(t, q.dtype, q.shape, name)
+    for name, t in (("alpha_log", alpha_log), ("mu_log", mu_log), ("beta", beta), ("eta", eta)):
+        _need(t, torch.float32, (B, T, H), name)
+    for name, t in (("S0", S0), ("M0", M0), ("dS_T", dS_T), ("dM_T", dM_T)):
+        _need(t, torch.float32, (B, H, D, D), name)
+    f32 = lambda *s_: torch.empty(s_, dtype=torch.float32, device=q.device)
+    g = dict(dq=f32(B, T, H, D), dk=f32(B, T, H, D), dv=f32(B, T, H, D),
+             dalpha_log=f32(B, T, H), dmu_log=f32(B, T, H), dbeta=f32(B, T, H),
+             deta=f32(B, T, H), dS0=f32(B, H, D, D), dM0=f32(B, H, D, D))
+    lib = library()
+    ws_bytes = int(lib.mdn_chunk_bwd_workspace_size(B, T, H, D, D, C, code))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    status = lib.mdn_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(alpha_log), _ptr(mu_log), _ptr(beta), _ptr(eta),
+        float(d), _ptr(S0), _ptr(M0), _ptr(vtilde), _ptr(d_o), _ptr(dS_T), _ptr(dM_T),
+        B, T, H, D, D, C, *(_ptr(g[n]) for n in ("dq", "dk", "dv", "dalpha_log", "dmu_log",
+                                                  "dbeta", "deta", "dS0", "dM0")),
+        _ptr(workspace), workspace.numel(), 0, _stream_handle(stream))
+    _check(status, "mdn_chunk_bwd")
+    return g
+
+
 def chunk_fwd_varlen(q, k, v, alpha_log, mu_log, beta, eta, cu_seqlens: torch.Tensor,
                      d: float = 0.5, S0=None, M0=None, C: int = 64, *, out=None,
                      workspace: Optional[torch.Tensor] = None, flags: int = 0,

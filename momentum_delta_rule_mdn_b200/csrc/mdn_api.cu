@@ -253,6 +253,110 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     return run_pass(a, in_dtype, flags, s, (size_t)B * T * H * D, (size_t)B * H);
 }
 
+// ---------------------------------------------------------------- backward
+namespace {
+
+struct BwdLayout {
+    size_t la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec, total;
+};
+
+BwdLayout bwd_layout(long long BH, int NT, int D)
+{
+    const size_t chunks = (size_t)BH * NT, rows = chunks * kChunk;
+    BwdLayout w;
+    size_t off = 0;
+    w.la = off;    off += align_up(rows * sizeof(float));
+    w.lm = off;    off += align_up(rows * sizeof(float));
+    w.lc = off;    off += align_up(rows * sizeof(float));
+    w.bco = off;   off += align_up(rows * sizeof(float));
+    w.gamma = off; off += align_up(rows * kChunk * sizeof(float));
+    w.att = off;   off += align_up(rows * kChunk * sizeof(float));
+    w.tmat = off;  off += align_up(rows * kChunk * sizeof(float));
+    w.SS = off;    off += align_up(chunks * 2 * D * D * sizeof(float));
+    w.dSS = off;   off += align_up(chunks * 2 * D * D * sizeof(float));
+    w.rec = off;   off += align_up(chunks * kBwdRec * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    mdn_dtype in_dtype)
+{
+    if (check_sizes(B, T, H, dk, dv, C, in_dtype) != MDN_OK) return 0;
+    return bwd_layout((long long)B * H, (T + C - 1) / C, dk).total;
+}
+
+mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                         const float* alpha_log, const float* mu_log, const float* beta,
+                         const float* eta, float d_corr, const float* S0, const float* M0,
+                         const void* vtilde, const void* d_o, const float* dS_T,
+                         const float* dM_T, int B, int T, int H, int dk, int dv, int C,
+                         float* dq, float* dk_out, float* dv_out, float* dalpha_log,
+                         float* dmu_log, float* dbeta, float* deta, float* dS0, float* dM0,
+                         void* workspace, size_t ws_bytes, int flags, mdn_stream_t stream)
+{
+    mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
+    if (st != MDN_OK) return st;
+    if (flags != 0) return MDN_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return MDN_OK;
+    if (!dS0 || !dM0 || !aligned16(dS0) || !aligned16(dM0)) return MDN_ERR_INVALID_ARG;
+    const void* opt[] = {S0, M0, dS_T, dM_T};
+    for (const void* p : opt)
+        if (p && !aligned16(p)) return MDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = dk;
+    if (T > 0) {
+        const void* tok[] = {q, k, v, vtilde, d_o, dq, dk_out, dv_out};
+        for (const void* p : tok)
+            if (!p || !aligned16(p)) return MDN_ERR_INVALID_ARG;
+        const void* g[] = {alpha_log, mu_log, beta, eta, dalpha_log, dmu_log, dbeta, deta};
+        for (const void* p : g)
+            if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
+    }
+    const int NT = (T + C - 1) / C;
+    const BwdLayout w = bwd_layout((long long)B * H, NT, D);
+    if (T > 0 && (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign))
+        return MDN_ERR_INVALID_ARG;
+    if (T > 0 && ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
+    const size_t state_bytes = (size_t)B * H * D * D * sizeof(float);
+    cudaError_t e;
+    if (T == 0) {  // S_T = S0, M_T = M0: the adjoints pass straight through
+        if (dS_T) e = cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, s);
+        else e = cudaMemsetAsync(dS0, 0, state_bytes, s);
+        if (e == cudaSuccess) {
+            if (dM_T) e = cudaMemcpyAsync(dM0, dM_T, state_bytes, cudaMemcpyDeviceToDevice, s);
+            else e = cudaMemsetAsync(dM0, 0, state_bytes, s);
+        }
+        return cuda_status(e);
+    }
+    char* ws = static_cast<char*>(workspace);
+    BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.vt = vtilde; a.dout = d_o;
+    a.alpha_log = alpha_log; a.mu_log = mu_log; a.beta = beta; a.eta = eta;
+    a.dcorr = d_corr; a.S0 = S0; a.M0 = M0; a.dS_T = dS_T; a.dM_T = dM_T;
+    a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
+    a.la = reinterpret_cast<float*>(ws + w.la);
+    a.lm = reinterpret_cast<float*>(ws + w.lm);
+    a.lc = reinterpret_cast<float*>(ws + w.lc);
+    a.bco = reinterpret_cast<float*>(ws + w.bco);
+    a.gamma = reinterpret_cast<float*>(ws + w.gamma);
+    a.att = reinterpret_cast<float*>(ws + w.att);
+    a.tmat = reinterpret_cast<float*>(ws + w.tmat);
+    a.SS = reinterpret_cast<float*>(ws + w.SS);
+    a.dSS = reinterpret_cast<float*>(ws + w.dSS);
+    a.crec_bw = reinterpret_cast<float*>(ws + w.rec);
+    a.dq = dq; a.dk = dk_out; a.dv = dv_out;
+    a.dalpha_log = dalpha_log; a.dmu_log = dmu_log; a.dbeta = dbeta; a.deta = deta;
+    a.dS0 = dS0; a.dM0 = dM0;
+    if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
+                              a.gamma, s)))
+        return mdn::cuda_fail(e);
+    if ((e = launch_chunk_bwd_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
+    return MDN_OK;
+}
+
 // ---------------------------------------------------------------- variable length
 namespace {
 

@@ -116,6 +116,47 @@ struct ChunkArgs {
     int nseq = 0;
 };
 
+// Everything one mdn_chunk_bwd call needs, with the workspace carved.
+constexpr int kBwdRec = 6 * kChunk;  // floats of the per-chunk coefficient-adjoint record
+struct BwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* vt;    // Vtilde saved by the forward pass
+    const void* dout;  // cotangent of o
+    const float* alpha_log;
+    const float* mu_log;
+    const float* beta;
+    const float* eta;
+    float dcorr;
+    const float* S0;    // may be null
+    const float* M0;
+    const float* dS_T;  // cotangents of S_T, M_T; may be null
+    const float* dM_T;
+    int B, T, H, D, NT;
+    // scratch
+    float* la;       // [B*H, NT*C] chunk coefficients (gate preparation)
+    float* lm;
+    float* lc;
+    float* bco;
+    float* gamma;    // [B*H*NT, C, C]
+    float* att;      // [B*H*NT, C, C]  (Qhat K^T) o Gamma
+    float* tmat;     // [B*H*NT, C, C]  T = (I + A)^{-1}
+    float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk
+    float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk
+    float* crec_bw;  // [B*H*NT, kBwdRec]  coefficient adjoints from the state products
+    // outputs (fp32)
+    float* dq;
+    float* dk;
+    float* dv;
+    float* dalpha_log;
+    float* dmu_log;
+    float* dbeta;
+    float* deta;
+    float* dS0;
+    float* dM0;
+};
+
 // One chain of the sequential pass: a state head and its run of chunks.
 struct Chain {
     long long sh;      // state head (index into S0 .. M_T, in units of D*D)
@@ -195,7 +236,8 @@ __device__ __forceinline__ ChunkOut chunk_out(const ChunkArgs& a, int b, int n)
 // Kernel kinds known to the optional timing facility (profile.cu).
 enum KernelKind {
     kGatePrep = 0, kIntraSimt, kInterSimt, kOutputSimt, kStep, kFiniteCheck,
-    kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kVarlen, kKernelKinds
+    kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kVarlen, kBwdPrep, kBwdStates,
+    kBwdChain, kBwdStateGrads, kBwdLocal, kKernelKinds
 };
 // Record a start event for a launch of kind k on s (returns a slot, or -1 when
 // timing is off); prof_end records the matching stop event.
@@ -213,6 +255,8 @@ cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const 
                              const float* eta, int B, int T, int H, float* la, float* lm,
                              float* lc, float* bco, float* gamma, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
+// The backward pass (fp32, CUDA cores); K-1's outputs must already be in a's scratch.
+cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, mdn_dtype dt, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and

@@ -170,3 +170,25 @@ def test_varlen_workspace_and_validation(lib):
     assert vl(flags=E.MDN_TEST_NO_INTRA) == E.MDN_ERR_INVALID_ARG
     assert vl(N=-1) == E.MDN_ERR_INVALID_ARG
     assert vl(N=0, cu=None) == E.MDN_OK
+
+
+def test_bwd_workspace_and_validation(lib):
+    E = _lib
+    ws = lib.mdn_chunk_bwd_workspace_size
+    assert ws(4, 2048, 8, 128, 128, 64, E.MDN_BF16) > 0
+    assert ws(4, 2048, 8, 96, 96, 64, E.MDN_BF16) == 0
+    assert ws(1, 65, 1, 64, 64, 64, E.MDN_F32) == ws(1, 128, 1, 64, 64, 64, E.MDN_F32)
+    need = ws(1, 100, 1, 64, 64, 64, E.MDN_F32)
+
+    def bw(T=100, flags=0, wsb=need, dq=FAKE, vt=FAKE, dS0=FAKE, dST=None, gate=FAKE):
+        return lib.mdn_chunk_bwd(FAKE, FAKE, FAKE, E.MDN_F32, gate, FAKE, FAKE, FAKE, 0.5, None,
+                                 None, vt, FAKE, dST, None, 1, T, 1, 64, 64, 64, dq, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, FAKE, dS0, FAKE, FAKE, wsb, flags, None)
+    assert bw(flags=1) == E.MDN_ERR_INVALID_ARG
+    assert bw(vt=None) == E.MDN_ERR_INVALID_ARG
+    assert bw(dq=FAKE + 4) == E.MDN_ERR_INVALID_ARG
+    assert bw(dS0=None) == E.MDN_ERR_INVALID_ARG
+    assert bw(dST=FAKE + 8) == E.MDN_ERR_INVALID_ARG
+    assert bw(gate=FAKE + 2) == E.MDN_ERR_INVALID_ARG
+    assert bw(wsb=need - 1) == E.MDN_ERR_INVALID_ARG
+    assert bw(T=-1) == E.MDN_ERR_INVALID_ARG
