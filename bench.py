@@ -238,10 +238,11 @@ def run_ours(args, rank, world, device):
 
     # ---- end to end through the public call, host (pinned) buffers
     e2e = None if args.no_e2e else run_e2e(args, mdn, inp, tok, spec, device, world)
-    decode = None if args.no_decode else run_decode(args, mdn, device, hbm)
-    gates = None if args.no_decode else run_gate_params(args, mdn, device, hbm, B * T * H)
-    varlen = None if args.no_decode else run_varlen(args, mdn, device, spec0)
-    backward = None if args.no_decode else run_backward(args, mdn, device, spec0)
+    side = set() if args.no_decode else set(args.side.split(","))
+    decode = run_decode(args, mdn, device, hbm) if "decode" in side else None
+    gates = run_gate_params(args, mdn, device, hbm, B * T * H) if "gates" in side else None
+    varlen = run_varlen(args, mdn, device, spec0) if "varlen" in side else None
+    backward = run_backward(args, mdn, device, spec0) if "backward" in side else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -627,7 +628,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the side measurements (decode shape, gate kernel, packed sequences, backward)")
+    ap.add_argument("--no-decode", action="store_true", help="skip every side measurement")
+    ap.add_argument("--side", default="decode,gates,varlen,backward",
+                    help="side measurements after the timed step (comma list of decode, gates, "
+                         "varlen, backward)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
