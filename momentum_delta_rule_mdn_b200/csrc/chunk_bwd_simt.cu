@@ -79,35 +79,60 @@ bwd_prep_kernel(BwdArgs a)
     __syncthreads();
     const float* G = a.gamma + chunk * C * C;
     float* att = a.att + chunk * C * C;
-    for (int idx = tid; idx < C * C; idx += 256) {
-        const int r = idx / C, i = idx % C;
-        float av = 0.f, tv = 0.f;
-        if (i <= r) {
-            float kk = 0.f, qk = 0.f;
-#pragma unroll 8
-            for (int c = 0; c < D; ++c) {
-                const float ki = Ks[i * KS + c];
-                kk = fmaf(Ks[r * KS + c], ki, kk);
-                qk = fmaf(Qs[r * KS + c], ki, qk);
+    {
+        // K K^T and Qhat K^T over 4 x 4 register tiles: rows rg + 16 u, columns ig + 16 v
+        const int rg = tid >> 4, ig = tid & 15;
+        float kk[4][4], qk[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) kk[u][v] = qk[u][v] = 0.f;
+        for (int c = 0; c < D; ++c) {
+            float rk[4], rq[4], ik[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                rk[u] = Ks[(rg + 16 * u) * KS + c];
+                rq[u] = Qs[(rg + 16 * u) * KS + c];
             }
-            tv = qk * G[r * C + i];
-            if (i < r) av = alpha_s[r] * kk * G[(r - 1) * C + i];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) ik[v] = Ks[(ig + 16 * v) * KS + c];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    kk[u][v] = fmaf(rk[u], ik[v], kk[u][v]);
+                    qk[u][v] = fmaf(rq[u], ik[v], qk[u][v]);
+                }
         }
-        As[r * AS + i] = av;
-        att[idx] = tv;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int r = rg + 16 * u, i = ig + 16 * v;
+                float av = 0.f, tv = 0.f;
+                if (i <= r) {
+                    tv = qk[u][v] * G[r * C + i];
+                    if (i < r) av = alpha_s[r] * kk[u][v] * G[(r - 1) * C + i];
+                }
+                As[r * AS + i] = av;
+                att[r * C + i] = tv;
+            }
     }
     __syncthreads();
-    // unit lower-triangular inverse by forward substitution, one column per thread
-    if (tid < C) {
-        const int c = tid;
-        for (int r = 0; r < C; ++r) {
-            float s = 0.f;
-            if (r == c) {
-                s = 1.f;
-            } else if (r > c) {
-                for (int i = c; i < r; ++i) s = fmaf(-As[r * AS + i], Ts[i * AS + c], s);
-            }
-            Ts[r * AS + c] = s;
+    // unit lower-triangular inverse by forward substitution: column c on the
+    // four lanes 4c .. 4c + 3, each summing every fourth term
+    {
+        const int c = tid >> 2, part = tid & 3;
+        if (part == 0) Ts[c] = (c == 0) ? 1.f : 0.f;  // row 0
+        __syncwarp();
+        for (int r = 1; r < C; ++r) {
+            float acc = 0.f;
+            if (r > c)
+                for (int i = c + part; i < r; i += 4) acc = fmaf(As[r * AS + i], Ts[i * AS + c], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (part == 0) Ts[r * AS + c] = (r == c) ? 1.f : (r > c ? -acc : 0.f);
+            __syncwarp();
         }
     }
     __syncthreads();
@@ -172,18 +197,25 @@ bwd_states_kernel(BwdArgs a)
             }
         }
         __syncthreads();
-#pragma unroll 4
+        float dS[EPT], dM[EPT];
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) dS[e] = dM[e] = 0.f;
+        for (int r = 0; r < C; ++r) {
+            const float v = Vs[r * VS + j];
+            const float vg = v * gl[r], vw = v * wv[r];
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) {
+                const float kv = Ks[r * KS + rg + 8 * e];  // one word per warp: a broadcast
+                dS[e] = fmaf(kv, vg, dS[e]);
+                dM[e] = fmaf(kv, vw, dM[e]);
+            }
+        }
+#pragma unroll
         for (int e = 0; e < EPT; ++e) {
             const int i = rg + 8 * e;
-            float dS = 0.f, dM = 0.f;
-            for (int r = 0; r < C; ++r) {
-                const float kv = Ks[r * KS + i] * Vs[r * VS + j];
-                dS = fmaf(kv, gl[r], dS);
-                dM = fmaf(kv, wv[r], dM);
-            }
             const float s = Ss[i * NS + j], m = Ms[i * NS + j];
-            Ss[i * NS + j] = scal[0] * s - scal[1] * m + dS;
-            Ms[i * NS + j] = scal[2] * m - dM;
+            Ss[i * NS + j] = scal[0] * s - scal[1] * m + dS[e];
+            Ms[i * NS + j] = scal[2] * m - dM[e];
         }
     }
 }
@@ -271,26 +303,39 @@ bwd_chain_kernel(BwdArgs a)
         }
         __syncthreads();
         // dVtilde = Att^T dO + Gamma_C o (K dS) - w o (K dM)
+        {
+            float kds[RPT], kdm[RPT], ad[RPT];
 #pragma unroll
-        for (int e = 0; e < RPT; ++e) {
-            const int r = rg + 8 * e;
-            float kds = 0.f, kdm = 0.f, ad = 0.f;
+            for (int e = 0; e < RPT; ++e) kds[e] = kdm[e] = ad[e] = 0.f;
             for (int i = 0; i < D; ++i) {
-                const float kv = Ks[r * KS + i];
-                kds = fmaf(kv, dSs[i * NS + j], kds);
-                kdm = fmaf(kv, dMs[i * NS + j], kdm);
+                const float ds = dSs[i * NS + j], dm = dMs[i * NS + j];
+#pragma unroll
+                for (int e = 0; e < RPT; ++e) {
+                    const float kv = Ks[(rg + 8 * e) * KS + i];
+                    kds[e] = fmaf(kv, ds, kds[e]);
+                    kdm[e] = fmaf(kv, dm, kdm[e]);
+                }
             }
-            for (int r2 = r; r2 < C; ++r2) ad = fmaf(Att[r2 * AS + r], dOs[r2 * VS + j], ad);
-            X[r * VS + j] = ad + gl[r] * kds - wv[r] * kdm;
+            // Att is lower triangular (zeros above the diagonal): full sums are exact
+            for (int r2 = rg; r2 < C; ++r2) {
+                const float od = dOs[r2 * VS + j];
+#pragma unroll
+                for (int e = 0; e < RPT; ++e) ad[e] = fmaf(Att[r2 * AS + rg + 8 * e], od, ad[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < RPT; ++e) {
+                const int r = rg + 8 * e;
+                X[r * VS + j] = ad[e] + gl[r] * kds[e] - wv[r] * kdm[e];
+            }
         }
         __syncthreads();
         float dy[RPT];
 #pragma unroll
-        for (int e = 0; e < RPT; ++e) {
-            const int r = rg + 8 * e;
-            float s = 0.f;
-            for (int r2 = r; r2 < C; ++r2) s = fmaf(Tm[r2 * AS + r], X[r2 * VS + j], s);
-            dy[e] = s;
+        for (int e = 0; e < RPT; ++e) dy[e] = 0.f;
+        for (int r2 = rg; r2 < C; ++r2) {  // T lower triangular as well
+            const float xv = X[r2 * VS + j];
+#pragma unroll
+            for (int e = 0; e < RPT; ++e) dy[e] = fmaf(Tm[r2 * AS + rg + 8 * e], xv, dy[e]);
         }
         __syncthreads();
 #pragma unroll
@@ -301,21 +346,27 @@ bwd_chain_kernel(BwdArgs a)
         }
         __syncthreads();
         const float aC = scal[0], bC = scal[1], mC = scal[2];
-#pragma unroll 4
+        float us[EPT], um[EPT];  // qhat^T (.) dO - K^T (.) dY terms of dS and dM
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) us[e] = um[e] = 0.f;
+        for (int r = 0; r < C; ++r) {
+            const float od = dOs[r * VS + j], xd = X[r * VS + j];
+            const float ab = abar[r];
+            const float qa = od * ab, qb = od * bco[r], xa = xd * ab, x2 = xd * d2[r];
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) {
+                const int i = rg + 8 * e;
+                const float qv = Qs[r * KS + i], kv = Ks[r * KS + i];
+                us[e] = fmaf(qv, qa, fmaf(-kv, xa, us[e]));
+                um[e] = fmaf(kv, x2, fmaf(-qv, qb, um[e]));
+            }
+        }
+#pragma unroll
         for (int e = 0; e < EPT; ++e) {
             const int i = rg + 8 * e;
-            float qs = 0.f, qm = 0.f, ks = 0.f, km = 0.f;
-            for (int r = 0; r < C; ++r) {
-                const float qd = Qs[r * KS + i] * dOs[r * VS + j];
-                const float kd = Ks[r * KS + i] * X[r * VS + j];
-                qs = fmaf(qd, abar[r], qs);
-                qm = fmaf(qd, bco[r], qm);
-                ks = fmaf(kd, abar[r], ks);
-                km = fmaf(kd, d2[r], km);
-            }
             const float ds = dSs[i * NS + j], dm = dMs[i * NS + j];
-            dSs[i * NS + j] = aC * ds + qs - ks;
-            dMs[i * NS + j] = -bC * ds + mC * dm - qm + km;
+            dSs[i * NS + j] = aC * ds + us[e];
+            dMs[i * NS + j] = -bC * ds + mC * dm + um[e];
         }
     }
     __syncthreads();
@@ -329,10 +380,11 @@ bwd_chain_kernel(BwdArgs a)
 // ------------------------------------------------------------------ B-3a
 // Products with the entering states S, M and the leaving adjoints dS, dM:
 // P1 = dO S^T, P2 = dO M^T, P3 = Vt dS^T, P4 = Vt dM^T, P5 = dY S^T,
-// P6 = dY M^T (C x d_k each), streamed over panels of KP rows of d_k.
-// Writes dq's and dk's parts from them, and per chunk the coefficient
-// adjoints they carry (row sums) plus <S,dS>, <M,dS>, <M,dM>.
-constexpr int KP = 16;
+// P6 = dY M^T (C x d_k each), streamed over panels of KP rows of d_k; a
+// thread holds 2 rows x 4 columns of all six.  Writes dq's and dk's parts
+// from them, and per chunk the coefficient adjoints they carry (row sums)
+// plus <S,dS>, <M,dS>, <M,dM>.
+constexpr int KP = 32;
 
 template <typename Tin, int D>
 __global__ void __launch_bounds__(256)
@@ -386,15 +438,25 @@ bwd_state_grads_kernel(BwdArgs a)
         red[warp * 3 + 1] = s2;
         red[warp * 3 + 2] = s3;
     }
-    const int r = tid >> 2, q4 = tid & 3;  // row of the chunk; k = k0 + q4 + 4m
-    const int t = n * C + r;
-    const float abar = expf(a.la[crow + r]), bco = a.bco[crow + r];
-    const float al = t < a.T ? expf(a.alpha_log[tok_idx(a, b, t, h)]) : 1.f;
-    const float d2 = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
-    const float gl = a.gamma[chunk * C * C + (C - 1) * C + r];
-    const float et = t < a.T ? a.eta[tok_idx(a, b, t, h)] : 0.f;
-    const float w = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
-    float sa = 0.f, sb = 0.f, sd2 = 0.f, sgl = 0.f, sw = 0.f;
+    const int rp = tid >> 3, kq = tid & 7;  // rows 2 rp, 2 rp + 1; k = k0 + kq + 8 m
+    float abar[2], bco[2], d2[2], gl[2], w[2];
+    bool in[2];
+    size_t gt[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int r = 2 * rp + u, t = n * C + r;
+        in[u] = t < a.T;
+        gt[u] = in[u] ? tok_idx(a, b, t, h) : 0;
+        abar[u] = expf(a.la[crow + r]);
+        bco[u] = a.bco[crow + r];
+        const float al = in[u] ? expf(a.alpha_log[gt[u]]) : 1.f;
+        d2[u] = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
+        gl[u] = a.gamma[chunk * C * C + (C - 1) * C + r];
+        const float et = in[u] ? a.eta[gt[u]] : 0.f;
+        w[u] = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
+    }
+    float sa[2] = {0.f, 0.f}, sb[2] = {0.f, 0.f}, sd2[2] = {0.f, 0.f}, sgl[2] = {0.f, 0.f},
+          sw[2] = {0.f, 0.f};
     for (int k0 = 0; k0 < D; k0 += KP) {
         __syncthreads();
         for (int idx = tid; idx < KP * D; idx += 256) {
@@ -406,67 +468,87 @@ bwd_state_grads_kernel(BwdArgs a)
             Pn[3 * KP * TS + kk * TS + c] = dMn[g];
         }
         __syncthreads();
-        float p[6][KP / 4];
+        float p[6][2][4];
 #pragma unroll
-        for (int m = 0; m < KP / 4; ++m)
+        for (int x = 0; x < 6; ++x)
 #pragma unroll
-            for (int u = 0; u < 6; ++u) p[u][m] = 0.f;
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) p[x][u][m] = 0.f;
         for (int c = 0; c < D; ++c) {
-            const float o = dOs[r * TS + c], vv = Vts[r * TS + c], y = dYs[r * TS + c];
+            float o[2], vv[2], y[2];
 #pragma unroll
-            for (int m = 0; m < KP / 4; ++m) {
-                const int kk = q4 + 4 * m;
+            for (int u = 0; u < 2; ++u) {
+                o[u] = dOs[(2 * rp + u) * TS + c];
+                vv[u] = Vts[(2 * rp + u) * TS + c];
+                y[u] = dYs[(2 * rp + u) * TS + c];
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int kk = kq + 8 * m;
                 const float sv = Pn[kk * TS + c], mv = Pn[KP * TS + kk * TS + c];
                 const float dsv = Pn[2 * KP * TS + kk * TS + c];
                 const float dmv = Pn[3 * KP * TS + kk * TS + c];
-                p[0][m] = fmaf(o, sv, p[0][m]);
-                p[1][m] = fmaf(o, mv, p[1][m]);
-                p[2][m] = fmaf(vv, dsv, p[2][m]);
-                p[3][m] = fmaf(vv, dmv, p[3][m]);
-                p[4][m] = fmaf(y, sv, p[4][m]);
-                p[5][m] = fmaf(y, mv, p[5][m]);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    p[0][u][m] = fmaf(o[u], sv, p[0][u][m]);
+                    p[1][u][m] = fmaf(o[u], mv, p[1][u][m]);
+                    p[2][u][m] = fmaf(vv[u], dsv, p[2][u][m]);
+                    p[3][u][m] = fmaf(vv[u], dmv, p[3][u][m]);
+                    p[4][u][m] = fmaf(y[u], sv, p[4][u][m]);
+                    p[5][u][m] = fmaf(y[u], mv, p[5][u][m]);
+                }
             }
         }
-        if (t < a.T) {
 #pragma unroll
-            for (int m = 0; m < KP / 4; ++m) {
-                const int k = k0 + q4 + 4 * m;
-                const size_t g = tok_idx(a, b, t, h) * D + k;
+        for (int u = 0; u < 2; ++u) {
+            if (!in[u]) continue;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int k = k0 + kq + 8 * m;
+                const size_t g = gt[u] * D + k;
                 const float kv = ldt<Tin>(a.k, g);
                 const float qh = ldt<Tin>(a.q, g) - a.dcorr * kv;
-                a.dq[g] = abar * p[0][m] - bco * p[1][m];
-                a.dk[g] = gl * p[2][m] - w * p[3][m] - abar * p[4][m] + d2 * p[5][m];
-                sa = fmaf(qh, p[0][m], sa);
-                sa = fmaf(-kv, p[4][m], sa);
-                sb = fmaf(-qh, p[1][m], sb);
-                sd2 = fmaf(kv, p[5][m], sd2);
-                sgl = fmaf(kv, p[2][m], sgl);
-                sw = fmaf(-kv, p[3][m], sw);
+                a.dq[g] = abar[u] * p[0][u][m] - bco[u] * p[1][u][m];
+                a.dk[g] = gl[u] * p[2][u][m] - w[u] * p[3][u][m] - abar[u] * p[4][u][m] +
+                          d2[u] * p[5][u][m];
+                sa[u] = fmaf(qh, p[0][u][m], fmaf(-kv, p[4][u][m], sa[u]));
+                sb[u] = fmaf(-qh, p[1][u][m], sb[u]);
+                sd2[u] = fmaf(kv, p[5][u][m], sd2[u]);
+                sgl[u] = fmaf(kv, p[2][u][m], sgl[u]);
+                sw[u] = fmaf(-kv, p[3][u][m], sw[u]);
             }
         }
     }
-    // the four threads of a row hold its partial sums
+    // the eight threads of a row pair hold its partial sums
 #pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-        sa += __shfl_xor_sync(0xffffffffu, sa, off);
-        sb += __shfl_xor_sync(0xffffffffu, sb, off);
-        sd2 += __shfl_xor_sync(0xffffffffu, sd2, off);
-        sgl += __shfl_xor_sync(0xffffffffu, sgl, off);
-        sw += __shfl_xor_sync(0xffffffffu, sw, off);
+    for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            sa[u] += __shfl_xor_sync(0xffffffffu, sa[u], off);
+            sb[u] += __shfl_xor_sync(0xffffffffu, sb[u], off);
+            sd2[u] += __shfl_xor_sync(0xffffffffu, sd2[u], off);
+            sgl[u] += __shfl_xor_sync(0xffffffffu, sgl[u], off);
+            sw[u] += __shfl_xor_sync(0xffffffffu, sw[u], off);
+        }
     }
     float* rec = a.crec_bw + chunk * kBwdRec;
-    if (q4 == 0) {
-        rec[r] = sa;
-        rec[C + r] = sb;
-        rec[2 * C + r] = sd2;
-        rec[3 * C + r] = sgl;
-        rec[4 * C + r] = sw;
+    if (kq == 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = 2 * rp + u;
+            rec[r] = sa[u];
+            rec[C + r] = sb[u];
+            rec[2 * C + r] = sd2[u];
+            rec[3 * C + r] = sgl[u];
+            rec[4 * C + r] = sw[u];
+        }
     }
     __syncthreads();
     if (tid < 3) {
-        float s = 0.f;
-        for (int w8 = 0; w8 < 8; ++w8) s += red[w8 * 3 + tid];
-        rec[5 * C + tid] = s;
+        float acc = 0.f;
+        for (int w8 = 0; w8 < 8; ++w8) acc += red[w8 * 3 + tid];
+        rec[5 * C + tid] = acc;
     }
 }
 
@@ -545,79 +627,129 @@ bwd_local_grads_kernel(BwdArgs a)
             }
         }
     }
-    // the four C x C products, 16 entries per thread
-    constexpr int EC = C * C / 256;
-    float dov[EC], qk[EC], dyv[EC], kk[EC];
+    // the four C x C products over 4 x 4 register tiles: rows rg + 16 u, columns ig + 16 v
+    const int rg = tid >> 4, ig = tid & 15;
+    float dov[4][4], qk[4][4], dyv[4][4], kk[4][4];
 #pragma unroll
-    for (int e = 0; e < EC; ++e) {
-        const int idx = tid + 256 * e, r = idx / C, i = idx % C;
-        float x1 = 0.f, x2 = 0.f, x3 = 0.f, x4 = 0.f;
-        if (i <= r) {
-#pragma unroll 4
-            for (int c = 0; c < D; ++c) {
-                const float vi = Vts[i * TS + c], ki = Ks[i * TS + c];
-                x1 = fmaf(dOs[r * TS + c], vi, x1);
-                x2 = fmaf(Qs[r * TS + c], ki, x2);
-                x3 = fmaf(dYs[r * TS + c], vi, x3);
-                x4 = fmaf(Ks[r * TS + c], ki, x4);
-            }
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dov[u][v] = qk[u][v] = dyv[u][v] = kk[u][v] = 0.f;
+    for (int c = 0; c < D; ++c) {
+        float ro[4], rq[4], ry[4], rk[4], iv[4], ik[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = rg + 16 * u;
+            ro[u] = dOs[r * TS + c];
+            rq[u] = Qs[r * TS + c];
+            ry[u] = dYs[r * TS + c];
+            rk[u] = Ks[r * TS + c];
         }
-        dov[e] = x1;
-        qk[e] = x2;
-        dyv[e] = x3;
-        kk[e] = x4;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int i = ig + 16 * v;
+            iv[v] = Vts[i * TS + c];
+            ik[v] = Ks[i * TS + c];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                dov[u][v] = fmaf(ro[u], iv[v], dov[u][v]);
+                qk[u][v] = fmaf(rq[u], ik[v], qk[u][v]);
+                dyv[u][v] = fmaf(ry[u], iv[v], dyv[u][v]);
+                kk[u][v] = fmaf(rk[u], ik[v], kk[u][v]);
+            }
     }
     __syncthreads();  // dO and dY tiles are no longer read; Gp is complete
     float* dOVG = dOs;  // [C][C+1]
     float* dPK = dYs;   // [C][C+1]
 #pragma unroll
-    for (int e = 0; e < EC; ++e) {
-        const int idx = tid + 256 * e, r = idx / C, i = idx % C;
-        const float g = v_et[i] * Gp[r * AS + i];
-        float ovg = 0.f, pk = 0.f, dg = 0.f;
-        if (i <= r) {
-            ovg = dov[e] * g;
-            dg = dov[e] * qk[e];
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int r = rg + 16 * u, i = ig + 16 * v;
+            const float g = v_et[i] * Gp[r * AS + i];
+            float ovg = 0.f, pk = 0.f, dg = 0.f;
+            if (i <= r) {
+                ovg = dov[u][v] * g;
+                dg = dov[u][v] * qk[u][v];
+            }
+            if (i < r) pk = -dyv[u][v] * v_et[i] * Gp[(r - 1) * AS + i];  // dA o Gamma-
+            dOVG[r * AS + i] = ovg;
+            dPK[r * AS + i] = pk;
+            dG[r * AS + i] = dg;
         }
-        if (i < r) pk = -dyv[e] * v_et[i] * Gp[(r - 1) * AS + i];  // dA o Gamma-
-        dOVG[r * AS + i] = ovg;
-        dPK[r * AS + i] = pk;
-        dG[r * AS + i] = dg;
-    }
     __syncthreads();
     // Gamma-_{r,i} = Gamma_{r-1,i}: dA o (P K^T) lands on row r - 1 (one writer per entry)
 #pragma unroll
-    for (int e = 0; e < EC; ++e) {
-        const int idx = tid + 256 * e, r = idx / C, i = idx % C;
-        if (i < r) dG[(r - 1) * AS + i] += -dyv[e] * v_al[r] * kk[e];
-    }
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int r = rg + 16 * u, i = ig + 16 * v;
+            if (i < r) dG[(r - 1) * AS + i] += -dyv[u][v] * v_al[r] * kk[u][v];
+        }
     const float* rec = a.crec_bw + chunk * kBwdRec;
     __syncthreads();
     if (tid < C) dG[(C - 1) * AS + tid] += rec[3 * C + tid];  // Gamma_{C,i} in the state update
-    // dQhat += dOVG K ; dK += dOVG^T Qhat + dPK^T P + Diag(alpha) dPK K ; d alpha from P
+    // dQhat += dOVG K ; dK += dOVG^T Qhat + dPK^T P + Diag(alpha) dPK K ; d alpha from P.
+    // A thread holds rows 2 rp, 2 rp + 1 and columns cg + 8 m.  dOVG and dPK are
+    // stored with zeros outside their triangles, so full-range sums are exact.
     {
-        const int r = tid >> 2, q4 = tid & 3, t = n * C + r;
-        const float alr = v_al[r];
-        float dar = 0.f;
-        for (int c = q4; c < D; c += 4) {
-            float dq = 0.f, dk = 0.f, dp = 0.f;
-            for (int i = 0; i <= r; ++i) dq = fmaf(dOVG[r * AS + i], Ks[i * TS + c], dq);
-            for (int r2 = r; r2 < C; ++r2) dk = fmaf(dOVG[r2 * AS + r], Qs[r2 * TS + c], dk);
-            for (int r2 = r + 1; r2 < C; ++r2)
-                dk = fmaf(dPK[r2 * AS + r] * v_al[r2], Ks[r2 * TS + c], dk);
-            for (int i = 0; i < r; ++i) dp = fmaf(dPK[r * AS + i], Ks[i * TS + c], dp);
-            dk = fmaf(alr, dp, dk);
-            dar = fmaf(dp, Ks[r * TS + c], dar);
-            if (t < a.T) {
-                const size_t g = tok_idx(a, b, t, h) * D + c;
-                const float dqt = a.dq[g] + dq;
-                a.dq[g] = dqt;
-                a.dk[g] = a.dk[g] + dk - a.dcorr * dqt;
+        constexpr int NM = D / 8;
+        const int rp = tid >> 3, cg = tid & 7;
+        float dq[2][NM], dp[2][NM];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int m = 0; m < NM; ++m) dq[u][m] = dp[u][m] = 0.f;
+        for (int i = 0; i <= 2 * rp + 1; ++i) {
+            const float g0 = dOVG[(2 * rp) * AS + i], g1 = dOVG[(2 * rp + 1) * AS + i];
+            const float p0 = dPK[(2 * rp) * AS + i], p1 = dPK[(2 * rp + 1) * AS + i];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const float kv = Ks[i * TS + cg + 8 * m];
+                dq[0][m] = fmaf(g0, kv, dq[0][m]);
+                dq[1][m] = fmaf(g1, kv, dq[1][m]);
+                dp[0][m] = fmaf(p0, kv, dp[0][m]);
+                dp[1][m] = fmaf(p1, kv, dp[1][m]);
             }
         }
-        dar += __shfl_xor_sync(0xffffffffu, dar, 1);
-        dar += __shfl_xor_sync(0xffffffffu, dar, 2);
-        if (q4 == 0) v_da[r] = dar;
+        float dk[2][NM];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int m = 0; m < NM; ++m) dk[u][m] = 0.f;
+        for (int r2 = 2 * rp; r2 < C; ++r2) {
+            const float al2 = v_al[r2];
+            const float g0 = dOVG[r2 * AS + 2 * rp], g1 = dOVG[r2 * AS + 2 * rp + 1];
+            const float p0 = dPK[r2 * AS + 2 * rp] * al2, p1 = dPK[r2 * AS + 2 * rp + 1] * al2;
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const float qv = Qs[r2 * TS + cg + 8 * m], kv = Ks[r2 * TS + cg + 8 * m];
+                dk[0][m] = fmaf(g0, qv, fmaf(p0, kv, dk[0][m]));
+                dk[1][m] = fmaf(g1, qv, fmaf(p1, kv, dk[1][m]));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = 2 * rp + u, t = n * C + r;
+            const float alr = v_al[r];
+            float dar = 0.f;
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const int c = cg + 8 * m;
+                dar = fmaf(dp[u][m], Ks[r * TS + c], dar);
+                if (t < a.T) {
+                    const size_t g = tok_idx(a, b, t, h) * D + c;
+                    const float dqt = a.dq[g] + dq[u][m];
+                    a.dq[g] = dqt;
+                    a.dk[g] = a.dk[g] + fmaf(alr, dp[u][m], dk[u][m]) - a.dcorr * dqt;
+                }
+            }
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) dar += __shfl_xor_sync(0xffffffffu, dar, off);
+            if (cg == 0) v_da[r] = dar;
+        }
     }
     __syncthreads();
     // coefficient adjoints -> la, lm, beta, eta, alpha
