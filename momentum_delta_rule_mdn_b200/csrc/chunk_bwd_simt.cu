@@ -849,6 +849,22 @@ bwd_local_grads_kernel(BwdArgs a)
     }
 }
 
+// A non-blocking stream of the current device for work forked off a call's
+// stream, created on first use by each host thread and kept.
+cudaError_t side_stream(cudaStream_t* out)
+{
+    thread_local cudaStream_t streams[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!streams[dev] &&
+        (e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking)) != cudaSuccess)
+        return e;
+    *out = streams[dev];
+    return cudaSuccess;
+}
+
 template <typename Tin, int D>
 cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
 {
@@ -871,14 +887,32 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     MDN_SET_SMEM((bwd_state_grads_kernel<Tin, D>), sm3a)
     MDN_SET_SMEM((bwd_local_grads_kernel<Tin, D>), sm3b)
 #undef MDN_SET_SMEM
+    // The state rebuild depends only on the chunk coefficients and is needed
+    // only by B-3a: it runs on a side stream, beside B-0 and the reverse chain
+    // (both chains leave most of each SM idle), and joins before B-3a.
+    cudaStream_t side;
+    if ((e = side_stream(&side))) return e;
+    cudaEvent_t fork, join;
+    if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming))) return e;
+    if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming))) {
+        cudaEventDestroy(fork);
+        return e;
+    }
+    // released once the device is done with them
+    struct Events {
+        cudaEvent_t a, b;
+        ~Events() { cudaEventDestroy(a); cudaEventDestroy(b); }
+    } ev{fork, join};
+    if ((e = cudaEventRecord(fork, s)) || (e = cudaStreamWaitEvent(side, fork, 0))) return e;
+    {
+        ProfScope ps(kBwdStates, side);
+        bwd_states_kernel<Tin, D><<<(unsigned)chains, 256, sm1, side>>>(a);
+    }
+    if ((e = cudaGetLastError())) return e;
+    if ((e = cudaEventRecord(join, side))) return e;
     {
         ProfScope ps(kBwdPrep, s);
         bwd_prep_kernel<Tin, D><<<(unsigned)chunks, 256, sm0, s>>>(a);
-    }
-    if ((e = cudaGetLastError())) return e;
-    {
-        ProfScope ps(kBwdStates, s);
-        bwd_states_kernel<Tin, D><<<(unsigned)chains, 256, sm1, s>>>(a);
     }
     if ((e = cudaGetLastError())) return e;
     {
@@ -886,6 +920,7 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
         bwd_chain_kernel<Tin, D><<<(unsigned)chains, 256, sm2, s>>>(a);
     }
     if ((e = cudaGetLastError())) return e;
+    if ((e = cudaStreamWaitEvent(s, join, 0))) return e;
     {
         ProfScope ps(kBwdStateGrads, s);
         bwd_state_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3a, s>>>(a);

@@ -96,3 +96,32 @@ def test_bwd_layer_workload_sampled_heads():
             mine = got[n][b:b + 1, :, h:h + 1] if n not in ("dS0", "dM0") else got[n][b:b + 1, h:h + 1]
             e = rel_l2(mine, ref[n])
             assert e <= TOL["bf16"], (b, h, n, e)
+
+
+def test_bwd_cuda_graph_replay_matches_eager():
+    """The backward call (which forks the state rebuild onto a side stream and
+    joins it back) captured in a CUDA graph and replayed gives the eager
+    results bit for bit."""
+    spec = mi.Spec("bwd_graph", B=1, T=320, H=3, d=128, state_std=0.02, seed=503)
+    inp = mi.make_inputs(spec)
+    dev = mi.to_torch(inp, "cuda")
+    o, vt, _, _ = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in GATES),
+                                inp.d_corr, dev["S0"], dev["M0"])
+    do = torch.randn_like(o)
+    args = (dev["q"], dev["k"], dev["v"], *(dev[g] for g in GATES), inp.d_corr, vt, do,
+            dev["S0"], dev["M0"])
+    eager = mdn.chunk_bwd(*args)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        mdn.chunk_bwd(*args)  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        got = mdn.chunk_bwd(*args)
+    graph.replay()
+    torch.cuda.synchronize()
+    for n in NAMES:
+        assert torch.equal(got[n], eager[n]), n
