@@ -146,13 +146,14 @@ template <typename Tin, int D>
 __global__ void __launch_bounds__(256)
 bwd_states_kernel(BwdArgs a)
 {
-    constexpr int NS = NSB, KS = D + 1, VS = NS + 1;
-    constexpr int EPT = D * NS / 256;
+    // a thread owns rows rg + 16 e and the column pair 2 j2, 2 j2 + 1 of the slice
+    constexpr int NS = NSB, KS = D + 1, VS = NS + 2;
+    constexpr int EP = D / 16;     // rows per thread
     extern __shared__ float smem[];
     float* Ss = smem;              // [D][NS]
     float* Ms = Ss + D * NS;
     float* Ks = Ms + D * NS;       // [C][D+1]
-    float* Vs = Ks + C * KS;       // [C][NS+1]
+    float* Vs = Ks + C * KS;       // [C][NS+2] (8-byte aligned rows)
     float* gl = Vs + C * VS;       // [C] Gamma_{C,r}
     float* wv = gl + C;            // [C] w_r
     float* scal = wv + C;          // alphabar_C, b_C, mubar_C
@@ -160,22 +161,29 @@ bwd_states_kernel(BwdArgs a)
     const int slice = blockIdx.x % (D / NS);
     const long long bh = blockIdx.x / (D / NS);
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
-    const int j0 = slice * NS, j = tid % NS, rg = tid / NS;
+    const int j0 = slice * NS, j2 = tid & 15, rg = tid >> 4, jc = 2 * j2;
     const size_t st = (size_t)bh * D * D;
-    for (int e = 0; e < EPT; ++e) {
-        const int i = rg + 8 * e;
-        Ss[i * NS + j] = a.S0 ? a.S0[st + (size_t)i * D + j0 + j] : 0.f;
-        Ms[i * NS + j] = a.M0 ? a.M0[st + (size_t)i * D + j0 + j] : 0.f;
+    for (int e = 0; e < EP; ++e) {
+        const int i = rg + 16 * e;
+        const size_t g = st + (size_t)i * D + j0 + jc;
+        *reinterpret_cast<float2*>(Ss + i * NS + jc) =
+            a.S0 ? make_float2(a.S0[g], a.S0[g + 1]) : make_float2(0.f, 0.f);
+        *reinterpret_cast<float2*>(Ms + i * NS + jc) =
+            a.M0 ? make_float2(a.M0[g], a.M0[g + 1]) : make_float2(0.f, 0.f);
     }
     for (int n = 0; n < a.NT; ++n) {
         const size_t chunk = (size_t)bh * a.NT + n;
         const size_t crow = chunk * C;
         float* SSn = a.SS + chunk * 2 * D * D;
         __syncthreads();
-        for (int e = 0; e < EPT; ++e) {
-            const int i = rg + 8 * e;
-            SSn[(size_t)i * D + j0 + j] = Ss[i * NS + j];
-            SSn[(size_t)D * D + (size_t)i * D + j0 + j] = Ms[i * NS + j];
+        for (int e = 0; e < EP; ++e) {
+            const int i = rg + 16 * e;
+            const float2 sv = *reinterpret_cast<const float2*>(Ss + i * NS + jc);
+            const float2 mv = *reinterpret_cast<const float2*>(Ms + i * NS + jc);
+            SSn[(size_t)i * D + j0 + jc] = sv.x;
+            SSn[(size_t)i * D + j0 + jc + 1] = sv.y;
+            SSn[(size_t)D * D + (size_t)i * D + j0 + jc] = mv.x;
+            SSn[(size_t)D * D + (size_t)i * D + j0 + jc + 1] = mv.y;
         }
         for (int idx = tid; idx < C * D; idx += 256) {
             const int r = idx / D, c = idx % D, t = n * C + r;
@@ -197,25 +205,31 @@ bwd_states_kernel(BwdArgs a)
             }
         }
         __syncthreads();
-        float dS[EPT], dM[EPT];
+        float dS[EP][2], dM[EP][2];
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) dS[e] = dM[e] = 0.f;
+        for (int e = 0; e < EP; ++e) dS[e][0] = dS[e][1] = dM[e][0] = dM[e][1] = 0.f;
         for (int r = 0; r < C; ++r) {
-            const float v = Vs[r * VS + j];
-            const float vg = v * gl[r], vw = v * wv[r];
+            const float2 v = *reinterpret_cast<const float2*>(Vs + r * VS + jc);
+            const float g = gl[r], w = wv[r];
+            const float vg0 = v.x * g, vg1 = v.y * g, vw0 = v.x * w, vw1 = v.y * w;
 #pragma unroll
-            for (int e = 0; e < EPT; ++e) {
-                const float kv = Ks[r * KS + rg + 8 * e];  // one word per warp: a broadcast
-                dS[e] = fmaf(kv, vg, dS[e]);
-                dM[e] = fmaf(kv, vw, dM[e]);
+            for (int e = 0; e < EP; ++e) {
+                const float kv = Ks[r * KS + rg + 16 * e];
+                dS[e][0] = fmaf(kv, vg0, dS[e][0]);
+                dS[e][1] = fmaf(kv, vg1, dS[e][1]);
+                dM[e][0] = fmaf(kv, vw0, dM[e][0]);
+                dM[e][1] = fmaf(kv, vw1, dM[e][1]);
             }
         }
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int i = rg + 8 * e;
-            const float s = Ss[i * NS + j], m = Ms[i * NS + j];
-            Ss[i * NS + j] = scal[0] * s - scal[1] * m + dS[e];
-            Ms[i * NS + j] = scal[2] * m - dM[e];
+        for (int e = 0; e < EP; ++e) {
+            const int i = rg + 16 * e;
+            float2* sp = reinterpret_cast<float2*>(Ss + i * NS + jc);
+            float2* mp = reinterpret_cast<float2*>(Ms + i * NS + jc);
+            const float2 sv = *sp, mv = *mp;
+            *sp = make_float2(scal[0] * sv.x - scal[1] * mv.x + dS[e][0],
+                              scal[0] * sv.y - scal[1] * mv.y + dS[e][1]);
+            *mp = make_float2(scal[2] * mv.x - dM[e][0], scal[2] * mv.y - dM[e][1]);
         }
     }
 }
@@ -227,9 +241,10 @@ template <typename Tin, int D>
 __global__ void __launch_bounds__(256)
 bwd_chain_kernel(BwdArgs a)
 {
-    constexpr int NS = NSB, KS = D + 1, VS = NS + 1, AS = C + 1;
-    constexpr int EPT = D * NS / 256;   // state entries per thread
-    constexpr int RPT = C * NS / 256;   // chunk rows per thread
+    // a thread owns the column pair 2 j2, 2 j2 + 1 of the slice, rows rg + 16 e
+    constexpr int NS = NSB, KS = D + 1, VS = NS + 2, AS = C + 1;
+    constexpr int EP = D / 16;     // state rows per thread
+    constexpr int RP = C / 16;     // chunk rows per thread
     extern __shared__ float smem[];
     float* dSs = smem;             // [D][NS]
     float* dMs = dSs + D * NS;
@@ -237,8 +252,8 @@ bwd_chain_kernel(BwdArgs a)
     float* Qs = Ks + C * KS;       // [C][D+1]
     float* Att = Qs + C * KS;      // [C][C+1]
     float* Tm = Att + C * AS;      // [C][C+1]
-    float* dOs = Tm + C * AS;      // [C][NS+1]
-    float* X = dOs + C * VS;       // [C][NS+1]  dVtilde, then dY
+    float* dOs = Tm + C * AS;      // [C][NS+2]
+    float* X = dOs + C * VS;       // [C][NS+2]  dVtilde, then dY
     float* abar = X + C * VS;      // [C]
     float* bco = abar + C;
     float* d2 = bco + C;           // b_{r-1} alpha_r
@@ -249,22 +264,29 @@ bwd_chain_kernel(BwdArgs a)
     const int slice = blockIdx.x % (D / NS);
     const long long bh = blockIdx.x / (D / NS);
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
-    const int j0 = slice * NS, j = tid % NS, rg = tid / NS;
+    const int j0 = slice * NS, j2 = tid & 15, rg = tid >> 4, jc = 2 * j2;
     const size_t st = (size_t)bh * D * D;
-    for (int e = 0; e < EPT; ++e) {
-        const int i = rg + 8 * e;
-        dSs[i * NS + j] = a.dS_T ? a.dS_T[st + (size_t)i * D + j0 + j] : 0.f;
-        dMs[i * NS + j] = a.dM_T ? a.dM_T[st + (size_t)i * D + j0 + j] : 0.f;
+    for (int e = 0; e < EP; ++e) {
+        const int i = rg + 16 * e;
+        const size_t g = st + (size_t)i * D + j0 + jc;
+        *reinterpret_cast<float2*>(dSs + i * NS + jc) =
+            a.dS_T ? make_float2(a.dS_T[g], a.dS_T[g + 1]) : make_float2(0.f, 0.f);
+        *reinterpret_cast<float2*>(dMs + i * NS + jc) =
+            a.dM_T ? make_float2(a.dM_T[g], a.dM_T[g + 1]) : make_float2(0.f, 0.f);
     }
     for (int n = a.NT - 1; n >= 0; --n) {
         const size_t chunk = (size_t)bh * a.NT + n;
         const size_t crow = chunk * C;
         float* dSSn = a.dSS + chunk * 2 * D * D;
         __syncthreads();
-        for (int e = 0; e < EPT; ++e) {
-            const int i = rg + 8 * e;
-            dSSn[(size_t)i * D + j0 + j] = dSs[i * NS + j];
-            dSSn[(size_t)D * D + (size_t)i * D + j0 + j] = dMs[i * NS + j];
+        for (int e = 0; e < EP; ++e) {
+            const int i = rg + 16 * e;
+            const float2 sv = *reinterpret_cast<const float2*>(dSs + i * NS + jc);
+            const float2 mv = *reinterpret_cast<const float2*>(dMs + i * NS + jc);
+            dSSn[(size_t)i * D + j0 + jc] = sv.x;
+            dSSn[(size_t)i * D + j0 + jc + 1] = sv.y;
+            dSSn[(size_t)D * D + (size_t)i * D + j0 + jc] = mv.x;
+            dSSn[(size_t)D * D + (size_t)i * D + j0 + jc + 1] = mv.y;
         }
         for (int idx = tid; idx < C * D; idx += 256) {
             const int r = idx / D, c = idx % D, t = n * C + r;
@@ -304,76 +326,106 @@ bwd_chain_kernel(BwdArgs a)
         __syncthreads();
         // dVtilde = Att^T dO + Gamma_C o (K dS) - w o (K dM)
         {
-            float kds[RPT], kdm[RPT], ad[RPT];
+            float kds[RP][2], kdm[RP][2], ad[RP][2];
 #pragma unroll
-            for (int e = 0; e < RPT; ++e) kds[e] = kdm[e] = ad[e] = 0.f;
+            for (int e = 0; e < RP; ++e)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) kds[e][c] = kdm[e][c] = ad[e][c] = 0.f;
             for (int i = 0; i < D; ++i) {
-                const float ds = dSs[i * NS + j], dm = dMs[i * NS + j];
+                const float2 ds = *reinterpret_cast<const float2*>(dSs + i * NS + jc);
+                const float2 dm = *reinterpret_cast<const float2*>(dMs + i * NS + jc);
 #pragma unroll
-                for (int e = 0; e < RPT; ++e) {
-                    const float kv = Ks[(rg + 8 * e) * KS + i];
-                    kds[e] = fmaf(kv, ds, kds[e]);
-                    kdm[e] = fmaf(kv, dm, kdm[e]);
+                for (int e = 0; e < RP; ++e) {
+                    const float kv = Ks[(rg + 16 * e) * KS + i];
+                    kds[e][0] = fmaf(kv, ds.x, kds[e][0]);
+                    kds[e][1] = fmaf(kv, ds.y, kds[e][1]);
+                    kdm[e][0] = fmaf(kv, dm.x, kdm[e][0]);
+                    kdm[e][1] = fmaf(kv, dm.y, kdm[e][1]);
                 }
             }
             // Att is lower triangular (zeros above the diagonal): full sums are exact
             for (int r2 = rg; r2 < C; ++r2) {
-                const float od = dOs[r2 * VS + j];
+                const float2 od = *reinterpret_cast<const float2*>(dOs + r2 * VS + jc);
 #pragma unroll
-                for (int e = 0; e < RPT; ++e) ad[e] = fmaf(Att[r2 * AS + rg + 8 * e], od, ad[e]);
+                for (int e = 0; e < RP; ++e) {
+                    const float at = Att[r2 * AS + rg + 16 * e];
+                    ad[e][0] = fmaf(at, od.x, ad[e][0]);
+                    ad[e][1] = fmaf(at, od.y, ad[e][1]);
+                }
             }
 #pragma unroll
-            for (int e = 0; e < RPT; ++e) {
-                const int r = rg + 8 * e;
-                X[r * VS + j] = ad[e] + gl[r] * kds[e] - wv[r] * kdm[e];
+            for (int e = 0; e < RP; ++e) {
+                const int r = rg + 16 * e;
+                *reinterpret_cast<float2*>(X + r * VS + jc) =
+                    make_float2(ad[e][0] + gl[r] * kds[e][0] - wv[r] * kdm[e][0],
+                                ad[e][1] + gl[r] * kds[e][1] - wv[r] * kdm[e][1]);
             }
         }
         __syncthreads();
-        float dy[RPT];
+        float dy[RP][2];
 #pragma unroll
-        for (int e = 0; e < RPT; ++e) dy[e] = 0.f;
+        for (int e = 0; e < RP; ++e) dy[e][0] = dy[e][1] = 0.f;
         for (int r2 = rg; r2 < C; ++r2) {  // T lower triangular as well
-            const float xv = X[r2 * VS + j];
+            const float2 xv = *reinterpret_cast<const float2*>(X + r2 * VS + jc);
 #pragma unroll
-            for (int e = 0; e < RPT; ++e) dy[e] = fmaf(Tm[r2 * AS + rg + 8 * e], xv, dy[e]);
+            for (int e = 0; e < RP; ++e) {
+                const float tv = Tm[r2 * AS + rg + 16 * e];
+                dy[e][0] = fmaf(tv, xv.x, dy[e][0]);
+                dy[e][1] = fmaf(tv, xv.y, dy[e][1]);
+            }
         }
         __syncthreads();
 #pragma unroll
-        for (int e = 0; e < RPT; ++e) {
-            const int r = rg + 8 * e, t = n * C + r;
-            X[r * VS + j] = dy[e];
-            if (t < a.T) a.dv[tok_idx(a, b, t, h) * D + j0 + j] = dy[e];
+        for (int e = 0; e < RP; ++e) {
+            const int r = rg + 16 * e, t = n * C + r;
+            *reinterpret_cast<float2*>(X + r * VS + jc) = make_float2(dy[e][0], dy[e][1]);
+            if (t < a.T) {
+                float* dst = a.dv + tok_idx(a, b, t, h) * D + j0 + jc;
+                dst[0] = dy[e][0];
+                dst[1] = dy[e][1];
+            }
         }
         __syncthreads();
         const float aC = scal[0], bC = scal[1], mC = scal[2];
-        float us[EPT], um[EPT];  // qhat^T (.) dO - K^T (.) dY terms of dS and dM
+        float us[EP][2], um[EP][2];  // qhat^T (.) dO - K^T (.) dY terms of dS and dM
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) us[e] = um[e] = 0.f;
+        for (int e = 0; e < EP; ++e) us[e][0] = us[e][1] = um[e][0] = um[e][1] = 0.f;
         for (int r = 0; r < C; ++r) {
-            const float od = dOs[r * VS + j], xd = X[r * VS + j];
-            const float ab = abar[r];
-            const float qa = od * ab, qb = od * bco[r], xa = xd * ab, x2 = xd * d2[r];
+            const float2 od = *reinterpret_cast<const float2*>(dOs + r * VS + jc);
+            const float2 xd = *reinterpret_cast<const float2*>(X + r * VS + jc);
+            const float ab = abar[r], bb = bco[r], dd = d2[r];
+            const float qa0 = od.x * ab, qa1 = od.y * ab, qb0 = od.x * bb, qb1 = od.y * bb;
+            const float xa0 = xd.x * ab, xa1 = xd.y * ab, x20 = xd.x * dd, x21 = xd.y * dd;
 #pragma unroll
-            for (int e = 0; e < EPT; ++e) {
-                const int i = rg + 8 * e;
+            for (int e = 0; e < EP; ++e) {
+                const int i = rg + 16 * e;
                 const float qv = Qs[r * KS + i], kv = Ks[r * KS + i];
-                us[e] = fmaf(qv, qa, fmaf(-kv, xa, us[e]));
-                um[e] = fmaf(kv, x2, fmaf(-qv, qb, um[e]));
+                us[e][0] = fmaf(qv, qa0, fmaf(-kv, xa0, us[e][0]));
+                us[e][1] = fmaf(qv, qa1, fmaf(-kv, xa1, us[e][1]));
+                um[e][0] = fmaf(kv, x20, fmaf(-qv, qb0, um[e][0]));
+                um[e][1] = fmaf(kv, x21, fmaf(-qv, qb1, um[e][1]));
             }
         }
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-            const int i = rg + 8 * e;
-            const float ds = dSs[i * NS + j], dm = dMs[i * NS + j];
-            dSs[i * NS + j] = aC * ds + us[e];
-            dMs[i * NS + j] = -bC * ds + mC * dm + um[e];
+        for (int e = 0; e < EP; ++e) {
+            const int i = rg + 16 * e;
+            float2* sp = reinterpret_cast<float2*>(dSs + i * NS + jc);
+            float2* mp = reinterpret_cast<float2*>(dMs + i * NS + jc);
+            const float2 ds = *sp, dm = *mp;
+            *sp = make_float2(aC * ds.x + us[e][0], aC * ds.y + us[e][1]);
+            *mp = make_float2(-bC * ds.x + mC * dm.x + um[e][0], -bC * ds.y + mC * dm.y + um[e][1]);
         }
     }
     __syncthreads();
-    for (int e = 0; e < EPT; ++e) {
-        const int i = rg + 8 * e;
-        a.dS0[st + (size_t)i * D + j0 + j] = dSs[i * NS + j];
-        a.dM0[st + (size_t)i * D + j0 + j] = dMs[i * NS + j];
+    for (int e = 0; e < EP; ++e) {
+        const int i = rg + 16 * e;
+        const float2 sv = *reinterpret_cast<const float2*>(dSs + i * NS + jc);
+        const float2 mv = *reinterpret_cast<const float2*>(dMs + i * NS + jc);
+        const size_t g = st + (size_t)i * D + j0 + jc;
+        a.dS0[g] = sv.x;
+        a.dS0[g + 1] = sv.y;
+        a.dM0[g] = mv.x;
+        a.dM0[g + 1] = mv.y;
     }
 }
 
@@ -871,9 +923,9 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     const long long chunks = (long long)a.B * a.H * a.NT;
     const long long chains = (long long)a.B * a.H * (D / NSB);
     const size_t sm0 = sizeof(float) * (2 * C * (D + 1) + 2 * C * (C + 1) + C);
-    const size_t sm1 = sizeof(float) * (2 * D * NSB + C * (D + 1) + C * (NSB + 1) + 2 * C + 4);
+    const size_t sm1 = sizeof(float) * (2 * D * NSB + C * (D + 1) + C * (NSB + 2) + 2 * C + 4);
     const size_t sm2 = sizeof(float) * (2 * D * NSB + 2 * C * (D + 1) + 2 * C * (C + 1) +
-                                        2 * C * (NSB + 1) + 5 * C + 4);
+                                        2 * C * (NSB + 2) + 5 * C + 4);
     const size_t sm3a = sizeof(float) * (3 * C * (D + 1) + 4 * KP * (D + 1) + 24);
     const size_t sm3b = sizeof(float) * (5 * C * (D + 1) + 2 * C * (C + 1) + 12 * C);
     cudaError_t e;

@@ -161,3 +161,21 @@ def test_step_delta_norm_of_a_still_state_is_zero():
     torch.cuda.synchronize()
     assert torch.equal(S, S0)
     assert torch.count_nonzero(dn).item() == 0
+
+
+def test_step_delta_norm_decode_workload():
+    """The decode workload's shape (B = 256, H = 16, d = 128, bf16): one token from
+    random states; every head's norm against the oracle's fp64 step."""
+    spec = mi.replace(mi.CONFIGS[4], T=1, state_std=0.02, seed=1204)
+    inp = mi.make_inputs(spec)
+    dev = mi.to_torch(inp, "cuda")
+    keys = ("q", "k", "v", "alpha_log", "mu_log", "beta", "eta")
+    tok = {k: dev[k][:, 0].contiguous() for k in keys}
+    S, M = dev["S0"].clone(), dev["M0"].clone()
+    _, _, dn = mdn.step_with_delta_norm(*(tok[k] for k in keys), inp.d_corr, S, M)
+    torch.cuda.synchronize()
+    _, _, S1, _ = oracle.step(*(np.ascontiguousarray(getattr(inp, k)[:, 0]) for k in keys),
+                              inp.d_corr, inp.S0, inp.M0)
+    ref = oracle.step_delta_norm(inp.S0, S1)
+    got = to_np(dn)
+    assert np.max(np.abs(got - ref) / ref) < 5e-3
