@@ -171,11 +171,15 @@ size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   workspace   at least mdn_chunk_bwd_workspace_size(...) bytes, 256-byte
  *               aligned (about (4 d^2 + 3 C^2 + 10 C) x 4 bytes per chunk of C
  *               tokens of each head).
- *   flags       0.
+ *   flags       0 or MDN_CHECK_FINITE (synchronise, then report non-finite
+ *               outputs or an expired device wait).
  *
- * This build computes the backward pass in fp32 on CUDA cores, for every
- * supported d and dtype.  Support and errors as mdn_chunk_fwd (T = 0 copies
- * dS_T, dM_T to dS0, dM0).  Asynchronous on `stream`; enqueues six kernels.
+ * bf16 inputs with d = 128 run the products with the states on tcgen05
+ * tensor cores (bf16 operands, fp32 accumulation); everything else, and
+ * every other input combination, runs in fp32 on CUDA cores.  Support and
+ * errors as mdn_chunk_fwd (T = 0 copies dS_T, dM_T to dS0, dM0).
+ * Asynchronous on `stream` (except with MDN_CHECK_FINITE); enqueues six
+ * kernels, one of them on a side stream of the library that joins back.
  */
 mdn_status mdn_chunk_bwd(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
                          const float *alpha_log, const float *mu_log,

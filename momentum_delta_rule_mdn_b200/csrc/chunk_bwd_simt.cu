@@ -26,6 +26,8 @@
 // chunks, d_v split in slices); B-2 the reverse chain of (dS, dM); B-3a the
 // products with the states (dO S^T, ..., per chunk); B-3b the chunk-local
 // products and the gate gradients.  All outputs are fp32.
+#include <type_traits>
+
 #include "mdn_internal.cuh"
 
 namespace mdn {
@@ -973,11 +975,14 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     }
     if ((e = cudaGetLastError())) return e;
     if ((e = cudaStreamWaitEvent(s, join, 0))) return e;
-    {
+    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        // bf16 inputs: the six state products on tensor cores
+        if ((e = launch_bwd_state_grads_tc(a, s))) return e;
+    } else {
         ProfScope ps(kBwdStateGrads, s);
         bwd_state_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3a, s>>>(a);
+        if ((e = cudaGetLastError())) return e;
     }
-    if ((e = cudaGetLastError())) return e;
     {
         ProfScope ps(kBwdLocal, s);
         bwd_local_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3b, s>>>(a);

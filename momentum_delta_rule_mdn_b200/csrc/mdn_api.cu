@@ -257,7 +257,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 namespace {
 
 struct BwdLayout {
-    size_t la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec, total;
+    size_t status, la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec, total;
 };
 
 BwdLayout bwd_layout(long long BH, int NT, int D)
@@ -265,6 +265,7 @@ BwdLayout bwd_layout(long long BH, int NT, int D)
     const size_t chunks = (size_t)BH * NT, rows = chunks * kChunk;
     BwdLayout w;
     size_t off = 0;
+    w.status = off; off += align_up(64);
     w.la = off;    off += align_up(rows * sizeof(float));
     w.lm = off;    off += align_up(rows * sizeof(float));
     w.lc = off;    off += align_up(rows * sizeof(float));
@@ -299,7 +300,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
 {
     mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
     if (st != MDN_OK) return st;
-    if (flags != 0) return MDN_ERR_INVALID_ARG;
+    if (flags & ~MDN_CHECK_FINITE) return MDN_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return MDN_OK;
     if (!dS0 || !dM0 || !aligned16(dS0) || !aligned16(dM0)) return MDN_ERR_INVALID_ARG;
     const void* opt[] = {S0, M0, dS_T, dM_T};
@@ -337,6 +338,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.alpha_log = alpha_log; a.mu_log = mu_log; a.beta = beta; a.eta = eta;
     a.dcorr = d_corr; a.S0 = S0; a.M0 = M0; a.dS_T = dS_T; a.dM_T = dM_T;
     a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
+    a.status = reinterpret_cast<unsigned*>(ws + w.status);
     a.la = reinterpret_cast<float*>(ws + w.la);
     a.lm = reinterpret_cast<float*>(ws + w.lm);
     a.lc = reinterpret_cast<float*>(ws + w.lc);
@@ -350,10 +352,29 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.dq = dq; a.dk = dk_out; a.dv = dv_out;
     a.dalpha_log = dalpha_log; a.dmu_log = dmu_log; a.dbeta = dbeta; a.deta = deta;
     a.dS0 = dS0; a.dM0 = dM0;
+    const bool check = flags & MDN_CHECK_FINITE;
+    if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
     if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
                               a.gamma, s)))
         return mdn::cuda_fail(e);
     if ((e = launch_chunk_bwd_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
+    if (!check) return MDN_OK;
+    const size_t ntok = (size_t)B * T * H * D, ngate = (size_t)B * T * H;
+    const float* outs[] = {dq, dk_out, dv_out};
+    for (const float* p : outs)
+        if ((e = launch_finite_check(p, ntok, false, a.status, s))) return mdn::cuda_fail(e);
+    const float* gouts[] = {dalpha_log, dmu_log, dbeta, deta};
+    for (const float* p : gouts)
+        if ((e = launch_finite_check(p, ngate, false, a.status, s))) return mdn::cuda_fail(e);
+    if ((e = launch_finite_check(dS0, (size_t)B * H * D * D, false, a.status, s)) ||
+        (e = launch_finite_check(dM0, (size_t)B * H * D * D, false, a.status, s)))
+        return mdn::cuda_fail(e);
+    unsigned host_status[2] = {0, 0};
+    if ((e = cudaMemcpyAsync(host_status, a.status, sizeof(host_status), cudaMemcpyDeviceToHost, s)))
+        return mdn::cuda_fail(e);
+    if ((e = cudaStreamSynchronize(s))) return mdn::cuda_fail(e);
+    if (host_status[1]) return MDN_ERR_TIMEOUT;
+    if (host_status[0]) return MDN_ERR_NONFINITE;
     return MDN_OK;
 }
 

@@ -135,6 +135,7 @@ struct BwdArgs {
     const float* dM_T;
     int B, T, H, D, NT;
     // scratch
+    unsigned* status;  // [0]: non-finite flag, [1]: timeout flag
     float* la;       // [B*H, NT*C] chunk coefficients (gate preparation)
     float* lm;
     float* lc;
@@ -257,6 +258,8 @@ cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const 
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // The backward pass (fp32, CUDA cores); K-1's outputs must already be in a's scratch.
 cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, mdn_dtype dt, cudaStream_t s);
+// B-3a of the backward pass on tcgen05 (bf16 inputs, d = 128).
+cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and
