@@ -1,0 +1,168 @@
+// Shared by the two versions of the backward pass's chunk-local kernel (CUDA
+// cores and tcgen05): the per-chunk coefficient vectors and the last phase,
+// which turns the adjoints of the chunk coefficients into the gate gradients.
+//
+// Coefficients of one chunk (chunk-local prefix sums of the log gates la, lm):
+//   alphabar_r = exp(la_r), b_r = sum_{j<=r} exp(la_r - la_j) beta_j mubar_j,
+//   Gamma_{r,i} = eta_i Gp_{r,i},  Gp_{r,i} = sum_{j=i}^{r} exp(la_r - la_j) beta_j exp(lm_j - lm_i),
+//   w_r = eta_r mubar_C / mubar_r, D2_r = b_{r-1} alpha_r.
+// Given the adjoints of alphabar, b, D2, w (row sums of the state products,
+// in the chunk's record), of Gamma (dG) and the chunk-end scalars, the
+// gradients of the log gates follow by reverse recurrences along the chunk:
+// R_{j,i} = dG_{j,i} + alpha_{j+1} R_{j+1,i} folds the sum over r >= j of
+// dG_{r,i} exp(la_r - la_j), and the reverse cumulative sums of the la, lm
+// adjoints give those of alpha_log and mu_log.
+#pragma once
+
+#include "mdn_internal.cuh"
+
+namespace mdn {
+
+// Per-chunk vectors (C floats each) in shared memory.
+struct BwdVec {
+    float *al, *be, *et, *la, *lm, *b, *da, *db, *dla, *dlm, *de, *dbe;
+};
+constexpr int kBwdVecFloats = 12 * kChunk;
+
+__device__ __forceinline__ BwdVec bwd_vec(float* base) {
+    constexpr int C = kChunk;
+    BwdVec v;
+    v.al = base;           // alpha
+    v.be = v.al + C;       // beta
+    v.et = v.be + C;       // eta
+    v.la = v.et + C;       // la
+    v.lm = v.la + C;       // lm
+    v.b = v.lm + C;        // b
+    v.da = v.b + C;        // adjoint of alpha (its direct uses: P = Diag(alpha) K, D2)
+    v.db = v.da + C;       // adjoint of b
+    v.dla = v.db + C;      // adjoint of la
+    v.dlm = v.dla + C;     // adjoint of lm
+    v.de = v.dlm + C;      // adjoint of eta
+    v.dbe = v.de + C;      // adjoint of beta
+    return v;
+}
+
+// The last phase (every thread of a 256-thread CTA calls it): dG ([C][C+1],
+// overwritten), Gp ([C][C+1]), the record of the state products (rec_g, in
+// global memory; rec: kBwdRec floats of shared scratch), v.da holding the
+// direct adjoint of alpha from P.  Writes the four gate gradients of the
+// chunk's tokens.
+__device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* rec_g,
+                                                const BwdVec& v, float* dG, const float* Gp,
+                                                float* rec, int tid, int n, int b, int h)
+{
+    constexpr int C = kChunk, AS = kChunk + 1;
+    // the chunk's record into shared memory first (rec: kBwdRec floats), so
+    // that the single-thread loops below read no global memory
+    for (int i = tid; i < kBwdRec; i += 256) rec[i] = rec_g[i];
+    __syncthreads();
+    float* v_al = v.al;
+    float* v_be = v.be;
+    float* v_et = v.et;
+    float* v_la = v.la;
+    float* v_lm = v.lm;
+    float* v_b = v.b;
+    float* v_da = v.da;
+    float* v_db = v.db;
+    float* v_dla = v.dla;
+    float* v_dlm = v.dlm;
+    float* v_de = v.de;
+    float* v_dbe = v.dbe;
+    // coefficient adjoints -> la, lm, beta, eta, alpha
+    if (tid < C) {
+        const int r = tid;
+        const float dD2 = rec[2 * C + r];
+        const float b_prev = r > 0 ? v_b[r - 1] : 0.f;
+        v_da[r] += dD2 * b_prev;                           // D2_r = b_{r-1} alpha_r
+        float db = rec[C + r];
+        if (r + 1 < C) db += rec[2 * C + r + 1] * v_al[r + 1];
+        float dabar = rec[r];
+        if (r == C - 1) {
+            dabar += rec[5 * C];                           // alphabar_C S
+            db -= rec[5 * C + 1];                          // - b_C M
+        }
+        v_db[r] = db;
+        const float abar = expf(v_la[r]);
+        v_dla[r] = dabar * abar + db * v_b[r];
+        const float wr = v_et[r] * expf(v_lm[C - 1] - v_lm[r]);
+        const float dw = rec[4 * C + r];
+        v_dlm[r] = -dw * wr;
+        v_de[r] = dw * expf(v_lm[C - 1] - v_lm[r]);
+        v_dbe[r] = 0.f;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float s = rec[5 * C + 2] * expf(v_lm[C - 1]);      // mubar_C M
+        for (int r = 0; r < C; ++r) s += rec[4 * C + r] * v_et[r] * expf(v_lm[C - 1] - v_lm[r]);
+        v_dlm[C - 1] += s;
+        // b_r = sum_{j<=r} exp(la_r - la_j) beta_j mubar_j: reverse recurrence
+        float Rb = 0.f;
+        for (int j = C - 1; j >= 0; --j) {
+            Rb = v_db[j] + (j + 1 < C ? v_al[j + 1] * Rb : 0.f);
+            const float mb = expf(v_lm[j]);
+            const float tj = v_be[j] * mb * Rb;
+            v_dbe[j] += mb * Rb;
+            v_dla[j] -= tj;
+            v_dlm[j] += tj;
+        }
+    }
+    __syncthreads();
+    // Gamma = eta o Gp: row and column sums of dG o Gamma, and eta's share
+    if (tid < C) {
+        const int x = tid;
+        float rs = 0.f, cs = 0.f, ce = 0.f;
+        for (int y = 0; y <= x; ++y) rs = fmaf(dG[x * AS + y], v_et[y] * Gp[x * AS + y], rs);
+        for (int y = x; y < C; ++y) {
+            const float gp = Gp[y * AS + x];
+            cs = fmaf(dG[y * AS + x], v_et[x] * gp, cs);
+            ce = fmaf(dG[y * AS + x], gp, ce);
+        }
+        v_dla[x] += rs;
+        v_dlm[x] -= cs;
+        v_de[x] += ce;
+    }
+    __syncthreads();
+    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place, one column per thread
+    if (tid < C) {
+        const int i = tid;
+        float R = 0.f;
+        for (int j = C - 1; j >= i; --j) {
+            R = dG[j * AS + i] + (j + 1 < C ? v_al[j + 1] * R : 0.f);
+            dG[j * AS + i] = R;
+        }
+    }
+    __syncthreads();
+    // U_j = sum_{i<=j} eta_i exp(lm_j - lm_i) R_{j,i}
+    if (tid < C) {
+        const int j = tid;
+        float U = 0.f;
+        for (int i = 0; i <= j; ++i) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[j * AS + i], U);
+        v_dbe[j] += U;
+        v_dla[j] -= v_be[j] * U;
+        v_dlm[j] += v_be[j] * U;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // reverse cumulative sums: la, lm are inclusive prefix sums of the log gates
+        float sla = 0.f, slm = 0.f;
+        for (int j = C - 1; j >= 0; --j) {
+            sla += v_dla[j];
+            slm += v_dlm[j];
+            v_dla[j] = sla;
+            v_dlm[j] = slm;
+        }
+    }
+    __syncthreads();
+    if (tid < C) {
+        const int j = tid, t = n * C + j;
+        if (t < a.T) {
+            const size_t gi = ((size_t)b * a.T + t) * a.H + h;
+            a.dalpha_log[gi] = v_da[j] * v_al[j] + v_dla[j];
+            a.dmu_log[gi] = v_dlm[j];
+            a.dbeta[gi] = v_dbe[j];
+            a.deta[gi] = v_de[j];
+        }
+    }
+}
+
+}  // namespace mdn

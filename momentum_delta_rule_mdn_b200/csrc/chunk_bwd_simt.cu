@@ -28,6 +28,7 @@
 // products and the gate gradients.  All outputs are fp32.
 #include <type_traits>
 
+#include "bwd_common.cuh"
 #include "mdn_internal.cuh"
 
 namespace mdn {
@@ -621,18 +622,14 @@ bwd_local_grads_kernel(BwdArgs a)
     float* dYs = dOs + C * TS;     // dY, then dPK                [C][C+1]
     float* Gp = dYs + C * TS;      // [C][C+1] Gamma without eta
     float* dG = Gp + C * AS;       // [C][C+1] adjoint of Gamma, then R
-    float* v_al = dG + C * AS;     // alpha
-    float* v_be = v_al + C;        // beta
-    float* v_et = v_be + C;        // eta
-    float* v_la = v_et + C;        // la (chunk-local cumulative log alpha)
-    float* v_lm = v_la + C;        // lm
-    float* v_b = v_lm + C;         // b
-    float* v_da = v_b + C;         // d alpha (direct)
-    float* v_db = v_da + C;        // adjoint of b
-    float* v_dla = v_db + C;       // adjoint of la
-    float* v_dlm = v_dla + C;      // adjoint of lm
-    float* v_de = v_dlm + C;       // adjoint of eta
-    float* v_dbe = v_de + C;       // adjoint of beta
+    const BwdVec v = bwd_vec(dG + C * AS);
+    float* v_al = v.al;
+    float* v_be = v.be;
+    float* v_et = v.et;
+    float* v_la = v.la;
+    float* v_lm = v.lm;
+    float* v_b = v.b;
+    float* v_da = v.da;
     const int tid = threadIdx.x;
     const int n = blockIdx.x % a.NT;
     const long long bh = blockIdx.x / a.NT;
@@ -790,14 +787,22 @@ bwd_local_grads_kernel(BwdArgs a)
             const float alr = v_al[r];
             float dar = 0.f;
 #pragma unroll
-            for (int m = 0; m < NM; ++m) {
-                const int c = cg + 8 * m;
-                dar = fmaf(dp[u][m], Ks[r * TS + c], dar);
-                if (t < a.T) {
-                    const size_t g = tok_idx(a, b, t, h) * D + c;
-                    const float dqt = a.dq[g] + dq[u][m];
-                    a.dq[g] = dqt;
-                    a.dk[g] = a.dk[g] + fmaf(alr, dp[u][m], dk[u][m]) - a.dcorr * dqt;
+            for (int m = 0; m < NM; ++m) dar = fmaf(dp[u][m], Ks[r * TS + cg + 8 * m], dar);
+            if (t < a.T) {
+                // every load before any store: the stores would otherwise pin the
+                // loads that follow them in program order
+                const size_t g0 = tok_idx(a, b, t, h) * D + cg;
+                float qo[NM], ko[NM];
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                    qo[m] = a.dq[g0 + 8 * m];
+                    ko[m] = a.dk[g0 + 8 * m];
+                }
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                    const float dqt = qo[m] + dq[u][m];
+                    a.dq[g0 + 8 * m] = dqt;
+                    a.dk[g0 + 8 * m] = ko[m] + fmaf(alr, dp[u][m], dk[u][m]) - a.dcorr * dqt;
                 }
             }
 #pragma unroll
@@ -806,101 +811,7 @@ bwd_local_grads_kernel(BwdArgs a)
         }
     }
     __syncthreads();
-    // coefficient adjoints -> la, lm, beta, eta, alpha
-    if (tid < C) {
-        const int r = tid;
-        const float dD2 = rec[2 * C + r];
-        const float b_prev = r > 0 ? v_b[r - 1] : 0.f;
-        v_da[r] += dD2 * b_prev;                           // D2_r = b_{r-1} alpha_r
-        float db = rec[C + r];
-        if (r + 1 < C) db += rec[2 * C + r + 1] * v_al[r + 1];
-        float dabar = rec[r];
-        if (r == C - 1) {
-            dabar += rec[5 * C];                           // alphabar_C S
-            db -= rec[5 * C + 1];                          // - b_C M
-        }
-        v_db[r] = db;
-        const float abar = expf(v_la[r]);
-        v_dla[r] = dabar * abar + db * v_b[r];
-        const float wr = v_et[r] * expf(v_lm[C - 1] - v_lm[r]);
-        const float dw = rec[4 * C + r];
-        v_dlm[r] = -dw * wr;
-        v_de[r] = dw * expf(v_lm[C - 1] - v_lm[r]);
-        v_dbe[r] = 0.f;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float s = rec[5 * C + 2] * expf(v_lm[C - 1]);      // mubar_C M
-        for (int r = 0; r < C; ++r) s += rec[4 * C + r] * v_et[r] * expf(v_lm[C - 1] - v_lm[r]);
-        v_dlm[C - 1] += s;
-        // b_r = sum_{j<=r} exp(la_r - la_j) beta_j mubar_j: reverse recurrence
-        float Rb = 0.f;
-        for (int j = C - 1; j >= 0; --j) {
-            Rb = v_db[j] + (j + 1 < C ? v_al[j + 1] * Rb : 0.f);
-            const float mb = expf(v_lm[j]);
-            const float tj = v_be[j] * mb * Rb;
-            v_dbe[j] += mb * Rb;
-            v_dla[j] -= tj;
-            v_dlm[j] += tj;
-        }
-    }
-    __syncthreads();
-    // Gamma = eta o Gp: row and column sums of dG o Gamma, and eta's share
-    if (tid < C) {
-        const int x = tid;
-        float rs = 0.f, cs = 0.f, ce = 0.f;
-        for (int y = 0; y <= x; ++y) rs = fmaf(dG[x * AS + y], v_et[y] * Gp[x * AS + y], rs);
-        for (int y = x; y < C; ++y) {
-            const float gp = Gp[y * AS + x];
-            cs = fmaf(dG[y * AS + x], v_et[x] * gp, cs);
-            ce = fmaf(dG[y * AS + x], gp, ce);
-        }
-        v_dla[x] += rs;
-        v_dlm[x] -= cs;
-        v_de[x] += ce;
-    }
-    __syncthreads();
-    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place, one column per thread
-    if (tid < C) {
-        const int i = tid;
-        float R = 0.f;
-        for (int j = C - 1; j >= i; --j) {
-            R = dG[j * AS + i] + (j + 1 < C ? v_al[j + 1] * R : 0.f);
-            dG[j * AS + i] = R;
-        }
-    }
-    __syncthreads();
-    // U_j = sum_{i<=j} eta_i exp(lm_j - lm_i) R_{j,i}
-    if (tid < C) {
-        const int j = tid;
-        float U = 0.f;
-        for (int i = 0; i <= j; ++i) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[j * AS + i], U);
-        v_dbe[j] += U;
-        v_dla[j] -= v_be[j] * U;
-        v_dlm[j] += v_be[j] * U;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        // reverse cumulative sums: la, lm are inclusive prefix sums of the log gates
-        float sla = 0.f, slm = 0.f;
-        for (int j = C - 1; j >= 0; --j) {
-            sla += v_dla[j];
-            slm += v_dlm[j];
-            v_dla[j] = sla;
-            v_dlm[j] = slm;
-        }
-    }
-    __syncthreads();
-    if (tid < C) {
-        const int j = tid, t = n * C + j;
-        if (t < a.T) {
-            const size_t gi = tok_idx(a, b, t, h);
-            a.dalpha_log[gi] = v_da[j] * v_al[j] + v_dla[j];
-            a.dmu_log[gi] = v_dlm[j];
-            a.dbeta[gi] = v_dbe[j];
-            a.deta[gi] = v_de[j];
-        }
-    }
+    bwd_coeff_phase(a, rec, v, dG, Gp, v.dbe + C, tid, n, b, h);
 }
 
 // A non-blocking stream of the current device for work forked off a call's
@@ -929,7 +840,7 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     const size_t sm2 = sizeof(float) * (2 * D * NSB + 2 * C * (D + 1) + 2 * C * (C + 1) +
                                         2 * C * (NSB + 2) + 5 * C + 4);
     const size_t sm3a = sizeof(float) * (3 * C * (D + 1) + 4 * KP * (D + 1) + 24);
-    const size_t sm3b = sizeof(float) * (5 * C * (D + 1) + 2 * C * (C + 1) + 12 * C);
+    const size_t sm3b = sizeof(float) * (5 * C * (D + 1) + 2 * C * (C + 1) + kBwdVecFloats + kBwdRec);
     cudaError_t e;
 #define MDN_SET_SMEM(K, BYTES)                                                          \
     if ((e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
@@ -983,7 +894,9 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
         bwd_state_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3a, s>>>(a);
         if ((e = cudaGetLastError())) return e;
     }
-    {
+    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if ((e = launch_bwd_local_grads_tc(a, s))) return e;
+    } else {
         ProfScope ps(kBwdLocal, s);
         bwd_local_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3b, s>>>(a);
     }

@@ -15,6 +15,7 @@
 // kernel does.  Operands are staged by the threads themselves (fp32 states
 // and dY are rounded to bf16 on the way into shared memory), K-major with the
 // 128-byte swizzle.
+#include "bwd_common.cuh"
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -30,8 +31,8 @@ constexpr uint32_t SA1 = 0;          // [dO; dY]: 2 K-panels x 128 rows x 128 B
 constexpr uint32_t SA2 = 32768;      // [Vt; 0]
 constexpr uint32_t SB1 = 65536;      // [S | M] as 256 rows: 2 K-panels x 256 rows x 128 B
 constexpr uint32_t SB2 = 131072;     // [dS | dM]
-constexpr uint32_t SSUM = 196608;    // fp32 row sums [5][64], then scalars [8][3]
-constexpr uint32_t SBAR = SSUM + 1280 + 96;
+constexpr uint32_t SSUM = 196608;    // fp32 row-sum partials [12][64], then scalars [8][3]
+constexpr uint32_t SBAR = SSUM + 3072 + 96;
 constexpr uint32_t SMISC = SBAR + 16;
 constexpr uint32_t SMEM_BYTES = SMISC + 16 + 1024;  // + alignment slack
 constexpr int XS = 129;              // row stride (floats) of the dk exchange tile over SA1
@@ -52,8 +53,11 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     const long long bh = blockIdx.x / a.NT;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x, crow = chunk * C;
-    float* sums = reinterpret_cast<float*>(sm + SSUM);       // sa, sb, sd2, sgl, sw x 64 rows
-    float* wsum = sums + 5 * C;                              // [8 warps][3]
+    // row-sum partials, one slot per writer so that the sums are formed in a
+    // fixed order: sa from (row kind, column half) in slots 0..3, then sb,
+    // sd2, sgl, sw from the two column halves in slots 4..11
+    float* part = reinterpret_cast<float*>(sm + SSUM);
+    float* wsum = part + 12 * C;                             // [8 warps][3]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SBAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SMISC);
 
@@ -65,7 +69,7 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    for (int i = tid; i < 5 * C; i += kThr) sums[i] = 0.f;
+    for (int i = tid; i < 12 * C; i += kThr) part[i] = 0.f;
     // rows 64..127 of [Vt; 0]
     for (int i = tid; i < 1024; i += kThr) {
         const int p = i >> 9, w = i & 511;
@@ -237,19 +241,27 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     }
     // row sums of both column halves (and, for sa, of both row kinds)
     if (ok && in) {
-        atomicAdd(sums + r, sa);
+        const int kind = R < 64 ? 0 : 1;
+        part[(2 * kind + half) * C + r] = sa;
         if (R < 64) {
-            atomicAdd(sums + C + r, sb);
-            atomicAdd(sums + 3 * C + r, sgl);
-            atomicAdd(sums + 4 * C + r, sw);
+            part[(4 + half) * C + r] = sb;
+            part[(8 + half) * C + r] = sgl;
+            part[(10 + half) * C + r] = sw;
         } else {
-            atomicAdd(sums + 2 * C + r, sd2);
+            part[(6 + half) * C + r] = sd2;
         }
     }
     tc_fence_before_sync();
     __syncthreads();
     float* rec = a.crec_bw + chunk * kBwdRec;
-    for (int i = tid; i < 5 * C; i += kThr) rec[i] = sums[i];
+    if (tid < C) {
+        const float* p0 = part + tid;
+        rec[tid] = (p0[0] + p0[C]) + (p0[2 * C] + p0[3 * C]);
+        rec[C + tid] = p0[4 * C] + p0[5 * C];
+        rec[2 * C + tid] = p0[6 * C] + p0[7 * C];
+        rec[3 * C + tid] = p0[8 * C] + p0[9 * C];
+        rec[4 * C + tid] = p0[10 * C] + p0[11 * C];
+    }
     if (tid < 3) {
         float acc = 0.f;
         for (int w8 = 0; w8 < 8; ++w8) acc += wsum[w8 * 3 + tid];
@@ -260,6 +272,281 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// ---------------------------------------------------------------------------
+// B-3b on tcgen05: the chunk-local products of the backward pass.
+//   stage 1: [dO; dY] Vt^T -> dO Vt^T (lanes 0..63), dY Vt^T (64..127)     (N 64)
+//            [Qhat; K] K^T -> Qhat K^T, K K^T                               (N 64)
+//   SIMT:    dOVG = (dO Vt^T) o Gamma, dPK = -(dY Vt^T) o Gamma-, the adjoint
+//            of Gamma; bf16 operands [dOVG; dPK] and [dOVG^T | (dPK o alpha)^T]
+//   stage 2: [dOVG; dPK] K -> dQhat part (lanes 0..63), dP = dPK K (64..127) (N 128)
+//            [dOVG^T | (Diag(alpha) dPK)^T] [Qhat; K] -> dK part                (N 128)
+//   SIMT:    dq, dk written; the coefficient phase gives the gate gradients.
+constexpr uint32_t LA_DY = 0;        // [dO; dY]   K-major, 2 K-panels x 128 rows x 128 B
+constexpr uint32_t LA_QK = 32768;    // [Qhat; K]  K-major (its K rows double as B of K K^T)
+constexpr uint32_t LB_V = 65536;     // Vt         K-major, 2 K-panels x 64 rows x 128 B
+constexpr uint32_t LA_3 = 81920;     // [dOVG; dPK]          K = 64: 1 panel x 128 rows x 128 B
+constexpr uint32_t LA_4 = 98304;     // [dOVG^T | dPKa^T; 0] K = 128: 2 panels x 128 rows x 128 B
+constexpr uint32_t L_GP = 131072;    // fp32 Gp [64][65]
+constexpr uint32_t L_DG = L_GP + 16640;   // fp32 dG [64][65]
+constexpr uint32_t L_VEC = L_DG + 16640;  // 12 x 64 floats
+constexpr uint32_t L_REC = L_VEC + 3072;  // the chunk record (kBwdRec floats)
+constexpr uint32_t L_BAR = L_REC + kBwdRec * 4;
+constexpr uint32_t L_MISC = L_BAR + 16;
+constexpr uint32_t L_SMEM = L_MISC + 16 + 1024;
+constexpr int LAS = 65;                   // row stride of the fp32 C x C matrices
+
+__device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
+}
+// byte offset of element (row, k) in a K-major 128-byte-swizzled tile whose
+// K-panels (64 elements) are panel_bytes apart
+__device__ __forceinline__ uint32_t kmaj_off(int row, int k, uint32_t panel_bytes) {
+    return (k >> 6) * panel_bytes + sw128_off(row, (k & 63) >> 3) + (k & 7) * 2;
+}
+
+__global__ void __launch_bounds__(kThr, 1)
+bwd_local_grads_tc_kernel(BwdArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x % a.NT;
+    const long long bh = blockIdx.x / a.NT;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const size_t chunk = blockIdx.x, crow = chunk * C;
+    float* Gp = reinterpret_cast<float*>(sm + L_GP);
+    float* dG = reinterpret_cast<float*>(sm + L_DG);
+    const BwdVec v = bwd_vec(reinterpret_cast<float*>(sm + L_VEC));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L_MISC);
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major)
+    for (int i = tid; i < C * 16; i += kThr) {
+        const int r = i >> 4, c16 = i & 15, t = n * C + r;
+        const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
+        float o[8] = {0.f}, y[8] = {0.f}, q[8] = {0.f}, k[8] = {0.f}, vt[8] = {0.f};
+        if (t < a.T) {
+            const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g), o);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g), q);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g), k);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g), vt);
+            const float4 y0 = *reinterpret_cast<const float4*>(a.dv + g);
+            const float4 y1 = *reinterpret_cast<const float4*>(a.dv + g + 4);
+            y[0] = y0.x; y[1] = y0.y; y[2] = y0.z; y[3] = y0.w;
+            y[4] = y1.x; y[5] = y1.y; y[6] = y1.z; y[7] = y1.w;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q[e] -= a.dcorr * k[e];
+        }
+        st_bf16x8(sm + LA_DY + off, o);
+        st_bf16x8(sm + LA_DY + off + 64 * 128, y);
+        st_bf16x8(sm + LA_QK + off, q);
+        st_bf16x8(sm + LA_QK + off + 64 * 128, k);
+        st_bf16x8(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7), vt);
+    }
+    // rows 64..127 of the second stage-2 operand are zero
+    for (int i = tid; i < 1024; i += kThr) {
+        const int p = i >> 9, w = i & 511;
+        *reinterpret_cast<uint4*>(sm + LA_4 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
+    }
+    if (tid < C) {
+        const int r = tid, t = n * C + r;
+        const bool in = t < a.T;
+        const size_t gi = in ? tokrow(a, b, t, h) : 0;
+        v.al[r] = in ? expf(a.alpha_log[gi]) : 1.f;
+        v.be[r] = in ? a.beta[gi] : 0.f;
+        v.et[r] = in ? a.eta[gi] : 0.f;
+        v.la[r] = a.la[crow + r];
+        v.lm[r] = a.lm[crow + r];
+        v.b[r] = a.bco[crow + r];
+        v.da[r] = 0.f;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ka = (ks >> 2) * 16384 + (ks & 3) * 32;
+            const uint32_t kv = (ks >> 2) * 8192 + (ks & 3) * 32;
+            mma_bf16(tmem, smem_desc(sbase + LA_DY + ka, 16, 1024, kSw128),
+                     smem_desc(sbase + LB_V + kv, 16, 1024, kSw128), id1, ks > 0);
+            mma_bf16(tmem + 64, smem_desc(sbase + LA_QK + ka, 16, 1024, kSw128),
+                     smem_desc(sbase + LA_QK + 8192 + ka, 16, 1024, kSw128), id1, ks > 0);
+        }
+        mma_commit(&bars[0]);
+    }
+    // Gamma without eta, by its column recurrence (overlaps the products)
+    if (tid < C) {
+        const int i = tid;
+        float g = 0.f;
+        for (int r = 0; r < C; ++r) {
+            if (r < i) {
+                Gp[r * LAS + i] = 0.f;
+            } else {
+                g = (r == i) ? v.be[i] : fmaf(v.al[r], g, v.be[r] * expf(v.lm[r] - v.lm[i]));
+                Gp[r * LAS + i] = g;
+            }
+        }
+    }
+    bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
+    tc_fence_after_sync();
+
+    // stage-1 epilogue: warp w reads lanes 32 (w % 4) ..; warps w, w + 4 take
+    // columns i in [32 half, 32 half + 32)
+    const int quad = warp & 3, half = warp >> 2;
+    const int R = quad * 32 + lane, r = R & 63;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    float dgm[32];  // dY rows: dA o (P K^T), owed to dG[r - 1][i]
+    if (ok) {
+        float x1[32], x2[32];
+        tmem_ld32(tq + 32 * half, x1);        // dO Vt^T  (dY Vt^T on lanes 64..127)
+        tmem_ld32(tq + 64 + 32 * half, x2);   // Qhat K^T (K K^T)
+        tmem_wait_ld();
+        const float al_r = v.al[r];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int i = 32 * half + e;
+            if (R < 64) {
+                const float g = v.et[i] * Gp[r * LAS + i];
+                const float ovg = i <= r ? x1[e] * g : 0.f;
+                dG[r * LAS + i] = i <= r ? x1[e] * x2[e] : 0.f;
+                st_bf16(sm + LA_3 + kmaj_off(r, i, 16384), ovg);             // row r of [dOVG; .]
+                st_bf16(sm + LA_4 + kmaj_off(i, r, 16384), ovg);             // (dOVG^T)[i][r]
+            } else {
+                const float pk = i < r ? -x1[e] * v.et[i] * Gp[(r - 1) * LAS + i] : 0.f;
+                dgm[e] = i < r ? -x1[e] * al_r * x2[e] : 0.f;
+                st_bf16(sm + LA_3 + kmaj_off(64 + r, i, 16384), pk);        // row 64 + r: dPK
+                st_bf16(sm + LA_4 + kmaj_off(i, 64 + r, 16384), pk * al_r); // (Diag(alpha) dPK)^T
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (ok && R >= 64) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int i = 32 * half + e;
+            if (i < r) dG[(r - 1) * LAS + i] += dgm[e];  // one writer per entry
+        }
+    }
+    const float* rec = a.crec_bw + chunk * kBwdRec;
+    if (tid == 0 && ok) {
+        constexpr uint32_t id2 = idesc_bf16(128, 128, false, true);
+        // [dOVG; dPK] K: B = K (K-dim i = rows 64..127 of the [Qhat; K] tile, N = features)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tmem + 128, smem_desc(sbase + LA_3 + ks * 32, 16, 1024, kSw128),
+                     smem_desc(sbase + LA_QK + 8192 + ks * 2048, 16384, 1024, kSw128), id2, ks > 0);
+        // [dOVG^T | dPKa^T] [Qhat; K]: B = the whole [Qhat; K] tile, K-dim 128 rows
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + 256,
+                     smem_desc(sbase + LA_4 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128),
+                     smem_desc(sbase + LA_QK + ks * 2048, 16384, 1024, kSw128), id2, ks > 0);
+        mma_commit(&bars[1]);
+    }
+    __syncthreads();
+    if (tid < C) dG[(C - 1) * LAS + tid] += rec[3 * C + tid];  // Gamma_{C,i} in the state update
+    ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
+    tc_fence_after_sync();
+
+    // stage-2 epilogue: lanes 64..127 hold dP = dPK K; lanes 0..63 the dQhat
+    // and dK parts; warps w, w + 4 take feature columns [64 half, 64 half + 64)
+    float* X = reinterpret_cast<float*>(sm + LA_DY);  // alpha_r dP[r][c], [64][129], over the operands
+    const int t = n * C + r;
+    const bool in = t < a.T;
+    const size_t grow = in ? tokrow(a, b, t, h) * D : 0;
+    if (ok && R >= 64) {
+        float dar = 0.f;
+        const float al_r = v.al[r];
+        const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + grow;
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+            float dp[16], kv[16];
+            tmem_ld16(tq + 128 + c0, dp);
+            tmem_wait_ld();
+            if (in) {
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + c0), kv);
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + c0 + 8), kv + 8);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dar = fmaf(dp[e], kv[e], dar);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) X[r * 129 + c0 + e] = al_r * dp[e];
+        }
+        atomicAdd(v.da + r, dar);
+    }
+    __syncthreads();
+    if (ok && R < 64) {
+        // The exchange row is read into registers before any global store: X is
+        // reached through a generic pointer, so reads of it interleaved with the
+        // stores to dq and dk could not be hoisted and serialised the loop.
+        float xr[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) xr[e] = X[r * 129 + 64 * half + e];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = 64 * half + 16 * j;
+            float dqb[16], dkb[16];
+            tmem_ld16(tq + 128 + c0, dqb);
+            tmem_ld16(tq + 256 + c0, dkb);
+            tmem_wait_ld();
+            if (in) {
+                float4 q4[4], k4[4];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {  // every load of the group before any store
+                    q4[e4] = *reinterpret_cast<const float4*>(a.dq + grow + c0 + 4 * e4);
+                    k4[e4] = *reinterpret_cast<const float4*>(a.dk + grow + c0 + 4 * e4);
+                }
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float qo[4] = {q4[e4].x, q4[e4].y, q4[e4].z, q4[e4].w};
+                    const float ko[4] = {k4[e4].x, k4[e4].y, k4[e4].z, k4[e4].w};
+                    float qn[4], kn[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int x = 16 * j + 4 * e4 + e;
+                        qn[e] = qo[e] + dqb[4 * e4 + e];
+                        kn[e] = ko[e] + dkb[4 * e4 + e] + xr[x] - a.dcorr * qn[e];
+                    }
+                    *reinterpret_cast<float4*>(a.dq + grow + c0 + 4 * e4) =
+                        make_float4(qn[0], qn[1], qn[2], qn[3]);
+                    *reinterpret_cast<float4*>(a.dk + grow + c0 + 4 * e4) =
+                        make_float4(kn[0], kn[1], kn[2], kn[3]);
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+    if (!ok) {
+        if (tid == 0) atomicOr(a.status + 1, 1u);
+        return;
+    }
+    bwd_coeff_phase(a, rec, v, dG, Gp, reinterpret_cast<float*>(sm + L_REC), tid, n, b, h);
 }
 
 }  // namespace
@@ -274,6 +561,23 @@ cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     ProfScope ps(kBwdStateGrads, s);
     bwd_state_grads_tc_kernel<<<(unsigned)chunks, kThr, SMEM_BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace mdn
+
+namespace mdn {
+
+cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s)
+{
+    if (a.D != D) return cudaErrorNotSupported;
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    cudaError_t e = cudaFuncSetAttribute(bwd_local_grads_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L_SMEM);
+    if (e != cudaSuccess) return e;
+    ProfScope ps(kBwdLocal, s);
+    bwd_local_grads_tc_kernel<<<(unsigned)chunks, kThr, L_SMEM, s>>>(a);
     return cudaGetLastError();
 }
 

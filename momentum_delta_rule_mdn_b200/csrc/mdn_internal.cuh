@@ -260,6 +260,8 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, mdn_dtype dt, cudaStream_t s);
 // B-3a of the backward pass on tcgen05 (bf16 inputs, d = 128).
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s);
+// B-3b of the backward pass on tcgen05 (bf16 inputs, d = 128).
+cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and
