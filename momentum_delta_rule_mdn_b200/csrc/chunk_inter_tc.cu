@@ -559,8 +559,8 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
 // are reserved: the intra-chunk CTAs there take a single chunk, and the chain
 // starts one chunk's time after launch while the other SMs produce the rest
 // ahead of it.  Four slices per head when they fit in one wave (their chain
-// is the shortest per chunk), else two; SMs are reserved only when the
-// slices fit beside the intra-chunk kernel's share.
+// is the shortest per chunk; two waves for packed sequences), else two; SMs
+// are reserved only when the slices fit beside the intra-chunk kernel's share.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
@@ -570,7 +570,11 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     if (e != cudaSuccess) return e;
     const long long heads = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
     const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
-    if (ns == 0) ns = heads * 4 <= sms ? 32 : 64;
+    // Packed sequences of mixed lengths: chains of short sequences end early
+    // and free their SMs, so a second wave of 32-column chains costs little
+    // next to the longest chain, which runs in the first (sequences are laid
+    // out in order, the first ones on the lowest CTAs).
+    if (ns == 0) ns = heads * 4 <= (a.cu_chunks ? 2LL * sms : (long long)sms) ? 32 : 64;
     const long long ctas = heads * (D / ns);
     const int reserve = ctas <= room ? (int)ctas : 0;
     if (!a.test_no_intra && (e = launch_chunk_intra_tc(a, s, reserve)) != cudaSuccess) return e;
