@@ -277,7 +277,7 @@ def run_decode(args, mdn, device, hbm_peak):
     """mdn_step at the decode workload's shape (B=256, H=16, d=128): S and M
     (2 x 268 MB fp32) are read and written once per token, so no L2 flush is
     needed.  Reports tokens/s and the kernel's HBM fraction."""
-    spec = mi.CONFIGS[4]
+    spec = mi.WORKLOADS[4]
     B, H, d = spec.B, spec.H, spec.d
     tok = mi.make_inputs(mi.replace(spec, T=1, seed=spec.seed + 11))
     t = {k: v[:, 0].contiguous() for k, v in mi.to_torch(tok, device).items() if v is not None}
@@ -625,10 +625,10 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------- plumbing
 def workload_spec(w):
     if w is None:
-        return mi.CONFIGS[DEFAULT_WORKLOAD]
+        return mi.WORKLOADS[DEFAULT_WORKLOAD]
     if str(w).isdigit():
-        return mi.CONFIGS[int(w)]
-    for s in mi.CONFIGS:
+        return mi.WORKLOADS[int(w)]
+    for s in mi.WORKLOADS:
         if s.name == w:
             return s
     raise SystemExit(f"unknown workload {w!r}")

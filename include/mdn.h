@@ -53,7 +53,7 @@ typedef struct CUstream_st *mdn_stream_t;
 typedef enum {
     MDN_OK = 0,
     MDN_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment, bad size  */
-    MDN_ERR_UNSUPPORTED = 2,  /* valid but outside this build's support (d, C, dtype) */
+    MDN_ERR_UNSUPPORTED = 2,  /* valid but outside what the library supports (d, C, dtype) */
     MDN_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed                 */
     MDN_ERR_NONFINITE = 4,    /* MDN_CHECK_FINITE found a NaN/Inf in an output        */
     MDN_ERR_TIMEOUT = 5       /* a bounded on-device wait ran out (kernel gave up)    */
@@ -114,7 +114,7 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   alpha_log, mu_log, beta, eta  [B,T,H] fp32.
  *   d_corr      the scalar d of qhat = q - d k.
  *   S0, M0      [B,H,d,d] fp32 entering states; either may be NULL (zeros).
- *   C           chunk length; this build supports C = 64.
+ *   C           chunk length; the library supports C = 64.
  *   o, vtilde   [B,T,H,d] in_dtype outputs (vtilde is the materialised Vtilde).
  *   S_T, M_T    [B,H,d,d] fp32 outputs: the states after token T.  They may
  *               alias S0 / M0 (read before written, per head).

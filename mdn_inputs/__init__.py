@@ -25,7 +25,7 @@ from typing import Optional
 
 import numpy as np
 
-__all__ = ["Spec", "Inputs", "CONFIGS", "make_inputs", "bf16_round_bits",
+__all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "bf16_round_bits",
            "bf16_bits_to_f32", "replace"]
 
 
@@ -52,7 +52,7 @@ class Spec:
 
 
 # The five workloads.  Index i uses seed 1000 + i.
-CONFIGS = [
+WORKLOADS = [
     Spec("tiny_fp32_B1_H1_T256_d64", B=1, T=256, H=1, d=64, dtype="f32", seed=1000),
     Spec("layer400m_B4_H8_T2048_d128", B=4, T=2048, H=8, d=128, seed=1001),
     Spec("layer1p3b_B8_H16_T4096_d128", B=8, T=4096, H=16, d=128, state_std=0.01,

@@ -185,7 +185,7 @@ const char* mdn_status_string(mdn_status s)
     switch (s) {
         case MDN_OK: return "MDN_OK";
         case MDN_ERR_INVALID_ARG: return "MDN_ERR_INVALID_ARG: invalid argument";
-        case MDN_ERR_UNSUPPORTED: return "MDN_ERR_UNSUPPORTED: sizes or dtype outside this build's support";
+        case MDN_ERR_UNSUPPORTED: return "MDN_ERR_UNSUPPORTED: sizes or dtype outside the library's support";
         case MDN_ERR_CUDA: return "MDN_ERR_CUDA: a CUDA launch or runtime call failed";
         case MDN_ERR_NONFINITE: return "MDN_ERR_NONFINITE: an output holds NaN or Inf";
         case MDN_ERR_TIMEOUT: return "MDN_ERR_TIMEOUT: a bounded device wait ran out";

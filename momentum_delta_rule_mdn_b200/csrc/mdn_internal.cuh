@@ -10,7 +10,7 @@
 
 namespace mdn {
 
-constexpr int kChunk = 64;  // chunk length C supported by this build
+constexpr int kChunk = 64;  // the chunk length C the kernels support
 
 // Element loads/stores in the input dtype, computed in fp32.
 __device__ __forceinline__ float ld_elem(const float* p) { return *p; }

@@ -18,7 +18,7 @@ the chunk start; S, M are the states entering the chunk)
 
 The eta_i factor on write i, the "previous step" reading of the index range
 0..C-1 in Y and Z, and the chunk-end state update and output formula are
-this build's readings of the pages (they are not printed there); the CPU
+readings of the pages (they are not printed there); the CPU
 tests pin this restatement to the stepwise oracle for several C.
 It is independent of the oracle and of the CUDA library.
 """

@@ -7,7 +7,7 @@ the oracle with planted mistakes and checks that some pin fails each time.
 
 Sources ("MDN: Parallelizing Stepwise Momentum for Delta Linear Attention"):
   recurrence ............ paper.rainbus.top summary, step 1; ijyty.com, section 3
-  unrolled closed form .. summary, step 2 (eta_i on write i: this build's reading)
+  unrolled closed form .. summary, step 2 (eta_i on write i: a reading)
   row<->column reordering summary, step 3; ijyty.com, section 4
   chunkwise form ........ summary, step 4
   spectrum lambda+- ..... summary, step 6; novelty paragraph; ijyty.com, section 5

@@ -17,7 +17,7 @@ TOL = {"f32": 1e-4, "bf16": 2e-2}
 @functools.lru_cache(maxsize=None)
 def config_inputs(i: int) -> mi.Inputs:
     """The i-th workload's inputs, generated once per test session."""
-    return mi.make_inputs(mi.CONFIGS[i])
+    return mi.make_inputs(mi.WORKLOADS[i])
 
 
 def rel_l2(x, ref) -> float:

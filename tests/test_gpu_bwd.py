@@ -78,7 +78,7 @@ def test_bwd_zero_length_passes_state_cotangents():
 def test_bwd_layer_workload_sampled_heads():
     """The whole layer workload (B = 4, T = 2048, H = 8, d = 128, bf16) through the
     forward and backward passes; two heads against the oracle."""
-    inp = mi.make_inputs(mi.CONFIGS[1])
+    inp = mi.make_inputs(mi.WORKLOADS[1])
     dev = mi.to_torch(inp, "cuda")
     o, vt, _, _ = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in GATES),
                                 inp.d_corr)

@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("cfg,T", [(0, 256), (1, 300), (3, 1000)])
 def test_gate_prep_matches_oracle(cfg, T):
-    spec = mi.replace(mi.CONFIGS[cfg], B=2, H=3, T=T)
+    spec = mi.replace(mi.WORKLOADS[cfg], B=2, H=3, T=T)
     inp = mi.make_inputs(spec)
     dev = mi.to_torch(inp, "cuda")
     la, lm, lc, bco, gam = mdn.chunk_gate_prep(dev["alpha_log"], dev["mu_log"], dev["beta"],
@@ -47,7 +47,7 @@ def test_gate_prep_matches_oracle(cfg, T):
 def test_gate_prep_stress_regime():
     """alpha -> 1 with mu at its clamp e^-1: c_r - c_{i-1} cancels in the
     log-broadcast form; the column recurrence keeps Gamma accurate."""
-    spec = mi.replace(mi.CONFIGS[1], B=1, H=4, T=256, a_mean=6.0, x_mean=-1.5, c_mean=-5.0)
+    spec = mi.replace(mi.WORKLOADS[1], B=1, H=4, T=256, a_mean=6.0, x_mean=-1.5, c_mean=-5.0)
     inp = mi.make_inputs(spec)
     dev = mi.to_torch(inp, "cuda")
     *_, gam = mdn.chunk_gate_prep(dev["alpha_log"], dev["mu_log"], dev["beta"], dev["eta"])

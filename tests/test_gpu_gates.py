@@ -37,7 +37,7 @@ def _dev(*arrs):
 @pytest.mark.parametrize("cfg", [1, 3])
 def test_gate_params_workload_preactivations(act, cfg):
     """The pre-activations of the workloads ([B,T,H], n % 4 == 0: the float4 path)."""
-    spec = mi.replace(mi.CONFIGS[cfg], B=2, T=1000, H=mi.CONFIGS[cfg].H)
+    spec = mi.replace(mi.WORKLOADS[cfg], B=2, T=1000, H=mi.WORKLOADS[cfg].H)
     inp = mi.make_inputs(spec)
     pre = (inp.x_eta, inp.a_pre, inp.b_pre, inp.c_pre)
     got = mdn.gate_params(*_dev(*pre), s=spec.eta_scale, mu_log_min=spec.mu_log_min,
@@ -96,7 +96,7 @@ def test_gate_params_extreme_preactivations(act):
 def test_gate_params_feed_the_chunk_pass():
     """K-0's gates drive mdn_chunk_fwd to the oracle's result from the same
     pre-activations (the oracle forms its gates itself)."""
-    spec = mi.replace(mi.CONFIGS[1], B=1, T=320, H=4)
+    spec = mi.replace(mi.WORKLOADS[1], B=1, T=320, H=4)
     inp = mi.make_inputs(spec)
     dev = mi.to_torch(inp, "cuda")
     pre = (inp.x_eta, inp.a_pre, inp.b_pre, inp.c_pre)
@@ -166,7 +166,7 @@ def test_step_delta_norm_of_a_still_state_is_zero():
 def test_step_delta_norm_decode_workload():
     """The decode workload's shape (B = 256, H = 16, d = 128, bf16): one token from
     random states; every head's norm against the oracle's fp64 step."""
-    spec = mi.replace(mi.CONFIGS[4], T=1, state_std=0.02, seed=1204)
+    spec = mi.replace(mi.WORKLOADS[4], T=1, state_std=0.02, seed=1204)
     inp = mi.make_inputs(spec)
     dev = mi.to_torch(inp, "cuda")
     keys = ("q", "k", "v", "alpha_log", "mu_log", "beta", "eta")

@@ -22,12 +22,12 @@ def test_bf16_rounding_is_round_to_nearest_even():
     assert np.array_equal(mi.bf16_bits_to_f32(ref), torch.from_numpy(y).to(torch.bfloat16).float().numpy())
 
 
-@pytest.mark.parametrize("cfg", range(len(mi.CONFIGS)))
+@pytest.mark.parametrize("cfg", range(len(mi.WORKLOADS)))
 def test_gates_satisfy_stability_constraints(cfg):
     """Stability inequality -(1-a)(1-mu) <= a beta eta |k|^2 <= (1+a)(1+mu) (novelty
     paragraph of the paper.rainbus.top summary) and non-negative real parts of
     lambda+- (summary step 6), on the generated gates and stored keys."""
-    spec = mi.CONFIGS[cfg]
+    spec = mi.WORKLOADS[cfg]
     spec = mi.replace(spec, B=min(spec.B, 2), T=min(spec.T, 512))
     inp = mi.make_inputs(spec)
     a = np.exp(inp.alpha_log.astype(np.float64))
@@ -44,7 +44,7 @@ def test_gates_satisfy_stability_constraints(cfg):
 
 
 def test_generator_is_deterministic():
-    s = mi.replace(mi.CONFIGS[2], B=1, T=128, H=2)
+    s = mi.replace(mi.WORKLOADS[2], B=1, T=128, H=2)
     a, b = mi.make_inputs(s), mi.make_inputs(s)
     for f in ("q_store", "k_store", "v_store", "alpha_log", "mu_log", "beta", "eta", "S0", "M0"):
         assert np.array_equal(getattr(a, f), getattr(b, f))

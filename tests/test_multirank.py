@@ -34,7 +34,7 @@ def _rank_main(rank, world, port, out_dir):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        spec = bench.rank_spec(mi.CONFIGS[0], rank)
+        spec = bench.rank_spec(mi.WORKLOADS[0], rank)
         inp = mi.make_inputs(spec)
         # each replica runs the pass on its own batch (the oracle stands in for the GPU path)
         o, vt, S, M = oracle.chunk_fwd(inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log, inp.beta,
