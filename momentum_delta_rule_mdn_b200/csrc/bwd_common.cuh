@@ -14,9 +14,34 @@
 // adjoints give those of alpha_log and mu_log.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "mdn_internal.cuh"
 
 namespace mdn {
+
+// Eight consecutive elements of a token tensor from element idx (a multiple
+// of 8) as fp32: one 16-byte load for bf16, two for fp32.
+template <typename Tin>
+__device__ __forceinline__ void ld8(const void* base, size_t idx, float* x);
+template <>
+__device__ __forceinline__ void ld8<__nv_bfloat16>(const void* base, size_t idx, float* x) {
+    const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
+        x[2 * e] = __low2float(v);
+        x[2 * e + 1] = __high2float(v);
+    }
+}
+template <>
+__device__ __forceinline__ void ld8<float>(const void* base, size_t idx, float* x) {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
 
 // Per-chunk vectors (C floats each) in shared memory.
 struct BwdVec {

@@ -188,13 +188,32 @@ bwd_states_kernel(BwdArgs a)
             SSn[(size_t)D * D + (size_t)i * D + j0 + jc] = mv.x;
             SSn[(size_t)D * D + (size_t)i * D + j0 + jc + 1] = mv.y;
         }
-        for (int idx = tid; idx < C * D; idx += 256) {
-            const int r = idx / D, c = idx % D, t = n * C + r;
-            Ks[r * KS + c] = t < a.T ? ldt<Tin>(a.k, tok_idx(a, b, t, h) * D + c) : 0.f;
-        }
-        for (int idx = tid; idx < C * NS; idx += 256) {
-            const int r = idx / NS, c = idx % NS, t = n * C + r;
-            Vs[r * VS + c] = t < a.T ? ldt<Tin>(a.vt, tok_idx(a, b, t, h) * D + j0 + c) : 0.f;
+        {   // K (C x D) and the Vtilde slice (C x NS), eight elements per load,
+            // every load of a thread issued before its stores
+            constexpr int KU = C * D / 8 / 256, VU = C * NS / 8 / 256;
+            float kx[KU][8], vx[VU > 0 ? VU : 1][8];
+#pragma unroll
+            for (int u = 0; u < KU; ++u) {
+                const int idx = (tid + 256 * u) * 8, r = idx / D, c = idx % D, t = n * C + r;
+                if (t < a.T) ld8<Tin>(a.k, tok_idx(a, b, t, h) * D + c, kx[u]);
+                else for (int e = 0; e < 8; ++e) kx[u][e] = 0.f;
+            }
+            if (tid < C * NS / 8) {
+                const int idx = tid * 8, r = idx / NS, c = idx % NS, t = n * C + r;
+                if (t < a.T) ld8<Tin>(a.vt, tok_idx(a, b, t, h) * D + j0 + c, vx[0]);
+                else for (int e = 0; e < 8; ++e) vx[0][e] = 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < KU; ++u) {
+                const int idx = (tid + 256 * u) * 8, r = idx / D, c = idx % D;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Ks[r * KS + c + e] = kx[u][e];
+            }
+            if (tid < C * NS / 8) {
+                const int idx = tid * 8, r = idx / NS, c = idx % NS;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Vs[r * VS + c + e] = vx[0][e];
+            }
         }
         if (tid < C) {
             const int r = tid, t = n * C + r;
@@ -880,11 +899,14 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
         bwd_prep_kernel<Tin, D><<<(unsigned)chunks, 256, sm0, s>>>(a);
     }
     if ((e = cudaGetLastError())) return e;
-    {
+    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128 && a.bc_u) {
+        // bf16: the chain on tensor cores, after its chunk operands
+        if ((e = launch_bwd_chain_prep(a, s)) || (e = launch_bwd_chain_tc(a, s))) return e;
+    } else {
         ProfScope ps(kBwdChain, s);
         bwd_chain_kernel<Tin, D><<<(unsigned)chains, 256, sm2, s>>>(a);
+        if ((e = cudaGetLastError())) return e;
     }
-    if ((e = cudaGetLastError())) return e;
     if ((e = cudaStreamWaitEvent(s, join, 0))) return e;
     if (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         // bf16 inputs: the six state products on tensor cores

@@ -549,7 +549,191 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     bwd_coeff_phase(a, rec, v, dG, Gp, reinterpret_cast<float*>(sm + L_REC), tid, n, b, h);
 }
 
+// ---------------------------------------------------------------------------
+// The chunk-only operands of the tensor-core reverse chain (bf16, d = 128).
+// With T, Att from B-0, per chunk:
+//   U  = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T]   bf16 [256][64]  (A of U dVtilde)
+//   TT = [T^T ; 0]                                      bf16 [128][64]  (A of T^T dVtilde = dv)
+//   P  = Att^T dO     fp32, slice-major [D/32][64][32]  (dVtilde's chain-free part)
+//   E  = Qhat^T Diag(alphabar) dO,  F = Qhat^T Diag(b) dO   fp32 [2][128][128]
+//   record: Gamma_{C,r} (64), w_r (64), then alphabar_C, b_C, mubar_C at 192..194
+__global__ void __launch_bounds__(kThr, 1)
+bwd_chain_prep_kernel(BwdArgs a)
+{
+    constexpr int KS = D + 1, AS = C + 1;
+    extern __shared__ float fsm[];
+    float* Ks = fsm;              // [C][D+1]
+    float* Qs = Ks + C * KS;      // [C][D+1]  qhat
+    float* Os = Qs + C * KS;      // [C][D+1]  dO
+    float* Tm = Os + C * KS;      // [C][C+1]  T
+    float* At = Tm + C * AS;      // [C][C+1]  Att
+    float* ab = At + C * AS;      // [C] alphabar
+    float* bb = ab + C;           // [C] b
+    float* d2 = bb + C;           // [C] b_{r-1} alpha_r
+    const int tid = threadIdx.x;
+    const int n = blockIdx.x % a.NT;
+    const long long bh = blockIdx.x / a.NT;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const size_t chunk = blockIdx.x, crow = chunk * C;
+    {   // K, qhat, dO tiles and T, Att: every load of a thread before its stores
+        constexpr int U8 = C * D / 8 / kThr;  // 8-element groups per thread and tile
+        float kx[U8][8], qx[U8][8], ox[U8][8];
+#pragma unroll
+        for (int u = 0; u < U8; ++u) {
+            const int idx = (tid + kThr * u) * 8, r = idx / D, c = idx % D, t = n * C + r;
+            if (t < a.T) {
+                const size_t g = tokrow(a, b, t, h) * D + c;
+                ld8<__nv_bfloat16>(a.k, g, kx[u]);
+                ld8<__nv_bfloat16>(a.q, g, qx[u]);
+                ld8<__nv_bfloat16>(a.dout, g, ox[u]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) kx[u][e] = qx[u][e] = ox[u][e] = 0.f;
+            }
+        }
+        constexpr int U4 = C * C / 4 / kThr;
+        float4 tx[U4], ax[U4];
+#pragma unroll
+        for (int u = 0; u < U4; ++u) {
+            const int idx = (tid + kThr * u) * 4;
+            tx[u] = *reinterpret_cast<const float4*>(a.tmat + chunk * C * C + idx);
+            ax[u] = *reinterpret_cast<const float4*>(a.att + chunk * C * C + idx);
+        }
+#pragma unroll
+        for (int u = 0; u < U8; ++u) {
+            const int idx = (tid + kThr * u) * 8, r = idx / D, c = idx % D;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                Ks[r * KS + c + e] = kx[u][e];
+                Qs[r * KS + c + e] = qx[u][e] - a.dcorr * kx[u][e];
+                Os[r * KS + c + e] = ox[u][e];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U4; ++u) {
+            const int idx = (tid + kThr * u) * 4, r = idx / C, i = idx % C;
+            const float tv[4] = {tx[u].x, tx[u].y, tx[u].z, tx[u].w};
+            const float av[4] = {ax[u].x, ax[u].y, ax[u].z, ax[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                Tm[r * AS + i + e] = tv[e];
+                At[r * AS + i + e] = av[e];
+            }
+        }
+    }
+    float* rec = a.bc_rec + chunk * 256;
+    if (tid < C) {
+        const int r = tid, t = n * C + r;
+        const bool in = t < a.T;
+        ab[r] = expf(a.la[crow + r]);
+        bb[r] = a.bco[crow + r];
+        const float al = in ? expf(a.alpha_log[tokrow(a, b, t, h)]) : 1.f;
+        d2[r] = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
+        rec[r] = a.gamma[chunk * C * C + (C - 1) * C + r];
+        const float et = in ? a.eta[tokrow(a, b, t, h)] : 0.f;
+        rec[C + r] = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
+        if (r == 0) {
+            rec[3 * C] = expf(a.la[crow + C - 1]);
+            rec[3 * C + 1] = a.bco[crow + C - 1];
+            rec[3 * C + 2] = expf(a.lm[crow + C - 1]);
+        }
+    }
+    __syncthreads();
+    {   // U: rows i = ig + 64 e (e < 2) of the S and M halves, columns r = rq + 4 m
+        const int ig = tid & 63, rq = tid >> 6;
+        float us[2][16], um[2][16];
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int m = 0; m < 16; ++m) us[e][m] = um[e][m] = 0.f;
+        for (int r2 = 0; r2 < C; ++r2) {
+            const float k0 = Ks[r2 * KS + ig], k1 = Ks[r2 * KS + ig + 64];
+            const float as = -ab[r2], ad = d2[r2];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float tv = Tm[(rq + 4 * m) * AS + r2];  // T^T[r2][r] = T[r][r2]
+                us[0][m] = fmaf(k0 * as, tv, us[0][m]);
+                us[1][m] = fmaf(k1 * as, tv, us[1][m]);
+                um[0][m] = fmaf(k0 * ad, tv, um[0][m]);
+                um[1][m] = fmaf(k1 * ad, tv, um[1][m]);
+            }
+        }
+        __nv_bfloat16* U = a.bc_u + chunk * 256 * 64;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int i = ig + 64 * e, r = rq + 4 * m;
+                U[i * 64 + r] = __float2bfloat16_rn(us[e][m]);
+                U[(128 + i) * 64 + r] = __float2bfloat16_rn(um[e][m]);
+            }
+    }
+    {   // [T^T; 0]
+        __nv_bfloat16* TT = a.bc_tt + chunk * 128 * 64;
+        for (int idx = tid; idx < 128 * 64; idx += kThr) {
+            const int r = idx >> 6, r2 = idx & 63;
+            TT[idx] = __float2bfloat16_rn(r < C ? Tm[r2 * AS + r] : 0.f);
+        }
+    }
+    {   // P = Att^T dO, columns j = tid & 127, rows r = (tid >> 7) + 2 m, slice-major
+        const int j = tid & 127, rh = tid >> 7;
+        float acc[32];
+#pragma unroll
+        for (int m = 0; m < 32; ++m) acc[m] = 0.f;
+        for (int r2 = 0; r2 < C; ++r2) {
+            const float ov = Os[r2 * KS + j];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) acc[m] = fmaf(At[r2 * AS + rh + 2 * m], ov, acc[m]);
+        }
+        float* P = a.bc_p + chunk * C * D;
+        const int sl = j >> 5, jj = j & 31;
+#pragma unroll
+        for (int m = 0; m < 32; ++m) P[(sl * C + rh + 2 * m) * 32 + jj] = acc[m];
+    }
+    // E, F: rows i = ig + 16 u, columns j = jg + 16 v (8 x 8 per thread), one after the other
+    const int ig = tid & 15, jg = tid >> 4;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+        const float* coef = which == 0 ? ab : bb;
+        float acc[8][8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
+        for (int r = 0; r < C; ++r) {
+            const float cr = coef[r];
+            float qv[8], ov[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) qv[u] = Qs[r * KS + ig + 16 * u] * cr;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) ov[v] = Os[r * KS + jg + 16 * v];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(qv[u], ov[v], acc[u][v]);
+        }
+        float* Mx = a.bc_ef + (chunk * 2 + which) * D * D;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) Mx[(ig + 16 * u) * D + jg + 16 * v] = acc[u][v];
+    }
+}
+
+
 }  // namespace
+
+cudaError_t launch_bwd_chain_prep(const BwdArgs& a, cudaStream_t s)
+{
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    const size_t smem = sizeof(float) * (3 * C * (D + 1) + 2 * C * (C + 1) + 3 * C);
+    cudaError_t e = cudaFuncSetAttribute(bwd_chain_prep_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ProfScope ps(kBwdChainPrep, s);
+    bwd_chain_prep_kernel<<<(unsigned)chunks, kThr, smem, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
 {

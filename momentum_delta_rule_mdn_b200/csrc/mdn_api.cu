@@ -257,10 +257,13 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 namespace {
 
 struct BwdLayout {
-    size_t status, la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec, total;
+    size_t status, la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec;
+    size_t bc_u, bc_tt, bc_p, bc_ef, bc_rec;  // tensor-core reverse chain (bf16, d = 128)
+    size_t total;
 };
 
-BwdLayout bwd_layout(long long BH, int NT, int D)
+// tc: the tensor-core reverse chain's chunk operands are included.
+BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
 {
     const size_t chunks = (size_t)BH * NT, rows = chunks * kChunk;
     BwdLayout w;
@@ -276,6 +279,14 @@ BwdLayout bwd_layout(long long BH, int NT, int D)
     w.SS = off;    off += align_up(chunks * 2 * D * D * sizeof(float));
     w.dSS = off;   off += align_up(chunks * 2 * D * D * sizeof(float));
     w.rec = off;   off += align_up(chunks * kBwdRec * sizeof(float));
+    w.bc_u = w.bc_tt = w.bc_p = w.bc_ef = w.bc_rec = 0;
+    if (tc) {
+        w.bc_u = off;   off += align_up(chunks * 256 * 64 * 2);
+        w.bc_tt = off;  off += align_up(chunks * 128 * 64 * 2);
+        w.bc_p = off;   off += align_up(chunks * kChunk * D * sizeof(float));
+        w.bc_ef = off;  off += align_up(chunks * 2 * D * D * sizeof(float));
+        w.bc_rec = off; off += align_up(chunks * 256 * sizeof(float));
+    }
     w.total = off;
     return w;
 }
@@ -286,7 +297,7 @@ size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
                                     mdn_dtype in_dtype)
 {
     if (check_sizes(B, T, H, dk, dv, C, in_dtype) != MDN_OK) return 0;
-    return bwd_layout((long long)B * H, (T + C - 1) / C, dk).total;
+    return bwd_layout((long long)B * H, (T + C - 1) / C, dk, in_dtype == MDN_BF16 && dk == 128).total;
 }
 
 mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
@@ -317,7 +328,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
             if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
     }
     const int NT = (T + C - 1) / C;
-    const BwdLayout w = bwd_layout((long long)B * H, NT, D);
+    const BwdLayout w = bwd_layout((long long)B * H, NT, D, in_dtype == MDN_BF16 && D == 128);
     if (T > 0 && (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign))
         return MDN_ERR_INVALID_ARG;
     if (T > 0 && ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
@@ -349,6 +360,12 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.SS = reinterpret_cast<float*>(ws + w.SS);
     a.dSS = reinterpret_cast<float*>(ws + w.dSS);
     a.crec_bw = reinterpret_cast<float*>(ws + w.rec);
+    const bool tc = in_dtype == MDN_BF16 && D == 128;
+    a.bc_u = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_u) : nullptr;
+    a.bc_tt = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_tt) : nullptr;
+    a.bc_p = tc ? reinterpret_cast<float*>(ws + w.bc_p) : nullptr;
+    a.bc_ef = tc ? reinterpret_cast<float*>(ws + w.bc_ef) : nullptr;
+    a.bc_rec = tc ? reinterpret_cast<float*>(ws + w.bc_rec) : nullptr;
     a.dq = dq; a.dk = dk_out; a.dv = dv_out;
     a.dalpha_log = dalpha_log; a.dmu_log = dmu_log; a.dbeta = dbeta; a.deta = deta;
     a.dS0 = dS0; a.dM0 = dM0;

@@ -146,6 +146,12 @@ struct BwdArgs {
     float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk
     float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk
     float* crec_bw;  // [B*H*NT, kBwdRec]  coefficient adjoints from the state products
+    // chunk-only operands of the tensor-core reverse chain (null on the CUDA-core path)
+    __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]
+    __nv_bfloat16* bc_tt;  // [B*H*NT, 128, 64]  [T^T; 0]
+    float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
+    float* bc_ef;          // [B*H*NT, 2, D, D]  Qhat^T Diag(alphabar) dO, Qhat^T Diag(b) dO
+    float* bc_rec;         // [B*H*NT, 256]  Gamma_C, w, then alphabar_C, b_C, mubar_C
     // outputs (fp32)
     float* dq;
     float* dk;
@@ -238,7 +244,7 @@ __device__ __forceinline__ ChunkOut chunk_out(const ChunkArgs& a, int b, int n)
 enum KernelKind {
     kGatePrep = 0, kIntraSimt, kInterSimt, kOutputSimt, kStep, kFiniteCheck,
     kChunkTc, kIntraTc, kInterTc, kOutputTc, kGateParams, kVarlen, kBwdPrep, kBwdStates,
-    kBwdChain, kBwdStateGrads, kBwdLocal, kKernelKinds
+    kBwdChain, kBwdStateGrads, kBwdLocal, kBwdChainPrep, kKernelKinds
 };
 // Record a start event for a launch of kind k on s (returns a slot, or -1 when
 // timing is off); prof_end records the matching stop event.
@@ -262,6 +268,9 @@ cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, mdn_dtype dt, cudaStream_t s
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s);
 // B-3b of the backward pass on tcgen05 (bf16 inputs, d = 128).
 cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s);
+// The tensor-core reverse chain (bf16, d = 128): its chunk-only operands, then the chain.
+cudaError_t launch_bwd_chain_prep(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and

@@ -33,7 +33,7 @@ Profiler& prof() {
 const char* const kNames[kKernelKinds] = {
     "gate_prep", "intra_simt", "inter_simt", "output_simt", "step", "finite_check",
     "chunk_tc", "intra_tc", "inter_tc", "output_tc", "gate_params", "varlen_prep", "bwd_prep", "bwd_states", "bwd_chain",
-    "bwd_state_grads", "bwd_local_grads",
+    "bwd_state_grads", "bwd_local_grads", "bwd_chain_prep",
 };
 
 // Fold every recorded pair into the totals (caller holds the lock).
