@@ -871,6 +871,21 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     MDN_SET_SMEM((bwd_state_grads_kernel<Tin, D>), sm3a)
     MDN_SET_SMEM((bwd_local_grads_kernel<Tin, D>), sm3b)
 #undef MDN_SET_SMEM
+    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128 && a.bc_u) {
+        // bf16, d = 128: T and Att on CUDA cores, then the chain's operands and
+        // the rebuild increments on tensor cores, the entering states by an
+        // elementwise scan, the reverse chain and both per-chunk product
+        // kernels on tensor cores
+        {
+            ProfScope ps(kBwdPrep, s);
+            bwd_prep_kernel<Tin, D><<<(unsigned)chunks, 256, sm0, s>>>(a);
+        }
+        if ((e = cudaGetLastError())) return e;
+        if ((e = launch_bwd_chain_prep_tc(a, s))) return e;
+        if ((e = launch_bwd_chain_tc(a, s))) return e;
+        if ((e = launch_bwd_state_grads_tc(a, s))) return e;
+        return launch_bwd_local_grads_tc(a, s);
+    }
     // The state rebuild depends only on the chunk coefficients and is needed
     // only by B-3a: it runs on a side stream, beside B-0 and the reverse chain
     // (both chains leave most of each SM idle), and joins before B-3a.
@@ -899,26 +914,18 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
         bwd_prep_kernel<Tin, D><<<(unsigned)chunks, 256, sm0, s>>>(a);
     }
     if ((e = cudaGetLastError())) return e;
-    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128 && a.bc_u) {
-        // bf16: the chain on tensor cores, after its chunk operands
-        if ((e = launch_bwd_chain_prep(a, s)) || (e = launch_bwd_chain_tc(a, s))) return e;
-    } else {
+    {
         ProfScope ps(kBwdChain, s);
         bwd_chain_kernel<Tin, D><<<(unsigned)chains, 256, sm2, s>>>(a);
-        if ((e = cudaGetLastError())) return e;
     }
+    if ((e = cudaGetLastError())) return e;
     if ((e = cudaStreamWaitEvent(s, join, 0))) return e;
-    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
-        // bf16 inputs: the six state products on tensor cores
-        if ((e = launch_bwd_state_grads_tc(a, s))) return e;
-    } else {
+    {
         ProfScope ps(kBwdStateGrads, s);
         bwd_state_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3a, s>>>(a);
-        if ((e = cudaGetLastError())) return e;
     }
-    if (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
-        if ((e = launch_bwd_local_grads_tc(a, s))) return e;
-    } else {
+    if ((e = cudaGetLastError())) return e;
+    {
         ProfScope ps(kBwdLocal, s);
         bwd_local_grads_kernel<Tin, D><<<(unsigned)chunks, 256, sm3b, s>>>(a);
     }

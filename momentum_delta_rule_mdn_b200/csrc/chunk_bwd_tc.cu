@@ -550,48 +550,141 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 }
 
 // ---------------------------------------------------------------------------
-// The chunk-only operands of the tensor-core reverse chain (bf16, d = 128).
-// With T, Att from B-0, per chunk:
+// The chunk-only operands of the tensor-core reverse chain (bf16, d = 128):
 //   U  = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T]   bf16 [256][64]  (A of U dVtilde)
 //   TT = [T^T ; 0]                                      bf16 [128][64]  (A of T^T dVtilde = dv)
 //   P  = Att^T dO     fp32, slice-major [D/32][64][32]  (dVtilde's chain-free part)
 //   E  = Qhat^T Diag(alphabar) dO,  F = Qhat^T Diag(b) dO   fp32 [2][128][128]
 //   record: Gamma_{C,r} (64), w_r (64), then alphabar_C, b_C, mubar_C at 192..194
+// plus the increments of the state rebuild, D_S = K^T Diag(Gamma_C) Vtilde and
+// D_M = K^T Diag(w) Vtilde, which turn the rebuild into an elementwise scan
+// over the chunks.  Products
+// (A operands K-major, transposed while they are staged):
+//   E = Qhat^T (Diag(alphabar) dO), F = Qhat^T (Diag(b) dO)    M 128, N 128, K 64
+//   U = K^T [Diag(-alphabar) T^T | Diag(D2) T^T]                M 128, N 64 + 64
+//   P = Att^T dO                                                 M 64 (of 128), N 128
+//   D = K^T [Diag(Gamma_C) Vtilde | Diag(w) Vtilde]             M 128, N 128 + 128 (second round)
+constexpr uint32_t PA_QT = 0;        // Qhat^T  [128 i][64 r]  K-major, 16 KB
+constexpr uint32_t PA_KT = 16384;    // K^T     [128 i][64 r]
+constexpr uint32_t PA_AT = 32768;    // Att^T   [128 r (64 used)][64 r2]
+constexpr uint32_t PB_OA = 49152;    // Diag(alphabar) dO  [64 r][128 j]  MN-major: 2 N-panels x 64 rows
+constexpr uint32_t PB_OB = 65536;    // Diag(b) dO
+constexpr uint32_t PB_O = 81920;     // dO
+constexpr uint32_t PB_VG = 98304;    // Diag(Gamma_C) Vtilde
+constexpr uint32_t PB_VW = 114688;   // Diag(w) Vtilde
+constexpr uint32_t PB_TS = 131072;   // -alphabar_{r2} T[r][r2]  [64 r][64 r2]  K-major, 8 KB
+constexpr uint32_t PB_TM = 139264;   //  D2_{r2} T[r][r2]
+constexpr uint32_t P_VEC = 147456;   // alphabar, b, D2, Gamma_C, w
+constexpr uint32_t P_BAR = P_VEC + 1280;
+constexpr uint32_t P_MISC = P_BAR + 16;
+constexpr uint32_t P_SMEM = P_MISC + 16 + 1024;
+
+// byte offset of element (row, col) of an MN-major tile with 64-element
+// column panels of `rows` rows (128-byte swizzle)
+__device__ __forceinline__ uint32_t mn_off(int row, int col, int rows) {
+    return (col >> 6) * rows * 128 + sw128_off(row, (col & 63) >> 3) + (col & 7) * 2;
+}
+
 __global__ void __launch_bounds__(kThr, 1)
-bwd_chain_prep_kernel(BwdArgs a)
+bwd_chain_prep_tc_kernel(BwdArgs a)
 {
-    constexpr int KS = D + 1, AS = C + 1;
-    extern __shared__ float fsm[];
-    float* Ks = fsm;              // [C][D+1]
-    float* Qs = Ks + C * KS;      // [C][D+1]  qhat
-    float* Os = Qs + C * KS;      // [C][D+1]  dO
-    float* Tm = Os + C * KS;      // [C][C+1]  T
-    float* At = Tm + C * AS;      // [C][C+1]  Att
-    float* ab = At + C * AS;      // [C] alphabar
-    float* bb = ab + C;           // [C] b
-    float* d2 = bb + C;           // [C] b_{r-1} alpha_r
-    const int tid = threadIdx.x;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x % a.NT;
     const long long bh = blockIdx.x / a.NT;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x, crow = chunk * C;
-    {   // K, qhat, dO tiles and T, Att: every load of a thread before its stores
-        constexpr int U8 = C * D / 8 / kThr;  // 8-element groups per thread and tile
-        float kx[U8][8], qx[U8][8], ox[U8][8];
+    float* v_ab = reinterpret_cast<float*>(sm + P_VEC);
+    float* v_b = v_ab + C;
+    float* v_d2 = v_b + C;
+    float* v_g = v_d2 + C;
+    float* v_w = v_g + C;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P_MISC);
+    float* rec = a.bc_rec + chunk * 256;
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (tid < C) {
+        const int r = tid, t = n * C + r;
+        const bool in = t < a.T;
+        const float ab = expf(a.la[crow + r]);
+        const float al = in ? expf(a.alpha_log[tokrow(a, b, t, h)]) : 1.f;
+        const float gl = a.gamma[chunk * C * C + (C - 1) * C + r];
+        const float et = in ? a.eta[tokrow(a, b, t, h)] : 0.f;
+        const float w = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
+        v_ab[r] = ab;
+        v_b[r] = a.bco[crow + r];
+        v_d2[r] = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
+        v_g[r] = gl;
+        v_w[r] = w;
+        rec[r] = gl;
+        rec[C + r] = w;
+        if (r == 0) {
+            rec[3 * C] = expf(a.la[crow + C - 1]);
+            rec[3 * C + 1] = a.bco[crow + C - 1];
+            rec[3 * C + 2] = expf(a.lm[crow + C - 1]);
+        }
+    }
+    // rows 64..127 of Att^T are zero
+    for (int i = tid; i < 512; i += kThr)
+        *reinterpret_cast<uint4*>(sm + PA_AT + 8192 + i * 16) = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    // token tiles: 64 rows x 16 groups of 8; the loads of a thread before its stores
+    {
+        constexpr int U8 = C * 16 / kThr;  // 4
+        float kx[U8][8], qx[U8][8], ox[U8][8], vx[U8][8];
 #pragma unroll
         for (int u = 0; u < U8; ++u) {
-            const int idx = (tid + kThr * u) * 8, r = idx / D, c = idx % D, t = n * C + r;
+            const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8, t = n * C + r;
             if (t < a.T) {
-                const size_t g = tokrow(a, b, t, h) * D + c;
+                const size_t g = tokrow(a, b, t, h) * D + c8;
                 ld8<__nv_bfloat16>(a.k, g, kx[u]);
                 ld8<__nv_bfloat16>(a.q, g, qx[u]);
                 ld8<__nv_bfloat16>(a.dout, g, ox[u]);
+                ld8<__nv_bfloat16>(a.vt, g, vx[u]);
             } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) kx[u][e] = qx[u][e] = ox[u][e] = 0.f;
+                for (int e = 0; e < 8; ++e) kx[u][e] = qx[u][e] = ox[u][e] = vx[u][e] = 0.f;
             }
         }
-        constexpr int U4 = C * C / 4 / kThr;
+#pragma unroll
+        for (int u = 0; u < U8; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8;
+            const float ab = v_ab[r], bb = v_b[r], gl = v_g[r], w = v_w[r];
+            float oa[8], ob[8], vg[8], vw[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float qh = qx[u][e] - a.dcorr * kx[u][e];
+                // transposed into the K-major A operands
+                st_bf16(sm + PA_QT + kmaj_off(c8 + e, r, 16384), qh);
+                st_bf16(sm + PA_KT + kmaj_off(c8 + e, r, 16384), kx[u][e]);
+                oa[e] = ab * ox[u][e];
+                ob[e] = bb * ox[u][e];
+                vg[e] = gl * vx[u][e];
+                vw[e] = w * vx[u][e];
+            }
+            const uint32_t o = mn_off(r, c8, 64);
+            st_bf16x8(sm + PB_OA + o, oa);
+            st_bf16x8(sm + PB_OB + o, ob);
+            st_bf16x8(sm + PB_O + o, ox[u]);
+            st_bf16x8(sm + PB_VG + o, vg);
+            st_bf16x8(sm + PB_VW + o, vw);
+        }
+    }
+    // T and Att: the scaled T tiles (K-major), Att^T (K-major), and [T^T; 0] to global
+    {
+        constexpr int U4 = C * C / 4 / kThr;  // 4
         float4 tx[U4], ax[U4];
 #pragma unroll
         for (int u = 0; u < U4; ++u) {
@@ -599,141 +692,166 @@ bwd_chain_prep_kernel(BwdArgs a)
             tx[u] = *reinterpret_cast<const float4*>(a.tmat + chunk * C * C + idx);
             ax[u] = *reinterpret_cast<const float4*>(a.att + chunk * C * C + idx);
         }
-#pragma unroll
-        for (int u = 0; u < U8; ++u) {
-            const int idx = (tid + kThr * u) * 8, r = idx / D, c = idx % D;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                Ks[r * KS + c + e] = kx[u][e];
-                Qs[r * KS + c + e] = qx[u][e] - a.dcorr * kx[u][e];
-                Os[r * KS + c + e] = ox[u][e];
-            }
-        }
+        __nv_bfloat16* TT = a.bc_tt + chunk * 128 * 64;
 #pragma unroll
         for (int u = 0; u < U4; ++u) {
-            const int idx = (tid + kThr * u) * 4, r = idx / C, i = idx % C;
+            const int idx = (tid + kThr * u) * 4, r = idx / C, r2 = idx % C;
             const float tv[4] = {tx[u].x, tx[u].y, tx[u].z, tx[u].w};
             const float av[4] = {ax[u].x, ax[u].y, ax[u].z, ax[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                Tm[r * AS + i + e] = tv[e];
-                At[r * AS + i + e] = av[e];
+                st_bf16(sm + PB_TS + kmaj_off(r, r2 + e, 8192), -v_ab[r2 + e] * tv[e]);
+                st_bf16(sm + PB_TM + kmaj_off(r, r2 + e, 8192), v_d2[r2 + e] * tv[e]);
+                st_bf16(sm + PA_AT + kmaj_off(r2 + e, r, 16384), av[e]);  // Att^T[r2 + e][r]
+                TT[(r2 + e) * 64 + r] = __float2bfloat16_rn(tv[e]);       // T^T
             }
         }
+        for (int i = tid; i < 64 * 64; i += kThr) TT[64 * 64 + i] = __float2bfloat16_rn(0.f);
     }
-    float* rec = a.bc_rec + chunk * 256;
-    if (tid < C) {
-        const int r = tid, t = n * C + r;
-        const bool in = t < a.T;
-        ab[r] = expf(a.la[crow + r]);
-        bb[r] = a.bco[crow + r];
-        const float al = in ? expf(a.alpha_log[tokrow(a, b, t, h)]) : 1.f;
-        d2[r] = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
-        rec[r] = a.gamma[chunk * C * C + (C - 1) * C + r];
-        const float et = in ? a.eta[tokrow(a, b, t, h)] : 0.f;
-        rec[C + r] = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
-        if (r == 0) {
-            rec[3 * C] = expf(a.la[crow + C - 1]);
-            rec[3 * C + 1] = a.bco[crow + C - 1];
-            rec[3 * C + 2] = expf(a.lm[crow + C - 1]);
-        }
-    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
     __syncthreads();
-    {   // U: rows i = ig + 64 e (e < 2) of the S and M halves, columns r = rq + 4 m
-        const int ig = tid & 63, rq = tid >> 6;
-        float us[2][16], um[2][16];
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        constexpr uint32_t idmn = idesc_bf16(128, 128, false, true);
+        constexpr uint32_t idk = idesc_bf16(128, 64, false, false);
 #pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int m = 0; m < 16; ++m) us[e][m] = um[e][m] = 0.f;
-        for (int r2 = 0; r2 < C; ++r2) {
-            const float k0 = Ks[r2 * KS + ig], k1 = Ks[r2 * KS + ig + 64];
-            const float as = -ab[r2], ad = d2[r2];
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float tv = Tm[(rq + 4 * m) * AS + r2];  // T^T[r2][r] = T[r][r2]
-                us[0][m] = fmaf(k0 * as, tv, us[0][m]);
-                us[1][m] = fmaf(k1 * as, tv, us[1][m]);
-                um[0][m] = fmaf(k0 * ad, tv, um[0][m]);
-                um[1][m] = fmaf(k1 * ad, tv, um[1][m]);
-            }
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t aq = smem_desc(sbase + PA_QT + ks * 32, 16, 1024, kSw128);
+            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
+            const uint64_t aa = smem_desc(sbase + PA_AT + ks * 32, 16, 1024, kSw128);
+            mma_bf16(tmem, aq, smem_desc(sbase + PB_OA + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
+            mma_bf16(tmem + 128, aq, smem_desc(sbase + PB_OB + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
+            mma_bf16(tmem + 256, ak, smem_desc(sbase + PB_TS + ks * 32, 16, 1024, kSw128), idk, ks > 0);
+            mma_bf16(tmem + 320, ak, smem_desc(sbase + PB_TM + ks * 32, 16, 1024, kSw128), idk, ks > 0);
+            mma_bf16(tmem + 384, aa, smem_desc(sbase + PB_O + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
         }
-        __nv_bfloat16* U = a.bc_u + chunk * 256 * 64;
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const int i = ig + 64 * e, r = rq + 4 * m;
-                U[i * 64 + r] = __float2bfloat16_rn(us[e][m]);
-                U[(128 + i) * 64 + r] = __float2bfloat16_rn(um[e][m]);
-            }
+        mma_commit(&bars[0]);
     }
-    {   // [T^T; 0]
-        __nv_bfloat16* TT = a.bc_tt + chunk * 128 * 64;
-        for (int idx = tid; idx < 128 * 64; idx += kThr) {
-            const int r = idx >> 6, r2 = idx & 63;
-            TT[idx] = __float2bfloat16_rn(r < C ? Tm[r2 * AS + r] : 0.f);
-        }
-    }
-    {   // P = Att^T dO, columns j = tid & 127, rows r = (tid >> 7) + 2 m, slice-major
-        const int j = tid & 127, rh = tid >> 7;
-        float acc[32];
-#pragma unroll
-        for (int m = 0; m < 32; ++m) acc[m] = 0.f;
-        for (int r2 = 0; r2 < C; ++r2) {
-            const float ov = Os[r2 * KS + j];
-#pragma unroll
-            for (int m = 0; m < 32; ++m) acc[m] = fmaf(At[r2 * AS + rh + 2 * m], ov, acc[m]);
-        }
-        float* P = a.bc_p + chunk * C * D;
-        const int sl = j >> 5, jj = j & 31;
-#pragma unroll
-        for (int m = 0; m < 32; ++m) P[(sl * C + rh + 2 * m) * 32 + jj] = acc[m];
-    }
-    // E, F: rows i = ig + 16 u, columns j = jg + 16 v (8 x 8 per thread), one after the other
-    const int ig = tid & 15, jg = tid >> 4;
+    bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
+    tc_fence_after_sync();
+    const int quad = warp & 3, half = warp >> 2;
+    const int R = quad * 32 + lane;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    if (ok) {
+        // E, F: row i = R, columns [64 half, 64 half + 64)
+        float* Eo = a.bc_ef + (chunk * 2) * D * D + (size_t)R * D;
 #pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-        const float* coef = which == 0 ? ab : bb;
-        float acc[8][8];
+        for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
+            float e16[16], f16[16];
+            tmem_ld16(tq + k0, e16);
+            tmem_ld16(tq + 128 + k0, f16);
+            tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-#pragma unroll
-            for (int v = 0; v < 8; ++v) acc[u][v] = 0.f;
-        for (int r = 0; r < C; ++r) {
-            const float cr = coef[r];
-            float qv[8], ov[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) qv[u] = Qs[r * KS + ig + 16 * u] * cr;
-#pragma unroll
-            for (int v = 0; v < 8; ++v) ov[v] = Os[r * KS + jg + 16 * v];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(qv[u], ov[v], acc[u][v]);
+            for (int q = 0; q < 4; ++q) {
+                *reinterpret_cast<float4*>(Eo + k0 + 4 * q) =
+                    make_float4(e16[4 * q], e16[4 * q + 1], e16[4 * q + 2], e16[4 * q + 3]);
+                *reinterpret_cast<float4*>(Eo + D * D + k0 + 4 * q) =
+                    make_float4(f16[4 * q], f16[4 * q + 1], f16[4 * q + 2], f16[4 * q + 3]);
+            }
         }
-        float* Mx = a.bc_ef + (chunk * 2 + which) * D * D;
+        // U: row i = R of the S half (half 0) or of the M half (half 1)
+        {
+            float u32[32];
+            uint4* Uo = reinterpret_cast<uint4*>(a.bc_u + chunk * 256 * 64 + (size_t)(128 * half + R) * 64);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+            for (int g = 0; g < 2; ++g) {
+                tmem_ld32(tq + 256 + 64 * half + 32 * g, u32);
+                tmem_wait_ld();
 #pragma unroll
-            for (int v = 0; v < 8; ++v) Mx[(ig + 16 * u) * D + jg + 16 * v] = acc[u][v];
+                for (int q = 0; q < 4; ++q) Uo[4 * g + q] = bf16x8(u32 + 8 * q);
+            }
+        }
+        // P = Att^T dO: rows r = R < 64, columns [64 half, 64 half + 64), by 32-column slice
+        if (R < 64) {
+            float* Po = a.bc_p + chunk * C * D;
+#pragma unroll 1
+            for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
+                float p16[16];
+                tmem_ld16(tq + 384 + k0, p16);
+                tmem_wait_ld();
+                const int sl = k0 >> 5, jj = k0 & 31;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4*>(Po + (sl * C + R) * 32 + jj + 4 * q) =
+                        make_float4(p16[4 * q], p16[4 * q + 1], p16[4 * q + 2], p16[4 * q + 3]);
+            }
+        }  // (R < 64 is warp-uniform: quadrants 0, 1)
     }
+    // second round: the rebuild increments into the columns of E and F
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (tid == 0 && ok) {
+        constexpr uint32_t idmn = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
+            mma_bf16(tmem, ak, smem_desc(sbase + PB_VG + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
+            mma_bf16(tmem + 128, ak, smem_desc(sbase + PB_VW + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
+        }
+        mma_commit(&bars[1]);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
+    tc_fence_after_sync();
+    if (ok) {
+        float* Do = a.bc_d + (chunk * 2) * D * D + (size_t)R * D;
+#pragma unroll 1
+        for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
+            float s16[16], m16[16];
+            tmem_ld16(tq + k0, s16);
+            tmem_ld16(tq + 128 + k0, m16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                *reinterpret_cast<float4*>(Do + k0 + 4 * q) =
+                    make_float4(s16[4 * q], s16[4 * q + 1], s16[4 * q + 2], s16[4 * q + 3]);
+                *reinterpret_cast<float4*>(Do + D * D + k0 + 4 * q) =
+                    make_float4(m16[4 * q], m16[4 * q + 1], m16[4 * q + 2], m16[4 * q + 3]);
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+    if (!ok && tid == 0) atomicOr(a.status + 1, 1u);
 }
 
+// The states entering every chunk by the elementwise recurrence
+// S <- alphabar_C S - b_C M + D_S, M <- mubar_C M - D_M (one element of a
+// head's d x d states per lane group of four).
+__global__ void __launch_bounds__(256)
+bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0,
+                      const float* __restrict__ dinc, const float* __restrict__ rec,
+                      float* __restrict__ SS, int NT, long long heads)
+{
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long per = D * D / 4;
+    if (gid >= heads * per) return;
+    const long long bh = gid / per;
+    const int e4 = (int)(gid % per) * 4;
+    float4 s = S0 ? *reinterpret_cast<const float4*>(S0 + bh * D * D + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 m = M0 ? *reinterpret_cast<const float4*>(M0 + bh * D * D + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int nn = 0; nn < NT; ++nn) {
+        const size_t chunk = (size_t)bh * NT + nn;
+        const float4 ds = __ldg(reinterpret_cast<const float4*>(dinc + chunk * 2 * D * D + e4));
+        const float4 dm = __ldg(reinterpret_cast<const float4*>(dinc + chunk * 2 * D * D + D * D + e4));
+        const float aC = __ldg(rec + chunk * 256 + 3 * C), bC = __ldg(rec + chunk * 256 + 3 * C + 1);
+        const float mC = __ldg(rec + chunk * 256 + 3 * C + 2);
+        *reinterpret_cast<float4*>(SS + chunk * 2 * D * D + e4) = s;
+        *reinterpret_cast<float4*>(SS + chunk * 2 * D * D + D * D + e4) = m;
+        s = make_float4(aC * s.x - bC * m.x + ds.x, aC * s.y - bC * m.y + ds.y,
+                        aC * s.z - bC * m.z + ds.z, aC * s.w - bC * m.w + ds.w);
+        m = make_float4(mC * m.x - dm.x, mC * m.y - dm.y, mC * m.z - dm.z, mC * m.w - dm.w);
+    }
+}
 
 }  // namespace
 
-cudaError_t launch_bwd_chain_prep(const BwdArgs& a, cudaStream_t s)
-{
-    const long long chunks = (long long)a.B * a.H * a.NT;
-    const size_t smem = sizeof(float) * (3 * C * (D + 1) + 2 * C * (C + 1) + 3 * C);
-    cudaError_t e = cudaFuncSetAttribute(bwd_chain_prep_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ProfScope ps(kBwdChainPrep, s);
-    bwd_chain_prep_kernel<<<(unsigned)chunks, kThr, smem, s>>>(a);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
 {
@@ -762,6 +880,31 @@ cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     ProfScope ps(kBwdLocal, s);
     bwd_local_grads_tc_kernel<<<(unsigned)chunks, kThr, L_SMEM, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace mdn
+
+namespace mdn {
+
+cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s)
+{
+    if (a.D != D) return cudaErrorNotSupported;
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    cudaError_t e = cudaFuncSetAttribute(bwd_chain_prep_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)P_SMEM);
+    if (e != cudaSuccess) return e;
+    {
+        ProfScope ps(kBwdChainPrep, s);
+        bwd_chain_prep_tc_kernel<<<(unsigned)chunks, kThr, P_SMEM, s>>>(a);
+    }
+    if ((e = cudaGetLastError())) return e;
+    const long long heads = (long long)a.B * a.H;
+    const long long threads = heads * D * D / 4;
+    ProfScope ps(kBwdStates, s);
+    bwd_state_scan_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+        a.S0, a.M0, a.bc_d, a.bc_rec, a.SS, a.NT, heads);
     return cudaGetLastError();
 }
 

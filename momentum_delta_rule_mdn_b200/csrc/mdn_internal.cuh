@@ -152,6 +152,7 @@ struct BwdArgs {
     float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
     float* bc_ef;          // [B*H*NT, 2, D, D]  Qhat^T Diag(alphabar) dO, Qhat^T Diag(b) dO
     float* bc_rec;         // [B*H*NT, 256]  Gamma_C, w, then alphabar_C, b_C, mubar_C
+    float* bc_d;           // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde
     // outputs (fp32)
     float* dq;
     float* dk;
@@ -268,9 +269,10 @@ cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, mdn_dtype dt, cudaStream_t s
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s);
 // B-3b of the backward pass on tcgen05 (bf16 inputs, d = 128).
 cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s);
-// The tensor-core reverse chain (bf16, d = 128): its chunk-only operands, then the chain.
-cudaError_t launch_bwd_chain_prep(const BwdArgs& a, cudaStream_t s);
+// The tensor-core reverse chain (bf16, d = 128).
 cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s);
+// tcgen05 version of the chain's operands plus the rebuilt entering states (a scan).
+cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and
