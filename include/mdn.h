@@ -171,8 +171,9 @@ size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   workspace   at least mdn_chunk_bwd_workspace_size(...) bytes, 256-byte
  *               aligned (about (4 d^2 + 3 C^2 + 10 C) x 4 bytes per chunk of C
  *               tokens of each head).
- *   flags       0 or MDN_CHECK_FINITE (synchronise, then report non-finite
- *               outputs or an expired device wait).
+ *   flags       0, or MDN_CHECK_FINITE (synchronise, then report non-finite
+ *               outputs or an expired device wait) and/or MDN_FORCE_SIMT (the
+ *               CUDA-core kernels for bf16 d = 128 too).
  *
  * bf16 inputs with d = 128 run the products with the states on tcgen05
  * tensor cores (bf16 operands, fp32 accumulation); everything else, and

@@ -130,7 +130,7 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0
 
 def chunk_bwd(q, k, v, alpha_log, mu_log, beta, eta, d: float, vtilde, d_o, S0=None, M0=None,
               dS_T=None, dM_T=None, C: int = 64, *, workspace: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None) -> dict:
+              flags: int = 0, stream: Optional[torch.cuda.Stream] = None) -> dict:
     """Backward pass of :func:`chunk_fwd` from its saved ``vtilde``.  Returns a
     dict of fp32 tensors: dq, dk, dv, dalpha_log, dmu_log, dbeta, deta, dS0, dM0."""
     B, T, H, D = q.shape
@@ -154,7 +154,7 @@ def chunk_bwd(q, k, v, alpha_log, mu_log, beta, eta, d: float, vtilde, d_o, S0=N
         float(d), _ptr(S0), _ptr(M0), _ptr(vtilde), _ptr(d_o), _ptr(dS_T), _ptr(dM_T),
         B, T, H, D, D, C, *(_ptr(g[n]) for n in ("dq", "dk", "dv", "dalpha_log", "dmu_log",
                                                   "dbeta", "deta", "dS0", "dM0")),
-        _ptr(workspace), workspace.numel(), 0, _stream_handle(stream))
+        _ptr(workspace), workspace.numel(), int(flags), _stream_handle(stream))
     _check(status, "mdn_chunk_bwd")
     return g
 

@@ -312,7 +312,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
 {
     mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
     if (st != MDN_OK) return st;
-    if (flags & ~MDN_CHECK_FINITE) return MDN_ERR_INVALID_ARG;
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT)) return MDN_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return MDN_OK;
     if (!dS0 || !dM0 || !aligned16(dS0) || !aligned16(dM0)) return MDN_ERR_INVALID_ARG;
     const void* opt[] = {S0, M0, dS_T, dM_T};
@@ -361,7 +361,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.SS = reinterpret_cast<float*>(ws + w.SS);
     a.dSS = reinterpret_cast<float*>(ws + w.dSS);
     a.crec_bw = reinterpret_cast<float*>(ws + w.rec);
-    const bool tc = in_dtype == MDN_BF16 && D == 128;
+    const bool tc = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
     a.bc_u = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_u) : nullptr;
     a.bc_tt = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_tt) : nullptr;
     a.bc_p = tc ? reinterpret_cast<float*>(ws + w.bc_p) : nullptr;

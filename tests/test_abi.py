@@ -184,7 +184,7 @@ def test_bwd_workspace_and_validation(lib):
         return lib.mdn_chunk_bwd(FAKE, FAKE, FAKE, E.MDN_F32, gate, FAKE, FAKE, FAKE, 0.5, None,
                                  None, vt, FAKE, dST, None, 1, T, 1, 64, 64, 64, dq, FAKE, FAKE,
                                  FAKE, FAKE, FAKE, FAKE, dS0, FAKE, FAKE, wsb, flags, None)
-    assert bw(flags=2) == E.MDN_ERR_INVALID_ARG
+    assert bw(flags=4) == E.MDN_ERR_INVALID_ARG
     assert bw(vt=None) == E.MDN_ERR_INVALID_ARG
     assert bw(dq=FAKE + 4) == E.MDN_ERR_INVALID_ARG
     assert bw(dS0=None) == E.MDN_ERR_INVALID_ARG

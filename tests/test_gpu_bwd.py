@@ -125,3 +125,24 @@ def test_bwd_cuda_graph_replay_matches_eager():
     torch.cuda.synchronize()
     for n in NAMES:
         assert torch.equal(got[n], eager[n]), n
+
+
+def test_bwd_tensor_core_path_matches_cuda_core_path():
+    """bf16, d = 128: the tcgen05 kernels (reverse chain, its operands, the
+    state scan, both product kernels) against the fp32 CUDA-core kernels on the
+    same inputs and the same saved Vtilde."""
+    from momentum_delta_rule_mdn_b200 import _lib
+    spec = mi.Spec("bwd_paths", B=2, T=300, H=3, d=128, state_std=0.03, seed=504)
+    inp = mi.make_inputs(spec)
+    dev = mi.to_torch(inp, "cuda")
+    o, vt, _, _ = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in GATES),
+                                inp.d_corr, dev["S0"], dev["M0"])
+    do = torch.randn_like(o)
+    dS = torch.randn(2, 3, 128, 128, device="cuda")
+    args = (dev["q"], dev["k"], dev["v"], *(dev[g] for g in GATES), inp.d_corr, vt, do,
+            dev["S0"], dev["M0"], dS, None)
+    tc = mdn.chunk_bwd(*args, flags=_lib.MDN_CHECK_FINITE)
+    simt = mdn.chunk_bwd(*args, flags=_lib.MDN_CHECK_FINITE | _lib.MDN_FORCE_SIMT)
+    for n in NAMES:
+        e = rel_l2(to_np(tc[n]), to_np(simt[n]))
+        assert e <= 1e-2, (n, e)
