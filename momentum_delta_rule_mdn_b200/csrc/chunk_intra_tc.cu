@@ -27,7 +27,9 @@
 // set of SMs take a single chunk) and follows the flags.  K and Q of a CTA's
 // next chunk are loaded by TMA into a second buffer while the current chunk
 // computes, and the gate scan of the next chunk runs on a warp that the
-// column pass leaves idle.  Column i of Gamma never leaves the registers of
+// column pass leaves idle.  The loop's code is kept compact (the loops over
+// 16-row groups and output halves are not unrolled): two CTAs at different
+// phases share each SM's instruction cache.  Column i of Gamma never leaves the registers of
 // the thread that owns it: that thread writes column i of A and K-row i of
 // the MN-major [I; Att] operand directly.  T is solved in place over A: the
 // diagonal blocks replace A_ii, B_ik replaces A_ik, and T_ij (i > j) goes to
@@ -86,8 +88,9 @@ struct IntraArgs {
 // Chunk-major order: the c-th chunk is chunk n of head bh; returns its index
 // in the head-major layout of the workspace.
 __device__ __forceinline__ long long chunk_of(long long c, const IntraArgs& a, int& n, int& bh) {
-    n = (int)(c / a.BH);
-    bh = (int)(c % a.BH);
+    const unsigned cu = (unsigned)c, q = cu / (unsigned)a.BH;  // chunk counts fit 32 bits
+    n = (int)q;
+    bh = (int)(cu - q * (unsigned)a.BH);
     return (long long)bh * a.NT + n;
 }
 
@@ -100,8 +103,9 @@ __device__ __forceinline__ void publish_chunk(unsigned* ready, long long chunk) 
 }
 
 // Gate record of one chunk (one warp): la, lm, b, alpha, beta, eta per
-// position; positions past T are steps that leave the state unchanged.
-__device__ __forceinline__ void gate_record(const IntraArgs& a, int n, int bh, float* rec, int lane) {
+// position; positions past T are steps that leave the state unchanged.  Not
+// inlined: the kernel's loop is kept small for the instruction cache.
+__device__ __noinline__ void gate_record(const IntraArgs& a, int n, int bh, float* rec, int lane) {
     const int b = bh / a.H, h = bh % a.H;
     const int t0 = n * C + 2 * lane;
     float ga[2] = {0.f, 0.f}, gm[2] = {0.f, 0.f}, gb[2] = {0.f, 0.f}, ge[2] = {0.f, 0.f};
@@ -266,7 +270,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         clk.lap(0);
 
         // ---- Qhat = Q - d K in place (the Q rows of both panels); chunk record
-#pragma unroll
+#pragma unroll 2
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u;
             const int pn = idx >> 9, w = idx & 511, r = w >> 3, cc = w & 7;
@@ -329,7 +333,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const float* be = rec + 4 * C;
             const float eta_i = rec[5 * C + i];
             float gam = 0.f, f = 1.f;
-#pragma unroll
+#pragma unroll 1
             for (int r16 = 0; r16 < C; r16 += 16) {
                 float kk[16], kh[16];
                 tmem_ld16(tmem + lane_sel + TM_G + r16, kk);      // k_i.k_r
@@ -468,7 +472,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int r = tid & 63, hf = tid >> 6;  // row r of T, columns 32 hf .. 32 hf + 31
             const int bi = r >> 4;
             const float g = wg[r], w = -wv[r];
-#pragma unroll
+#pragma unroll 1
             for (int q = 0; q < 2; ++q) {
                 const int bj = 2 * hf + q;  // 16-column block of T
                 float x[16];
@@ -544,7 +548,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         clk.lap(9);
 
         // ---- A2T rows (lane, 128 + lane) into the current K/Q buffer (K has been read)
-#pragma unroll
+#pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2, *reinterpret_cast<float(*)[32]>(v));
             tmem_ld32(tmem + lane_sel + TM_R + 64 * q2 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
