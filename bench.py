@@ -413,7 +413,9 @@ def run_backward(args, mdn, device, spec0):
     kern = mdn.profile_read(reset=True)
     mdn.profile_enable(False)
     return {"workload": spec0.name, "ms": round(ms, 4), "tokens_per_s": round(B * T / (ms * 1e-3), 1),
-            "calls": n, "path": "fp32 CUDA cores",
+            "calls": n,
+            "path": ("tcgen05 (bf16, d = 128), fp32 accumulation" if o.dtype == torch.bfloat16 and d == 128
+                     else "fp32 CUDA cores"),
             "kernels_ms": {k: round(v[0] / v[1], 4) for k, v in kern.items()}}
 
 
