@@ -39,6 +39,8 @@
 // while chunk n+1 computes.  Every wait is bounded; a wait that runs out
 // raises the CTA's abort flag, every role leaves its loop, in-flight copies
 // and MMAs are drained, and status[1] is set.
+#include <algorithm>
+
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -553,14 +555,46 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
 // The tensor-core path: the intra-chunk kernel, then the sequential
 // inter-chunk kernel as its programmatic dependent, both on stream s.
 //
-// Slice width (ns = 0 chooses) and overlap: the inter-chunk kernel's CTAs
-// can only start on SMs that the intra-chunk kernel has left.  When its CTAs
-// fit in the SMs minus a share kept for the intra-chunk kernel, that many SMs
-// are reserved: the intra-chunk CTAs there take a single chunk, and the chain
-// starts one chunk's time after launch while the other SMs produce the rest
-// ahead of it.  Four slices per head when they fit in one wave (their chain
-// is the shortest per chunk; two waves for packed sequences), else two; SMs
-// are reserved only when the slices fit beside the intra-chunk kernel's share.
+// Reserved SMs for the chains, and the chunk limit of the intra-chunk CTAs
+// on them.  The inter-chunk kernel's CTAs can only start on SMs that the
+// intra-chunk kernel (two CTAs per SM) has left, and each chain then takes
+// one chunk of its head per step.  With the intra-chunk CTAs on the chains'
+// SMs limited to L chunks, the chains start after about L chunk times while
+// the CTAs on the other SMs (U of them) produce the remaining chunks, which
+// the chunk-major order makes the last ones the chains need.  An
+// intra-chunk chunk costs about r chain steps (two CTAs per SM, ~17k cycles;
+// a 32-column chain step ~3.3k, a 64-column one ~4.6k), so L minimises
+//     L r + max(NT, rest / U r + 1),   rest = chunks - 2 SMs L.
+struct Reserve {
+    int sms = 0;    // CTAs on SMs 0 .. sms-1 are limited
+    int limit = 1;
+};
+static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, int ns)
+{
+    Reserve rv;
+    if (ctas > sms) return rv;
+    const double r = ns == 32 ? 5.0 : 3.7;
+    const long long U = 2LL * (sms - ctas), per_round = 2LL * sms;
+    const int lmax = (int)((chunks + per_round - 1) / per_round);
+    double best = 0.0;
+    for (int L = 1; L <= lmax; ++L) {
+        const long long rest = chunks - per_round * L;
+        if (rest > 0 && U == 0) continue;
+        const double t = L * r + std::max((double)nt, rest > 0 ? (double)rest / U * r + 1.0 : 0.0);
+        if (rv.sms == 0 || t < best) {
+            best = t;
+            rv.sms = (int)ctas;
+            rv.limit = L;
+        }
+    }
+    return rv;
+}
+
+// Slice width (ns = 0 chooses): four slices per head when they fit in one
+// wave (their chain is the shortest per chunk; two waves for packed
+// sequences), else two.  Packed sequences reserve SMs (one chunk each) only
+// when the slices fit beside a quarter of the SMs kept for the intra-chunk
+// kernel: their chains' lengths are not known on the host.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
@@ -576,8 +610,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     // out in order, the first ones on the lowest CTAs).
     if (ns == 0) ns = heads * 4 <= (a.cu_chunks ? 2LL * sms : (long long)sms) ? 32 : 64;
     const long long ctas = heads * (D / ns);
-    const int reserve = ctas <= room ? (int)ctas : 0;
-    if (!a.test_no_intra && (e = launch_chunk_intra_tc(a, s, reserve)) != cudaSuccess) return e;
+    Reserve rv;
+    if (a.cu_chunks) {
+        if (ctas <= room) rv.sms = (int)ctas;
+    } else {
+        rv = plan_reserve(heads * a.NT, ctas, sms, a.NT, ns);
+    }
+    if (!a.test_no_intra && (e = launch_chunk_intra_tc(a, s, rv.sms, rv.limit)) != cudaSuccess)
+        return e;
     return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
 }
 

@@ -24,7 +24,7 @@
 // in chunk-major order (chunk 0 of every head first), publishing a ready flag
 // per chunk; the inter-chunk kernel, launched as their programmatic
 // dependent, starts on the SMs whose CTAs leave first (the CTAs on a reserved
-// set of SMs take a single chunk) and follows the flags.  K and Q of a CTA's
+// set of SMs take at most a given number of chunks) and follows the flags.  K and Q of a CTA's
 // next chunk are loaded by TMA into a second buffer while the current chunk
 // computes, and the gate scan of the next chunk runs on a warp that the
 // column pass leaves idle.  The loop's code is kept compact (the loops over
@@ -81,8 +81,8 @@ struct IntraArgs {
     float* dbg;              // diagnostics: phase clocks of CTA 0 (null in normal use)
     float dcorr;
     int T, H, NT, BH;
-    int reserve;             // CTAs on SMs 0 .. reserve-1 take one chunk only, freeing
-                             // those SMs early for the inter-chunk kernel
+    int reserve;             // CTAs on SMs 0 .. reserve-1 take at most `limit` chunks,
+    int limit;               // freeing those SMs early for the inter-chunk kernel
 };
 
 // Chunk-major order: the c-th chunk is chunk n of head bh; returns its index
@@ -215,7 +215,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (tid == kTmaTid) {
         uint32_t smid_;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));
-        if ((int)smid_ < a.reserve) limit = 1;
+        if ((int)smid_ < a.reserve) limit = a.limit;
         mbar_init(&bars[B_LD], 1);
         mbar_init(&bars[B_LD + 1], 1);
         mbar_init(&bars[B_MMA], 1);
@@ -596,7 +596,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 }  // namespace
 
-cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve)
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve, int limit)
 {
     const long long chunks = (long long)a.B * a.H * a.NT;
     CUtensorMap mq, mk, mqh, mtat, ma2t;
@@ -615,6 +615,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserv
     t.ready = a.ready;
     t.queue = a.ready + chunks;
     t.reserve = reserve;
+    t.limit = limit > 0 ? limit : 1;
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;
     t.dcorr = a.dcorr;

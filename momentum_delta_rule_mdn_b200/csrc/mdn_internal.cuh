@@ -280,7 +280,7 @@ cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s);
 mdn_status cuda_fail(cudaError_t e);
 // ns: columns of d_v per inter-chunk CTA (32 or 64), 0 = choose by batch size
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);
-cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve);
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve, int limit);
 // ds_norm (nullable, [B*H]): receives ||S_t - S_{t-1}||_F of each head.
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,
                         const float* alpha_log, const float* mu_log, const float* beta,
