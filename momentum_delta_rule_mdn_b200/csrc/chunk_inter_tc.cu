@@ -28,8 +28,9 @@
 // that nothing else sits on that chain:
 //   warp 0      one lane issues every tcgen05.mma and commit
 //   warp 1      one lane issues every TMA load, up to two chunks ahead
-//   NS/4 chain warps: warp w owns TMEM lanes 32(w%4).. and 16 columns; it
-//               holds those columns of one row of S and M in fp32 registers
+//   16 chain warps: warp w owns TMEM lanes 32(w%4).. and NH columns (8 at
+//               NS = 32, 16 at NS = 64: the epilogues on the chain are short
+//               per thread); it holds those columns of one row of S and M in fp32 registers
 //               for the whole sequence (their bf16 copy in shared memory is
 //               the B operand of A1); the warps on lanes 0..63 also form Y
 //   4 output warps: Vtilde and o of chunk n from A3 and A1, written to
@@ -50,13 +51,13 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int NH = 16;           // columns per chain thread
 constexpr int kChainWarp0 = 2;   // warps 0, 1: MMA issue, loads
 
 // Per-width layout.  NS = d_v columns per CTA (32 or 64).
 template <int NS>
 struct Cfg {
-    static constexpr int CW = NS / 4;                 // chain warps: 4 lane quadrants x NS/16 column groups
+    static constexpr int NH = NS == 32 ? 8 : 16;      // columns per chain thread
+    static constexpr int CW = 4 * (NS / NH);          // chain warps: 4 lane quadrants x NS/NH column groups
     static constexpr int kOutWarp0 = kChainWarp0 + CW;
     static constexpr int kThreads = (kOutWarp0 + 4) * 32;
     // one CTA per SM; registers are granted to warps in groups of four
@@ -163,6 +164,13 @@ __device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* a
     }
 }
 
+// N (8 or 16) consecutive columns of this thread's TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+    if constexpr (N == 16) tmem_ld16(taddr, v);
+    else tmem_ld8(taddr, v);
+}
+
 // Warp-uniform form: every lane waits, and the warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
@@ -176,6 +184,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 {
     using L = Cfg<NS>;
     constexpr int CW = L::CW;
+    constexpr int NH = L::NH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -372,20 +381,17 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 clk.lap(1);
                 tc_fence_after_sync();
                 const uint32_t a1 = tq + L::TM_A1 + 2 * NS * s2 + NH * hc;
+                float x[NH], y[NH];
+                tmem_ld_cols<NH>(a1, x);
+                tmem_ld_cols<NH>(a1 + NS, y);
+                tmem_wait_ld();
 #pragma unroll
-                for (int q16 = 0; q16 < NH / 16; ++q16) {
-                    float x[16], y[16];
-                    tmem_ld16(a1 + 16 * q16, x);
-                    tmem_ld16(a1 + NS + 16 * q16, y);
-                    tmem_wait_ld();
+                for (int c = 0; c < NH / 8; ++c) {
+                    float vv[8];
+                    unpack_bf16x8(vrow[c], vv);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float vv[8];
-                        unpack_bf16x8(vrow[2 * q16 + c], vv);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) vv[e] -= fmaf(c_ab, x[8 * c + e], -c_d2 * y[8 * c + e]);
-                        st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + 2 * q16 + c), vv);
-                    }
+                    for (int e = 0; e < 8; ++e) vv[e] -= fmaf(c_ab, x[8 * c + e], -c_d2 * y[8 * c + e]);
+                    st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + c), vv);
                 }
                 clk.lap(2);
                 fence_proxy_async_smem();
@@ -403,18 +409,16 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
             clk.lap(4);
             tc_fence_after_sync();
-#pragma unroll
-            for (int q16 = 0; q16 < NH / 16; ++q16) {
-                float dS[16], dM[16];
-                tmem_ld16(tq + L::TM_A2 + NH * hc + 16 * q16, dS);
-                tmem_ld16(tq + L::TM_A2 + NS + NH * hc + 16 * q16, dM);
+            {
+                float dS[NH], dM[NH];
+                tmem_ld_cols<NH>(tq + L::TM_A2 + NH * hc, dS);
+                tmem_ld_cols<NH>(tq + L::TM_A2 + NS + NH * hc, dM);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int jj = 16 * q16 + j;
-                    const float sn = fmaf(abC, s[jj], fmaf(-bC, m[jj], dS[j]));
-                    m[jj] = fmaf(mbC, m[jj], dM[j]);
-                    s[jj] = sn;
+                for (int j = 0; j < NH; ++j) {
+                    const float sn = fmaf(abC, s[j], fmaf(-bC, m[j], dS[j]));
+                    m[j] = fmaf(mbC, m[j], dM[j]);
+                    s[j] = sn;
                 }
             }
 #pragma unroll
