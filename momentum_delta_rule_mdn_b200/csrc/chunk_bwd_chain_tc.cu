@@ -18,9 +18,12 @@
 //     A3 = [T^T; 0] dVtilde = dY         (M 128, N NS, K 64; off the chain)
 // This is the shape of the forward pass's inter-chunk kernel, whose warp
 // roles, hand-offs and bounded waits this kernel keeps: one lane issues the
-// MMAs, one lane the TMA and bulk loads (two chunks ahead), NS/4 chain warps
-// hold rows of dS and dM in fp32 registers (their bf16 copy is A1's B
-// operand), 4 output warps write dv.  NS = 32: four CTAs per head.
+// MMAs, one lane the TMA and bulk loads (two chunks ahead), 16 chain warps
+// hold rows of dS and dM in fp32 registers, 8 columns each (their bf16 copy is
+// A1's B operand), 4 output warps write dv.  NS = 32: four CTAs per head.
+// E, F and the adjoints leaving each chunk are in chain order (see
+// chain_off), so that the chain warps' global loads (E, F one chunk ahead)
+// and stores are 512 contiguous bytes per warp instruction.
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -30,13 +33,13 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int NH = 16;           // columns per chain thread
 constexpr int kChainWarp0 = 2;   // warps 0, 1: MMA issue, loads
 
 // Per-width layout.  NS = d_v columns per CTA (32 or 64).
 template <int NS>
 struct Cfg {
-    static constexpr int CW = NS / 4;                 // chain warps: 4 lane quadrants x NS/16 column groups
+    static constexpr int NH = NS == 32 ? 8 : 16;      // columns per chain thread
+    static constexpr int CW = 4 * (NS / NH);          // chain warps: 4 lane quadrants x NS/NH column groups
     static constexpr int kOutWarp0 = kChainWarp0 + CW;
     static constexpr int kThreads = (kOutWarp0 + 4) * 32;
     // one CTA per SM; registers are granted to warps in groups of four
@@ -124,6 +127,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
         }
     }
 }
+// N (8 or 16) consecutive columns of this thread's TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+    if constexpr (N == 16) tmem_ld16(taddr, v);
+    else tmem_ld8(taddr, v);
+}
+
 // Warp-uniform form: every lane waits, and the warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
@@ -136,6 +146,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 {
     using L = Cfg<NS>;
     constexpr int CW = L::CW;
+    constexpr int NH = L::NH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -314,29 +325,41 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         const int r = lane & 63;
         PhaseClock clk;
         clk.start(nullptr);
-        for (int n = 0; n < NT; ++n) {
+        // E and F of a chunk, in chain order (a warp's float4 at one quarter is
+        // 512 contiguous bytes); loaded one chunk ahead of their use
+        float ef[NH], ff[NH];
+        auto load_ef = [&](long long c, float* e, float* f) {
+            const float* src = a.ef + (size_t)c * 2 * D * D;
+#pragma unroll
+            for (int q = 0; q < NH / 4; ++q) {
+                const int o = chain_off(lane, j0 + NH * hc + 4 * q);
+                const float4 e4 = *reinterpret_cast<const float4*>(src + o);
+                const float4 f4 = *reinterpret_cast<const float4*>(src + D * D + o);
+                e[4 * q] = e4.x; e[4 * q + 1] = e4.y; e[4 * q + 2] = e4.z; e[4 * q + 3] = e4.w;
+                f[4 * q] = f4.x; f[4 * q + 1] = f4.y; f[4 * q + 2] = f4.z; f[4 * q + 3] = f4.w;
+            }
+        };
+        // One chunk of the chain; E, F of this chunk are in (ec, fc), and those
+        // of the next are loaded into (en, fn).  The loop below alternates the
+        // two register sets, so a load is only waited for a chunk later.
+        auto step = [&](int n, const float* ec, const float* fc, float* en, float* fn) -> bool {
             const int s2 = n & 1, sv = n % L::NVC;
             const long long chunk = ch.chunk0 + (NT - 1 - n);
             // the adjoints of the states leaving this chunk, kept for the
-            // chunk-local gradients; E and F of this chunk, for the update below
-            float ef[NH], ff[NH];
+            // chunk-local gradients
             {
-                const size_t off = (size_t)chunk * 2 * D * D + (size_t)lane * D + j0 + NH * hc;
-                float* dst = a.dss + off;
-                const float* e_src = a.ef + off;
+                float* dst = a.dss + (size_t)chunk * 2 * D * D;
 #pragma unroll
                 for (int q = 0; q < NH / 4; ++q) {
-                    *reinterpret_cast<float4*>(dst + 4 * q) =
+                    const int o = chain_off(lane, j0 + NH * hc + 4 * q);
+                    *reinterpret_cast<float4*>(dst + o) =
                         make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-                    *reinterpret_cast<float4*>(dst + D * D + 4 * q) =
+                    *reinterpret_cast<float4*>(dst + D * D + o) =
                         make_float4(m[4 * q], m[4 * q + 1], m[4 * q + 2], m[4 * q + 3]);
-                    const float4 e4 = *reinterpret_cast<const float4*>(e_src + 4 * q);
-                    const float4 f4 = *reinterpret_cast<const float4*>(e_src + D * D + 4 * q);
-                    ef[4 * q] = e4.x; ef[4 * q + 1] = e4.y; ef[4 * q + 2] = e4.z; ef[4 * q + 3] = e4.w;
-                    ff[4 * q] = f4.x; ff[4 * q + 1] = f4.y; ff[4 * q + 2] = f4.z; ff[4 * q + 3] = f4.w;
                 }
             }
-            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
+            if (n + 1 < NT) load_ef(chunk - 1, en, fn);  // the next chunk in chain order
+            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) return false;
             clk.lap(0);
             const float* cr = reinterpret_cast<const float*>(sm + L::CR0 + sv * 1024);
             const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
@@ -344,24 +367,21 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 const float c_g = cr[r], c_w = cr[C + r];
                 const float* prow =
                     reinterpret_cast<const float*>(sm + L::V0 + sv * L::V_BYTES) + r * NS + NH * hc;
-                if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
+                if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) return false;
                 clk.lap(1);
                 tc_fence_after_sync();
                 const uint32_t a1 = tq + L::TM_A1 + 2 * NS * s2 + NH * hc;
+                float x[NH], y[NH];
+                tmem_ld_cols<NH>(a1, x);
+                tmem_ld_cols<NH>(a1 + NS, y);
+                tmem_wait_ld();
 #pragma unroll
-                for (int q16 = 0; q16 < NH / 16; ++q16) {
-                    float x[16], y[16];
-                    tmem_ld16(a1 + 16 * q16, x);
-                    tmem_ld16(a1 + NS + 16 * q16, y);
-                    tmem_wait_ld();
+                for (int c = 0; c < NH / 8; ++c) {
+                    float vv[8];  // dVtilde = Att^T dO + Gamma_C K dS - w K dM
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float vv[8];  // dVtilde = Att^T dO + Gamma_C K dS - w K dM
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            vv[e] = prow[16 * q16 + 8 * c + e] + fmaf(c_g, x[8 * c + e], -c_w * y[8 * c + e]);
-                        st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + 2 * q16 + c), vv);
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        vv[e] = prow[8 * c + e] + fmaf(c_g, x[8 * c + e], -c_w * y[8 * c + e]);
+                    st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + c), vv);
                 }
                 clk.lap(2);
                 fence_proxy_async_smem();
@@ -376,21 +396,19 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 __syncwarp();
                 if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
             }
-            if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
+            if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) return false;
             clk.lap(4);
             tc_fence_after_sync();
-#pragma unroll
-            for (int q16 = 0; q16 < NH / 16; ++q16) {
-                float dS[16], dM[16];
-                tmem_ld16(tq + L::TM_A2 + NH * hc + 16 * q16, dS);
-                tmem_ld16(tq + L::TM_A2 + NS + NH * hc + 16 * q16, dM);
+            {
+                float dS[NH], dM[NH];
+                tmem_ld_cols<NH>(tq + L::TM_A2 + NH * hc, dS);
+                tmem_ld_cols<NH>(tq + L::TM_A2 + NS + NH * hc, dM);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int jj = 16 * q16 + j;
-                    const float sn = fmaf(abC, s[jj], dS[j] + ef[jj]);
-                    m[jj] = fmaf(mbC, m[jj], fmaf(-bC, s[jj], dM[j] - ff[jj]));
-                    s[jj] = sn;
+                for (int j = 0; j < NH; ++j) {
+                    const float sn = fmaf(abC, s[j], dS[j] + ec[j]);
+                    m[j] = fmaf(mbC, m[j], fmaf(-bC, s[j], dM[j] - fc[j]));
+                    s[j] = sn;
                 }
             }
 #pragma unroll
@@ -404,6 +422,13 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             __syncwarp();
             if (lid == 0) mbar_arrive(&bars[B_SR]);
             clk.lap(6);
+            return true;
+        };
+        float ef2[NH], ff2[NH];
+        if (NT > 0) load_ef(ch.chunk0 + NT - 1, ef, ff);
+        for (int n = 0; n < NT; n += 2) {
+            if (!step(n, ef, ff, ef2, ff2)) break;
+            if (n + 1 < NT && !step(n + 1, ef2, ff2, ef, ff)) break;
         }
         clk.flush();
     } else {

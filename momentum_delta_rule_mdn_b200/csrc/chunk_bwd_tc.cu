@@ -99,18 +99,21 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     const float* dSn = a.dSS + chunk * 2 * D * D;
     const float* dMn = dSn + D * D;
     float s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    // all four in chain order: consecutive threads take consecutive rows, so a
+    // warp's float4 loads are 512 contiguous bytes
     for (int i = tid; i < D * 16; i += kThr) {
-        const int row = i >> 4, c16 = i & 15;
-        const size_t g = (size_t)row * D + c16 * 8;
+        const int rest = i >> 5, c16 = rest >> 2;
+        const int row = ((rest & 3) << 5) | (i & 31);
+        const int g = chain_off(row, c16 * 8), g4 = chain_off(row, c16 * 8 + 4);
         float sv[8], mv[8], dsv[8], dmv[8];
         *reinterpret_cast<float4*>(sv) = *reinterpret_cast<const float4*>(Sn + g);
-        *reinterpret_cast<float4*>(sv + 4) = *reinterpret_cast<const float4*>(Sn + g + 4);
+        *reinterpret_cast<float4*>(sv + 4) = *reinterpret_cast<const float4*>(Sn + g4);
         *reinterpret_cast<float4*>(mv) = *reinterpret_cast<const float4*>(Mn + g);
-        *reinterpret_cast<float4*>(mv + 4) = *reinterpret_cast<const float4*>(Mn + g + 4);
+        *reinterpret_cast<float4*>(mv + 4) = *reinterpret_cast<const float4*>(Mn + g4);
         *reinterpret_cast<float4*>(dsv) = *reinterpret_cast<const float4*>(dSn + g);
-        *reinterpret_cast<float4*>(dsv + 4) = *reinterpret_cast<const float4*>(dSn + g + 4);
+        *reinterpret_cast<float4*>(dsv + 4) = *reinterpret_cast<const float4*>(dSn + g4);
         *reinterpret_cast<float4*>(dmv) = *reinterpret_cast<const float4*>(dMn + g);
-        *reinterpret_cast<float4*>(dmv + 4) = *reinterpret_cast<const float4*>(dMn + g + 4);
+        *reinterpret_cast<float4*>(dmv + 4) = *reinterpret_cast<const float4*>(dMn + g4);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             s1 = fmaf(sv[e], dsv[e], s1);
@@ -735,8 +738,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     const int R = quad * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     if (ok) {
-        // E, F: row i = R, columns [64 half, 64 half + 64)
-        float* Eo = a.bc_ef + (chunk * 2) * D * D + (size_t)R * D;
+        // E, F: row i = R, columns [64 half, 64 half + 64), in chain order
+        float* Eo = a.bc_ef + (chunk * 2) * D * D;
 #pragma unroll 1
         for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
             float e16[16], f16[16];
@@ -745,9 +748,10 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                *reinterpret_cast<float4*>(Eo + k0 + 4 * q) =
+                const int o = chain_off(R, k0 + 4 * q);
+                *reinterpret_cast<float4*>(Eo + o) =
                     make_float4(e16[4 * q], e16[4 * q + 1], e16[4 * q + 2], e16[4 * q + 3]);
-                *reinterpret_cast<float4*>(Eo + D * D + k0 + 4 * q) =
+                *reinterpret_cast<float4*>(Eo + D * D + o) =
                     make_float4(f16[4 * q], f16[4 * q + 1], f16[4 * q + 2], f16[4 * q + 3]);
             }
         }
@@ -796,7 +800,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
     tc_fence_after_sync();
     if (ok) {
-        float* Do = a.bc_d + (chunk * 2) * D * D + (size_t)R * D;
+        float* Do = a.bc_d + (chunk * 2) * D * D;  // chain order
 #pragma unroll 1
         for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
             float s16[16], m16[16];
@@ -805,9 +809,10 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                *reinterpret_cast<float4*>(Do + k0 + 4 * q) =
+                const int o = chain_off(R, k0 + 4 * q);
+                *reinterpret_cast<float4*>(Do + o) =
                     make_float4(s16[4 * q], s16[4 * q + 1], s16[4 * q + 2], s16[4 * q + 3]);
-                *reinterpret_cast<float4*>(Do + D * D + k0 + 4 * q) =
+                *reinterpret_cast<float4*>(Do + D * D + o) =
                     make_float4(m16[4 * q], m16[4 * q + 1], m16[4 * q + 2], m16[4 * q + 3]);
             }
         }
@@ -833,9 +838,12 @@ bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0
     const long long per = D * D / 4;
     if (gid >= heads * per) return;
     const long long bh = gid / per;
-    const int e4 = (int)(gid % per) * 4;
-    float4 s = S0 ? *reinterpret_cast<const float4*>(S0 + bh * D * D + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 m = M0 ? *reinterpret_cast<const float4*>(M0 + bh * D * D + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int e4 = (int)(gid % per) * 4;  // chain order; S0, M0 are row-major
+    int i0, j0;
+    chain_ij(e4, i0, j0);
+    const int r4 = i0 * D + j0;
+    float4 s = S0 ? *reinterpret_cast<const float4*>(S0 + bh * D * D + r4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 m = M0 ? *reinterpret_cast<const float4*>(M0 + bh * D * D + r4) : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int nn = 0; nn < NT; ++nn) {
         const size_t chunk = (size_t)bh * NT + nn;
         const float4 ds = __ldg(reinterpret_cast<const float4*>(dinc + chunk * 2 * D * D + e4));

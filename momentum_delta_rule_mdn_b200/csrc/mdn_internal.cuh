@@ -118,6 +118,20 @@ struct ChunkArgs {
 
 // Everything one mdn_chunk_bwd call needs, with the workspace carved.
 constexpr int kBwdRec = 6 * kChunk;  // floats of the per-chunk coefficient-adjoint record
+
+// "Chain order" of a 128 x 128 per-chunk matrix on the backward tensor-core
+// path (the reverse chain's operands E, F and its results, the adjoints
+// leaving each chunk; the state rebuild's increments and the entering
+// states): column quarters (4 columns) outermost, then rows, then the 4
+// columns of the quarter.  The reverse chain's threads hold one row and
+// whole quarters each, 32 consecutive rows per warp, so a warp's float4
+// access at one quarter is 512 contiguous bytes.
+__device__ __forceinline__ int chain_off(int i, int j) { return (((j >> 2) * 128 + i) << 2) | (j & 3); }
+// The row i and column j of the element at chain-order offset o.
+__device__ __forceinline__ void chain_ij(int o, int& i, int& j) {
+    i = (o >> 2) & 127;
+    j = ((o >> 9) << 2) | (o & 3);
+}
 struct BwdArgs {
     const void* q;
     const void* k;
@@ -143,16 +157,16 @@ struct BwdArgs {
     float* gamma;    // [B*H*NT, C, C]
     float* att;      // [B*H*NT, C, C]  (Qhat K^T) o Gamma
     float* tmat;     // [B*H*NT, C, C]  T = (I + A)^{-1}
-    float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk
-    float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk
+    float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk (tensor-core path: chain order)
+    float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk (idem)
     float* crec_bw;  // [B*H*NT, kBwdRec]  coefficient adjoints from the state products
     // chunk-only operands of the tensor-core reverse chain (null on the CUDA-core path)
     __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]
     __nv_bfloat16* bc_tt;  // [B*H*NT, 128, 64]  [T^T; 0]
     float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
-    float* bc_ef;          // [B*H*NT, 2, D, D]  Qhat^T Diag(alphabar) dO, Qhat^T Diag(b) dO
+    float* bc_ef;          // [B*H*NT, 2, D, D]  Qhat^T Diag(alphabar) dO, Qhat^T Diag(b) dO (chain order)
     float* bc_rec;         // [B*H*NT, 256]  Gamma_C, w, then alphabar_C, b_C, mubar_C
-    float* bc_d;           // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde
+    float* bc_d;           // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde (chain order)
     // outputs (fp32)
     float* dq;
     float* dk;
