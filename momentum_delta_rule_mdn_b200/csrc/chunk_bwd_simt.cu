@@ -64,27 +64,52 @@ bwd_prep_kernel(BwdArgs a)
     const long long bh = blockIdx.x / a.NT;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x;
-    for (int idx = tid; idx < C * D; idx += 256) {
-        const int r = idx / D, c = idx % D, t = n * C + r;
-        float kv = 0.f, qv = 0.f;
-        if (t < a.T) {
-            const size_t g = tok_idx(a, b, t, h) * D + c;
-            kv = ldt<Tin>(a.k, g);
-            qv = ldt<Tin>(a.q, g) - a.dcorr * kv;
+    // K, Qhat: 8-element vector loads, all issued before the shared-memory stores
+    {
+        constexpr int PER = C * D / 8 / 256;  // vectors per thread and tensor
+        float kx[PER][8], qx[PER][8];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int idx = tid + 256 * u, r = idx / (D / 8), c8 = idx % (D / 8), t = n * C + r;
+            if (t < a.T) {
+                const size_t g = tok_idx(a, b, t, h) * D + 8 * c8;
+                ld8<Tin>(a.k, g, kx[u]);
+                ld8<Tin>(a.q, g, qx[u]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) kx[u][e] = qx[u][e] = 0.f;
+            }
         }
-        Ks[r * KS + c] = kv;
-        Qs[r * KS + c] = qv;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int idx = tid + 256 * u, r = idx / (D / 8), c8 = idx % (D / 8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                Ks[r * KS + 8 * c8 + e] = kx[u][e];
+                Qs[r * KS + 8 * c8 + e] = qx[u][e] - a.dcorr * kx[u][e];
+            }
+        }
     }
     if (tid < C) {
         const int t = n * C + tid;
         alpha_s[tid] = t < a.T ? expf(a.alpha_log[tok_idx(a, b, t, h)]) : 1.f;
     }
-    __syncthreads();
     const float* G = a.gamma + chunk * C * C;
     float* att = a.att + chunk * C * C;
+    // Gamma at this thread's tile (rows r and r - 1), loaded before the products
+    const int rg = tid >> 4, ig = tid & 15;
+    float g_r[4][4], g_m[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int r = rg + 16 * u, i = ig + 16 * v;
+            g_r[u][v] = i <= r ? __ldg(G + r * C + i) : 0.f;
+            g_m[u][v] = i < r ? __ldg(G + (r - 1) * C + i) : 0.f;
+        }
+    __syncthreads();
     {
         // K K^T and Qhat K^T over 4 x 4 register tiles: rows rg + 16 u, columns ig + 16 v
-        const int rg = tid >> 4, ig = tid & 15;
         float kk[4][4], qk[4][4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -114,8 +139,8 @@ bwd_prep_kernel(BwdArgs a)
                 const int r = rg + 16 * u, i = ig + 16 * v;
                 float av = 0.f, tv = 0.f;
                 if (i <= r) {
-                    tv = qk[u][v] * G[r * C + i];
-                    if (i < r) av = alpha_s[r] * kk[u][v] * G[(r - 1) * C + i];
+                    tv = qk[u][v] * g_r[u][v];
+                    if (i < r) av = alpha_s[r] * kk[u][v] * g_m[u][v];
                 }
                 As[r * AS + i] = av;
                 att[r * C + i] = tv;
