@@ -116,33 +116,62 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_dbe[r] = 0.f;
     }
     __syncthreads();
-    if (tid == 0) {
-        float s = rec[5 * C + 2] * expf(v_lm[C - 1]);      // mubar_C M
-        for (int r = 0; r < C; ++r) s += rec[4 * C + r] * v_et[r] * expf(v_lm[C - 1] - v_lm[r]);
-        v_dlm[C - 1] += s;
-        // b_r = sum_{j<=r} exp(la_r - la_j) beta_j mubar_j: reverse recurrence
-        float Rb = 0.f;
-        for (int j = C - 1; j >= 0; --j) {
-            Rb = v_db[j] + (j + 1 < C ? v_al[j + 1] * Rb : 0.f);
+    if (tid < 32) {
+        // warp 0, positions j = 2 lane, 2 lane + 1
+        const int j0 = 2 * tid, j1 = j0 + 1;
+        // mubar_C M plus sum_r dw_r eta_r exp(lm_C - lm_r): a warp sum
+        float s = rec[4 * C + j0] * v_et[j0] * expf(v_lm[C - 1] - v_lm[j0]) +
+                  rec[4 * C + j1] * v_et[j1] * expf(v_lm[C - 1] - v_lm[j1]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        // b_r = sum_{j<=r} exp(la_r - la_j) beta_j mubar_j gives the reverse
+        // recurrence Rb_j = db_j + alpha_{j+1} Rb_{j+1} (Rb_C = 0): a suffix
+        // scan of the affine maps x -> db_j + alpha_{j+1} x, composed as
+        // (b1, a1) o (b2, a2) = (b1 + a1 b2, a1 a2)
+        const float a0 = v_al[j1], a1 = j1 + 1 < C ? v_al[j1 + 1] : 0.f;
+        const float b0 = v_db[j0], b1 = v_db[j1];
+        float sb = fmaf(a0, b1, b0), sa = a0 * a1;  // f_j0 o f_j1
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float ob = __shfl_down_sync(0xffffffffu, sb, off);
+            const float oa = __shfl_down_sync(0xffffffffu, sa, off);
+            if (tid + off < 32) {
+                sb = fmaf(sa, ob, sb);
+                sa *= oa;
+            }
+        }
+        float next = __shfl_down_sync(0xffffffffu, sb, 1);  // Rb at j1 + 1
+        if (tid == 31) next = 0.f;
+        const float Rb0 = sb, Rb1 = fmaf(a1, next, b1);
+        const float rb[2] = {Rb0, Rb1};
+        const int jj[2] = {j0, j1};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int j = jj[e];
             const float mb = expf(v_lm[j]);
-            const float tj = v_be[j] * mb * Rb;
-            v_dbe[j] += mb * Rb;
+            const float tj = v_be[j] * mb * rb[e];
+            v_dbe[j] += mb * rb[e];
             v_dla[j] -= tj;
             v_dlm[j] += tj;
         }
+        if (tid == 31) v_dlm[C - 1] += s + rec[5 * C + 2] * expf(v_lm[C - 1]);  // mubar_C M
     }
     __syncthreads();
-    // Gamma = eta o Gp: row and column sums of dG o Gamma, and eta's share
+    // Gamma = eta o Gp: row sums of dG o Gamma (threads 0..63), column sums
+    // and eta's share (threads 64..127)
     if (tid < C) {
         const int x = tid;
-        float rs = 0.f, cs = 0.f, ce = 0.f;
+        float rs = 0.f;
         for (int y = 0; y <= x; ++y) rs = fmaf(dG[x * AS + y], v_et[y] * Gp[x * AS + y], rs);
+        v_dla[x] += rs;
+    } else if (tid < 2 * C) {
+        const int x = tid - C;
+        float cs = 0.f, ce = 0.f;
         for (int y = x; y < C; ++y) {
             const float gp = Gp[y * AS + x];
             cs = fmaf(dG[y * AS + x], v_et[x] * gp, cs);
             ce = fmaf(dG[y * AS + x], gp, ce);
         }
-        v_dla[x] += rs;
         v_dlm[x] -= cs;
         v_de[x] += ce;
     }
@@ -167,15 +196,27 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_dlm[j] += v_be[j] * U;
     }
     __syncthreads();
-    if (tid == 0) {
-        // reverse cumulative sums: la, lm are inclusive prefix sums of the log gates
-        float sla = 0.f, slm = 0.f;
-        for (int j = C - 1; j >= 0; --j) {
-            sla += v_dla[j];
-            slm += v_dlm[j];
-            v_dla[j] = sla;
-            v_dlm[j] = slm;
+    if (tid < 32) {
+        // reverse cumulative sums (la, lm are inclusive prefix sums of the log
+        // gates): a warp suffix scan, two positions per lane
+        const int j0 = 2 * tid, j1 = j0 + 1;
+        const float xa1 = v_dla[j1], xm1 = v_dlm[j1];
+        float sa = v_dla[j0] + xa1, sm = v_dlm[j0] + xm1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float oa = __shfl_down_sync(0xffffffffu, sa, off);
+            const float om = __shfl_down_sync(0xffffffffu, sm, off);
+            if (tid + off < 32) {
+                sa += oa;
+                sm += om;
+            }
         }
+        float na = __shfl_down_sync(0xffffffffu, sa, 1), nm = __shfl_down_sync(0xffffffffu, sm, 1);
+        if (tid == 31) na = nm = 0.f;
+        v_dla[j0] = sa;
+        v_dlm[j0] = sm;
+        v_dla[j1] = xa1 + na;
+        v_dlm[j1] = xm1 + nm;
     }
     __syncthreads();
     if (tid < C) {

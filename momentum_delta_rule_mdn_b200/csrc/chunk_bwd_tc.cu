@@ -75,23 +75,35 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         const int p = i >> 9, w = i & 511;
         *reinterpret_cast<uint4*>(sm + SA2 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
     }
-    // dO, Vt (bf16 copies) and dY (fp32 -> bf16), 64 rows x 16 chunks of 8 each
-    for (int i = tid; i < C * 16; i += kThr) {
-        const int r = i >> 4, c16 = i & 15, t = n * C + r;
-        const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
-        uint4 o = make_uint4(0, 0, 0, 0), v = o, y = o;
-        if (t < a.T) {
-            const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
-            o = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
-            v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
-            const float4 y0 = *reinterpret_cast<const float4*>(a.dv + g);
-            const float4 y1 = *reinterpret_cast<const float4*>(a.dv + g + 4);
-            const float yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-            y = bf16x8(yy);
+    // dO, Vt (bf16 copies) and dY (fp32 -> bf16), 64 rows x 16 chunks of 8
+    // each; a thread's global loads are all issued before its stores
+    {
+        constexpr int PER = C * 16 / kThr;
+        uint4 ro[PER], rv[PER];
+        float4 ry0[PER], ry1[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15, t = n * C + r;
+            ro[u] = rv[u] = make_uint4(0, 0, 0, 0);
+            ry0[u] = ry1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < a.T) {
+                const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
+                ro[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
+                rv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
+                ry0[u] = *reinterpret_cast<const float4*>(a.dv + g);
+                ry1[u] = *reinterpret_cast<const float4*>(a.dv + g + 4);
+            }
         }
-        *reinterpret_cast<uint4*>(sm + SA1 + off) = o;
-        *reinterpret_cast<uint4*>(sm + SA1 + off + 64 * 128) = y;   // rows 64..127
-        *reinterpret_cast<uint4*>(sm + SA2 + off) = v;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15;
+            const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
+            const float yy[8] = {ry0[u].x, ry0[u].y, ry0[u].z, ry0[u].w,
+                                 ry1[u].x, ry1[u].y, ry1[u].z, ry1[u].w};
+            *reinterpret_cast<uint4*>(sm + SA1 + off) = ro[u];
+            *reinterpret_cast<uint4*>(sm + SA1 + off + 64 * 128) = bf16x8(yy);   // rows 64..127
+            *reinterpret_cast<uint4*>(sm + SA2 + off) = rv[u];
+        }
     }
     // S, M, dS, dM (fp32 -> bf16), 128 rows x 16 chunks each; the three scalars
     const float* Sn = a.SS + chunk * 2 * D * D;
@@ -101,30 +113,40 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     float s1 = 0.f, s2 = 0.f, s3 = 0.f;
     // all four in chain order: consecutive threads take consecutive rows, so a
     // warp's float4 loads are 512 contiguous bytes
-    for (int i = tid; i < D * 16; i += kThr) {
-        const int rest = i >> 5, c16 = rest >> 2;
-        const int row = ((rest & 3) << 5) | (i & 31);
-        const int g = chain_off(row, c16 * 8), g4 = chain_off(row, c16 * 8 + 4);
-        float sv[8], mv[8], dsv[8], dmv[8];
-        *reinterpret_cast<float4*>(sv) = *reinterpret_cast<const float4*>(Sn + g);
-        *reinterpret_cast<float4*>(sv + 4) = *reinterpret_cast<const float4*>(Sn + g4);
-        *reinterpret_cast<float4*>(mv) = *reinterpret_cast<const float4*>(Mn + g);
-        *reinterpret_cast<float4*>(mv + 4) = *reinterpret_cast<const float4*>(Mn + g4);
-        *reinterpret_cast<float4*>(dsv) = *reinterpret_cast<const float4*>(dSn + g);
-        *reinterpret_cast<float4*>(dsv + 4) = *reinterpret_cast<const float4*>(dSn + g4);
-        *reinterpret_cast<float4*>(dmv) = *reinterpret_cast<const float4*>(dMn + g);
-        *reinterpret_cast<float4*>(dmv + 4) = *reinterpret_cast<const float4*>(dMn + g4);
+    // (two row pieces per round, their loads issued before the stores)
+#pragma unroll 1
+    for (int i0 = tid; i0 < D * 16; i0 += 2 * kThr) {
+        float sv[2][8], mv[2][8], dsv[2][8], dmv[2][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            s1 = fmaf(sv[e], dsv[e], s1);
-            s2 = fmaf(mv[e], dsv[e], s2);
-            s3 = fmaf(mv[e], dmv[e], s3);
+        for (int u = 0; u < 2; ++u) {
+            const int i = i0 + kThr * u, rest = i >> 5, c16 = rest >> 2;
+            const int row = ((rest & 3) << 5) | (i & 31);
+            const int g = chain_off(row, c16 * 8), g4 = chain_off(row, c16 * 8 + 4);
+            *reinterpret_cast<float4*>(sv[u]) = *reinterpret_cast<const float4*>(Sn + g);
+            *reinterpret_cast<float4*>(sv[u] + 4) = *reinterpret_cast<const float4*>(Sn + g4);
+            *reinterpret_cast<float4*>(mv[u]) = *reinterpret_cast<const float4*>(Mn + g);
+            *reinterpret_cast<float4*>(mv[u] + 4) = *reinterpret_cast<const float4*>(Mn + g4);
+            *reinterpret_cast<float4*>(dsv[u]) = *reinterpret_cast<const float4*>(dSn + g);
+            *reinterpret_cast<float4*>(dsv[u] + 4) = *reinterpret_cast<const float4*>(dSn + g4);
+            *reinterpret_cast<float4*>(dmv[u]) = *reinterpret_cast<const float4*>(dMn + g);
+            *reinterpret_cast<float4*>(dmv[u] + 4) = *reinterpret_cast<const float4*>(dMn + g4);
         }
-        const uint32_t pan = (c16 >> 3) * 32768;
-        st_bf16x8(sm + SB1 + pan + sw128_off(row, c16 & 7), sv);
-        st_bf16x8(sm + SB1 + pan + sw128_off(row + 128, c16 & 7), mv);
-        st_bf16x8(sm + SB2 + pan + sw128_off(row, c16 & 7), dsv);
-        st_bf16x8(sm + SB2 + pan + sw128_off(row + 128, c16 & 7), dmv);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = i0 + kThr * u, rest = i >> 5, c16 = rest >> 2;
+            const int row = ((rest & 3) << 5) | (i & 31);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                s1 = fmaf(sv[u][e], dsv[u][e], s1);
+                s2 = fmaf(mv[u][e], dsv[u][e], s2);
+                s3 = fmaf(mv[u][e], dmv[u][e], s3);
+            }
+            const uint32_t pan = (c16 >> 3) * 32768;
+            st_bf16x8(sm + SB1 + pan + sw128_off(row, c16 & 7), sv[u]);
+            st_bf16x8(sm + SB1 + pan + sw128_off(row + 128, c16 & 7), mv[u]);
+            st_bf16x8(sm + SB2 + pan + sw128_off(row, c16 & 7), dsv[u]);
+            st_bf16x8(sm + SB2 + pan + sw128_off(row + 128, c16 & 7), dmv[u]);
+        }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -336,29 +358,44 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major)
-    for (int i = tid; i < C * 16; i += kThr) {
-        const int r = i >> 4, c16 = i & 15, t = n * C + r;
-        const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
-        float o[8] = {0.f}, y[8] = {0.f}, q[8] = {0.f}, k[8] = {0.f}, vt[8] = {0.f};
-        if (t < a.T) {
-            const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g), o);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g), q);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g), k);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g), vt);
-            const float4 y0 = *reinterpret_cast<const float4*>(a.dv + g);
-            const float4 y1 = *reinterpret_cast<const float4*>(a.dv + g + 4);
-            y[0] = y0.x; y[1] = y0.y; y[2] = y0.z; y[3] = y0.w;
-            y[4] = y1.x; y[5] = y1.y; y[6] = y1.z; y[7] = y1.w;
+    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major).  Every global load
+    // of a thread (four row pieces) is issued before its shared-memory stores.
+    {
+        constexpr int PER = C * 16 / kThr;
+        uint4 ro[PER], rq[PER], rk[PER], rv[PER];
+        float4 ry0[PER], ry1[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15, t = n * C + r;
+            ro[u] = rq[u] = rk[u] = rv[u] = make_uint4(0, 0, 0, 0);
+            ry0[u] = ry1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < a.T) {
+                const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
+                ro[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
+                rq[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
+                rk[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
+                rv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
+                ry0[u] = *reinterpret_cast<const float4*>(a.dv + g);
+                ry1[u] = *reinterpret_cast<const float4*>(a.dv + g + 4);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15;
+            const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
+            float q[8], k[8];
+            unpack_bf16x8(rq[u], q);
+            unpack_bf16x8(rk[u], k);
 #pragma unroll
             for (int e = 0; e < 8; ++e) q[e] -= a.dcorr * k[e];
+            const float y[8] = {ry0[u].x, ry0[u].y, ry0[u].z, ry0[u].w,
+                                ry1[u].x, ry1[u].y, ry1[u].z, ry1[u].w};
+            *reinterpret_cast<uint4*>(sm + LA_DY + off) = ro[u];
+            st_bf16x8(sm + LA_DY + off + 64 * 128, y);
+            st_bf16x8(sm + LA_QK + off, q);
+            *reinterpret_cast<uint4*>(sm + LA_QK + off + 64 * 128) = rk[u];
+            *reinterpret_cast<uint4*>(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7)) = rv[u];
         }
-        st_bf16x8(sm + LA_DY + off, o);
-        st_bf16x8(sm + LA_DY + off + 64 * 128, y);
-        st_bf16x8(sm + LA_QK + off, q);
-        st_bf16x8(sm + LA_QK + off + 64 * 128, k);
-        st_bf16x8(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7), vt);
     }
     // rows 64..127 of the second stage-2 operand are zero
     for (int i = tid; i < 1024; i += kThr) {
@@ -376,6 +413,7 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         v.lm[r] = a.lm[crow + r];
         v.b[r] = a.bco[crow + r];
         v.da[r] = 0.f;
+        v.de[r] = in ? expf(a.mu_log[gi]) : 1.f;  // mu_r, until the coefficient phase
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
@@ -395,15 +433,18 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         }
         mma_commit(&bars[0]);
     }
-    // Gamma without eta, by its column recurrence (overlaps the products)
+    // Gamma without eta, by its column recurrence (overlaps the products):
+    // Gp_{r,i} = alpha_r Gp_{r-1,i} + beta_r mubar_r / mubar_i, the ratio as a
+    // running product of mu (held in v.de until the coefficient phase)
     if (tid < C) {
         const int i = tid;
-        float g = 0.f;
+        float g = 0.f, f = 1.f;
         for (int r = 0; r < C; ++r) {
             if (r < i) {
                 Gp[r * LAS + i] = 0.f;
             } else {
-                g = (r == i) ? v.be[i] : fmaf(v.al[r], g, v.be[r] * expf(v.lm[r] - v.lm[i]));
+                if (r > i) f *= v.de[r];
+                g = (r == i) ? v.be[i] : fmaf(v.al[r], g, v.be[r] * f);
                 Gp[r * LAS + i] = g;
             }
         }
