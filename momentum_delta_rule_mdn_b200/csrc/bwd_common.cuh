@@ -74,13 +74,17 @@ __device__ __forceinline__ BwdVec bwd_vec(float* base) {
 // chunk's tokens.
 __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* rec_g,
                                                 const BwdVec& v, float* dG, const float* Gp,
-                                                float* rec, int tid, int n, int b, int h)
+                                                float* rec, int tid, int n, int b, int h,
+                                                bool rec_loaded = false)
 {
     constexpr int C = kChunk, AS = kChunk + 1;
-    // the chunk's record into shared memory first (rec: kBwdRec floats), so
-    // that the single-thread loops below read no global memory
-    for (int i = tid; i < kBwdRec; i += 256) rec[i] = rec_g[i];
-    __syncthreads();
+    // the chunk's record in shared memory (rec: kBwdRec floats), so that the
+    // loops below read no global memory; a caller that copied it earlier
+    // (and synchronised since) passes rec_loaded
+    if (!rec_loaded) {
+        for (int i = tid; i < kBwdRec; i += 256) rec[i] = rec_g[i];
+        __syncthreads();
+    }
     float* v_al = v.al;
     float* v_be = v.be;
     float* v_et = v.et;

@@ -358,10 +358,14 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major).  Every global load
-    // of a thread (four row pieces) is issued before its shared-memory stores.
+    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major), and the chunk's
+    // coefficient-adjoint record.  Every global load of a thread (four row
+    // pieces, two record entries) is issued before its shared-memory stores.
     {
         constexpr int PER = C * 16 / kThr;
+        static_assert(kBwdRec <= 2 * kThr, "record copy");
+        const float* rec_g = a.crec_bw + chunk * kBwdRec;
+        const float rc0 = rec_g[tid], rc1 = tid + kThr < kBwdRec ? rec_g[tid + kThr] : 0.f;
         uint4 ro[PER], rq[PER], rk[PER], rv[PER];
         float4 ry0[PER], ry1[PER];
 #pragma unroll
@@ -396,6 +400,9 @@ bwd_local_grads_tc_kernel(BwdArgs a)
             *reinterpret_cast<uint4*>(sm + LA_QK + off + 64 * 128) = rk[u];
             *reinterpret_cast<uint4*>(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7)) = rv[u];
         }
+        float* recs = reinterpret_cast<float*>(sm + L_REC);
+        recs[tid] = rc0;
+        if (tid + kThr < kBwdRec) recs[tid + kThr] = rc1;
     }
     // rows 64..127 of the second stage-2 operand are zero
     for (int i = tid; i < 1024; i += kThr) {
@@ -548,34 +555,42 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 #pragma unroll
         for (int e = 0; e < 64; ++e) xr[e] = X[r * 129 + 64 * half + e];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c0 = 64 * half + 16 * j;
-            float dqb[16], dkb[16];
-            tmem_ld16(tq + 128 + c0, dqb);
-            tmem_ld16(tq + 256 + c0, dkb);
-            tmem_wait_ld();
+        for (int j2 = 0; j2 < 4; j2 += 2) {  // two 16-column groups per round
+            float4 q4[2][4], k4[2][4];
             if (in) {
-                float4 q4[4], k4[4];
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {  // every load of the group before any store
-                    q4[e4] = *reinterpret_cast<const float4*>(a.dq + grow + c0 + 4 * e4);
-                    k4[e4] = *reinterpret_cast<const float4*>(a.dk + grow + c0 + 4 * e4);
-                }
+                for (int g = 0; g < 2; ++g)
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float qo[4] = {q4[e4].x, q4[e4].y, q4[e4].z, q4[e4].w};
-                    const float ko[4] = {k4[e4].x, k4[e4].y, k4[e4].z, k4[e4].w};
-                    float qn[4], kn[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int x = 16 * j + 4 * e4 + e;
-                        qn[e] = qo[e] + dqb[4 * e4 + e];
-                        kn[e] = ko[e] + dkb[4 * e4 + e] + xr[x] - a.dcorr * qn[e];
+                    for (int e4 = 0; e4 < 4; ++e4) {  // every load of the round before any store
+                        const int c = 64 * half + 16 * (j2 + g) + 4 * e4;
+                        q4[g][e4] = *reinterpret_cast<const float4*>(a.dq + grow + c);
+                        k4[g][e4] = *reinterpret_cast<const float4*>(a.dk + grow + c);
                     }
-                    *reinterpret_cast<float4*>(a.dq + grow + c0 + 4 * e4) =
-                        make_float4(qn[0], qn[1], qn[2], qn[3]);
-                    *reinterpret_cast<float4*>(a.dk + grow + c0 + 4 * e4) =
-                        make_float4(kn[0], kn[1], kn[2], kn[3]);
+            }
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const int j = j2 + g, c0 = 64 * half + 16 * j;
+                float dqb[16], dkb[16];
+                tmem_ld16(tq + 128 + c0, dqb);
+                tmem_ld16(tq + 256 + c0, dkb);
+                tmem_wait_ld();
+                if (in) {
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float qo[4] = {q4[g][e4].x, q4[g][e4].y, q4[g][e4].z, q4[g][e4].w};
+                        const float ko[4] = {k4[g][e4].x, k4[g][e4].y, k4[g][e4].z, k4[g][e4].w};
+                        float qn[4], kn[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int x = 16 * j + 4 * e4 + e;
+                            qn[e] = qo[e] + dqb[4 * e4 + e];
+                            kn[e] = ko[e] + dkb[4 * e4 + e] + xr[x] - a.dcorr * qn[e];
+                        }
+                        *reinterpret_cast<float4*>(a.dq + grow + c0 + 4 * e4) =
+                            make_float4(qn[0], qn[1], qn[2], qn[3]);
+                        *reinterpret_cast<float4*>(a.dk + grow + c0 + 4 * e4) =
+                            make_float4(kn[0], kn[1], kn[2], kn[3]);
+                    }
                 }
             }
         }
@@ -590,7 +605,7 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         if (tid == 0) atomicOr(a.status + 1, 1u);
         return;
     }
-    bwd_coeff_phase(a, rec, v, dG, Gp, reinterpret_cast<float*>(sm + L_REC), tid, n, b, h);
+    bwd_coeff_phase(a, rec, v, dG, Gp, reinterpret_cast<float*>(sm + L_REC), tid, n, b, h, true);
 }
 
 // ---------------------------------------------------------------------------
