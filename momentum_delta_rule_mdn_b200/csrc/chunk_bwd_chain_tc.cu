@@ -11,19 +11,21 @@
 // with E = Qhat^T Diag(alphabar) dO, F = Qhat^T Diag(b) dO.  Folding T into
 // U = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T] (chunk data, formed with
 // Att^T dO, E, F and [T^T; 0] by a parallel kernel first), a chunk is
-//     A1 = [K; K] [dS | dM]              (M 128, N 2 NS, K 128; lanes 0..63 used)
+//     A1 = [K; Qhat] [dS | dM]           (M 128, N 2 NS, K 128; lanes 0..63 used)
 //     dVtilde = Att^T dO + Diag(Gamma_C) A1_S - Diag(w) A1_M      (epilogue)
 //     A2 = U dVtilde                     (two M 128, N NS, K 64)
 //     dS, dM <- (alphabar_C dS + E, -b_C dS + mubar_C dM - F) + A2   (epilogue)
+//   with E = Qhat^T Diag(alphabar) dO and -F = Qhat^T (-Diag(b) dO) issued into
+//   A2's accumulators right after A1 (M 128, N NS, K 64, A MN-major from the
+//   Qhat rows of the [K; Qhat] tile), while the chain warps form dVtilde
 //     A3 = [T^T; 0] dVtilde = dY         (M 128, N NS, K 64; off the chain)
 // This is the shape of the forward pass's inter-chunk kernel, whose warp
 // roles, hand-offs and bounded waits this kernel keeps: one lane issues the
 // MMAs, one lane the TMA and bulk loads (two chunks ahead), 16 chain warps
 // hold rows of dS and dM in fp32 registers, 8 columns each (their bf16 copy is
 // A1's B operand), 4 output warps write dv.  NS = 32: four CTAs per head.
-// E, F and the adjoints leaving each chunk are in chain order (see
-// chain_off), so that the chain warps' global loads (E, F one chunk ahead)
-// and stores are 512 contiguous bytes per warp instruction.
+// The adjoints leaving each chunk are stored in chain order (see chain_off),
+// so that each chain warp's stores are 512 contiguous bytes per instruction.
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -44,7 +46,7 @@ struct Cfg {
     static constexpr int kThreads = (kOutWarp0 + 4) * 32;
     // one CTA per SM; registers are granted to warps in groups of four
     static constexpr int kMaxRegs = (65536 / (((kThreads / 32 + 3) / 4) * 128)) & ~7;
-    static constexpr int NVC = NS == 32 ? 4 : 2;      // V / coefficient slots
+    static constexpr int NVC = 2;                     // P, E/F operand and coefficient slots
     static constexpr uint32_t kTmemCols = NS == 32 ? 256 : 512;
     // shared memory (byte offsets from a 1024-byte aligned base)
     static constexpr uint32_t KQ0 = 0;                // [K; Qhat], 2 slots x 2 panels x (128 rows x 128 B)
@@ -56,15 +58,17 @@ struct Cfg {
     static constexpr uint32_t YB_BYTES = 64 * NS * 2;
     static constexpr uint32_t V0 = YB + YB_BYTES;      // Att^T dO slice 64 rows x NS fp32, NVC slots
     static constexpr uint32_t V_BYTES = 64 * NS * 4;
-    static constexpr uint32_t CR0 = V0 + NVC * V_BYTES;  // chunk coefficients (256 floats), NVC slots
+    static constexpr uint32_t E0 = V0 + NVC * V_BYTES;   // Diag(alphabar) dO, -Diag(b) dO slices, NVC slots
+    static constexpr uint32_t E_BYTES = 2 * 64 * NS * 2;  // (bf16, 64 rows x NS, MN-major: B of E, F)
+    static constexpr uint32_t CR0 = E0 + NVC * E_BYTES;  // chunk coefficients (256 floats), NVC slots
     static constexpr uint32_t BARS = CR0 + NVC * 1024;
     static constexpr uint32_t MISC = BARS + 256;
     static constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory map too large");
-    static_assert(ST % 1024 == 0 && YB % 1024 == 0 && V0 % 16 == 0, "operand alignment");
+    static_assert(ST % 1024 == 0 && YB % 1024 == 0 && V0 % 16 == 0 && E0 % 1024 == 0, "operand alignment");
     // TMEM columns: A1 (KS | KM, QhatS | QhatM) in two slots, A2 (dS | dM), A3 in two slots
     static constexpr uint32_t TM_A1 = 0, TM_A2 = 4 * NS, TM_A3 = 6 * NS;
-    static constexpr uint32_t kTxVC = V_BYTES + 1024;
+    static constexpr uint32_t kTxVC = V_BYTES + E_BYTES + 1024;
     // byte offset of 16-byte chunk c (8 columns) of row i of S, resp. M, in ST
     __device__ static __forceinline__ uint32_t s_off(int i, int c) { return sw128_off(i, c); }
     __device__ static __forceinline__ uint32_t m_off(int i, int c) {
@@ -91,12 +95,13 @@ constexpr int B_YR = 17;   //     Y written (the chain warps on lanes 0..63)
 constexpr int B_SR = 18;   //     next state written (every chain warp)
 constexpr int B_OD = 19;   // [2] A1 / A3 slot read by the output warps (4 warps)
 constexpr int B_FIN = 21;  //     every MMA complete (exit)
-constexpr int kBars = 22;
+constexpr int B_MQ = 22;   // [2] A1 and the E / F products complete: the [K; Qhat] slot is free
+constexpr int kBars = 24;
 
 struct ChainArgs {
     const float* crec;      // [chunks][256]: Gamma_C, w, ..., alphabar_C, b_C, mubar_C at 192..194
     const float* pp;        // [chunks][D/32][64][32]  Att^T dO by slice
-    const float* ef;        // [chunks][2][D][D]  E, F
+    const uint8_t* eo;      // [chunks][D/32][2][4096 B]  Diag(alphabar) dO, -Diag(b) dO by slice
     const float* dS_T;      // cotangents of S_T, M_T (may be null)
     const float* dM_T;
     float* dS0;
@@ -141,10 +146,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 template <int NS>
 __global__ void __launch_bounds__(Cfg<NS>::kThreads) __maxnreg__(Cfg<NS>::kMaxRegs)
-chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_tat,
-                       const __grid_constant__ CUtensorMap tm_a2t, const ChainArgs a)
+chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_qh,
+                       const __grid_constant__ CUtensorMap tm_tat, const __grid_constant__ CUtensorMap tm_a2t,
+                       const ChainArgs a)
 {
     using L = Cfg<NS>;
+    static_assert(NS == 32, "the E/F operand slices are laid out for 32 columns");
     constexpr int CW = L::CW;
     constexpr int NH = L::NH;
     extern __shared__ uint8_t smem_raw[];
@@ -217,6 +224,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             constexpr uint32_t ystep = (16 * NS * 2) >> 4;  // 16 rows of Y
             constexpr uint32_t id1 = idesc_bf16(128, 2 * NS, false, true);
             constexpr uint32_t id2 = idesc_bf16(128, NS, false, true);
+            constexpr uint32_t idef = idesc_bf16(128, NS, true, true);  // Qhat^T: MN-major A
             // K, Qhat of chunk n and the A1 / A3 slot of chunk n are waited for
             // while chunk n - 1 waits for its Y, so that only the state hand-off
             // separates the last product of one chunk from the first of the next.
@@ -234,6 +242,23 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                     mma_bf16(a1, dkq + (((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
                              d_st + ks * (2048 >> 4), id1, ks > 0);
                 mma_commit(&bars[B_M1 + s2]);
+                // E = Qhat^T Diag(alphabar) dO and -F = Qhat^T (-Diag(b) dO) into the
+                // accumulators of A2 (read by the last state epilogue, which has
+                // signalled), while the chain warps form dVtilde
+                {
+                    const int sv = n % L::NVC;
+                    if (!wait_bar(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
+                    const uint32_t qh = sbase + L::KQ0 + s2 * 32768 + 8192;
+                    const uint32_t eo = sbase + L::E0 + sv * L::E_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t aq = smem_desc(qh + ks * 2048, 16384, 1024, kSw128);
+                        mma_bf16(tmem + L::TM_A2, aq, smem_desc(eo + ks * 1024, 4096, 512, kSw64), idef, ks > 0);
+                        mma_bf16(tmem + L::TM_A2 + NS, aq, smem_desc(eo + 4096 + ks * 1024, 4096, 512, kSw64),
+                                 idef, ks > 0);
+                    }
+                    mma_commit(&bars[B_MQ + s2]);  // the last reads of this [K; Qhat] slot
+                }
                 clk.lap(2);
                 if (!wait_bar(&bars[B_FFB + s2], (n >> 1) & 1, abort_flag)) break;
                 if (n + 1 < NT) {
@@ -249,8 +274,8 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t yd = d_y + ks * ystep;
-                    mma_bf16(tmem + L::TM_A2, dfb + (16384 >> 4) + ks * 2, yd, id2, ks > 0);
-                    mma_bf16(tmem + L::TM_A2 + NS, dfb + (32768 >> 4) + ks * 2, yd, id2, ks > 0);
+                    mma_bf16(tmem + L::TM_A2, dfb + (16384 >> 4) + ks * 2, yd, id2, true);
+                    mma_bf16(tmem + L::TM_A2 + NS, dfb + (32768 >> 4) + ks * 2, yd, id2, true);
                 }
                 mma_commit(&bars[B_M2]);
                 clk.lap(5);
@@ -276,7 +301,8 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 const int s2 = n & 1, sv = n % L::NVC;
                 const int mm = NT - 1 - n;  // chunks are walked backwards
                 const long long chunk = ch.chunk0 + mm;
-                if (n >= 2 && !wait_bar(&bars[B_M1 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
+                // the slot's previous chunk (n - 2) has been read by A1 and by E, F
+                if (n >= 2 && !wait_bar(&bars[B_MQ + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
                 clk.lap(0);
                 uint64_t* fb = &bars[B_FKQ + s2];
                 mbar_arrive_expect_tx(fb, kTxKQ);
@@ -284,7 +310,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 for (int p = 0; p < 2; ++p) {
                     uint8_t* dst = sm + L::KQ0 + s2 * 32768 + p * 16384;
                     tma_load_4d(dst, &tm_k, p * 64, h, (ch.n0 + mm) * C, b, fb);
-                    tma_load_4d(dst + 8192, &tm_k, p * 64, h, (ch.n0 + mm) * C, b, fb);
+                    tma_load_3d(dst + 8192, &tm_qh, p * 64, 0, (int)chunk, fb);
                 }
                 issued_kq = n + 1;
                 if (n >= 2 && !wait_bar(&bars[B_M3 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
@@ -304,6 +330,8 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 mbar_arrive_expect_tx(fb, L::kTxVC);
                 bulk_load(sm + L::V0 + sv * L::V_BYTES, a.pp + (chunk * (D / NS) + slice) * 64 * NS,
                           L::V_BYTES, fb);
+                bulk_load(sm + L::E0 + sv * L::E_BYTES, a.eo + (chunk * (D / NS) + slice) * L::E_BYTES,
+                          L::E_BYTES, fb);
                 bulk_load(sm + L::CR0 + sv * 1024, a.crec + chunk * 256, 1024, fb);
                 issued_vc = n + 1;
             }
@@ -325,24 +353,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         const int r = lane & 63;
         PhaseClock clk;
         clk.start(nullptr);
-        // E and F of a chunk, in chain order (a warp's float4 at one quarter is
-        // 512 contiguous bytes); loaded one chunk ahead of their use
-        float ef[NH], ff[NH];
-        auto load_ef = [&](long long c, float* e, float* f) {
-            const float* src = a.ef + (size_t)c * 2 * D * D;
-#pragma unroll
-            for (int q = 0; q < NH / 4; ++q) {
-                const int o = chain_off(lane, j0 + NH * hc + 4 * q);
-                const float4 e4 = *reinterpret_cast<const float4*>(src + o);
-                const float4 f4 = *reinterpret_cast<const float4*>(src + D * D + o);
-                e[4 * q] = e4.x; e[4 * q + 1] = e4.y; e[4 * q + 2] = e4.z; e[4 * q + 3] = e4.w;
-                f[4 * q] = f4.x; f[4 * q + 1] = f4.y; f[4 * q + 2] = f4.z; f[4 * q + 3] = f4.w;
-            }
-        };
-        // One chunk of the chain; E, F of this chunk are in (ec, fc), and those
-        // of the next are loaded into (en, fn).  The loop below alternates the
-        // two register sets, so a load is only waited for a chunk later.
-        auto step = [&](int n, const float* ec, const float* fc, float* en, float* fn) -> bool {
+        for (int n = 0; n < NT; ++n) {
             const int s2 = n & 1, sv = n % L::NVC;
             const long long chunk = ch.chunk0 + (NT - 1 - n);
             // the adjoints of the states leaving this chunk, kept for the
@@ -358,8 +369,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                         make_float4(m[4 * q], m[4 * q + 1], m[4 * q + 2], m[4 * q + 3]);
                 }
             }
-            if (n + 1 < NT) load_ef(chunk - 1, en, fn);  // the next chunk in chain order
-            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) return false;
+            if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
             clk.lap(0);
             const float* cr = reinterpret_cast<const float*>(sm + L::CR0 + sv * 1024);
             const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
@@ -367,7 +377,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 const float c_g = cr[r], c_w = cr[C + r];
                 const float* prow =
                     reinterpret_cast<const float*>(sm + L::V0 + sv * L::V_BYTES) + r * NS + NH * hc;
-                if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) return false;
+                if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
                 clk.lap(1);
                 tc_fence_after_sync();
                 const uint32_t a1 = tq + L::TM_A1 + 2 * NS * s2 + NH * hc;
@@ -387,16 +397,13 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lid == 0) {
-                    mbar_arrive(&bars[B_YR]);
-                    mbar_arrive(&bars[B_EVC + sv]);
-                }
+                if (lid == 0) mbar_arrive(&bars[B_YR]);
                 clk.lap(3);
-            } else {
-                __syncwarp();
-                if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
             }
-            if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) return false;
+            if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
+            // the products of this chunk (E and F among them) have read the
+            // slot: it may be refilled
+            if (lid == 0) mbar_arrive(&bars[B_EVC + sv]);
             clk.lap(4);
             tc_fence_after_sync();
             {
@@ -406,8 +413,9 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < NH; ++j) {
-                    const float sn = fmaf(abC, s[j], dS[j] + ec[j]);
-                    m[j] = fmaf(mbC, m[j], fmaf(-bC, s[j], dM[j] - fc[j]));
+                    // dS holds E + U_S dVtilde, dM holds -F + U_M dVtilde
+                    const float sn = fmaf(abC, s[j], dS[j]);
+                    m[j] = fmaf(mbC, m[j], fmaf(-bC, s[j], dM[j]));
                     s[j] = sn;
                 }
             }
@@ -422,13 +430,6 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             __syncwarp();
             if (lid == 0) mbar_arrive(&bars[B_SR]);
             clk.lap(6);
-            return true;
-        };
-        float ef2[NH], ff2[NH];
-        if (NT > 0) load_ef(ch.chunk0 + NT - 1, ef, ff);
-        for (int n = 0; n < NT; n += 2) {
-            if (!step(n, ef, ff, ef2, ff2)) break;
-            if (n + 1 < NT && !step(n + 1, ef2, ff2, ef, ff)) break;
         }
         clk.flush();
     } else {
@@ -489,16 +490,17 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     constexpr int NS = 32;
     using L = Cfg<NS>;
     if (a.D != D) return cudaErrorNotSupported;
-    CUtensorMap mk, mtt, mu;
+    CUtensorMap mk, mqh, mtt, mu;
     const long long chunks = (long long)a.B * a.H * a.NT;
     if (!make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
+        !make_chunk_map(&mqh, a.bc_qh, chunks, C, D, C) ||
         !make_chunk_map(&mtt, a.bc_tt, chunks, 2 * C, C, 2 * C) ||
         !make_chunk_map(&mu, a.bc_u, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
     ChainArgs t;
     t.crec = a.bc_rec;
     t.pp = a.bc_p;
-    t.ef = a.bc_ef;
+    t.eo = a.bc_eo;
     t.dS_T = a.dS_T;
     t.dM_T = a.dM_T;
     t.dS0 = a.dS0;
@@ -517,7 +519,7 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)a.B * a.H * (D / NS);
     ProfScope ps(kBwdChain, s);
-    chunk_bwd_chain_kernel<NS><<<(unsigned)blocks, L::kThreads, L::SMEM_BYTES, s>>>(mk, mtt, mu, t);
+    chunk_bwd_chain_kernel<NS><<<(unsigned)blocks, L::kThreads, L::SMEM_BYTES, s>>>(mk, mqh, mtt, mu, t);
     return cudaGetLastError();
 }
 

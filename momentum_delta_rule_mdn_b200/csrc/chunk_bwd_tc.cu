@@ -613,27 +613,27 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 //   U  = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T]   bf16 [256][64]  (A of U dVtilde)
 //   TT = [T^T ; 0]                                      bf16 [128][64]  (A of T^T dVtilde = dv)
 //   P  = Att^T dO     fp32, slice-major [D/32][64][32]  (dVtilde's chain-free part)
-//   E  = Qhat^T Diag(alphabar) dO,  F = Qhat^T Diag(b) dO   fp32 [2][128][128]
+//   Qhat rows (bf16 [64][128]) and Diag(alphabar) dO, -Diag(b) dO by 32-column
+//   slice (bf16, the reverse chain's shared-memory image of its B operands)
 //   record: Gamma_{C,r} (64), w_r (64), then alphabar_C, b_C, mubar_C at 192..194
 // plus the increments of the state rebuild, D_S = K^T Diag(Gamma_C) Vtilde and
 // D_M = K^T Diag(w) Vtilde, which turn the rebuild into an elementwise scan
 // over the chunks.  Products
 // (A operands K-major, transposed while they are staged):
-//   E = Qhat^T (Diag(alphabar) dO), F = Qhat^T (Diag(b) dO)    M 128, N 128, K 64
 //   U = K^T [Diag(-alphabar) T^T | Diag(D2) T^T]                M 128, N 64 + 64
 //   P = Att^T dO                                                 M 64 (of 128), N 128
 //   D = K^T [Diag(Gamma_C) Vtilde | Diag(w) Vtilde]             M 128, N 128 + 128 (second round)
-constexpr uint32_t PA_QT = 0;        // Qhat^T  [128 i][64 r]  K-major, 16 KB
-constexpr uint32_t PA_KT = 16384;    // K^T     [128 i][64 r]
-constexpr uint32_t PA_AT = 32768;    // Att^T   [128 r (64 used)][64 r2]
-constexpr uint32_t PB_OA = 49152;    // Diag(alphabar) dO  [64 r][128 j]  MN-major: 2 N-panels x 64 rows
-constexpr uint32_t PB_OB = 65536;    // Diag(b) dO
-constexpr uint32_t PB_O = 81920;     // dO
-constexpr uint32_t PB_VG = 98304;    // Diag(Gamma_C) Vtilde
-constexpr uint32_t PB_VW = 114688;   // Diag(w) Vtilde
-constexpr uint32_t PB_TS = 131072;   // -alphabar_{r2} T[r][r2]  [64 r][64 r2]  K-major, 8 KB
-constexpr uint32_t PB_TM = 139264;   //  D2_{r2} T[r][r2]
-constexpr uint32_t P_VEC = 147456;   // alphabar, b, D2, Gamma_C, w
+// E = Qhat^T Diag(alphabar) dO and F = Qhat^T Diag(b) dO are formed in the
+// reverse chain itself (by the MMA lane while it waits for each chunk's
+// dVtilde), from Qhat and the scaled dO slices written here.
+constexpr uint32_t PA_KT = 0;        // K^T     [128 i][64 r]  K-major, 16 KB
+constexpr uint32_t PA_AT = 16384;    // Att^T   [128 r (64 used)][64 r2]
+constexpr uint32_t PB_O = 32768;     // dO      [64 r][128 j]  MN-major: 2 N-panels x 64 rows
+constexpr uint32_t PB_VG = 49152;    // Diag(Gamma_C) Vtilde
+constexpr uint32_t PB_VW = 65536;    // Diag(w) Vtilde
+constexpr uint32_t PB_TS = 81920;    // -alphabar_{r2} T[r][r2]  [64 r][64 r2]  K-major, 8 KB
+constexpr uint32_t PB_TM = 90112;    //  D2_{r2} T[r][r2]
+constexpr uint32_t P_VEC = 98304;    // alphabar, b, D2, Gamma_C, w
 constexpr uint32_t P_BAR = P_VEC + 1280;
 constexpr uint32_t P_MISC = P_BAR + 16;
 constexpr uint32_t P_SMEM = P_MISC + 16 + 1024;
@@ -721,24 +721,27 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         for (int u = 0; u < U8; ++u) {
             const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8;
             const float ab = v_ab[r], bb = v_b[r], gl = v_g[r], w = v_w[r];
-            float oa[8], ob[8], vg[8], vw[8];
+            float qh[8], oa[8], ob[8], vg[8], vw[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float qh = qx[u][e] - a.dcorr * kx[u][e];
-                // transposed into the K-major A operands
-                st_bf16(sm + PA_QT + kmaj_off(c8 + e, r, 16384), qh);
+                qh[e] = qx[u][e] - a.dcorr * kx[u][e];
+                // transposed into the K-major A operand
                 st_bf16(sm + PA_KT + kmaj_off(c8 + e, r, 16384), kx[u][e]);
                 oa[e] = ab * ox[u][e];
-                ob[e] = bb * ox[u][e];
+                ob[e] = -bb * ox[u][e];
                 vg[e] = gl * vx[u][e];
                 vw[e] = w * vx[u][e];
             }
             const uint32_t o = mn_off(r, c8, 64);
-            st_bf16x8(sm + PB_OA + o, oa);
-            st_bf16x8(sm + PB_OB + o, ob);
             st_bf16x8(sm + PB_O + o, ox[u]);
             st_bf16x8(sm + PB_VG + o, vg);
             st_bf16x8(sm + PB_VW + o, vw);
+            // Qhat rows, and the reverse chain's E / F operands Diag(alphabar) dO and
+            // -Diag(b) dO by 32-column slice, each in the chain's shared-memory image
+            *reinterpret_cast<uint4*>(a.bc_qh + (chunk * C + r) * D + c8) = bf16x8(qh);
+            uint8_t* eo = a.bc_eo + (chunk * (D / 32) + (c8 >> 5)) * 8192 + sw64_off(r, (c8 & 31) >> 3);
+            *reinterpret_cast<uint4*>(eo) = bf16x8(oa);
+            *reinterpret_cast<uint4*>(eo + 4096) = bf16x8(ob);
         }
     }
     // T and Att: the scaled T tiles (K-major), Att^T (K-major), and [T^T; 0] to global
@@ -777,11 +780,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         constexpr uint32_t idk = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t aq = smem_desc(sbase + PA_QT + ks * 32, 16, 1024, kSw128);
             const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
             const uint64_t aa = smem_desc(sbase + PA_AT + ks * 32, 16, 1024, kSw128);
-            mma_bf16(tmem, aq, smem_desc(sbase + PB_OA + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
-            mma_bf16(tmem + 128, aq, smem_desc(sbase + PB_OB + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
             mma_bf16(tmem + 256, ak, smem_desc(sbase + PB_TS + ks * 32, 16, 1024, kSw128), idk, ks > 0);
             mma_bf16(tmem + 320, ak, smem_desc(sbase + PB_TM + ks * 32, 16, 1024, kSw128), idk, ks > 0);
             mma_bf16(tmem + 384, aa, smem_desc(sbase + PB_O + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
@@ -794,23 +794,6 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     const int R = quad * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     if (ok) {
-        // E, F: row i = R, columns [64 half, 64 half + 64), in chain order
-        float* Eo = a.bc_ef + (chunk * 2) * D * D;
-#pragma unroll 1
-        for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
-            float e16[16], f16[16];
-            tmem_ld16(tq + k0, e16);
-            tmem_ld16(tq + 128 + k0, f16);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int o = chain_off(R, k0 + 4 * q);
-                *reinterpret_cast<float4*>(Eo + o) =
-                    make_float4(e16[4 * q], e16[4 * q + 1], e16[4 * q + 2], e16[4 * q + 3]);
-                *reinterpret_cast<float4*>(Eo + D * D + o) =
-                    make_float4(f16[4 * q], f16[4 * q + 1], f16[4 * q + 2], f16[4 * q + 3]);
-            }
-        }
         // U: row i = R of the S half (half 0) or of the M half (half 1)
         {
             float u32[32];
@@ -839,7 +822,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             }
         }  // (R < 64 is warp-uniform: quadrants 0, 1)
     }
-    // second round: the rebuild increments into the columns of E and F
+    // second round: the rebuild increments into TMEM columns 0..255 (unused in the first)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();

@@ -164,7 +164,11 @@ struct BwdArgs {
     __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]
     __nv_bfloat16* bc_tt;  // [B*H*NT, 128, 64]  [T^T; 0]
     float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
-    float* bc_ef;          // [B*H*NT, 2, D, D]  Qhat^T Diag(alphabar) dO, Qhat^T Diag(b) dO (chain order)
+    __nv_bfloat16* bc_qh;  // [B*H*NT, C, D]  Qhat = Q - d K (bf16, rows of the chunk)
+    uint8_t* bc_eo;        // [B*H*NT, D/32, 2, 4096 B]  Diag(alphabar) dO and -Diag(b) dO by
+                           // 32-column slice, bf16, each the shared-memory image of the reverse
+                           // chain's B operand (MN-major, 64-byte swizzle); with Qhat^T they
+                           // give E and F inside the chain
     float* bc_rec;         // [B*H*NT, 256]  Gamma_C, w, then alphabar_C, b_C, mubar_C
     float* bc_d;           // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde (chain order)
     // outputs (fp32)
