@@ -67,6 +67,27 @@ __device__ __forceinline__ BwdVec bwd_vec(float* base) {
     return v;
 }
 
+// T = (I + A)^{-1} for a strictly lower C x C matrix A (shared memory, row
+// stride C + 1) into Ts (same layout), by forward substitution: column c on
+// the four lanes 4c .. 4c + 3 of a 256-thread CTA, each summing every fourth
+// term.  The caller synchronises before and after.
+__device__ __forceinline__ void bwd_unit_lower_inverse(const float* As, float* Ts, int tid)
+{
+    constexpr int C = kChunk, AS = kChunk + 1;
+    const int c = tid >> 2, part = tid & 3;
+    if (part == 0) Ts[c] = (c == 0) ? 1.f : 0.f;  // row 0
+    __syncwarp();
+    for (int r = 1; r < C; ++r) {
+        float acc = 0.f;
+        if (r > c)
+            for (int i = c + part; i < r; i += 4) acc = fmaf(As[r * AS + i], Ts[i * AS + c], acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (part == 0) Ts[r * AS + c] = (r == c) ? 1.f : (r > c ? -acc : 0.f);
+        __syncwarp();
+    }
+}
+
 // The last phase (every thread of a 256-thread CTA calls it): dG ([C][C+1],
 // overwritten), Gp ([C][C+1]), the record of the state products (rec_g, in
 // global memory; rec: kBwdRec floats of shared scratch), v.da holding the

@@ -149,20 +149,7 @@ bwd_prep_kernel(BwdArgs a)
     __syncthreads();
     // unit lower-triangular inverse by forward substitution: column c on the
     // four lanes 4c .. 4c + 3, each summing every fourth term
-    {
-        const int c = tid >> 2, part = tid & 3;
-        if (part == 0) Ts[c] = (c == 0) ? 1.f : 0.f;  // row 0
-        __syncwarp();
-        for (int r = 1; r < C; ++r) {
-            float acc = 0.f;
-            if (r > c)
-                for (int i = c + part; i < r; i += 4) acc = fmaf(As[r * AS + i], Ts[i * AS + c], acc);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (part == 0) Ts[r * AS + c] = (r == c) ? 1.f : (r > c ? -acc : 0.f);
-            __syncwarp();
-        }
-    }
+    bwd_unit_lower_inverse(As, Ts, tid);
     __syncthreads();
     float* Tm = a.tmat + chunk * C * C;
     for (int idx = tid; idx < C * C; idx += 256) Tm[idx] = Ts[(idx / C) * AS + idx % C];
@@ -897,15 +884,11 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s)
     MDN_SET_SMEM((bwd_local_grads_kernel<Tin, D>), sm3b)
 #undef MDN_SET_SMEM
     if (std::is_same<Tin, __nv_bfloat16>::value && D == 128 && a.bc_u) {
-        // bf16, d = 128: T and Att on CUDA cores, then the chain's operands and
-        // the rebuild increments on tensor cores, the entering states by an
-        // elementwise scan, the reverse chain and both per-chunk product
-        // kernels on tensor cores
-        {
-            ProfScope ps(kBwdPrep, s);
-            bwd_prep_kernel<Tin, D><<<(unsigned)chunks, 256, sm0, s>>>(a);
-        }
-        if ((e = cudaGetLastError())) return e;
+        // bf16, d = 128: T and Att, the chain's operands and the rebuild
+        // increments on tensor cores, the entering states by an elementwise
+        // scan, the reverse chain and both per-chunk product kernels on
+        // tensor cores
+        if ((e = launch_bwd_prep_tc(a, s))) return e;
         if ((e = launch_bwd_chain_prep_tc(a, s))) return e;
         if ((e = launch_bwd_chain_tc(a, s))) return e;
         if ((e = launch_bwd_state_grads_tc(a, s))) return e;

@@ -609,6 +609,143 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// T = (I + A)^{-1} with A = (P K^T) o Gamma-, and Att = (Qhat K^T) o Gamma, per
+// chunk (bf16, d = 128): the forward pass's intra-chunk product on tcgen05,
+//   G = [K; Qhat] [K; Qhat]^T   (M 128, N 128, K 128; lane i < 64: k_i.k_r in
+//                                columns r, k_i.qhat_r in columns 64 + r)
+// then thread i forms column i of A and Att from lane i, and the forward
+// substitution of the CUDA-core version gives T.  Qhat is rounded to bf16 as
+// in the forward pass.
+constexpr uint32_t Q_KQ = 0;                 // [K; Qhat] K-major: 2 panels x 128 rows x 128 B
+constexpr uint32_t Q_A = 32768;              // fp32 A [64][65]
+constexpr uint32_t Q_T = Q_A + 16640;        // fp32 Gamma [64][65], then T
+constexpr uint32_t Q_AL = Q_T + 16640;       // alpha_r
+constexpr uint32_t Q_BAR = Q_AL + 256;
+constexpr uint32_t Q_MISC = Q_BAR + 16;
+constexpr uint32_t Q_SMEM = Q_MISC + 16 + 1024;
+
+__global__ void __launch_bounds__(kThr)
+bwd_prep_tc_kernel(BwdArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int n = blockIdx.x % a.NT;
+    const long long bh = blockIdx.x / a.NT;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const size_t chunk = blockIdx.x;
+    float* As = reinterpret_cast<float*>(sm + Q_A);
+    float* Ts = reinterpret_cast<float*>(sm + Q_T);
+    float* alpha_s = reinterpret_cast<float*>(sm + Q_AL);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Q_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Q_MISC);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    // K, Q rows and Gamma: every global load of a thread before its stores
+    {
+        constexpr int PER = C * 16 / kThr;   // 16-byte pieces of K (and of Q) per thread
+        constexpr int PG = C * C / 4 / kThr;  // float4 of Gamma per thread
+        uint4 rk[PER], rq[PER];
+        float4 rg[PG];
+        const float* G = a.gamma + chunk * C * C;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15, t = n * C + r;
+            rk[u] = rq[u] = make_uint4(0, 0, 0, 0);
+            if (t < a.T) {
+                const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
+                rk[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
+                rq[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < PG; ++u) rg[u] = __ldg(reinterpret_cast<const float4*>(G) + tid + kThr * u);
+        float al = 1.f;
+        if (tid < C && n * C + tid < a.T) al = expf(a.alpha_log[tokrow(a, b, n * C + tid, h)]);
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15;
+            const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
+            float k[8], q[8];
+            unpack_bf16x8(rk[u], k);
+            unpack_bf16x8(rq[u], q);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q[e] -= a.dcorr * k[e];
+            *reinterpret_cast<uint4*>(sm + Q_KQ + off) = rk[u];
+            *reinterpret_cast<uint4*>(sm + Q_KQ + off + 8192) = bf16x8(q);  // rows 64..127
+        }
+#pragma unroll
+        for (int u = 0; u < PG; ++u) {
+            const int idx = (tid + kThr * u) * 4, r = idx / C, c = idx % C;
+            Ts[r * LAS + c] = rg[u].x;
+            Ts[r * LAS + c + 1] = rg[u].y;
+            Ts[r * LAS + c + 2] = rg[u].z;
+            Ts[r * LAS + c + 3] = rg[u].w;
+        }
+        if (tid < C) alpha_s[tid] = al;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        constexpr uint32_t id = idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t ad = smem_desc(sbase + Q_KQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128);
+            mma_bf16(tmem, ad, ad, id, ks > 0);
+        }
+        mma_commit(bar);
+    }
+    const bool ok = __syncthreads_and(mbar_wait(bar, 0));
+    tc_fence_after_sync();
+    float* att = a.att + chunk * C * C;
+    if (ok && tid < C) {
+        // column i of A and of Att from TMEM lane i (warps 0, 1: lanes 0..63)
+        const int i = tid;
+        const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll 1
+        for (int r16 = 0; r16 < C; r16 += 16) {
+            float kk[16], kh[16];
+            tmem_ld16(tmem + lane_sel + r16, kk);      // k_i . k_r
+            tmem_ld16(tmem + lane_sel + C + r16, kh);  // k_i . qhat_r
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int r = r16 + e;
+                const float av = i < r ? alpha_s[r] * kk[e] * Ts[(r - 1) * LAS + i] : 0.f;
+                const float tv = i <= r ? kh[e] * Ts[r * LAS + i] : 0.f;
+                As[r * LAS + i] = av;
+                att[r * C + i] = tv;
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();  // A complete; Gamma read
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 128);
+    }
+    if (!ok) {
+        if (tid == 0) atomicOr(a.status + 1, 1u);
+        return;
+    }
+    bwd_unit_lower_inverse(As, Ts, tid);
+    __syncthreads();
+    float* Tm = a.tmat + chunk * C * C;
+    for (int idx = tid; idx < C * C; idx += kThr) Tm[idx] = Ts[(idx / C) * LAS + idx % C];
+}
+
+// ---------------------------------------------------------------------------
 // The chunk-only operands of the tensor-core reverse chain (bf16, d = 128):
 //   U  = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T]   bf16 [256][64]  (A of U dVtilde)
 //   TT = [T^T ; 0]                                      bf16 [128][64]  (A of T^T dVtilde = dv)
@@ -933,6 +1070,18 @@ cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s)
 }  // namespace mdn
 
 namespace mdn {
+
+cudaError_t launch_bwd_prep_tc(const BwdArgs& a, cudaStream_t s)
+{
+    if (a.D != D) return cudaErrorNotSupported;
+    const long long chunks = (long long)a.B * a.H * a.NT;
+    cudaError_t e = cudaFuncSetAttribute(bwd_prep_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Q_SMEM);
+    if (e != cudaSuccess) return e;
+    ProfScope ps(kBwdPrep, s);
+    bwd_prep_tc_kernel<<<(unsigned)chunks, kThr, Q_SMEM, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s)
 {

@@ -291,6 +291,7 @@ cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s);
 // tcgen05 version of the chain's operands plus the rebuilt entering states (a scan).
 cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_prep_tc(const BwdArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) path: bf16 q, k, v with d = 128.  Returns cudaErrorNotSupported
 // when the arguments are outside what it handles.
 // Records e as this thread's last CUDA error (mdn_last_cuda_error) and
