@@ -613,16 +613,107 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 // chunk (bf16, d = 128): the forward pass's intra-chunk product on tcgen05,
 //   G = [K; Qhat] [K; Qhat]^T   (M 128, N 128, K 128; lane i < 64: k_i.k_r in
 //                                columns r, k_i.qhat_r in columns 64 + r)
-// then thread i forms column i of A and Att from lane i, and the forward
-// substitution of the CUDA-core version gives T.  Qhat is rounded to bf16 as
-// in the forward pass.
+// then thread i forms column i of A and Att from lane i, and T follows by
+// 16 x 16 blocks (inverse_blocked).  Qhat is rounded to bf16 as in the
+// forward pass.
 constexpr uint32_t Q_KQ = 0;                 // [K; Qhat] K-major: 2 panels x 128 rows x 128 B
-constexpr uint32_t Q_A = 32768;              // fp32 A [64][65]
-constexpr uint32_t Q_T = Q_A + 16640;        // fp32 Gamma [64][65], then T
-constexpr uint32_t Q_AL = Q_T + 16640;       // alpha_r
+constexpr uint32_t Q_A = 32768;              // fp32 A [64][LDF], then B_ik in place
+constexpr uint32_t Q_T = Q_A + 64 * LDF * 4; // fp32 Gamma [64][LDF], then T
+constexpr uint32_t Q_AL = Q_T + 64 * LDF * 4; // alpha_r
 constexpr uint32_t Q_BAR = Q_AL + 256;
 constexpr uint32_t Q_MISC = Q_BAR + 16;
 constexpr uint32_t Q_SMEM = Q_MISC + 16 + 1024;
+
+// acc0, acc1 += rows r0, r0 + 1 of the 16 x 16 block at X times columns
+// c0 .. c0 + 3 of the block at Y (row stride LDF).
+__device__ __forceinline__ void blk_2x4(const float* X, const float* Y, int r0, int c0, float4& acc0,
+                                        float4& acc1) {
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 a0 = lds4(X + r0 * LDF + 4 * k4), a1 = lds4(X + (r0 + 1) * LDF + 4 * k4);
+        const float x0[4] = {a0.x, a0.y, a0.z, a0.w}, x1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float4 y = lds4(Y + (4 * k4 + e) * LDF + c0);
+            acc0.x = fmaf(x0[e], y.x, acc0.x); acc0.y = fmaf(x0[e], y.y, acc0.y);
+            acc0.z = fmaf(x0[e], y.z, acc0.z); acc0.w = fmaf(x0[e], y.w, acc0.w);
+            acc1.x = fmaf(x1[e], y.x, acc1.x); acc1.y = fmaf(x1[e], y.y, acc1.y);
+            acc1.z = fmaf(x1[e], y.z, acc1.z); acc1.w = fmaf(x1[e], y.w, acc1.w);
+        }
+    }
+}
+
+// T = (I + A)^{-1} for a strictly lower 64 x 64 A (row stride LDF) into T (same
+// stride, row-major), by 16 x 16 blocks: the diagonal blocks by forward
+// substitution (one column per thread), B_ik = -T_ii A_ik in place of A_ik,
+// then T_ij = sum_{k=j}^{i-1} B_ik T_kj level by level (i - j = 1, 2, 3).
+// Every thread of the 256-thread CTA calls it; it synchronises.
+__device__ void inverse_blocked(float* A, float* T, int tid)
+{
+    if (tid < C) {
+        const int o = 16 * (tid >> 4), cl = tid & 15;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) t[r] = (r == cl) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+            float av[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 v4 = lds4(A + (o + r) * LDF + o + 4 * q4);
+                av[4 * q4] = v4.x; av[4 * q4 + 1] = v4.y; av[4 * q4 + 2] = v4.z; av[4 * q4 + 3] = v4.w;
+            }
+            float acc0 = 0.f, acc1 = 0.f;  // two partial sums: a shorter dependency chain
+#pragma unroll
+            for (int kk = 0; kk < r; kk += 2) {
+                acc0 = fmaf(av[kk], t[kk], acc0);
+                if (kk + 1 < r) acc1 = fmaf(av[kk + 1], t[kk + 1], acc1);
+            }
+            if (r > cl) t[r] = -(acc0 + acc1);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) T[(o + r) * LDF + o + cl] = t[r];
+    } else {
+        // the six blocks above the diagonal are zero
+        for (int idx = tid - C; idx < 6 * 256; idx += kThr - C) {
+            const int bidx = idx >> 8, w = idx & 255;
+            const int bi = bidx < 3 ? 0 : (bidx < 5 ? 1 : 2);
+            const int bj = bidx < 3 ? bidx + 1 : (bidx < 5 ? bidx - 1 : 3);
+            T[(16 * bi + (w >> 4)) * LDF + 16 * bj + (w & 15)] = 0.f;
+        }
+    }
+    __syncthreads();
+    // B_ik = -T_ii A_ik, blocks (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2): 32 tiles of 2 x 4 each
+    float4 r0v = make_float4(0.f, 0.f, 0.f, 0.f), r1v = r0v;
+    int where = -1;
+    if (tid < 192) {
+        const int bidx = tid >> 5;
+        const int bi = bidx < 1 ? 1 : (bidx < 3 ? 2 : 3);
+        const int bk = bidx < 1 ? 0 : (bidx < 3 ? bidx - 1 : bidx - 3);
+        const int r0 = 2 * ((tid >> 2) & 7), c0 = 4 * (tid & 3);
+        blk_2x4(T + 16 * bi * LDF + 16 * bi, A + 16 * bi * LDF + 16 * bk, r0, c0, r0v, r1v);
+        where = (16 * bi + r0) * LDF + 16 * bk + c0;
+    }
+    __syncthreads();  // every read of A_ik precedes its overwrite
+    if (where >= 0) {
+        *reinterpret_cast<float4*>(A + where) = make_float4(-r0v.x, -r0v.y, -r0v.z, -r0v.w);
+        *reinterpret_cast<float4*>(A + where + LDF) = make_float4(-r1v.x, -r1v.y, -r1v.z, -r1v.w);
+    }
+    __syncthreads();
+    for (int L = 1; L < 4; ++L) {
+        if (tid < (4 - L) * 32) {
+            const int i = L + (tid >> 5), j = i - L;
+            const int r0 = 2 * ((tid >> 2) & 7), c0 = 4 * (tid & 3);
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+            for (int kb = j; kb < i; ++kb)
+                blk_2x4(A + 16 * i * LDF + 16 * kb, T + 16 * kb * LDF + 16 * j, r0, c0, acc0, acc1);
+            float* t = T + (16 * i + r0) * LDF + 16 * j + c0;
+            *reinterpret_cast<float4*>(t) = acc0;
+            *reinterpret_cast<float4*>(t + LDF) = acc1;
+        }
+        __syncthreads();
+    }
+}
 
 __global__ void __launch_bounds__(kThr)
 bwd_prep_tc_kernel(BwdArgs a)
@@ -685,10 +776,7 @@ bwd_prep_tc_kernel(BwdArgs a)
 #pragma unroll
         for (int u = 0; u < PG; ++u) {
             const int idx = (tid + kThr * u) * 4, r = idx / C, c = idx % C;
-            Ts[r * LAS + c] = rg[u].x;
-            Ts[r * LAS + c + 1] = rg[u].y;
-            Ts[r * LAS + c + 2] = rg[u].z;
-            Ts[r * LAS + c + 3] = rg[u].w;
+            *reinterpret_cast<float4*>(Ts + r * LDF + c) = rg[u];
         }
         if (tid < C) alpha_s[tid] = al;
     }
@@ -722,9 +810,9 @@ bwd_prep_tc_kernel(BwdArgs a)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int r = r16 + e;
-                const float av = i < r ? alpha_s[r] * kk[e] * Ts[(r - 1) * LAS + i] : 0.f;
-                const float tv = i <= r ? kh[e] * Ts[r * LAS + i] : 0.f;
-                As[r * LAS + i] = av;
+                const float av = i < r ? alpha_s[r] * kk[e] * Ts[(r - 1) * LDF + i] : 0.f;
+                const float tv = i <= r ? kh[e] * Ts[r * LDF + i] : 0.f;
+                As[r * LDF + i] = av;
                 att[r * C + i] = tv;
             }
         }
@@ -739,10 +827,9 @@ bwd_prep_tc_kernel(BwdArgs a)
         if (tid == 0) atomicOr(a.status + 1, 1u);
         return;
     }
-    bwd_unit_lower_inverse(As, Ts, tid);
-    __syncthreads();
-    float* Tm = a.tmat + chunk * C * C;
-    for (int idx = tid; idx < C * C; idx += kThr) Tm[idx] = Ts[(idx / C) * LAS + idx % C];
+    inverse_blocked(As, Ts, tid);
+    float4* Tm = reinterpret_cast<float4*>(a.tmat + chunk * C * C);
+    for (int idx = tid; idx < C * C / 4; idx += kThr) Tm[idx] = lds4(Ts + (idx >> 4) * LDF + 4 * (idx & 15));
 }
 
 // ---------------------------------------------------------------------------
