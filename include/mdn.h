@@ -170,17 +170,19 @@ size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   dS0, dM0    [B,H,d,d] fp32 outputs (the gradients of the entering states).
  *   workspace   at least mdn_chunk_bwd_workspace_size(...) bytes, 256-byte
  *               aligned (about (4 d^2 + 3 C^2 + 10 C) x 4 bytes per chunk of C
- *               tokens of each head).
+ *               tokens of each head, plus about 260 KB per chunk for the
+ *               tensor-core path's chunk operands).
  *   flags       0, or MDN_CHECK_FINITE (synchronise, then report non-finite
  *               outputs or an expired device wait) and/or MDN_FORCE_SIMT (the
  *               CUDA-core kernels for bf16 d = 128 too).
  *
- * bf16 inputs with d = 128 run the products with the states on tcgen05
- * tensor cores (bf16 operands, fp32 accumulation); everything else, and
- * every other input combination, runs in fp32 on CUDA cores.  Support and
- * errors as mdn_chunk_fwd (T = 0 copies dS_T, dM_T to dS0, dM0).
- * Asynchronous on `stream` (except with MDN_CHECK_FINITE); enqueues six
- * kernels, one of them on a side stream of the library that joins back.
+ * bf16 inputs with d = 128 run every product on tcgen05 tensor cores (bf16
+ * operands, fp32 accumulation; the reverse chain of the state adjoints as a
+ * warp-specialised chain like the forward pass's): seven kernels on `stream`.
+ * Every other input combination runs in fp32 on CUDA cores: six kernels, the
+ * state rebuild on a side stream of the library that joins back.  Support
+ * and errors as mdn_chunk_fwd (T = 0 copies dS_T, dM_T to dS0, dM0).
+ * Asynchronous on `stream` (except with MDN_CHECK_FINITE).
  */
 mdn_status mdn_chunk_bwd(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
                          const float *alpha_log, const float *mu_log,
