@@ -28,7 +28,8 @@ sys.path.insert(0, ROOT)
 import mdn_inputs as mi  # noqa: E402
 
 METRIC = "MDN chunk-fwd tokens/s (d=128, bf16 in/fp32 state) and % tensor/HBM roofline"
-DEFAULT_WORKLOAD = 1           # B=4, H=8, T=2048, d=128, bf16
+DEFAULT_WORKLOAD = 2           # the largest single-GPU workload: B=8, H=16, T=4096, d=128, S0/M0 != 0
+SIDE_WORKLOADS = (1, 3)        # timed the same way, reported beside the headline
 L2_FLUSH_BYTES = 256 << 20     # > 126 MB of L2
 FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x FP32 lanes x FMA x max clock
 
@@ -52,20 +53,41 @@ def load_traffic():
         return {}
 
 
+def pass_work(spec: mi.Spec):
+    """The chunk pass's algorithmic minimum (the method's own contractions and
+    the bytes it must move), per token-head: flops = 12 C d + 12 d^2 (the six
+    C^2-type products K K^T, Qhat K^T, T V, T Y, T Z and the intra-chunk output,
+    and the six C d^2-type products Y S, Z M, Qhat S, Qhat M and the two state
+    increments; the T solve and Gamma excluded); bytes = q, k, v read and o,
+    vtilde written in the input dtype, plus four fp32 gates; plus, per head, the
+    fp32 S_T, M_T written and S0, M0 read when given.  Returns (bytes, flops)."""
+    th = spec.B * spec.T * spec.H
+    d, C = spec.d, spec.C
+    elt = 2 if spec.dtype == "bf16" else 4
+    heads = spec.B * spec.H
+    states = 2 * heads * d * d * 4 * (2 if spec.state_std > 0 else 1)
+    return th * (5 * d * elt + 16) + states, th * (12.0 * C * d + 12.0 * d * d)
+
+
+def token_bytes(spec: mi.Spec) -> int:
+    """One decode token for every head: S and M read and written (fp32), q, k,
+    v read, o written, four gates."""
+    heads, d = spec.B * spec.H, spec.d
+    elt = 2 if spec.dtype == "bf16" else 4
+    return heads * (4 * d * d * 4 + 4 * d * elt + 16)
+
+
 def kernel_work(name: str, spec: mi.Spec):
     """Algorithmic work of one launch of a kernel: (bound, amount, unit-of-peak).
-    Chunk kernels process every token-head of the batch per launch; the decode
-    kernel processes every head once."""
+    The tensor-core chunk kernels are charged the whole pass's algorithmic
+    bytes (they split one pass between them; neither alone has a minimum of
+    its own), the CUDA-core kernels their fp32 flops, the decode step its
+    bytes."""
     th = spec.B * spec.T * spec.H          # token-heads
     d, C = spec.d, spec.C
     heads = spec.B * spec.H
-    states = 2 * heads * d * d * 4 * (2 if spec.state_std > 0 else 1)  # S_T,M_T (+S0,M0)
-    if name == "inter_tc":
-        # the bytes it must move: q, k, v read and o, vtilde written (bf16), plus the states
-        return "hbm", th * (5 * d * 2) + states, "GB/s"
-    if name == "intra_tc":
-        # q, k, gates read; Qhat, [T; Att T], A2T and the chunk record written
-        return "hbm", th * (2 * d * 2 + 16) + th * (d * 2 + 2 * C * 2 + 2 * d * 2 + 16), "GB/s"
+    if name in ("inter_tc", "intra_tc"):
+        return "hbm", pass_work(spec)[0], "GB/s"
     if name == "inter_simt":
         return "alu", th * 12.0 * d * d, "TFLOP/s"
     if name == "intra_simt":
@@ -77,6 +99,18 @@ def kernel_work(name: str, spec: mi.Spec):
     if name == "step":
         return "hbm", heads * (4 * d * d * 4 + 3 * d * 2 + 16 + 2 * d * 2), "GB/s"
     return None, 0.0, ""
+
+
+def fractions(nbytes: float, flops: float, sec: float, hbm: float, bf16: float) -> dict:
+    """HBM, tensor and roofline fractions of work done in `sec` seconds:
+    roofline = max(flops / tensor peak, bytes / HBM peak) / sec."""
+    if sec <= 0:
+        return {"hbm_frac": None, "tensor_frac": None, "roofline_frac": None}
+    return {"achieved_gbs": round(nbytes / sec / 1e9, 1),
+            "achieved_tflops": round(flops / sec / 1e12, 2),
+            "hbm_frac": round(nbytes / sec / 1e9 / hbm, 4),
+            "tensor_frac": round(flops / sec / 1e12 / bf16, 4),
+            "roofline_frac": round(max(flops / (bf16 * 1e12), nbytes / (hbm * 1e9)) / sec, 4)}
 
 
 # ---------------------------------------------------------------- clocks
@@ -147,102 +181,179 @@ def decode_token(spec: mi.Spec, seed: int):
     return inp
 
 
+class Pass:
+    """One workload's step (mdn_chunk_fwd over the batch + one decode token that
+    continues from its (S_T, M_T)) with its device buffers, ready to time."""
+
+    def __init__(self, mdn, spec: mi.Spec, device):
+        self.mdn, self.spec = mdn, spec
+        self.inp = mi.make_inputs(spec)
+        self.tok = decode_token(spec, spec.seed + 1)
+        self.dev = mi.to_torch(self.inp, device)
+        self.dtok = {k: (v[:, 0].contiguous() if v is not None else None)
+                     for k, v in mi.to_torch(self.tok, device).items()}
+        B, T, H, d = spec.B, spec.T, spec.H, spec.d
+        self.ws = torch.empty(mdn.chunk_fwd_workspace_size(B, T, H, d, spec.C, self.dev["q"].dtype),
+                              dtype=torch.uint8, device=device)
+        self.out = (torch.empty_like(self.dev["q"]), torch.empty_like(self.dev["q"]),
+                    torch.empty((B, H, d, d), dtype=torch.float32, device=device),
+                    torch.empty((B, H, d, d), dtype=torch.float32, device=device))
+        self.o1 = torch.empty_like(self.dtok["q"])
+
+    def step(self):
+        g = ("alpha_log", "mu_log", "beta", "eta")
+        dev, dtok, spec = self.dev, self.dtok, self.spec
+        self.mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[x] for x in g), self.inp.d_corr,
+                           dev["S0"], dev["M0"], spec.C, out=self.out, workspace=self.ws)
+        self.mdn.step(dtok["q"], dtok["k"], dtok["v"], *(dtok[x] for x in g), self.inp.d_corr,
+                      self.out[2], self.out[3], o=self.o1, want_vtilde=False)
+
+    def time(self, steps: int, warmup: int, flush, world: int, clock=None):
+        """Per-step device times (ms) of `steps` steps after `warmup` untimed ones,
+        L2 flushed (untimed) before each; then the library's per-kernel times
+        from a second, untimed pass over the same number of steps (its events
+        between kernels would otherwise serialise the two chunk kernels, which
+        overlap in the timed pass)."""
+        mdn = self.mdn
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with (clock if clock is not None else _Null()):
+            for i in range(steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                self.step()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        mdn.profile_enable(True)
+        mdn.profile_read(reset=True)
+        for _ in range(steps):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        kernels = mdn.profile_read(reset=True)
+        mdn.profile_enable(False)
+        status = mdn.chunk_fwd_status(self.ws)
+        if status != 0:
+            raise RuntimeError(f"chunk pass reported {mdn.status_string(status)}")
+        return step_ms, kernels
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def pass_summary(spec: mi.Spec, ms: float, kernels: dict, steps: int, hbm: float, bf16: float):
+    """Throughput and roofline fractions of one workload's step: over the whole
+    step (pass + decode token) and over the pass's dominant kernel."""
+    nbytes, flops = pass_work(spec)
+    tb = token_bytes(spec)
+    out = {"workload": spec.name, "ms_per_step": round(ms, 5),
+           "tokens_per_s": round(spec.B * spec.T / (ms * 1e-3), 1),
+           "step": fractions(nbytes + tb, flops, ms * 1e-3, hbm, bf16),
+           "kernels_us": {k: round(v[0] / v[1] * 1e3, 2) for k, v in kernels.items()}}
+    chunk = {k: v for k, v in kernels.items() if k != "step"}
+    if chunk:
+        name, (tot, n) = max(chunk.items(), key=lambda kv: kv[1][0])
+        out["dominant"] = dict(kernel=name, us=round(tot / n * 1e3, 2),
+                               **fractions(nbytes, flops, tot / n * 1e-3, hbm, bf16))
+    return out
+
+
+def config_block(spec: mi.Spec, world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H, "d_k": spec.d,
+            "d_v": spec.d, "C": spec.C, "inputs": spec.dtype, "state": "fp32",
+            "S0_M0": "N(0, %g^2)" % spec.state_std if spec.state_std > 0 else "zero",
+            "step": "mdn_chunk_fwd over the batch + 1 mdn_step token",
+            "l2": "flushed before every timed step (256 MiB write, untimed)",
+            "parallelism": f"replicas x{world} (independent heads, no collective)",
+            "global_batch": spec.B * world, "seq_len": spec.T}
+
+
 def run_ours(args, rank, world, device):
     import momentum_delta_rule_mdn_b200 as mdn
 
     spec0 = workload_spec(args.workload)
     spec = rank_spec(spec0, rank)
-    inp = mi.make_inputs(spec)
-    tok = decode_token(spec, spec.seed + 1)
-    dev = mi.to_torch(inp, device)
-    dtok = {k: (v[:, 0].contiguous() if v is not None else None)
-            for k, v in mi.to_torch(tok, device).items()}
-    B, T, H, d = spec.B, spec.T, spec.H, spec.d
-    ws = torch.empty(mdn.chunk_fwd_workspace_size(B, T, H, d, spec.C, dev["q"].dtype),
-                     dtype=torch.uint8, device=device)
-    o = torch.empty_like(dev["q"])
-    vt = torch.empty_like(dev["q"])
-    S_T = torch.empty((B, H, d, d), dtype=torch.float32, device=device)
-    M_T = torch.empty_like(S_T)
-    o1 = torch.empty_like(dtok["q"])
+    hbm, bf16, peak_src = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    gates = ("alpha_log", "mu_log", "beta", "eta")
-
-    def step():
-        mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), inp.d_corr,
-                      dev["S0"], dev["M0"], spec.C, out=(o, vt, S_T, M_T), workspace=ws)
-        mdn.step(dtok["q"], dtok["k"], dtok["v"], *(dtok[g] for g in gates), inp.d_corr,
-                 S_T, M_T, o=o1, want_vtilde=False)
-
-    stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-
-    # ---- timed region: K steps, L2 flushed (untimed) before each
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(device.index) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-
-    # ---- per-kernel device times, from a second (untimed) pass over the same
-    # steps: the library's events between kernels would serialise the
-    # intra- and inter-chunk kernels, which overlap in the timed pass
-    mdn.profile_enable(True)
-    mdn.profile_read(reset=True)
-    for i in range(args.steps):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    kernels = mdn.profile_read(reset=True)
-    mdn.profile_enable(False)
+    main = Pass(mdn, spec, device)
+    B, T, H, d = spec.B, spec.T, spec.H, spec.d
+    clk = ClockSampler(device.index)   # sampled during the timed steps only
+    step_ms, kernels = main.time(args.steps, args.warmup, flush, world, clock=clk)
+    clocks = clk.summary()
     ms = float(np.mean(step_ms))
     ms_max = max_over_ranks(ms, world, device)
-
     value = whole_job_value(B * T, world, ms_max)
 
-    # ---- dominant kernel and its roofline
-    hbm, bf16, peak_src = load_peaks()
-    dom = max(kernels.items(), key=lambda kv: kv[1][0]) if kernels else None
+    # ---- dominant kernel and its roofline: the pass's algorithmic bytes and
+    # flops (pass_work) over that kernel's average device time
+    nbytes, flops = pass_work(spec)
     roofline = None
     gpu_launches = sum(n for _, n in kernels.values())
-    if dom:
-        name, (tot_ms, n) = dom
+    chunk = {k: v for k, v in kernels.items() if k != "step"}
+    if chunk:
+        name, (tot_ms, n) = max(chunk.items(), key=lambda kv: kv[1][0])
         bound, work, unit = kernel_work(name, spec)
         avg_s = tot_ms / n * 1e-3
         if bound == "hbm":
             achieved, peak = work / avg_s / 1e9, hbm
-        elif bound == "tensor":
-            achieved, peak = work / avg_s / 1e12, bf16
         else:
             achieved, peak = work / avg_s / 1e12, FP32_ALU_PEAK_TFLOPS
         tr = load_traffic().get(name, {})
         traffic = tr.get("bytes_per_launch") if tr.get("workload") == spec0.name else None
+        fr = fractions(nbytes, flops, avg_s, hbm, bf16)
         roofline = {"kernel": name, "bound": bound, "achieved": round(achieved, 3),
                     "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
                     "traffic": traffic,
-                    "peak_source": peak_src if bound != "alu" else
-                    "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz",
+                    "peak_source": (f"{peak_src} (MEASURED_PEAKS.json: copy GB/s, bf16 burst TFLOP/s)"
+                                    if bound != "alu" else
+                                    "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz"),
+                    "work": {"bytes": int(nbytes), "flops": flops,
+                             "per_token_head": {"bytes": (5 * d * (2 if spec.dtype == "bf16" else 4)
+                                                          + 16),
+                                                "flops": 12 * spec.C * d + 12 * d * d},
+                             "states_bytes": int(nbytes - B * T * H * (5 * d * (2 if spec.dtype == "bf16" else 4) + 16))},
+                    "tensor": {"achieved_tflops": fr["achieved_tflops"], "peak": bf16,
+                               "frac": fr["tensor_frac"]},
+                    "roofline_frac": fr["roofline_frac"],
                     "kernel_ms_avg": round(tot_ms / n, 5),
-                    "share_of_step": round(tot_ms / args.steps / ms, 4)}
+                    "share_of_step": round(tot_ms / args.steps / ms, 4),
+                    "step": fractions(nbytes + token_bytes(spec), flops, ms_max * 1e-3, hbm, bf16)}
+
+    # ---- the other workloads, timed the same way (rank 0's batch shapes)
+    configs = {}
+    if not args.no_side_configs:
+        for w in SIDE_WORKLOADS:
+            if mi.WORKLOADS[w].name == spec0.name:
+                continue
+            sp = rank_spec(mi.WORKLOADS[w], rank)
+            p = Pass(mdn, sp, device)
+            sms, sk = p.time(max(5, min(args.steps, 20)), args.warmup, flush, world)
+            configs[sp.name] = pass_summary(sp, float(np.mean(sms)), sk, len(sms), hbm, bf16)
+            del p
+    main_summary = pass_summary(spec, ms, kernels, args.steps, hbm, bf16)
 
     # ---- end to end through the public call, host (pinned) buffers
-    e2e = None if args.no_e2e else run_e2e(args, mdn, inp, tok, spec, device, world)
+    e2e = None if args.no_e2e else run_e2e(args, mdn, main.inp, main.tok, spec, device, world)
     side = set() if args.no_decode else set(args.side.split(","))
     decode = run_decode(args, mdn, device, hbm) if "decode" in side else None
     gates = run_gate_params(args, mdn, device, hbm, B * T * H) if "gates" in side else None
     varlen = run_varlen(args, mdn, device, spec0) if "varlen" in side else None
-    backward = run_backward(args, mdn, device, spec0) if "backward" in side else None
+    backward = run_backward(args, mdn, device, mi.WORKLOADS[1]) if "backward" in side else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -250,17 +361,14 @@ def run_ours(args, rank, world, device):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if "inter_tc" in kernels else "f32",
         "data": "synthetic (seeded generator; gates from the stable parameterisation)",
-        "config": {"workload": spec0.name, "B": B, "T": T, "H": H, "d_k": d, "d_v": d,
-                   "C": spec.C, "inputs": spec.dtype, "state": "fp32",
-                   "step": "mdn_chunk_fwd over the batch + 1 mdn_step token",
-                   "l2": "flushed before every timed step (256 MiB write, untimed)",
-                   "parallelism": f"replicas x{world} (independent heads, no collective)",
-                   "global_batch": B * world, "seq_len": T},
+        "config": config_block(spec0, world),
         "roofline": roofline,
         "kernels": {k: {"ms_total": round(v[0], 4), "launches": v[1]} for k, v in kernels.items()},
         "gpu_launches": gpu_launches,
         "e2e": e2e,
-        "clocks": clk.summary(),
+        "clocks": clocks,
+        "headline": main_summary,
+        "configs": configs,
     }
     if decode:
         line["decode"] = decode
@@ -615,10 +723,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
-                       "d_k": spec.d, "d_v": spec.d, "C": spec.C,
-                       "step": "oracle forward over the sample + 1 decode token",
-                       "global_batch": spec.B, "seq_len": spec.T},
+            "config": config_block(spec, world),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -667,13 +772,15 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=None, help="config name or index (default: 1)")
+    ap.add_argument("--workload", default=None, help="config name or index (default: 2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip every side measurement")
     ap.add_argument("--side", default="decode,gates,varlen,backward",
                     help="side measurements after the timed step (comma list of decode, gates, "
                          "varlen, backward)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-side-configs", action="store_true",
+                    help="skip timing the other workloads beside the headline one")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

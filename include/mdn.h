@@ -98,11 +98,40 @@ const char *mdn_status_string(mdn_status status);
 const char *mdn_last_cuda_error(void);
 
 /*
- * Bytes of device scratch that mdn_chunk_fwd needs for these sizes, or 0 if
- * the sizes are invalid or unsupported.  Pure host function.
+ * Bytes of device scratch that mdn_chunk_fwd needs for these sizes with
+ * flags = 0, or 0 if the sizes are invalid or unsupported.  Pure host
+ * function.  The scratch is sized for the path the call takes: bf16 input
+ * with d = 128 runs on the tensor cores and needs about 1 KB per chunk of C
+ * tokens of each head (the per-chunk operands of the sequential kernel); every
+ * other case runs on CUDA cores and needs about (C + 4 d + 4) x 4 bytes per
+ * token and head.
  */
 size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
                                     mdn_dtype in_dtype);
+
+/*
+ * As mdn_chunk_fwd_workspace_size, for the path that `flags` selects (with
+ * MDN_FORCE_SIMT, bf16 d = 128 input takes the CUDA-core path and needs its
+ * larger scratch).  A workspace sized for flags = 0 is too small for such a
+ * call, which then returns MDN_ERR_INVALID_ARG.  Pure host function.
+ */
+size_t mdn_chunk_fwd_workspace_size_flags(int B, int T, int H, int dk, int dv, int C,
+                                          mdn_dtype in_dtype, int flags);
+
+/*
+ * What the kernels of the last mdn_chunk_fwd or mdn_chunk_fwd_varlen call on
+ * this workspace recorded on the device, for callers that do not pass
+ * MDN_CHECK_FINITE (which makes the pass itself synchronise and report).  Synchronises `stream` (the stream that call used)
+ * and returns MDN_OK, MDN_ERR_TIMEOUT (a bounded device wait ran out: the
+ * call's outputs are undefined), MDN_ERR_INVALID_ARG (packed sequences only:
+ * cu_seqlens broke its rules, every sequence was treated as empty) or
+ * MDN_ERR_NONFINITE (only after a call with MDN_CHECK_FINITE).  Every chunk
+ * pass clears these words before its kernels run.  (mdn_chunk_fwd_noalloc has
+ * no caller workspace; pass it MDN_CHECK_FINITE to have it report.)
+ *   workspace   the workspace pointer passed to that call (256-byte aligned).
+ * Errors: MDN_ERR_INVALID_ARG (null or unaligned workspace), MDN_ERR_CUDA.
+ */
+mdn_status mdn_chunk_fwd_status(const void *workspace, mdn_stream_t stream);
 
 /*
  * Chunkwise forward pass over a whole sequence (summary, steps 2-5; the
@@ -118,8 +147,10 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   o, vtilde   [B,T,H,d] in_dtype outputs (vtilde is the materialised Vtilde).
  *   S_T, M_T    [B,H,d,d] fp32 outputs: the states after token T.  They may
  *               alias S0 / M0 (read before written, per head).
- *   workspace   device scratch of at least mdn_chunk_fwd_workspace_size(...)
- *               bytes, 256-byte aligned; its contents on entry do not matter.
+ *   workspace   device scratch of at least
+ *               mdn_chunk_fwd_workspace_size_flags(..., flags) bytes (for
+ *               flags without MDN_FORCE_SIMT, mdn_chunk_fwd_workspace_size),
+ *               256-byte aligned; its contents on entry do not matter.
  *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT, plus at most one of
  *               MDN_SLICE32 / MDN_SLICE64 (and MDN_TEST_NO_INTRA in tests).
  *
@@ -129,10 +160,13 @@ size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  * Errors: MDN_ERR_INVALID_ARG (null required pointer, negative size,
  * unaligned pointer, too-small workspace), MDN_ERR_UNSUPPORTED (d, C or dtype
  * outside support), MDN_ERR_CUDA (launch failure), and with MDN_CHECK_FINITE
- * also MDN_ERR_NONFINITE / MDN_ERR_TIMEOUT.
+ * also MDN_ERR_NONFINITE / MDN_ERR_TIMEOUT.  Without MDN_CHECK_FINITE an
+ * expired device wait (MDN_ERR_TIMEOUT; the outputs are then undefined) is
+ * only recorded in the workspace: mdn_chunk_fwd_status reads it.
  *
- * Asynchronous on `stream` (except with MDN_CHECK_FINITE).  The bf16 d = 128
- * path enqueues a small memset of the workspace and two kernels, the second
+ * Asynchronous on `stream` (except with MDN_CHECK_FINITE).  Every call first
+ * clears the workspace's status words with a small memset.  The bf16 d = 128
+ * path then enqueues two kernels, the second
  * launched as the first one's programmatic dependent; the sequence can be
  * captured in a CUDA graph and replayed.  Calls that may run concurrently
  * need separate workspaces.
@@ -200,6 +234,13 @@ mdn_status mdn_chunk_bwd(const void *q, const void *k, const void *v, mdn_dtype 
  */
 size_t mdn_chunk_fwd_varlen_workspace_size(int N, int total_T, int H, int dk, int dv, int C,
                                            mdn_dtype in_dtype);
+
+/*
+ * As mdn_chunk_fwd_varlen_workspace_size, for the path that `flags` selects
+ * (see mdn_chunk_fwd_workspace_size_flags).  Pure host function.
+ */
+size_t mdn_chunk_fwd_varlen_workspace_size_flags(int N, int total_T, int H, int dk, int dv,
+                                                 int C, mdn_dtype in_dtype, int flags);
 
 /*
  * mdn_chunk_fwd over N independent sequences of different lengths packed
@@ -336,8 +377,12 @@ mdn_status mdn_chunk_gate_prep(const float *alpha_log, const float *mu_log,
  * The scratch is one fixed array of 64 MiB in device memory per GPU, created
  * when the library is loaded on that GPU and held until the process exits.
  * Arguments and results are exactly those of mdn_chunk_fwd (minus workspace
- * and ws_bytes).  Sizes whose scratch need, mdn_chunk_fwd_workspace_size(...),
- * exceeds 64 MiB are rejected with MDN_ERR_UNSUPPORTED before anything runs.
+ * and ws_bytes).  Sizes whose scratch need,
+ * mdn_chunk_fwd_workspace_size_flags(..., flags), exceeds 64 MiB are rejected
+ * with MDN_ERR_UNSUPPORTED before anything runs (on the tensor-core path that
+ * is about 63,000 chunks of 64 tokens, e.g. B*H = 32 heads of T = 120,000);
+ * invalid or unsupported arguments get mdn_chunk_fwd's own error, also
+ * before any device work.
  *
  * - The scratch of the CURRENT device is used; `stream` must belong to it.
  * - The first call on a device looks up the array's device address (a

@@ -26,6 +26,8 @@ SIGNATURES = {
     "mdn_status_string": (ctypes.c_char_p, [_i]),
     "mdn_last_cuda_error": (ctypes.c_char_p, []),
     "mdn_chunk_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "mdn_chunk_fwd_workspace_size_flags": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "mdn_chunk_fwd_status": (_i, [_vp, _vp]),
     "mdn_chunk_fwd": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                            _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp]),
     "mdn_step": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
@@ -39,6 +41,7 @@ SIGNATURES = {
                            _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                            _vp, _vp, _vp, _vp, _sz, _i, _vp]),
     "mdn_chunk_fwd_varlen_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "mdn_chunk_fwd_varlen_workspace_size_flags": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "mdn_chunk_fwd_varlen": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _i, _i,
                                   _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i,
                                   _vp]),

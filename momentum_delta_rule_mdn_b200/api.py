@@ -71,9 +71,17 @@ def _need(t: Optional[torch.Tensor], dtype, shape, name):
 
 
 def chunk_fwd_workspace_size(B: int, T: int, H: int, d: int, C: int = 64,
-                             dtype: torch.dtype = torch.bfloat16) -> int:
+                             dtype: torch.dtype = torch.bfloat16, flags: int = 0) -> int:
+    """Scratch bytes of :func:`chunk_fwd` for these sizes and flags (the path they select)."""
     code = _lib.MDN_BF16 if dtype == torch.bfloat16 else _lib.MDN_F32
-    return int(library().mdn_chunk_fwd_workspace_size(B, T, H, d, d, C, code))
+    return int(library().mdn_chunk_fwd_workspace_size_flags(B, T, H, d, d, C, code, int(flags)))
+
+
+def chunk_fwd_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises ``stream`` and returns the status code that the kernels of the
+    last chunk pass on ``workspace`` recorded (0 = MDN_OK; MDN_ERR_TIMEOUT means a
+    bounded device wait ran out and the outputs are undefined)."""
+    return int(library().mdn_chunk_fwd_status(_ptr(workspace), _stream_handle(stream)))
 
 
 def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0=None,
@@ -117,7 +125,7 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0
         _need(S_T, torch.float32, (B, H, D, D), "S_T")
         _need(M_T, torch.float32, (B, H, D, D), "M_T")
     lib = library()
-    ws_bytes = int(lib.mdn_chunk_fwd_workspace_size(B, T, H, D, D, C, code))
+    ws_bytes = int(lib.mdn_chunk_fwd_workspace_size_flags(B, T, H, D, D, C, code, int(flags)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     status = lib.mdn_chunk_fwd(
@@ -193,7 +201,8 @@ def chunk_fwd_varlen(q, k, v, alpha_log, mu_log, beta, eta, cu_seqlens: torch.Te
         _need(S_T, torch.float32, (N, H, D, D), "S_T")
         _need(M_T, torch.float32, (N, H, D, D), "M_T")
     lib = library()
-    ws_bytes = int(lib.mdn_chunk_fwd_varlen_workspace_size(N, total_T, H, D, D, C, code))
+    ws_bytes = int(lib.mdn_chunk_fwd_varlen_workspace_size_flags(N, total_T, H, D, D, C, code,
+                                                                 int(flags)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     status = lib.mdn_chunk_fwd_varlen(

@@ -23,30 +23,45 @@ bool aligned_elem(const void* p, mdn_dtype dt) {
 }
 
 struct WsLayout {
-    size_t status, la, lm, lc, bco, gamma, U, Y, Z, Oi, qhat, tat, a2t, crec, ready, total;
+    size_t status, ready, la, lm, lc, bco, gamma, U, Y, Z, Oi, qhat, tat, a2t, crec, total;
+    size_t head;  // bytes from the start that every call zeroes: status words and ready flags
 };
 
-// Byte offsets of every scratch region for these sizes.
-WsLayout ws_layout(long long BH, int NT, int D)
+// Whether a chunk pass with these arguments runs on the tensor cores.
+bool uses_tensor_cores(mdn_dtype dt, int D, int flags)
 {
-    const size_t rows = (size_t)BH * NT * kChunk;  // positions, padded to whole chunks
-    WsLayout w;
+    return dt == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
+}
+
+// Byte offsets of the scratch regions of the path that will run (tc: the
+// tensor-core path; else the CUDA-core path).  The status words and the
+// ready flags sit together at the start so that one memset clears both.
+WsLayout ws_layout(long long BH, int NT, int D, bool tc)
+{
+    const size_t chunks = (size_t)BH * NT;
+    const size_t rows = chunks * kChunk;  // positions, padded to whole chunks
+    WsLayout w = {};
     size_t off = 0;
-    w.status = off; off += align_up(64);
-    w.la = off;     off += align_up(rows * sizeof(float));
-    w.lm = off;     off += align_up(rows * sizeof(float));
-    w.lc = off;     off += align_up(rows * sizeof(float));
-    w.bco = off;    off += align_up(rows * sizeof(float));
-    w.gamma = off;  off += align_up(rows * kChunk * sizeof(float));
-    w.U = off;      off += align_up(rows * D * sizeof(float));
-    w.Y = off;      off += align_up(rows * D * sizeof(float));
-    w.Z = off;      off += align_up(rows * D * sizeof(float));
-    w.Oi = off;     off += align_up(rows * D * sizeof(float));
-    w.qhat = off;   off += align_up(rows * D * 2);
-    w.tat = off;    off += align_up(rows * 2 * kChunk * 2);
-    w.a2t = off;    off += align_up(rows * 2 * D * 2);
-    w.crec = off;   off += align_up(rows * 4 * sizeof(float));
-    w.ready = off;  off += align_up(((size_t)BH * NT + 1) * sizeof(unsigned));
+    w.status = off; off += 64;
+    w.ready = off;  off += (chunks + 1) * sizeof(unsigned);
+    w.head = off;
+    off = align_up(off);
+    if (tc) {
+        w.qhat = off;   off += align_up(rows * D * 2);
+        w.tat = off;    off += align_up(rows * 2 * kChunk * 2);
+        w.a2t = off;    off += align_up(rows * 2 * D * 2);
+        w.crec = off;   off += align_up(rows * 4 * sizeof(float));
+    } else {
+        w.la = off;     off += align_up(rows * sizeof(float));
+        w.lm = off;     off += align_up(rows * sizeof(float));
+        w.lc = off;     off += align_up(rows * sizeof(float));
+        w.bco = off;    off += align_up(rows * sizeof(float));
+        w.gamma = off;  off += align_up(rows * kChunk * sizeof(float));
+        w.U = off;      off += align_up(rows * D * sizeof(float));
+        w.Y = off;      off += align_up(rows * D * sizeof(float));
+        w.Z = off;      off += align_up(rows * D * sizeof(float));
+        w.Oi = off;     off += align_up(rows * D * sizeof(float));
+    }
     w.total = off;
     return w;
 }
@@ -66,39 +81,42 @@ mdn_status check_sizes(int B, int T, int H, int dk, int dv, int C, mdn_dtype dt)
 
 mdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MDN_OK : mdn::cuda_fail(e); }
 
-// Points the scratch members of a at their regions of ws.
+// Points the scratch members of a at their regions of ws (null for the
+// regions the other path uses).
 void carve(ChunkArgs& a, char* ws, const WsLayout& w)
 {
+    auto at = [ws](size_t off) -> char* { return off ? ws + off : nullptr; };
     a.status = reinterpret_cast<unsigned*>(ws + w.status);
-    a.la = reinterpret_cast<float*>(ws + w.la);
-    a.lm = reinterpret_cast<float*>(ws + w.lm);
-    a.lc = reinterpret_cast<float*>(ws + w.lc);
-    a.bco = reinterpret_cast<float*>(ws + w.bco);
-    a.gamma = reinterpret_cast<float*>(ws + w.gamma);
-    a.U = reinterpret_cast<float*>(ws + w.U);
-    a.Y = reinterpret_cast<float*>(ws + w.Y);
-    a.Z = reinterpret_cast<float*>(ws + w.Z);
-    a.Oi = reinterpret_cast<float*>(ws + w.Oi);
-    a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + w.qhat);
-    a.tat = reinterpret_cast<__nv_bfloat16*>(ws + w.tat);
-    a.a2t = reinterpret_cast<__nv_bfloat16*>(ws + w.a2t);
-    a.crec = reinterpret_cast<float*>(ws + w.crec);
     a.ready = reinterpret_cast<unsigned*>(ws + w.ready);
+    a.la = reinterpret_cast<float*>(at(w.la));
+    a.lm = reinterpret_cast<float*>(at(w.lm));
+    a.lc = reinterpret_cast<float*>(at(w.lc));
+    a.bco = reinterpret_cast<float*>(at(w.bco));
+    a.gamma = reinterpret_cast<float*>(at(w.gamma));
+    a.U = reinterpret_cast<float*>(at(w.U));
+    a.Y = reinterpret_cast<float*>(at(w.Y));
+    a.Z = reinterpret_cast<float*>(at(w.Z));
+    a.Oi = reinterpret_cast<float*>(at(w.Oi));
+    a.qhat = reinterpret_cast<__nv_bfloat16*>(at(w.qhat));
+    a.tat = reinterpret_cast<__nv_bfloat16*>(at(w.tat));
+    a.a2t = reinterpret_cast<__nv_bfloat16*>(at(w.a2t));
+    a.crec = reinterpret_cast<float*>(at(w.crec));
 }
 
-// The chunk pass over a (scratch carved; status zeroed by the caller when
-// MDN_CHECK_FINITE is set).  ntok: elements of o and of vt; nstate: heads of
-// S_T and M_T.
-mdn_status run_pass(ChunkArgs& a, mdn_dtype in_dtype, int flags, cudaStream_t s, size_t ntok,
-                    size_t nstate)
+// The chunk pass over a (scratch carved from layout w).  The status words
+// and ready flags are zeroed first on every call, so that
+// mdn_chunk_fwd_status can report what this call's kernels recorded.
+// ntok: elements of o and of vt; nstate: heads of S_T and M_T.
+// zero_head: false when the caller has already zeroed the head (packed
+// sequences zero it before their offset check writes status[2]).
+mdn_status run_pass(ChunkArgs& a, const WsLayout& w, mdn_dtype in_dtype, int flags,
+                    cudaStream_t s, size_t ntok, size_t nstate, bool zero_head = true)
 {
     cudaError_t e;
     const int D = a.D;
-    const bool tensor_cores = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
-    if (tensor_cores) {
+    if (zero_head && (e = cudaMemsetAsync(a.status, 0, w.head, s))) return mdn::cuda_fail(e);
+    if (uses_tensor_cores(in_dtype, D, flags)) {
         const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
-        if ((e = cudaMemsetAsync(a.ready, 0, ((size_t)a.B * a.H * a.NT + 1) * sizeof(unsigned), s)))
-            return mdn::cuda_fail(e);
         a.test_no_intra = (flags & MDN_TEST_NO_INTRA) != 0;
         if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
     } else {
@@ -193,12 +211,33 @@ const char* mdn_status_string(mdn_status s)
     return "unknown mdn_status";
 }
 
-size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
-                                    mdn_dtype in_dtype)
+size_t mdn_chunk_fwd_workspace_size_flags(int B, int T, int H, int dk, int dv, int C,
+                                          mdn_dtype in_dtype, int flags)
 {
     if (check_sizes(B, T, H, dk, dv, C, in_dtype) != MDN_OK) return 0;
     const int NT = (T + C - 1) / C;
-    return ws_layout((long long)B * H, NT, dk).total;
+    return ws_layout((long long)B * H, NT, dk, uses_tensor_cores(in_dtype, dk, flags)).total;
+}
+
+size_t mdn_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    mdn_dtype in_dtype)
+{
+    return mdn_chunk_fwd_workspace_size_flags(B, T, H, dk, dv, C, in_dtype, 0);
+}
+
+mdn_status mdn_chunk_fwd_status(const void* workspace, mdn_stream_t stream)
+{
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned host_status[3] = {0, 0, 0};
+    cudaError_t e = cudaMemcpyAsync(host_status, workspace, sizeof(host_status),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return mdn::cuda_fail(e);
+    if (host_status[2]) return MDN_ERR_INVALID_ARG;
+    if (host_status[1]) return MDN_ERR_TIMEOUT;
+    if (host_status[0]) return MDN_ERR_NONFINITE;
+    return MDN_OK;
 }
 
 mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
@@ -237,7 +276,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
         if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
     if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MDN_ERR_INVALID_ARG;
     const int NT = (T + C - 1) / C;
-    const WsLayout w = ws_layout((long long)B * H, NT, D);
+    const WsLayout w = ws_layout((long long)B * H, NT, D, uses_tensor_cores(in_dtype, D, flags));
     if (ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
 
     ChunkArgs a;
@@ -247,10 +286,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
     a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
     carve(a, static_cast<char*>(workspace), w);
-    cudaError_t e;
-    if ((flags & MDN_CHECK_FINITE) && (e = cudaMemsetAsync(a.status, 0, 64, s)))
-        return mdn::cuda_fail(e);
-    return run_pass(a, in_dtype, flags, s, (size_t)B * T * H * D, (size_t)B * H);
+    return run_pass(a, w, in_dtype, flags, s, (size_t)B * T * H * D, (size_t)B * H);
 }
 
 // ---------------------------------------------------------------- backward
@@ -403,14 +439,15 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
 namespace {
 
 struct VarlenLayout {
-    size_t cu_s, cu_c, q, k, v, al, ml, be, et, chunk, total;
-    int NT;  // padded chunks (an upper bound on the sequences' chunk count)
+    size_t cu_s, cu_c, q, k, v, al, ml, be, et, total;
+    WsLayout chunk;  // the chunk pass's scratch, at the start of the workspace
+    int NT;          // padded chunks (an upper bound on the sequences' chunk count)
 };
 
 // NT = floor(total_T / C) + N bounds sum_s ceil(len_s / C) for any split of
 // total_T tokens into N sequences.
 mdn_status varlen_layout(int N, int total_T, int H, int dk, int dv, int C, mdn_dtype dt,
-                         VarlenLayout& v)
+                         int flags, VarlenLayout& v)
 {
     if (N < 0 || total_T < 0 || C <= 0) return MDN_ERR_INVALID_ARG;
     const long long NT = (long long)total_T / (C > 0 ? C : 1) + N;
@@ -421,7 +458,8 @@ mdn_status varlen_layout(int N, int total_T, int H, int dk, int dv, int C, mdn_d
     const size_t rows = (size_t)NT * C * H;  // padded token-heads
     const size_t elt = dt == MDN_F32 ? 4 : 2;
     v.NT = (int)NT;
-    size_t off = 0;
+    v.chunk = ws_layout(H, v.NT, dk, uses_tensor_cores(dt, dk, flags));
+    size_t off = v.chunk.total;
     v.cu_s = off; off += align_up((size_t)(N + 1) * sizeof(int));
     v.cu_c = off; off += align_up((size_t)(N + 1) * sizeof(int));
     v.q = off;    off += align_up(rows * dk * elt);
@@ -431,19 +469,24 @@ mdn_status varlen_layout(int N, int total_T, int H, int dk, int dv, int C, mdn_d
     v.ml = off;   off += align_up(rows * sizeof(float));
     v.be = off;   off += align_up(rows * sizeof(float));
     v.et = off;   off += align_up(rows * sizeof(float));
-    v.chunk = off;
-    v.total = off + ws_layout(H, v.NT, dk).total;
+    v.total = off;
     return MDN_OK;
 }
 
 }  // namespace
 
+size_t mdn_chunk_fwd_varlen_workspace_size_flags(int N, int total_T, int H, int dk, int dv,
+                                                 int C, mdn_dtype in_dtype, int flags)
+{
+    VarlenLayout v;
+    if (varlen_layout(N, total_T, H, dk, dv, C, in_dtype, flags, v) != MDN_OK) return 0;
+    return v.total;
+}
+
 size_t mdn_chunk_fwd_varlen_workspace_size(int N, int total_T, int H, int dk, int dv, int C,
                                            mdn_dtype in_dtype)
 {
-    VarlenLayout v;
-    if (varlen_layout(N, total_T, H, dk, dv, C, in_dtype, v) != MDN_OK) return 0;
-    return v.total;
+    return mdn_chunk_fwd_varlen_workspace_size_flags(N, total_T, H, dk, dv, C, in_dtype, 0);
 }
 
 mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
@@ -454,7 +497,7 @@ mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn
                                 void* workspace, size_t ws_bytes, int flags, mdn_stream_t stream)
 {
     VarlenLayout L;
-    mdn_status st = varlen_layout(N, total_T, H, dk, dv, C, in_dtype, L);
+    mdn_status st = varlen_layout(N, total_T, H, dk, dv, C, in_dtype, flags, L);
     if (st != MDN_OK) return st;
     if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64))
         return MDN_ERR_INVALID_ARG;
@@ -489,10 +532,10 @@ mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn
     a.B = 1; a.T = L.NT * C; a.H = H; a.D = D; a.NT = L.NT;
     a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
     a.cu_seqlens = cu_s; a.cu_chunks = cu_c; a.nseq = N;
-    carve(a, ws + L.chunk, ws_layout(H, L.NT, D));
+    carve(a, ws, L.chunk);
 
     cudaError_t e;
-    if ((e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
+    if ((e = cudaMemsetAsync(a.status, 0, L.chunk.head, s))) return mdn::cuda_fail(e);
     if ((e = launch_varlen_setup(cu_seqlens, N, total_T, cu_s, cu_c, a.status + 2, s)))
         return mdn::cuda_fail(e);
     const size_t elt = in_dtype == MDN_F32 ? 4 : 2;
@@ -502,7 +545,8 @@ mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn
                                   const_cast<float*>(a.mu_log), const_cast<float*>(a.beta),
                                   const_cast<float*>(a.eta), s)))
         return mdn::cuda_fail(e);
-    return run_pass(a, in_dtype, flags, s, (size_t)total_T * H * D, (size_t)N * H);
+    return run_pass(a, L.chunk, in_dtype, flags, s, (size_t)total_T * H * D, (size_t)N * H,
+                    /*zero_head=*/false);
 }
 
 namespace {

@@ -47,7 +47,15 @@ extern "C" mdn_status mdn_chunk_fwd_noalloc(
     const float* M0, int B, int T, int H, int dk, int dv, int C, void* o, void* vtilde,
     float* S_T, float* M_T, int flags, mdn_stream_t stream)
 {
-    const size_t need = mdn_chunk_fwd_workspace_size(B, T, H, dk, dv, C, in_dtype);
+    const size_t need =
+        mdn_chunk_fwd_workspace_size_flags(B, T, H, dk, dv, C, in_dtype, flags);
+    if (need == 0 || B == 0 || H == 0 || T == 0) {
+        // Invalid or unsupported sizes (mdn_chunk_fwd's own validation reports
+        // them before anything touches a device), or nothing that needs
+        // scratch (no heads; T = 0 only copies the states): no array needed.
+        return mdn_chunk_fwd(q, k, v, in_dtype, alpha_log, mu_log, beta, eta, d_corr, S0, M0,
+                             B, T, H, dk, dv, C, o, vtilde, S_T, M_T, nullptr, 0, flags, stream);
+    }
     if (need > kStaticScratchBytes) return MDN_ERR_UNSUPPORTED;
     void* ws = nullptr;
     const cudaError_t e = scratch_on_current_device(&ws);

@@ -73,3 +73,22 @@ def compare_heads(got, inp: mi.Inputs, heads, tol: float, T0: int = 0, T1=None,
     bad = [f"{n}: rel-L2 {e:.3e}" for n, e in zip(names, errs) if not e <= tol]
     assert not bad, f"{bad} > {tol:.1e}; all: {dict(zip(names, errs))}"
     return errs
+
+
+@functools.lru_cache(maxsize=3)
+def oracle_all(i: int):
+    """The oracle over the whole batch of the i-th workload (parallel over heads),
+    computed once per test session."""
+    inp = config_inputs(i)
+    return oracle.chunk_fwd(inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log, inp.beta, inp.eta,
+                            inp.d_corr, inp.S0, inp.M0)
+
+
+def compare_all(got, ref, tol: float):
+    """got = (o, vt, S_T, M_T) device tensors, ref = the oracle's four arrays for
+    the same batch: every head, every token.  Returns the four rel-L2 errors."""
+    names = ("o", "vtilde", "S_T", "M_T")
+    errs = [rel_l2(to_np(g), r) for g, r in zip(got, ref)]
+    bad = [f"{n}: rel-L2 {e:.3e}" for n, e in zip(names, errs) if not e <= tol]
+    assert not bad, f"{bad} > {tol:.1e}; all: {dict(zip(names, errs))}"
+    return errs

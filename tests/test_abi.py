@@ -65,7 +65,75 @@ def test_workspace_size_rules(lib):
     assert ws(1, 129, 1, 64, 64, 64, 0) > ws(1, 128, 1, 64, 64, 64, 0)
 
 
+def test_workspace_sized_by_path(lib):
+    """The scratch holds only the regions of the path that runs: the tensor-core
+    path (bf16, d = 128) its bf16 chunk operands and coefficient records, the
+    CUDA-core path its fp32 coefficients, Gamma and U/Y/Z/O_inter."""
+    wsf = lib.mdn_chunk_fwd_workspace_size_flags
+    E = _lib
+    MiB = 1 << 20
+    for (B, T, H) in ((4, 2048, 8), (8, 4096, 16), (1, 16384, 16), (2, 200, 3)):
+        chunks = B * H * ((T + 63) // 64)
+        rows = chunks * 64
+        up = lambda x: (x + 255) // 256 * 256
+        tc = up(64 + (chunks + 1) * 4) + up(rows * 128 * 2) + up(rows * 128 * 2) \
+            + up(rows * 256 * 2) + up(rows * 16)
+        assert wsf(B, T, H, 128, 128, 64, E.MDN_BF16, 0) == tc
+        assert lib.mdn_chunk_fwd_workspace_size(B, T, H, 128, 128, 64, E.MDN_BF16) == tc
+        simt = up(64 + (chunks + 1) * 4) + 4 * up(rows * 4) + up(rows * 64 * 4) \
+            + 4 * up(rows * 128 * 4)
+        assert wsf(B, T, H, 128, 128, 64, E.MDN_BF16, E.MDN_FORCE_SIMT) == simt
+        assert wsf(B, T, H, 128, 128, 64, E.MDN_F32, 0) == simt      # fp32 runs on CUDA cores
+    assert wsf(4, 2048, 8, 128, 128, 64, E.MDN_BF16, 0) <= 70 * MiB
+    assert wsf(8, 4096, 16, 128, 128, 64, E.MDN_BF16, 0) <= 0.6 * 1024 * MiB
+    # d = 64 has no tensor-core path: the flag changes nothing
+    assert wsf(1, 256, 2, 64, 64, 64, E.MDN_BF16, 0) == \
+        wsf(1, 256, 2, 64, 64, 64, E.MDN_BF16, E.MDN_FORCE_SIMT)
+    vws = lib.mdn_chunk_fwd_varlen_workspace_size_flags
+    assert vws(3, 1000, 4, 128, 128, 64, E.MDN_BF16, 0) < \
+        vws(3, 1000, 4, 128, 128, 64, E.MDN_BF16, E.MDN_FORCE_SIMT)
+    assert lib.mdn_chunk_fwd_varlen_workspace_size(3, 1000, 4, 128, 128, 64, E.MDN_BF16) == \
+        vws(3, 1000, 4, 128, 128, 64, E.MDN_BF16, 0)
+
+
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_too_small_workspace_for_the_requested_path(lib):
+    """A workspace sized for the default (tensor-core) path is rejected before any
+    device work when MDN_FORCE_SIMT asks for the CUDA-core path."""
+    E = _lib
+    need_tc = lib.mdn_chunk_fwd_workspace_size_flags(1, 128, 1, 128, 128, 64, E.MDN_BF16, 0)
+    need_simt = lib.mdn_chunk_fwd_workspace_size_flags(1, 128, 1, 128, 128, 64, E.MDN_BF16,
+                                                       E.MDN_FORCE_SIMT)
+    assert need_simt > need_tc
+    assert _chunk(lib, dk=128, dv=128, wsb=need_tc, flags=E.MDN_FORCE_SIMT) == \
+        E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, dk=128, dv=128, wsb=need_tc - 1) == E.MDN_ERR_INVALID_ARG
+
+
+def test_status_query_validation(lib):
+    assert lib.mdn_chunk_fwd_status(None, None) == _lib.MDN_ERR_INVALID_ARG
+    assert lib.mdn_chunk_fwd_status(FAKE + 16, None) == _lib.MDN_ERR_INVALID_ARG
+
+
+def test_noalloc_validates_before_any_device_work(lib):
+    """Invalid or unsupported sizes get mdn_chunk_fwd's own errors without the
+    library touching a device (this machine may have none: a device call would
+    come back as MDN_ERR_CUDA); sizes beyond the fixed scratch are refused."""
+    E = _lib
+
+    def na(B=1, T=128, H=1, d=128, C=64, dt=E.MDN_BF16, flags=0, q=FAKE):
+        return lib.mdn_chunk_fwd_noalloc(q, FAKE, FAKE, dt, FAKE, FAKE, FAKE, FAKE, 0.5, None,
+                                         None, B, T, H, d, d, C, FAKE, FAKE, FAKE, FAKE, flags,
+                                         None)
+    assert na(d=96) == E.MDN_ERR_UNSUPPORTED
+    assert na(C=32) == E.MDN_ERR_UNSUPPORTED
+    assert na(dt=7) == E.MDN_ERR_UNSUPPORTED
+    assert na(B=-1) == E.MDN_ERR_INVALID_ARG
+    assert na(T=-5) == E.MDN_ERR_INVALID_ARG
+    assert na(B=0) == E.MDN_OK
+    assert na(B=8, T=4096, H=16) == E.MDN_ERR_UNSUPPORTED              # beyond 64 MiB
 
 
 def _chunk(lib, **kw):

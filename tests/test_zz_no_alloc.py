@@ -66,3 +66,25 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
                                    0.5, None, None, B, T, H, d, d, 64, fake, fake, fake, fake,
                                    0, None)
     assert st == _lib.MDN_ERR_UNSUPPORTED
+
+
+def test_noalloc_invalid_sizes_then_a_valid_call(lib):
+    """Unsupported d or C and a negative size get mdn_chunk_fwd's own errors
+    through the no-allocation entry point; a valid call right after is still
+    correct."""
+    fake = 0x10000
+    bad = lambda d, C, B=1: lib.mdn_chunk_fwd_noalloc(
+        fake, fake, fake, _lib.MDN_BF16, fake, fake, fake, fake, 0.5, None, None, B, 128, 2,
+        d, d, C, fake, fake, fake, fake, 0, None)
+    assert bad(96, 64) == _lib.MDN_ERR_UNSUPPORTED
+    assert bad(128, 32) == _lib.MDN_ERR_UNSUPPORTED
+    assert bad(128, 64, B=-1) == _lib.MDN_ERR_INVALID_ARG
+    spec = mi.Spec("noalloc_c", B=1, T=130, H=2, d=128, state_std=0.01, seed=503)
+    inp = mi.make_inputs(spec)
+    dev = mi.to_torch(inp, "cuda")
+    got = _noalloc(lib, dev, spec, inp.d_corr)
+    ref = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha_log"], dev["mu_log"],
+                        dev["beta"], dev["eta"], inp.d_corr, dev["S0"], dev["M0"])
+    torch.cuda.synchronize()
+    for g, r in zip(got, ref):
+        assert rel_l2(to_np(g), to_np(r)) <= TOL["bf16"]
