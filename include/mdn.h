@@ -72,10 +72,10 @@ typedef enum {
 #define MDN_FORCE_SIMT   0x2  /* use the fp32 CUDA-core kernels even for bf16 input */
 #define MDN_SLICE32      0x4  /* tensor-core path: the inter-chunk kernel gives each CTA
                                  32 columns of d_v (four CTAs per head) */
-#define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head).  Neither flag:
-                                 32 when B*H*4 CTAs fit on the SMs at once, else 64.
-                                 Both widths compute the same result; the flags
-                                 exist for tuning and testing. */
+#define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head) */
+#define MDN_SLICE128     0x10 /* ... all 128 columns (one CTA per head), the default.
+                                 At most one of the three; every width computes the
+                                 same result; the flags exist for tuning and testing. */
 #define MDN_TEST_NO_INTRA 0x100 /* testing the failure path only: the tensor-core
                                  path does not launch its intra-chunk kernel, so the
                                  inter-chunk kernel's wait for each chunk's operands
@@ -152,7 +152,8 @@ mdn_status mdn_chunk_fwd_status(const void *workspace, mdn_stream_t stream);
  *               flags without MDN_FORCE_SIMT, mdn_chunk_fwd_workspace_size),
  *               256-byte aligned; its contents on entry do not matter.
  *   flags       0 or MDN_CHECK_FINITE | MDN_FORCE_SIMT, plus at most one of
- *               MDN_SLICE32 / MDN_SLICE64 (and MDN_TEST_NO_INTRA in tests).
+ *               MDN_SLICE32 / MDN_SLICE64 / MDN_SLICE128 (and MDN_TEST_NO_INTRA
+ *               in tests).
  *
  * Support: d in {64, 128}, C = 64, any T >= 0 (a short last chunk is handled
  * as if padded with steps that leave S and M unchanged), B, H >= 0 with
@@ -342,6 +343,31 @@ mdn_status mdn_gate_params(const float *x_eta, const float *a, const float *b, c
                            long long n, float s, float mu_log_min, int eta_act,
                            float *alpha_log, float *mu_log, float *beta, float *eta,
                            mdn_stream_t stream);
+
+/*
+ * mdn_chunk_fwd with the gate parameterisation fused into the pass: the four
+ * gates are computed from their raw per-token pre-activations (the stable
+ * gating of summary step 6 and ijyty.com sections 5 and 8, exactly as
+ * mdn_gate_params computes them) inside the kernels that read them, so no
+ * gate array is written or read back.
+ *
+ *   x_eta, a_pre, b_pre, c_pre   [B,T,H] fp32 pre-activations of eta, alpha,
+ *                beta and mu (4-byte aligned).
+ *   s, mu_log_min, eta_act       as mdn_gate_params (s and the clamp finite;
+ *                eta_act MDN_ETA_TANH or MDN_ETA_2SIGMOID).
+ * Every other argument, the workspace size (mdn_chunk_fwd_workspace_size...),
+ * the support and the errors are those of mdn_chunk_fwd (plus
+ * MDN_ERR_INVALID_ARG for a bad eta_act, s or clamp).  The result equals
+ * mdn_gate_params followed by mdn_chunk_fwd up to the rounding of the gates.
+ */
+mdn_status mdn_chunk_fwd_preact(const void *q, const void *k, const void *v, mdn_dtype in_dtype,
+                                const float *x_eta, const float *a_pre, const float *b_pre,
+                                const float *c_pre, float s, float mu_log_min, int eta_act,
+                                float d_corr, const float *S0, const float *M0,
+                                int B, int T, int H, int dk, int dv, int C,
+                                void *o, void *vtilde, float *S_T, float *M_T,
+                                void *workspace, size_t ws_bytes, int flags,
+                                mdn_stream_t stream);
 
 /*
  * The chunk coefficients alone (the gate-preparation stage of mdn_chunk_fwd;

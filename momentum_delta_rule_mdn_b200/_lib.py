@@ -14,6 +14,7 @@ MDN_CHECK_FINITE = 0x1
 MDN_FORCE_SIMT = 0x2
 MDN_SLICE32 = 0x4
 MDN_SLICE64 = 0x8
+MDN_SLICE128 = 0x10
 MDN_TEST_NO_INTRA = 0x100
 MDN_ETA_TANH = 0
 MDN_ETA_2SIGMOID = 1
@@ -44,6 +45,9 @@ SIGNATURES = {
     "mdn_chunk_fwd_varlen_workspace_size_flags": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "mdn_chunk_fwd_varlen": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _i, _i,
                                   _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i,
+                                  _vp]),
+    "mdn_chunk_fwd_preact": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _f, _i, _f, _vp,
+                                  _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i,
                                   _vp]),
     "mdn_chunk_gate_prep": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                  _vp, _vp, _vp, _vp, _vp, _vp]),

@@ -136,6 +136,41 @@ def chunk_fwd(q, k, v, alpha_log, mu_log, beta, eta, d: float = 0.5, S0=None, M0
     return o, vt, S_T, M_T
 
 
+def chunk_fwd_preact(q, k, v, x_eta, a, b, c, s: float = 1.0, mu_log_min: float = -2.0,
+                     eta_act: str = "tanh", d: float = 0.5, S0=None, M0=None, C: int = 64, *,
+                     out=None, workspace: Optional[torch.Tensor] = None, flags: int = 0,
+                     stream: Optional[torch.cuda.Stream] = None):
+    """:func:`chunk_fwd` with the gates computed inside the pass from their
+    pre-activations x_eta, a, b, c ([B,T,H] float32; see :func:`gate_params`).
+    Returns (o, vtilde, S_T, M_T)."""
+    if eta_act not in _ETA_ACT:
+        raise ValueError(f"eta_act must be one of {sorted(_ETA_ACT)}, got {eta_act!r}")
+    B, T, H, D = q.shape
+    code = _dtype_code(q)
+    for name, t in (("k", k), ("v", v)):
+        _need(t, q.dtype, q.shape, name)
+    for name, t in (("x_eta", x_eta), ("a", a), ("b", b), ("c", c)):
+        _need(t, torch.float32, (B, T, H), name)
+    _need(S0, torch.float32, (B, H, D, D), "S0")
+    _need(M0, torch.float32, (B, H, D, D), "M0")
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(q),
+               torch.empty((B, H, D, D), dtype=torch.float32, device=q.device),
+               torch.empty((B, H, D, D), dtype=torch.float32, device=q.device))
+    o, vt, S_T, M_T = out
+    lib = library()
+    ws_bytes = int(lib.mdn_chunk_fwd_workspace_size_flags(B, T, H, D, D, C, code, int(flags)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    status = lib.mdn_chunk_fwd_preact(
+        _ptr(q), _ptr(k), _ptr(v), code, _ptr(x_eta), _ptr(a), _ptr(b), _ptr(c), float(s),
+        float(mu_log_min), _ETA_ACT[eta_act], float(d), _ptr(S0), _ptr(M0), B, T, H, D, D, C,
+        _ptr(o), _ptr(vt), _ptr(S_T), _ptr(M_T), _ptr(workspace), workspace.numel(), int(flags),
+        _stream_handle(stream))
+    _check(status, "mdn_chunk_fwd_preact")
+    return o, vt, S_T, M_T
+
+
 def chunk_bwd(q, k, v, alpha_log, mu_log, beta, eta, d: float, vtilde, d_o, S0=None, M0=None,
               dS_T=None, dM_T=None, C: int = 64, *, workspace: Optional[torch.Tensor] = None,
               flags: int = 0, stream: Optional[torch.cuda.Stream] = None) -> dict:

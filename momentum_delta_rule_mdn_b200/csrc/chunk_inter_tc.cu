@@ -42,14 +42,14 @@
 // and MMAs are drained, and status[1] is set.
 #include <algorithm>
 
-#include "mdn_internal.cuh"
-#include "tc_common.cuh"
+#include "inter_common.cuh"
 
 namespace mdn {
 namespace {
 
 using namespace sm100;
 using namespace tc;
+using namespace inter;
 
 constexpr int kChainWarp0 = 2;   // warps 0, 1: MMA issue, loads
 
@@ -111,69 +111,11 @@ constexpr int B_OD = 19;   // [2] A1 / A3 slot read by the output warps (4 warps
 constexpr int B_FIN = 21;  //     every MMA complete (exit)
 constexpr int kBars = 22;
 
-struct InterArgs {
-    const float* crec;
-    const unsigned* ready;  // [chunks] set by the intra-chunk kernel once a chunk is written
-    const float* S0;
-    const float* M0;
-    float* S_T;
-    float* M_T;
-    __nv_bfloat16* o;
-    __nv_bfloat16* vt;
-    unsigned* status;
-    float* dbg;  // diagnostics: phase clocks of the MMA and load lanes of CTA 0 (null in normal use)
-    int T, H, NT;
-    const int* cu_seqlens;  // variable-length mode (see ChunkArgs); null otherwise
-    const int* cu_chunks;
-};
-
-constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
-
-// Wait for the phase of `bar` with this parity.  Gives up when another role
-// has raised the abort flag, or after ~1 s (then raises it itself).
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitNs || i > (1u << 26)) {
-                *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-}
-// Wait until the intra-chunk kernel has published a chunk (it may still be
-// running: this kernel is launched as its programmatic dependent).  Gives up
-// like wait_bar.
-__device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* abort_flag) {
-    if (ld_acquire_gpu(flag) != 0u) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = 1;; ++i) {
-        __nanosleep(64);
-        if (ld_acquire_gpu(flag) != 0u) return true;
-        if ((i & 15u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitNs || i > (1u << 24)) {
-                *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-}
-
 // N (8 or 16) consecutive columns of this thread's TMEM lane.
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
     if constexpr (N == 16) tmem_ld16(taddr, v);
     else tmem_ld8(taddr, v);
-}
-
-// Warp-uniform form: every lane waits, and the warp agrees on the outcome.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
 }
 
 template <int NS>
@@ -515,22 +457,7 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
         !make_chunk_map(&mtat, a.tat, chunks, 2 * C, C, 2 * C) ||
         !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
-    InterArgs t;
-    t.crec = a.crec;
-    t.ready = a.ready;
-    t.S0 = a.S0;
-    t.M0 = a.M0;
-    t.S_T = a.S_T;
-    t.M_T = a.M_T;
-    t.o = static_cast<__nv_bfloat16*>(a.o);
-    t.vt = static_cast<__nv_bfloat16*>(a.vt);
-    t.status = a.status;
-    t.dbg = a.dbg;
-    t.T = a.T;
-    t.H = a.H;
-    t.NT = a.NT;
-    t.cu_seqlens = a.cu_seqlens;
-    t.cu_chunks = a.cu_chunks;
+    const InterArgs t = inter_args(a);
     cudaError_t e = cudaFuncSetAttribute(chunk_inter_kernel<NS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::SMEM_BYTES);
@@ -577,7 +504,7 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
 {
     Reserve rv;
     if (ctas > sms) return rv;
-    const double r = ns == 32 ? 5.0 : 3.7;
+    const double r = ns == 32 ? 5.0 : ns == 64 ? 3.7 : 6.0;
     const long long U = 2LL * (sms - ctas), per_round = 2LL * sms;
     const int lmax = (int)((chunks + per_round - 1) / per_round);
     double best = 0.0;
@@ -594,11 +521,11 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
     return rv;
 }
 
-// Slice width (ns = 0 chooses): four slices per head when they fit in one
-// wave (their chain is the shortest per chunk; two waves for packed
-// sequences), else two.  Packed sequences reserve SMs (one chunk each) only
-// when the slices fit beside a quarter of the SMs kept for the intra-chunk
-// kernel: their chains' lengths are not known on the host.
+// Chain width (ns = 0 chooses): 128 columns, one CTA per head, whose products
+// are the widest; 32- and 64-column slices (four or two CTAs per head) are
+// kept for tuning and testing.  Packed sequences reserve SMs (one chunk each)
+// only when the chains fit beside a quarter of the SMs kept for the
+// intra-chunk kernel: their chains' lengths are not known on the host.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
@@ -608,11 +535,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     if (e != cudaSuccess) return e;
     const long long heads = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
     const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
-    // Packed sequences of mixed lengths: chains of short sequences end early
-    // and free their SMs, so a second wave of 32-column chains costs little
-    // next to the longest chain, which runs in the first (sequences are laid
-    // out in order, the first ones on the lowest CTAs).
-    if (ns == 0) ns = heads * 4 <= (a.cu_chunks ? 2LL * sms : (long long)sms) ? 32 : 64;
+    if (ns == 0) ns = 128;
     const long long ctas = heads * (D / ns);
     Reserve rv;
     if (a.cu_chunks) {
@@ -622,6 +545,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     }
     if (!a.test_no_intra && (e = launch_chunk_intra_tc(a, s, rv.sms, rv.limit)) != cudaSuccess)
         return e;
+    if (ns == 128) return launch_inter_head(a, s);
     return ns == 64 ? launch_inter<64>(a, s) : launch_inter<32>(a, s);
 }
 

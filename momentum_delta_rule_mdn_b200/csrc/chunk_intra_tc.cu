@@ -70,10 +70,7 @@ constexpr uint32_t TM_G = 0, TM_P = 0, TM_R = 128;  // P reuses G's columns once
 constexpr int B_LD = 0, B_MMA = 2;
 
 struct IntraArgs {
-    const float* alpha_log;  // [B, T, H] gates
-    const float* mu_log;
-    const float* beta;
-    const float* eta;
+    GateSrc gates;           // [B, T, H] gates, or their pre-activations
     float* crec;             // [chunks][256]
     unsigned* ready;         // [chunks] set to 1 once a chunk's operands are in global memory
     unsigned* queue;         // next chunk (in chunk-major order) to hand out; zero on entry
@@ -103,7 +100,8 @@ __device__ __forceinline__ void publish_chunk(unsigned* ready, long long chunk) 
 }
 
 // Gate record of one chunk (one warp): la, lm, b, alpha, beta, eta per
-// position; positions past T are steps that leave the state unchanged.  Not
+// position, from the gates or from their pre-activations (the fused
+// parameterisation); positions past T are steps that leave the state unchanged.  Not
 // inlined: the kernel's loop is kept small for the instruction cache.
 __device__ __noinline__ void gate_record(const IntraArgs& a, int n, int bh, float* rec, int lane) {
     const int b = bh / a.H, h = bh % a.H;
@@ -112,11 +110,7 @@ __device__ __noinline__ void gate_record(const IntraArgs& a, int n, int bh, floa
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         if (t0 + e < a.T) {
-            const size_t gi = ((size_t)b * a.T + t0 + e) * a.H + h;
-            ga[e] = a.alpha_log[gi];
-            gm[e] = a.mu_log[gi];
-            gb[e] = a.beta[gi];
-            ge[e] = a.eta[gi];
+            gates_at(a.gates, ((size_t)b * a.T + t0 + e) * a.H + h, ga[e], gm[e], gb[e], ge[e]);
         }
     }
     float la[2], lm[2], lc[2];
@@ -607,10 +601,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserv
         !make_chunk_map(&ma2t, a.a2t, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
     IntraArgs t;
-    t.alpha_log = a.alpha_log;
-    t.mu_log = a.mu_log;
-    t.beta = a.beta;
-    t.eta = a.eta;
+    t.gates = a.gates();
     t.crec = a.crec;
     t.ready = a.ready;
     t.queue = a.ready + chunks;

@@ -69,7 +69,12 @@ intra_simt_kernel(ChunkArgs a)
     }
     if (tid < C) {
         const int r = tid, t = n * C + r;
-        const float ar = (t < a.T) ? expf(a.alpha_log[((size_t)b * a.T + t) * a.H + h]) : 1.f;
+        float ar = 1.f;
+        if (t < a.T) {
+            float al, ml, be, et;
+            gates_at(a.gates(), ((size_t)b * a.T + t) * a.H + h, al, ml, be, et);
+            ar = expf(al);
+        }
         const float abar_prev = (r > 0) ? expf(a.la[crow + r - 1]) : 1.f;
         const float b_prev = (r > 0) ? a.bco[crow + r - 1] : 0.f;
         alpha_s[r] = ar;
@@ -166,7 +171,11 @@ inter_simt_kernel(ChunkArgs a)
             abar_s[r] = expf(a.la[crow + r]);
             b_s[r] = a.bco[crow + r];
             wS[r] = a.gamma[chunk * C * C + (C - 1) * C + r];
-            const float et = (t < a.T) ? a.eta[((size_t)b * a.T + t) * a.H + h] : 0.f;
+            float et = 0.f;
+            if (t < a.T) {
+                float al, ml, be;
+                gates_at(a.gates(), ((size_t)b * a.T + t) * a.H + h, al, ml, be, et);
+            }
             wM[r] = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
             if (r == 0) {
                 scal[0] = expf(a.la[crow + C - 1]);

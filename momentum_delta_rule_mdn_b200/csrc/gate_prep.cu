@@ -6,6 +6,9 @@
 // logcumsumexp.  One warp owns one chunk of 64 positions (two per lane); the
 // prefix sums and the log-sum-exp prefix are warp-shuffle scans.
 //
+// The gates are read as given, or computed from their pre-activations as
+// they are read (the fused parameterisation, see GateSrc).
+//
 // Positions past the end of the sequence act as steps that leave S and M
 // unchanged (alpha = mu = 1, beta = eta = 0), so a short last chunk needs no
 // special case downstream.
@@ -24,9 +27,7 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 
 __global__ void __launch_bounds__(128)
-gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ mu_log,
-                 const float* __restrict__ beta, const float* __restrict__ eta,
-                 int B, int T, int H, int NT, float* __restrict__ la, float* __restrict__ lm,
+gate_prep_kernel(const GateSrc src, int B, int T, int H, int NT, float* __restrict__ la, float* __restrict__ lm,
                  float* __restrict__ lc, float* __restrict__ bco, float* __restrict__ gamma)
 {
     const int lane = threadIdx.x & 31;
@@ -43,11 +44,7 @@ gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
     for (int e = 0; e < 2; ++e) {
         const int t = t0 + e;
         if (t < T) {
-            const size_t g = ((size_t)b * T + t) * H + h;
-            a[e] = alpha_log[g];
-            m[e] = mu_log[g];
-            be[e] = beta[g];
-            et[e] = eta[g];
+            gates_at(src, ((size_t)b * T + t) * H + h, a[e], m[e], be[e], et[e]);
         }
     }
     float la_v[2], lm_v[2], lc_v[2];
@@ -89,8 +86,7 @@ gate_prep_kernel(const float* __restrict__ alpha_log, const float* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
-                             const float* eta, int B, int T, int H, float* la, float* lm,
+cudaError_t launch_gate_prep(const GateSrc& g, int B, int T, int H, float* la, float* lm,
                              float* lc, float* bco, float* gamma, cudaStream_t s)
 {
     const int NT = (T + kChunk - 1) / kChunk;
@@ -100,7 +96,7 @@ cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const 
     const long long blocks = (chunks + warps_per_block - 1) / warps_per_block;
     ProfScope ps(kGatePrep, s);
     gate_prep_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, s>>>(
-        alpha_log, mu_log, beta, eta, B, T, H, NT, la, lm, lc, bco, gamma);
+        g, B, T, H, NT, la, lm, lc, bco, gamma);
     return cudaGetLastError();
 }
 

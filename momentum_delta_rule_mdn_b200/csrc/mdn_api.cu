@@ -16,6 +16,13 @@ constexpr int kAbiVersion = 1;
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+constexpr int kSliceFlags = MDN_SLICE32 | MDN_SLICE64 | MDN_SLICE128;
+// At most one chain-width flag.
+bool one_slice_flag(int flags)
+{
+    const int f = flags & kSliceFlags;
+    return (f & (f - 1)) == 0;
+}
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool aligned_elem(const void* p, mdn_dtype dt) {
@@ -116,12 +123,12 @@ mdn_status run_pass(ChunkArgs& a, const WsLayout& w, mdn_dtype in_dtype, int fla
     const int D = a.D;
     if (zero_head && (e = cudaMemsetAsync(a.status, 0, w.head, s))) return mdn::cuda_fail(e);
     if (uses_tensor_cores(in_dtype, D, flags)) {
-        const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64 : 0;
+        const int ns = (flags & MDN_SLICE32) ? 32 : (flags & MDN_SLICE64) ? 64
+                     : (flags & MDN_SLICE128) ? 128 : 0;
         a.test_no_intra = (flags & MDN_TEST_NO_INTRA) != 0;
         if ((e = launch_chunk_tc(a, s, ns))) return mdn::cuda_fail(e);
     } else {
-        if ((e = launch_gate_prep(a.alpha_log, a.mu_log, a.beta, a.eta, a.B, a.T, a.H, a.la, a.lm,
-                                  a.lc, a.bco, a.gamma, s)))
+        if ((e = launch_gate_prep(a.gates(), a.B, a.T, a.H, a.la, a.lm, a.lc, a.bco, a.gamma, s)))
             return mdn::cuda_fail(e);
         if ((e = launch_chunk_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
     }
@@ -240,18 +247,19 @@ mdn_status mdn_chunk_fwd_status(const void* workspace, mdn_stream_t stream)
     return MDN_OK;
 }
 
-mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
-                         const float* alpha_log, const float* mu_log, const float* beta,
-                         const float* eta, float d_corr, const float* S0, const float* M0,
-                         int B, int T, int H, int dk, int dv, int C, void* o, void* vtilde,
-                         float* S_T, float* M_T, void* workspace, size_t ws_bytes, int flags,
-                         mdn_stream_t stream)
+namespace {
+// mdn_chunk_fwd with the gates from `g` (the gate arrays, or pre-activations).
+mdn_status chunk_fwd_impl(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                          const GateSrc& g, float d_corr, const float* S0, const float* M0,
+                          int B, int T, int H, int dk, int dv, int C, void* o, void* vtilde,
+                          float* S_T, float* M_T, void* workspace, size_t ws_bytes, int flags,
+                          mdn_stream_t stream)
 {
     mdn_status st = check_sizes(B, T, H, dk, dv, C, in_dtype);
     if (st != MDN_OK) return st;
-    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64 | MDN_TEST_NO_INTRA))
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | kSliceFlags | MDN_TEST_NO_INTRA))
         return MDN_ERR_INVALID_ARG;
-    if ((flags & MDN_SLICE32) && (flags & MDN_SLICE64)) return MDN_ERR_INVALID_ARG;
+    if (!one_slice_flag(flags)) return MDN_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return MDN_OK;
     if (!S_T || !M_T || !aligned16(S_T) || !aligned16(M_T)) return MDN_ERR_INVALID_ARG;
     if ((S0 && !aligned16(S0)) || (M0 && !aligned16(M0))) return MDN_ERR_INVALID_ARG;
@@ -271,8 +279,7 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
     const void* tok[] = {q, k, v, o, vtilde};
     for (const void* p : tok)
         if (!p || !aligned16(p)) return MDN_ERR_INVALID_ARG;
-    const void* gates[] = {alpha_log, mu_log, beta, eta};
-    for (const void* p : gates)
+    for (const void* p : g.g)
         if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
     if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign) return MDN_ERR_INVALID_ARG;
     const int NT = (T + C - 1) / C;
@@ -281,12 +288,42 @@ mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype 
 
     ChunkArgs a;
     a.q = q; a.k = k; a.v = v;
-    a.alpha_log = alpha_log; a.mu_log = mu_log; a.beta = beta; a.eta = eta;
+    a.alpha_log = g.g[0]; a.mu_log = g.g[1]; a.beta = g.g[2]; a.eta = g.g[3];
+    a.gate_pre = g.pre; a.gate_s = g.s; a.gate_mu_min = g.mu_min;
     a.dcorr = d_corr; a.S0 = S0; a.M0 = M0;
     a.B = B; a.T = T; a.H = H; a.D = D; a.NT = NT;
     a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
     carve(a, static_cast<char*>(workspace), w);
     return run_pass(a, w, in_dtype, flags, s, (size_t)B * T * H * D, (size_t)B * H);
+}
+}  // namespace
+
+mdn_status mdn_chunk_fwd(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                         const float* alpha_log, const float* mu_log, const float* beta,
+                         const float* eta, float d_corr, const float* S0, const float* M0,
+                         int B, int T, int H, int dk, int dv, int C, void* o, void* vtilde,
+                         float* S_T, float* M_T, void* workspace, size_t ws_bytes, int flags,
+                         mdn_stream_t stream)
+{
+    return chunk_fwd_impl(q, k, v, in_dtype, GateSrc{{alpha_log, mu_log, beta, eta}, 0, 1.f, 0.f},
+                          d_corr, S0, M0, B, T, H, dk, dv, C, o, vtilde, S_T, M_T, workspace,
+                          ws_bytes, flags, stream);
+}
+
+mdn_status mdn_chunk_fwd_preact(const void* q, const void* k, const void* v, mdn_dtype in_dtype,
+                                const float* x_eta, const float* a_pre, const float* b_pre,
+                                const float* c_pre, float s, float mu_log_min, int eta_act,
+                                float d_corr, const float* S0, const float* M0, int B, int T,
+                                int H, int dk, int dv, int C, void* o, void* vtilde, float* S_T,
+                                float* M_T, void* workspace, size_t ws_bytes, int flags,
+                                mdn_stream_t stream)
+{
+    if (eta_act != MDN_ETA_TANH && eta_act != MDN_ETA_2SIGMOID) return MDN_ERR_INVALID_ARG;
+    if (!std::isfinite(s) || !std::isfinite(mu_log_min)) return MDN_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, in_dtype,
+                          GateSrc{{x_eta, a_pre, b_pre, c_pre}, 1 + eta_act, s, mu_log_min},
+                          d_corr, S0, M0, B, T, H, dk, dv, C, o, vtilde, S_T, M_T, workspace,
+                          ws_bytes, flags, stream);
 }
 
 // ---------------------------------------------------------------- backward
@@ -411,7 +448,8 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.dS0 = dS0; a.dM0 = dM0;
     const bool check = flags & MDN_CHECK_FINITE;
     if (check && (e = cudaMemsetAsync(a.status, 0, 64, s))) return mdn::cuda_fail(e);
-    if ((e = launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, a.la, a.lm, a.lc, a.bco,
+    if ((e = launch_gate_prep(GateSrc{{alpha_log, mu_log, beta, eta}, 0, 1.f, 0.f}, B, T, H,
+                              a.la, a.lm, a.lc, a.bco,
                               a.gamma, s)))
         return mdn::cuda_fail(e);
     if ((e = launch_chunk_bwd_simt(a, in_dtype, s))) return mdn::cuda_fail(e);
@@ -499,9 +537,8 @@ mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn
     VarlenLayout L;
     mdn_status st = varlen_layout(N, total_T, H, dk, dv, C, in_dtype, flags, L);
     if (st != MDN_OK) return st;
-    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | MDN_SLICE32 | MDN_SLICE64))
-        return MDN_ERR_INVALID_ARG;
-    if ((flags & MDN_SLICE32) && (flags & MDN_SLICE64)) return MDN_ERR_INVALID_ARG;
+    if (flags & ~(MDN_CHECK_FINITE | MDN_FORCE_SIMT | kSliceFlags)) return MDN_ERR_INVALID_ARG;
+    if (!one_slice_flag(flags)) return MDN_ERR_INVALID_ARG;
     if (N == 0 || H == 0) return MDN_OK;
     if (!cu_seqlens || !aligned4(cu_seqlens)) return MDN_ERR_INVALID_ARG;
     if (!S_T || !M_T || !aligned16(S_T) || !aligned16(M_T)) return MDN_ERR_INVALID_ARG;
@@ -628,7 +665,8 @@ mdn_status mdn_chunk_gate_prep(const float* alpha_log, const float* mu_log, cons
         if (!p || (reinterpret_cast<uintptr_t>(p) & 7u)) return MDN_ERR_INVALID_ARG;
     if (gamma && !aligned4(gamma)) return MDN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return cuda_status(launch_gate_prep(alpha_log, mu_log, beta, eta, B, T, H, la, lm, lc, b,
+    return cuda_status(launch_gate_prep(GateSrc{{alpha_log, mu_log, beta, eta}, 0, 1.f, 0.f},
+                                        B, T, H, la, lm, lc, b,
                                         gamma, s));
 }
 

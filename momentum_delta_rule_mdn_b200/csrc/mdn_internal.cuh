@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "gate_math.cuh"
 #include "mdn.h"
 
 namespace mdn {
@@ -68,6 +69,30 @@ __device__ __forceinline__ void chunk_log_coeffs(const float (&a)[2], const floa
     lc[1] = log_add_exp(lc[0], x[1]);
 }
 
+// The gates a chunk pass reads: the four gate arrays [B, T, H]
+// (alpha_log, mu_log, beta, eta), or, with pre != 0, four pre-activation
+// arrays of the same layout (x_eta, a, b, c) from which every kernel that
+// needs a gate computes it as it reads it (the stable parameterisation of
+// gate_math.cuh; pre = 1 + the eta activation, s and mu_min its constants).
+struct GateSrc {
+    const float* g[4];
+    int pre;
+    float s, mu_min;
+};
+__device__ __forceinline__ void gates_at(const GateSrc& G, size_t i, float& al, float& ml,
+                                         float& be, float& et)
+{
+    if (G.pre == 0) {
+        al = G.g[0][i];
+        ml = G.g[1][i];
+        be = G.g[2][i];
+        et = G.g[3][i];
+    } else {
+        gate::gate_one_rt(G.pre - 1, G.g[0][i], G.g[1][i], G.g[2][i], G.g[3][i], G.s, G.mu_min,
+                          al, ml, be, et);
+    }
+}
+
 // Everything one mdn_chunk_fwd call needs, with the workspace already carved.
 struct ChunkArgs {
     const void* q;
@@ -114,6 +139,13 @@ struct ChunkArgs {
     const int* cu_seqlens = nullptr;
     const int* cu_chunks = nullptr;
     int nseq = 0;
+    // Fused gate parameterisation: with gate_pre != 0, alpha_log, mu_log,
+    // beta and eta above hold the pre-activations x_eta, a, b, c (see GateSrc).
+    int gate_pre = 0;
+    float gate_s = 1.f, gate_mu_min = -2.f;
+    __host__ __device__ GateSrc gates() const {
+        return GateSrc{{alpha_log, mu_log, beta, eta}, gate_pre, gate_s, gate_mu_min};
+    }
 };
 
 // Everything one mdn_chunk_bwd call needs, with the workspace carved.
@@ -277,8 +309,7 @@ struct ProfScope {
 };
 
 // Launchers (each returns the launch's cudaGetLastError()).
-cudaError_t launch_gate_prep(const float* alpha_log, const float* mu_log, const float* beta,
-                             const float* eta, int B, int T, int H, float* la, float* lm,
+cudaError_t launch_gate_prep(const GateSrc& g, int B, int T, int H, float* la, float* lm,
                              float* lc, float* bco, float* gamma, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, mdn_dtype dt, cudaStream_t s);
 // The backward pass (fp32, CUDA cores); K-1's outputs must already be in a's scratch.
@@ -299,6 +330,7 @@ cudaError_t launch_bwd_prep_tc(const BwdArgs& a, cudaStream_t s);
 mdn_status cuda_fail(cudaError_t e);
 // ns: columns of d_v per inter-chunk CTA (32 or 64), 0 = choose by batch size
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns);
+cudaError_t launch_inter_head(const ChunkArgs& a, cudaStream_t s);
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserve, int limit);
 // ds_norm (nullable, [B*H]): receives ||S_t - S_{t-1}||_F of each head.
 cudaError_t launch_step(const void* q, const void* k, const void* v, mdn_dtype dt,

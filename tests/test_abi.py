@@ -156,6 +156,8 @@ def test_chunk_fwd_validation(lib):
     assert _chunk(lib, C=0) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, flags=0x100) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, flags=_lib.MDN_SLICE32 | _lib.MDN_SLICE64) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, flags=_lib.MDN_SLICE64 | _lib.MDN_SLICE128) == E.MDN_ERR_INVALID_ARG
+    assert _chunk(lib, flags=_lib.MDN_SLICE32 | _lib.MDN_SLICE128) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, q=None) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, vt=None) == E.MDN_ERR_INVALID_ARG
     assert _chunk(lib, ST=None) == E.MDN_ERR_INVALID_ARG
@@ -260,3 +262,22 @@ def test_bwd_workspace_and_validation(lib):
     assert bw(gate=FAKE + 2) == E.MDN_ERR_INVALID_ARG
     assert bw(wsb=need - 1) == E.MDN_ERR_INVALID_ARG
     assert bw(T=-1) == E.MDN_ERR_INVALID_ARG
+
+
+def test_preact_validation(lib):
+    """The fused-gate pass validates its gate constants and pointers before any
+    device work."""
+    E = _lib
+    inf = float("inf")
+
+    def pa(act=E.MDN_ETA_TANH, s=1.0, mn=-2.0, x=FAKE, d=64, B=1):
+        return lib.mdn_chunk_fwd_preact(FAKE, FAKE, FAKE, E.MDN_BF16, x, FAKE, FAKE, FAKE, s, mn,
+                                        act, 0.5, None, None, B, 128, 1, d, d, 64, FAKE, FAKE,
+                                        FAKE, FAKE, FAKE, 0, 0, None)
+    assert pa(act=2) == E.MDN_ERR_INVALID_ARG
+    assert pa(s=inf) == E.MDN_ERR_INVALID_ARG
+    assert pa(mn=float("nan")) == E.MDN_ERR_INVALID_ARG
+    assert pa(x=None) == E.MDN_ERR_INVALID_ARG
+    assert pa(x=FAKE + 2) == E.MDN_ERR_INVALID_ARG
+    assert pa(d=96) == E.MDN_ERR_UNSUPPORTED
+    assert pa(B=0) == E.MDN_OK

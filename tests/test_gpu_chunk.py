@@ -55,11 +55,12 @@ def test_small_cases(name, B, T, H, d, dtype, std):
     compare_heads(run(inp), inp, all_heads(inp.spec), TOL[dtype])
 
 
-@pytest.mark.parametrize("flags", [_lib.MDN_SLICE32, _lib.MDN_SLICE64])
+@pytest.mark.parametrize("flags", [_lib.MDN_SLICE32, _lib.MDN_SLICE64, _lib.MDN_SLICE128])
 @pytest.mark.parametrize("name,B,T,H", [("ragged", 2, 200, 3), ("T1", 1, 1, 2), ("T65", 1, 65, 1),
-                                         ("long", 1, 1000, 2)])
+                                         ("long", 1, 1000, 2), ("many_heads", 3, 130, 60)])
 def test_inter_slice_widths(name, B, T, H, flags):
-    """Both column-slice widths of the inter-chunk kernel against the oracle."""
+    """Every chain width of the inter-chunk kernel against the oracle (180 heads:
+    more chains than SMs, so the chains run in more than one wave)."""
     inp = mi.make_inputs(mi.Spec("slice_" + name, B=B, T=T, H=H, d=128, dtype="bf16",
                                  state_std=0.01, seed=zlib.crc32(name.encode()) % 1000 + 3000))
     compare_heads(run(inp, flags=flags), inp, all_heads(inp.spec), TOL["bf16"])
