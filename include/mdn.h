@@ -73,9 +73,11 @@ typedef enum {
 #define MDN_SLICE32      0x4  /* tensor-core path: the inter-chunk kernel gives each CTA
                                  32 columns of d_v (four CTAs per head) */
 #define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head) */
-#define MDN_SLICE128     0x10 /* ... all 128 columns (one CTA per head), the default.
-                                 At most one of the three; every width computes the
-                                 same result; the flags exist for tuning and testing. */
+#define MDN_SLICE128     0x10 /* ... all 128 columns (one CTA per head).  None of the
+                                 three: 32 when B*H*4 CTAs fit on the SMs at once,
+                                 else 128 (packed sequences: 32 up to two waves, else
+                                 64).  At most one; every width computes the same
+                                 result; the flags exist for tuning and testing. */
 #define MDN_TEST_NO_INTRA 0x100 /* testing the failure path only: the tensor-core
                                  path does not launch its intra-chunk kernel, so the
                                  inter-chunk kernel's wait for each chunk's operands

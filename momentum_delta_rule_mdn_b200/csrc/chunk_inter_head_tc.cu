@@ -33,9 +33,10 @@
 //   warp 1        one lane issues every TMA load and bulk copy
 //   16 chain warps  warp w reads TMEM lanes 32(w%4).. and 32 columns; the eight on
 //                 lanes 0..63 form Y, the eight on lanes 64..127 form Oi; after
-//                 A2 all sixteen write the state's bf16 copy (the B operand of
-//                 the next A1), then rescale the fp32 state in TMEM
-//   8 output warps  Vtilde and o of chunk n from A3, to global memory
+//                 A2 all sixteen read the state once, write its bf16 copy (the B
+//                 operand of the next A1) and store it back rescaled in TMEM
+//   8 output warps  Vtilde and o of chunk n from A3, read out of TMEM (which
+//                 frees it for the next A1) before they go to global memory
 // Hand-offs are mbarriers only; every wait is bounded (as in the slice
 // kernel: a wait that runs out raises the CTA's abort flag, every role leaves
 // its loop, copies and MMAs in flight are drained, and status[1] is set).
@@ -251,6 +252,9 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int c16 = (grp & 1) * 4;      // their first 16-byte chunk in a 128-byte row
         const uint32_t s_col = TM_S + 32 * grp, m_col = TM_M + 32 * grp;
         bool ok = true;
+        PhaseClock clk;  // diagnostics: a Y warp (quad 0) and an Oi warp (quad 2) of CTA 0
+        clk.start((a.dbg && blockIdx.x == 0 && lid == 0 && grp == 0 && (quad == 0 || quad == 2))
+                      ? a.dbg + (quad == 0 ? 20 : 40) : nullptr);
         // the entering state: its bf16 copy, and the fp32 state rescaled for chunk 0
         if (NT > 0) {
             ok = warp_wait(&bars[B_FCR], 0, abort_flag);
@@ -298,13 +302,16 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int n = 0; n < NT && ok; ++n) {
             const int s2 = n & 1, sc = n & 3;
             const float* cr = reinterpret_cast<const float*>(sm + CR0 + sc * 1024);
+            clk.lap(0);
             if (!warp_wait(&bars[B_FCR + sc], (n >> 2) & 1, abort_flag)) break;
             if (quad < 2) {
                 // ---- Y = V - (D1 KS - D2 KM) for rows 0..63, then clear those columns
                 const int r = lane;
                 const float c_ab = cr[r], c_d2 = cr[C + r];
                 if (!warp_wait(&bars[B_FV], n & 1, abort_flag)) break;
+                clk.lap(1);
                 if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
+                clk.lap(2);
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int p = 0; p < 2; ++p) {
@@ -326,10 +333,12 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                     for (int e = 0; e < 16; ++e) x[e] = 0.f;
                     tmem_st16(tq + col, x);
                 }
+                clk.lap(3);
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
                 __syncwarp();
+                clk.lap(4);
                 if (lid == 0) {
                     mbar_arrive(&bars[B_YR]);
                     mbar_arrive(&bars[B_ECR + sc]);
@@ -338,7 +347,9 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                 // ---- Oi = Diag(alphabar) QhatS - Diag(b) QhatM for rows 64..127, in place
                 const int r = lane - 64;
                 const float c_ab = cr[r], c_b = cr[2 * C + r];
+                clk.lap(1);
                 if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
+                clk.lap(2);
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int p = 0; p < 2; ++p) {
@@ -351,16 +362,20 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                     for (int e = 0; e < 16; ++e) x[e] = fmaf(c_ab, x[e], -c_b * y[e]);
                     tmem_st16(tq + col, x);
                 }
+                clk.lap(3);
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncwarp();
+                clk.lap(4);
                 if (lid == 0) {
                     mbar_arrive(&bars[B_OI]);
                     mbar_arrive(&bars[B_ECR + sc]);
                 }
             }
             // ---- the state after chunk n
+            clk.lap(5);
             if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
+            clk.lap(6);
             tc_fence_after_sync();
             if (n + 1 == NT) {
                 // S_T, M_T (nothing reads the bf16 copy or the rescaled state any more)
@@ -380,6 +395,14 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
                 break;
             }
+            // bf16 copy for the next A1, and the fp32 state rescaled in place for
+            // the next A2 (chunk n + 1's record was loaded with its K, Qhat), from
+            // one read of the state
+            const int sn = (n + 1) & 3;
+            if (!warp_wait(&bars[B_FCR + sn], ((n + 1) >> 2) & 1, abort_flag)) break;
+            const float* crn = reinterpret_cast<const float*>(sm + CR0 + sn * 1024);
+            const float abC = crn[3 * C], bC = crn[3 * C + 1], mbC = crn[3 * C + 2];
+            clk.lap(7);
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
                 float s[16], m[16];
@@ -391,22 +414,6 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                 st_bf16x8(sm + ST + pan * 16384 + sw128_off(lane, cc + 1), s + 8);
                 st_bf16x8(sm + ST + (2 + pan) * 16384 + sw128_off(lane, cc), m);
                 st_bf16x8(sm + ST + (2 + pan) * 16384 + sw128_off(lane, cc + 1), m + 8);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lid == 0) mbar_arrive(&bars[B_SR]);
-            // rescale for chunk n + 1 (its record was loaded with its K, Qhat)
-            const int sn = (n + 1) & 3;
-            if (!warp_wait(&bars[B_FCR + sn], ((n + 1) >> 2) & 1, abort_flag)) break;
-            const float* crn = reinterpret_cast<const float*>(sm + CR0 + sn * 1024);
-            const float abC = crn[3 * C], bC = crn[3 * C + 1], mbC = crn[3 * C + 2];
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                float s[16], m[16];
-                tmem_ld16(tq + s_col + 16 * p, s);
-                tmem_ld16(tq + m_col + 16 * p, m);
-                tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     s[j] = fmaf(abC, s[j], -bC * m[j]);
@@ -415,40 +422,62 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
                 tmem_st16(tq + s_col + 16 * p, s);
                 tmem_st16(tq + m_col + 16 * p, m);
             }
+            clk.lap(8);
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lid == 0) mbar_arrive(&bars[B_SR]);
+            clk.lap(9);
             tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
             if (lid == 0) mbar_arrive(&bars[B_PS]);
+            clk.lap(10);
         }
+        clk.flush();
     } else {
         // ------------------------------------------------------------ outputs
         const int half = (warp - kOutWarp0) >> 2;  // columns 64 half .. 64 half + 63
         const bool orow = quad >= 2;               // lanes 64..127: rows of o; 0..63: of Vtilde
         const int r = lane & 63;
         __nv_bfloat16* const out = orow ? a.o : a.vt;
+        PhaseClock clk;  // diagnostics: one output warp of CTA 0
+        clk.start((a.dbg && blockIdx.x == 0 && lid == 0 && warp == kOutWarp0) ? a.dbg + 60 : nullptr);
         for (int n = 0; n < NT; ++n) {
+            clk.lap(0);
             if (!warp_wait(&bars[B_M3], n & 1, abort_flag)) break;
+            clk.lap(1);
             tc_fence_after_sync();
-            const int t = n * C + r;  // token of the chain
-            uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(ch.out0 + t) * a.H + h) * D +
-                                                  64 * half);
-#pragma unroll 1
+            // read the 64 columns and pack them to bf16 first: the TMEM columns
+            // are released (for the next chunk's A1) before the global stores
+            uint32_t pk[32];
+#pragma unroll
             for (int p = 0; p < 2; ++p) {
                 float x[16], y[16];
                 tmem_ld16(tq + TM_A1 + 64 * half + 32 * p, x);
                 tmem_ld16(tq + TM_A1 + 64 * half + 32 * p + 16, y);
                 tmem_wait_ld();
-                if (t < ch.len) {
-                    dst[4 * p] = bf16x8(x);
-                    dst[4 * p + 1] = bf16x8(x + 8);
-                    dst[4 * p + 2] = bf16x8(y);
-                    dst[4 * p + 3] = bf16x8(y + 8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pk[16 * p + e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+                    pk[16 * p + 8 + e] = pack_bf16(y[2 * e], y[2 * e + 1]);
                 }
             }
+            clk.lap(2);
             tc_fence_before_sync();
             __syncwarp();
             if (lid == 0) mbar_arrive(&bars[B_OD]);
+            const int t = n * C + r;  // token of the chain
+            if (t < ch.len) {
+                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(ch.out0 + t) * a.H + h) * D +
+                                                      64 * half);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4)
+                    dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            }
+            clk.lap(3);
         }
+        clk.flush();
     }
 
     tc_fence_before_sync();

@@ -504,7 +504,7 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
 {
     Reserve rv;
     if (ctas > sms) return rv;
-    const double r = ns == 32 ? 5.0 : ns == 64 ? 3.7 : 6.0;
+    const double r = ns == 32 ? 5.0 : ns == 64 ? 3.7 : 2.0;
     const long long U = 2LL * (sms - ctas), per_round = 2LL * sms;
     const int lmax = (int)((chunks + per_round - 1) / per_round);
     double best = 0.0;
@@ -521,9 +521,14 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
     return rv;
 }
 
-// Chain width (ns = 0 chooses): 128 columns, one CTA per head, whose products
-// are the widest; 32- and 64-column slices (four or two CTAs per head) are
-// kept for tuning and testing.  Packed sequences reserve SMs (one chunk each)
+// Chain width (ns = 0 chooses).  A chain step costs about 3.1k cycles with
+// 32-column slices, 4.8k with 64 and 9k with the whole head: the epilogues of
+// one CTA move data in proportion to its width, and that, not the tensor
+// pipe, bounds the step.  So four 32-column slices per head when they all fit
+// on the SMs at once (the shortest chain); otherwise one CTA per head, which
+// takes the least SM time per chunk (9k against 4 x 3.1k or 2 x 4.8k) and
+// leaves the fewest waves.  Packed sequences keep 32 up to two waves, else 64
+// (their chains end at different times), and reserve SMs (one chunk each)
 // only when the chains fit beside a quarter of the SMs kept for the
 // intra-chunk kernel: their chains' lengths are not known on the host.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
@@ -535,7 +540,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     if (e != cudaSuccess) return e;
     const long long heads = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
     const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
-    if (ns == 0) ns = 128;
+    if (ns == 0) {
+        if (a.cu_chunks) ns = heads * 4 <= 2LL * sms ? 32 : 64;
+        else ns = heads * 4 <= sms ? 32 : 128;
+    }
     const long long ctas = heads * (D / ns);
     Reserve rv;
     if (a.cu_chunks) {
