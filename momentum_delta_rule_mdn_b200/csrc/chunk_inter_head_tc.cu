@@ -467,13 +467,38 @@ chunk_inter_head_kernel(const __grid_constant__ CUtensorMap tm_k,
             tc_fence_before_sync();
             __syncwarp();
             if (lid == 0) mbar_arrive(&bars[B_OD]);
-            const int t = n * C + r;  // token of the chain
-            if (t < ch.len) {
-                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(ch.out0 + t) * a.H + h) * D +
-                                                      64 * half);
+            // Transpose 16-byte chunks within each group of eight lanes (three
+            // butterfly exchanges): lane 8 o + j then holds chunk j of rows
+            // 8 o .. 8 o + 7 of the warp, so that one store instruction writes four
+            // whole 128-byte rows instead of 32 scattered 16-byte pieces.
+            uint4 ch16[8];
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4)
-                    dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int c = 0; c < 8; ++c)
+                ch16[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            const int j8 = lid & 7;
+#pragma unroll
+            for (int m = 4; m >= 1; m >>= 1) {
+                const bool hi = (j8 & m) != 0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (c & m) continue;
+                    const uint4 snd = hi ? ch16[c] : ch16[c | m];
+                    uint4 rcv;
+                    rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, m);
+                    rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, m);
+                    rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, m);
+                    rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, m);
+                    if (hi) ch16[c] = rcv;
+                    else ch16[c | m] = rcv;
+                }
+            }
+            const int rbase = (r & ~31) + (lid & ~7);  // first row of this lane's group of eight
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = n * C + rbase + k;  // token of the chain
+                if (t < ch.len)
+                    reinterpret_cast<uint4*>(out + ((size_t)(ch.out0 + t) * a.H + h) * D +
+                                             64 * half)[j8] = ch16[k];
             }
             clk.lap(3);
         }

@@ -496,6 +496,10 @@ cudaError_t launch_inter(const ChunkArgs& a, cudaStream_t s)
 // intra-chunk chunk costs about r chain steps (two CTAs per SM, ~17k cycles;
 // a 32-column chain step ~3.3k, a 64-column one ~4.6k), so L minimises
 //     L r + max(NT, rest / U r + 1),   rest = chunks - 2 SMs L.
+// For whole-head chains (~9k cycles a step) r = 6 is not that ratio but the
+// value that measured best on the 1.3B-layer workload: both kernels are then
+// bound by SM time, not by the chain, and the plan keeps the intra-chunk
+// kernel on every SM until nearly all chunks are done.
 struct Reserve {
     int sms = 0;    // CTAs on SMs 0 .. sms-1 are limited
     int limit = 1;
@@ -504,7 +508,7 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
 {
     Reserve rv;
     if (ctas > sms) return rv;
-    const double r = ns == 32 ? 5.0 : ns == 64 ? 3.7 : 2.0;
+    const double r = ns == 32 ? 5.0 : ns == 64 ? 3.7 : 6.0;
     const long long U = 2LL * (sms - ctas), per_round = 2LL * sms;
     const int lmax = (int)((chunks + per_round - 1) / per_round);
     double best = 0.0;

@@ -10,8 +10,9 @@
 //   A      = (P K^T) o Gamma-:  A_{r,i} = alpha_r k_r.k_i Gamma_{r-1,i}  (i < r)
 //   Att    = (Qhat K^T) o Gamma:  Att_{r,i} = qhat_r.k_i Gamma_{r,i}  (i <= r)
 //   T      = (I + A)^{-1} in fp32 over 16 x 16 blocks: diagonal blocks by forward
-//            substitution, B_ik = -T_ii A_ik, then T_ij = sum_{k=j}^{i-1} B_ik T_kj
-//            by distance from the diagonal
+//            substitution, B_ik = -T_ii A_ik, then the blocks off the diagonal in
+//            two dependent steps (T_10, T_21, T_32 with C_3k = B_3k + B_32 B_2k, then
+//            T_20, T_31 and T_30 = C_30 T_00 + C_31 T_10)
 //   P      = [I; Att] T = [T; Att T]                    (M=128, N=64,  K=64)
 //   R      = K^T [Diag(Gamma_C) T | -Diag(w) T]          (M=128, N=128, K=64)
 //            with w_r = eta_r mubar_C / mubar_r
@@ -32,8 +33,8 @@
 // phases share each SM's instruction cache.  Column i of Gamma never leaves the registers of
 // the thread that owns it: that thread writes column i of A and K-row i of
 // the MN-major [I; Att] operand directly.  T is solved in place over A: the
-// diagonal blocks replace A_ii, B_ik replaces A_ik, and T_ij (i > j) goes to
-// the unused block (j, i).
+// diagonal blocks replace A_ii, B_ik replaces A_ik (C_30 replaces B_30, C_31
+// goes to a scratch block), and T_ij (i > j) goes to the unused block (j, i).
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -63,6 +64,7 @@ static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 constexpr uint32_t TB_OFF = 8192;    // T bf16 (B of P): the Q half of panel 0 of the current buffer
 constexpr uint32_t DT0_OFF = 24576;  // N-panel 0 of [D_G T | -D_w T] (B of R): the Q half of panel 1
 constexpr uint32_t STG_TAT = AM;     // [T; Att T] staging: over T once the bf16 copies are made
+constexpr uint32_t C31 = DT1;        // C_31 (fp32, row stride LDF) during the T solve
 // TMEM columns
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t TM_G = 0, TM_P = 0, TM_R = 128;  // P reuses G's columns once G is read
@@ -438,23 +440,68 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncthreads();
         clk.lap(5);
 
-        // ---- T_ij = sum_{k=j}^{i-1} B_ik T_kj by distance L = i - j, into block (j, i)
-        for (int L = 1; L < 4; ++L) {
-            if (tid < (4 - L) * 32) {
-                const int i = L + (tid >> 5), j = i - L;
-                const int r0 = 2 * ((tid >> 2) & 7), c0 = 4 * (tid & 3);
+        // ---- T off the diagonal in two dependent steps instead of three levels:
+        //      step 1: T_10 = B_10 T_00, T_21 = B_21 T_11, T_32 = B_32 T_22 into blocks
+        //      (0,1), (1,2), (2,3), and C_30 = B_30 + B_32 B_20 over B_30, C_31 = B_31 +
+        //      B_32 B_21 into a scratch block over DT1 (free until the bf16 copies);
+        //      step 2: T_20 = B_20 T_00 + B_21 T_10, T_31 = B_31 T_11 + B_32 T_21,
+        //      T_30 = C_30 T_00 + C_31 T_10 (= B_30 T_00 + B_31 T_10 + B_32 T_20)
+#pragma unroll 1
+        for (int rep = 0; rep < 2; ++rep) {
+            const int tt = tid + 128 * rep;
+            if (tt < 160) {
+                const int job = tt >> 5;
+                const int r0 = 2 * ((tt >> 2) & 7), c0 = 4 * (tt & 3);
                 float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-                for (int kb = j; kb < i; ++kb) {
-                    // T_kj: the diagonal block for kb == j, else stored at block (j, kb)
-                    tile_2x4(Am + 16 * i * LDF + 16 * kb, Am + 16 * j * LDF + 16 * kb, r0, c0,
+                float* dst;
+                if (job < 3) {  // T_{j+1,j} = B_{j+1,j} T_jj
+                    const int j = job;
+                    tile_2x4(Am + 16 * (j + 1) * LDF + 16 * j, Am + 16 * j * LDF + 16 * j, r0, c0,
                              acc0, acc1);
+                    dst = Am + (16 * j + r0) * LDF + 16 * (j + 1) + c0;
+                } else {        // C_3k = B_3k + B_32 B_2k, k = 0, 1
+                    const int kb = job - 3;
+                    const float* b3k = Am + (48 + r0) * LDF + 16 * kb + c0;
+                    acc0 = lds4(b3k);
+                    acc1 = lds4(b3k + LDF);
+                    tile_2x4(Am + 48 * LDF + 32, Am + 32 * LDF + 16 * kb, r0, c0, acc0, acc1);
+                    dst = kb == 0 ? Am + (48 + r0) * LDF + c0
+                                  : reinterpret_cast<float*>(sm + C31) + r0 * LDF + c0;
                 }
-                float* t = Am + (16 * j + r0) * LDF + 16 * i + c0;
-                *reinterpret_cast<float4*>(t) = acc0;
-                *reinterpret_cast<float4*>(t + LDF) = acc1;
+                *reinterpret_cast<float4*>(dst) = acc0;
+                *reinterpret_cast<float4*>(dst + LDF) = acc1;
             }
-            __syncthreads();
         }
+        __syncthreads();
+        if (tid < 96) {
+            const int job = tid >> 5;
+            const int r0 = 2 * ((tid >> 2) & 7), c0 = 4 * (tid & 3);
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+            const float* x0;
+            const float* y0;
+            const float* x1;
+            const float* y1;
+            float* dst;
+            if (job == 0) {
+                x0 = Am + 32 * LDF;      y0 = Am;                  // B_20, T_00
+                x1 = Am + 32 * LDF + 16; y1 = Am + 16;             // B_21, T_10
+                dst = Am + r0 * LDF + 32 + c0;
+            } else if (job == 1) {
+                x0 = Am + 48 * LDF + 16; y0 = Am + 16 * LDF + 16;  // B_31, T_11
+                x1 = Am + 48 * LDF + 32; y1 = Am + 16 * LDF + 32;  // B_32, T_21
+                dst = Am + (16 + r0) * LDF + 48 + c0;
+            } else {
+                x0 = Am + 48 * LDF;      y0 = Am;                  // C_30, T_00
+                x1 = reinterpret_cast<const float*>(sm + C31);     // C_31
+                y1 = Am + 16;                                      // T_10
+                dst = Am + r0 * LDF + 48 + c0;
+            }
+            tile_2x4(x0, y0, r0, c0, acc0, acc1);
+            tile_2x4(x1, y1, r0, c0, acc0, acc1);
+            *reinterpret_cast<float4*>(dst) = acc0;
+            *reinterpret_cast<float4*>(dst + LDF) = acc1;
+        }
+        __syncthreads();
         clk.lap(6);
 
         // ---- bf16 copies of T: T (B of P) into the Q half of panel 0, and

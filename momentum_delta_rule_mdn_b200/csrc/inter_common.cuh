@@ -65,6 +65,10 @@ __device__ __forceinline__ bool wait_ready(const unsigned* flag, volatile int* a
 }
 
 // Warp-uniform form: every lane waits, and the warp agrees on the outcome.
+// Warp-uniform form: every lane waits, and the warp agrees on the outcome.
+// (Polling from one lane and broadcasting the result was measured slower on
+// the 32-column chains: it adds a shuffle and a second probe to every hand-off
+// on their critical path.)
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
 }
