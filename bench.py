@@ -313,8 +313,8 @@ def run_ours(args, rank, world, device):
             achieved, peak = work / avg_s / 1e9, hbm
         else:
             achieved, peak = work / avg_s / 1e12, FP32_ALU_PEAK_TFLOPS
-        tr = load_traffic().get(name, {})
-        traffic = tr.get("bytes_per_launch") if tr.get("workload") == spec0.name else None
+        tr = load_traffic().get(name, {}).get(spec0.name, {})
+        traffic = tr.get("bytes_per_launch")
         fr = fractions(nbytes, flops, avg_s, hbm, bf16)
         roofline = {"kernel": name, "bound": bound, "achieved": round(achieved, 3),
                     "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),

@@ -15,8 +15,8 @@
 //
 // Gamma_{r,i} = eta_i (alphabar_r / mubar_i)(c_r - c_{i-1}) is accumulated
 // down each column i by its first-order recurrence
-//     Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r exp(lm_r - lm_i),
-// a sum of non-negative terms.  Evaluating the difference c_r - c_{i-1} from
+//     Gamma_{r,i} = alpha_r Gamma_{r-1,i} + eta_i beta_r mubar_r / mubar_i,
+// a sum of non-negative terms (mubar_r / mubar_i as a running product of mu).  Evaluating the difference c_r - c_{i-1} from
 // lc (the pages' log-broadcast) cancels catastrophically in fp32 when
 // mu/alpha < 1 over a run of tokens; the recurrence has no subtraction.
 #include "mdn_internal.cuh"
@@ -59,7 +59,10 @@ gate_prep_kernel(const GateSrc src, int B, int T, int H, int NT, float* __restri
 
     if (gamma == nullptr) return;
     // Column recurrence; this lane owns columns i0 = lane and i1 = lane + 32.
+    // mubar_r / mubar_i is kept as a running product of mu (non-negative
+    // factors; no exponential per element).
     const float ea[2] = {expf(a[0]), expf(a[1])};
+    const float em[2] = {expf(m[0]), expf(m[1])};
     const int i0 = lane, i1 = lane + 32;
     // Position p sits in lane p/2, element p%2: fetch both elements, pick locally.
     auto fetch = [&](const float (&x)[2], int p) {
@@ -67,20 +70,24 @@ gate_prep_kernel(const GateSrc src, int B, int T, int H, int NT, float* __restri
         const float e1 = __shfl_sync(kFull, x[1], p >> 1);
         return (p & 1) ? e1 : e0;
     };
-    const float eta_i0 = fetch(et, i0), lm_i0 = fetch(lm_v, i0);
-    const float eta_i1 = fetch(et, i1), lm_i1 = fetch(lm_v, i1);
-    float g0 = 0.f, g1 = 0.f;
+    const float eta_i0 = fetch(et, i0), eta_i1 = fetch(et, i1);
+    float g0 = 0.f, g1 = 0.f, f0 = 1.f, f1 = 1.f;
     float* G = gamma + (size_t)chunk * kChunk * kChunk;
-    for (int r = 0; r < kChunk; ++r) {
-        const int src = r >> 1;
-        const bool odd = r & 1;
-        const float ar = __shfl_sync(kFull, odd ? ea[1] : ea[0], src);
-        const float br = __shfl_sync(kFull, odd ? be[1] : be[0], src);
-        const float lmr = __shfl_sync(kFull, odd ? lm_v[1] : lm_v[0], src);
-        g0 = (r >= i0) ? fmaf(ar, g0, eta_i0 * br * expf(lmr - lm_i0)) : 0.f;
-        g1 = (r >= i1) ? fmaf(ar, g1, eta_i1 * br * expf(lmr - lm_i1)) : 0.f;
-        G[r * kChunk + i0] = g0;
-        G[r * kChunk + i1] = g1;
+#pragma unroll 2
+    for (int s = 0; s < kChunk / 2; ++s) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int r = 2 * s + e;
+            const float ar = __shfl_sync(kFull, ea[e], s);
+            const float br = __shfl_sync(kFull, be[e], s);
+            const float mr = __shfl_sync(kFull, em[e], s);
+            f0 = (r > i0) ? f0 * mr : 1.f;
+            f1 = (r > i1) ? f1 * mr : 1.f;
+            g0 = (r >= i0) ? fmaf(ar, g0, eta_i0 * br * f0) : 0.f;
+            g1 = (r >= i1) ? fmaf(ar, g1, eta_i1 * br * f1) : 0.f;
+            G[r * kChunk + i0] = g0;
+            G[r * kChunk + i1] = g1;
+        }
     }
 }
 
