@@ -202,15 +202,17 @@ def test_chunk_fwd_cuda_graph_replay():
         compare_heads(out, inps[r], all_heads(inps[r].spec), TOL["bf16"])
 
 
-def test_timeout_path_reports_and_recovers():
+@pytest.mark.parametrize("width", [0, _lib.MDN_SLICE128])
+def test_timeout_path_reports_and_recovers(width):
     """Failure injected on the host: the intra-chunk kernel is not launched, so
     the inter-chunk kernel's bounded wait for the first chunk's operands runs
     out; its CTAs stop cleanly and the call reports MDN_ERR_TIMEOUT.  The
-    context stays usable: the next normal call is correct."""
+    context stays usable: the next normal call is correct.  Both chain kernels
+    (32-column slices, chosen for these two heads, and one CTA per head)."""
     inp = mi.make_inputs(mi.Spec("timeout", B=1, T=130, H=2, d=128, dtype="bf16",
                                  state_std=0.01, seed=4200))
     with pytest.raises(mdn.MDNError) as err:
-        run(inp, flags=_lib.MDN_TEST_NO_INTRA | _lib.MDN_CHECK_FINITE)
+        run(inp, flags=_lib.MDN_TEST_NO_INTRA | _lib.MDN_CHECK_FINITE | width)
     assert err.value.status == _lib.MDN_ERR_TIMEOUT
     compare_heads(run(inp), inp, all_heads(inp.spec), TOL["bf16"])
     # without MDN_CHECK_FINITE the call returns at once; the status query reports
@@ -220,8 +222,8 @@ def test_timeout_path_reports_and_recovers():
     ws = torch.empty(mdn.chunk_fwd_workspace_size(B, T, H, d), dtype=torch.uint8, device="cuda")
     args = (dev["q"], dev["k"], dev["v"], dev["alpha_log"], dev["mu_log"], dev["beta"],
             dev["eta"], inp.d_corr, dev["S0"], dev["M0"])
-    mdn.chunk_fwd(*args, workspace=ws, flags=_lib.MDN_TEST_NO_INTRA)
+    mdn.chunk_fwd(*args, workspace=ws, flags=_lib.MDN_TEST_NO_INTRA | width)
     assert mdn.chunk_fwd_status(ws) == _lib.MDN_ERR_TIMEOUT
-    out = mdn.chunk_fwd(*args, workspace=ws)
+    out = mdn.chunk_fwd(*args, workspace=ws, flags=width)
     assert mdn.chunk_fwd_status(ws) == _lib.MDN_OK
     compare_heads(out, inp, all_heads(inp.spec), TOL["bf16"])

@@ -50,9 +50,9 @@ def decode_cfg():
     return config_inputs(4)
 
 
-def test_step_decode_config_sampled_heads(decode_cfg):
-    """512 consecutive mdn_step calls at B=256, H=16, d=128 (bf16); sampled heads
-    against the oracle recurrence."""
+def test_step_decode_config_every_head(decode_cfg):
+    """512 consecutive mdn_step calls at B=256, H=16, d=128 (bf16); every head
+    against the oracle recurrence (one oracle call over the whole batch)."""
     inp = decode_cfg
     dev = mi.to_torch(inp, "cuda")
     B, T, H, d = inp.q.shape
@@ -65,16 +65,13 @@ def test_step_decode_config_sampled_heads(decode_cfg):
         mdn.step(*(steps[k][t] for k in ("q", "k", "v", "alpha_log", "mu_log", "beta", "eta")),
                  inp.d_corr, S, M, o=o_all[t], vtilde=vt_all[t])
     torch.cuda.synchronize()
-    heads = [(0, 0), (17, 5), (101, 15), (255, 9), (200, 3), (64, 12)]
     o_np, vt_np, S_np, M_np = to_np(o_all), to_np(vt_all), to_np(S), to_np(M)
-    for (b, h) in heads:
-        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
-        ro, rvt, rS, rM = oracle.chunk_fwd(inp.q[sl], inp.k[sl], inp.v[sl], inp.alpha_log[sl],
-                                           inp.mu_log[sl], inp.beta[sl], inp.eta[sl], inp.d_corr)
-        assert rel_l2(o_np[:, b, h], ro[0, :, 0]) <= TOL["bf16"]
-        assert rel_l2(vt_np[:, b, h], rvt[0, :, 0]) <= TOL["bf16"]
-        assert rel_l2(S_np[b, h], rS[0, 0]) <= TOL["bf16"]
-        assert rel_l2(M_np[b, h], rM[0, 0]) <= TOL["bf16"]
+    ro, rvt, rS, rM = oracle.chunk_fwd(inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log, inp.beta,
+                                       inp.eta, inp.d_corr)
+    errs = [rel_l2(o_np, ro.transpose(1, 0, 2, 3)), rel_l2(vt_np, rvt.transpose(1, 0, 2, 3)),
+            rel_l2(S_np, rS), rel_l2(M_np, rM)]
+    print("decode 512 steps rel-L2 (o, vtilde, S, M):", ", ".join(f"{e:.3e}" for e in errs))
+    assert max(errs) <= TOL["bf16"], errs
     # the same 512-token sequence through the chunkwise pass ("training == inference")
     o_c, vt_c, S_c, M_c = mdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha_log"],
                                         dev["mu_log"], dev["beta"], dev["eta"], inp.d_corr)
