@@ -185,7 +185,8 @@ mdn_status mdn_chunk_fwd(const void *q, const void *k, const void *v, mdn_dtype 
 
 /*
  * Bytes of device scratch that mdn_chunk_bwd needs, or 0 if the sizes are
- * invalid or unsupported.  Pure host function.
+ * invalid or unsupported.  For bf16 at d = 128 it covers both paths (the
+ * tensor-core path needs more than MDN_FORCE_SIMT's).  Pure host function.
  */
 size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
                                     mdn_dtype in_dtype);
@@ -207,8 +208,9 @@ size_t mdn_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
  *   dS0, dM0    [B,H,d,d] fp32 outputs (the gradients of the entering states).
  *   workspace   at least mdn_chunk_bwd_workspace_size(...) bytes, 256-byte
  *               aligned (about (4 d^2 + 3 C^2 + 10 C) x 4 bytes per chunk of C
- *               tokens of each head, plus about 260 KB per chunk for the
- *               tensor-core path's chunk operands).
+ *               tokens of each head on CUDA cores; on the tensor-core path
+ *               the states and adjoints are kept in bf16 (2 d^2 x 2 bytes
+ *               less) and the chunk operands add about 260 KB per chunk).
  *   flags       0, or MDN_CHECK_FINITE (synchronise, then report non-finite
  *               outputs or an expired device wait) and/or MDN_FORCE_SIMT (the
  *               CUDA-core kernels for bf16 d = 128 too).

@@ -88,22 +88,37 @@ __device__ __forceinline__ void bwd_unit_lower_inverse(const float* As, float* T
     }
 }
 
-// The last phase (every thread of a 256-thread CTA calls it): dG ([C][C+1],
-// overwritten), Gp ([C][C+1]), the record of the state products (rec_g, in
-// global memory; rec: kBwdRec floats of shared scratch), v.da holding the
-// direct adjoint of alpha from P.  Writes the four gate gradients of the
-// chunk's tokens.
+// Storage of the lower-triangular C x C matrices Gp and dG in shared memory
+// (element (r, i), i <= r): rows of C + 1 floats, or the lower triangle
+// packed by rows.  Both are conflict-free for a warp that walks a row (one
+// column per lane) and for one that walks a column (one row per lane: the
+// triangular numbers are distinct modulo 32 over 32 consecutive rows).
+struct PaddedLower {
+    __device__ __forceinline__ int operator()(int r, int i) const { return r * (kChunk + 1) + i; }
+};
+struct PackedLower {
+    static constexpr int kFloats = kChunk * (kChunk + 1) / 2;
+    __device__ __forceinline__ int operator()(int r, int i) const { return ((r * (r + 1)) >> 1) + i; }
+};
+
+// The last phase (every thread of a CTA of at least 128 threads calls it): dG
+// (overwritten) and Gp, lower triangles stored as Idx says, the record of the
+// state products (rec_g, in global memory; rec: kBwdRec floats of shared
+// scratch), v.da holding the direct adjoint of alpha from P.  Writes the four
+// gate gradients of the chunk's tokens.
+template <class Idx = PaddedLower>
 __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* rec_g,
                                                 const BwdVec& v, float* dG, const float* Gp,
                                                 float* rec, int tid, int n, int b, int h,
-                                                bool rec_loaded = false)
+                                                bool rec_loaded = false, int nthreads = 256)
 {
-    constexpr int C = kChunk, AS = kChunk + 1;
+    constexpr int C = kChunk;
+    const Idx at;
     // the chunk's record in shared memory (rec: kBwdRec floats), so that the
     // loops below read no global memory; a caller that copied it earlier
     // (and synchronised since) passes rec_loaded
     if (!rec_loaded) {
-        for (int i = tid; i < kBwdRec; i += 256) rec[i] = rec_g[i];
+        for (int i = tid; i < kBwdRec; i += nthreads) rec[i] = rec_g[i];
         __syncthreads();
     }
     float* v_al = v.al;
@@ -187,15 +202,15 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
     if (tid < C) {
         const int x = tid;
         float rs = 0.f;
-        for (int y = 0; y <= x; ++y) rs = fmaf(dG[x * AS + y], v_et[y] * Gp[x * AS + y], rs);
+        for (int y = 0; y <= x; ++y) rs = fmaf(dG[at(x, y)], v_et[y] * Gp[at(x, y)], rs);
         v_dla[x] += rs;
     } else if (tid < 2 * C) {
         const int x = tid - C;
         float cs = 0.f, ce = 0.f;
         for (int y = x; y < C; ++y) {
-            const float gp = Gp[y * AS + x];
-            cs = fmaf(dG[y * AS + x], v_et[x] * gp, cs);
-            ce = fmaf(dG[y * AS + x], gp, ce);
+            const float gp = Gp[at(y, x)];
+            cs = fmaf(dG[at(y, x)], v_et[x] * gp, cs);
+            ce = fmaf(dG[at(y, x)], gp, ce);
         }
         v_dlm[x] -= cs;
         v_de[x] += ce;
@@ -206,8 +221,8 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         const int i = tid;
         float R = 0.f;
         for (int j = C - 1; j >= i; --j) {
-            R = dG[j * AS + i] + (j + 1 < C ? v_al[j + 1] * R : 0.f);
-            dG[j * AS + i] = R;
+            R = dG[at(j, i)] + (j + 1 < C ? v_al[j + 1] * R : 0.f);
+            dG[at(j, i)] = R;
         }
     }
     __syncthreads();
@@ -215,7 +230,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
     if (tid < C) {
         const int j = tid;
         float U = 0.f;
-        for (int i = 0; i <= j; ++i) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[j * AS + i], U);
+        for (int i = 0; i <= j; ++i) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[at(j, i)], U);
         v_dbe[j] += U;
         v_dla[j] -= v_be[j] * U;
         v_dlm[j] += v_be[j] * U;

@@ -24,8 +24,8 @@
 // MMAs, one lane the TMA and bulk loads (two chunks ahead), 16 chain warps
 // hold rows of dS and dM in fp32 registers, 8 columns each (their bf16 copy is
 // A1's B operand), 4 output warps write dv.  NS = 32: four CTAs per head.
-// The adjoints leaving each chunk are stored in chain order (see chain_off),
-// so that each chain warp's stores are 512 contiguous bytes per instruction.
+// The adjoints leaving each chunk are stored in bf16 as the state products'
+// operand image (state_img_off), which those products copy in whole.
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
 
@@ -106,7 +106,7 @@ struct ChainArgs {
     const float* dM_T;
     float* dS0;
     float* dM0;
-    float* dss;             // [chunks][2][D][D]: adjoints of the states leaving each chunk
+    uint8_t* dss_img;       // [chunks][kStateImgBytes]: adjoints of the states leaving each chunk (bf16)
     float* dv;              // [B, T, H, D] fp32
     unsigned* status;
     int T, H, NT;
@@ -356,17 +356,15 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         for (int n = 0; n < NT; ++n) {
             const int s2 = n & 1, sv = n % L::NVC;
             const long long chunk = ch.chunk0 + (NT - 1 - n);
-            // the adjoints of the states leaving this chunk, kept for the
-            // chunk-local gradients
+            // the adjoints of the states leaving this chunk, kept (bf16, as
+            // the state products' operand image) for the chunk-local gradients
             {
-                float* dst = a.dss + (size_t)chunk * 2 * D * D;
+                uint8_t* dst = a.dss_img + (size_t)chunk * kStateImgBytes;
 #pragma unroll
-                for (int q = 0; q < NH / 4; ++q) {
-                    const int o = chain_off(lane, j0 + NH * hc + 4 * q);
-                    *reinterpret_cast<float4*>(dst + o) =
-                        make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-                    *reinterpret_cast<float4*>(dst + D * D + o) =
-                        make_float4(m[4 * q], m[4 * q + 1], m[4 * q + 2], m[4 * q + 3]);
+                for (int c = 0; c < NH / 8; ++c) {
+                    const int g = (j0 + NH * hc) / 8 + c;
+                    st_bf16x8(dst + state_img_off(lane, g), s + 8 * c);
+                    st_bf16x8(dst + state_img_off(lane + D, g), m + 8 * c);
                 }
             }
             if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
@@ -505,7 +503,7 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     t.dM_T = a.dM_T;
     t.dS0 = a.dS0;
     t.dM0 = a.dM0;
-    t.dss = a.dSS;
+    t.dss_img = a.dss_img;
     t.dv = a.dv;
     t.status = a.status;
     t.T = a.T;

@@ -12,9 +12,10 @@
 //     dq = Diag(alphabar) P1 - Diag(b) P2
 //     dk = Diag(Gamma_C) P3 - Diag(w) P4 - Diag(alphabar) P5 + Diag(D2) P6
 // and the row sums that feed the gate gradients, exactly as the CUDA-core
-// kernel does.  Operands are staged by the threads themselves (fp32 states
-// and dY are rounded to bf16 on the way into shared memory), K-major with the
-// 128-byte swizzle.
+// kernel does.  The states and adjoints arrive as bf16 images of the B
+// operands (written by the state scan and the reverse chain), two bulk
+// copies; dO, Vt and dY (fp32, rounded to bf16) are staged by the threads,
+// K-major with the 128-byte swizzle.
 #include "bwd_common.cuh"
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
@@ -33,7 +34,7 @@ constexpr uint32_t SB1 = 65536;      // [S | M] as 256 rows: 2 K-panels x 256 ro
 constexpr uint32_t SB2 = 131072;     // [dS | dM]
 constexpr uint32_t SSUM = 196608;    // fp32 row-sum partials [12][64], then scalars [8][3]
 constexpr uint32_t SBAR = SSUM + 3072 + 96;
-constexpr uint32_t SMISC = SBAR + 16;
+constexpr uint32_t SMISC = SBAR + 16;  // after two mbarriers (MMAs done, state images landed)
 constexpr uint32_t SMEM_BYTES = SMISC + 16 + 1024;  // + alignment slack
 constexpr int XS = 129;              // row stride (floats) of the dk exchange tile over SA1
 
@@ -62,8 +63,17 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SMISC);
 
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         mbar_fence_init();
+        // [S | M] entering the chunk and [dS | dM] leaving it: bf16 images of
+        // the B operands, copied in whole
+        mbar_arrive_expect_tx(&bar[1], 2 * kStateImgBytes);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            bulk_load(sm + SB1 + p * 16384, a.ss_img + chunk * kStateImgBytes + p * 16384, 16384, &bar[1]);
+            bulk_load(sm + SB2 + p * 16384, a.dss_img + chunk * kStateImgBytes + p * 16384, 16384, &bar[1]);
+        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -105,47 +115,28 @@ bwd_state_grads_tc_kernel(BwdArgs a)
             *reinterpret_cast<uint4*>(sm + SA2 + off) = rv[u];
         }
     }
-    // S, M, dS, dM (fp32 -> bf16), 128 rows x 16 chunks each; the three scalars
-    const float* Sn = a.SS + chunk * 2 * D * D;
-    const float* Mn = Sn + D * D;
-    const float* dSn = a.dSS + chunk * 2 * D * D;
-    const float* dMn = dSn + D * D;
+    fence_proxy_async_smem();
+    __syncthreads();
+    // the chunk-end scalars' adjoints: <S, dS>, <M, dS>, <M, dM> over the
+    // bf16 states the products use (a warp reads 32 consecutive rows of one
+    // 8-column group: conflict-free under the swizzle)
+    bool ok = mbar_wait(&bar[1], 0);
     float s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    // all four in chain order: consecutive threads take consecutive rows, so a
-    // warp's float4 loads are 512 contiguous bytes
-    // (two row pieces per round, their loads issued before the stores)
-#pragma unroll 1
-    for (int i0 = tid; i0 < D * 16; i0 += 2 * kThr) {
-        float sv[2][8], mv[2][8], dsv[2][8], dmv[2][8];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = i0 + kThr * u, rest = i >> 5, c16 = rest >> 2;
-            const int row = ((rest & 3) << 5) | (i & 31);
-            const int g = chain_off(row, c16 * 8), g4 = chain_off(row, c16 * 8 + 4);
-            *reinterpret_cast<float4*>(sv[u]) = *reinterpret_cast<const float4*>(Sn + g);
-            *reinterpret_cast<float4*>(sv[u] + 4) = *reinterpret_cast<const float4*>(Sn + g4);
-            *reinterpret_cast<float4*>(mv[u]) = *reinterpret_cast<const float4*>(Mn + g);
-            *reinterpret_cast<float4*>(mv[u] + 4) = *reinterpret_cast<const float4*>(Mn + g4);
-            *reinterpret_cast<float4*>(dsv[u]) = *reinterpret_cast<const float4*>(dSn + g);
-            *reinterpret_cast<float4*>(dsv[u] + 4) = *reinterpret_cast<const float4*>(dSn + g4);
-            *reinterpret_cast<float4*>(dmv[u]) = *reinterpret_cast<const float4*>(dMn + g);
-            *reinterpret_cast<float4*>(dmv[u] + 4) = *reinterpret_cast<const float4*>(dMn + g4);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = i0 + kThr * u, rest = i >> 5, c16 = rest >> 2;
-            const int row = ((rest & 3) << 5) | (i & 31);
+    if (ok) {
+#pragma unroll 2
+        for (int i = tid; i < D * 16; i += kThr) {
+            const int row = i & (D - 1), g = i >> 7;
+            float sv[8], mv[8], dsv[8], dmv[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + SB1 + state_img_off(row, g)), sv);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + SB1 + state_img_off(row + D, g)), mv);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + SB2 + state_img_off(row, g)), dsv);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + SB2 + state_img_off(row + D, g)), dmv);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                s1 = fmaf(sv[u][e], dsv[u][e], s1);
-                s2 = fmaf(mv[u][e], dsv[u][e], s2);
-                s3 = fmaf(mv[u][e], dmv[u][e], s3);
+                s1 = fmaf(sv[e], dsv[e], s1);
+                s2 = fmaf(mv[e], dsv[e], s2);
+                s3 = fmaf(mv[e], dmv[e], s3);
             }
-            const uint32_t pan = (c16 >> 3) * 32768;
-            st_bf16x8(sm + SB1 + pan + sw128_off(row, c16 & 7), sv[u]);
-            st_bf16x8(sm + SB1 + pan + sw128_off(row + 128, c16 & 7), mv[u]);
-            st_bf16x8(sm + SB2 + pan + sw128_off(row, c16 & 7), dsv[u]);
-            st_bf16x8(sm + SB2 + pan + sw128_off(row + 128, c16 & 7), dmv[u]);
         }
     }
 #pragma unroll
@@ -159,13 +150,12 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         wsum[warp * 3 + 1] = s2;
         wsum[warp * 3 + 2] = s3;
     }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (tid == 0) {
+    if (tid == 0 && ok) {
         constexpr uint32_t id = idesc_bf16(128, 256, false, false);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -179,9 +169,9 @@ bwd_state_grads_tc_kernel(BwdArgs a)
             mma_bf16(tmem + 256, smem_desc(sbase + SA2 + ko, 16, 1024, kSw128),
                      smem_desc(sbase + SB2 + kb, 16, 1024, kSw128), id, ks > 0);
         }
-        mma_commit(bar);
+        mma_commit(&bar[0]);
     }
-    const bool ok = __syncthreads_and(mbar_wait(bar, 0));
+    ok = __syncthreads_and(ok && mbar_wait(&bar[0], 0));
     tc_fence_after_sync();
 
     // Epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..; warps w and w + 4 take
@@ -292,7 +282,10 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         for (int w8 = 0; w8 < 8; ++w8) acc += wsum[w8 * 3 + tid];
         rec[5 * C + tid] = acc;
     }
-    if (!ok && tid == 0) atomicOr(a.status + 1, 1u);
+    if (!ok && tid == 0) {
+        atomicOr(a.status + 1, 1u);
+        (void)mbar_wait(&bar[1], 0);  // the state copies land before shared memory is released
+    }
     if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
@@ -308,19 +301,29 @@ bwd_state_grads_tc_kernel(BwdArgs a)
 //   stage 2: [dOVG; dPK] K -> dQhat part (lanes 0..63), dP = dPK K (64..127) (N 128)
 //            [dOVG^T | (Diag(alpha) dPK)^T] [Qhat; K] -> dK part                (N 128)
 //   SIMT:    dq, dk written; the coefficient phase gives the gate gradients.
-constexpr uint32_t LA_DY = 0;        // [dO; dY]   K-major, 2 K-panels x 128 rows x 128 B
-constexpr uint32_t LA_QK = 32768;    // [Qhat; K]  K-major (its K rows double as B of K K^T)
-constexpr uint32_t LB_V = 65536;     // Vt         K-major, 2 K-panels x 64 rows x 128 B
-constexpr uint32_t LA_3 = 81920;     // [dOVG; dPK]          K = 64: 1 panel x 128 rows x 128 B
-constexpr uint32_t LA_4 = 98304;     // [dOVG^T | dPKa^T; 0] K = 128: 2 panels x 128 rows x 128 B
-constexpr uint32_t L_GP = 131072;    // fp32 Gp [64][65]
-constexpr uint32_t L_DG = L_GP + 16640;   // fp32 dG [64][65]
-constexpr uint32_t L_VEC = L_DG + 16640;  // 12 x 64 floats
+// Two CTAs share an SM, so that one chunk's serial phases overlap another's:
+// stage 2 accumulates over stage 1's TMEM columns (256 in all), its operands
+// are written over stage 1's once those have been read, the exchange tile of
+// the last epilogue over stage 2's, and Gamma's factor Gp and the adjoint dG
+// are kept as packed lower triangles (about 102 KB of shared memory).
+constexpr uint32_t LA_QK = 0;        // [Qhat; K]  K-major, 2 K-panels x 128 rows x 128 B (its K rows double as B of K K^T)
+constexpr uint32_t LA_DY = 32768;    // [dO; dY]   K-major (stage 1)
+constexpr uint32_t LB_V = 65536;     // Vt         K-major, 2 K-panels x 64 rows x 128 B (stage 1)
+constexpr uint32_t LA_3 = 32768;     // [dOVG; dPK]          K = 64: 1 panel x 128 rows x 128 B (stage 2)
+constexpr uint32_t LA_4 = 49152;     // [dOVG^T | dPKa^T; 0] K = 128: 2 panels x 128 rows x 128 B (stage 2)
+constexpr uint32_t L_X = 32768;      // fp32 alpha_r dP [64][129] (once stage 2 has completed)
+constexpr int LXS = 129;             // its row stride (floats)
+constexpr uint32_t L_GP = 81920;     // fp32 Gp, packed lower triangle
+constexpr uint32_t L_DG = L_GP + PackedLower::kFloats * 4;   // fp32 dG, packed lower triangle
+constexpr uint32_t L_VEC = L_DG + PackedLower::kFloats * 4;  // 12 x 64 floats
 constexpr uint32_t L_REC = L_VEC + 3072;  // the chunk record (kBwdRec floats)
 constexpr uint32_t L_BAR = L_REC + kBwdRec * 4;
 constexpr uint32_t L_MISC = L_BAR + 16;
 constexpr uint32_t L_SMEM = L_MISC + 16 + 1024;
-constexpr int LAS = 65;                   // row stride of the fp32 C x C matrices
+constexpr uint32_t kLocalTmemCols = 256;
+static_assert(L_X + 64 * LXS * 4 <= L_GP, "exchange tile");
+static_assert(LA_4 + 32768 <= L_GP && LB_V + 16384 <= L_GP, "operand map");
+static_assert(2 * (L_SMEM + 1024) <= 233472, "two CTAs per SM");
 
 __device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
     *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
@@ -330,8 +333,11 @@ __device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
 __device__ __forceinline__ uint32_t kmaj_off(int row, int k, uint32_t panel_bytes) {
     return (k >> 6) * panel_bytes + sw128_off(row, (k & 63) >> 3) + (k & 7) * 2;
 }
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThr, 2)
 bwd_local_grads_tc_kernel(BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -343,8 +349,10 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     const long long bh = blockIdx.x / a.NT;
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x, crow = chunk * C;
+    const PackedLower at;
     float* Gp = reinterpret_cast<float*>(sm + L_GP);
     float* dG = reinterpret_cast<float*>(sm + L_DG);
+    float* recs = reinterpret_cast<float*>(sm + L_REC);
     const BwdVec v = bwd_vec(reinterpret_cast<float*>(sm + L_VEC));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L_MISC);
@@ -355,7 +363,7 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         mbar_fence_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, kLocalTmemCols);
         tmem_relinquish();
     }
     // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major), and the chunk's
@@ -400,14 +408,8 @@ bwd_local_grads_tc_kernel(BwdArgs a)
             *reinterpret_cast<uint4*>(sm + LA_QK + off + 64 * 128) = rk[u];
             *reinterpret_cast<uint4*>(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7)) = rv[u];
         }
-        float* recs = reinterpret_cast<float*>(sm + L_REC);
         recs[tid] = rc0;
         if (tid + kThr < kBwdRec) recs[tid + kThr] = rc1;
-    }
-    // rows 64..127 of the second stage-2 operand are zero
-    for (int i = tid; i < 1024; i += kThr) {
-        const int p = i >> 9, w = i & 511;
-        *reinterpret_cast<uint4*>(sm + LA_4 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
     }
     if (tid < C) {
         const int r = tid, t = n * C + r;
@@ -440,51 +442,73 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         }
         mma_commit(&bars[0]);
     }
+    // the rows of dq and dk that the last epilogue reads back (written by the
+    // state products), pulled into L2 meanwhile: 64 rows x 2 x 512 B
+    {
+        const int r = tid >> 2, t = n * C + r;
+        if (t < a.T) {
+            const size_t g = tokrow(a, b, t, h) * D + (tid & 3) * 32;
+            prefetch_l2(a.dq + g);
+            prefetch_l2(a.dk + g);
+        }
+    }
     // Gamma without eta, by its column recurrence (overlaps the products):
     // Gp_{r,i} = alpha_r Gp_{r-1,i} + beta_r mubar_r / mubar_i, the ratio as a
     // running product of mu (held in v.de until the coefficient phase)
     if (tid < C) {
         const int i = tid;
-        float g = 0.f, f = 1.f;
-        for (int r = 0; r < C; ++r) {
-            if (r < i) {
-                Gp[r * LAS + i] = 0.f;
-            } else {
-                if (r > i) f *= v.de[r];
-                g = (r == i) ? v.be[i] : fmaf(v.al[r], g, v.be[r] * f);
-                Gp[r * LAS + i] = g;
-            }
+        float g = v.be[i], f = 1.f;
+        Gp[at(i, i)] = g;
+        for (int r = i + 1; r < C; ++r) {
+            f *= v.de[r];
+            g = fmaf(v.al[r], g, v.be[r] * f);
+            Gp[at(r, i)] = g;
         }
     }
     bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
     tc_fence_after_sync();
 
     // stage-1 epilogue: warp w reads lanes 32 (w % 4) ..; warps w, w + 4 take
-    // columns i in [32 half, 32 half + 32)
+    // columns i in [32 half, 32 half + 32), 16 at a time
     const int quad = warp & 3, half = warp >> 2;
     const int R = quad * 32 + lane, r = R & 63;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     float dgm[32];  // dY rows: dA o (P K^T), owed to dG[r - 1][i]
     if (ok) {
-        float x1[32], x2[32];
-        tmem_ld32(tq + 32 * half, x1);        // dO Vt^T  (dY Vt^T on lanes 64..127)
-        tmem_ld32(tq + 64 + 32 * half, x2);   // Qhat K^T (K K^T)
-        tmem_wait_ld();
+        // rows 64..127 of the second stage-2 operand are zero (over stage 1's
+        // operands, which the completed products have read)
+        for (int i = tid; i < 1024; i += kThr) {
+            const int p = i >> 9, w = i & 511;
+            *reinterpret_cast<uint4*>(sm + LA_4 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
+        }
         const float al_r = v.al[r];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int i = 32 * half + e;
-            if (R < 64) {
-                const float g = v.et[i] * Gp[r * LAS + i];
-                const float ovg = i <= r ? x1[e] * g : 0.f;
-                dG[r * LAS + i] = i <= r ? x1[e] * x2[e] : 0.f;
-                st_bf16(sm + LA_3 + kmaj_off(r, i, 16384), ovg);             // row r of [dOVG; .]
-                st_bf16(sm + LA_4 + kmaj_off(i, r, 16384), ovg);             // (dOVG^T)[i][r]
-            } else {
-                const float pk = i < r ? -x1[e] * v.et[i] * Gp[(r - 1) * LAS + i] : 0.f;
-                dgm[e] = i < r ? -x1[e] * al_r * x2[e] : 0.f;
-                st_bf16(sm + LA_3 + kmaj_off(64 + r, i, 16384), pk);        // row 64 + r: dPK
-                st_bf16(sm + LA_4 + kmaj_off(i, 64 + r, 16384), pk * al_r); // (Diag(alpha) dPK)^T
+        for (int p2 = 0; p2 < 2; ++p2) {
+            float x1[16], x2[16];
+            tmem_ld16(tq + 32 * half + 16 * p2, x1);        // dO Vt^T  (dY Vt^T on lanes 64..127)
+            tmem_ld16(tq + 64 + 32 * half + 16 * p2, x2);   // Qhat K^T (K K^T)
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int i = 32 * half + 16 * p2 + e;
+                if (R < 64) {
+                    float ovg = 0.f;
+                    if (i <= r) {
+                        ovg = x1[e] * (v.et[i] * Gp[at(r, i)]);
+                        dG[at(r, i)] = x1[e] * x2[e];
+                    }
+                    st_bf16(sm + LA_3 + kmaj_off(r, i, 16384), ovg);             // row r of [dOVG; .]
+                    st_bf16(sm + LA_4 + kmaj_off(i, r, 16384), ovg);             // (dOVG^T)[i][r]
+                } else {
+                    float pk = 0.f, dm = 0.f;
+                    if (i < r) {
+                        pk = -x1[e] * v.et[i] * Gp[at(r - 1, i)];
+                        dm = -x1[e] * al_r * x2[e];
+                    }
+                    dgm[16 * p2 + e] = dm;
+                    st_bf16(sm + LA_3 + kmaj_off(64 + r, i, 16384), pk);        // row 64 + r: dPK
+                    st_bf16(sm + LA_4 + kmaj_off(i, 64 + r, 16384), pk * al_r); // (Diag(alpha) dPK)^T
+                }
             }
         }
     }
@@ -496,33 +520,32 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int i = 32 * half + e;
-            if (i < r) dG[(r - 1) * LAS + i] += dgm[e];  // one writer per entry
+            if (i < r) dG[at(r - 1, i)] += dgm[e];  // one writer per entry
         }
     }
-    const float* rec = a.crec_bw + chunk * kBwdRec;
     if (tid == 0 && ok) {
         constexpr uint32_t id2 = idesc_bf16(128, 128, false, true);
         // [dOVG; dPK] K: B = K (K-dim i = rows 64..127 of the [Qhat; K] tile, N = features)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tmem + 128, smem_desc(sbase + LA_3 + ks * 32, 16, 1024, kSw128),
+            mma_bf16(tmem, smem_desc(sbase + LA_3 + ks * 32, 16, 1024, kSw128),
                      smem_desc(sbase + LA_QK + 8192 + ks * 2048, 16384, 1024, kSw128), id2, ks > 0);
         // [dOVG^T | dPKa^T] [Qhat; K]: B = the whole [Qhat; K] tile, K-dim 128 rows
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tmem + 256,
+            mma_bf16(tmem + 128,
                      smem_desc(sbase + LA_4 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSw128),
                      smem_desc(sbase + LA_QK + ks * 2048, 16384, 1024, kSw128), id2, ks > 0);
         mma_commit(&bars[1]);
     }
     __syncthreads();
-    if (tid < C) dG[(C - 1) * LAS + tid] += rec[3 * C + tid];  // Gamma_{C,i} in the state update
+    if (tid < C) dG[at(C - 1, tid)] += recs[3 * C + tid];  // Gamma_{C,i} in the state update
     ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
     tc_fence_after_sync();
 
     // stage-2 epilogue: lanes 64..127 hold dP = dPK K; lanes 0..63 the dQhat
     // and dK parts; warps w, w + 4 take feature columns [64 half, 64 half + 64)
-    float* X = reinterpret_cast<float*>(sm + LA_DY);  // alpha_r dP[r][c], [64][129], over the operands
+    float* X = reinterpret_cast<float*>(sm + L_X);  // alpha_r dP[r][c], over stage 2's operands
     const int t = n * C + r;
     const bool in = t < a.T;
     const size_t grow = in ? tokrow(a, b, t, h) * D : 0;
@@ -533,7 +556,7 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float dp[16], kv[16];
-            tmem_ld16(tq + 128 + c0, dp);
+            tmem_ld16(tq + c0, dp);
             tmem_wait_ld();
             if (in) {
                 unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + c0), kv);
@@ -542,18 +565,14 @@ bwd_local_grads_tc_kernel(BwdArgs a)
                 for (int e = 0; e < 16; ++e) dar = fmaf(dp[e], kv[e], dar);
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) X[r * 129 + c0 + e] = al_r * dp[e];
+            for (int e = 0; e < 16; ++e) X[r * LXS + c0 + e] = al_r * dp[e];
         }
-        atomicAdd(v.da + r, dar);
+        atomicAdd(v.da + r, dar);  // two addends onto 0: the same sum in either order
     }
     __syncthreads();
     if (ok && R < 64) {
-        // The exchange row is read into registers before any global store: X is
-        // reached through a generic pointer, so reads of it interleaved with the
-        // stores to dq and dk could not be hoisted and serialised the loop.
-        float xr[64];
-#pragma unroll
-        for (int e = 0; e < 64; ++e) xr[e] = X[r * 129 + 64 * half + e];
+        float* __restrict__ dqr = a.dq + grow;
+        float* __restrict__ dkr = a.dk + grow;
 #pragma unroll
         for (int j2 = 0; j2 < 4; j2 += 2) {  // two 16-column groups per round
             float4 q4[2][4], k4[2][4];
@@ -563,16 +582,18 @@ bwd_local_grads_tc_kernel(BwdArgs a)
 #pragma unroll
                     for (int e4 = 0; e4 < 4; ++e4) {  // every load of the round before any store
                         const int c = 64 * half + 16 * (j2 + g) + 4 * e4;
-                        q4[g][e4] = *reinterpret_cast<const float4*>(a.dq + grow + c);
-                        k4[g][e4] = *reinterpret_cast<const float4*>(a.dk + grow + c);
+                        q4[g][e4] = *reinterpret_cast<const float4*>(dqr + c);
+                        k4[g][e4] = *reinterpret_cast<const float4*>(dkr + c);
                     }
             }
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
-                const int j = j2 + g, c0 = 64 * half + 16 * j;
-                float dqb[16], dkb[16];
-                tmem_ld16(tq + 128 + c0, dqb);
-                tmem_ld16(tq + 256 + c0, dkb);
+                const int c0 = 64 * half + 16 * (j2 + g);
+                float dqb[16], dkb[16], xr[16];
+                tmem_ld16(tq + c0, dqb);
+                tmem_ld16(tq + 128 + c0, dkb);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) xr[e] = X[r * LXS + c0 + e];
                 tmem_wait_ld();
                 if (in) {
 #pragma unroll
@@ -582,14 +603,11 @@ bwd_local_grads_tc_kernel(BwdArgs a)
                         float qn[4], kn[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int x = 16 * j + 4 * e4 + e;
                             qn[e] = qo[e] + dqb[4 * e4 + e];
-                            kn[e] = ko[e] + dkb[4 * e4 + e] + xr[x] - a.dcorr * qn[e];
+                            kn[e] = ko[e] + dkb[4 * e4 + e] + xr[4 * e4 + e] - a.dcorr * qn[e];
                         }
-                        *reinterpret_cast<float4*>(a.dq + grow + c0 + 4 * e4) =
-                            make_float4(qn[0], qn[1], qn[2], qn[3]);
-                        *reinterpret_cast<float4*>(a.dk + grow + c0 + 4 * e4) =
-                            make_float4(kn[0], kn[1], kn[2], kn[3]);
+                        *reinterpret_cast<float4*>(dqr + c0 + 4 * e4) = make_float4(qn[0], qn[1], qn[2], qn[3]);
+                        *reinterpret_cast<float4*>(dkr + c0 + 4 * e4) = make_float4(kn[0], kn[1], kn[2], kn[3]);
                     }
                 }
             }
@@ -599,13 +617,13 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kLocalTmemCols);
     }
     if (!ok) {
         if (tid == 0) atomicOr(a.status + 1, 1u);
         return;
     }
-    bwd_coeff_phase(a, rec, v, dG, Gp, reinterpret_cast<float*>(sm + L_REC), tid, n, b, h, true);
+    bwd_coeff_phase<PackedLower>(a, recs, v, dG, Gp, recs, tid, n, b, h, true, kThr);
 }
 
 // ---------------------------------------------------------------------------
@@ -1090,34 +1108,52 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 }
 
 // The states entering every chunk by the elementwise recurrence
-// S <- alphabar_C S - b_C M + D_S, M <- mubar_C M - D_M (one element of a
-// head's d x d states per lane group of four).
+// S <- alphabar_C S - b_C M + D_S, M <- mubar_C M - D_M, in fp32 registers;
+// each chunk's entering pair is stored as the bf16 image the state products
+// copy in (state_img_off).  A thread owns 8 columns of one row of a head's
+// S and M; a warp takes 32 consecutive rows, so its loads of the increments
+// (chain order) are 512 contiguous bytes.
 __global__ void __launch_bounds__(256)
 bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0,
                       const float* __restrict__ dinc, const float* __restrict__ rec,
-                      float* __restrict__ SS, int NT, long long heads)
+                      uint8_t* __restrict__ img, int NT, long long heads)
 {
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long per = D * D / 4;
+    constexpr int per = D * (D / 8);
     if (gid >= heads * per) return;
     const long long bh = gid / per;
-    const int e4 = (int)(gid % per) * 4;  // chain order; S0, M0 are row-major
-    int i0, j0;
-    chain_ij(e4, i0, j0);
-    const int r4 = i0 * D + j0;
-    float4 s = S0 ? *reinterpret_cast<const float4*>(S0 + bh * D * D + r4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 m = M0 ? *reinterpret_cast<const float4*>(M0 + bh * D * D + r4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int rem = (int)(gid % per), g = rem / D, i = rem % D;
+    float s[8], m[8];
+    const size_t r0 = (size_t)bh * D * D + (size_t)i * D + 8 * g;  // S0, M0 are row-major
+#pragma unroll
+    for (int h4 = 0; h4 < 2; ++h4) {
+        const float4 a = S0 ? *reinterpret_cast<const float4*>(S0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b = M0 ? *reinterpret_cast<const float4*>(M0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[4 * h4] = a.x; s[4 * h4 + 1] = a.y; s[4 * h4 + 2] = a.z; s[4 * h4 + 3] = a.w;
+        m[4 * h4] = b.x; m[4 * h4 + 1] = b.y; m[4 * h4 + 2] = b.z; m[4 * h4 + 3] = b.w;
+    }
+    const int o0 = chain_off(i, 8 * g), o1 = chain_off(i, 8 * g + 4);
+    const uint32_t ps = state_img_off(i, g), pm = state_img_off(i + D, g);
     for (int nn = 0; nn < NT; ++nn) {
         const size_t chunk = (size_t)bh * NT + nn;
-        const float4 ds = __ldg(reinterpret_cast<const float4*>(dinc + chunk * 2 * D * D + e4));
-        const float4 dm = __ldg(reinterpret_cast<const float4*>(dinc + chunk * 2 * D * D + D * D + e4));
+        const float* dn = dinc + chunk * 2 * D * D;
+        const float4 ds0 = __ldg(reinterpret_cast<const float4*>(dn + o0));
+        const float4 ds1 = __ldg(reinterpret_cast<const float4*>(dn + o1));
+        const float4 dm0 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o0));
+        const float4 dm1 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o1));
         const float aC = __ldg(rec + chunk * 256 + 3 * C), bC = __ldg(rec + chunk * 256 + 3 * C + 1);
         const float mC = __ldg(rec + chunk * 256 + 3 * C + 2);
-        *reinterpret_cast<float4*>(SS + chunk * 2 * D * D + e4) = s;
-        *reinterpret_cast<float4*>(SS + chunk * 2 * D * D + D * D + e4) = m;
-        s = make_float4(aC * s.x - bC * m.x + ds.x, aC * s.y - bC * m.y + ds.y,
-                        aC * s.z - bC * m.z + ds.z, aC * s.w - bC * m.w + ds.w);
-        m = make_float4(mC * m.x - dm.x, mC * m.y - dm.y, mC * m.z - dm.z, mC * m.w - dm.w);
+        uint8_t* im = img + chunk * kStateImgBytes;
+        *reinterpret_cast<uint4*>(im + ps) = bf16x8(s);
+        *reinterpret_cast<uint4*>(im + pm) = bf16x8(m);
+        const float dsv[8] = {ds0.x, ds0.y, ds0.z, ds0.w, ds1.x, ds1.y, ds1.z, ds1.w};
+        const float dmv[8] = {dm0.x, dm0.y, dm0.z, dm0.w, dm1.x, dm1.y, dm1.z, dm1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float sn = fmaf(aC, s[e], fmaf(-bC, m[e], dsv[e]));
+            m[e] = fmaf(mC, m[e], -dmv[e]);
+            s[e] = sn;
+        }
     }
 }
 
@@ -1148,6 +1184,9 @@ cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(bwd_local_grads_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L_SMEM);
+    if (e == cudaSuccess)  // two CTAs per SM need the larger carve-out
+        e = cudaFuncSetAttribute(bwd_local_grads_tc_kernel,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     ProfScope ps(kBwdLocal, s);
     bwd_local_grads_tc_kernel<<<(unsigned)chunks, kThr, L_SMEM, s>>>(a);
@@ -1184,10 +1223,10 @@ cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s)
     }
     if ((e = cudaGetLastError())) return e;
     const long long heads = (long long)a.B * a.H;
-    const long long threads = heads * D * D / 4;
+    const long long threads = heads * D * (D / 8);
     ProfScope ps(kBwdStates, s);
     bwd_state_scan_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
-        a.S0, a.M0, a.bc_d, a.bc_rec, a.SS, a.NT, heads);
+        a.S0, a.M0, a.bc_d, a.bc_rec, a.ss_img, a.NT, heads);
     return cudaGetLastError();
 }
 

@@ -335,7 +335,9 @@ struct BwdLayout {
     size_t total;
 };
 
-// tc: the tensor-core reverse chain's chunk operands are included.
+// tc: the tensor-core path (bf16 state images instead of fp32 states, and the
+// reverse chain's chunk operands).  For bf16 at d = 128 its total is the
+// larger of the two paths'.
 BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
 {
     const size_t chunks = (size_t)BH * NT, rows = chunks * kChunk;
@@ -349,8 +351,9 @@ BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
     w.gamma = off; off += align_up(rows * kChunk * sizeof(float));
     w.att = off;   off += align_up(rows * kChunk * sizeof(float));
     w.tmat = off;  off += align_up(rows * kChunk * sizeof(float));
-    w.SS = off;    off += align_up(chunks * 2 * D * D * sizeof(float));
-    w.dSS = off;   off += align_up(chunks * 2 * D * D * sizeof(float));
+    const size_t state_bytes = tc ? (size_t)kStateImgBytes : 2 * D * D * sizeof(float);
+    w.SS = off;    off += align_up(chunks * state_bytes);
+    w.dSS = off;   off += align_up(chunks * state_bytes);
     w.rec = off;   off += align_up(chunks * kBwdRec * sizeof(float));
     w.bc_u = w.bc_tt = w.bc_p = w.bc_qh = w.bc_eo = w.bc_rec = w.bc_d = 0;
     if (tc) {
@@ -403,7 +406,8 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
             if (!p || !aligned4(p)) return MDN_ERR_INVALID_ARG;
     }
     const int NT = (T + C - 1) / C;
-    const BwdLayout w = bwd_layout((long long)B * H, NT, D, in_dtype == MDN_BF16 && D == 128);
+    const bool tc = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
+    const BwdLayout w = bwd_layout((long long)B * H, NT, D, tc);
     if (T > 0 && (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign))
         return MDN_ERR_INVALID_ARG;
     if (T > 0 && ws_bytes < w.total) return MDN_ERR_INVALID_ARG;
@@ -432,10 +436,11 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.gamma = reinterpret_cast<float*>(ws + w.gamma);
     a.att = reinterpret_cast<float*>(ws + w.att);
     a.tmat = reinterpret_cast<float*>(ws + w.tmat);
-    a.SS = reinterpret_cast<float*>(ws + w.SS);
-    a.dSS = reinterpret_cast<float*>(ws + w.dSS);
+    a.SS = tc ? nullptr : reinterpret_cast<float*>(ws + w.SS);
+    a.dSS = tc ? nullptr : reinterpret_cast<float*>(ws + w.dSS);
+    a.ss_img = tc ? reinterpret_cast<uint8_t*>(ws + w.SS) : nullptr;
+    a.dss_img = tc ? reinterpret_cast<uint8_t*>(ws + w.dSS) : nullptr;
     a.crec_bw = reinterpret_cast<float*>(ws + w.rec);
-    const bool tc = in_dtype == MDN_BF16 && D == 128 && !(flags & MDN_FORCE_SIMT);
     a.bc_u = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_u) : nullptr;
     a.bc_tt = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_tt) : nullptr;
     a.bc_p = tc ? reinterpret_cast<float*>(ws + w.bc_p) : nullptr;

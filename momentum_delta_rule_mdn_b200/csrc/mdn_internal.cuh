@@ -164,6 +164,15 @@ __device__ __forceinline__ void chain_ij(int o, int& i, int& j) {
     i = (o >> 2) & 127;
     j = ((o >> 9) << 2) | (o & 3);
 }
+// A pair of d x d states [X | Y] (d = 128) in bf16 as one 64 KB image: 256
+// rows (X's rows, then Y's), K-major, two 64-column panels of 256 rows x 128 B
+// with the 128-byte swizzle.  It is the shared-memory form of the B operand
+// of products by X^T and Y^T, so a plain bulk copy moves it in.  Byte offset
+// of the 16-byte piece holding columns 8g .. 8g + 7 of row `row`:
+constexpr uint32_t kStateImgBytes = 2u * 128u * 128u * 2u;
+__device__ __forceinline__ uint32_t state_img_off(int row, int g) {
+    return (uint32_t)(g >> 3) * 32768u + (uint32_t)row * 128u + ((uint32_t)((g ^ row) & 7) << 4);
+}
 struct BwdArgs {
     const void* q;
     const void* k;
@@ -189,8 +198,13 @@ struct BwdArgs {
     float* gamma;    // [B*H*NT, C, C]
     float* att;      // [B*H*NT, C, C]  (Qhat K^T) o Gamma
     float* tmat;     // [B*H*NT, C, C]  T = (I + A)^{-1}
-    float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk (tensor-core path: chain order)
-    float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk (idem)
+    float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk (CUDA-core path)
+    float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk (CUDA-core path)
+    // tensor-core path (null otherwise): the same states and adjoints as bf16,
+    // each chunk's [S | M] and [dS | dM] as the 64 KB shared-memory image of
+    // the state products' B operand (see state_img_off)
+    uint8_t* ss_img;   // [B*H*NT][kStateImgBytes]
+    uint8_t* dss_img;  // [B*H*NT][kStateImgBytes]
     float* crec_bw;  // [B*H*NT, kBwdRec]  coefficient adjoints from the state products
     // chunk-only operands of the tensor-core reverse chain (null on the CUDA-core path)
     __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]

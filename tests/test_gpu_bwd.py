@@ -47,10 +47,13 @@ def test_bwd_matches_gradient_oracle(dtype, d, T):
     three cotangents."""
     spec = mi.Spec("bwd", B=1, T=T, H=2, d=d, dtype=dtype, state_std=0.05, seed=501)
     g, ref = _run(spec)
+    errs = {}
     for n in NAMES:
         got = to_np(g[n])
         assert np.all(np.isfinite(got)), n
-        e = rel_l2(got, ref[n])
+        errs[n] = rel_l2(got, ref[n])
+    print(f"bwd {dtype} d={d} T={T} rel-L2:", " ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+    for n, e in errs.items():
         assert e <= TOL[dtype], (n, e)
 
 
@@ -59,8 +62,9 @@ def test_bwd_layer_shape_sampled():
     H = 2, zero entering states, o's cotangent only."""
     spec = mi.Spec("bwd_layer", B=2, T=512, H=2, d=128, seed=502)
     g, ref = _run(spec, with_state_cot=False)
-    for n in NAMES:
-        e = rel_l2(to_np(g[n]), ref[n])
+    errs = {n: rel_l2(to_np(g[n]), ref[n]) for n in NAMES}
+    print("bwd layer shape B2 T512 H2 rel-L2:", " ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+    for n, e in errs.items():
         assert e <= TOL["bf16"], (n, e)
 
 
