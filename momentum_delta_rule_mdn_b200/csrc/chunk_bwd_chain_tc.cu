@@ -10,7 +10,7 @@
 //     dM     <- -b_C dS + mubar_C dM - F + K^T Diag(D2) dY
 // with E = Qhat^T Diag(alphabar) dO, F = Qhat^T Diag(b) dO.  Folding T into
 // U = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T] (chunk data, formed with
-// Att^T dO, E, F and [T^T; 0] by a parallel kernel first), a chunk is
+// Att^T dO, E, F and T by a parallel kernel first), a chunk is
 //     A1 = [K; Qhat] [dS | dM]           (M 128, N 2 NS, K 128; lanes 0..63 used)
 //     dVtilde = Att^T dO + Diag(Gamma_C) A1_S - Diag(w) A1_M      (epilogue)
 //     A2 = U dVtilde                     (two M 128, N NS, K 64)
@@ -18,7 +18,8 @@
 //   with E = Qhat^T Diag(alphabar) dO and -F = Qhat^T (-Diag(b) dO) issued into
 //   A2's accumulators right after A1 (M 128, N NS, K 64, A MN-major from the
 //   Qhat rows of the [K; Qhat] tile), while the chain warps form dVtilde
-//     A3 = [T^T; 0] dVtilde = dY         (M 128, N NS, K 64; off the chain)
+//     A3 = T^T dVtilde = dY              (M 128 with rows 64..127 unused, N NS, K 64;
+//                                         off the chain; T^T MN-major from T's rows)
 // This is the shape of the forward pass's inter-chunk kernel, whose warp
 // roles, hand-offs and bounded waits this kernel keeps: one lane issues the
 // MMAs, one lane the TMA and bulk loads (two chunks ahead), 16 chain warps
@@ -50,7 +51,7 @@ struct Cfg {
     static constexpr uint32_t kTmemCols = NS == 32 ? 256 : 512;
     // shared memory (byte offsets from a 1024-byte aligned base)
     static constexpr uint32_t KQ0 = 0;                // [K; Qhat], 2 slots x 2 panels x (128 rows x 128 B)
-    static constexpr uint32_t FB0 = 2 * 32768;        // [T; Att T] (16 KB), [A2T_S | A2T_M] (2 x 16 KB), 2 slots
+    static constexpr uint32_t FB0 = 2 * 32768;        // T (8 KB of a 16 KB part), [U_S | U_M] (2 x 16 KB), 2 slots
     static constexpr uint32_t FB_BYTES = 49152;
     static constexpr uint32_t ST = FB0 + 2 * FB_BYTES;  // [S | M] bf16, 128 rows, MN-major 128-byte swizzle
     static constexpr uint32_t ST_BYTES = 128 * 2 * NS * 2;
@@ -81,7 +82,7 @@ struct Cfg {
 };
 
 constexpr uint32_t kTxKQ = 32768;   // K, Qhat
-constexpr uint32_t kTxFB = 49152;   // [T; Att T], A2T
+constexpr uint32_t kTxFB = 8192 + 32768;  // T (64 x 64), U
 
 // mbarriers (index into the array at BARS); as in the inter-chunk kernel
 constexpr int B_FKQ = 0;   // [2] K, Qhat landed
@@ -108,6 +109,7 @@ struct ChainArgs {
     float* dM0;
     uint8_t* dss_img;       // [chunks][kStateImgBytes]: adjoints of the states leaving each chunk (bf16)
     float* dv;              // [B, T, H, D] fp32
+    uint8_t* dy_img;        // [chunks][kDyImgBytes]: dv of each chunk in bf16 (operand image)
     unsigned* status;
     int T, H, NT;
     const int* cu_seqlens;  // unused here (one batch row per sequence)
@@ -279,9 +281,13 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 }
                 mma_commit(&bars[B_M2]);
                 clk.lap(5);
+                // A3 = T^T dVtilde: T^T is the MN-major form of T's row-major rows (M-panel 0;
+                // the output rows of panel 1, from the rest of the slot, are not read)
+                const uint32_t tt = sbase + L::FB0 + s2 * L::FB_BYTES;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + L::TM_A3 + NS * s2, dfb + ks * 2, d_y + ks * ystep, id2, ks > 0);
+                    mma_bf16(tmem + L::TM_A3 + NS * s2, smem_desc(tt + ks * 2048, 8192, 1024, kSw128),
+                             d_y + ks * ystep, idef, ks > 0);
                 mma_commit(&bars[B_M3 + s2]);
                 clk.lap(6);
             }
@@ -444,17 +450,27 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             if (yrow) {
                 const int t = (NT - 1 - n) * C + r;  // token of the chain
                 float* dst = a.dv + ((size_t)(ch.out0 + t) * a.H + h) * D + j0;
+                // dY in bf16 as the chunk-local kernels' operand image (2 panels of
+                // 64 rows x 128 B, 128-byte swizzle; zero past the end of the sequence)
+                uint8_t* im = a.dy_img + (size_t)(ch.chunk0 + (NT - 1 - n)) * kDyImgBytes;
 #pragma unroll 1
                 for (int q16 = 0; q16 < NS / 16; ++q16) {
                     float x[16];
                     tmem_ld16(tq + L::TM_A3 + NS * s2 + 16 * q16, x);
                     tmem_wait_ld();
-                    if (t < ch.len) {
+                    const bool keep = t < ch.len;
+                    if (keep) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             *reinterpret_cast<float4*>(dst + 16 * q16 + 4 * q) =
                                 make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
                     }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x[e] = keep ? x[e] : 0.f;
+                    const int c = j0 + 16 * q16;
+                    uint8_t* row = im + (c >> 6) * 8192;
+                    st_bf16x8(row + sw128_off(r, (c & 63) >> 3), x);
+                    st_bf16x8(row + sw128_off(r, ((c & 63) >> 3) + 1), x + 8);
                 }
             }
             tc_fence_before_sync();
@@ -492,7 +508,7 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     const long long chunks = (long long)a.B * a.H * a.NT;
     if (!make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
         !make_chunk_map(&mqh, a.bc_qh, chunks, C, D, C) ||
-        !make_chunk_map(&mtt, a.bc_tt, chunks, 2 * C, C, 2 * C) ||
+        !make_chunk_map(&mtt, a.bc_tt, chunks, C, C, C) ||
         !make_chunk_map(&mu, a.bc_u, chunks, 2 * D, C, 128))
         return cudaErrorInvalidValue;
     ChainArgs t;
@@ -505,6 +521,7 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     t.dM0 = a.dM0;
     t.dss_img = a.dss_img;
     t.dv = a.dv;
+    t.dy_img = a.dy_img;
     t.status = a.status;
     t.T = a.T;
     t.H = a.H;

@@ -5,17 +5,17 @@
 // the saved Vtilde).  Per chunk, with S, M the states entering it and dS, dM
 // the adjoints of the states leaving it, the six products
 //     [dO; dY] [S | M]^T   -> P1 = dO S^T, P2 = dO M^T, P5 = dY S^T, P6 = dY M^T
-//     [Vt; 0]  [dS | dM]^T -> P3 = Vt dS^T, P4 = Vt dM^T
+//     [Vt; .]  [dS | dM]^T -> P3 = Vt dS^T, P4 = Vt dM^T  (product rows 64..127 unused)
 // are two groups of eight tcgen05.mma (M 128, N 256, K 128; bf16 operands,
 // fp32 accumulators in 512 TMEM columns).  The epilogue forms the parts of dq
 // and dk they carry,
 //     dq = Diag(alphabar) P1 - Diag(b) P2
 //     dk = Diag(Gamma_C) P3 - Diag(w) P4 - Diag(alphabar) P5 + Diag(D2) P6
 // and the row sums that feed the gate gradients, exactly as the CUDA-core
-// kernel does.  The states and adjoints arrive as bf16 images of the B
-// operands (written by the state scan and the reverse chain), two bulk
-// copies; dO, Vt and dY (fp32, rounded to bf16) are staged by the threads,
-// K-major with the 128-byte swizzle.
+// kernel does.  Every operand arrives by the copy engines, K-major with the
+// 128-byte swizzle: the states and adjoints as bf16 images of the B operands
+// (written by the state scan and the reverse chain) and dY as the reverse
+// chain's bf16 image, by bulk copies; the dO, Vt, K and Q rows by TMA.
 #include "bwd_common.cuh"
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
@@ -29,10 +29,12 @@ using namespace tc;
 constexpr int kThr = 256;
 // shared memory (byte offsets from a 1024-byte aligned base)
 constexpr uint32_t SA1 = 0;          // [dO; dY]: 2 K-panels x 128 rows x 128 B
-constexpr uint32_t SA2 = 32768;      // [Vt; 0]
+constexpr uint32_t SA2 = 32768;      // [Vt; K]: the product rows of K are not read; the
+                                     // epilogue reads K from there
 constexpr uint32_t SB1 = 65536;      // [S | M] as 256 rows: 2 K-panels x 256 rows x 128 B
 constexpr uint32_t SB2 = 131072;     // [dS | dM]
-constexpr uint32_t SSUM = 196608;    // fp32 row-sum partials [12][64], then scalars [8][3]
+constexpr uint32_t SQ = 196608;      // Q rows for the epilogue: 2 K-panels x 64 rows x 128 B
+constexpr uint32_t SSUM = SQ + 16384;  // fp32 row-sum partials [12][64], then scalars [8][3]
 constexpr uint32_t SBAR = SSUM + 3072 + 96;
 constexpr uint32_t SMISC = SBAR + 16;  // after two mbarriers (MMAs done, state images landed)
 constexpr uint32_t SMEM_BYTES = SMISC + 16 + 1024;  // + alignment slack
@@ -43,7 +45,9 @@ __device__ __forceinline__ size_t tokrow(const BwdArgs& a, int b, int t, int h) 
 }
 
 __global__ void __launch_bounds__(kThr, 1)
-bwd_state_grads_tc_kernel(BwdArgs a)
+bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_vt,
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                          BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -66,13 +70,23 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         mbar_fence_init();
-        // [S | M] entering the chunk and [dS | dM] leaving it: bf16 images of
-        // the B operands, copied in whole
-        mbar_arrive_expect_tx(&bar[1], 2 * kStateImgBytes);
+        // every operand by the copy engines: [S | M] entering the chunk and
+        // [dS | dM] leaving it (bf16 images of the B operands), dY (the reverse
+        // chain's bf16 image), and the dO, Vt, K, Q rows by TMA (rows past the
+        // end of the sequence read as zero)
+        mbar_arrive_expect_tx(&bar[1], 2 * kStateImgBytes + kDyImgBytes + 4 * 16384);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             bulk_load(sm + SB1 + p * 16384, a.ss_img + chunk * kStateImgBytes + p * 16384, 16384, &bar[1]);
             bulk_load(sm + SB2 + p * 16384, a.dss_img + chunk * kStateImgBytes + p * 16384, 16384, &bar[1]);
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_4d(sm + SA1 + p * 16384, &tm_do, p * 64, h, n * C, b, &bar[1]);
+            bulk_load(sm + SA1 + p * 16384 + 8192, a.dy_img + chunk * kDyImgBytes + p * 8192, 8192, &bar[1]);
+            tma_load_4d(sm + SA2 + p * 16384, &tm_vt, p * 64, h, n * C, b, &bar[1]);
+            tma_load_4d(sm + SA2 + p * 16384 + 8192, &tm_k, p * 64, h, n * C, b, &bar[1]);
+            tma_load_4d(sm + SQ + p * 8192, &tm_q, p * 64, h, n * C, b, &bar[1]);
         }
     }
     if (warp == 0) {
@@ -80,41 +94,6 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         tmem_relinquish();
     }
     for (int i = tid; i < 12 * C; i += kThr) part[i] = 0.f;
-    // rows 64..127 of [Vt; 0]
-    for (int i = tid; i < 1024; i += kThr) {
-        const int p = i >> 9, w = i & 511;
-        *reinterpret_cast<uint4*>(sm + SA2 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
-    }
-    // dO, Vt (bf16 copies) and dY (fp32 -> bf16), 64 rows x 16 chunks of 8
-    // each; a thread's global loads are all issued before its stores
-    {
-        constexpr int PER = C * 16 / kThr;
-        uint4 ro[PER], rv[PER];
-        float4 ry0[PER], ry1[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15, t = n * C + r;
-            ro[u] = rv[u] = make_uint4(0, 0, 0, 0);
-            ry0[u] = ry1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < a.T) {
-                const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
-                ro[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
-                rv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
-                ry0[u] = *reinterpret_cast<const float4*>(a.dv + g);
-                ry1[u] = *reinterpret_cast<const float4*>(a.dv + g + 4);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15;
-            const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
-            const float yy[8] = {ry0[u].x, ry0[u].y, ry0[u].z, ry0[u].w,
-                                 ry1[u].x, ry1[u].y, ry1[u].z, ry1[u].w};
-            *reinterpret_cast<uint4*>(sm + SA1 + off) = ro[u];
-            *reinterpret_cast<uint4*>(sm + SA1 + off + 64 * 128) = bf16x8(yy);   // rows 64..127
-            *reinterpret_cast<uint4*>(sm + SA2 + off) = rv[u];
-        }
-    }
     fence_proxy_async_smem();
     __syncthreads();
     // the chunk-end scalars' adjoints: <S, dS>, <M, dS>, <M, dM> over the
@@ -171,11 +150,9 @@ bwd_state_grads_tc_kernel(BwdArgs a)
         }
         mma_commit(&bar[0]);
     }
-    ok = __syncthreads_and(ok && mbar_wait(&bar[0], 0));
-    tc_fence_after_sync();
-
     // Epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..; warps w and w + 4 take
-    // the two halves of the 128 columns of each product.
+    // the two halves of the 128 columns of each product.  Its coefficients are
+    // loaded while the products run; K and Q come from shared memory.
     const int quad = warp & 3, half = warp >> 2;
     const int R = quad * 32 + lane;               // TMEM lane: dO rows 0..63, dY rows 64..127
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -189,8 +166,14 @@ bwd_state_grads_tc_kernel(BwdArgs a)
     const float gl = a.gamma[chunk * C * C + (C - 1) * C + r];
     const float et = in ? a.eta[tokrow(a, b, t, h)] : 0.f;
     const float w = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
-    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + grow;
-    const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + grow;
+    // row r of K (rows 64.. of the [Vt; K] tile) and of Q, 16 columns at k0
+    auto ld_row16 = [&](uint32_t tile, uint32_t panel, int row, int k0, float* x) {
+        const uint32_t o = tile + (k0 >> 6) * panel + sw128_off(row, (k0 & 63) >> 3);
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + o), x);
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + (o ^ 16)), x + 8);
+    };
+    ok = __syncthreads_and(ok && mbar_wait(&bar[0], 0));
+    tc_fence_after_sync();
     float sa = 0.f, sb = 0.f, sd2 = 0.f, sgl = 0.f, sw = 0.f;
     if (ok && R >= 64) {
         // dY rows: dk part -Diag(alphabar) P5 + Diag(D2) P6, into the exchange tile
@@ -199,14 +182,8 @@ bwd_state_grads_tc_kernel(BwdArgs a)
             float p5[16], p6[16], kv[16];
             tmem_ld16(tq + k0, p5);
             tmem_ld16(tq + 128 + k0, p6);
+            ld_row16(SA2, 16384, 64 + r, k0, kv);
             tmem_wait_ld();
-            if (in) {
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + k0), kv);
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + k0 + 8), kv + 8);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) kv[e] = 0.f;
-            }
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 sa = fmaf(-kv[e], p5[e], sa);
@@ -227,12 +204,10 @@ bwd_state_grads_tc_kernel(BwdArgs a)
             tmem_ld16(tq + 128 + k0, p2);
             tmem_ld16(tq + 256 + k0, p3);
             tmem_ld16(tq + 384 + k0, p4);
+            ld_row16(SA2, 16384, 64 + r, k0, kv);
+            ld_row16(SQ, 8192, r, k0, qh);
             tmem_wait_ld();
             if (in) {  // the TMEM loads above stay warp-uniform
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + k0), kv);
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + k0 + 8), kv + 8);
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(qg + k0), qh);
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(qg + k0 + 8), qh + 8);
                 float dq[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -310,15 +285,16 @@ constexpr uint32_t LA_QK = 0;        // [Qhat; K]  K-major, 2 K-panels x 128 row
 constexpr uint32_t LA_DY = 32768;    // [dO; dY]   K-major (stage 1)
 constexpr uint32_t LB_V = 65536;     // Vt         K-major, 2 K-panels x 64 rows x 128 B (stage 1)
 constexpr uint32_t LA_3 = 32768;     // [dOVG; dPK]          K = 64: 1 panel x 128 rows x 128 B (stage 2)
-constexpr uint32_t LA_4 = 49152;     // [dOVG^T | dPKa^T; 0] K = 128: 2 panels x 128 rows x 128 B (stage 2)
+constexpr uint32_t LA_4 = 49152;     // [dOVG^T | dPKa^T; .] K = 128: 2 panels x 128 rows x 128 B (stage 2;
+                                     // rows 64..127 unused)
 constexpr uint32_t L_X = 32768;      // fp32 alpha_r dP [64][129] (once stage 2 has completed)
 constexpr int LXS = 129;             // its row stride (floats)
 constexpr uint32_t L_GP = 81920;     // fp32 Gp, packed lower triangle
 constexpr uint32_t L_DG = L_GP + PackedLower::kFloats * 4;   // fp32 dG, packed lower triangle
 constexpr uint32_t L_VEC = L_DG + PackedLower::kFloats * 4;  // 12 x 64 floats
 constexpr uint32_t L_REC = L_VEC + 3072;  // the chunk record (kBwdRec floats)
-constexpr uint32_t L_BAR = L_REC + kBwdRec * 4;
-constexpr uint32_t L_MISC = L_BAR + 16;
+constexpr uint32_t L_BAR = L_REC + kBwdRec * 4;  // MMA stage 1, stage 2, operand copies
+constexpr uint32_t L_MISC = L_BAR + 32;
 constexpr uint32_t L_SMEM = L_MISC + 16 + 1024;
 constexpr uint32_t kLocalTmemCols = 256;
 static_assert(L_X + 64 * LXS * 4 <= L_GP, "exchange tile");
@@ -338,7 +314,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 }
 
 __global__ void __launch_bounds__(kThr, 2)
-bwd_local_grads_tc_kernel(BwdArgs a)
+bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_qh,
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_vt,
+                          BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -360,76 +338,67 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
         mbar_fence_init();
+        // operands by the copy engines, K-major with the 128-byte swizzle: dO,
+        // K and Vt rows by TMA (zero past the end of the sequence), Qhat rows
+        // (bf16, from the chain's operand kernel) by TMA, dY as the reverse
+        // chain's bf16 image
+        mbar_arrive_expect_tx(&bars[2], 4 * 16384 + kDyImgBytes);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            tma_load_4d(sm + LA_DY + p * 16384, &tm_do, p * 64, h, n * C, b, &bars[2]);
+            bulk_load(sm + LA_DY + p * 16384 + 8192, a.dy_img + chunk * kDyImgBytes + p * 8192, 8192, &bars[2]);
+            tma_load_3d(sm + LA_QK + p * 16384, &tm_qh, p * 64, 0, (int)chunk, &bars[2]);
+            tma_load_4d(sm + LA_QK + p * 16384 + 8192, &tm_k, p * 64, h, n * C, b, &bars[2]);
+            tma_load_4d(sm + LB_V + p * 8192, &tm_vt, p * 64, h, n * C, b, &bars[2]);
+        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kLocalTmemCols);
         tmem_relinquish();
     }
-    // operands: dO, dY, Qhat, K, Vt rows (bf16, K-major), and the chunk's
-    // coefficient-adjoint record.  Every global load of a thread (four row
-    // pieces, two record entries) is issued before its shared-memory stores.
+    // the chunk's coefficient-adjoint record and gate vectors (every global
+    // load of a thread before its shared-memory stores)
     {
-        constexpr int PER = C * 16 / kThr;
         static_assert(kBwdRec <= 2 * kThr, "record copy");
         const float* rec_g = a.crec_bw + chunk * kBwdRec;
         const float rc0 = rec_g[tid], rc1 = tid + kThr < kBwdRec ? rec_g[tid + kThr] : 0.f;
-        uint4 ro[PER], rq[PER], rk[PER], rv[PER];
-        float4 ry0[PER], ry1[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15, t = n * C + r;
-            ro[u] = rq[u] = rk[u] = rv[u] = make_uint4(0, 0, 0, 0);
-            ry0[u] = ry1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < a.T) {
-                const size_t g = tokrow(a, b, t, h) * D + c16 * 8;
-                ro[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
-                rq[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
-                rk[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
-                rv[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
-                ry0[u] = *reinterpret_cast<const float4*>(a.dv + g);
-                ry1[u] = *reinterpret_cast<const float4*>(a.dv + g + 4);
+        float gal = 0.f, gbe = 0.f, get = 0.f, gla = 0.f, glm = 0.f, gb = 0.f, gmu = 0.f;
+        const int tg = n * C + tid;
+        const bool gin = tid < C && tg < a.T;
+        if (tid < C) {
+            const size_t gi = gin ? tokrow(a, b, tg, h) : 0;
+            if (gin) {
+                gal = a.alpha_log[gi];
+                gbe = a.beta[gi];
+                get = a.eta[gi];
+                gmu = a.mu_log[gi];
             }
-        }
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int i = tid + kThr * u, r = i >> 4, c16 = i & 15;
-            const uint32_t off = (c16 >> 3) * 16384 + sw128_off(r, c16 & 7);
-            float q[8], k[8];
-            unpack_bf16x8(rq[u], q);
-            unpack_bf16x8(rk[u], k);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) q[e] -= a.dcorr * k[e];
-            const float y[8] = {ry0[u].x, ry0[u].y, ry0[u].z, ry0[u].w,
-                                ry1[u].x, ry1[u].y, ry1[u].z, ry1[u].w};
-            *reinterpret_cast<uint4*>(sm + LA_DY + off) = ro[u];
-            st_bf16x8(sm + LA_DY + off + 64 * 128, y);
-            st_bf16x8(sm + LA_QK + off, q);
-            *reinterpret_cast<uint4*>(sm + LA_QK + off + 64 * 128) = rk[u];
-            *reinterpret_cast<uint4*>(sm + LB_V + (c16 >> 3) * 8192 + sw128_off(r, c16 & 7)) = rv[u];
+            gla = a.la[crow + tid];
+            glm = a.lm[crow + tid];
+            gb = a.bco[crow + tid];
         }
         recs[tid] = rc0;
         if (tid + kThr < kBwdRec) recs[tid + kThr] = rc1;
+        if (tid < C) {
+            const int r = tid;
+            v.al[r] = gin ? expf(gal) : 1.f;
+            v.be[r] = gbe;
+            v.et[r] = get;
+            v.la[r] = gla;
+            v.lm[r] = glm;
+            v.b[r] = gb;
+            v.da[r] = 0.f;
+            v.de[r] = gin ? expf(gmu) : 1.f;  // mu_r, until the coefficient phase
+        }
     }
-    if (tid < C) {
-        const int r = tid, t = n * C + r;
-        const bool in = t < a.T;
-        const size_t gi = in ? tokrow(a, b, t, h) : 0;
-        v.al[r] = in ? expf(a.alpha_log[gi]) : 1.f;
-        v.be[r] = in ? a.beta[gi] : 0.f;
-        v.et[r] = in ? a.eta[gi] : 0.f;
-        v.la[r] = a.la[crow + r];
-        v.lm[r] = a.lm[crow + r];
-        v.b[r] = a.bco[crow + r];
-        v.da[r] = 0.f;
-        v.de[r] = in ? expf(a.mu_log[gi]) : 1.f;  // mu_r, until the coefficient phase
-    }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
-    __syncthreads();
+    __syncthreads();  // the barriers' initialisation and the TMEM address are visible from here
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
+    bool ok = __syncthreads_and(mbar_wait(&bars[2], 0));
+    if (tid == 0 && ok) {
         constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -465,7 +434,7 @@ bwd_local_grads_tc_kernel(BwdArgs a)
             Gp[at(r, i)] = g;
         }
     }
-    bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
+    ok = __syncthreads_and(ok && mbar_wait(&bars[0], 0));
     tc_fence_after_sync();
 
     // stage-1 epilogue: warp w reads lanes 32 (w % 4) ..; warps w, w + 4 take
@@ -475,12 +444,8 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     float dgm[32];  // dY rows: dA o (P K^T), owed to dG[r - 1][i]
     if (ok) {
-        // rows 64..127 of the second stage-2 operand are zero (over stage 1's
-        // operands, which the completed products have read)
-        for (int i = tid; i < 1024; i += kThr) {
-            const int p = i >> 9, w = i & 511;
-            *reinterpret_cast<uint4*>(sm + LA_4 + p * 16384 + 8192 + w * 16) = make_uint4(0, 0, 0, 0);
-        }
+        // (rows 64..127 of the second stage-2 operand are left as they are: the
+        // product rows they give, lanes 64..127 of the dK part, are not read)
         const float al_r = v.al[r];
 #pragma unroll
         for (int p2 = 0; p2 < 2; ++p2) {
@@ -552,15 +517,15 @@ bwd_local_grads_tc_kernel(BwdArgs a)
     if (ok && R >= 64) {
         float dar = 0.f;
         const float al_r = v.al[r];
-        const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + grow;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float dp[16], kv[16];
             tmem_ld16(tq + c0, dp);
+            // row r of K from the [Qhat; K] tile (zero past the end of the sequence)
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + LA_QK + kmaj_off(64 + r, c0, 16384)), kv);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + LA_QK + kmaj_off(64 + r, c0 + 8, 16384)), kv + 8);
             tmem_wait_ld();
             if (in) {
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + c0), kv);
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(kg + c0 + 8), kv + 8);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) dar = fmaf(dp[e], kv[e], dar);
             }
@@ -620,7 +585,10 @@ bwd_local_grads_tc_kernel(BwdArgs a)
         tmem_dealloc(tmem, kLocalTmemCols);
     }
     if (!ok) {
-        if (tid == 0) atomicOr(a.status + 1, 1u);
+        if (tid == 0) {
+            atomicOr(a.status + 1, 1u);
+            (void)mbar_wait(&bars[2], 0);  // the operand copies land before shared memory is released
+        }
         return;
     }
     bwd_coeff_phase<PackedLower>(a, recs, v, dG, Gp, recs, tid, n, b, h, true, kThr);
@@ -853,7 +821,8 @@ bwd_prep_tc_kernel(BwdArgs a)
 // ---------------------------------------------------------------------------
 // The chunk-only operands of the tensor-core reverse chain (bf16, d = 128):
 //   U  = [-K^T Diag(alphabar) T^T ; K^T Diag(D2) T^T]   bf16 [256][64]  (A of U dVtilde)
-//   TT = [T^T ; 0]                                      bf16 [128][64]  (A of T^T dVtilde = dv)
+//   T  row-major                                        bf16 [64][64]   (T^T as the MN-major A
+//                                                                        of T^T dVtilde = dv)
 //   P  = Att^T dO     fp32, slice-major [D/32][64][32]  (dVtilde's chain-free part)
 //   Qhat rows (bf16 [64][128]) and Diag(alphabar) dO, -Diag(b) dO by 32-column
 //   slice (bf16, the reverse chain's shared-memory image of its B operands)
@@ -864,12 +833,15 @@ bwd_prep_tc_kernel(BwdArgs a)
 // (A operands K-major, transposed while they are staged):
 //   U = K^T [Diag(-alphabar) T^T | Diag(D2) T^T]                M 128, N 64 + 64
 //   P = Att^T dO                                                 M 64 (of 128), N 128
-//   D = K^T [Diag(Gamma_C) Vtilde | Diag(w) Vtilde]             M 128, N 128 + 128 (second round)
+//   D = K^T [Diag(Gamma_C) Vtilde | Diag(w) Vtilde]             M 128, N 128 + 128 (second round,
+//                                                                over the first round's columns)
 // E = Qhat^T Diag(alphabar) dO and F = Qhat^T Diag(b) dO are formed in the
 // reverse chain itself (by the MMA lane while it waits for each chunk's
-// dVtilde), from Qhat and the scaled dO slices written here.
+// dVtilde), from Qhat and the scaled dO slices written here.  Two CTAs share
+// an SM (256 TMEM columns, about 100 KB of shared memory each).
 constexpr uint32_t PA_KT = 0;        // K^T     [128 i][64 r]  K-major, 16 KB
-constexpr uint32_t PA_AT = 16384;    // Att^T   [128 r (64 used)][64 r2]
+constexpr uint32_t PA_AT = 16384;    // Att^T   [128 r][64 r2]: rows 64..127 are left as they are
+                                     // (the product rows they give are not read)
 constexpr uint32_t PB_O = 32768;     // dO      [64 r][128 j]  MN-major: 2 N-panels x 64 rows
 constexpr uint32_t PB_VG = 49152;    // Diag(Gamma_C) Vtilde
 constexpr uint32_t PB_VW = 65536;    // Diag(w) Vtilde
@@ -879,6 +851,7 @@ constexpr uint32_t P_VEC = 98304;    // alphabar, b, D2, Gamma_C, w
 constexpr uint32_t P_BAR = P_VEC + 1280;
 constexpr uint32_t P_MISC = P_BAR + 16;
 constexpr uint32_t P_SMEM = P_MISC + 16 + 1024;
+static_assert(2 * (P_SMEM + 1024) <= 233472, "two CTAs per SM");
 
 // byte offset of element (row, col) of an MN-major tile with 64-element
 // column panels of `rows` rows (128-byte swizzle)
@@ -886,7 +859,7 @@ __device__ __forceinline__ uint32_t mn_off(int row, int col, int rows) {
     return (col >> 6) * rows * 128 + sw128_off(row, (col & 63) >> 3) + (col & 7) * 2;
 }
 
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThr, 2)
 bwd_chain_prep_tc_kernel(BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -913,7 +886,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         mbar_fence_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
     if (tid < C) {
@@ -937,45 +910,46 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             rec[3 * C + 2] = expf(a.lm[crow + C - 1]);
         }
     }
-    // rows 64..127 of Att^T are zero
-    for (int i = tid; i < 512; i += kThr)
-        *reinterpret_cast<uint4*>(sm + PA_AT + 8192 + i * 16) = make_uint4(0, 0, 0, 0);
     __syncthreads();
-    // token tiles: 64 rows x 16 groups of 8; the loads of a thread before its stores
+    // token tiles: 64 rows x 16 groups of 8; the loads of a thread (kept as
+    // packed bf16) before its stores
     {
         constexpr int U8 = C * 16 / kThr;  // 4
-        float kx[U8][8], qx[U8][8], ox[U8][8], vx[U8][8];
+        uint4 kx[U8], qx[U8], ox[U8], vx[U8];
 #pragma unroll
         for (int u = 0; u < U8; ++u) {
             const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8, t = n * C + r;
+            kx[u] = qx[u] = ox[u] = vx[u] = make_uint4(0, 0, 0, 0);
             if (t < a.T) {
                 const size_t g = tokrow(a, b, t, h) * D + c8;
-                ld8<__nv_bfloat16>(a.k, g, kx[u]);
-                ld8<__nv_bfloat16>(a.q, g, qx[u]);
-                ld8<__nv_bfloat16>(a.dout, g, ox[u]);
-                ld8<__nv_bfloat16>(a.vt, g, vx[u]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) kx[u][e] = qx[u][e] = ox[u][e] = vx[u][e] = 0.f;
+                kx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
+                qx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
+                ox[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
+                vx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
             }
         }
 #pragma unroll
         for (int u = 0; u < U8; ++u) {
             const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8;
             const float ab = v_ab[r], bb = v_b[r], gl = v_g[r], w = v_w[r];
+            float kf[8], qf[8], of[8], vf[8];
+            unpack_bf16x8(kx[u], kf);
+            unpack_bf16x8(qx[u], qf);
+            unpack_bf16x8(ox[u], of);
+            unpack_bf16x8(vx[u], vf);
             float qh[8], oa[8], ob[8], vg[8], vw[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                qh[e] = qx[u][e] - a.dcorr * kx[u][e];
+                qh[e] = qf[e] - a.dcorr * kf[e];
                 // transposed into the K-major A operand
-                st_bf16(sm + PA_KT + kmaj_off(c8 + e, r, 16384), kx[u][e]);
-                oa[e] = ab * ox[u][e];
-                ob[e] = -bb * ox[u][e];
-                vg[e] = gl * vx[u][e];
-                vw[e] = w * vx[u][e];
+                st_bf16(sm + PA_KT + kmaj_off(c8 + e, r, 16384), kf[e]);
+                oa[e] = ab * of[e];
+                ob[e] = -bb * of[e];
+                vg[e] = gl * vf[e];
+                vw[e] = w * vf[e];
             }
             const uint32_t o = mn_off(r, c8, 64);
-            st_bf16x8(sm + PB_O + o, ox[u]);
+            *reinterpret_cast<uint4*>(sm + PB_O + o) = ox[u];
             st_bf16x8(sm + PB_VG + o, vg);
             st_bf16x8(sm + PB_VW + o, vw);
             // Qhat rows, and the reverse chain's E / F operands Diag(alphabar) dO and
@@ -986,7 +960,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             *reinterpret_cast<uint4*>(eo + 4096) = bf16x8(ob);
         }
     }
-    // T and Att: the scaled T tiles (K-major), Att^T (K-major), and [T^T; 0] to global
+    // T and Att: the scaled T tiles (K-major), Att^T (K-major), and T (bf16,
+    // row-major) to global
     {
         constexpr int U4 = C * C / 4 / kThr;  // 4
         float4 tx[U4], ax[U4];
@@ -996,7 +971,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             tx[u] = *reinterpret_cast<const float4*>(a.tmat + chunk * C * C + idx);
             ax[u] = *reinterpret_cast<const float4*>(a.att + chunk * C * C + idx);
         }
-        __nv_bfloat16* TT = a.bc_tt + chunk * 128 * 64;
+        __nv_bfloat16* Tg = a.bc_tt + chunk * C * C;
 #pragma unroll
         for (int u = 0; u < U4; ++u) {
             const int idx = (tid + kThr * u) * 4, r = idx / C, r2 = idx % C;
@@ -1007,10 +982,14 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
                 st_bf16(sm + PB_TS + kmaj_off(r, r2 + e, 8192), -v_ab[r2 + e] * tv[e]);
                 st_bf16(sm + PB_TM + kmaj_off(r, r2 + e, 8192), v_d2[r2 + e] * tv[e]);
                 st_bf16(sm + PA_AT + kmaj_off(r2 + e, r, 16384), av[e]);  // Att^T[r2 + e][r]
-                TT[(r2 + e) * 64 + r] = __float2bfloat16_rn(tv[e]);       // T^T
             }
+            const __nv_bfloat162 t01 = __floats2bfloat162_rn(tv[0], tv[1]);
+            const __nv_bfloat162 t23 = __floats2bfloat162_rn(tv[2], tv[3]);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&t01);
+            pk.y = *reinterpret_cast<const uint32_t*>(&t23);
+            *reinterpret_cast<uint2*>(Tg + idx) = pk;
         }
-        for (int i = tid; i < 64 * 64; i += kThr) TT[64 * 64 + i] = __float2bfloat16_rn(0.f);
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
@@ -1024,9 +1003,9 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         for (int ks = 0; ks < 4; ++ks) {
             const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
             const uint64_t aa = smem_desc(sbase + PA_AT + ks * 32, 16, 1024, kSw128);
-            mma_bf16(tmem + 256, ak, smem_desc(sbase + PB_TS + ks * 32, 16, 1024, kSw128), idk, ks > 0);
-            mma_bf16(tmem + 320, ak, smem_desc(sbase + PB_TM + ks * 32, 16, 1024, kSw128), idk, ks > 0);
-            mma_bf16(tmem + 384, aa, smem_desc(sbase + PB_O + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
+            mma_bf16(tmem, ak, smem_desc(sbase + PB_TS + ks * 32, 16, 1024, kSw128), idk, ks > 0);
+            mma_bf16(tmem + 64, ak, smem_desc(sbase + PB_TM + ks * 32, 16, 1024, kSw128), idk, ks > 0);
+            mma_bf16(tmem + 128, aa, smem_desc(sbase + PB_O + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
         }
         mma_commit(&bars[0]);
     }
@@ -1038,14 +1017,14 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     if (ok) {
         // U: row i = R of the S half (half 0) or of the M half (half 1)
         {
-            float u32[32];
             uint4* Uo = reinterpret_cast<uint4*>(a.bc_u + chunk * 256 * 64 + (size_t)(128 * half + R) * 64);
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                tmem_ld32(tq + 256 + 64 * half + 32 * g, u32);
+            for (int g = 0; g < 4; ++g) {
+                float u16[16];
+                tmem_ld16(tq + 64 * half + 16 * g, u16);
                 tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 4; ++q) Uo[4 * g + q] = bf16x8(u32 + 8 * q);
+                Uo[2 * g] = bf16x8(u16);
+                Uo[2 * g + 1] = bf16x8(u16 + 8);
             }
         }
         // P = Att^T dO: rows r = R < 64, columns [64 half, 64 half + 64), by 32-column slice
@@ -1054,7 +1033,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 #pragma unroll 1
             for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
                 float p16[16];
-                tmem_ld16(tq + 384 + k0, p16);
+                tmem_ld16(tq + 128 + k0, p16);
                 tmem_wait_ld();
                 const int sl = k0 >> 5, jj = k0 & 31;
 #pragma unroll
@@ -1064,7 +1043,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             }
         }  // (R < 64 is warp-uniform: quadrants 0, 1)
     }
-    // second round: the rebuild increments into TMEM columns 0..255 (unused in the first)
+    // second round: the rebuild increments, over the first round's columns
+    // (every TMEM read above has completed: tmem_wait_ld, then the barrier)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -1102,7 +1082,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, 256);
     }
     if (!ok && tid == 0) atomicOr(a.status + 1, 1u);
 }
@@ -1110,9 +1090,11 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 // The states entering every chunk by the elementwise recurrence
 // S <- alphabar_C S - b_C M + D_S, M <- mubar_C M - D_M, in fp32 registers;
 // each chunk's entering pair is stored as the bf16 image the state products
-// copy in (state_img_off).  A thread owns 8 columns of one row of a head's
-// S and M; a warp takes 32 consecutive rows, so its loads of the increments
-// (chain order) are 512 contiguous bytes.
+// copy in (state_img_off).  A thread owns 8 columns of one row of a head's S
+// and M; eight consecutive lanes take the eight 16-byte pieces of one row of
+// a 64-column panel, so a warp's stores fill four whole 128-byte lines (its
+// loads of the increments, in chain order, are eight runs of 64 bytes).  Each
+// thread keeps the next two chunks' increments in flight.
 __global__ void __launch_bounds__(256)
 bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0,
                       const float* __restrict__ dinc, const float* __restrict__ rec,
@@ -1122,36 +1104,48 @@ bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0
     constexpr int per = D * (D / 8);
     if (gid >= heads * per) return;
     const long long bh = gid / per;
-    const int rem = (int)(gid % per), g = rem / D, i = rem % D;
+    const int rem = (int)(gid % per), i = (rem & 1023) >> 3, g = (rem >> 10) * 8 + (rem & 7);
     float s[8], m[8];
     const size_t r0 = (size_t)bh * D * D + (size_t)i * D + 8 * g;  // S0, M0 are row-major
 #pragma unroll
     for (int h4 = 0; h4 < 2; ++h4) {
-        const float4 a = S0 ? *reinterpret_cast<const float4*>(S0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 b = M0 ? *reinterpret_cast<const float4*>(M0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        s[4 * h4] = a.x; s[4 * h4 + 1] = a.y; s[4 * h4 + 2] = a.z; s[4 * h4 + 3] = a.w;
-        m[4 * h4] = b.x; m[4 * h4 + 1] = b.y; m[4 * h4 + 2] = b.z; m[4 * h4 + 3] = b.w;
+        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 y = M0 ? *reinterpret_cast<const float4*>(M0 + r0 + 4 * h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[4 * h4] = x.x; s[4 * h4 + 1] = x.y; s[4 * h4 + 2] = x.z; s[4 * h4 + 3] = x.w;
+        m[4 * h4] = y.x; m[4 * h4 + 1] = y.y; m[4 * h4 + 2] = y.z; m[4 * h4 + 3] = y.w;
     }
     const int o0 = chain_off(i, 8 * g), o1 = chain_off(i, 8 * g + 4);
     const uint32_t ps = state_img_off(i, g), pm = state_img_off(i + D, g);
+    struct Step { float4 ds0, ds1, dm0, dm1; float aC, bC, mC; };
+    auto load = [&](int nn) {
+        Step st;
+        if (nn < NT) {
+            const size_t chunk = (size_t)bh * NT + nn;
+            const float* dn = dinc + chunk * 2 * D * D;
+            st.ds0 = __ldg(reinterpret_cast<const float4*>(dn + o0));
+            st.ds1 = __ldg(reinterpret_cast<const float4*>(dn + o1));
+            st.dm0 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o0));
+            st.dm1 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o1));
+            st.aC = __ldg(rec + chunk * 256 + 3 * C);
+            st.bC = __ldg(rec + chunk * 256 + 3 * C + 1);
+            st.mC = __ldg(rec + chunk * 256 + 3 * C + 2);
+        }
+        return st;
+    };
+    Step n1 = load(0), n2 = load(1);
     for (int nn = 0; nn < NT; ++nn) {
-        const size_t chunk = (size_t)bh * NT + nn;
-        const float* dn = dinc + chunk * 2 * D * D;
-        const float4 ds0 = __ldg(reinterpret_cast<const float4*>(dn + o0));
-        const float4 ds1 = __ldg(reinterpret_cast<const float4*>(dn + o1));
-        const float4 dm0 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o0));
-        const float4 dm1 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o1));
-        const float aC = __ldg(rec + chunk * 256 + 3 * C), bC = __ldg(rec + chunk * 256 + 3 * C + 1);
-        const float mC = __ldg(rec + chunk * 256 + 3 * C + 2);
-        uint8_t* im = img + chunk * kStateImgBytes;
+        const Step cu = n1;
+        n1 = n2;
+        n2 = load(nn + 2);
+        uint8_t* im = img + ((size_t)bh * NT + nn) * kStateImgBytes;
         *reinterpret_cast<uint4*>(im + ps) = bf16x8(s);
         *reinterpret_cast<uint4*>(im + pm) = bf16x8(m);
-        const float dsv[8] = {ds0.x, ds0.y, ds0.z, ds0.w, ds1.x, ds1.y, ds1.z, ds1.w};
-        const float dmv[8] = {dm0.x, dm0.y, dm0.z, dm0.w, dm1.x, dm1.y, dm1.z, dm1.w};
+        const float dsv[8] = {cu.ds0.x, cu.ds0.y, cu.ds0.z, cu.ds0.w, cu.ds1.x, cu.ds1.y, cu.ds1.z, cu.ds1.w};
+        const float dmv[8] = {cu.dm0.x, cu.dm0.y, cu.dm0.z, cu.dm0.w, cu.dm1.x, cu.dm1.y, cu.dm1.z, cu.dm1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float sn = fmaf(aC, s[e], fmaf(-bC, m[e], dsv[e]));
-            m[e] = fmaf(mC, m[e], -dmv[e]);
+            const float sn = fmaf(cu.aC, s[e], fmaf(-cu.bC, m[e], dsv[e]));
+            m[e] = fmaf(cu.mC, m[e], -dmv[e]);
             s[e] = sn;
         }
     }
@@ -1168,8 +1162,14 @@ cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    CUtensorMap mdo, mvt, mk, mq;
+    if (!make_token_map(&mdo, a.dout, a.B, a.T, a.H, 64, true) ||
+        !make_token_map(&mvt, a.vt, a.B, a.T, a.H, 64, true) ||
+        !make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
+        !make_token_map(&mq, a.q, a.B, a.T, a.H, 64, true))
+        return cudaErrorInvalidValue;
     ProfScope ps(kBwdStateGrads, s);
-    bwd_state_grads_tc_kernel<<<(unsigned)chunks, kThr, SMEM_BYTES, s>>>(a);
+    bwd_state_grads_tc_kernel<<<(unsigned)chunks, kThr, SMEM_BYTES, s>>>(mdo, mvt, mk, mq, a);
     return cudaGetLastError();
 }
 
@@ -1188,8 +1188,14 @@ cudaError_t launch_bwd_local_grads_tc(const BwdArgs& a, cudaStream_t s)
         e = cudaFuncSetAttribute(bwd_local_grads_tc_kernel,
                                  cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
+    CUtensorMap mdo, mqh, mk, mvt;
+    if (!make_token_map(&mdo, a.dout, a.B, a.T, a.H, 64, true) ||
+        !make_chunk_map(&mqh, a.bc_qh, chunks, C, D, C) ||
+        !make_token_map(&mk, a.k, a.B, a.T, a.H, 64, true) ||
+        !make_token_map(&mvt, a.vt, a.B, a.T, a.H, 64, true))
+        return cudaErrorInvalidValue;
     ProfScope ps(kBwdLocal, s);
-    bwd_local_grads_tc_kernel<<<(unsigned)chunks, kThr, L_SMEM, s>>>(a);
+    bwd_local_grads_tc_kernel<<<(unsigned)chunks, kThr, L_SMEM, s>>>(mdo, mqh, mk, mvt, a);
     return cudaGetLastError();
 }
 
@@ -1216,6 +1222,9 @@ cudaError_t launch_bwd_chain_prep_tc(const BwdArgs& a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(bwd_chain_prep_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)P_SMEM);
+    if (e == cudaSuccess)  // two CTAs per SM need the larger carve-out
+        e = cudaFuncSetAttribute(bwd_chain_prep_tc_kernel,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     {
         ProfScope ps(kBwdChainPrep, s);

@@ -331,7 +331,7 @@ namespace {
 
 struct BwdLayout {
     size_t status, la, lm, lc, bco, gamma, att, tmat, SS, dSS, rec;
-    size_t bc_u, bc_tt, bc_p, bc_qh, bc_eo, bc_rec, bc_d;  // tensor-core path (bf16, d = 128)
+    size_t bc_u, bc_tt, bc_p, bc_qh, bc_eo, bc_rec, bc_d, dy;  // tensor-core path (bf16, d = 128)
     size_t total;
 };
 
@@ -355,15 +355,16 @@ BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
     w.SS = off;    off += align_up(chunks * state_bytes);
     w.dSS = off;   off += align_up(chunks * state_bytes);
     w.rec = off;   off += align_up(chunks * kBwdRec * sizeof(float));
-    w.bc_u = w.bc_tt = w.bc_p = w.bc_qh = w.bc_eo = w.bc_rec = w.bc_d = 0;
+    w.bc_u = w.bc_tt = w.bc_p = w.bc_qh = w.bc_eo = w.bc_rec = w.bc_d = w.dy = 0;
     if (tc) {
         w.bc_u = off;   off += align_up(chunks * 256 * 64 * 2);
-        w.bc_tt = off;  off += align_up(chunks * 128 * 64 * 2);
+        w.bc_tt = off;  off += align_up(chunks * 64 * 64 * 2);
         w.bc_p = off;   off += align_up(chunks * kChunk * D * sizeof(float));
         w.bc_qh = off;  off += align_up(chunks * kChunk * D * 2);
         w.bc_eo = off;  off += align_up(chunks * (D / 32) * 2 * 4096);
         w.bc_rec = off; off += align_up(chunks * 256 * sizeof(float));
         w.bc_d = off;   off += align_up(chunks * 2 * D * D * sizeof(float));
+        w.dy = off;     off += align_up(chunks * kDyImgBytes);
     }
     w.total = off;
     return w;
@@ -448,6 +449,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.bc_eo = tc ? reinterpret_cast<uint8_t*>(ws + w.bc_eo) : nullptr;
     a.bc_rec = tc ? reinterpret_cast<float*>(ws + w.bc_rec) : nullptr;
     a.bc_d = tc ? reinterpret_cast<float*>(ws + w.bc_d) : nullptr;
+    a.dy_img = tc ? reinterpret_cast<uint8_t*>(ws + w.dy) : nullptr;
     a.dq = dq; a.dk = dk_out; a.dv = dv_out;
     a.dalpha_log = dalpha_log; a.dmu_log = dmu_log; a.dbeta = dbeta; a.deta = deta;
     a.dS0 = dS0; a.dM0 = dM0;

@@ -173,6 +173,10 @@ constexpr uint32_t kStateImgBytes = 2u * 128u * 128u * 2u;
 __device__ __forceinline__ uint32_t state_img_off(int row, int g) {
     return (uint32_t)(g >> 3) * 32768u + (uint32_t)row * 128u + ((uint32_t)((g ^ row) & 7) << 4);
 }
+// The 64 x 128 bf16 rows of one chunk (d = 128) as a K-major operand image:
+// two 64-column panels of 64 rows x 128 B, 128-byte swizzle (row r, columns
+// 8g .. 8g + 7 at (g >> 3) * 8192 + sw128 offset of (r, g & 7)).
+constexpr uint32_t kDyImgBytes = 2u * 64u * 128u;
 struct BwdArgs {
     const void* q;
     const void* k;
@@ -205,10 +209,11 @@ struct BwdArgs {
     // the state products' B operand (see state_img_off)
     uint8_t* ss_img;   // [B*H*NT][kStateImgBytes]
     uint8_t* dss_img;  // [B*H*NT][kStateImgBytes]
+    uint8_t* dy_img;   // [B*H*NT][kDyImgBytes]  dv of each chunk in bf16 (tensor-core path)
     float* crec_bw;  // [B*H*NT, kBwdRec]  coefficient adjoints from the state products
     // chunk-only operands of the tensor-core reverse chain (null on the CUDA-core path)
     __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]
-    __nv_bfloat16* bc_tt;  // [B*H*NT, 128, 64]  [T^T; 0]
+    __nv_bfloat16* bc_tt;  // [B*H*NT, 64, 64]  T, row-major (the MN-major form of T^T)
     float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
     __nv_bfloat16* bc_qh;  // [B*H*NT, C, D]  Qhat = Q - d K (bf16, rows of the chunk)
     uint8_t* bc_eo;        // [B*H*NT, D/32, 2, 4096 B]  Diag(alphabar) dO and -Diag(b) dO by

@@ -9,6 +9,8 @@ CASE      chunk      mdn_chunk_fwd over the workload's batch (both chunk kernels
                      (B=256, H=16, d=128: S and M are 2 x 268 MB, far above L2)
           gate_prep  mdn_chunk_gate_prep (la, lm, lc, b and Gamma) on the workload's gates
           gates      mdn_gate_params on the workload's pre-activations
+          bwd        mdn_chunk_bwd over the batch, from the forward pass's vtilde and a
+                     seeded cotangent of o (every backward kernel)
 WORKLOAD  index or name of a synthetic workload (default 2, the 1.3B-layer shape)
 REPS      calls (default 3)
 
@@ -53,8 +55,15 @@ def main(argv) -> None:
         inp = mi.make_inputs(spec)
         dev = mi.to_torch(inp, "cuda")
         pre = [torch.from_numpy(p).cuda() for p in (inp.x_eta, inp.a_pre, inp.b_pre, inp.c_pre)]
+        if case == "bwd":
+            o, vt, _, _ = api.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates),
+                                        inp.d_corr)
+            do = torch.randn(o.shape, generator=torch.Generator().manual_seed(3)).to(o)
         for _ in range(reps):
-            if case == "chunk":
+            if case == "bwd":
+                api.chunk_bwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), inp.d_corr,
+                              vt, do)
+            elif case == "chunk":
                 api.chunk_fwd(dev["q"], dev["k"], dev["v"], *(dev[g] for g in gates), inp.d_corr,
                               dev["S0"], dev["M0"])
             elif case == "preact":
