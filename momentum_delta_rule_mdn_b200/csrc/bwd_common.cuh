@@ -106,12 +106,22 @@ struct PackedLower {
 // state products (rec_g, in global memory; rec: kBwdRec floats of shared
 // scratch), v.da holding the direct adjoint of alpha from P.  Writes the four
 // gate gradients of the chunk's tokens.
-template <class Idx = PaddedLower>
+// A phase timer that does nothing (the default of the coefficient phase's
+// optional per-phase timer; diagnostic builds pass one that records cycles).
+struct NoPhaseTimer {
+    __device__ __forceinline__ void lap(int) {}
+};
+
+template <class Idx = PaddedLower, class Timer = NoPhaseTimer>
 __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* rec_g,
                                                 const BwdVec& v, float* dG, const float* Gp,
                                                 float* rec, int tid, int n, int b, int h,
-                                                bool rec_loaded = false, int nthreads = 256)
+                                                bool rec_loaded = false, int nthreads = 256,
+                                                Timer* timer = nullptr)
 {
+    auto lap = [&](int k) {
+        if (timer) timer->lap(k);
+    };
     constexpr int C = kChunk;
     const Idx at;
     // the chunk's record in shared memory (rec: kBwdRec floats), so that the
@@ -156,6 +166,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_dbe[r] = 0.f;
     }
     __syncthreads();
+    lap(0);
     if (tid < 32) {
         // warp 0, positions j = 2 lane, 2 lane + 1
         const int j0 = 2 * tid, j1 = j0 + 1;
@@ -197,6 +208,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         if (tid == 31) v_dlm[C - 1] += s + rec[5 * C + 2] * expf(v_lm[C - 1]);  // mubar_C M
     }
     __syncthreads();
+    lap(1);
     // Gamma = eta o Gp: row sums of dG o Gamma (threads 0..63), column sums
     // and eta's share (threads 64..127)
     if (tid < C) {
@@ -216,16 +228,25 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_de[x] += ce;
     }
     __syncthreads();
-    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place, one column per thread
+    lap(2);
+    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place, one column per
+    // thread (the next row's operands are read before this row's store)
     if (tid < C) {
         const int i = tid;
         float R = 0.f;
+        float dg_n = dG[at(C - 1, i)], al_n = 0.f;  // al_n: alpha_{j+1} (none past the chunk)
         for (int j = C - 1; j >= i; --j) {
-            R = dG[at(j, i)] + (j + 1 < C ? v_al[j + 1] * R : 0.f);
+            const float dg = dg_n, al = al_n;
+            if (j > i) {
+                dg_n = dG[at(j - 1, i)];
+                al_n = v_al[j];
+            }
+            R = dg + (j + 1 < C ? al * R : 0.f);
             dG[at(j, i)] = R;
         }
     }
     __syncthreads();
+    lap(3);
     // U_j = sum_{i<=j} eta_i exp(lm_j - lm_i) R_{j,i}
     if (tid < C) {
         const int j = tid;
@@ -236,6 +257,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_dlm[j] += v_be[j] * U;
     }
     __syncthreads();
+    lap(4);
     if (tid < 32) {
         // reverse cumulative sums (la, lm are inclusive prefix sums of the log
         // gates): a warp suffix scan, two positions per lane
@@ -259,6 +281,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
         v_dlm[j1] = xm1 + nm;
     }
     __syncthreads();
+    lap(5);
     if (tid < C) {
         const int j = tid, t = n * C + j;
         if (t < a.T) {
@@ -269,6 +292,7 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
             a.deta[gi] = v_de[j];
         }
     }
+    lap(6);
 }
 
 }  // namespace mdn

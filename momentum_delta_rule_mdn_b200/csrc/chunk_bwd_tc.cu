@@ -39,10 +39,53 @@ constexpr uint32_t SBAR = SSUM + 3072 + 96;
 constexpr uint32_t SMISC = SBAR + 16;  // after two mbarriers (MMAs done, state images landed)
 constexpr uint32_t SMEM_BYTES = SMISC + 16 + 1024;  // + alignment slack
 constexpr int XS = 129;              // row stride (floats) of the dk exchange tile over SA1
+constexpr int kRowS = 132;           // row stride (floats) of the dq / dk staging tiles: rows
+                                     // 16-byte aligned, float4 accesses of 8 rows conflict-free
+static_assert(2 * 64 * kRowS * 4 <= SQ - SB1, "dq / dk staging tiles over the state images");
 
 __device__ __forceinline__ size_t tokrow(const BwdArgs& a, int b, int t, int h) {
     return ((size_t)b * a.T + t) * a.H + h;
 }
+
+// Per-phase cycle counts of the per-chunk kernels, as seen by thread 0 of
+// every CTA and summed over CTAs (slot kBwdClkCtas of each kernel's block
+// counts them).  Diagnostic builds only (MDN_PHASE_CLOCKS, with the buffer set
+// by mdn_diag_bwd_clock); otherwise every call is empty.
+constexpr int kBwdClkSlots = 32, kBwdClkCtas = 31;
+#ifdef MDN_PHASE_CLOCKS
+__device__ float* g_bwd_clk = nullptr;
+struct BwdClock {
+    long long t;
+    float acc[kBwdClkSlots];
+    bool on;
+    __device__ __forceinline__ void start(bool o) {
+        on = o;
+#pragma unroll
+        for (int k = 0; k < kBwdClkSlots; ++k) acc[k] = 0.f;
+        t = clock_now();
+    }
+    __device__ __forceinline__ void lap(int k) {
+        if (on) {
+            const long long now = clock_now();
+            acc[k] += (float)(now - t);
+            t = now;
+        }
+    }
+    __device__ __forceinline__ void flush(int block) {
+        float* out = g_bwd_clk;
+        if (!on || !out) return;
+        out += block * kBwdClkSlots;
+        for (int k = 0; k < kBwdClkCtas; ++k) atomicAdd(out + k, acc[k]);
+        atomicAdd(out + kBwdClkCtas, 1.f);
+    }
+};
+#else
+struct BwdClock {
+    __device__ __forceinline__ void start(bool) {}
+    __device__ __forceinline__ void lap(int) {}
+    __device__ __forceinline__ void flush(int) {}
+};
+#endif
 
 __global__ void __launch_bounds__(kThr, 1)
 bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_vt,
@@ -65,6 +108,8 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     float* wsum = part + 12 * C;                             // [8 warps][3]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SBAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SMISC);
+    BwdClock clk;
+    clk.start(tid == 0);
 
     if (tid == 0) {
         mbar_init(&bar[0], 1);
@@ -96,6 +141,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     for (int i = tid; i < 12 * C; i += kThr) part[i] = 0.f;
     fence_proxy_async_smem();
     __syncthreads();
+    clk.lap(0);
     // the chunk-end scalars' adjoints: <S, dS>, <M, dS>, <M, dM> over the
     // bf16 states the products use (a warp reads 32 consecutive rows of one
     // 8-column group: conflict-free under the swizzle)
@@ -132,6 +178,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     tc_fence_before_sync();
     ok = __syncthreads_and(ok);
     tc_fence_after_sync();
+    clk.lap(1);
     const uint32_t tmem = *tmem_slot;
 
     if (tid == 0 && ok) {
@@ -157,6 +204,10 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     const int R = quad * 32 + lane;               // TMEM lane: dO rows 0..63, dY rows 64..127
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     float* X = reinterpret_cast<float*>(sm + SA1);  // dk of the dY rows, [64][XS], over the operands
+    // rows of dq and dk staged for bulk stores (row stride kRowS floats), over
+    // the state images
+    float* QT = reinterpret_cast<float*>(sm + SB1);
+    float* KT = QT + C * kRowS;
     const int r = R & 63, t = n * C + r;
     const bool in = t < a.T;
     const size_t grow = in ? tokrow(a, b, t, h) * D : 0;
@@ -174,6 +225,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     };
     ok = __syncthreads_and(ok && mbar_wait(&bar[0], 0));
     tc_fence_after_sync();
+    clk.lap(2);
     float sa = 0.f, sb = 0.f, sd2 = 0.f, sgl = 0.f, sw = 0.f;
     if (ok && R >= 64) {
         // dY rows: dk part -Diag(alphabar) P5 + Diag(D2) P6, into the exchange tile
@@ -196,6 +248,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         }
     }
     __syncthreads();
+    clk.lap(3);
     if (ok && R < 64) {
 #pragma unroll 1
         for (int k0 = half * 64; k0 < half * 64 + 64; k0 += 16) {
@@ -217,13 +270,15 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
                     sgl = fmaf(kv[e], p3[e], sgl);
                     sw = fmaf(-kv[e], p4[e], sw);
                     dq[e] = fmaf(abar, p1[e], -bco * p2[e]);
-                    dk[e] = fmaf(gl, p3[e], -w * p4[e]) + X[r * XS + k0 + e];
+                    // dk carries -d dq (Qhat = Q - d K) for this part of dq; the
+                    // chunk-local kernel adds its parts of both
+                    dk[e] = fmaf(-a.dcorr, dq[e], fmaf(gl, p3[e], -w * p4[e]) + X[r * XS + k0 + e]);
                 }
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    *reinterpret_cast<float4*>(a.dq + grow + k0 + 4 * e4) =
+                    *reinterpret_cast<float4*>(QT + r * kRowS + k0 + 4 * e4) =
                         make_float4(dq[4 * e4], dq[4 * e4 + 1], dq[4 * e4 + 2], dq[4 * e4 + 3]);
-                    *reinterpret_cast<float4*>(a.dk + grow + k0 + 4 * e4) =
+                    *reinterpret_cast<float4*>(KT + r * kRowS + k0 + 4 * e4) =
                         make_float4(dk[4 * e4], dk[4 * e4 + 1], dk[4 * e4 + 2], dk[4 * e4 + 3]);
                 }
             }
@@ -241,9 +296,18 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
             part[(6 + half) * C + r] = sd2;
         }
     }
+    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
+    // one 512-byte bulk store per row of dq and of dk
+    if (ok && tid < 2 * C && n * C + (tid & (C - 1)) < a.T) {
+        const int row = tid & (C - 1);
+        const size_t g = tokrow(a, b, n * C + row, h) * D;
+        bulk_store((tid < C ? a.dq : a.dk) + g, (tid < C ? QT : KT) + row * kRowS, D * 4);
+        bulk_commit_group();
+    }
     float* rec = a.crec_bw + chunk * kBwdRec;
+    clk.lap(4);
     if (tid < C) {
         const float* p0 = part + tid;
         rec[tid] = (p0[0] + p0[C]) + (p0[2 * C] + p0[3 * C]);
@@ -261,10 +325,13 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         atomicOr(a.status + 1, 1u);
         (void)mbar_wait(&bar[1], 0);  // the state copies land before shared memory is released
     }
+    bulk_wait_group_read<0>();  // the row stores have read their staging tiles
     if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
+    clk.lap(5);
+    clk.flush(0);
 }
 
 // ---------------------------------------------------------------------------
@@ -287,8 +354,10 @@ constexpr uint32_t LB_V = 65536;     // Vt         K-major, 2 K-panels x 64 rows
 constexpr uint32_t LA_3 = 32768;     // [dOVG; dPK]          K = 64: 1 panel x 128 rows x 128 B (stage 2)
 constexpr uint32_t LA_4 = 49152;     // [dOVG^T | dPKa^T; .] K = 128: 2 panels x 128 rows x 128 B (stage 2;
                                      // rows 64..127 unused)
-constexpr uint32_t L_X = 32768;      // fp32 alpha_r dP [64][129] (once stage 2 has completed)
-constexpr int LXS = 129;             // its row stride (floats)
+constexpr uint32_t L_Q = 0;          // fp32 dq part [64][LXS] (once stage 2 has completed)
+constexpr uint32_t L_X = 33792;      // fp32 alpha_r dP [64][LXS], then the dk part in place
+constexpr int LXS = 132;             // their row stride (floats): rows 16-byte aligned for the
+                                     // bulk reductions, float4 accesses of 8 rows conflict-free
 constexpr uint32_t L_GP = 81920;     // fp32 Gp, packed lower triangle
 constexpr uint32_t L_DG = L_GP + PackedLower::kFloats * 4;   // fp32 dG, packed lower triangle
 constexpr uint32_t L_VEC = L_DG + PackedLower::kFloats * 4;  // 12 x 64 floats
@@ -297,7 +366,7 @@ constexpr uint32_t L_BAR = L_REC + kBwdRec * 4;  // MMA stage 1, stage 2, operan
 constexpr uint32_t L_MISC = L_BAR + 32;
 constexpr uint32_t L_SMEM = L_MISC + 16 + 1024;
 constexpr uint32_t kLocalTmemCols = 256;
-static_assert(L_X + 64 * LXS * 4 <= L_GP, "exchange tile");
+static_assert(L_Q + 64 * LXS * 4 <= L_X && L_X + 64 * LXS * 4 <= L_GP, "staging tiles");
 static_assert(LA_4 + 32768 <= L_GP && LB_V + 16384 <= L_GP, "operand map");
 static_assert(2 * (L_SMEM + 1024) <= 233472, "two CTAs per SM");
 
@@ -309,8 +378,10 @@ __device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
 __device__ __forceinline__ uint32_t kmaj_off(int row, int k, uint32_t panel_bytes) {
     return (k >> 6) * panel_bytes + sw128_off(row, (k & 63) >> 3) + (k & 7) * 2;
 }
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+// p[0..3] += (x, y, z, w) in L2, no value returned (16-byte aligned p)
+__device__ __forceinline__ void red_add_v4(float* p, float x, float y, float z, float w) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(x), "f"(y), "f"(z), "f"(w)
+                 : "memory");
 }
 
 __global__ void __launch_bounds__(kThr, 2)
@@ -334,6 +405,8 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     const BwdVec v = bwd_vec(reinterpret_cast<float*>(sm + L_VEC));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L_MISC);
+    BwdClock clk;
+    clk.start(tid == 0);
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -397,7 +470,9 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     __syncthreads();  // the barriers' initialisation and the TMEM address are visible from here
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    clk.lap(0);
     bool ok = __syncthreads_and(mbar_wait(&bars[2], 0));
+    clk.lap(1);
     if (tid == 0 && ok) {
         constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
 #pragma unroll
@@ -411,31 +486,36 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         }
         mma_commit(&bars[0]);
     }
-    // the rows of dq and dk that the last epilogue reads back (written by the
-    // state products), pulled into L2 meanwhile: 64 rows x 2 x 512 B
-    {
-        const int r = tid >> 2, t = n * C + r;
-        if (t < a.T) {
-            const size_t g = tokrow(a, b, t, h) * D + (tid & 3) * 32;
-            prefetch_l2(a.dq + g);
-            prefetch_l2(a.dk + g);
-        }
-    }
     // Gamma without eta, by its column recurrence (overlaps the products):
     // Gp_{r,i} = alpha_r Gp_{r-1,i} + beta_r mubar_r / mubar_i, the ratio as a
     // running product of mu (held in v.de until the coefficient phase)
+    // (the next row's alpha, beta, mu are read before this row's store, so that
+    // the shared-memory latency overlaps the recurrence)
     if (tid < C) {
         const int i = tid;
         float g = v.be[i], f = 1.f;
         Gp[at(i, i)] = g;
+        float al_n = 0.f, be_n = 0.f, de_n = 1.f;
+        if (i + 1 < C) {
+            al_n = v.al[i + 1];
+            be_n = v.be[i + 1];
+            de_n = v.de[i + 1];
+        }
         for (int r = i + 1; r < C; ++r) {
-            f *= v.de[r];
-            g = fmaf(v.al[r], g, v.be[r] * f);
+            const float al_r = al_n, be_r = be_n, de_r = de_n;
+            if (r + 1 < C) {
+                al_n = v.al[r + 1];
+                be_n = v.be[r + 1];
+                de_n = v.de[r + 1];
+            }
+            f *= de_r;
+            g = fmaf(al_r, g, be_r * f);
             Gp[at(r, i)] = g;
         }
     }
     ok = __syncthreads_and(ok && mbar_wait(&bars[0], 0));
     tc_fence_after_sync();
+    clk.lap(2);
 
     // stage-1 epilogue: warp w reads lanes 32 (w % 4) ..; warps w, w + 4 take
     // columns i in [32 half, 32 half + 32), 16 at a time
@@ -447,6 +527,15 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         // (rows 64..127 of the second stage-2 operand are left as they are: the
         // product rows they give, lanes 64..127 of the dK part, are not read)
         const float al_r = v.al[r];
+        // Gamma's row (r, resp. r - 1 on the dY rows) over this thread's
+        // columns, read before any store of the epilogue
+        const int gr = R < 64 ? r : r - 1;
+        float gam[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int i = 32 * half + e;
+            gam[e] = i <= gr ? v.et[i] * Gp[at(gr, i)] : 0.f;
+        }
 #pragma unroll
         for (int p2 = 0; p2 < 2; ++p2) {
             float x1[16], x2[16];
@@ -456,10 +545,11 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = 32 * half + 16 * p2 + e;
+                const float g = gam[16 * p2 + e];
                 if (R < 64) {
                     float ovg = 0.f;
                     if (i <= r) {
-                        ovg = x1[e] * (v.et[i] * Gp[at(r, i)]);
+                        ovg = x1[e] * g;
                         dG[at(r, i)] = x1[e] * x2[e];
                     }
                     st_bf16(sm + LA_3 + kmaj_off(r, i, 16384), ovg);             // row r of [dOVG; .]
@@ -467,7 +557,7 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
                 } else {
                     float pk = 0.f, dm = 0.f;
                     if (i < r) {
-                        pk = -x1[e] * v.et[i] * Gp[at(r - 1, i)];
+                        pk = -x1[e] * g;
                         dm = -x1[e] * al_r * x2[e];
                     }
                     dgm[16 * p2 + e] = dm;
@@ -481,11 +571,18 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (ok && R >= 64) {
+    clk.lap(3);
+    if (ok && R >= 64) {  // one writer per entry; every read before the first write
+        float cur[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int i = 32 * half + e;
-            if (i < r) dG[at(r - 1, i)] += dgm[e];  // one writer per entry
+            cur[e] = i < r ? dG[at(r - 1, i)] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int i = 32 * half + e;
+            if (i < r) dG[at(r - 1, i)] = cur[e] + dgm[e];
         }
     }
     if (tid == 0 && ok) {
@@ -507,6 +604,7 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     if (tid < C) dG[at(C - 1, tid)] += recs[3 * C + tid];  // Gamma_{C,i} in the state update
     ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
     tc_fence_after_sync();
+    clk.lap(4);
 
     // stage-2 epilogue: lanes 64..127 hold dP = dPK K; lanes 0..63 the dQhat
     // and dK parts; warps w, w + 4 take feature columns [64 half, 64 half + 64)
@@ -530,60 +628,54 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
                 for (int e = 0; e < 16; ++e) dar = fmaf(dp[e], kv[e], dar);
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) X[r * LXS + c0 + e] = al_r * dp[e];
+            for (int e4 = 0; e4 < 4; ++e4)
+                *reinterpret_cast<float4*>(X + r * LXS + c0 + 4 * e4) =
+                    make_float4(al_r * dp[4 * e4], al_r * dp[4 * e4 + 1], al_r * dp[4 * e4 + 2],
+                                al_r * dp[4 * e4 + 3]);
         }
         atomicAdd(v.da + r, dar);  // two addends onto 0: the same sum in either order
     }
     __syncthreads();
+    clk.lap(5);
     if (ok && R < 64) {
-        float* __restrict__ dqr = a.dq + grow;
-        float* __restrict__ dkr = a.dk + grow;
+        // this kernel's parts of dq and dk, staged by rows (dk over the row of
+        // X it has read) and added to the state products' by bulk reductions
+        float* QL = reinterpret_cast<float*>(sm + L_Q);
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+            float dqb[16], dkb[16];
+            tmem_ld16(tq + c0, dqb);
+            tmem_ld16(tq + 128 + c0, dkb);
+            float4 xr[4];
 #pragma unroll
-        for (int j2 = 0; j2 < 4; j2 += 2) {  // two 16-column groups per round
-            float4 q4[2][4], k4[2][4];
-            if (in) {
+            for (int e4 = 0; e4 < 4; ++e4) xr[e4] = *reinterpret_cast<const float4*>(X + r * LXS + c0 + 4 * e4);
+            tmem_wait_ld();
 #pragma unroll
-                for (int g = 0; g < 2; ++g)
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {  // every load of the round before any store
-                        const int c = 64 * half + 16 * (j2 + g) + 4 * e4;
-                        q4[g][e4] = *reinterpret_cast<const float4*>(dqr + c);
-                        k4[g][e4] = *reinterpret_cast<const float4*>(dkr + c);
-                    }
-            }
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                const int c0 = 64 * half + 16 * (j2 + g);
-                float dqb[16], dkb[16], xr[16];
-                tmem_ld16(tq + c0, dqb);
-                tmem_ld16(tq + 128 + c0, dkb);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) xr[e] = X[r * LXS + c0 + e];
-                tmem_wait_ld();
-                if (in) {
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float qo[4] = {q4[g][e4].x, q4[g][e4].y, q4[g][e4].z, q4[g][e4].w};
-                        const float ko[4] = {k4[g][e4].x, k4[g][e4].y, k4[g][e4].z, k4[g][e4].w};
-                        float qn[4], kn[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            qn[e] = qo[e] + dqb[4 * e4 + e];
-                            kn[e] = ko[e] + dkb[4 * e4 + e] + xr[4 * e4 + e] - a.dcorr * qn[e];
-                        }
-                        *reinterpret_cast<float4*>(dqr + c0 + 4 * e4) = make_float4(qn[0], qn[1], qn[2], qn[3]);
-                        *reinterpret_cast<float4*>(dkr + c0 + 4 * e4) = make_float4(kn[0], kn[1], kn[2], kn[3]);
-                    }
-                }
+            for (int e4 = 0; e4 < 4; ++e4) {
+                const float* q4 = dqb + 4 * e4;
+                const float* k4 = dkb + 4 * e4;
+                *reinterpret_cast<float4*>(QL + r * LXS + c0 + 4 * e4) = make_float4(q4[0], q4[1], q4[2], q4[3]);
+                *reinterpret_cast<float4*>(X + r * LXS + c0 + 4 * e4) =
+                    make_float4(k4[0] + xr[e4].x - a.dcorr * q4[0], k4[1] + xr[e4].y - a.dcorr * q4[1],
+                                k4[2] + xr[e4].z - a.dcorr * q4[2], k4[3] + xr[e4].w - a.dcorr * q4[3]);
             }
         }
     }
+    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, kLocalTmemCols);
     }
+    // one 512-byte bulk reduction per row of dq and of dk (one addition per element)
+    if (ok && tid < 2 * C && n * C + (tid & (C - 1)) < a.T) {
+        const int row = tid & (C - 1);
+        const size_t g = tokrow(a, b, n * C + row, h) * D;
+        bulk_reduce_add_f32((tid < C ? a.dq : a.dk) + g, sm + (tid < C ? L_Q : L_X) + row * LXS * 4, D * 4);
+        bulk_commit_group();
+    }
+    clk.lap(6);
     if (!ok) {
         if (tid == 0) {
             atomicOr(a.status + 1, 1u);
@@ -591,7 +683,13 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         }
         return;
     }
-    bwd_coeff_phase<PackedLower>(a, recs, v, dG, Gp, recs, tid, n, b, h, true, kThr);
+    struct Sub {  // the coefficient phase's laps in slots 7 ..
+        BwdClock* c;
+        __device__ __forceinline__ void lap(int k) { c->lap(7 + k); }
+    } sub{&clk};
+    bwd_coeff_phase<PackedLower>(a, recs, v, dG, Gp, recs, tid, n, b, h, true, kThr, &sub);
+    bulk_wait_group_read<0>();  // the row reductions have read their staging tiles
+    clk.flush(1);
 }
 
 // ---------------------------------------------------------------------------
@@ -829,8 +927,8 @@ bwd_prep_tc_kernel(BwdArgs a)
 //   record: Gamma_{C,r} (64), w_r (64), then alphabar_C, b_C, mubar_C at 192..194
 // plus the increments of the state rebuild, D_S = K^T Diag(Gamma_C) Vtilde and
 // D_M = K^T Diag(w) Vtilde, which turn the rebuild into an elementwise scan
-// over the chunks.  Products
-// (A operands K-major, transposed while they are staged):
+// over the chunks.  Products (K^T and Att^T are the MN-major forms of K's and
+// Att's rows, so nothing is transposed on the way into shared memory):
 //   U = K^T [Diag(-alphabar) T^T | Diag(D2) T^T]                M 128, N 64 + 64
 //   P = Att^T dO                                                 M 64 (of 128), N 128
 //   D = K^T [Diag(Gamma_C) Vtilde | Diag(w) Vtilde]             M 128, N 128 + 128 (second round,
@@ -839,9 +937,10 @@ bwd_prep_tc_kernel(BwdArgs a)
 // reverse chain itself (by the MMA lane while it waits for each chunk's
 // dVtilde), from Qhat and the scaled dO slices written here.  Two CTAs share
 // an SM (256 TMEM columns, about 100 KB of shared memory each).
-constexpr uint32_t PA_KT = 0;        // K^T     [128 i][64 r]  K-major, 16 KB
-constexpr uint32_t PA_AT = 16384;    // Att^T   [128 r][64 r2]: rows 64..127 are left as they are
-                                     // (the product rows they give are not read)
+constexpr uint32_t PA_KT = 0;        // K^T as an MN-major A: K's rows [64 r][128 i], 2 M-panels
+                                     // of 64 rows x 128 B, 16 KB
+constexpr uint32_t PA_AT = 16384;    // Att^T as an MN-major A: Att's rows [64 r][64 i] (M-panel 0;
+                                     // the product rows of panel 1 are not read)
 constexpr uint32_t PB_O = 32768;     // dO      [64 r][128 j]  MN-major: 2 N-panels x 64 rows
 constexpr uint32_t PB_VG = 49152;    // Diag(Gamma_C) Vtilde
 constexpr uint32_t PB_VW = 65536;    // Diag(w) Vtilde
@@ -879,6 +978,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + P_MISC);
     float* rec = a.bc_rec + chunk * 256;
+    BwdClock clk;
+    clk.start(tid == 0);
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -889,45 +990,61 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
+    // one round of global loads: this position's gate values (threads < C)
+    // and the token tiles (64 rows x 16 groups of 8, kept as packed bf16)
+    constexpr int U8 = C * 16 / kThr;  // 4
+    uint4 kx[U8], qx[U8], ox[U8], vx[U8];
+    float g_la = 0.f, g_al = 0.f, g_gl = 0.f, g_et = 0.f, g_lm = 0.f, g_b = 0.f, g_bp = 0.f;
+    float g_laC = 0.f, g_lmC = 0.f;
+    const bool gin = tid < C && n * C + tid < a.T;
     if (tid < C) {
-        const int r = tid, t = n * C + r;
-        const bool in = t < a.T;
-        const float ab = expf(a.la[crow + r]);
-        const float al = in ? expf(a.alpha_log[tokrow(a, b, t, h)]) : 1.f;
-        const float gl = a.gamma[chunk * C * C + (C - 1) * C + r];
-        const float et = in ? a.eta[tokrow(a, b, t, h)] : 0.f;
-        const float w = et * expf(a.lm[crow + C - 1] - a.lm[crow + r]);
-        v_ab[r] = ab;
-        v_b[r] = a.bco[crow + r];
-        v_d2[r] = r > 0 ? a.bco[crow + r - 1] * al : 0.f;
-        v_g[r] = gl;
+        const int r = tid;
+        g_la = a.la[crow + r];
+        if (gin) {
+            g_al = a.alpha_log[tokrow(a, b, n * C + r, h)];
+            g_et = a.eta[tokrow(a, b, n * C + r, h)];
+        }
+        g_gl = a.gamma[chunk * C * C + (C - 1) * C + r];
+        g_lm = a.lm[crow + r];
+        g_lmC = a.lm[crow + C - 1];
+        g_laC = a.la[crow + C - 1];
+        g_b = a.bco[crow + r];
+        g_bp = r > 0 ? a.bco[crow + r - 1] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U8; ++u) {
+        const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8, t = n * C + r;
+        kx[u] = qx[u] = ox[u] = vx[u] = make_uint4(0, 0, 0, 0);
+        if (t < a.T) {
+            const size_t g = tokrow(a, b, t, h) * D + c8;
+            kx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
+            qx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
+            ox[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
+            vx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
+        }
+    }
+    if (tid < C) {
+        const int r = tid;
+        const float al = gin ? expf(g_al) : 1.f;
+        const float w = g_et * expf(g_lmC - g_lm);
+        v_ab[r] = expf(g_la);
+        v_b[r] = g_b;
+        v_d2[r] = r > 0 ? g_bp * al : 0.f;
+        v_g[r] = g_gl;
         v_w[r] = w;
-        rec[r] = gl;
+        rec[r] = g_gl;
         rec[C + r] = w;
         if (r == 0) {
-            rec[3 * C] = expf(a.la[crow + C - 1]);
+            rec[3 * C] = expf(g_laC);
             rec[3 * C + 1] = a.bco[crow + C - 1];
-            rec[3 * C + 2] = expf(a.lm[crow + C - 1]);
+            rec[3 * C + 2] = expf(g_lmC);
         }
     }
     __syncthreads();
-    // token tiles: 64 rows x 16 groups of 8; the loads of a thread (kept as
-    // packed bf16) before its stores
+    clk.lap(0);
+    // the token tiles into shared memory (nothing transposed) and the chain's
+    // per-chunk copies to global memory
     {
-        constexpr int U8 = C * 16 / kThr;  // 4
-        uint4 kx[U8], qx[U8], ox[U8], vx[U8];
-#pragma unroll
-        for (int u = 0; u < U8; ++u) {
-            const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8, t = n * C + r;
-            kx[u] = qx[u] = ox[u] = vx[u] = make_uint4(0, 0, 0, 0);
-            if (t < a.T) {
-                const size_t g = tokrow(a, b, t, h) * D + c8;
-                kx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + g);
-                qx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + g);
-                ox[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + g);
-                vx[u] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.vt) + g);
-            }
-        }
 #pragma unroll
         for (int u = 0; u < U8; ++u) {
             const int i = tid + kThr * u, r = i >> 4, c8 = (i & 15) * 8;
@@ -941,14 +1058,13 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 qh[e] = qf[e] - a.dcorr * kf[e];
-                // transposed into the K-major A operand
-                st_bf16(sm + PA_KT + kmaj_off(c8 + e, r, 16384), kf[e]);
                 oa[e] = ab * of[e];
                 ob[e] = -bb * of[e];
                 vg[e] = gl * vf[e];
                 vw[e] = w * vf[e];
             }
             const uint32_t o = mn_off(r, c8, 64);
+            *reinterpret_cast<uint4*>(sm + PA_KT + o) = kx[u];
             *reinterpret_cast<uint4*>(sm + PB_O + o) = ox[u];
             st_bf16x8(sm + PB_VG + o, vg);
             st_bf16x8(sm + PB_VW + o, vw);
@@ -977,18 +1093,17 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             const int idx = (tid + kThr * u) * 4, r = idx / C, r2 = idx % C;
             const float tv[4] = {tx[u].x, tx[u].y, tx[u].z, tx[u].w};
             const float av[4] = {ax[u].x, ax[u].y, ax[u].z, ax[u].w};
+            float ts[4], tm[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                st_bf16(sm + PB_TS + kmaj_off(r, r2 + e, 8192), -v_ab[r2 + e] * tv[e]);
-                st_bf16(sm + PB_TM + kmaj_off(r, r2 + e, 8192), v_d2[r2 + e] * tv[e]);
-                st_bf16(sm + PA_AT + kmaj_off(r2 + e, r, 16384), av[e]);  // Att^T[r2 + e][r]
+                ts[e] = -v_ab[r2 + e] * tv[e];
+                tm[e] = v_d2[r2 + e] * tv[e];
             }
-            const __nv_bfloat162 t01 = __floats2bfloat162_rn(tv[0], tv[1]);
-            const __nv_bfloat162 t23 = __floats2bfloat162_rn(tv[2], tv[3]);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&t01);
-            pk.y = *reinterpret_cast<const uint32_t*>(&t23);
-            *reinterpret_cast<uint2*>(Tg + idx) = pk;
+            // four consecutive elements of row r: 8 bytes in each tile
+            *reinterpret_cast<uint2*>(sm + PB_TS + kmaj_off(r, r2, 8192)) = bf16x4(ts);
+            *reinterpret_cast<uint2*>(sm + PB_TM + kmaj_off(r, r2, 8192)) = bf16x4(tm);
+            *reinterpret_cast<uint2*>(sm + PA_AT + kmaj_off(r, r2, 8192)) = bf16x4(av);
+            *reinterpret_cast<uint2*>(Tg + idx) = bf16x4(tv);
         }
     }
     fence_proxy_async_smem();
@@ -996,13 +1111,14 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    clk.lap(1);
     if (tid == 0) {
-        constexpr uint32_t idmn = idesc_bf16(128, 128, false, true);
-        constexpr uint32_t idk = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t idmn = idesc_bf16(128, 128, true, true);   // A, B MN-major
+        constexpr uint32_t idk = idesc_bf16(128, 64, true, false);    // A MN-major, B K-major
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
-            const uint64_t aa = smem_desc(sbase + PA_AT + ks * 32, 16, 1024, kSw128);
+            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 2048, 8192, 1024, kSw128);
+            const uint64_t aa = smem_desc(sbase + PA_AT + ks * 2048, 8192, 1024, kSw128);
             mma_bf16(tmem, ak, smem_desc(sbase + PB_TS + ks * 32, 16, 1024, kSw128), idk, ks > 0);
             mma_bf16(tmem + 64, ak, smem_desc(sbase + PB_TM + ks * 32, 16, 1024, kSw128), idk, ks > 0);
             mma_bf16(tmem + 128, aa, smem_desc(sbase + PB_O + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
@@ -1011,6 +1127,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     }
     bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
     tc_fence_after_sync();
+    clk.lap(2);
     const int quad = warp & 3, half = warp >> 2;
     const int R = quad * 32 + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -1049,10 +1166,10 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     __syncthreads();
     tc_fence_after_sync();
     if (tid == 0 && ok) {
-        constexpr uint32_t idmn = idesc_bf16(128, 128, false, true);
+        constexpr uint32_t idmn = idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 32, 16, 1024, kSw128);
+            const uint64_t ak = smem_desc(sbase + PA_KT + ks * 2048, 8192, 1024, kSw128);
             mma_bf16(tmem, ak, smem_desc(sbase + PB_VG + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
             mma_bf16(tmem + 128, ak, smem_desc(sbase + PB_VW + ks * 2048, 8192, 1024, kSw128), idmn, ks > 0);
         }
@@ -1060,6 +1177,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     }
     ok = __syncthreads_and(ok && mbar_wait(&bars[1], 0));
     tc_fence_after_sync();
+    clk.lap(3);
     if (ok) {
         float* Do = a.bc_d + (chunk * 2) * D * D;  // chain order
 #pragma unroll 1
@@ -1084,6 +1202,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         tc_fence_after_sync();
         tmem_dealloc(tmem, 256);
     }
+    clk.lap(4);
+    clk.flush(2);
     if (!ok && tid == 0) atomicOr(a.status + 1, 1u);
 }
 
@@ -1153,6 +1273,15 @@ bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0
 
 }  // namespace
 
+
+#ifdef MDN_PHASE_CLOCKS
+// Diagnostic builds: where the per-phase cycle sums go (3 x kBwdClkSlots
+// floats: state products, local products, chain operands), or null.
+extern "C" int mdn_diag_bwd_clock(float* p)
+{
+    return cudaMemcpyToSymbol(g_bwd_clk, &p, sizeof(p)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
 {

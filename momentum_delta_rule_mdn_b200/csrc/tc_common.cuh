@@ -25,6 +25,10 @@ __device__ __forceinline__ uint4 bf16x8(const float* x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                       pack_bf16(x[6], x[7]));
 }
+// Four floats as four bf16 (round to nearest even), packed for an 8-byte store.
+__device__ __forceinline__ uint2 bf16x4(const float* x) {
+    return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+}
 __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* x) {
     *reinterpret_cast<uint4*>(p) = bf16x8(x);
 }
