@@ -69,6 +69,28 @@ def pass_work(spec: mi.Spec):
     return th * (5 * d * elt + 16) + states, th * (12.0 * C * d + 12.0 * d * d)
 
 
+def bwd_work(spec: mi.Spec, with_state_cot: bool = False):
+    """The backward pass's algorithmic work per token-head, from its chunkwise
+    form (per chunk of C tokens, d_k = d_v = d):
+      C^2 d products: K K^T and Qhat K^T (T and Att rebuilt), Att^T dO, T^T dVtilde,
+        dO Vt^T, dY Vt^T, Qhat K^T, K K^T (the chunk-local adjoints), [dOVG; dPK] K
+        and [dOVG^T | dPKa^T] [Qhat; K]: 28 C^2 d flops
+      C d^2 products: U = K^T [.. T^T] (counted as 4 C^2 d above), D = K^T [Gamma Vt |
+        w Vt], K [dS | dM], U dVtilde, E and F, and the six state products dO S^T,
+        dO M^T, dY S^T, dY M^T, Vt dS^T, Vt dM^T: 28 C d^2 flops
+    so 28 C d + 28 d^2 flops per token-head (2.33 times the forward's); bytes =
+    q, k, vtilde, d_o read in the input dtype and four fp32 gates read, dq, dk,
+    dv and four gate gradients written in fp32; per head, dS0 and dM0 written
+    and S0, M0 (and dS_T, dM_T when given) read in fp32.  Returns (bytes, flops)."""
+    th = spec.B * spec.T * spec.H
+    d, C = spec.d, spec.C
+    elt = 2 if spec.dtype == "bf16" else 4
+    heads = spec.B * spec.H
+    n_state = 2 + (2 if spec.state_std > 0 else 0) + (2 if with_state_cot else 0)
+    return (th * (4 * d * elt + 16 + 3 * d * 4 + 16) + heads * n_state * d * d * 4,
+            th * (28.0 * C * d + 28.0 * d * d))
+
+
 def token_bytes(spec: mi.Spec) -> int:
     """One decode token for every head: S and M read and written (fp32), q, k,
     v read, o written, four gates."""
@@ -520,8 +542,15 @@ def run_backward(args, mdn, device, spec0):
     torch.cuda.synchronize()
     kern = mdn.profile_read(reset=True)
     mdn.profile_enable(False)
+    nbytes, flops = bwd_work(spec0)
+    hbm, bf16, src = load_peaks()
+    roof = {"bound": "latency (serial per-chunk phases; see the kernel times)",
+            "work": {"bytes": nbytes, "flops": flops,
+                     "per_token_head": {"bytes": int(nbytes // (B * T * H)), "flops": 28 * spec0.C * d + 28 * d * d}},
+            **fractions(nbytes, flops, ms * 1e-3, hbm, bf16),
+            "peak": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": src}}
     return {"workload": spec0.name, "ms": round(ms, 4), "tokens_per_s": round(B * T / (ms * 1e-3), 1),
-            "calls": n,
+            "calls": n, "roofline": roof,
             "path": ("tcgen05 (bf16, d = 128), fp32 accumulation" if o.dtype == torch.bfloat16 and d == 128
                      else "fp32 CUDA cores"),
             "kernels_ms": {k: round(v[0] / v[1], 4) for k, v in kern.items()}}
