@@ -16,8 +16,9 @@
 //     A2 = U dVtilde                     (two M 128, N NS, K 64)
 //     dS, dM <- (alphabar_C dS + E, -b_C dS + mubar_C dM - F) + A2   (epilogue)
 //   with E = Qhat^T Diag(alphabar) dO and -F = Qhat^T (-Diag(b) dO) issued into
-//   A2's accumulators right after A1 (M 128, N NS, K 64, A MN-major from the
-//   Qhat rows of the [K; Qhat] tile), while the chain warps form dVtilde
+//   A2's accumulators right after A1 (one product of M 128, N 2 NS, K 64, A
+//   MN-major from the Qhat rows of the [K; Qhat] tile), while the chain warps
+//   form dVtilde
 //     A3 = T^T dVtilde = dY              (M 128 with rows 64..127 unused, N NS, K 64;
 //                                         off the chain; T^T MN-major from T's rows)
 // This is the shape of the forward pass's inter-chunk kernel, whose warp
@@ -118,6 +119,18 @@ struct ChainArgs {
 
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
 
+// Per-phase cycle sums of CTA 0's MMA lane (slots 0..19), TMA lane (20..39)
+// and first chain warp (40..59), in diagnostic builds (MDN_PHASE_CLOCKS, the
+// buffer set by mdn_diag_chain_clock); null otherwise.
+#ifdef MDN_PHASE_CLOCKS
+__device__ float* g_chain_clk = nullptr;
+__device__ __forceinline__ float* chain_clk(int slot) {
+    return (blockIdx.x == 0 && g_chain_clk) ? g_chain_clk + slot : nullptr;
+}
+#else
+__device__ __forceinline__ float* chain_clk(int) { return nullptr; }
+#endif
+
 // Wait for the phase of `bar` with this parity.  Gives up when another role
 // has raised the abort flag, or after ~1 s (then raises it itself).
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -216,7 +229,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         // ------------------------------------------------------------ MMA issue
         if (lid == 0) {
             PhaseClock clk;
-            clk.start(nullptr);
+            clk.start(chain_clk(0));
             const uint64_t d_kq0 = smem_desc(sbase + L::KQ0, 16, 1024, kSw128);
             // B of A1: [S | M], N = 2 NS; for NS = 64 the S and M halves are two 128-byte panels
             const uint64_t d_st = smem_desc(sbase + L::ST, NS == 32 ? 8192 : 16384, 1024, kSw128);
@@ -252,22 +265,18 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                     if (!wait_bar(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
                     const uint32_t qh = sbase + L::KQ0 + s2 * 32768 + 8192;
                     const uint32_t eo = sbase + L::E0 + sv * L::E_BYTES;
+                    // one product of N = 2 NS: B = [Diag(alphabar) dO | -Diag(b) dO] (the two
+                    // 32-column MN atoms 4096 B apart), D = the [dS | dM] accumulators
+                    constexpr uint32_t idef2 = idesc_bf16(128, 2 * NS, true, true);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t aq = smem_desc(qh + ks * 2048, 16384, 1024, kSw128);
-                        mma_bf16(tmem + L::TM_A2, aq, smem_desc(eo + ks * 1024, 4096, 512, kSw64), idef, ks > 0);
-                        mma_bf16(tmem + L::TM_A2 + NS, aq, smem_desc(eo + 4096 + ks * 1024, 4096, 512, kSw64),
-                                 idef, ks > 0);
+                        mma_bf16(tmem + L::TM_A2, aq, smem_desc(eo + ks * 1024, 4096, 512, kSw64), idef2, ks > 0);
                     }
                     mma_commit(&bars[B_MQ + s2]);  // the last reads of this [K; Qhat] slot
                 }
                 clk.lap(2);
                 if (!wait_bar(&bars[B_FFB + s2], (n >> 1) & 1, abort_flag)) break;
-                if (n + 1 < NT) {
-                    const int t2 = (n + 1) & 1;
-                    if (!wait_bar(&bars[B_FKQ + t2], ((n + 1) >> 1) & 1, abort_flag)) break;
-                    if (n >= 1 && !wait_bar(&bars[B_OD + t2], ((n - 1) >> 1) & 1, abort_flag)) break;
-                }
                 clk.lap(3);
                 if (!wait_bar(&bars[B_YR], n & 1, abort_flag)) break;
                 clk.lap(4);
@@ -290,6 +299,15 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                              d_y + ks * ystep, idef, ks > 0);
                 mma_commit(&bars[B_M3 + s2]);
                 clk.lap(6);
+                // K, Qhat of chunk n + 1 and the A1 / A3 slot it reuses (read by the
+                // output warps of chunk n - 1), waited for while the chain warps
+                // form the state of chunk n + 1
+                if (n + 1 < NT) {
+                    const int t2 = (n + 1) & 1;
+                    if (!wait_bar(&bars[B_FKQ + t2], ((n + 1) >> 1) & 1, abort_flag)) break;
+                    if (n >= 1 && !wait_bar(&bars[B_OD + t2], ((n - 1) >> 1) & 1, abort_flag)) break;
+                }
+                clk.lap(7);
             }
             clk.flush();
             // every issued MMA has completed before TMEM and shared memory are released
@@ -301,7 +319,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         // ------------------------------------------------------------ TMA loads
         if (lid == 0) {
             PhaseClock clk;
-            clk.start(nullptr);
+            clk.start(chain_clk(20));
             int issued_kq = 0, issued_fb = 0, issued_vc = 0;
             for (int n = 0; n < NT; ++n) {
                 const int s2 = n & 1, sv = n % L::NVC;
@@ -319,19 +337,13 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                     tma_load_3d(dst + 8192, &tm_qh, p * 64, 0, (int)chunk, fb);
                 }
                 issued_kq = n + 1;
-                if (n >= 2 && !wait_bar(&bars[B_M3 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
-                clk.lap(1);
-                fb = &bars[B_FFB + s2];
-                mbar_arrive_expect_tx(fb, kTxFB);
-                uint8_t* dst = sm + L::FB0 + s2 * L::FB_BYTES;
-                tma_load_3d(dst, &tm_tat, 0, 0, (int)chunk, fb);
-                tma_load_3d(dst + 16384, &tm_a2t, 0, 0, (int)chunk, fb);
-                tma_load_3d(dst + 32768, &tm_a2t, 0, 128, (int)chunk, fb);
-                issued_fb = n + 1;
+                // the chunk's slices of Att^T dO, of the scaled dO and its
+                // coefficients first: the chain warps need them before anything
+                // else of the chunk, and their slot frees before the T / U slot
                 if (n >= L::NVC &&
                     !wait_bar(&bars[B_EVC + sv], ((n / L::NVC) - 1) & 1, abort_flag))
                     break;
-                clk.lap(2);
+                clk.lap(1);
                 fb = &bars[B_FVC + sv];
                 mbar_arrive_expect_tx(fb, L::kTxVC);
                 bulk_load(sm + L::V0 + sv * L::V_BYTES, a.pp + (chunk * (D / NS) + slice) * 64 * NS,
@@ -340,6 +352,15 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                           L::E_BYTES, fb);
                 bulk_load(sm + L::CR0 + sv * 1024, a.crec + chunk * 256, 1024, fb);
                 issued_vc = n + 1;
+                if (n >= 2 && !wait_bar(&bars[B_M3 + s2], ((n - 2) >> 1) & 1, abort_flag)) break;
+                clk.lap(2);
+                fb = &bars[B_FFB + s2];
+                mbar_arrive_expect_tx(fb, kTxFB);
+                uint8_t* dst = sm + L::FB0 + s2 * L::FB_BYTES;
+                tma_load_3d(dst, &tm_tat, 0, 0, (int)chunk, fb);
+                tma_load_3d(dst + 16384, &tm_a2t, 0, 0, (int)chunk, fb);
+                tma_load_3d(dst + 32768, &tm_a2t, 0, 128, (int)chunk, fb);
+                issued_fb = n + 1;
             }
             clk.flush();
             // Copies that were issued must land before shared memory is
@@ -358,21 +379,10 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         const bool ypart = quad < 2;  // lanes 0..63: rows of K, so this warp forms Y
         const int r = lane & 63;
         PhaseClock clk;
-        clk.start(nullptr);
+        clk.start(warp == kChainWarp0 + 2 && lid == 0 ? chain_clk(40) : nullptr);
         for (int n = 0; n < NT; ++n) {
             const int s2 = n & 1, sv = n % L::NVC;
             const long long chunk = ch.chunk0 + (NT - 1 - n);
-            // the adjoints of the states leaving this chunk, kept (bf16, as
-            // the state products' operand image) for the chunk-local gradients
-            {
-                uint8_t* dst = a.dss_img + (size_t)chunk * kStateImgBytes;
-#pragma unroll
-                for (int c = 0; c < NH / 8; ++c) {
-                    const int g = (j0 + NH * hc) / 8 + c;
-                    st_bf16x8(dst + state_img_off(lane, g), s + 8 * c);
-                    st_bf16x8(dst + state_img_off(lane + D, g), m + 8 * c);
-                }
-            }
             if (!warp_wait(&bars[B_FVC + sv], (n / L::NVC) & 1, abort_flag)) break;
             clk.lap(0);
             const float* cr = reinterpret_cast<const float*>(sm + L::CR0 + sv * 1024);
@@ -404,6 +414,20 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 if (lid == 0) mbar_arrive(&bars[B_YR]);
                 clk.lap(3);
             }
+            // the adjoints of the states leaving this chunk, kept (bf16, as the
+            // state products' operand image) for the chunk-local gradients;
+            // stored once Y is on its way (the stores' issue stalls would
+            // otherwise delay Y)
+            {
+                uint8_t* dst = a.dss_img + (size_t)chunk * kStateImgBytes;
+#pragma unroll
+                for (int c = 0; c < NH / 8; ++c) {
+                    const int g = (j0 + NH * hc) / 8 + c;
+                    st_bf16x8(dst + state_img_off(lane, g), s + 8 * c);
+                    st_bf16x8(dst + state_img_off(lane + D, g), m + 8 * c);
+                }
+            }
+            clk.lap(7);
             if (!warp_wait(&bars[B_M2], n & 1, abort_flag)) break;
             // the products of this chunk (E and F among them) have read the
             // slot: it may be refilled
@@ -498,6 +522,13 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 }
 
 }  // namespace
+
+#ifdef MDN_PHASE_CLOCKS
+extern "C" int mdn_diag_chain_clock(float* p)
+{
+    return cudaMemcpyToSymbol(g_chain_clk, &p, sizeof(p)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
 {
