@@ -115,6 +115,7 @@ struct ChainArgs {
     int T, H, NT;
     const int* cu_seqlens;  // unused here (one batch row per sequence)
     const int* cu_chunks;
+    const int* seq_order;   // unused here
 };
 
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
@@ -559,6 +560,7 @@ cudaError_t launch_bwd_chain_tc(const BwdArgs& a, cudaStream_t s)
     t.NT = a.NT;
     t.cu_seqlens = nullptr;
     t.cu_chunks = nullptr;
+    t.seq_order = nullptr;
     cudaError_t e = cudaFuncSetAttribute(chunk_bwd_chain_kernel<NS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::SMEM_BYTES);

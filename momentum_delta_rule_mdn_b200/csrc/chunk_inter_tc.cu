@@ -545,13 +545,23 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
     const long long heads = a.cu_chunks ? (long long)a.nseq * a.H : (long long)a.B * a.H;
     const long long room = sms - sms / 4;  // SMs the chain may take beside the intra kernel
     if (ns == 0) {
-        if (a.cu_chunks) ns = heads * 4 <= 2LL * sms ? 32 : 64;
+        // packed sequences: the chains are ordered longest first, and the
+        // longest one is the critical path; 32-column slices (the shortest
+        // step) while the slices fit in four waves, else 64
+        if (a.cu_chunks) ns = heads * 4 <= 4LL * sms ? 32 : 64;
         else ns = heads * 4 <= sms ? 32 : 128;
     }
     const long long ctas = heads * (D / ns);
     Reserve rv;
     if (a.cu_chunks) {
-        if (ctas <= room) rv.sms = (int)ctas;
+        // SMs from the start for the chains of the longest sequence (the
+        // first H slices' worth of CTAs); the intra-chunk kernel keeps the
+        // rest, so that it produces that sequence's chunks faster than its
+        // chains take them; the other chains follow as SMs free up
+        const long long first = (long long)a.H * (D / ns);
+        long long want = first < ctas ? first : ctas;
+        if (want > room) want = room;
+        rv.sms = (int)want;
     } else {
         rv = plan_reserve(heads * a.NT, ctas, sms, a.NT, ns);
     }

@@ -82,13 +82,15 @@ struct IntraArgs {
     int T, H, NT, BH;
     int reserve;             // CTAs on SMs 0 .. reserve-1 take at most `limit` chunks,
     int limit;               // freeing those SMs early for the inter-chunk kernel
+    const int* chunk_order;  // variable-length mode: the order of the padded chunks; else null
 };
 
-// Chunk-major order: the c-th chunk is chunk n of head bh; returns its index
-// in the head-major layout of the workspace.
+// Chunk-major order: the c-th chunk is chunk n of head bh (n taken through
+// chunk_order in variable-length mode: the longest sequence's chunks first);
+// returns its index in the head-major layout of the workspace.
 __device__ __forceinline__ long long chunk_of(long long c, const IntraArgs& a, int& n, int& bh) {
     const unsigned cu = (unsigned)c, q = cu / (unsigned)a.BH;  // chunk counts fit 32 bits
-    n = (int)q;
+    n = a.chunk_order ? a.chunk_order[q] : (int)q;
     bh = (int)(cu - q * (unsigned)a.BH);
     return (long long)bh * a.NT + n;
 }
@@ -653,6 +655,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a, cudaStream_t s, int reserv
     t.ready = a.ready;
     t.queue = a.ready + chunks;
     t.reserve = reserve;
+    t.chunk_order = a.chunk_order;
     t.limit = limit > 0 ? limit : 1;
     t.status = a.status;
     t.dbg = a.dbg ? a.dbg + 80512 : nullptr;

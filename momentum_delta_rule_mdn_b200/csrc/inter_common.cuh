@@ -25,6 +25,7 @@ struct InterArgs {
     int T, H, NT;
     const int* cu_seqlens;  // variable-length mode (see ChunkArgs); null otherwise
     const int* cu_chunks;
+    const int* seq_order;
 };
 
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
@@ -92,6 +93,7 @@ inline InterArgs inter_args(const ChunkArgs& a)
     t.NT = a.NT;
     t.cu_seqlens = a.cu_seqlens;
     t.cu_chunks = a.cu_chunks;
+    t.seq_order = a.seq_order;
     return t;
 }
 

@@ -484,7 +484,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
 namespace {
 
 struct VarlenLayout {
-    size_t cu_s, cu_c, q, k, v, al, ml, be, et, total;
+    size_t cu_s, cu_c, seq_order, chunk_order, q, k, v, al, ml, be, et, total;
     WsLayout chunk;  // the chunk pass's scratch, at the start of the workspace
     int NT;          // padded chunks (an upper bound on the sequences' chunk count)
 };
@@ -507,6 +507,8 @@ mdn_status varlen_layout(int N, int total_T, int H, int dk, int dv, int C, mdn_d
     size_t off = v.chunk.total;
     v.cu_s = off; off += align_up((size_t)(N + 1) * sizeof(int));
     v.cu_c = off; off += align_up((size_t)(N + 1) * sizeof(int));
+    v.seq_order = off;   off += align_up((size_t)N * sizeof(int));
+    v.chunk_order = off; off += align_up((size_t)NT * sizeof(int));
     v.q = off;    off += align_up(rows * dk * elt);
     v.k = off;    off += align_up(rows * dk * elt);
     v.v = off;    off += align_up(rows * dv * elt);
@@ -576,11 +578,15 @@ mdn_status mdn_chunk_fwd_varlen(const void* q, const void* k, const void* v, mdn
     a.B = 1; a.T = L.NT * C; a.H = H; a.D = D; a.NT = L.NT;
     a.o = o; a.vt = vtilde; a.S_T = S_T; a.M_T = M_T;
     a.cu_seqlens = cu_s; a.cu_chunks = cu_c; a.nseq = N;
+    int* seq_order = reinterpret_cast<int*>(ws + L.seq_order);
+    int* chunk_order = reinterpret_cast<int*>(ws + L.chunk_order);
+    a.seq_order = seq_order; a.chunk_order = chunk_order;
     carve(a, ws, L.chunk);
 
     cudaError_t e;
     if ((e = cudaMemsetAsync(a.status, 0, L.chunk.head, s))) return mdn::cuda_fail(e);
-    if ((e = launch_varlen_setup(cu_seqlens, N, total_T, cu_s, cu_c, a.status + 2, s)))
+    if ((e = launch_varlen_setup(cu_seqlens, N, total_T, L.NT, cu_s, cu_c, seq_order, chunk_order,
+                                 a.status + 2, s)))
         return mdn::cuda_fail(e);
     const size_t elt = in_dtype == MDN_F32 ? 4 : 2;
     if ((e = launch_varlen_gather(q, k, v, elt, alpha_log, mu_log, beta, eta, cu_s, cu_c, N, H, D,

@@ -139,6 +139,13 @@ struct ChunkArgs {
     const int* cu_seqlens = nullptr;
     const int* cu_chunks = nullptr;
     int nseq = 0;
+    // Work order in variable-length mode: seq_order lists the sequences by
+    // decreasing chunk count (chain CTA sh takes sequence seq_order[sh / H]),
+    // chunk_order the padded chunks with the longest sequence's first (the
+    // intra-chunk kernel's q-th chunk index), so that the longest chain, the
+    // pass's critical path, starts first and is fed first.
+    const int* seq_order = nullptr;
+    const int* chunk_order = nullptr;
     // Fused gate parameterisation: with gate_pre != 0, alpha_log, mu_log,
     // beta and eta above hold the pre-activations x_eta, a, b, c (see GateSrc).
     int gate_pre = 0;
@@ -253,8 +260,9 @@ __device__ __forceinline__ Chain chain_of(const A& a, long long sh)
     c.sh = sh;
     c.h = (int)(sh % a.H);
     if (a.cu_chunks) {
-        const int seq = (int)(sh / a.H);
+        const int seq = a.seq_order ? a.seq_order[sh / a.H] : (int)(sh / a.H);
         const int c0 = a.cu_chunks[seq];
+        c.sh = (long long)seq * a.H + c.h;  // states are [nseq, H, D, D] in sequence order
         c.b = 0;
         c.chunk0 = (long long)c.h * a.NT + c0;
         c.n0 = c0;
@@ -369,8 +377,9 @@ cudaError_t launch_finite_check(const void* x, size_t n, bool bf16, unsigned* fl
 // makes every sequence empty.  Gather: the chunk-aligned padded inputs
 // (NT*C rows; padding rows are steps that change nothing: k = v = q = 0,
 // alpha = mu = 1, beta = eta = 0).
-cudaError_t launch_varlen_setup(const int* cu_seqlens, int N, int total_T, int* cu_s, int* cu_c,
-                                unsigned* bad, cudaStream_t s);
+cudaError_t launch_varlen_setup(const int* cu_seqlens, int N, int total_T, int NT, int* cu_s,
+                                int* cu_c, int* seq_order, int* chunk_order, unsigned* bad,
+                                cudaStream_t s);
 cudaError_t launch_varlen_gather(const void* q, const void* k, const void* v, size_t elt,
                                  const float* alpha_log, const float* mu_log, const float* beta,
                                  const float* eta, const int* cu_s, const int* cu_c, int N, int H,

@@ -9,7 +9,10 @@
 // up to the chunk boundary are steps that change nothing (k = v = q = 0,
 // alpha = mu = 1, beta = eta = 0), as for a ragged last chunk.  The chain
 // kernels then run one chain per (sequence, head) over that sequence's chunks
-// and write o and vt straight back to the packed rows.
+// and write o and vt straight back to the packed rows.  The longest chain is
+// the pass's critical path, so the setup also ranks the sequences by length:
+// the chain kernels start the longest sequences' chains first, and the
+// intra-chunk kernel produces their chunks first.
 #include "mdn_internal.cuh"
 
 namespace mdn {
@@ -44,11 +47,17 @@ __device__ int block_incl_sum(int x, int* warp_tot, int& total)
     return r;
 }
 
+// Sequences are ranked by chunk count (for the work order) when there are at
+// most this many; beyond it they keep their call order.
+constexpr int kRankMax = 2048;
+
 __global__ void __launch_bounds__(kSetupThreads)
-varlen_setup_kernel(const int* __restrict__ cu, int N, int total_T, int* __restrict__ cu_s,
-                    int* __restrict__ cu_c, unsigned* __restrict__ bad)
+varlen_setup_kernel(const int* __restrict__ cu, int N, int total_T, int NT, int* __restrict__ cu_s,
+                    int* __restrict__ cu_c, int* __restrict__ seq_order,
+                    int* __restrict__ chunk_order, unsigned* __restrict__ bad)
 {
     __shared__ int warp_tot[32];
+    __shared__ int cnt_sh[kRankMax];
     const int tid = threadIdx.x;
     int my_bad = 0;
     for (int i = tid; i <= N; i += kSetupThreads) {
@@ -71,6 +80,39 @@ varlen_setup_kernel(const int* __restrict__ cu, int N, int total_T, int* __restr
         carry += total;
     }
     if (tid == 0 && any_bad) atomicOr(bad, 1u);
+    __syncthreads();  // cu_c is complete
+
+    // seq_order: the sequences by decreasing chunk count (ties in call order)
+    if (!any_bad && N <= kRankMax) {
+        for (int i = tid; i < N; i += kSetupThreads) cnt_sh[i] = cu_c[i + 1] - cu_c[i];
+        __syncthreads();
+        for (int i = tid; i < N; i += kSetupThreads) {
+            const int ci = cnt_sh[i];
+            int rank = 0;
+            for (int j = 0; j < N; ++j) {
+                const int cj = cnt_sh[j];
+                rank += (cj > ci) || (cj == ci && j < i);
+            }
+            seq_order[rank] = i;
+        }
+    } else {
+        for (int i = tid; i < N; i += kSetupThreads) seq_order[i] = i;
+    }
+    __syncthreads();
+    // chunk_order: the padded chunks of seq_order[0], then of seq_order[1], ...,
+    // then the unused padded chunks
+    carry = 0;
+    for (int base = 0; base < N; base += kSetupThreads) {  // uniform trip count
+        const int r = base + tid;
+        const int sq = r < N ? seq_order[r] : 0;
+        const int cnt = r < N ? cu_c[sq + 1] - cu_c[sq] : 0;
+        int total;
+        const int incl = block_incl_sum(cnt, warp_tot, total);
+        const int start = carry + incl - cnt;
+        for (int t = 0; t < cnt; ++t) chunk_order[start + t] = cu_c[sq] + t;
+        carry += total;
+    }
+    for (int j = cu_c[N] + tid; j < NT; j += kSetupThreads) chunk_order[j] = j;
 }
 
 // One warp per padded row: the row's H*D values of q, k, v (16-byte units)
@@ -129,11 +171,13 @@ varlen_gather_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
 
 }  // namespace
 
-cudaError_t launch_varlen_setup(const int* cu_seqlens, int N, int total_T, int* cu_s, int* cu_c,
-                                unsigned* bad, cudaStream_t s)
+cudaError_t launch_varlen_setup(const int* cu_seqlens, int N, int total_T, int NT, int* cu_s,
+                                int* cu_c, int* seq_order, int* chunk_order, unsigned* bad,
+                                cudaStream_t s)
 {
     ProfScope ps(kVarlen, s);
-    varlen_setup_kernel<<<1, kSetupThreads, 0, s>>>(cu_seqlens, N, total_T, cu_s, cu_c, bad);
+    varlen_setup_kernel<<<1, kSetupThreads, 0, s>>>(cu_seqlens, N, total_T, NT, cu_s, cu_c,
+                                                     seq_order, chunk_order, bad);
     return cudaGetLastError();
 }
 
