@@ -531,10 +531,9 @@ static Reserve plan_reserve(long long chunks, long long ctas, int sms, int nt, i
 // pipe, bounds the step.  So four 32-column slices per head when they all fit
 // on the SMs at once (the shortest chain); otherwise one CTA per head, which
 // takes the least SM time per chunk (9k against 4 x 3.1k or 2 x 4.8k) and
-// leaves the fewest waves.  Packed sequences keep 32 up to two waves, else 64
-// (their chains end at different times), and reserve SMs (one chunk each)
-// only when the chains fit beside a quarter of the SMs kept for the
-// intra-chunk kernel: their chains' lengths are not known on the host.
+// leaves the fewest waves.  Packed sequences keep 32 up to four waves, else
+// 64 (their chains end at different times), and reserve SMs (one chunk
+// each) for the chains of the longest sequence, which start first.
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t s, int ns)
 {
     if (a.D != D) return cudaErrorNotSupported;
