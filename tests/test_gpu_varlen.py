@@ -105,6 +105,44 @@ def test_varlen_layer_budget_length_mix():
         assert rel_l2(to_np(g), r) <= TOL["bf16"], name
 
 
+def test_varlen_many_sequences_beyond_the_rank_limit():
+    """More sequences (2,100) than the setup ranks by length (2,048): the work
+    order falls back to the call order; lengths 0..150 at random, H = 1,
+    bf16, d = 128, against the oracle over the whole batch and per sequence."""
+    rng = np.random.default_rng(405)
+    lens = [int(x) for x in rng.integers(0, 151, size=2100)]
+    inp, dev, cu, cu_dev, S0n, M0n, S0, M0 = _packed(lens, 1, 128, "bf16", seed=406,
+                                                     state_std=0.01)
+    o, vt, S_T, M_T = mdn.chunk_fwd_varlen(*(dev[k] for k in ("q", "k", "v")),
+                                           *(dev[g] for g in GATES), cu_dev, inp.d_corr,
+                                           S0, M0, flags=_lib.MDN_CHECK_FINITE)
+    torch.cuda.synchronize()
+    ro, rvt, rS, rM = _ref(inp, cu, S0n, M0n)
+    for name, g, r in (("o", o, ro), ("vtilde", vt, rvt), ("S_T", S_T, rS), ("M_T", M_T, rM)):
+        assert rel_l2(to_np(g), r) <= TOL["bf16"], name
+    S_np = to_np(S_T)
+    worst = max(rel_l2(S_np[s], rS[s]) for s in range(len(lens)) if lens[s] > 0)
+    assert worst <= TOL["bf16"], worst
+
+
+def test_varlen_longest_sequence_last_and_first():
+    """The work order ranks the sequences by length (chains and chunks of the
+    longest first): a call with the longest sequence last and one with it
+    first both match the oracle."""
+    lens = [130, 64, 1, 700, 65, 2000]
+    outs = []
+    for order in (lens, lens[::-1]):
+        inp, dev, cu, cu_dev, S0n, M0n, S0, M0 = _packed(order, 2, 128, "bf16", seed=407,
+                                                         state_std=0.02)
+        o, vt, S_T, M_T = mdn.chunk_fwd_varlen(*(dev[k] for k in ("q", "k", "v")),
+                                               *(dev[g] for g in GATES), cu_dev, inp.d_corr,
+                                               S0, M0)
+        torch.cuda.synchronize()
+        ro, rvt, rS, rM = _ref(inp, cu, S0n, M0n)
+        for name, g, r in (("o", o, ro), ("vtilde", vt, rvt), ("S_T", S_T, rS), ("M_T", M_T, rM)):
+            assert rel_l2(to_np(g), r) <= TOL["bf16"], (name, order)
+
+
 @pytest.mark.parametrize("cu_list,total", [
     ([0, 100, 50, 200], 200),   # decreasing
     ([0, 100, 150], 200),       # does not end at total_T
