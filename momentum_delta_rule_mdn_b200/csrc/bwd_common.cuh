@@ -101,7 +101,7 @@ struct PackedLower {
     __device__ __forceinline__ int operator()(int r, int i) const { return ((r * (r + 1)) >> 1) + i; }
 };
 
-// The last phase (every thread of a CTA of at least 128 threads calls it): dG
+// The last phase (every thread of a CTA of at least 256 threads calls it): dG
 // (overwritten) and Gp, lower triangles stored as Idx says, the record of the
 // state products (rec_g, in global memory; rec: kBwdRec floats of shared
 // scratch), v.da holding the direct adjoint of alpha from P.  Writes the four
@@ -209,52 +209,90 @@ __device__ __forceinline__ void bwd_coeff_phase(const BwdArgs& a, const float* r
     }
     __syncthreads();
     lap(1);
-    // Gamma = eta o Gp: row sums of dG o Gamma (threads 0..63), column sums
-    // and eta's share (threads 64..127)
-    if (tid < C) {
-        const int x = tid;
-        float rs = 0.f;
-        for (int y = 0; y <= x; ++y) rs = fmaf(dG[at(x, y)], v_et[y] * Gp[at(x, y)], rs);
-        v_dla[x] += rs;
-    } else if (tid < 2 * C) {
-        const int x = tid - C;
-        float cs = 0.f, ce = 0.f;
-        for (int y = x; y < C; ++y) {
-            const float gp = Gp[at(y, x)];
-            cs = fmaf(dG[at(y, x)], v_et[x] * gp, cs);
-            ce = fmaf(dG[at(y, x)], gp, ce);
+    // Gamma = eta o Gp: row sums of dG o Gamma (threads 0..127, two per row),
+    // column sums and eta's share (threads 128..255, two per column); the two
+    // halves of a sum (alternate terms) are joined by a shuffle
+    if (tid < 4 * C) {
+        const bool rows = tid < 2 * C;
+        const int x = (tid & (2 * C - 1)) >> 1, part = tid & 1;
+        float s0 = 0.f, s1 = 0.f;
+        if (rows) {
+            for (int y = part; y <= x; y += 2) s0 = fmaf(dG[at(x, y)], v_et[y] * Gp[at(x, y)], s0);
+        } else {
+            for (int y = x + part; y < C; y += 2) {
+                const float gp = Gp[at(y, x)];
+                s0 = fmaf(dG[at(y, x)], v_et[x] * gp, s0);
+                s1 = fmaf(dG[at(y, x)], gp, s1);
+            }
         }
-        v_dlm[x] -= cs;
-        v_de[x] += ce;
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        if (part == 0) {
+            if (rows) {
+                v_dla[x] += s0;
+            } else {
+                v_dlm[x] -= s0;
+                v_de[x] += s1;
+            }
+        }
     }
     __syncthreads();
     lap(2);
-    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place, one column per
-    // thread (the next row's operands are read before this row's store)
-    if (tid < C) {
-        const int i = tid;
-        float R = 0.f;
-        float dg_n = dG[at(C - 1, i)], al_n = 0.f;  // al_n: alpha_{j+1} (none past the chunk)
-        for (int j = C - 1; j >= i; --j) {
-            const float dg = dg_n, al = al_n;
-            if (j > i) {
-                dg_n = dG[at(j - 1, i)];
-                al_n = v_al[j];
-            }
-            R = dg + (j + 1 < C ? al * R : 0.f);
-            dG[at(j, i)] = R;
+    // R_{j,i} = sum_{r>=j} dG_{r,i} exp(la_r - la_j), in place: the reverse
+    // recurrence R_j = dG_j + alpha_{j+1} R_{j+1} down each column, by blocks
+    // of 16 rows on four threads per column (thread part p owns rows
+    // 16p .. 16p + 15).  Each thread runs its block from a zero carry, keeping
+    // L_j and the decay P_j = alpha_{j+1} .. alpha_{hi+1} to its block's top;
+    // the carries R_{16(p+1)} come down the four lanes, and R_j = L_j + P_j R.
+    if (tid < 4 * C) {
+        const int i = tid >> 2, part = tid & 3, lo = 16 * part;
+        float L[16], P[16], al1[16];
+        // every read of the block before any write
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int j = lo + e;
+            L[e] = j >= i ? dG[at(j, i)] : 0.f;
+            al1[e] = j + 1 < C ? v_al[j + 1] : 0.f;  // alpha_{j+1}; none past the chunk
+        }
+        float l = 0.f, pr = 1.f;
+#pragma unroll
+        for (int e = 15; e >= 0; --e) {
+            pr *= al1[e];
+            l = L[e] + al1[e] * l;
+            L[e] = l;
+            P[e] = pr;
+        }
+        // (L, P) at the block's lowest row, from the blocks above
+        const unsigned full = 0xffffffffu;
+        const int base = (threadIdx.x & 31) & ~3;
+        float carry = 0.f;
+#pragma unroll
+        for (int q = 3; q >= 1; --q) {
+            const float lq = __shfl_sync(full, L[0], base + q);
+            const float pq = __shfl_sync(full, P[0], base + q);
+            if (q > part) carry = lq + pq * carry;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int j = lo + e;
+            if (j >= i) dG[at(j, i)] = L[e] + P[e] * carry;
         }
     }
     __syncthreads();
     lap(3);
-    // U_j = sum_{i<=j} eta_i exp(lm_j - lm_i) R_{j,i}
-    if (tid < C) {
-        const int j = tid;
+    // U_j = sum_{i<=j} eta_i exp(lm_j - lm_i) R_{j,i}: four threads per row
+    // (every fourth term each), joined by shuffles
+    if (tid < 4 * C) {
+        const int j = tid >> 2, part = tid & 3;
         float U = 0.f;
-        for (int i = 0; i <= j; ++i) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[at(j, i)], U);
-        v_dbe[j] += U;
-        v_dla[j] -= v_be[j] * U;
-        v_dlm[j] += v_be[j] * U;
+        for (int i = part; i <= j; i += 4) U = fmaf(v_et[i] * expf(v_lm[j] - v_lm[i]), dG[at(j, i)], U);
+        U += __shfl_xor_sync(0xffffffffu, U, 1);
+        U += __shfl_xor_sync(0xffffffffu, U, 2);
+        if (part == 0) {
+            v_dbe[j] += U;
+            v_dla[j] -= v_be[j] * U;
+            v_dlm[j] += v_be[j] * U;
+        }
     }
     __syncthreads();
     lap(4);

@@ -487,30 +487,59 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         mma_commit(&bars[0]);
     }
     // Gamma without eta, by its column recurrence (overlaps the products):
-    // Gp_{r,i} = alpha_r Gp_{r-1,i} + beta_r mubar_r / mubar_i, the ratio as a
-    // running product of mu (held in v.de until the coefficient phase)
-    // (the next row's alpha, beta, mu are read before this row's store, so that
-    // the shared-memory latency overlaps the recurrence)
-    if (tid < C) {
-        const int i = tid;
-        float g = v.be[i], f = 1.f;
-        Gp[at(i, i)] = g;
-        float al_n = 0.f, be_n = 0.f, de_n = 1.f;
-        if (i + 1 < C) {
-            al_n = v.al[i + 1];
-            be_n = v.be[i + 1];
-            de_n = v.de[i + 1];
+    // Gp_{r,i} = alpha_r Gp_{r-1,i} + beta_r f_r with f_r = mubar_r / mubar_i a
+    // running product of mu (held in v.de until the coefficient phase), by
+    // blocks of 16 rows on four threads per column (part p owns rows 16p ..).
+    // The block's rows map a carry (g, f) entering it to (A g + f G, f F);
+    // the maps of the blocks below give each block its carry, and a second
+    // pass over the block writes Gp.
+    {
+        const int i = tid >> 2, part = tid & 3, lo = 16 * part;
+        float ar[16], br[16], mr[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            ar[e] = v.al[lo + e];
+            br[e] = v.be[lo + e];
+            mr[e] = v.de[lo + e];
         }
-        for (int r = i + 1; r < C; ++r) {
-            const float al_r = al_n, be_r = be_n, de_r = de_n;
-            if (r + 1 < C) {
-                al_n = v.al[r + 1];
-                be_n = v.be[r + 1];
-                de_n = v.de[r + 1];
+        float A = 1.f, G = 0.f, F = 1.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int r = lo + e;
+            if (r == i) {
+                A = 0.f;
+                G = br[e];
+                F = 1.f;
+            } else if (r > i) {
+                G = fmaf(ar[e], G, br[e] * mr[e] * F);
+                A *= ar[e];
+                F *= mr[e];
             }
-            f *= de_r;
-            g = fmaf(al_r, g, be_r * f);
-            Gp[at(r, i)] = g;
+        }
+        const unsigned full = 0xffffffffu;
+        const int base = lane & ~3;
+        float g = 0.f, f = 1.f;  // the carry entering this block
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            const float aq = __shfl_sync(full, A, base + q);
+            const float gq = __shfl_sync(full, G, base + q);
+            const float fq = __shfl_sync(full, F, base + q);
+            if (q < part) {
+                g = fmaf(aq, g, f * gq);
+                f *= fq;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int r = lo + e;
+            if (r == i) {
+                f = 1.f;
+                g = br[e];
+            } else if (r > i) {
+                f *= mr[e];
+                g = fmaf(ar[e], g, br[e] * f);
+            }
+            if (r >= i) Gp[at(r, i)] = g;
         }
     }
     ok = __syncthreads_and(ok && mbar_wait(&bars[0], 0));
@@ -542,6 +571,7 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
             tmem_ld16(tq + 32 * half + 16 * p2, x1);        // dO Vt^T  (dY Vt^T on lanes 64..127)
             tmem_ld16(tq + 64 + 32 * half + 16 * p2, x2);   // Qhat K^T (K K^T)
             tmem_wait_ld();
+            float row3[16];  // this row's 16 entries of [dOVG; dPK], two 16-byte stores
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int i = 32 * half + 16 * p2 + e;
@@ -552,7 +582,7 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
                         ovg = x1[e] * g;
                         dG[at(r, i)] = x1[e] * x2[e];
                     }
-                    st_bf16(sm + LA_3 + kmaj_off(r, i, 16384), ovg);             // row r of [dOVG; .]
+                    row3[e] = ovg;                                               // row r of [dOVG; .]
                     st_bf16(sm + LA_4 + kmaj_off(i, r, 16384), ovg);             // (dOVG^T)[i][r]
                 } else {
                     float pk = 0.f, dm = 0.f;
@@ -561,9 +591,15 @@ bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
                         dm = -x1[e] * al_r * x2[e];
                     }
                     dgm[16 * p2 + e] = dm;
-                    st_bf16(sm + LA_3 + kmaj_off(64 + r, i, 16384), pk);        // row 64 + r: dPK
+                    row3[e] = pk;                                                // row 64 + r: dPK
                     st_bf16(sm + LA_4 + kmaj_off(i, 64 + r, 16384), pk * al_r); // (Diag(alpha) dPK)^T
                 }
+            }
+            {
+                const int k0 = 32 * half + 16 * p2;  // a multiple of 16: two whole 16-byte chunks
+                const uint32_t o = kmaj_off(R < 64 ? r : 64 + r, k0, 16384);
+                st_bf16x8(sm + LA_3 + o, row3);
+                st_bf16x8(sm + LA_3 + (o ^ 16), row3 + 8);
             }
         }
     }
