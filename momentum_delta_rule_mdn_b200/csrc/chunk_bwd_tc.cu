@@ -34,8 +34,10 @@ constexpr uint32_t SA2 = 32768;      // [Vt; K]: the product rows of K are not r
 constexpr uint32_t SB1 = 65536;      // [S | M] as 256 rows: 2 K-panels x 256 rows x 128 B
 constexpr uint32_t SB2 = 131072;     // [dS | dM]
 constexpr uint32_t SQ = 196608;      // Q rows for the epilogue: 2 K-panels x 64 rows x 128 B
-constexpr uint32_t SSUM = SQ + 16384;  // fp32 row-sum partials [12][64], then scalars [8][3]
-constexpr uint32_t SBAR = SSUM + 3072 + 96;
+constexpr int kThrS = 384;           // threads of the state-product kernel (3 warps per TMEM quadrant)
+constexpr int kSumSlots = 18;        // row-sum partial slots (see the kernel)
+constexpr uint32_t SSUM = SQ + 16384;  // fp32 row-sum partials [18][64], then scalars [12][3]
+constexpr uint32_t SBAR = SSUM + kSumSlots * 64 * 4 + (kThrS / 32) * 3 * 4;
 constexpr uint32_t SMISC = SBAR + 16;  // after two mbarriers (MMAs done, state images landed)
 constexpr uint32_t SMEM_BYTES = SMISC + 16 + 1024;  // + alignment slack
 constexpr int XS = 129;              // row stride (floats) of the dk exchange tile over SA1
@@ -87,7 +89,7 @@ struct BwdClock {
 };
 #endif
 
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThrS, 1)
 bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_vt,
                           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                           BwdArgs a)
@@ -102,10 +104,10 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     const int b = (int)(bh / a.H), h = (int)(bh % a.H);
     const size_t chunk = blockIdx.x, crow = chunk * C;
     // row-sum partials, one slot per writer so that the sums are formed in a
-    // fixed order: sa from (row kind, column half) in slots 0..3, then sb,
-    // sd2, sgl, sw from the two column halves in slots 4..11
+    // fixed order: sa from (row kind, column group) in slots 0..5, then sb,
+    // sd2, sgl, sw from the three column groups in slots 6..17
     float* part = reinterpret_cast<float*>(sm + SSUM);
-    float* wsum = part + 12 * C;                             // [8 warps][3]
+    float* wsum = part + kSumSlots * C;                      // [12 warps][3]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + SBAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SMISC);
     BwdClock clk;
@@ -138,7 +140,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    for (int i = tid; i < 12 * C; i += kThr) part[i] = 0.f;
+    for (int i = tid; i < kSumSlots * C; i += kThrS) part[i] = 0.f;
     fence_proxy_async_smem();
     __syncthreads();
     clk.lap(0);
@@ -149,7 +151,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     float s1 = 0.f, s2 = 0.f, s3 = 0.f;
     if (ok) {
 #pragma unroll 2
-        for (int i = tid; i < D * 16; i += kThr) {
+        for (int i = tid; i < D * 16; i += kThrS) {
             const int row = i & (D - 1), g = i >> 7;
             float sv[8], mv[8], dsv[8], dmv[8];
             unpack_bf16x8(*reinterpret_cast<const uint4*>(sm + SB1 + state_img_off(row, g)), sv);
@@ -197,10 +199,12 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
         }
         mma_commit(&bar[0]);
     }
-    // Epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..; warps w and w + 4 take
-    // the two halves of the 128 columns of each product.  Its coefficients are
-    // loaded while the products run; K and Q come from shared memory.
-    const int quad = warp & 3, half = warp >> 2;
+    // Epilogue.  Warp w reads TMEM lanes 32 (w % 4) ..; warps w, w + 4, w + 8
+    // take columns [0, 48), [48, 96), [96, 128) of each product.  Its
+    // coefficients are loaded while the products run; K and Q come from
+    // shared memory.
+    const int quad = warp & 3, grp = warp >> 2;
+    const int c_lo = 48 * grp, c_hi = grp == 2 ? 128 : c_lo + 48;
     const int R = quad * 32 + lane;               // TMEM lane: dO rows 0..63, dY rows 64..127
     const uint32_t tq = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     float* X = reinterpret_cast<float*>(sm + SA1);  // dk of the dY rows, [64][XS], over the operands
@@ -230,7 +234,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     if (ok && R >= 64) {
         // dY rows: dk part -Diag(alphabar) P5 + Diag(D2) P6, into the exchange tile
 #pragma unroll 1
-        for (int k0 = half * 64; k0 < half * 64 + 64; k0 += 16) {
+        for (int k0 = c_lo; k0 < c_hi; k0 += 16) {
             float p5[16], p6[16], kv[16];
             tmem_ld16(tq + k0, p5);
             tmem_ld16(tq + 128 + k0, p6);
@@ -251,7 +255,7 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     clk.lap(3);
     if (ok && R < 64) {
 #pragma unroll 1
-        for (int k0 = half * 64; k0 < half * 64 + 64; k0 += 16) {
+        for (int k0 = c_lo; k0 < c_hi; k0 += 16) {
             float p1[16], p2[16], p3[16], p4[16], kv[16], qh[16];
             tmem_ld16(tq + k0, p1);
             tmem_ld16(tq + 128 + k0, p2);
@@ -284,16 +288,16 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
             }
         }
     }
-    // row sums of both column halves (and, for sa, of both row kinds)
+    // row sums of the three column groups (and, for sa, of both row kinds)
     if (ok && in) {
         const int kind = R < 64 ? 0 : 1;
-        part[(2 * kind + half) * C + r] = sa;
+        part[(3 * kind + grp) * C + r] = sa;
         if (R < 64) {
-            part[(4 + half) * C + r] = sb;
-            part[(8 + half) * C + r] = sgl;
-            part[(10 + half) * C + r] = sw;
+            part[(6 + grp) * C + r] = sb;
+            part[(12 + grp) * C + r] = sgl;
+            part[(15 + grp) * C + r] = sw;
         } else {
-            part[(6 + half) * C + r] = sd2;
+            part[(9 + grp) * C + r] = sd2;
         }
     }
     fence_proxy_async_smem();
@@ -310,15 +314,16 @@ bwd_state_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __gri
     clk.lap(4);
     if (tid < C) {
         const float* p0 = part + tid;
-        rec[tid] = (p0[0] + p0[C]) + (p0[2 * C] + p0[3 * C]);
-        rec[C + tid] = p0[4 * C] + p0[5 * C];
-        rec[2 * C + tid] = p0[6 * C] + p0[7 * C];
-        rec[3 * C + tid] = p0[8 * C] + p0[9 * C];
-        rec[4 * C + tid] = p0[10 * C] + p0[11 * C];
+        auto sum3 = [&](int s0) { return (p0[s0 * C] + p0[(s0 + 1) * C]) + p0[(s0 + 2) * C]; };
+        rec[tid] = sum3(0) + sum3(3);
+        rec[C + tid] = sum3(6);
+        rec[2 * C + tid] = sum3(9);
+        rec[3 * C + tid] = sum3(12);
+        rec[4 * C + tid] = sum3(15);
     }
     if (tid < 3) {
         float acc = 0.f;
-        for (int w8 = 0; w8 < 8; ++w8) acc += wsum[w8 * 3 + tid];
+        for (int w = 0; w < kThrS / 32; ++w) acc += wsum[w * 3 + tid];
         rec[5 * C + tid] = acc;
     }
     if (!ok && tid == 0) {
@@ -1334,7 +1339,7 @@ cudaError_t launch_bwd_state_grads_tc(const BwdArgs& a, cudaStream_t s)
         !make_token_map(&mq, a.q, a.B, a.T, a.H, 64, true))
         return cudaErrorInvalidValue;
     ProfScope ps(kBwdStateGrads, s);
-    bwd_state_grads_tc_kernel<<<(unsigned)chunks, kThr, SMEM_BYTES, s>>>(mdo, mvt, mk, mq, a);
+    bwd_state_grads_tc_kernel<<<(unsigned)chunks, kThrS, SMEM_BYTES, s>>>(mdo, mvt, mk, mq, a);
     return cudaGetLastError();
 }
 
