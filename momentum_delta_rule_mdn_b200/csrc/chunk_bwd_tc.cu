@@ -5,17 +5,20 @@
 // the saved Vtilde).  Per chunk, with S, M the states entering it and dS, dM
 // the adjoints of the states leaving it, the six products
 //     [dO; dY] [S | M]^T   -> P1 = dO S^T, P2 = dO M^T, P5 = dY S^T, P6 = dY M^T
-//     [Vt; .]  [dS | dM]^T -> P3 = Vt dS^T, P4 = Vt dM^T  (product rows 64..127 unused)
+//     [Vt; K]  [dS | dM]^T -> P3 = Vt dS^T, P4 = Vt dM^T  (product rows 64..127 unused)
 // are two groups of eight tcgen05.mma (M 128, N 256, K 128; bf16 operands,
 // fp32 accumulators in 512 TMEM columns).  The epilogue forms the parts of dq
 // and dk they carry,
 //     dq = Diag(alphabar) P1 - Diag(b) P2
-//     dk = Diag(Gamma_C) P3 - Diag(w) P4 - Diag(alphabar) P5 + Diag(D2) P6
-// and the row sums that feed the gate gradients, exactly as the CUDA-core
-// kernel does.  Every operand arrives by the copy engines, K-major with the
-// 128-byte swizzle: the states and adjoints as bf16 images of the B operands
-// (written by the state scan and the reverse chain) and dY as the reverse
-// chain's bf16 image, by bulk copies; the dO, Vt, K and Q rows by TMA.
+//     dk = Diag(Gamma_C) P3 - Diag(w) P4 - Diag(alphabar) P5 + Diag(D2) P6 - d dq
+// (the last term from Qhat = Q - d K, for this kernel's part of dq) and the
+// row sums that feed the gate gradients, as the CUDA-core kernel does.  Every
+// operand arrives by the copy engines, K-major with the 128-byte swizzle: the
+// states and adjoints as bf16 images of the B operands (written by the state
+// scan and the reverse chain) and dY as the reverse chain's bf16 image, by
+// bulk copies; the dO, Vt, K and Q rows by TMA.  12 warps, three per TMEM lane
+// quadrant, each a third of the columns; dq and dk leave as 512-byte row
+// stores from staging tiles over the state images.
 #include "bwd_common.cuh"
 #include "mdn_internal.cuh"
 #include "tc_common.cuh"
