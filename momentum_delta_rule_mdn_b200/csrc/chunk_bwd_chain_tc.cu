@@ -58,8 +58,8 @@ struct Cfg {
     static constexpr uint32_t ST_BYTES = 128 * 2 * NS * 2;
     static constexpr uint32_t YB = ST + ST_BYTES;      // Y 64 rows x NS bf16, MN-major (64 / 128-byte swizzle)
     static constexpr uint32_t YB_BYTES = 64 * NS * 2;
-    static constexpr uint32_t V0 = YB + YB_BYTES;      // Att^T dO slice 64 rows x NS fp32, NVC slots
-    static constexpr uint32_t V_BYTES = 64 * NS * 4;
+    static constexpr uint32_t V0 = YB + YB_BYTES;      // Att^T dO slice 64 rows x NS bf16, NVC slots
+    static constexpr uint32_t V_BYTES = 64 * NS * 2;
     static constexpr uint32_t E0 = V0 + NVC * V_BYTES;   // Diag(alphabar) dO, -Diag(b) dO slices, NVC slots
     static constexpr uint32_t E_BYTES = 2 * 64 * NS * 2;  // (bf16, 64 rows x NS, MN-major: B of E, F)
     static constexpr uint32_t CR0 = E0 + NVC * E_BYTES;  // chunk coefficients (256 floats), NVC slots
@@ -102,7 +102,7 @@ constexpr int kBars = 24;
 
 struct ChainArgs {
     const float* crec;      // [chunks][256]: Gamma_C, w, ..., alphabar_C, b_C, mubar_C at 192..194
-    const float* pp;        // [chunks][D/32][64][32]  Att^T dO by slice
+    const __nv_bfloat16* pp;  // [chunks][D/32][64][32]  Att^T dO by slice (bf16)
     const uint8_t* eo;      // [chunks][D/32][2][4096 B]  Diag(alphabar) dO, -Diag(b) dO by slice
     const float* dS_T;      // cotangents of S_T, M_T (may be null)
     const float* dM_T;
@@ -390,8 +390,8 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             const float abC = cr[3 * C], bC = cr[3 * C + 1], mbC = cr[3 * C + 2];
             if (ypart) {
                 const float c_g = cr[r], c_w = cr[C + r];
-                const float* prow =
-                    reinterpret_cast<const float*>(sm + L::V0 + sv * L::V_BYTES) + r * NS + NH * hc;
+                const uint4* prow = reinterpret_cast<const uint4*>(
+                    sm + L::V0 + sv * L::V_BYTES + (r * NS + NH * hc) * 2);
                 if (!warp_wait(&bars[B_M1 + s2], (n >> 1) & 1, abort_flag)) break;
                 clk.lap(1);
                 tc_fence_after_sync();
@@ -403,9 +403,10 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 #pragma unroll
                 for (int c = 0; c < NH / 8; ++c) {
                     float vv[8];  // dVtilde = Att^T dO + Gamma_C K dS - w K dM
+                    unpack_bf16x8(prow[c], vv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        vv[e] = prow[8 * c + e] + fmaf(c_g, x[8 * c + e], -c_w * y[8 * c + e]);
+                        vv[e] += fmaf(c_g, x[8 * c + e], -c_w * y[8 * c + e]);
                     st_bf16x8(sm + L::YB + L::y_off(r, hc * (NH / 8) + c), vv);
                 }
                 clk.lap(2);

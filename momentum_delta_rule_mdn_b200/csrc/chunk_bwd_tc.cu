@@ -924,7 +924,7 @@ bwd_prep_tc_kernel(BwdArgs a)
     }
     const bool ok = __syncthreads_and(mbar_wait(bar, 0));
     tc_fence_after_sync();
-    float* att = a.att + chunk * C * C;
+    __nv_bfloat16* att = reinterpret_cast<__nv_bfloat16*>(a.att) + chunk * C * C;  // bf16 on this path
     if (ok && tid < C) {
         // column i of A and of Att from TMEM lane i (warps 0, 1: lanes 0..63)
         const int i = tid;
@@ -941,7 +941,7 @@ bwd_prep_tc_kernel(BwdArgs a)
                 const float av = i < r ? alpha_s[r] * kk[e] * Ts[(r - 1) * LDF + i] : 0.f;
                 const float tv = i <= r ? kh[e] * Ts[r * LDF + i] : 0.f;
                 As[r * LDF + i] = av;
-                att[r * C + i] = tv;
+                att[r * C + i] = __float2bfloat16_rn(tv);
             }
         }
     }
@@ -956,8 +956,14 @@ bwd_prep_tc_kernel(BwdArgs a)
         return;
     }
     inverse_blocked(As, Ts, tid);
-    float4* Tm = reinterpret_cast<float4*>(a.tmat + chunk * C * C);
-    for (int idx = tid; idx < C * C / 4; idx += kThr) Tm[idx] = lds4(Ts + (idx >> 4) * LDF + 4 * (idx & 15));
+    // T in bf16, row-major: the chain-operand kernel's input and the reverse
+    // chain's MN-major A of T^T dVtilde
+    uint2* Tm = reinterpret_cast<uint2*>(a.bc_tt + chunk * C * C);
+    for (int idx = tid; idx < C * C / 4; idx += kThr) {
+        const float4 t4 = lds4(Ts + (idx >> 4) * LDF + 4 * (idx & 15));
+        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+        Tm[idx] = bf16x4(tv);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1120,23 +1126,25 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             *reinterpret_cast<uint4*>(eo + 4096) = bf16x8(ob);
         }
     }
-    // T and Att: the scaled T tiles (K-major), Att^T (K-major), and T (bf16,
-    // row-major) to global
+    // T and Att (bf16, row-major, from the prep kernel): the scaled T tiles
+    // (K-major) and Att's rows (the MN-major form of Att^T)
     {
         constexpr int U4 = C * C / 4 / kThr;  // 4
-        float4 tx[U4], ax[U4];
+        uint2 tx[U4], ax[U4];
+        const __nv_bfloat16* Tg = a.bc_tt + chunk * C * C;
+        const __nv_bfloat16* Ag = reinterpret_cast<const __nv_bfloat16*>(a.att) + chunk * C * C;
 #pragma unroll
         for (int u = 0; u < U4; ++u) {
             const int idx = (tid + kThr * u) * 4;
-            tx[u] = *reinterpret_cast<const float4*>(a.tmat + chunk * C * C + idx);
-            ax[u] = *reinterpret_cast<const float4*>(a.att + chunk * C * C + idx);
+            tx[u] = *reinterpret_cast<const uint2*>(Tg + idx);
+            ax[u] = *reinterpret_cast<const uint2*>(Ag + idx);
         }
-        __nv_bfloat16* Tg = a.bc_tt + chunk * C * C;
 #pragma unroll
         for (int u = 0; u < U4; ++u) {
             const int idx = (tid + kThr * u) * 4, r = idx / C, r2 = idx % C;
-            const float tv[4] = {tx[u].x, tx[u].y, tx[u].z, tx[u].w};
-            const float av[4] = {ax[u].x, ax[u].y, ax[u].z, ax[u].w};
+            float tv[4], av[4];
+            unpack_bf16x4(tx[u], tv);
+            unpack_bf16x4(ax[u], av);
             float ts[4], tm[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -1146,8 +1154,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
             // four consecutive elements of row r: 8 bytes in each tile
             *reinterpret_cast<uint2*>(sm + PB_TS + kmaj_off(r, r2, 8192)) = bf16x4(ts);
             *reinterpret_cast<uint2*>(sm + PB_TM + kmaj_off(r, r2, 8192)) = bf16x4(tm);
-            *reinterpret_cast<uint2*>(sm + PA_AT + kmaj_off(r, r2, 8192)) = bf16x4(av);
-            *reinterpret_cast<uint2*>(Tg + idx) = bf16x4(tv);
+            *reinterpret_cast<uint2*>(sm + PA_AT + kmaj_off(r, r2, 8192)) = ax[u];
         }
     }
     fence_proxy_async_smem();
@@ -1190,17 +1197,16 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
         }
         // P = Att^T dO: rows r = R < 64, columns [64 half, 64 half + 64), by 32-column slice
         if (R < 64) {
-            float* Po = a.bc_p + chunk * C * D;
+            __nv_bfloat16* Po = a.bc_p + chunk * C * D;
 #pragma unroll 1
             for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
                 float p16[16];
                 tmem_ld16(tq + 128 + k0, p16);
                 tmem_wait_ld();
                 const int sl = k0 >> 5, jj = k0 & 31;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4*>(Po + (sl * C + R) * 32 + jj + 4 * q) =
-                        make_float4(p16[4 * q], p16[4 * q + 1], p16[4 * q + 2], p16[4 * q + 3]);
+                uint4* dst = reinterpret_cast<uint4*>(Po + (sl * C + R) * 32 + jj);
+                dst[0] = bf16x8(p16);
+                dst[1] = bf16x8(p16 + 8);
             }
         }  // (R < 64 is warp-uniform: quadrants 0, 1)
     }

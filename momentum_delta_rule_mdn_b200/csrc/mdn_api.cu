@@ -359,7 +359,7 @@ BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
     if (tc) {
         w.bc_u = off;   off += align_up(chunks * 256 * 64 * 2);
         w.bc_tt = off;  off += align_up(chunks * 64 * 64 * 2);
-        w.bc_p = off;   off += align_up(chunks * kChunk * D * sizeof(float));
+        w.bc_p = off;   off += align_up(chunks * kChunk * D * 2);
         w.bc_qh = off;  off += align_up(chunks * kChunk * D * 2);
         w.bc_eo = off;  off += align_up(chunks * (D / 32) * 2 * 4096);
         w.bc_rec = off; off += align_up(chunks * 256 * sizeof(float));
@@ -444,7 +444,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.crec_bw = reinterpret_cast<float*>(ws + w.rec);
     a.bc_u = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_u) : nullptr;
     a.bc_tt = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_tt) : nullptr;
-    a.bc_p = tc ? reinterpret_cast<float*>(ws + w.bc_p) : nullptr;
+    a.bc_p = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_p) : nullptr;
     a.bc_qh = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_qh) : nullptr;
     a.bc_eo = tc ? reinterpret_cast<uint8_t*>(ws + w.bc_eo) : nullptr;
     a.bc_rec = tc ? reinterpret_cast<float*>(ws + w.bc_rec) : nullptr;

@@ -207,8 +207,9 @@ struct BwdArgs {
     float* lc;
     float* bco;
     float* gamma;    // [B*H*NT, C, C]
-    float* att;      // [B*H*NT, C, C]  (Qhat K^T) o Gamma
-    float* tmat;     // [B*H*NT, C, C]  T = (I + A)^{-1}
+    float* att;      // [B*H*NT, C, C]  (Qhat K^T) o Gamma (tensor-core path: bf16 in the same place)
+    float* tmat;     // [B*H*NT, C, C]  T = (I + A)^{-1} (CUDA-core path; the tensor-core path
+                     // keeps T in bf16 in bc_tt)
     float* SS;       // [B*H*NT, 2, D, D]  S, M entering each chunk (CUDA-core path)
     float* dSS;      // [B*H*NT, 2, D, D]  adjoints of S, M leaving each chunk (CUDA-core path)
     // tensor-core path (null otherwise): the same states and adjoints as bf16,
@@ -221,7 +222,8 @@ struct BwdArgs {
     // chunk-only operands of the tensor-core reverse chain (null on the CUDA-core path)
     __nv_bfloat16* bc_u;   // [B*H*NT, 256, 64]  [-K^T Diag(alphabar) T^T; K^T Diag(D2) T^T]
     __nv_bfloat16* bc_tt;  // [B*H*NT, 64, 64]  T, row-major (the MN-major form of T^T)
-    float* bc_p;           // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice
+    __nv_bfloat16* bc_p;   // [B*H*NT, D/32, 64, 32]  Att^T dO, by 32-column slice (bf16: the
+                           // chain rounds dVtilde, of which it is a term, to bf16 anyway)
     __nv_bfloat16* bc_qh;  // [B*H*NT, C, D]  Qhat = Q - d K (bf16, rows of the chunk)
     uint8_t* bc_eo;        // [B*H*NT, D/32, 2, 4096 B]  Diag(alphabar) dO and -Diag(b) dO by
                            // 32-column slice, bf16, each the shared-memory image of the reverse

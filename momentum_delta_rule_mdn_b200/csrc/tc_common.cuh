@@ -29,6 +29,14 @@ __device__ __forceinline__ uint4 bf16x8(const float* x) {
 __device__ __forceinline__ uint2 bf16x4(const float* x) {
     return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
 }
+__device__ __forceinline__ void unpack_bf16x4(const uint2 w, float* x) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w.y);
+    x[0] = __low2float(a);
+    x[1] = __high2float(a);
+    x[2] = __low2float(b);
+    x[3] = __high2float(b);
+}
 __device__ __forceinline__ void st_bf16x8(uint8_t* p, const float* x) {
     *reinterpret_cast<uint4*>(p) = bf16x8(x);
 }
