@@ -1229,7 +1229,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
     tc_fence_after_sync();
     clk.lap(3);
     if (ok) {
-        float* Do = a.bc_d + (chunk * 2) * D * D;  // chain order
+        __nv_bfloat16* Do = a.bc_d + (chunk * 2) * D * D;  // chain order
 #pragma unroll 1
         for (int k0 = 64 * half; k0 < 64 * half + 64; k0 += 16) {
             float s16[16], m16[16];
@@ -1239,10 +1239,8 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int o = chain_off(R, k0 + 4 * q);
-                *reinterpret_cast<float4*>(Do + o) =
-                    make_float4(s16[4 * q], s16[4 * q + 1], s16[4 * q + 2], s16[4 * q + 3]);
-                *reinterpret_cast<float4*>(Do + D * D + o) =
-                    make_float4(m16[4 * q], m16[4 * q + 1], m16[4 * q + 2], m16[4 * q + 3]);
+                *reinterpret_cast<uint2*>(Do + o) = bf16x4(s16 + 4 * q);
+                *reinterpret_cast<uint2*>(Do + D * D + o) = bf16x4(m16 + 4 * q);
             }
         }
     }
@@ -1267,7 +1265,7 @@ bwd_chain_prep_tc_kernel(BwdArgs a)
 // thread keeps the next two chunks' increments in flight.
 __global__ void __launch_bounds__(256)
 bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0,
-                      const float* __restrict__ dinc, const float* __restrict__ rec,
+                      const __nv_bfloat16* __restrict__ dinc, const float* __restrict__ rec,
                       uint8_t* __restrict__ img, int NT, long long heads)
 {
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1286,16 +1284,16 @@ bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0
     }
     const int o0 = chain_off(i, 8 * g), o1 = chain_off(i, 8 * g + 4);
     const uint32_t ps = state_img_off(i, g), pm = state_img_off(i + D, g);
-    struct Step { float4 ds0, ds1, dm0, dm1; float aC, bC, mC; };
+    struct Step { uint2 ds0, ds1, dm0, dm1; float aC, bC, mC; };
     auto load = [&](int nn) {
         Step st;
         if (nn < NT) {
             const size_t chunk = (size_t)bh * NT + nn;
-            const float* dn = dinc + chunk * 2 * D * D;
-            st.ds0 = __ldg(reinterpret_cast<const float4*>(dn + o0));
-            st.ds1 = __ldg(reinterpret_cast<const float4*>(dn + o1));
-            st.dm0 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o0));
-            st.dm1 = __ldg(reinterpret_cast<const float4*>(dn + D * D + o1));
+            const __nv_bfloat16* dn = dinc + chunk * 2 * D * D;
+            st.ds0 = __ldg(reinterpret_cast<const uint2*>(dn + o0));
+            st.ds1 = __ldg(reinterpret_cast<const uint2*>(dn + o1));
+            st.dm0 = __ldg(reinterpret_cast<const uint2*>(dn + D * D + o0));
+            st.dm1 = __ldg(reinterpret_cast<const uint2*>(dn + D * D + o1));
             st.aC = __ldg(rec + chunk * 256 + 3 * C);
             st.bC = __ldg(rec + chunk * 256 + 3 * C + 1);
             st.mC = __ldg(rec + chunk * 256 + 3 * C + 2);
@@ -1310,8 +1308,11 @@ bwd_state_scan_kernel(const float* __restrict__ S0, const float* __restrict__ M0
         uint8_t* im = img + ((size_t)bh * NT + nn) * kStateImgBytes;
         *reinterpret_cast<uint4*>(im + ps) = bf16x8(s);
         *reinterpret_cast<uint4*>(im + pm) = bf16x8(m);
-        const float dsv[8] = {cu.ds0.x, cu.ds0.y, cu.ds0.z, cu.ds0.w, cu.ds1.x, cu.ds1.y, cu.ds1.z, cu.ds1.w};
-        const float dmv[8] = {cu.dm0.x, cu.dm0.y, cu.dm0.z, cu.dm0.w, cu.dm1.x, cu.dm1.y, cu.dm1.z, cu.dm1.w};
+        float dsv[8], dmv[8];
+        unpack_bf16x4(cu.ds0, dsv);
+        unpack_bf16x4(cu.ds1, dsv + 4);
+        unpack_bf16x4(cu.dm0, dmv);
+        unpack_bf16x4(cu.dm1, dmv + 4);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float sn = fmaf(cu.aC, s[e], fmaf(-cu.bC, m[e], dsv[e]));

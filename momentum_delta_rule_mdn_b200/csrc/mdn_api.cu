@@ -363,7 +363,7 @@ BwdLayout bwd_layout(long long BH, int NT, int D, bool tc)
         w.bc_qh = off;  off += align_up(chunks * kChunk * D * 2);
         w.bc_eo = off;  off += align_up(chunks * (D / 32) * 2 * 4096);
         w.bc_rec = off; off += align_up(chunks * 256 * sizeof(float));
-        w.bc_d = off;   off += align_up(chunks * 2 * D * D * sizeof(float));
+        w.bc_d = off;   off += align_up(chunks * 2 * D * D * 2);
         w.dy = off;     off += align_up(chunks * kDyImgBytes);
     }
     w.total = off;
@@ -448,7 +448,7 @@ mdn_status mdn_chunk_bwd(const void* q, const void* k, const void* v, mdn_dtype 
     a.bc_qh = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_qh) : nullptr;
     a.bc_eo = tc ? reinterpret_cast<uint8_t*>(ws + w.bc_eo) : nullptr;
     a.bc_rec = tc ? reinterpret_cast<float*>(ws + w.bc_rec) : nullptr;
-    a.bc_d = tc ? reinterpret_cast<float*>(ws + w.bc_d) : nullptr;
+    a.bc_d = tc ? reinterpret_cast<__nv_bfloat16*>(ws + w.bc_d) : nullptr;
     a.dy_img = tc ? reinterpret_cast<uint8_t*>(ws + w.dy) : nullptr;
     a.dq = dq; a.dk = dk_out; a.dv = dv_out;
     a.dalpha_log = dalpha_log; a.dmu_log = dmu_log; a.dbeta = dbeta; a.deta = deta;

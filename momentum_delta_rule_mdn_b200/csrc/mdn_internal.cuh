@@ -230,7 +230,8 @@ struct BwdArgs {
                            // chain's B operand (MN-major, 64-byte swizzle); with Qhat^T they
                            // give E and F inside the chain
     float* bc_rec;         // [B*H*NT, 256]  Gamma_C, w, then alphabar_C, b_C, mubar_C
-    float* bc_d;           // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde (chain order)
+    __nv_bfloat16* bc_d;   // [B*H*NT, 2, D, D]  K^T Diag(Gamma_C) Vtilde, K^T Diag(w) Vtilde (chain
+                           // order, bf16: increments of the fp32 rebuild)
     // outputs (fp32)
     float* dq;
     float* dk;

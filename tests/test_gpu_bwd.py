@@ -96,9 +96,12 @@ def test_bwd_layer_workload_sampled_heads():
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
         ref = ob.chunk_bwd(inp.q[sl], inp.k[sl], inp.v[sl], inp.alpha_log[sl], inp.mu_log[sl],
                            inp.beta[sl], inp.eta[sl], inp.d_corr, None, None, do[sl])
+        errs = {}
         for n in NAMES:
             mine = got[n][b:b + 1, :, h:h + 1] if n not in ("dS0", "dM0") else got[n][b:b + 1, h:h + 1]
-            e = rel_l2(mine, ref[n])
+            errs[n] = rel_l2(mine, ref[n])
+        print(f"bwd layer400m head ({b},{h}) rel-L2:", " ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+        for n, e in errs.items():
             assert e <= TOL["bf16"], (b, h, n, e)
 
 
