@@ -105,6 +105,21 @@ def test_bwd_layer_workload_sampled_heads():
             assert e <= TOL["bf16"], (b, h, n, e)
 
 
+def test_bwd_long_sequence_long_memory():
+    """64 chunks with the long-context gates (alpha and mu close to 1, as in the
+    16K-context workload): the state rebuild carries each chunk's increment
+    (stored in bf16) far down the sequence, so its rounding would build up
+    here if anywhere.  B = H = 1, T = 4096, d = 128, bf16, against the fp64
+    gradient oracle."""
+    spec = mi.Spec("bwd_long", B=1, T=4096, H=1, d=128, a_mean=3.0, c_mean=3.0,
+                   state_std=0.01, seed=506)
+    g, ref = _run(spec)
+    errs = {n: rel_l2(to_np(g[n]), ref[n]) for n in NAMES}
+    print("bwd long memory T4096 rel-L2:", " ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+    for n, e in errs.items():
+        assert e <= TOL["bf16"], (n, e)
+
+
 def test_bwd_cuda_graph_replay_matches_eager():
     """The backward call (which forks the state rebuild onto a side stream and
     joins it back) captured in a CUDA graph and replayed gives the eager
