@@ -386,11 +386,6 @@ __device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
 __device__ __forceinline__ uint32_t kmaj_off(int row, int k, uint32_t panel_bytes) {
     return (k >> 6) * panel_bytes + sw128_off(row, (k & 63) >> 3) + (k & 7) * 2;
 }
-// p[0..3] += (x, y, z, w) in L2, no value returned (16-byte aligned p)
-__device__ __forceinline__ void red_add_v4(float* p, float x, float y, float z, float w) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(x), "f"(y), "f"(z), "f"(w)
-                 : "memory");
-}
 
 __global__ void __launch_bounds__(kThr, 2)
 bwd_local_grads_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_qh,
