@@ -59,10 +59,16 @@ gate_prep_kernel(const GateSrc src, int B, int T, int H, int NT, float* __restri
 
     if (gamma == nullptr) return;
     // Column recurrence; this lane owns columns i0 = lane and i1 = lane + 32.
-    // mubar_r / mubar_i is kept as a running product of mu (non-negative
-    // factors; no exponential per element).
-    const float ea[2] = {expf(a[0]), expf(a[1])};
-    const float em[2] = {expf(m[0]), expf(m[1])};
+    // With f started at 0, f_r = mu_r f_{r-1} + [r == i] is mubar_r / mubar_i
+    // from the diagonal down (a running product of mu: non-negative factors,
+    // no exponential per element) and 0 above it, so
+    //     h_r = alpha_r h_{r-1} + beta_r f_r,   Gamma_{r,i} = eta_i h_r
+    // needs no case for the rows above the diagonal.  Each row's alpha, beta,
+    // mu come from shared memory as one broadcast 16-byte load.
+    __shared__ float4 rowc[4][kChunk];
+    float4* rc = rowc[threadIdx.x >> 5];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) rc[2 * lane + e] = make_float4(expf(a[e]), be[e], expf(m[e]), 0.f);
     const int i0 = lane, i1 = lane + 32;
     // Position p sits in lane p/2, element p%2: fetch both elements, pick locally.
     auto fetch = [&](const float (&x)[2], int p) {
@@ -71,23 +77,18 @@ gate_prep_kernel(const GateSrc src, int B, int T, int H, int NT, float* __restri
         return (p & 1) ? e1 : e0;
     };
     const float eta_i0 = fetch(et, i0), eta_i1 = fetch(et, i1);
-    float g0 = 0.f, g1 = 0.f, f0 = 1.f, f1 = 1.f;
+    __syncwarp();
+    float h0 = 0.f, h1 = 0.f, f0 = 0.f, f1 = 0.f;
     float* G = gamma + (size_t)chunk * kChunk * kChunk;
-#pragma unroll 2
-    for (int s = 0; s < kChunk / 2; ++s) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int r = 2 * s + e;
-            const float ar = __shfl_sync(kFull, ea[e], s);
-            const float br = __shfl_sync(kFull, be[e], s);
-            const float mr = __shfl_sync(kFull, em[e], s);
-            f0 = (r > i0) ? f0 * mr : 1.f;
-            f1 = (r > i1) ? f1 * mr : 1.f;
-            g0 = (r >= i0) ? fmaf(ar, g0, eta_i0 * br * f0) : 0.f;
-            g1 = (r >= i1) ? fmaf(ar, g1, eta_i1 * br * f1) : 0.f;
-            G[r * kChunk + i0] = g0;
-            G[r * kChunk + i1] = g1;
-        }
+#pragma unroll 4
+    for (int r = 0; r < kChunk; ++r) {
+        const float4 c = rc[r];
+        f0 = fmaf(c.z, f0, r == i0 ? 1.f : 0.f);
+        f1 = fmaf(c.z, f1, r == i1 ? 1.f : 0.f);
+        h0 = fmaf(c.x, h0, c.y * f0);
+        h1 = fmaf(c.x, h1, c.y * f1);
+        G[r * kChunk + i0] = eta_i0 * h0;
+        G[r * kChunk + i1] = eta_i1 * h1;
     }
 }
 
