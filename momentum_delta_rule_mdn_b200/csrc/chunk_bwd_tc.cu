@@ -56,8 +56,8 @@ __device__ __forceinline__ size_t tokrow(const BwdArgs& a, int b, int t, int h) 
 // every CTA and summed over CTAs (slot kBwdClkCtas of each kernel's block
 // counts them).  Diagnostic builds only (MDN_PHASE_CLOCKS, with the buffer set
 // by mdn_diag_bwd_clock); otherwise every call is empty.
-constexpr int kBwdClkSlots = 32, kBwdClkCtas = 31;
 #ifdef MDN_PHASE_CLOCKS
+constexpr int kBwdClkSlots = 32, kBwdClkCtas = 31;
 __device__ float* g_bwd_clk = nullptr;
 struct BwdClock {
     long long t;
