@@ -1,0 +1,130 @@
+"""CPU checks that the kernels' rewrites of the pages' definitions are exact.
+
+Each test emulates, in fp64 and in the order the kernel performs them, the
+steps of one of the chunk kernels' algorithms, and compares the result with
+the oracle or with a library routine.  They test the algorithms (their
+algebra and their schedules), not the CUDA code: the GPU parity tests cover
+the kernels themselves.
+
+"MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
+paper.rainbus.top summary, steps 4 and 5 (Gamma and T = (I + P K^T o Gamma-)^-1).
+"""
+import numpy as np
+
+import mdn_inputs as mi
+import oracle
+
+C = 64
+
+
+def _chunk_gates(seed=7):
+    """One chunk of the seeded generator's gates (fp64), as a kernel reads them."""
+    inp = mi.make_inputs(mi.Spec("algebra", B=1, T=3 * C, H=2, d=64, dtype="f32", seed=seed))
+    sl = (0, slice(C, 2 * C), 1)  # batch 0, chunk 1, head 1
+    return tuple(np.asarray(g, dtype=np.float64)[sl] for g in
+                 (inp.alpha_log, inp.mu_log, inp.beta, inp.eta)), inp
+
+
+def _oracle_gamma(inp):
+    _, _, _, gamma = oracle.chunk_coeffs(inp.alpha_log, inp.mu_log, inp.beta, inp.eta, C)
+    return gamma[0, 1, 1]  # batch 0, head 1, chunk 1
+
+
+def test_gamma_column_walk_zero_started_matches_oracle():
+    """The gate-prep kernel's walk down column i: f_r = mu_r f_{r-1} + [r = i]
+    from f = 0, h_r = alpha_r h_{r-1} + beta_r f_r, Gamma_{r,i} = eta_i h_r."""
+    (al, ml, be, et), inp = _chunk_gates()
+    a, m = np.exp(al), np.exp(ml)
+    G = np.zeros((C, C))
+    for i in range(C):
+        f = h = 0.0
+        for r in range(C):
+            f = m[r] * f + (1.0 if r == i else 0.0)
+            h = a[r] * h + be[r] * f
+            G[r, i] = et[i] * h
+    ref = _oracle_gamma(inp)
+    assert np.abs(G - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_gamma_column_walk_predicated_matches_oracle():
+    """The intra-chunk kernel's column pass: f = 1 on and above the diagonal and
+    f mu_r below it, Gamma = alpha_r Gamma_{r-1} + eta_i beta_r f on and below it."""
+    (al, ml, be, et), inp = _chunk_gates(seed=8)
+    a, m = np.exp(al), np.exp(ml)
+    G = np.zeros((C, C))
+    for i in range(C):
+        g, f = 0.0, 1.0
+        for r in range(C):
+            f = f * m[r] if r > i else 1.0
+            g = a[r] * g + et[i] * be[r] * f if r >= i else 0.0
+            G[r, i] = g
+    ref = _oracle_gamma(inp)
+    assert np.abs(G - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def _blocked_inverse(A):
+    """T = (I + A)^-1 for strictly lower A as the intra-chunk kernel solves it,
+    over 16 x 16 blocks: the diagonal blocks by forward substitution (one column
+    at a time), B_ik = -T_ii A_ik, then two dependent steps:
+        T_10 = B_10 T_00, T_21 = B_21 T_11, T_32 = B_32 T_22,
+        C_30 = B_30 + B_32 B_20, C_31 = B_31 + B_32 B_21;
+        T_20 = B_20 T_00 + B_21 T_10, T_31 = B_31 T_11 + B_32 T_21,
+        T_30 = C_30 T_00 + C_31 T_10."""
+    n = 16
+    blk = lambda M, i, j: M[n * i:n * (i + 1), n * j:n * (j + 1)]
+    Tii = []
+    for i in range(4):
+        Ai = blk(A, i, i)
+        Ti = np.zeros((n, n))
+        for cl in range(n):
+            t = np.zeros(n)
+            t[cl] = 1.0
+            for r in range(cl + 1, n):
+                t[r] = -sum(Ai[r, k] * t[k] for k in range(r))
+            Ti[:, cl] = t
+        Tii.append(Ti)
+    Bm = {(i, k): -Tii[i] @ blk(A, i, k) for i in range(4) for k in range(i)}
+    T = {(i, i): Tii[i] for i in range(4)}
+    T[1, 0] = Bm[1, 0] @ T[0, 0]
+    T[2, 1] = Bm[2, 1] @ T[1, 1]
+    T[3, 2] = Bm[3, 2] @ T[2, 2]
+    C30 = Bm[3, 0] + Bm[3, 2] @ Bm[2, 0]
+    C31 = Bm[3, 1] + Bm[3, 2] @ Bm[2, 1]
+    T[2, 0] = Bm[2, 0] @ T[0, 0] + Bm[2, 1] @ T[1, 0]
+    T[3, 1] = Bm[3, 1] @ T[1, 1] + Bm[3, 2] @ T[2, 1]
+    T[3, 0] = C30 @ T[0, 0] + C31 @ T[1, 0]
+    out = np.zeros((C, C))
+    for (i, j), M in T.items():
+        out[n * i:n * (i + 1), n * j:n * (j + 1)] = M
+    return out
+
+
+def test_blocked_two_step_inverse_matches_direct_inverse():
+    # A = (P K^T) o Gamma- as the kernel forms it, from one chunk of the
+    # generator's gates and keys
+    (al, ml, be, et), inp = _chunk_gates(seed=9)
+    k = np.asarray(inp.k, dtype=np.float64)[0, C:2 * C, 1]
+    gam = _oracle_gamma(inp)
+    gm = np.zeros((C, C))
+    gm[1:, :] = gam[:-1, :]                      # Gamma-_{r,i} = Gamma_{r-1,i}
+    A = np.tril(np.exp(al)[:, None] * (k @ k.T) * gm, -1)
+    T = _blocked_inverse(A)
+    ref = np.linalg.inv(np.eye(C) + A)
+    assert np.abs(T - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    # the schedule leaves the strict upper triangle at zero and the diagonal at one
+    assert np.all(np.triu(T, 1) == 0.0) and np.all(np.diag(T) == 1.0)
+
+
+def test_blocked_two_step_inverse_catches_a_wrong_schedule():
+    """The check above is sharp: dropping the B_32 B_20 term of C_30 (a
+    plausible slip in the two-step schedule) moves T_30 far outside it."""
+    rng = np.random.default_rng(3)
+    A = np.tril(rng.standard_normal((C, C)) * 0.2, -1)
+    ref = np.linalg.inv(np.eye(C) + A)
+    T = _blocked_inverse(A)
+    assert np.abs(T - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    n = 16
+    B = lambda i, k: -np.linalg.inv(np.eye(n) + A[n * i:n * (i + 1), n * i:n * (i + 1)]) @ \
+        A[n * i:n * (i + 1), n * k:n * (k + 1)]
+    wrong30 = B(3, 0) @ T[:n, :n] + (B(3, 1) + B(3, 2) @ B(2, 1)) @ T[n:2 * n, :n]
+    assert np.abs(wrong30 - ref[3 * n:, :n]).max() > 1e-3
