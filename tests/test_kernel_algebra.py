@@ -7,7 +7,8 @@ algebra and their schedules), not the CUDA code: the GPU parity tests cover
 the kernels themselves.
 
 "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
-paper.rainbus.top summary, steps 4 and 5 (Gamma and T = (I + P K^T o Gamma-)^-1).
+paper.rainbus.top summary, steps 3-5 and 7 (the chunk form, Gamma,
+T = (I + P K^T o Gamma-)^-1, q-hat).
 """
 import numpy as np
 
@@ -128,3 +129,52 @@ def test_blocked_two_step_inverse_catches_a_wrong_schedule():
         A[n * i:n * (i + 1), n * k:n * (k + 1)]
     wrong30 = B(3, 0) @ T[:n, :n] + (B(3, 1) + B(3, 2) @ B(2, 1)) @ T[n:2 * n, :n]
     assert np.abs(wrong30 - ref[3 * n:, :n]).max() > 1e-3
+
+
+def test_tensor_core_factorisation_matches_oracle():
+    """The tensor-core path's factorisation, step by step, against the stepwise
+    oracle over several chunks with non-zero entering states.  Per chunk the
+    intra-chunk kernel forms Qhat = Q - d K, A = (P K^T) o Gamma-, T = (I + A)^-1,
+    [T; Att T] with Att = (Qhat K^T) o Gamma, A2T = [K^T Diag(Gamma_C) T;
+    -K^T Diag(w) T] (w_r = eta_r mubar_C / mubar_r) and the records alphabar_r,
+    D2_r = alpha_r b_{r-1}, b_r; the chain then forms
+        Y = V - (alphabar_r K S - D2_r K M),  [Vtilde; Att T Y] = [T; Att T] Y,
+        o = alphabar_r Qhat S - b_r Qhat M + Att T Y,
+        S <- alphabar_C S - b_C M + A2T_S Y,  M <- mubar_C M + A2T_M Y."""
+    d, dcorr, NTc = 16, 0.5, 3
+    inp = mi.make_inputs(mi.Spec("factor", B=1, T=NTc * C, H=1, d=d, dtype="f32",
+                                 state_std=0.05, seed=11))
+    q, k, v = (np.asarray(x, dtype=np.float64)[0, :, 0] for x in (inp.q, inp.k, inp.v))
+    al, ml, be, et = (np.asarray(x, dtype=np.float64)[0, :, 0] for x in
+                      (inp.alpha_log, inp.mu_log, inp.beta, inp.eta))
+    _, _, _, gamma = oracle.chunk_coeffs(inp.alpha_log, inp.mu_log, inp.beta, inp.eta, C)
+    S = np.asarray(inp.S0, dtype=np.float64)[0, 0].copy()
+    M = np.asarray(inp.M0, dtype=np.float64)[0, 0].copy()
+    o = np.zeros((NTc * C, d))
+    vt = np.zeros((NTc * C, d))
+    for n in range(NTc):
+        sl = slice(n * C, (n + 1) * C)
+        K, Q, V = k[sl], q[sl], v[sl]
+        a, la, lm = np.exp(al[sl]), np.cumsum(al[sl]), np.cumsum(ml[sl])
+        abar, mbar = np.exp(la), np.exp(lm)
+        c = np.cumsum(be[sl] * mbar / abar)
+        b = abar * c
+        G = gamma[0, 0, n]
+        Gm = np.zeros((C, C))
+        Gm[1:, :] = G[:-1, :]
+        A = np.tril(a[:, None] * (K @ K.T) * Gm, -1)
+        T = np.linalg.inv(np.eye(C) + A)
+        Qh = Q - dcorr * K
+        Att = np.tril((Qh @ K.T) * G)
+        w = et[sl] * mbar[-1] / mbar
+        A2S = K.T @ (G[-1][:, None] * T)
+        A2M = -K.T @ (w[:, None] * T)
+        D2 = a * np.concatenate(([0.0], b[:-1]))
+        Y = V - (abar[:, None] * (K @ S) - D2[:, None] * (K @ M))
+        vt[sl] = T @ Y
+        o[sl] = abar[:, None] * (Qh @ S) - b[:, None] * (Qh @ M) + (Att @ T) @ Y
+        S, M = abar[-1] * S - b[-1] * M + A2S @ Y, mbar[-1] * M + A2M @ Y
+    ro, rvt, rS, rM = oracle.chunk_fwd(inp.q, inp.k, inp.v, inp.alpha_log, inp.mu_log,
+                                      inp.beta, inp.eta, dcorr, inp.S0, inp.M0)
+    for x, ref in ((o, ro[0, :, 0]), (vt, rvt[0, :, 0]), (S, rS[0, 0]), (M, rM[0, 0])):
+        assert np.abs(x - ref).max() <= 1e-9 * np.abs(ref).max()
