@@ -75,7 +75,7 @@ typedef enum {
 #define MDN_SLICE64      0x8  /* ... 64 columns (two CTAs per head) */
 #define MDN_SLICE128     0x10 /* ... all 128 columns (one CTA per head).  None of the
                                  three: 32 when B*H*4 CTAs fit on the SMs at once,
-                                 else 128 (packed sequences: 32 up to two waves, else
+                                 else 128 (packed sequences: 32 up to four waves, else
                                  64).  At most one; every width computes the same
                                  result; the flags exist for tuning and testing. */
 #define MDN_TEST_NO_INTRA 0x100 /* testing the failure path only: the tensor-core
