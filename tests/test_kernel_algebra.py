@@ -8,7 +8,8 @@ the kernels themselves.
 
 "MDN: Parallelizing Stepwise Momentum for Delta Linear Attention",
 paper.rainbus.top summary, steps 3-5 and 7 (the chunk form, Gamma,
-T = (I + P K^T o Gamma-)^-1, q-hat).
+T = (I + P K^T o Gamma-)^-1, q-hat), and the backward pass the pages train with
+(summary step 7; ijyty.com article section 6).
 """
 import numpy as np
 
@@ -178,3 +179,80 @@ def test_tensor_core_factorisation_matches_oracle():
                                       inp.beta, inp.eta, dcorr, inp.S0, inp.M0)
     for x, ref in ((o, ro[0, :, 0]), (vt, rvt[0, :, 0]), (S, rS[0, 0]), (M, rM[0, 0])):
         assert np.abs(x - ref).max() <= 1e-9 * np.abs(ref).max()
+
+
+def test_backward_blocked_column_recurrence():
+    """The backward coefficient phase's R_{j,i} = sum_{r>=j} dG_{r,i} alphabar_r /
+    alphabar_j, i.e. R_j = dG_j + alpha_{j+1} R_{j+1} down each column (rows
+    j >= i), as the kernel runs it: four blocks of 16 rows, each from a zero
+    carry keeping L_j and the decay P_j = alpha_{j+1} .. alpha_{16(p+1)} to its
+    block's end, then the carries passed up from the blocks below and
+    R_j = L_j + P_j carry."""
+    rng = np.random.default_rng(5)
+    al = rng.uniform(0.3, 1.0, C)
+    dG = np.tril(rng.standard_normal((C, C)))
+    al1 = np.append(al[1:], 0.0)                 # alpha_{j+1}; none past the chunk
+    ref = np.zeros((C, C))
+    for i in range(C):
+        R = 0.0
+        for j in range(C - 1, i - 1, -1):
+            R = dG[j, i] + al1[j] * R
+            ref[j, i] = R
+    out = np.zeros((C, C))
+    for i in range(C):
+        Ls, Ps = [], []
+        for part in range(4):
+            lo = 16 * part
+            L = np.array([dG[lo + e, i] if lo + e >= i else 0.0 for e in range(16)])
+            P = np.zeros(16)
+            l, pr = 0.0, 1.0
+            for e in range(15, -1, -1):
+                pr *= al1[lo + e]
+                l = L[e] + al1[lo + e] * l
+                L[e], P[e] = l, pr
+            Ls.append(L)
+            Ps.append(P)
+        for part in range(4):
+            carry = 0.0
+            for q in range(3, part, -1):
+                carry = Ls[q][0] + Ps[q][0] * carry
+            for e in range(16):
+                j = 16 * part + e
+                if j >= i:
+                    out[j, i] = Ls[part][e] + Ps[part][e] * carry
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_backward_affine_suffix_scan():
+    """Rb_j = db_j + alpha_{j+1} Rb_{j+1} (Rb_C = 0) as a warp's suffix scan:
+    lane l composes the maps of positions 2l, 2l+1 as (b0 + a0 b1, a0 a1), the
+    lanes combine with the ones `off` above (off = 1, 2, 4, 8, 16) by
+    (b, a) <- (b + a b', a a'), and position 2l+1 takes db + alpha Rb of 2l+2."""
+    rng = np.random.default_rng(6)
+    al = rng.uniform(0.3, 1.0, C)
+    db = rng.standard_normal(C)
+    ref = np.zeros(C)
+    R = 0.0
+    for j in range(C - 1, -1, -1):
+        R = db[j] + (al[j + 1] if j + 1 < C else 0.0) * R
+        ref[j] = R
+    sb = np.zeros(32)
+    sa = np.zeros(32)
+    a1s = np.zeros(32)
+    for lane in range(32):
+        j0, j1 = 2 * lane, 2 * lane + 1
+        a0, a1 = al[j1], (al[j1 + 1] if j1 + 1 < C else 0.0)
+        sb[lane], sa[lane], a1s[lane] = a0 * db[j1] + db[j0], a0 * a1, a1
+    off = 1
+    while off < 32:
+        ob = np.append(sb[off:], np.zeros(off))  # shuffle down: lane l reads lane l + off
+        oa = np.append(sa[off:], np.zeros(off))
+        live = np.arange(32) + off < 32
+        sb = np.where(live, sb + sa * ob, sb)
+        sa = np.where(live, sa * oa, sa)
+        off <<= 1
+    nxt = np.append(sb[1:], 0.0)
+    out = np.zeros(C)
+    out[0::2] = sb
+    out[1::2] = db[1::2] + a1s * nxt
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
