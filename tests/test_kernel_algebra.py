@@ -256,3 +256,37 @@ def test_backward_affine_suffix_scan():
     out[0::2] = sb
     out[1::2] = db[1::2] + a1s * nxt
     assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_backward_state_rebuild_from_saved_vtilde():
+    """The backward pass keeps only Vtilde from the forward pass and rebuilds
+    the chunk-entering states by the scan the state-rebuild kernel runs:
+        D_S = K^T Diag(Gamma_{C,.}) Vtilde,  D_M = K^T Diag(w) Vtilde,
+        S <- alphabar_C S - b_C M + D_S,     M <- mubar_C M - D_M.
+    Each rebuilt state equals the oracle's state after that many tokens."""
+    d, NTc = 16, 3
+    inp = mi.make_inputs(mi.Spec("rebuild", B=1, T=NTc * C, H=1, d=d, dtype="f32",
+                                 state_std=0.05, seed=12))
+    args = (inp.alpha_log, inp.mu_log, inp.beta, inp.eta)
+    _, vt, _, _ = oracle.chunk_fwd(inp.q, inp.k, inp.v, *args, inp.d_corr, inp.S0, inp.M0)
+    _, _, _, gamma = oracle.chunk_coeffs(*args, C)
+    k = np.asarray(inp.k, dtype=np.float64)[0, :, 0]
+    al, ml, be, et = (np.asarray(x, dtype=np.float64)[0, :, 0] for x in args)
+    S = np.asarray(inp.S0, dtype=np.float64)[0, 0].copy()
+    M = np.asarray(inp.M0, dtype=np.float64)[0, 0].copy()
+    for n in range(NTc):
+        sl = slice(n * C, (n + 1) * C)
+        la, lm = np.cumsum(al[sl]), np.cumsum(ml[sl])
+        abar, mbar = np.exp(la), np.exp(lm)
+        bC = abar[-1] * np.sum(be[sl] * mbar / abar)
+        w = et[sl] * mbar[-1] / mbar
+        V = vt[0, sl, 0]
+        DS = k[sl].T @ (gamma[0, 0, n][-1][:, None] * V)
+        DM = k[sl].T @ (w[:, None] * V)
+        S, M = abar[-1] * S - bC * M + DS, mbar[-1] * M - DM
+        T1 = (n + 1) * C
+        cut = lambda x: None if x is None else np.asarray(x)[:, :T1]
+        _, _, rS, rM = oracle.chunk_fwd(cut(inp.q), cut(inp.k), cut(inp.v),
+                                        *(cut(g) for g in args), inp.d_corr, inp.S0, inp.M0)
+        for x, ref in ((S, rS[0, 0]), (M, rM[0, 0])):
+            assert np.abs(x - ref).max() <= 1e-10 * np.abs(ref).max()
